@@ -1,0 +1,161 @@
+"""FP64 CPU oracle for exact softmax attention: test infrastructure only.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  It shares no code with the CUDA path
+(``exact_io_aware_63_b200``) and never imports it.
+
+The arithmetic lives in ``attention_oracle.c`` (plain C, double precision),
+which states the definition it follows: standard attention, which the pages
+("FlashAttention: Fast and Memory-Efficient Exact Attention with
+IO-Awareness", opendecode.dev summary, "The key idea"; "FlashAttention,
+Decoded", gloss of abstract sentence 4) say the tiled method reproduces
+exactly.  This module only builds that file with gcc and marshals numpy
+arrays to it.
+
+Functions (all arrays contiguous, float64 unless stated):
+
+* ``attention_forward(q, k, v, scale, causal, block_mask, kv_len)`` ->
+  ``(o, lse)`` for q, k, v of shape [B, H, N, d].
+* ``attention_backward(q, k, v, dout, scale, causal, block_mask, kv_len)`` ->
+  ``(dq, dk, dv, delta)`` by the chain rule on sum(O * dO).
+* ``attention_forward_rows(q_rows, rows, k, v, scale, causal, block_mask,
+  kv_len_b)`` -> ``(o_rows, lse_rows)`` for chosen query rows of one head.
+* ``tile_visits(B, N, causal, block_mask, kv_len, T=128, i_begin=0,
+  i_end=None)`` -> uint8 [B, i_end - i_begin, N // T]: 1 where a
+  (query tile, key tile) pair holds at least one allowed (row, key).
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "attention_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+_dp = ctypes.POINTER(ctypes.c_double)
+_u8p = ctypes.POINTER(ctypes.c_uint8)
+_i32p = ctypes.POINTER(ctypes.c_int32)
+_i64p = ctypes.POINTER(ctypes.c_int64)
+
+
+def build(force: bool = False) -> str:
+    """Compile attention_oracle.c into liboracle.so next to it (gcc -O2)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-Wall", "-shared", "-fPIC", "-o", tmp, _SRC,
+             "-lpthread", "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            lib.oracle_attention_forward.argtypes = [
+                _dp, _dp, _dp, _dp, _dp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                ctypes.c_double, ctypes.c_int, _u8p, _i32p, ctypes.c_int]
+            lib.oracle_attention_backward.argtypes = [
+                _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                ctypes.c_int, ctypes.c_double, ctypes.c_int, _u8p, _i32p, ctypes.c_int]
+            lib.oracle_attention_forward_rows.argtypes = [
+                _dp, _i64p, ctypes.c_int, _dp, _dp, _dp, _dp, ctypes.c_int, ctypes.c_int,
+                ctypes.c_double, ctypes.c_int, _u8p, ctypes.c_int]
+            lib.oracle_tile_visits.argtypes = [
+                _u8p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _u8p, _i32p,
+                ctypes.c_int, ctypes.c_int]
+            for fn in (lib.oracle_attention_forward, lib.oracle_attention_backward,
+                       lib.oracle_attention_forward_rows, lib.oracle_tile_visits):
+                fn.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def _f64(a):
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a, typ):
+    return a.ctypes.data_as(typ) if a is not None else None
+
+
+def _mask_args(block_mask, kv_len):
+    bm = None if block_mask is None else np.ascontiguousarray(np.asarray(block_mask, np.uint8))
+    kl = None if kv_len is None else np.ascontiguousarray(np.asarray(kv_len, np.int32))
+    return bm, kl
+
+
+def _threads(nthreads):
+    return int(nthreads) if nthreads else (os.cpu_count() or 1)
+
+
+def attention_forward(q, k, v, scale, causal=False, block_mask=None, kv_len=None, nthreads=None):
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, N, d = q.shape
+    assert k.shape == q.shape and v.shape == q.shape
+    bm, kl = _mask_args(block_mask, kv_len)
+    o = np.empty_like(q)
+    lse = np.empty((B, H, N), np.float64)
+    rc = _load().oracle_attention_forward(
+        _ptr(q, _dp), _ptr(k, _dp), _ptr(v, _dp), _ptr(o, _dp), _ptr(lse, _dp), B, H, N, d,
+        float(scale), int(bool(causal)), _ptr(bm, _u8p), _ptr(kl, _i32p), _threads(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attention_forward failed: {rc}")
+    return o, lse
+
+
+def attention_backward(q, k, v, dout, scale, causal=False, block_mask=None, kv_len=None,
+                       nthreads=None):
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, H, N, d = q.shape
+    bm, kl = _mask_args(block_mask, kv_len)
+    dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
+    delta = np.empty((B, H, N), np.float64)
+    rc = _load().oracle_attention_backward(
+        _ptr(q, _dp), _ptr(k, _dp), _ptr(v, _dp), _ptr(dout, _dp), _ptr(dq, _dp), _ptr(dk, _dp),
+        _ptr(dv, _dp), _ptr(delta, _dp), B, H, N, d, float(scale), int(bool(causal)),
+        _ptr(bm, _u8p), _ptr(kl, _i32p), _threads(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attention_backward failed: {rc}")
+    return dq, dk, dv, delta
+
+
+def attention_forward_rows(q_rows, rows, k, v, scale, causal=False, block_mask=None,
+                           kv_len_b=None):
+    """Forward for query rows ``rows`` (int array) of one head; q_rows is [R, d]."""
+    q_rows, k, v = _f64(q_rows), _f64(k), _f64(v)
+    rows = np.ascontiguousarray(np.asarray(rows, np.int64))
+    R, d = q_rows.shape
+    N = k.shape[0]
+    bm, _ = _mask_args(block_mask, None)
+    o = np.empty((R, d), np.float64)
+    lse = np.empty((R,), np.float64)
+    rc = _load().oracle_attention_forward_rows(
+        _ptr(q_rows, _dp), _ptr(rows, _i64p), R, _ptr(k, _dp), _ptr(v, _dp), _ptr(o, _dp),
+        _ptr(lse, _dp), N, d, float(scale), int(bool(causal)), _ptr(bm, _u8p),
+        -1 if kv_len_b is None else int(kv_len_b))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attention_forward_rows failed: {rc}")
+    return o, lse
+
+
+def tile_visits(B, N, causal=False, block_mask=None, kv_len=None, T=128, i_begin=0, i_end=None):
+    nt = N // T
+    i_end = nt if i_end is None else i_end
+    bm, kl = _mask_args(block_mask, kv_len)
+    out = np.zeros((B, i_end - i_begin, nt), np.uint8)
+    rc = _load().oracle_tile_visits(_ptr(out, _u8p), B, N, T, int(bool(causal)), _ptr(bm, _u8p),
+                                    _ptr(kl, _i32p), i_begin, i_end)
+    if rc != 0:
+        raise RuntimeError(f"oracle_tile_visits failed: {rc}")
+    return out

@@ -1,0 +1,318 @@
+/*
+ * Plain FP64 CPU oracle for exact softmax attention (forward and backward).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg may load this file's library.  It shares no
+ * code, header, table or helper with the CUDA path, and the CUDA path never
+ * calls it.
+ *
+ * What it computes.  "FlashAttention: Fast and Memory-Efficient Exact
+ * Attention with IO-Awareness" (opendecode.dev summary, section "The key
+ * idea") and "FlashAttention, Decoded" (abstract gloss, sentence 4) both say
+ * the tiled method gives an output identical to standard attention.  The
+ * oracle is therefore the plain definition of standard attention, written
+ * out one query row at a time:
+ *
+ *   M(r,c) = (!causal || c <= r) && (kv_len == NULL || c < kv_len[b])
+ *            && (block_mask == NULL || block_mask[(r/128)*(N/128) + c/128] != 0)
+ *   S_rc   = scale * sum_k Q_rk K_ck          if M(r,c), else -inf
+ *   m_r    = max_c S_rc,  l_r = sum_c exp(S_rc - m_r)
+ *   P_rc   = exp(S_rc - m_r) / l_r,  LSE_r = m_r + ln l_r  (natural log)
+ *   O_r    = sum_c P_rc V_c
+ *
+ * The backward pass is the chain rule on L = sum(O * dO):
+ *   dV_c = sum_r P_rc dO_r,  dP_rc = dO_r . V_c,  D_r = sum_c P_rc dP_rc,
+ *   dS_rc = P_rc (dP_rc - D_r),  dQ_r = scale sum_c dS_rc K_c,
+ *   dK_c = scale sum_r dS_rc Q_r.
+ *
+ * A row with no allowed key has O_r = 0, LSE_r = -inf and zero gradients.
+ * There is no tiling, no online softmax and no reordering: one full score
+ * row is formed, then normalised.  Work is split over (b, h) heads with
+ * POSIX threads; each head is computed by exactly one thread, so the result
+ * does not depend on the thread count.
+ *
+ * Layout: every tensor is contiguous [B][H][N][d] (row-major), LSE and D
+ * are [B][H][N].
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_MASK_TILE 128
+
+typedef struct {
+    const double *q, *k, *v, *dout;
+    double *o, *lse, *dq, *dk, *dv, *delta;
+    int B, H, N, d;
+    double scale;
+    int causal;
+    const uint8_t *block_mask;
+    const int32_t *kv_len;
+    int backward;
+    int next_head;          /* shared work counter, guarded by lock */
+    pthread_mutex_t lock;
+} oracle_job;
+
+/* The mask M(r,c) exactly as defined above. */
+static int allowed(int r, int c, int N, int causal, const uint8_t *block_mask, int L)
+{
+    if (causal && c > r) return 0;
+    if (L >= 0 && c >= L) return 0;
+    if (block_mask) {
+        int nt = N / ORACLE_MASK_TILE;
+        if (!block_mask[(size_t)(r / ORACLE_MASK_TILE) * nt + (c / ORACLE_MASK_TILE)]) return 0;
+    }
+    return 1;
+}
+
+/*
+ * One softmax row.  Fills p[0..N) with P_rc (0 where masked) and returns the
+ * row's m and l through the pointers.  Returns the number of allowed keys.
+ */
+static int softmax_row(const double *qr, int r, const double *K, int N, int d, double scale,
+                       int causal, const uint8_t *block_mask, int L, double *p,
+                       double *m_out, double *l_out)
+{
+    int count = 0;
+    double m = -INFINITY;
+    for (int c = 0; c < N; ++c) {
+        if (!allowed(r, c, N, causal, block_mask, L)) {
+            p[c] = -INFINITY;
+            continue;
+        }
+        const double *kc = K + (size_t)c * d;
+        double s = 0.0;
+        for (int x = 0; x < d; ++x) s += qr[x] * kc[x];
+        s *= scale;
+        p[c] = s;
+        if (s > m) m = s;
+        ++count;
+    }
+    double l = 0.0;
+    for (int c = 0; c < N; ++c) {
+        if (p[c] == -INFINITY) { p[c] = 0.0; continue; }
+        p[c] = exp(p[c] - m);
+        l += p[c];
+    }
+    if (count > 0)
+        for (int c = 0; c < N; ++c) p[c] /= l;
+    *m_out = m;
+    *l_out = l;
+    return count;
+}
+
+static void forward_head(const oracle_job *job, int bh, double *p)
+{
+    const int N = job->N, d = job->d;
+    const int b = bh / job->H;
+    const size_t off = (size_t)bh * N * d;
+    const double *Q = job->q + off, *K = job->k + off, *V = job->v + off;
+    double *O = job->o + off;
+    double *lse = job->lse + (size_t)bh * N;
+    const int L = job->kv_len ? job->kv_len[b] : -1;
+    for (int r = 0; r < N; ++r) {
+        double m, l;
+        int count = softmax_row(Q + (size_t)r * d, r, K, N, d, job->scale, job->causal,
+                                job->block_mask, L, p, &m, &l);
+        double *orow = O + (size_t)r * d;
+        for (int x = 0; x < d; ++x) orow[x] = 0.0;
+        if (count == 0) {
+            lse[r] = -INFINITY;
+            continue;
+        }
+        for (int c = 0; c < N; ++c) {
+            if (p[c] == 0.0) continue;
+            const double *vc = V + (size_t)c * d;
+            for (int x = 0; x < d; ++x) orow[x] += p[c] * vc[x];
+        }
+        lse[r] = m + log(l);
+    }
+}
+
+static void backward_head(const oracle_job *job, int bh, double *p, double *dp)
+{
+    const int N = job->N, d = job->d;
+    const int b = bh / job->H;
+    const size_t off = (size_t)bh * N * d;
+    const double *Q = job->q + off, *K = job->k + off, *V = job->v + off, *dO = job->dout + off;
+    double *dQ = job->dq + off, *dK = job->dk + off, *dV = job->dv + off;
+    const int L = job->kv_len ? job->kv_len[b] : -1;
+    memset(dK, 0, sizeof(double) * (size_t)N * d);
+    memset(dV, 0, sizeof(double) * (size_t)N * d);
+    for (int r = 0; r < N; ++r) {
+        const double *qr = Q + (size_t)r * d;
+        const double *dor = dO + (size_t)r * d;
+        double *dqr = dQ + (size_t)r * d;
+        double m, l;
+        int count = softmax_row(qr, r, K, N, d, job->scale, job->causal, job->block_mask, L, p,
+                                &m, &l);
+        for (int x = 0; x < d; ++x) dqr[x] = 0.0;
+        if (count == 0) {
+            if (job->delta) job->delta[(size_t)bh * N + r] = 0.0;
+            continue;
+        }
+        /* dP_rc = dO_r . V_c and D_r = sum_c P_rc dP_rc */
+        double D = 0.0;
+        for (int c = 0; c < N; ++c) {
+            if (p[c] == 0.0) { dp[c] = 0.0; continue; }
+            const double *vc = V + (size_t)c * d;
+            double s = 0.0;
+            for (int x = 0; x < d; ++x) s += dor[x] * vc[x];
+            dp[c] = s;
+            D += p[c] * s;
+        }
+        if (job->delta) job->delta[(size_t)bh * N + r] = D;
+        for (int c = 0; c < N; ++c) {
+            if (p[c] == 0.0) continue;
+            const double ds = p[c] * (dp[c] - D);
+            const double *kc = K + (size_t)c * d;
+            double *dkc = dK + (size_t)c * d;
+            double *dvc = dV + (size_t)c * d;
+            for (int x = 0; x < d; ++x) {
+                dqr[x] += job->scale * ds * kc[x];
+                dkc[x] += job->scale * ds * qr[x];
+                dvc[x] += p[c] * dor[x];
+            }
+        }
+    }
+}
+
+static void *worker(void *arg)
+{
+    oracle_job *job = (oracle_job *)arg;
+    double *p = (double *)malloc(sizeof(double) * (size_t)job->N);
+    double *dp = (double *)malloc(sizeof(double) * (size_t)job->N);
+    if (!p || !dp) {
+        free(p);
+        free(dp);
+        return (void *)1;
+    }
+    for (;;) {
+        pthread_mutex_lock(&job->lock);
+        int bh = job->next_head++;
+        pthread_mutex_unlock(&job->lock);
+        if (bh >= job->B * job->H) break;
+        if (job->backward)
+            backward_head(job, bh, p, dp);
+        else
+            forward_head(job, bh, p);
+    }
+    free(p);
+    free(dp);
+    return NULL;
+}
+
+static int run_job(oracle_job *job, int nthreads)
+{
+    if (job->B <= 0 || job->H <= 0 || job->N <= 0 || job->d <= 0) return -3;
+    if (job->block_mask && job->N % ORACLE_MASK_TILE != 0) return -3;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > job->B * job->H) nthreads = job->B * job->H;
+    pthread_mutex_init(&job->lock, NULL);
+    job->next_head = 0;
+    pthread_t *tids = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    int rc = 0, started = 0;
+    for (int t = 0; t < nthreads; ++t) {
+        if (pthread_create(&tids[t], NULL, worker, job) != 0) { rc = -6; break; }
+        ++started;
+    }
+    for (int t = 0; t < started; ++t) {
+        void *ret = NULL;
+        pthread_join(tids[t], &ret);
+        if (ret) rc = -6;
+    }
+    free(tids);
+    pthread_mutex_destroy(&job->lock);
+    return rc;
+}
+
+int oracle_attention_forward(const double *q, const double *k, const double *v, double *o,
+                             double *lse, int B, int H, int N, int d, double scale, int causal,
+                             const uint8_t *block_mask, const int32_t *kv_len, int nthreads)
+{
+    oracle_job job;
+    memset(&job, 0, sizeof(job));
+    job.q = q; job.k = k; job.v = v; job.o = o; job.lse = lse;
+    job.B = B; job.H = H; job.N = N; job.d = d; job.scale = scale; job.causal = causal;
+    job.block_mask = block_mask; job.kv_len = kv_len; job.backward = 0;
+    return run_job(&job, nthreads);
+}
+
+int oracle_attention_backward(const double *q, const double *k, const double *v,
+                              const double *dout, double *dq, double *dk, double *dv,
+                              double *delta, int B, int H, int N, int d, double scale, int causal,
+                              const uint8_t *block_mask, const int32_t *kv_len, int nthreads)
+{
+    oracle_job job;
+    memset(&job, 0, sizeof(job));
+    job.q = q; job.k = k; job.v = v; job.dout = dout;
+    job.dq = dq; job.dk = dk; job.dv = dv; job.delta = delta;
+    job.B = B; job.H = H; job.N = N; job.d = d; job.scale = scale; job.causal = causal;
+    job.block_mask = block_mask; job.kv_len = kv_len; job.backward = 1;
+    return run_job(&job, nthreads);
+}
+
+/*
+ * Forward for a chosen subset of query rows of ONE head.  q_rows is
+ * [R][d] (row i holds query number rows[i]); K and V are the head's full
+ * [N][d]; kv_len_b < 0 means no key padding.  Used to check sampled rows at
+ * sizes where the whole head is too slow on the CPU; each row is the same
+ * computation as in oracle_attention_forward.
+ */
+int oracle_attention_forward_rows(const double *q_rows, const int64_t *rows, int R,
+                                  const double *k, const double *v, double *o_rows,
+                                  double *lse_rows, int N, int d, double scale, int causal,
+                                  const uint8_t *block_mask, int kv_len_b)
+{
+    if (R < 0 || N <= 0 || d <= 0) return -3;
+    double *p = (double *)malloc(sizeof(double) * (size_t)N);
+    if (!p) return -6;
+    for (int i = 0; i < R; ++i) {
+        const int r = (int)rows[i];
+        double m, l;
+        int count = softmax_row(q_rows + (size_t)i * d, r, k, N, d, scale, causal, block_mask,
+                                kv_len_b, p, &m, &l);
+        double *orow = o_rows + (size_t)i * d;
+        for (int x = 0; x < d; ++x) orow[x] = 0.0;
+        if (count == 0) { lse_rows[i] = -INFINITY; continue; }
+        for (int c = 0; c < N; ++c) {
+            if (p[c] == 0.0) continue;
+            const double *vc = v + (size_t)c * d;
+            for (int x = 0; x < d; ++x) orow[x] += p[c] * vc[x];
+        }
+        lse_rows[i] = m + log(l);
+    }
+    free(p);
+    return 0;
+}
+
+/*
+ * Which (query tile, key tile) pairs hold at least one allowed (r, c).
+ * visits is [B][i_end - i_begin][n_t] with n_t = N / T: the entry for query
+ * tile i (i_begin <= i < i_end) and key tile j is 1 when some r in tile i and
+ * some c in tile j have M(r,c), else 0.  Brute force over the entries of each
+ * tile pair (stopping at the first allowed one), straight from the
+ * definition of M; heads share the mask, so only b matters.
+ */
+int oracle_tile_visits(uint8_t *visits, int B, int N, int T, int causal,
+                       const uint8_t *block_mask, const int32_t *kv_len, int i_begin, int i_end)
+{
+    if (T <= 0 || N % T != 0 || (block_mask && N % ORACLE_MASK_TILE != 0)) return -3;
+    const int nt = N / T;
+    if (i_begin < 0 || i_end > nt || i_begin > i_end) return -3;
+    const int ni = i_end - i_begin;
+    for (int b = 0; b < B; ++b) {
+        const int L = kv_len ? kv_len[b] : -1;
+        for (int i = i_begin; i < i_end; ++i)
+            for (int j = 0; j < nt; ++j) {
+                int any = 0;
+                for (int r = i * T; r < (i + 1) * T && !any; ++r)
+                    for (int c = j * T; c < (j + 1) * T; ++c)
+                        if (allowed(r, c, N, causal, block_mask, L)) { any = 1; break; }
+                visits[((size_t)b * ni + (i - i_begin)) * nt + j] = (uint8_t)any;
+            }
+    }
+    return 0;
+}

@@ -1,0 +1,338 @@
+"""Pins for the FP64 oracle: closed forms, invariants, brute force and a hand-worked case.
+
+None of these re-types the oracle's formula.  Each checks a fact that the
+mathematics (or the pages' "exact attention" claim, opendecode.dev summary,
+"The key idea") fixes, chosen so that a plausible slip in the oracle (a
+dropped scale, a wrong sign, a transposed operand, an off-by-one in the mask,
+a log base, a missing max-subtraction) fails at least one of them.
+"""
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def rand(shape, seed):
+    return np.random.default_rng(seed).standard_normal(shape)
+
+
+def allowed_count(N, r, causal, kv, bm):
+    """Number of allowed keys of row r, counted one key at a time."""
+    cnt = 0
+    for c in range(N):
+        ok = (not causal or c <= r) and (kv is None or c < kv)
+        if bm is not None:
+            ok = ok and bm[r // 128, c // 128] != 0
+        cnt += int(ok)
+    return cnt
+
+
+# ---------------------------------------------------------------------------
+# hand-worked example (tests/golden/two_key_attention.json)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("case", ["noncausal", "causal"])
+def test_golden_two_key(case):
+    g = json.load(open(os.path.join(GOLDEN, "two_key_attention.json")))
+    q = np.array(g["q"])[None, None]
+    k = np.array(g["k"])[None, None]
+    v = np.array(g["v"])[None, None]
+    do = np.array(g["dout"])[None, None]
+    causal = case == "causal"
+    exp = g[case]
+    o, lse = oracle.attention_forward(q, k, v, g["scale"], causal=causal)
+    np.testing.assert_allclose(o[0, 0], exp["o"], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(lse[0, 0], exp["lse"], rtol=0, atol=1e-14)
+    dq, dk, dv, delta = oracle.attention_backward(q, k, v, do, g["scale"], causal=causal)
+    np.testing.assert_allclose(dq[0, 0], exp["dq"], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(dk[0, 0], exp["dk"], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(dv[0, 0], exp["dv"], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(delta[0, 0], exp["delta"], rtol=0, atol=1e-14)
+
+
+# ---------------------------------------------------------------------------
+# closed forms
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("causal,kv,use_bm", [(False, None, False), (True, None, False),
+                                              (False, 300, False), (True, 200, True),
+                                              (False, None, True)])
+def test_zero_query_gives_mean_of_allowed_values(causal, kv, use_bm):
+    B, H, N, d = 1, 2, 384, 16
+    q = np.zeros((B, H, N, d))
+    k, v = rand((B, H, N, d), 1), rand((B, H, N, d), 2)
+    bm = None
+    if use_bm:
+        bm = np.array([[1, 0, 1], [1, 1, 0], [0, 1, 1]], np.uint8)
+    kvl = None if kv is None else np.array([kv], np.int32)
+    o, lse = oracle.attention_forward(q, k, v, 0.125, causal=causal, block_mask=bm, kv_len=kvl)
+    for r in [0, 1, 127, 128, 200, 255, 256, 383]:
+        keys = [c for c in range(N)
+                if (not causal or c <= r) and (kv is None or c < kv)
+                and (bm is None or bm[r // 128, c // 128])]
+        cnt = allowed_count(N, r, causal, kv, bm)
+        assert cnt == len(keys)
+        for h in range(H):
+            if cnt == 0:
+                assert np.all(o[0, h, r] == 0) and lse[0, h, r] == -np.inf
+                continue
+            np.testing.assert_allclose(o[0, h, r], v[0, h, keys].mean(axis=0), atol=1e-13)
+            assert abs(lse[0, h, r] - math.log(cnt)) < 1e-13
+
+
+def test_dominant_score_selects_one_value_row():
+    N, d = 64, 64
+    rng = np.random.default_rng(3)
+    # orthonormal key rows: each query aligned with one key gives score 50*scale*|k| for it,
+    # and 0 for every other key
+    basis, _ = np.linalg.qr(rng.standard_normal((d, d)))
+    k = basis[:N]
+    target = rng.permutation(N)
+    q = 400.0 * k[target]          # score 400*scale = 50 for the target key, 0 elsewhere
+    v = rng.standard_normal((N, d))
+    o, lse = oracle.attention_forward(q[None, None], k[None, None], v[None, None], 0.125)
+    np.testing.assert_allclose(o[0, 0], v[target], atol=1e-12 * 50)
+    # LSE = 50 + ln(1 + (N-1) e^-50)
+    np.testing.assert_allclose(lse[0, 0], 50.0 + np.log1p((N - 1) * np.exp(-50.0)), atol=1e-12)
+
+
+def test_large_scores_do_not_overflow():
+    # scores near 1000 overflow exp() unless the row max is subtracted first
+    N, d = 8, 4
+    q = np.zeros((N, d)); q[:, 0] = 1000.0
+    k = np.zeros((N, d)); k[:, 0] = 1.0; k[3, 0] = 1.001
+    v = rand((N, d), 4)
+    o, lse = oracle.attention_forward(q[None, None], k[None, None], v[None, None], 1.0)
+    w = np.exp(np.array([0.0] * 3 + [1.0] + [0.0] * 4))
+    np.testing.assert_allclose(o[0, 0, 0], (w[:, None] * v).sum(0) / w.sum(), atol=1e-12)
+    np.testing.assert_allclose(lse[0, 0, 0], 1000.0 + np.log(w.sum()), atol=1e-10)
+
+
+def test_causal_row_zero():
+    B, H, N, d = 2, 3, 256, 32
+    q, k, v = rand((B, H, N, d), 5), rand((B, H, N, d), 6), rand((B, H, N, d), 7)
+    s = 0.17
+    o, lse = oracle.attention_forward(q, k, v, s, causal=True)
+    assert np.array_equal(o[:, :, 0], v[:, :, 0])
+    np.testing.assert_allclose(lse[:, :, 0], s * np.einsum("bhx,bhx->bh", q[:, :, 0], k[:, :, 0]),
+                               atol=1e-13)
+
+
+def test_single_key():
+    q, k, v, do = (rand((1, 2, 1, 8), s) for s in range(4))
+    o, lse = oracle.attention_forward(q, k, v, 0.3)
+    assert np.array_equal(o, v)
+    dq, dk, dv, _ = oracle.attention_backward(q, k, v, do, 0.3)
+    assert np.all(dq == 0) and np.all(dk == 0)
+    assert np.array_equal(dv, do)
+
+
+def test_value_identity_gives_probability_rows():
+    # with V = I (d = N) the output row is the probability row itself: rows sum to 1,
+    # entries are non-negative and zero exactly on masked keys
+    N = 256
+    q, k = rand((1, 1, N, N), 8), rand((1, 1, N, N), 9)
+    v = np.eye(N)[None, None]
+    bm = np.array([[1, 0], [1, 1]], np.uint8)
+    for causal, kv, m in [(False, None, None), (True, None, None), (False, 100, None),
+                          (True, 200, bm)]:
+        kvl = None if kv is None else np.array([kv], np.int32)
+        p, _ = oracle.attention_forward(q, k, v, 0.05, causal=causal, block_mask=m, kv_len=kvl)
+        p = p[0, 0]
+        np.testing.assert_allclose(p.sum(axis=1), 1.0, atol=1e-14)
+        assert np.all(p >= 0)
+        for r in range(N):
+            for c in range(N):
+                ok = (not causal or c <= r) and (kv is None or c < kv) and \
+                     (m is None or m[r // 128, c // 128])
+                if not ok:
+                    assert p[r, c] == 0.0
+
+
+# ---------------------------------------------------------------------------
+# invariants
+# ---------------------------------------------------------------------------
+
+def test_joint_key_value_permutation():
+    B, H, N, d = 1, 2, 200, 16
+    q, k, v, do = (rand((B, H, N, d), s) for s in (10, 11, 12, 13))
+    perm = np.random.default_rng(14).permutation(N)
+    o1, l1 = oracle.attention_forward(q, k, v, 0.25)
+    o2, l2 = oracle.attention_forward(q, k[:, :, perm], v[:, :, perm], 0.25)
+    np.testing.assert_allclose(o1, o2, atol=1e-12)
+    np.testing.assert_allclose(l1, l2, atol=1e-12)
+    _, dk1, dv1, _ = oracle.attention_backward(q, k, v, do, 0.25)
+    _, dk2, dv2, _ = oracle.attention_backward(q, k[:, :, perm], v[:, :, perm], do, 0.25)
+    np.testing.assert_allclose(dk1[:, :, perm], dk2, atol=1e-12)
+    np.testing.assert_allclose(dv1[:, :, perm], dv2, atol=1e-12)
+
+
+def test_key_shift_shifts_lse_only():
+    B, H, N, d = 1, 1, 160, 8
+    q, k, v = (rand((B, H, N, d), s) for s in (15, 16, 17))
+    c = rand((d,), 18)
+    s = 0.3
+    o1, l1 = oracle.attention_forward(q, k, v, s, causal=True)
+    o2, l2 = oracle.attention_forward(q, k + c, v, s, causal=True)
+    np.testing.assert_allclose(o1, o2, atol=1e-12)
+    np.testing.assert_allclose(l2 - l1, s * q @ c, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal,kv", [(False, None), (True, None), (False, 150)])
+def test_gradient_sum_rules(causal, kv):
+    B, H, N, d = 1, 2, 256, 16
+    q, k, v, do = (rand((B, H, N, d), s) for s in (19, 20, 21, 22))
+    kvl = None if kv is None else np.array([kv], np.int32)
+    dq, dk, dv, delta = oracle.attention_backward(q, k, v, do, 0.2, causal=causal, kv_len=kvl)
+    # P rows sum to 1, so the value gradients add up to the output gradients
+    np.testing.assert_allclose(dv.sum(axis=2), do.sum(axis=2), atol=1e-11)
+    # sum_c dS_rc = D_r - D_r = 0, so the key gradients add up to 0 per head
+    np.testing.assert_allclose(dk.sum(axis=2), 0.0, atol=1e-11)
+    if kv is not None:
+        assert np.all(dk[:, :, kv:] == 0) and np.all(dv[:, :, kv:] == 0)
+    # D_r = sum_c P dP equals rowsum(dO * O)
+    o, _ = oracle.attention_forward(q, k, v, 0.2, causal=causal, kv_len=kvl)
+    np.testing.assert_allclose(delta, (do * o).sum(axis=3), atol=1e-12)
+
+
+def test_fully_masked_rows():
+    # causal with the first diagonal tile masked out: rows 0..127 see no key
+    B, H, N, d = 1, 1, 256, 8
+    q, k, v, do = (rand((B, H, N, d), s) for s in (23, 24, 25, 26))
+    bm = np.array([[0, 1], [1, 1]], np.uint8)
+    o, lse = oracle.attention_forward(q, k, v, 0.5, causal=True, block_mask=bm)
+    assert np.all(o[0, 0, :128] == 0) and np.all(np.isneginf(lse[0, 0, :128]))
+    assert np.all(np.isfinite(lse[0, 0, 128:]))
+    dq, dk, dv, _ = oracle.attention_backward(q, k, v, do, 0.5, causal=True, block_mask=bm)
+    assert np.all(dq[0, 0, :128] == 0)
+    assert np.all(np.isfinite(dk)) and np.all(np.isfinite(dv))
+
+
+# ---------------------------------------------------------------------------
+# brute force: finite differences of L = sum(O * dO)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("causal,kv", [(False, None), (True, None), (False, 11)])
+def test_finite_difference_gradients(causal, kv):
+    N, d, s = 16, 8, 0.4
+    q, k, v, do = (rand((1, 1, N, d), t) for t in (27, 28, 29, 30))
+    kvl = None if kv is None else np.array([kv], np.int32)
+
+    def loss(qq, kk, vv):
+        o, _ = oracle.attention_forward(qq, kk, vv, s, causal=causal, kv_len=kvl, nthreads=1)
+        return float((o * do).sum())
+
+    dq, dk, dv, _ = oracle.attention_backward(q, k, v, do, s, causal=causal, kv_len=kvl)
+    h = 1e-6
+    for which, grad in ((0, dq), (1, dk), (2, dv)):
+        num = np.zeros_like(grad)
+        for r in range(N):
+            for x in range(d):
+                args_p = [q.copy(), k.copy(), v.copy()]
+                args_m = [q.copy(), k.copy(), v.copy()]
+                args_p[which][0, 0, r, x] += h
+                args_m[which][0, 0, r, x] -= h
+                num[0, 0, r, x] = (loss(*args_p) - loss(*args_m)) / (2 * h)
+        err = np.linalg.norm(num - grad) / max(np.linalg.norm(grad), 1e-300)
+        assert err < 1e-7, (which, err)
+
+
+# ---------------------------------------------------------------------------
+# the pages' mechanism: tiled online softmax reaches the same numbers
+# ---------------------------------------------------------------------------
+
+def online_softmax_tiled(q, k, v, scale, causal, Br=32, Bc=48):
+    """Tiles of keys visited one at a time, keeping a running row max and row sum and
+    rescaling the partial output whenever the max grows (opendecode.dev summary,
+    'The key idea').  Test-only; unrelated to the oracle's code."""
+    N, d = q.shape
+    o = np.zeros((N, d))
+    lse = np.zeros(N)
+    for r0 in range(0, N, Br):
+        qi = q[r0:r0 + Br]
+        rows = np.arange(r0, min(r0 + Br, N))
+        m = np.full(len(rows), -np.inf)
+        l = np.zeros(len(rows))
+        acc = np.zeros((len(rows), d))
+        for c0 in range(0, N, Bc):
+            cols = np.arange(c0, min(c0 + Bc, N))
+            sc = scale * qi @ k[cols].T
+            if causal:
+                sc = np.where(cols[None, :] <= rows[:, None], sc, -np.inf)
+            m_new = np.maximum(m, sc.max(axis=1))
+            safe = np.where(np.isinf(m_new), 0.0, m_new)
+            alpha = np.exp(m - safe)
+            p = np.exp(sc - safe[:, None])
+            l = alpha * l + p.sum(axis=1)
+            acc = alpha[:, None] * acc + p @ v[cols]
+            m = m_new
+        o[rows] = acc / l[:, None]
+        lse[rows] = m + np.log(l)
+    return o, lse
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_online_softmax_matches_oracle(causal):
+    N, d = 230, 24
+    q, k, v = (rand((N, d), t) * 2 for t in (31, 32, 33))
+    o_t, l_t = online_softmax_tiled(q, k, v, 0.3, causal)
+    o, l = oracle.attention_forward(q[None, None], k[None, None], v[None, None], 0.3,
+                                    causal=causal)
+    np.testing.assert_allclose(o[0, 0], o_t, atol=1e-12)
+    np.testing.assert_allclose(l[0, 0], l_t, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# row-subset forward and tile visits
+# ---------------------------------------------------------------------------
+
+def test_forward_rows_match_full_forward():
+    N, d = 512, 16
+    q, k, v = (rand((1, 1, N, d), t) for t in (34, 35, 36))
+    bm = np.array([[1, 0, 0, 1], [1, 1, 0, 0], [0, 0, 1, 0], [1, 0, 1, 1]], np.uint8)
+    rows = np.array([0, 5, 130, 300, 511])
+    for causal, kv in [(False, None), (True, 333)]:
+        kvl = None if kv is None else np.array([kv], np.int32)
+        o, l = oracle.attention_forward(q, k, v, 0.2, causal=causal, block_mask=bm, kv_len=kvl)
+        orow, lrow = oracle.attention_forward_rows(q[0, 0, rows], rows, k[0, 0], v[0, 0], 0.2,
+                                                   causal=causal, block_mask=bm, kv_len_b=kv)
+        assert np.array_equal(orow, o[0, 0, rows]) and np.array_equal(lrow, l[0, 0, rows])
+
+
+def test_tile_visits_hand_enumerated():
+    # N = 512 -> 4 x 4 tiles.  Written out by hand from the mask definition.
+    causal_only = oracle.tile_visits(1, 512, causal=True)[0]
+    assert causal_only.tolist() == [[1, 0, 0, 0], [1, 1, 0, 0], [1, 1, 1, 0], [1, 1, 1, 1]]
+    # keys < 200 live in key tiles 0 and 1 (tile 1 holds keys 128..255)
+    kv = oracle.tile_visits(2, 512, kv_len=np.array([200, 512], np.int32))
+    assert kv[0].tolist() == [[1, 1, 0, 0]] * 4
+    assert kv[1].tolist() == [[1, 1, 1, 1]] * 4
+    both = oracle.tile_visits(1, 512, causal=True, kv_len=np.array([129], np.int32))[0]
+    assert both.tolist() == [[1, 0, 0, 0], [1, 1, 0, 0], [1, 1, 0, 0], [1, 1, 0, 0]]
+    bm = np.array([[1, 1, 0, 0], [0, 1, 0, 1], [1, 0, 0, 0], [0, 0, 1, 1]], np.uint8)
+    masked = oracle.tile_visits(1, 512, causal=True, block_mask=bm)[0]
+    assert masked.tolist() == [[1, 0, 0, 0], [0, 1, 0, 0], [1, 0, 0, 0], [0, 0, 1, 1]]
+    part = oracle.tile_visits(1, 512, causal=True, block_mask=bm, i_begin=2, i_end=4)[0]
+    assert part.tolist() == masked[2:].tolist()
+
+
+def test_tile_visits_agree_with_value_identity_probabilities():
+    # a tile pair is visited exactly when some probability inside it can be nonzero
+    N = 384
+    q, k = rand((1, 1, N, N), 37) * 0.01, rand((1, 1, N, N), 38) * 0.01
+    v = np.eye(N)[None, None]
+    bm = np.array([[1, 0, 1], [0, 1, 1], [1, 1, 0]], np.uint8)
+    kvl = np.array([300], np.int32)
+    p, _ = oracle.attention_forward(q, k, v, 1.0, causal=True, block_mask=bm, kv_len=kvl)
+    vis = oracle.tile_visits(1, N, causal=True, block_mask=bm, kv_len=kvl)[0]
+    for i in range(3):
+        for j in range(3):
+            blk = p[0, 0, i * 128:(i + 1) * 128, j * 128:(j + 1) * 128]
+            assert bool(vis[i, j]) == bool(np.any(blk > 0)), (i, j)
