@@ -1,0 +1,514 @@
+#!/usr/bin/env python
+"""Benchmark of the exact tiled attention path on B200: forward and forward+backward
+TFLOP/s and fraction of the B200 dense BF16 tensor peak.
+
+One step = one fa_fwd (O, LSE) and one fa_bwd (its three launches: preprocess,
+main, dQ conversion) over one batch of the chosen workload, with inputs
+resident in HBM.  FLOPs follow the metric's convention: 4*B*H*N^2*d for the
+forward (halved for causal masks, scaled by the kept-tile density for block
+masks and by sum(kv_len)/(B*N) for key padding), and 2.5 times that for the
+backward.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...     # the FP64 CPU oracle, timed
+
+Multi-GPU (under torchrun): every rank runs its own copy of the workload on
+its own GPU (independent problems, no data-path collective); the reported
+value is the FLOPs of all ranks over the slowest rank's time ("weak" scaling).
+Rank 0 prints one JSON line.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd and fwd+bwd TFLOP/s and % of B200 BF16 tensor peak"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DATASHEET_BF16_TFLOPS = 2250.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ----------------------------------------------------------------------------
+# workload arithmetic (metric convention)
+# ----------------------------------------------------------------------------
+
+def density(x):
+    """Fraction of the N x N score matrix the metric counts (mask-dependent)."""
+    B, H, N, d = x.q.shape
+    f = 1.0
+    if x.causal:
+        f *= 0.5
+    if x.block_mask is not None:
+        f *= float(x.block_mask.double().mean())
+    if x.kv_len is not None:
+        f *= float(x.kv_len.double().sum()) / (B * N)
+    return f
+
+
+def flops_fwd(x):
+    B, H, N, d = x.q.shape
+    return 4.0 * B * H * N * N * d * density(x)
+
+
+def ideal_bytes(x):
+    """Each input read once and each output written once (bytes)."""
+    B, H, N, d = x.q.shape
+    E, R = B * H * N * d, B * H * N
+    fwd = 3 * 2 * E + 2 * E + 4 * R                    # Q, K, V in; O, LSE out
+    bwd_main = 4 * 2 * E + 2 * 4 * R + 2 * 2 * E + 2 * 4 * E   # Q K V dO, lse2 D in; dK dV out; dQ acc
+    return fwd, bwd_main
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "exact_io_aware_63_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode())
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    ent = rec.get(workload, {}).get(kernel)
+    if not ent or ent.get("source_hash") != kernel_source_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------
+# clocks (nvidia-smi sampled during the load)
+# ----------------------------------------------------------------------------
+
+REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+
+class ClockSampler:
+    def __init__(self, index):
+        self.proc = None
+        self.index = index
+        self.path = None
+
+    def start(self):
+        q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             + ",".join("clocks_event_reasons." + r for r in REASONS))
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.index)], stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self, t_begin, t_end):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 10:
+                    continue
+                try:
+                    ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                    rows.append((ts, float(parts[2]), float(parts[3]), parts[6:10]))
+                except Exception:
+                    continue
+        os.unlink(self.path)
+        window = [r for r in rows if t_begin - 0.05 <= r[0] <= t_end + 0.05]
+        if not window:
+            window = rows
+        if not window:
+            return None
+        reasons = sorted({REASONS[i] for r in window for i, v in enumerate(r[3])
+                          if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[1] for r in window),
+                "sm_max_mhz": max(r[2] for r in window), "reasons": reasons,
+                "samples": len(window)}
+
+
+# ----------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    from exact_io_aware_63_b200 import binding, inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    binding.load(build_if_missing=False)
+
+    w = inputs.WORKLOADS[args.workload]
+    x = inputs.workload_inputs(args.workload)
+    B, H, N, d = x.q.shape
+    q, k, v, do = (t.to(dev) for t in (x.q, x.k, x.v, x.dout))
+    bm = None if x.block_mask is None else x.block_mask.to(dev)
+    kl = None if x.kv_len is None else x.kv_len.to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    ws_bytes = binding.fa_bwd_workspace_size(B, H, N, d)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    S = stream.cuda_stream
+    scale, causal = x.scale, x.causal
+
+    def check(rc, what):
+        if rc != 0:
+            raise RuntimeError(f"{what}: {binding.fa_status_string(rc)}")
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        check(binding.fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, bm, kl, S), "fa_fwd")
+        if ev is not None:
+            ev[1].record(stream)
+        for ph in range(3):
+            check(binding.fa_bwd_phase(ph, q, k, v, o, lse, do, dq, dk, dv, B, H, N, d, scale,
+                                       causal, bm, kl, ws, ws_bytes, S), "fa_bwd_phase")
+            if ev is not None:
+                ev[2 + ph].record(stream)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = binding.fa_get_device_status(S)
+    if st != 0:
+        raise RuntimeError("device status after warm-up: " + binding.fa_status_string(st))
+
+    cvd = os.environ.get("CUDA_VISIBLE_DEVICES")
+    smi_id = cvd.split(",")[local].strip() if cvd else str(local)
+    sampler = ClockSampler(smi_id)
+    sampler.start()
+    time.sleep(0.3)
+    t_load0 = time.time()
+    # untimed sustained load so that clock samples see the kernels running
+    t_end_sustain = time.time() + args.clock_window
+    while time.time() < t_end_sustain:
+        for _ in range(8):
+            flush.zero_()
+            step()
+        torch.cuda.synchronize()
+
+    n_ev = 5
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    for kk in range(args.steps):
+        flush.zero_()                      # L2 flushed between timed steps
+        step(evs[kk])
+    torch.cuda.synchronize()
+    barrier()
+    t1 = time.time()
+    clocks = sampler.stop(t_load0, t1)
+    st = binding.fa_get_device_status(S)
+    if st != 0:
+        raise RuntimeError("device status after timing: " + binding.fa_status_string(st))
+
+    step_ms = [e[0].elapsed_time(e[4]) for e in evs]
+    fwd_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    pre_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    main_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    post_ms = [e[3].elapsed_time(e[4]) for e in evs]
+    mean = lambda a: sum(a) / len(a)
+    m = torch.tensor([mean(step_ms), mean(fwd_ms), mean(pre_ms), mean(main_ms), mean(post_ms)],
+                     dtype=torch.float64, device=dev)
+    if dist is not None:
+        dist.all_reduce(m, op=dist.ReduceOp.MAX)
+    step_t, fwd_t, pre_t, main_t, post_t = (float(t) for t in m.cpu())
+
+    # ---------------------------------------------------------------- e2e
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv, hdo = (t.pin_memory() for t in (x.q, x.k, x.v, x.dout))
+        ho, hdq, hdk, hdv = (torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+                             for _ in range(4))
+        hlse = torch.empty((B, H, N), dtype=torch.float32).pin_memory()
+        e2e_steps = max(1, min(args.steps, 20))
+        for it in range(2 + e2e_steps):
+            if it == 2:
+                barrier()
+                torch.cuda.synchronize()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            do.copy_(hdo, non_blocking=True)
+            check(binding.fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, bm, kl, S), "fa_fwd")
+            check(binding.fa_bwd(q, k, v, o, lse, do, dq, dk, dv, B, H, N, d, scale, causal, bm, kl,
+                                 ws, ws_bytes, S), "fa_bwd")
+            ho.copy_(o, non_blocking=True)
+            hlse.copy_(lse, non_blocking=True)
+            hdq.copy_(dq, non_blocking=True)
+            hdk.copy_(dk, non_blocking=True)
+            hdv.copy_(dv, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = torch.tensor([e0.elapsed_time(e1) / e2e_steps], dtype=torch.float64, device=dev)
+        if dist is not None:
+            dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+        e2e_ms = float(e2e_ms)
+        E, R = B * H * N * d, B * H * N
+        h2d = 4 * 2 * E
+        d2h = 4 * 2 * E + 4 * R
+        total_flops = 3.5 * flops_fwd(x) * world
+        e2e = {"value": total_flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    # ---------------------------------------------------------------- report
+    peaks, peak_kind = load_peaks()
+    ff = flops_fwd(x)
+    fb = 2.5 * ff
+    value = 3.5 * ff * world / (step_t * 1e-3) / 1e12
+    fwd_tflops = ff / (fwd_t * 1e-3) / 1e12
+    main_tflops = fb / (main_t * 1e-3) / 1e12
+    bwd_tflops = fb / ((pre_t + main_t + post_t) * 1e-3) / 1e12
+    per_gpu = value / world
+    # dominant kernel by time: the backward main kernel or the forward kernel
+    if main_t >= fwd_t:
+        dom, dom_t, dom_flops, dom_bytes = "fa_bwd_kernel", main_t, fb, ideal_bytes(x)[1]
+    else:
+        dom, dom_t, dom_flops, dom_bytes = "fa_fwd_kernel", fwd_t, ff, ideal_bytes(x)[0]
+    achieved = dom_flops / (dom_t * 1e-3) / 1e12
+    roofline = {"kernel": dom, "bound": "tensor", "achieved": achieved,
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"],
+                "peak_source": f"{peak_kind} bf16_tflops (burst)",
+                "traffic": ncu_traffic(dom, args.workload),
+                "algorithmic_bytes": dom_bytes,
+                "algorithmic_flops": dom_flops,
+                "ms_per_launch": dom_t}
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_t, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "description": w.description,
+                   "B": B, "H": H, "N": N, "d": d, "causal": causal,
+                   "key_padding": x.kv_len is not None, "block_sparse": x.block_mask is not None,
+                   "flop_density": density(x), "seed": w.seed,
+                   "l2": "flushed between timed steps (256 MiB write)",
+                   "parallelism": f"replica x{world}"},
+        "fwd_tflops": fwd_tflops,
+        "bwd_tflops": bwd_tflops,
+        "fwd_bwd_pct_of_peak": per_gpu / peaks["bf16_tflops"],
+        "fwd_pct_of_peak": fwd_tflops / peaks["bf16_tflops"],
+        "peak_bf16_tflops": peaks["bf16_tflops"], "peak_source": peak_kind,
+        "datasheet_bf16_tflops": DATASHEET_BF16_TFLOPS,
+        "ms": {"fwd": fwd_t, "bwd_pre": pre_t, "bwd_main": main_t, "bwd_dq": post_t},
+        "bwd_main_tflops": main_tflops,
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": 4 * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(x, budget_s=args.cpu_budget)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------
+# the FP64 CPU oracle, timed on a bounded sample
+# ----------------------------------------------------------------------------
+
+def allowed_entries(x, rows):
+    """Allowed (row, key) entries of one head for the given query rows, per batch."""
+    import numpy as np
+    B, H, N, d = x.q.shape
+    rows = np.asarray(rows)
+    tot = np.zeros(B)
+    c = np.arange(N)
+    bm = None if x.block_mask is None else x.block_mask.numpy().astype(bool)
+    for b in range(B):
+        L = N if x.kv_len is None else int(x.kv_len[b])
+        for r in rows:
+            ok = c < L
+            if x.causal:
+                ok &= c <= r
+            if bm is not None:
+                ok &= np.repeat(bm[r // 128], 128)
+            tot[b] += ok.sum()
+    return tot
+
+
+def oracle_sample(x, n_heads, n_rows):
+    """The first n_heads heads (batch-major) and query rows [0, n_rows) of each."""
+    import torch
+    B, H, N, d = x.q.shape
+    heads = [(b, h) for b in range(B) for h in range(H)][:n_heads]
+    sel = lambda t: torch.stack([t[b, h] for b, h in heads])[:, None].to(torch.float64).numpy()
+    kl = None if x.kv_len is None else [int(x.kv_len[b]) for b, _ in heads]
+    return heads, sel(x.q), sel(x.k), sel(x.v), sel(x.dout), kl
+
+
+def time_oracle(x, n_heads, n_rows, threads):
+    import numpy as np
+    import oracle
+    heads, q, k, v, do, kl = oracle_sample(x, n_heads, n_rows)
+    bm = None if x.block_mask is None else x.block_mask.numpy()
+    kl = None if kl is None else np.array(kl, np.int32)
+    t0 = time.perf_counter()
+    oracle.attention_forward_band(q, k, v, x.scale, x.causal, bm, kl, 0, n_rows, threads)
+    oracle.attention_backward_band(q, k, v, do, x.scale, x.causal, bm, kl, 0, n_rows, threads)
+    dt = time.perf_counter() - t0
+    # metric FLOPs of the sample: the workload's per-entry rate times the sample's entries
+    B, H, N, d = x.q.shape
+    per_b = allowed_entries(x, range(n_rows))
+    entries = sum(per_b[b] for b, _ in heads)
+    all_entries = allowed_entries(x, range(N)).sum() * H
+    flops = 3.5 * flops_fwd(x) * entries / all_entries
+    return dt, flops, heads
+
+
+def sample_plan(x, threads):
+    B, H, N, d = x.q.shape
+    n_rows = N if N <= 4096 else 256
+    n_heads = min(B * H, max(1, threads))
+    return n_heads, n_rows
+
+
+def cpu_baseline(x, budget_s=20.0):
+    """Oracle throughput on a bounded sample: whole heads (or a band of rows for
+    N > 4096), grown until about budget_s CPU-seconds of work."""
+    threads = os.cpu_count() or 1
+    B, H, N, d = x.q.shape
+    n_heads, n_rows = sample_plan(x, threads)
+    while True:
+        dt, flops, heads = time_oracle(x, n_heads, n_rows, threads)
+        used = min(threads, len(heads))
+        if dt * used >= budget_s or (n_heads >= B * H and n_rows >= N) or dt > budget_s:
+            break
+        if n_heads < B * H:
+            n_heads = min(B * H, n_heads * 2)
+        else:
+            n_rows = min(N, n_rows * 2)
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": used, "kind": "oracle",
+            "host_cpus": threads, "seconds": dt,
+            "sample": f"FP64 oracle fwd+bwd on {len(heads)} of {B * H} heads, query rows "
+                      f"0..{n_rows - 1} of {N} (FLOPs counted as the metric counts them)"}
+
+
+def run_reference(args):
+    """The reference arm: the FP64 CPU oracle (as it stands) on the same workload, metric
+    and unit, one bounded sample per step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from exact_io_aware_63_b200 import inputs
+    w = inputs.WORKLOADS[args.workload]
+    x = inputs.workload_inputs(args.workload)
+    threads = os.cpu_count() or 1
+    B, H, N, d = x.q.shape
+    n_heads, n_rows = sample_plan(x, threads)
+    n_heads = min(n_heads, B * H)
+    for _ in range(args.warmup):
+        time_oracle(x, n_heads, n_rows, threads)
+    times, flops = [], 0.0
+    for _ in range(args.steps):
+        dt, flops, heads = time_oracle(x, n_heads, n_rows, threads)
+        times.append(dt)
+    ms = 1e3 * sum(times) / len(times)
+    value = flops / (ms * 1e-3) / 1e12
+    used = min(threads, n_heads)
+    sample = (f"FP64 oracle fwd+bwd on {n_heads} of {B * H} heads, query rows 0..{n_rows - 1} "
+              f"of {N}")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": args.workload, "description": w.description, "B": B, "H": H,
+                       "N": N, "d": d, "parallelism": "cpu threads"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": used, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="bert")
+    ap.add_argument("--clock-window", type=float, default=1.5,
+                    help="seconds of untimed load before timing, sampled for clocks")
+    ap.add_argument("--cpu-budget", type=float, default=20.0,
+                    help="CPU-seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("note: warm-up raised to 3 steps", file=sys.stderr)
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

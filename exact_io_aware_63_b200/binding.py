@@ -1,0 +1,198 @@
+"""ctypes binding of libfa_b200.so: the C ABI of ``include/fa.h`` with the same names.
+
+Argument marshalling only.  Tensors are torch CUDA tensors (device memory and
+streams come from PyTorch); every step of the attention path runs in the
+library's kernels.  There is no fallback: if the library is missing the
+import of a function raises.
+
+Raw entry points (same argument order as the C ABI; tensors are passed as
+torch tensors or None, the stream as a torch.cuda.Stream or None = current):
+``fa_fwd``, ``fa_fwd_traced``, ``fa_bwd``, ``fa_bwd_traced``, ``fa_bwd_phase``,
+``fa_bwd_workspace_size``, ``fa_get_device_status``, ``fa_status_string``,
+``fa_version``.
+
+Convenience wrappers that allocate outputs: ``attention_forward`` and
+``attention_backward``.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+from . import build as _build
+
+_lock = threading.Lock()
+_lib = None
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_f = ctypes.c_float
+_sz = ctypes.c_size_t
+
+_SIGS = {
+    "fa_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _vp, _vp]),
+    "fa_fwd_traced": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _vp, _vp, _vp]),
+    "fa_bwd_workspace_size": (_sz, [_i, _i, _i, _i]),
+    "fa_bwd": (_i, [_vp] * 9 + [_i, _i, _i, _i, _f, _i, _vp, _vp, _vp, _sz, _vp]),
+    "fa_bwd_traced": (_i, [_vp] * 9 + [_i, _i, _i, _i, _f, _i, _vp, _vp, _vp, _sz, _vp, _vp]),
+    "fa_bwd_phase": (_i, [_i] + [_vp] * 9 + [_i, _i, _i, _i, _f, _i, _vp, _vp, _vp, _sz, _vp]),
+    "fa_get_device_status": (_i, [_vp]),
+    "fa_status_string": (ctypes.c_char_p, [_i]),
+    "fa_version": (_i, []),
+}
+
+FA_OK = 0
+STATUS_NAMES = {0: "FA_OK", -1: "FA_ERR_NULL", -2: "FA_ERR_ALIGN", -3: "FA_ERR_SHAPE",
+                -4: "FA_ERR_UNSUPPORTED_D", -5: "FA_ERR_WORKSPACE", -6: "FA_ERR_CUDA",
+                -7: "FA_ERR_TIMEOUT", -8: "FA_ERR_ARG"}
+
+
+class FAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)} ({lib_status_string(status)})")
+        self.status = status
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def load(build_if_missing: bool = True):
+    """Load libfa_b200.so (building it first if it is missing or stale)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if build_if_missing and _build.needs_build():
+                _build.build()
+            if not os.path.exists(_build.LIB):
+                raise ImportError(f"{_build.LIB} is missing; run python -m exact_io_aware_63_b200.build")
+            lib = ctypes.CDLL(_build.LIB)
+            for name, (res, args) in _SIGS.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = lib
+    return _lib
+
+
+def lib_status_string(status: int) -> str:
+    return load().fa_status_string(int(status)).decode()
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+# ----------------------------------------------------------------------------
+# raw C-ABI calls (same names and argument order)
+# ----------------------------------------------------------------------------
+
+def fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, block_mask, kv_len, stream=None):
+    return load().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, float(scale),
+                         int(bool(causal)), _ptr(block_mask), _ptr(kv_len), _stream(stream))
+
+
+def fa_fwd_traced(q, k, v, o, lse, B, H, N, d, scale, causal, block_mask, kv_len, visited,
+                  stream=None):
+    return load().fa_fwd_traced(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
+                                float(scale), int(bool(causal)), _ptr(block_mask), _ptr(kv_len),
+                                _ptr(visited), _stream(stream))
+
+
+def fa_bwd_workspace_size(B, H, N, d):
+    return load().fa_bwd_workspace_size(B, H, N, d)
+
+
+def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, block_mask, kv_len,
+           workspace, workspace_bytes, stream=None):
+    return load().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq),
+                         _ptr(dk), _ptr(dv), B, H, N, d, float(scale), int(bool(causal)),
+                         _ptr(block_mask), _ptr(kv_len), _ptr(workspace), int(workspace_bytes),
+                         _stream(stream))
+
+
+def fa_bwd_traced(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, block_mask, kv_len,
+                  workspace, workspace_bytes, visited, stream=None):
+    return load().fa_bwd_traced(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
+                                _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, float(scale),
+                                int(bool(causal)), _ptr(block_mask), _ptr(kv_len), _ptr(workspace),
+                                int(workspace_bytes), _ptr(visited), _stream(stream))
+
+
+def fa_bwd_phase(phase, q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, block_mask,
+                 kv_len, workspace, workspace_bytes, stream=None):
+    return load().fa_bwd_phase(int(phase), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                               _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, float(scale),
+                               int(bool(causal)), _ptr(block_mask), _ptr(kv_len), _ptr(workspace),
+                               int(workspace_bytes), _stream(stream))
+
+
+def fa_get_device_status(stream=None):
+    return load().fa_get_device_status(_stream(stream))
+
+
+def fa_status_string(status):
+    return lib_status_string(status)
+
+
+def fa_version():
+    return load().fa_version()
+
+
+# ----------------------------------------------------------------------------
+# convenience wrappers (allocate outputs with torch, then call the C ABI)
+# ----------------------------------------------------------------------------
+
+def _check(rc, what):
+    if rc != FA_OK:
+        raise FAError(rc, what)
+
+
+def attention_forward(q, k, v, scale, causal=False, block_mask=None, kv_len=None, visited=None,
+                      stream=None):
+    """O, LSE for bf16 CUDA tensors q, k, v of shape [B, H, N, d]."""
+    import torch
+    B, H, N, d = q.shape
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    if visited is None:
+        rc = fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, block_mask, kv_len, stream)
+    else:
+        rc = fa_fwd_traced(q, k, v, o, lse, B, H, N, d, scale, causal, block_mask, kv_len,
+                           visited, stream)
+    _check(rc, "fa_fwd")
+    return o, lse
+
+
+def attention_backward(q, k, v, o, lse, dout, scale, causal=False, block_mask=None, kv_len=None,
+                       workspace=None, visited=None, stream=None):
+    """dQ, dK, dV for the forward that produced (o, lse)."""
+    import torch
+    B, H, N, d = q.shape
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws_bytes = fa_bwd_workspace_size(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    if visited is None:
+        rc = fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, block_mask,
+                    kv_len, workspace, workspace.numel(), stream)
+    else:
+        rc = fa_bwd_traced(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal,
+                           block_mask, kv_len, workspace, workspace.numel(), visited, stream)
+    _check(rc, "fa_bwd")
+    return dq, dk, dv

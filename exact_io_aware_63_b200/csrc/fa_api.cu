@@ -1,0 +1,342 @@
+// fa_api.cu - the C ABI declared in include/fa.h: argument checks, TMA tensor
+// map encoding, work-unit counts and kernel launches.  All arithmetic of the
+// attention path runs in the kernels of fa_fwd.cuh and fa_bwd.cuh.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fa.h"
+#include "fa_bwd.cuh"
+#include "fa_fwd.cuh"
+
+namespace {
+
+constexpr int kVersion = 10000;  // 1.0.0
+
+// ---------------------------------------------------------------------------
+// driver entry point for tensor-map encoding (no link-time libcuda dependency)
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// [rows][d] bf16 tensor, boxes of 128 rows x 64 columns, 128-byte swizzle.
+bool make_tmap(CUtensorMap* m, const void* base, long long rows, int d) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Shape checks shared by every entry point.  Returns FA_OK, an error, or 1
+// for "empty problem: nothing to do".
+int check_shape(int B, int H, int N, int d) {
+  if (B < 0 || H < 0 || N < 0) return FA_ERR_SHAPE;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED_D;
+  if (N % fa::kTile != 0) return FA_ERR_SHAPE;
+  if (B == 0 || H == 0 || N == 0) return 1;
+  const long long rows = static_cast<long long>(B) * H * N;
+  if (rows >= (1LL << 31)) return FA_ERR_SHAPE;
+  return FA_OK;
+}
+
+int check_scale(float scale) {
+  return (std::isfinite(scale) && scale > 0.f) ? FA_OK : FA_ERR_ARG;
+}
+
+// Makes the device that owns `ptr` current for this runtime instance and
+// returns its SM count (0 on failure).
+int select_device(const void* ptr) {
+  cudaPointerAttributes attr;
+  if (cudaPointerGetAttributes(&attr, ptr) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  int dev = attr.device;
+  if (dev < 0) return 0;
+  if (cudaSetDevice(dev) != cudaSuccess) return 0;
+  static int sm_count[64] = {0};
+  if (dev < 64 && sm_count[dev]) return sm_count[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev < 64) sm_count[dev] = n;
+  return n;
+}
+
+template <typename Kernel>
+bool set_smem(Kernel k, int bytes) {
+  return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct WsLayout {
+  size_t delta, lse2, dq_acc, total;
+};
+
+WsLayout ws_layout(int B, int H, int N, int d) {
+  const size_t R = static_cast<size_t>(B) * H * N;
+  WsLayout w;
+  w.delta = 0;
+  w.lse2 = round_up(w.delta + 4 * R, 256);
+  w.dq_acc = round_up(w.lse2 + 4 * R, 256);
+  w.total = round_up(w.dq_acc + 4 * R * d, 256);
+  return w;
+}
+
+template <int D>
+int launch_fwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o, float* lse, int B,
+               int H, int N, float scale, int causal, const uint8_t* block_mask,
+               const int32_t* kv_len, uint8_t* visited, cudaStream_t stream, int num_sms) {
+  using Cfg = fa::FwdCfg<D>;
+  const long long rows = static_cast<long long>(B) * H * N;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap(&tq, q, rows, D) || !make_tmap(&tk, k, rows, D) || !make_tmap(&tv, v, rows, D))
+    return FA_ERR_CUDA;
+  static bool smem_set = false;
+  if (!smem_set) {
+    if (!set_smem(fa::fa_fwd_kernel<D>, Cfg::kSmemBytes)) return FA_ERR_CUDA;
+    smem_set = true;
+  }
+  fa::FwdParams p;
+  p.o = o;
+  p.lse = lse;
+  p.block_mask = block_mask;
+  p.kv_len = kv_len;
+  p.visited = visited;
+  p.B = B;
+  p.H = H;
+  p.N = N;
+  p.n_t = N / fa::kTile;
+  p.num_pairs = (p.n_t + 1) / 2;
+  p.num_units = B * H * p.num_pairs;
+  p.causal = causal ? 1 : 0;
+  p.scale_log2 = scale * fa::kLog2e;
+  const int grid = p.num_units < num_sms ? p.num_units : num_sms;
+  fa::fa_fwd_kernel<D><<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <int D>
+int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf16* o,
+               const float* lse, const fa_bf16* dout, fa_bf16* dq, fa_bf16* dk, fa_bf16* dv, int B,
+               int H, int N, float scale, int causal, const uint8_t* block_mask,
+               const int32_t* kv_len, void* workspace, uint8_t* visited, cudaStream_t stream,
+               int num_sms, unsigned phases) {
+  using Cfg = fa::BwdCfg<D>;
+  const long long rows = static_cast<long long>(B) * H * N;
+  const WsLayout wl = ws_layout(B, H, N, D);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* delta = reinterpret_cast<float*>(ws + wl.delta);
+  float* lse2 = reinterpret_cast<float*>(ws + wl.lse2);
+  float* dq_acc = reinterpret_cast<float*>(ws + wl.dq_acc);
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_tmap(&tq, q, rows, D) || !make_tmap(&tk, k, rows, D) || !make_tmap(&tv, v, rows, D) ||
+      !make_tmap(&tdo, dout, rows, D))
+    return FA_ERR_CUDA;
+  static bool smem_set = false;
+  if (!smem_set) {
+    if (!set_smem(fa::fa_bwd_kernel<D>, Cfg::kSmemBytes)) return FA_ERR_CUDA;
+    smem_set = true;
+  }
+  // preprocess
+  if (phases & 1u) {
+    const int threads = 256;
+    long long blocks = (rows * (D / 4) + threads - 1) / threads;
+    const long long cap = static_cast<long long>(num_sms) * 8;
+    if (blocks > cap) blocks = cap;
+    fa::fa_bwd_pre_kernel<D><<<static_cast<int>(blocks), threads, 0, stream>>>(
+        o, dout, lse, delta, lse2, reinterpret_cast<float4*>(dq_acc), rows);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  // main
+  if (phases & 2u) {
+    fa::BwdParams p;
+    p.dq_acc = dq_acc;
+    p.delta = delta;
+    p.lse2 = lse2;
+    p.dk = dk;
+    p.dv = dv;
+    p.block_mask = block_mask;
+    p.kv_len = kv_len;
+    p.visited = visited;
+    p.B = B;
+    p.H = H;
+    p.N = N;
+    p.n_t = N / fa::kTile;
+    p.num_units = B * H * p.n_t;
+    p.causal = causal ? 1 : 0;
+    p.scale = scale;
+    p.scale_log2 = scale * fa::kLog2e;
+    const int grid = p.num_units < num_sms ? p.num_units : num_sms;
+    fa::fa_bwd_kernel<D><<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(tq, tk, tv, tdo, p);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  // dQ
+  if (phases & 4u) {
+    const int threads = 256;
+    const long long n8 = rows * D / 8;
+    long long blocks = (n8 + threads - 1) / threads;
+    const long long cap = static_cast<long long>(num_sms) * 8;
+    if (blocks > cap) blocks = cap;
+    fa::fa_bwd_dq_kernel<<<static_cast<int>(blocks), threads, 0, stream>>>(
+        reinterpret_cast<const float4*>(dq_acc), reinterpret_cast<uint4*>(dq), scale, n8);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+
+int fwd_impl(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o, float* lse, int B,
+             int H, int N, int d, float scale, int causal, const uint8_t* block_mask,
+             const int32_t* kv_len, uint8_t* visited, void* stream) {
+  int rc = check_shape(B, H, N, d);
+  if (rc == 1) return FA_OK;
+  if (rc != FA_OK) return rc;
+  if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+    return FA_ERR_ALIGN;
+  if (kv_len && !aligned(kv_len, 4)) return FA_ERR_ALIGN;
+  rc = check_scale(scale);
+  if (rc != FA_OK) return rc;
+  const int sms = select_device(q);
+  if (sms <= 0) return FA_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 64)
+    return launch_fwd<64>(q, k, v, o, lse, B, H, N, scale, causal, block_mask, kv_len, visited, s,
+                          sms);
+  return launch_fwd<128>(q, k, v, o, lse, B, H, N, scale, causal, block_mask, kv_len, visited, s,
+                         sms);
+}
+
+int bwd_impl(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf16* o,
+             const float* lse, const fa_bf16* dout, fa_bf16* dq, fa_bf16* dk, fa_bf16* dv, int B,
+             int H, int N, int d, float scale, int causal, const uint8_t* block_mask,
+             const int32_t* kv_len, void* workspace, size_t workspace_bytes, uint8_t* visited,
+             void* stream, unsigned phases = 7u) {
+  int rc = check_shape(B, H, N, d);
+  if (rc == 1) return FA_OK;
+  if (rc != FA_OK) return rc;
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA_ERR_NULL;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
+      !aligned(lse, 4))
+    return FA_ERR_ALIGN;
+  if (kv_len && !aligned(kv_len, 4)) return FA_ERR_ALIGN;
+  rc = check_scale(scale);
+  if (rc != FA_OK) return rc;
+  if (!workspace || workspace_bytes < ws_layout(B, H, N, d).total) return FA_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return FA_ERR_ALIGN;
+  const int sms = select_device(q);
+  if (sms <= 0) return FA_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 64)
+    return launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, scale, causal, block_mask,
+                          kv_len, workspace, visited, s, sms, phases);
+  return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, scale, causal, block_mask,
+                         kv_len, workspace, visited, s, sms, phases);
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_fwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o, float* lse, int B,
+           int H, int N, int d, float scale, int causal, const uint8_t* block_mask,
+           const int32_t* kv_len, void* stream) {
+  return fwd_impl(q, k, v, o, lse, B, H, N, d, scale, causal, block_mask, kv_len, nullptr, stream);
+}
+
+int fa_fwd_traced(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o, float* lse,
+                  int B, int H, int N, int d, float scale, int causal, const uint8_t* block_mask,
+                  const int32_t* kv_len, uint8_t* visited, void* stream) {
+  if (!visited && B > 0 && H > 0 && N > 0) return FA_ERR_NULL;
+  return fwd_impl(q, k, v, o, lse, B, H, N, d, scale, causal, block_mask, kv_len, visited, stream);
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
+  const int rc = check_shape(B, H, N, d);
+  if (rc != FA_OK) return 0;
+  return ws_layout(B, H, N, d).total;
+}
+
+int fa_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf16* o,
+           const float* lse, const fa_bf16* dout, fa_bf16* dq, fa_bf16* dk, fa_bf16* dv, int B,
+           int H, int N, int d, float scale, int causal, const uint8_t* block_mask,
+           const int32_t* kv_len, void* workspace, size_t workspace_bytes, void* stream) {
+  return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, block_mask, kv_len,
+                  workspace, workspace_bytes, nullptr, stream);
+}
+
+int fa_bwd_traced(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf16* o,
+                  const float* lse, const fa_bf16* dout, fa_bf16* dq, fa_bf16* dk, fa_bf16* dv,
+                  int B, int H, int N, int d, float scale, int causal, const uint8_t* block_mask,
+                  const int32_t* kv_len, void* workspace, size_t workspace_bytes,
+                  uint8_t* visited, void* stream) {
+  if (!visited && B > 0 && H > 0 && N > 0) return FA_ERR_NULL;
+  return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, block_mask, kv_len,
+                  workspace, workspace_bytes, visited, stream);
+}
+
+int fa_bwd_phase(int phase, const fa_bf16* q, const fa_bf16* k, const fa_bf16* v,
+                 const fa_bf16* o, const float* lse, const fa_bf16* dout, fa_bf16* dq, fa_bf16* dk,
+                 fa_bf16* dv, int B, int H, int N, int d, float scale, int causal,
+                 const uint8_t* block_mask, const int32_t* kv_len, void* workspace,
+                 size_t workspace_bytes, void* stream) {
+  if (phase < 0 || phase > 2) return FA_ERR_ARG;
+  return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, block_mask, kv_len,
+                  workspace, workspace_bytes, nullptr, stream, 1u << phase);
+}
+
+int fa_get_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, fa::g_device_status, sizeof(v)) != cudaSuccess) return FA_ERR_CUDA;
+  if (v != 0) {
+    const unsigned int z = 0;
+    if (cudaMemcpyToSymbol(fa::g_device_status, &z, sizeof(z)) != cudaSuccess) return FA_ERR_CUDA;
+    return FA_ERR_TIMEOUT;
+  }
+  return FA_OK;
+}
+
+const char* fa_status_string(int status) {
+  switch (status) {
+    case FA_OK: return "ok";
+    case FA_ERR_NULL: return "a required pointer is NULL";
+    case FA_ERR_ALIGN: return "a pointer is not aligned as required";
+    case FA_ERR_SHAPE: return "unsupported shape (negative size, N % 128 != 0, or B*H*N >= 2^31)";
+    case FA_ERR_UNSUPPORTED_D: return "head dimension d must be 64 or 128";
+    case FA_ERR_WORKSPACE: return "workspace missing or smaller than fa_bwd_workspace_size()";
+    case FA_ERR_CUDA: return "a CUDA runtime or driver call failed";
+    case FA_ERR_TIMEOUT: return "a device pipeline wait timed out; outputs are incomplete";
+    case FA_ERR_ARG: return "invalid argument (scale not finite or not > 0, or unknown phase)";
+    default: return "unknown status";
+  }
+}
+
+int fa_version(void) { return kVersion; }
+
+}  // extern "C"

@@ -1,0 +1,560 @@
+// fa_bwd.cuh - backward kernels: recompute the score and probability tiles on
+// chip from Q, K, V and the saved log-sum-exp instead of storing them
+// ("FlashAttention, Decoded", "The Hardware Picture": recomputation;
+// opendecode.dev summary, "The key idea": the matrix is recomputed from the
+// tiles in the backward pass).
+//
+// With S = scale * Q K^T, P = exp(S - LSE), O = P V and upstream gradient dO:
+//   dV = P^T dO,  dP = dO V^T,  D_r = sum_x dO_rx O_rx,  dS = P o (dP - D),
+//   dQ = scale * dS K,  dK = scale * dS^T Q.
+//
+// Three launches:
+//   fa_bwd_pre_kernel    D and LSE*log2(e) per row; zero the f32 dQ accumulator
+//   fa_bwd_kernel        one CTA per (b, h, 128-key tile j), persistent
+//   fa_bwd_dq_kernel     dQ = bf16(scale * accumulator)
+//
+// fa_bwd_kernel roles (12 warps):
+//   warp 0      TMA producer: K_j, V_j once per unit; Q_i, dO_i per visited
+//               query tile through a kStages-deep ring
+//   warp 1      MMA issuer (one thread), TMEM owner
+//   warps 4-7   "dS" group, one key row per thread (TMEM lane): P^T, dS^T,
+//               and the dK / dV epilogue of each unit
+//   warps 8-11  "dQ" group, one query row per thread: drains dQ partials from
+//               TMEM and adds them into the float32 accumulator in HBM
+// Per visited query tile i the MMA thread issues, all accumulating in TMEM:
+//   S^T  = K_j Q_i^T          (cols   0..127)
+//   dP^T = V_j dO_i^T         (cols 128..255)
+//   dV  += P^T dO_i           (A = P^T bf16 in TMEM over S^T's first 64 cols)
+//   dK  += dS^T Q_i           (A = dS^T bf16 in TMEM over dP^T's first 64 cols)
+//   dQ   = dS K_j             (A = dS from shared memory; result over cols 0..D-1)
+// dK and dV accumulate in cols 256..256+2D-1 for the whole unit.
+#pragma once
+
+#include "fa_fwd.cuh"
+
+namespace fa {
+
+// ---------------------------------------------------------------------------
+// preprocess: D_r = sum_x dO_rx O_rx (f32), lse2_r = LSE_r * log2(e)
+// (+inf for rows with no allowed key, so that exp2(s - lse2) = 0), and zero
+// the dQ accumulator.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const uint16_t* __restrict__ o,
+                                                         const uint16_t* __restrict__ dout,
+                                                         const float* __restrict__ lse,
+                                                         float* __restrict__ delta,
+                                                         float* __restrict__ lse2,
+                                                         float4* __restrict__ dq_acc,
+                                                         long long rows) {
+  constexpr int kLanesPerRow = D / 8;  // one 16-byte chunk (8 bf16) per lane
+  constexpr int kRowsPerWarp = 32 / kLanesPerRow;
+  const long long warp_global = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5;
+  const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int sub = lane / kLanesPerRow;
+  const int part = lane % kLanesPerRow;
+  for (long long r0 = warp_global * kRowsPerWarp; r0 < rows; r0 += nwarps * kRowsPerWarp) {
+    const long long r = r0 + sub;
+    float acc = 0.f;
+    if (r < rows) {
+      const uint4 a = __ldg(reinterpret_cast<const uint4*>(o + r * D) + part);
+      const uint4 b = __ldg(reinterpret_cast<const uint4*>(dout + r * D) + part);
+      const uint32_t av[4] = {a.x, a.y, a.z, a.w};
+      const uint32_t bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 fa2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&av[e]));
+        const float2 fb2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bv[e]));
+        acc = fmaf(fa2.x, fb2.x, acc);
+        acc = fmaf(fa2.y, fb2.y, acc);
+      }
+    }
+#pragma unroll
+    for (int off = kLanesPerRow / 2; off > 0; off >>= 1)
+      acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (r < rows && part == 0) {
+      delta[r] = acc;
+      const float l = lse[r];
+      lse2[r] = (l == -INFINITY) ? INFINITY : l * kLog2e;
+    }
+  }
+  const long long n4 = rows * (D / 4);
+  const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n4;
+       e += (long long)gridDim.x * blockDim.x)
+    dq_acc[e] = z;
+}
+
+// dQ = bf16(scale * accumulator), 8 elements per thread per step.
+__global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const float4* __restrict__ dq_acc,
+                                                        uint4* __restrict__ dq, float scale,
+                                                        long long n8) {
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n8;
+       e += (long long)gridDim.x * blockDim.x) {
+    const float4 a = __ldg(dq_acc + 2 * e);
+    const float4 b = __ldg(dq_acc + 2 * e + 1);
+    dq[e] = make_uint4(pack_bf16x2(a.x * scale, a.y * scale), pack_bf16x2(a.z * scale, a.w * scale),
+                       pack_bf16x2(b.x * scale, b.y * scale), pack_bf16x2(b.z * scale, b.w * scale));
+  }
+}
+
+// ---------------------------------------------------------------------------
+// main backward kernel
+// ---------------------------------------------------------------------------
+struct BwdParams {
+  float* dq_acc;
+  const float* delta;
+  const float* lse2;
+  uint16_t* dk;
+  uint16_t* dv;
+  const uint8_t* block_mask;
+  const int32_t* kv_len;
+  uint8_t* visited;
+  int B, H, N, n_t;
+  int num_units;
+  int causal;
+  float scale;
+  float scale_log2;
+};
+
+template <int D>
+struct BwdCfg {
+  static constexpr int kThreads = 384;
+  static constexpr int kTileBytes = kTile * D * 2;
+  static constexpr int kBoxes = D / 64;
+  static constexpr int kStages = (D == 64) ? 4 : 2;
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kOffK + kTileBytes;
+  static constexpr int kOffQ = kOffV + kTileBytes;
+  static constexpr int kOffDO = kOffQ + kStages * kTileBytes;
+  static constexpr int kOffDS = kOffDO + kStages * kTileBytes;  // 128 x 128 bf16
+  static constexpr int kOffBar = kOffDS + kTile * kTile * 2;
+  // kv_full, kv_empty, qdo_full[S], qdo_empty[S], s_full, dp_full, p_full, ds_full,
+  // ds_smem_empty, dq_full, dq_empty, dkv_full, drain
+  static constexpr int kNumBars = 2 + 2 * kStages + 9;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kColS = 0;      // S^T, then P^T (bf16), then dQ
+  static constexpr uint32_t kColDP = 128;   // dP^T, then dS^T (bf16)
+  static constexpr uint32_t kColDK = 256;
+  static constexpr uint32_t kColDV = 256 + D;
+};
+
+struct BwdUnit {
+  int bh, b, j, L, i_begin, any;
+};
+
+__device__ __forceinline__ bool bwd_tile_on(const BwdParams& p, const BwdUnit& w, int i) {
+  if (p.causal && w.j > i) return false;
+  if (w.j * kTile >= w.L) return false;
+  if (p.block_mask && __ldg(p.block_mask + (size_t)i * p.n_t + w.j) == 0) return false;
+  return true;
+}
+
+// First visited query tile >= i (or n_t).
+__device__ __forceinline__ int bwd_next(const BwdParams& p, const BwdUnit& w, int i) {
+  if (w.j * kTile >= w.L) return p.n_t;
+  for (; i < p.n_t; ++i)
+    if (bwd_tile_on(p, w, i)) return i;
+  return p.n_t;
+}
+
+__device__ __forceinline__ BwdUnit bwd_decode(const BwdParams& p, int u) {
+  BwdUnit w;
+  const int BH = p.B * p.H;
+  const int rank = u / BH;  // key tile; for causal masks tile 0 sees the most queries
+  w.bh = u - rank * BH;
+  w.b = w.bh / p.H;
+  w.j = rank;
+  int L = p.N;
+  if (p.kv_len) {
+    L = __ldg(p.kv_len + w.b);
+    L = L < 0 ? 0 : (L > p.N ? p.N : L);
+  }
+  w.L = L;
+  w.i_begin = p.causal ? w.j : 0;
+  w.any = bwd_next(p, w, w.i_begin) < p.n_t;
+  return w;
+}
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
+               "f"(c), "f"(d)
+               : "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
+    fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                  const BwdParams p) {
+  using Cfg = BwdCfg<D>;
+  constexpr int S = Cfg::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + Cfg::kOffBar;
+  const uint32_t kv_full = bar0, kv_empty = bar0 + 8;
+  auto qdo_full = [&](int s) { return bar0 + 8 * (2 + s); };
+  auto qdo_empty = [&](int s) { return bar0 + 8 * (2 + S + s); };
+  const uint32_t s_full = bar0 + 8 * (2 + 2 * S);
+  const uint32_t dp_full = s_full + 8, p_full = s_full + 16, ds_full = s_full + 24;
+  const uint32_t ds_smem_empty = s_full + 32, dq_full = s_full + 40, dq_empty = s_full + 48;
+  const uint32_t dkv_full = s_full + 56, drain_bar = s_full + 64;
+  uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kOffMisc + 4);
+
+  const int warp = warp_id();
+  const int lane = lane_id();
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    mbar_init(kv_empty, 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(qdo_full(s), 1);
+      mbar_init(qdo_empty(s), 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
+    mbar_init(p_full, 128);
+    mbar_init(ds_full, 128);
+    mbar_init(ds_smem_empty, 1);
+    mbar_init(dq_full, 1);
+    mbar_init(dq_empty, 128);
+    mbar_init(dkv_full, 1);
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    prefetch_tmap(&tm_do);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_base_slot), Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_base_slot;
+  const int G = gridDim.x;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t kv_cnt = 0, qdo_cnt = 0;
+      bool ok = true;
+      for (int round = 0; ok; ++round) {
+        const int u = unit_for_round(round, blockIdx.x, G);
+        if (u >= p.num_units) break;
+        const BwdUnit w = bwd_decode(p, u);
+        if (!w.any) continue;
+        ok = mbar_wait(kv_empty, (kv_cnt & 1) ^ 1);
+        if (!ok) break;
+        ++kv_cnt;
+        const int krow = w.bh * p.N + w.j * kTile;
+        mbar_arrive_expect_tx(kv_full, 2 * Cfg::kTileBytes);
+        for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
+          tma_load_2d(sbase + Cfg::kOffK + bx * 16384, &tm_k, bx * 64, krow, kv_full);
+          tma_load_2d(sbase + Cfg::kOffV + bx * 16384, &tm_v, bx * 64, krow, kv_full);
+        }
+        for (int i = bwd_next(p, w, w.i_begin); i < p.n_t && ok; i = bwd_next(p, w, i + 1)) {
+          const int s = qdo_cnt % S;
+          ok = mbar_wait(qdo_empty(s), ((qdo_cnt / S) & 1) ^ 1);
+          if (!ok) break;
+          const int qrow = w.bh * p.N + i * kTile;
+          mbar_arrive_expect_tx(qdo_full(s), 2 * Cfg::kTileBytes);
+          for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
+            tma_load_2d(sbase + Cfg::kOffQ + s * Cfg::kTileBytes + bx * 16384, &tm_q, bx * 64, qrow,
+                        qdo_full(s));
+            tma_load_2d(sbase + Cfg::kOffDO + s * Cfg::kTileBytes + bx * 16384, &tm_do, bx * 64,
+                        qrow, qdo_full(s));
+          }
+          ++qdo_cnt;
+        }
+        if (*abort_flag) ok = false;
+      }
+      if (!ok) *abort_flag = 1;
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_kk = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T
+      constexpr uint32_t idesc_tn = idesc_bf16_f32(128, D, 0, 1);    // dV, dK (A in TMEM)
+      constexpr uint32_t idesc_dq = idesc_bf16_f32(128, D, 1, 1);    // dQ (both MN-major)
+      uint32_t kv_cnt = 0, qdo_cnt = 0, p_cnt = 0, ds_cnt = 0, dq_cnt = 0;
+      bool ok = true;
+      const uint32_t ka = sbase + Cfg::kOffK, va = sbase + Cfg::kOffV;
+      const uint32_t dsa = sbase + Cfg::kOffDS;
+      for (int round = 0; ok; ++round) {
+        const int u = unit_for_round(round, blockIdx.x, G);
+        if (u >= p.num_units) break;
+        const BwdUnit w = bwd_decode(p, u);
+        if (!w.any) continue;
+        ok = mbar_wait(kv_full, kv_cnt & 1);
+        ++kv_cnt;
+        if (!ok) break;
+        int t = 0;
+        for (int i = bwd_next(p, w, w.i_begin); i < p.n_t && ok; i = bwd_next(p, w, i + 1), ++t) {
+          const int s = qdo_cnt % S;
+          ok = mbar_wait(qdo_full(s), (qdo_cnt / S) & 1);
+          if (!ok) break;
+          ok = mbar_wait(dq_empty, (dq_cnt & 1) ^ 1);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t qa = sbase + Cfg::kOffQ + s * Cfg::kTileBytes;
+          const uint32_t doa = sbase + Cfg::kOffDO + s * Cfg::kTileBytes;
+          // S^T = K_j Q_i^T
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            umma_ss(tmem + Cfg::kColS, sw128_desc(ka + off, 16, 1024),
+                    sw128_desc(qa + off, 16, 1024), idesc_kk, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(s_full);
+          if (p.visited) p.visited[((size_t)w.bh * p.n_t + i) * p.n_t + w.j] = 1;
+          // dP^T = V_j dO_i^T
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            umma_ss(tmem + Cfg::kColDP, sw128_desc(va + off, 16, 1024),
+                    sw128_desc(doa + off, 16, 1024), idesc_kk, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(dp_full);
+          // dV += P^T dO_i
+          ok = mbar_wait(p_full, p_cnt & 1);
+          ++p_cnt;
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            umma_ts(tmem + Cfg::kColDV, tmem + Cfg::kColS + kk * 8,
+                    sw128_desc(doa + kk * 2048, 16384, 1024), idesc_tn,
+                    (t > 0 || kk > 0) ? 1u : 0u);
+          // dK += dS^T Q_i ; dQ = dS K_j
+          ok = mbar_wait(ds_full, ds_cnt & 1);
+          ++ds_cnt;
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            umma_ts(tmem + Cfg::kColDK, tmem + Cfg::kColDP + kk * 8,
+                    sw128_desc(qa + kk * 2048, 16384, 1024), idesc_tn,
+                    (t > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            umma_ss(tmem + Cfg::kColS, sw128_desc(dsa + kk * 2048, 16384, 1024),
+                    sw128_desc(ka + kk * 2048, 16384, 1024), idesc_dq, kk > 0 ? 1u : 0u);
+          umma_commit(dq_full);
+          ++dq_cnt;
+          umma_commit(qdo_empty(s));
+          umma_commit(ds_smem_empty);
+          ++qdo_cnt;
+          if (*abort_flag) ok = false;
+        }
+        if (!ok) break;
+        umma_commit(kv_empty);
+        umma_commit(dkv_full);
+      }
+      if (!ok) *abort_flag = 1;
+      umma_commit(drain_bar);
+      mbar_wait(drain_bar, 0);
+    }
+    __syncwarp();
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------ dS group
+    const int quarter = warp & 3;
+    const int kr = quarter * 32 + lane;  // key row within the tile
+    const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
+    uint8_t* ds_smem = smem + Cfg::kOffDS;
+    uint32_t s_cnt = 0, dp_cnt = 0, dsm_cnt = 0, dkv_cnt = 0;
+    bool ok = true;
+    for (int round = 0; ok; ++round) {
+      const int u = unit_for_round(round, blockIdx.x, G);
+      if (u >= p.num_units) break;
+      const BwdUnit w = bwd_decode(p, u);
+      const int c_key = w.j * kTile + kr;  // key index within the head
+      const size_t krow = (size_t)w.bh * p.N + c_key;
+      uint4* dk_row = reinterpret_cast<uint4*>(p.dk + krow * D);
+      uint4* dv_row = reinterpret_cast<uint4*>(p.dv + krow * D);
+      if (!w.any) {
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) {
+          dk_row[c] = make_uint4(0, 0, 0, 0);
+          dv_row[c] = make_uint4(0, 0, 0, 0);
+        }
+        continue;
+      }
+      const bool key_valid = c_key < w.L;
+      for (int i = bwd_next(p, w, w.i_begin); i < p.n_t; i = bwd_next(p, w, i + 1)) {
+        const float* lse2_t = p.lse2 + (size_t)w.bh * p.N + i * kTile;
+        const float* dl_t = p.delta + (size_t)w.bh * p.N + i * kTile;
+        const bool diag = p.causal && (i == w.j);
+        ok = __all_sync(0xffffffffu, mbar_wait(s_full, s_cnt & 1));
+        ++s_cnt;
+        if (!ok) break;
+        tc_fence_after();
+        // P^T row: p[q] = exp2(S^T[kr][q] * scale*log2e - lse2[q]), masked -> 0
+        uint32_t ppk[64];
+        {
+          uint32_t r[4][32];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tmem_ld32(t_lane + Cfg::kColS + c * 32, r[c]);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            reg_fence32(r[c]);
+            float lz[32];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float4 v4 = __ldg(reinterpret_cast<const float4*>(lse2_t + c * 32) + e);
+              lz[4 * e] = v4.x; lz[4 * e + 1] = v4.y; lz[4 * e + 2] = v4.z; lz[4 * e + 3] = v4.w;
+            }
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int q0 = c * 32 + 2 * e;
+              float p0 = ex2_approx(fmaf(__uint_as_float(r[c][2 * e]), p.scale_log2, -lz[2 * e]));
+              float p1 =
+                  ex2_approx(fmaf(__uint_as_float(r[c][2 * e + 1]), p.scale_log2, -lz[2 * e + 1]));
+              if (!key_valid || (diag && kr > q0)) p0 = 0.f;
+              if (!key_valid || (diag && kr > q0 + 1)) p1 = 0.f;
+              pk[e] = pack_bf16x2(p0, p1);
+              ppk[c * 16 + e] = pk[e];
+            }
+            tmem_st16(t_lane + Cfg::kColS + c * 16, pk);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(p_full);
+        // dS^T row: ds[q] = p[q] * (dP^T[kr][q] - D[q])
+        ok = __all_sync(0xffffffffu, mbar_wait(dp_full, dp_cnt & 1));
+        ++dp_cnt;
+        if (!ok) break;
+        ok = __all_sync(0xffffffffu, mbar_wait(ds_smem_empty, (dsm_cnt & 1) ^ 1));
+        ++dsm_cnt;
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tmem_ld32(t_lane + Cfg::kColDP + c * 32, r);
+          tmem_wait_ld();
+          reg_fence32(r);
+          float dz[32];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float4 v4 = __ldg(reinterpret_cast<const float4*>(dl_t + c * 32) + e);
+            dz[4 * e] = v4.x; dz[4 * e + 1] = v4.y; dz[4 * e + 2] = v4.z; dz[4 * e + 3] = v4.w;
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float2 pp =
+                __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ppk[c * 16 + e]));
+            const float ds0 = pp.x * (__uint_as_float(r[2 * e]) - dz[2 * e]);
+            const float ds1 = pp.y * (__uint_as_float(r[2 * e + 1]) - dz[2 * e + 1]);
+            pk[e] = pack_bf16x2(ds0, ds1);
+          }
+          tmem_st16(t_lane + Cfg::kColDP + c * 16, pk);
+          // shared-memory copy for the dQ MMA: [key][query], 64-query chunks 16 KB
+          // apart, 128-byte rows, 16-byte granules swizzled by (key & 7)
+          uint8_t* rowp = ds_smem + (c >> 1) * 16384 + kr * 128;
+#pragma unroll
+          for (int g4 = 0; g4 < 4; ++g4) {
+            const int g = (c & 1) * 4 + g4;
+            *reinterpret_cast<uint4*>(rowp + ((g ^ (kr & 7)) << 4)) =
+                make_uint4(pk[4 * g4], pk[4 * g4 + 1], pk[4 * g4 + 2], pk[4 * g4 + 3]);
+          }
+        }
+        fence_proxy_async_smem();
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(ds_full);
+        if (*abort_flag) { ok = false; break; }
+      }
+      if (!ok) break;
+      // ---------------------------------------------- dK, dV epilogue
+      ok = __all_sync(0xffffffffu, mbar_wait(dkv_full, dkv_cnt & 1));
+      ++dkv_cnt;
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(t_lane + Cfg::kColDK + c * 32, r);
+        tmem_wait_ld();
+        reg_fence32(r);
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * p.scale,
+                              __uint_as_float(r[2 * e + 1]) * p.scale);
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4)
+          dk_row[c * 4 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+        tmem_ld32(t_lane + Cfg::kColDV + c * 32, r);
+        tmem_wait_ld();
+        reg_fence32(r);
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4)
+          dv_row[c * 4 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+      }
+      tc_fence_before();
+    }
+    if (!ok) *abort_flag = 1;
+  } else if (warp >= 8) {
+    // ------------------------------------------------------------ dQ group
+    const int quarter = warp & 3;
+    const int qr = quarter * 32 + lane;  // query row within the tile
+    const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
+    uint32_t dq_cnt = 0;
+    bool ok = true;
+    for (int round = 0; ok; ++round) {
+      const int u = unit_for_round(round, blockIdx.x, G);
+      if (u >= p.num_units) break;
+      const BwdUnit w = bwd_decode(p, u);
+      if (!w.any) continue;
+      for (int i = bwd_next(p, w, w.i_begin); i < p.n_t; i = bwd_next(p, w, i + 1)) {
+        ok = __all_sync(0xffffffffu, mbar_wait(dq_full, dq_cnt & 1));
+        ++dq_cnt;
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t r[D / 32][32];
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) tmem_ld32(t_lane + Cfg::kColS + c * 32, r[c]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) reg_fence32(r[c]);
+        tc_fence_before();
+        mbar_arrive(dq_empty);
+        float* dst = p.dq_acc + ((size_t)w.bh * p.N + i * kTile + qr) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c)
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            red_add_v4(dst + c * 32 + 4 * e, __uint_as_float(r[c][4 * e]),
+                       __uint_as_float(r[c][4 * e + 1]), __uint_as_float(r[c][4 * e + 2]),
+                       __uint_as_float(r[c][4 * e + 3]));
+        if (*abort_flag) { ok = false; break; }
+      }
+    }
+    if (!ok) *abort_flag = 1;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, Cfg::kTmemCols);
+}
+
+}  // namespace fa

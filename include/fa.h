@@ -1,0 +1,160 @@
+/*
+ * fa.h - C ABI of the B200 (sm_100a) exact tiled attention library
+ *        (libfa_b200.so).
+ *
+ * The operation.  Exact softmax attention, computed tile by tile so that
+ * the N x N score matrix never reaches HBM ("FlashAttention:
+ * Fast and Memory-Efficient Exact Attention with IO-Awareness",
+ * opendecode.dev summary, section "The key idea"; "FlashAttention,
+ * Decoded", gloss of abstract sentence 4 and "The Hardware Picture").  For
+ * every batch b and head h, with row r and key c:
+ *
+ *   allowed(r,c) = (!causal || c <= r) && (kv_len == NULL || c < kv_len[b])
+ *                  && (block_mask == NULL || block_mask[(r/128)*(N/128) + c/128] != 0)
+ *   S_rc  = scale * <Q_r, K_c>  (allowed), -inf (otherwise)
+ *   P_rc  = exp(S_rc - LSE_r),  LSE_r = ln sum_c exp(S_rc)
+ *   O_r   = sum_c P_rc V_c
+ *
+ * A row with no allowed key gets O_r = 0 and LSE_r = -inf.  The backward pass
+ * recomputes S and P on chip from Q, K, V and LSE ("The Hardware Picture":
+ * recomputation; opendecode.dev, "The key idea") and returns
+ * dQ = scale * dS K, dK = scale * dS^T Q, dV = P^T dO, with
+ * dS = P o (dO V^T - D) and D_r = sum_x dO_rx O_rx.
+ *
+ * Conventions for every entry point below.
+ *  - Tensors Q, K, V, O, dO, dQ, dK, dV are bfloat16 (raw 16-bit patterns,
+ *    type fa_bf16), contiguous [B][H][N][d] in device memory, base address
+ *    16-byte aligned.  LSE is float32 [B][H][N] (natural log), 4-byte aligned.
+ *  - d is 64 or 128.  N is a multiple of 128.  B, H, N >= 0; if any is 0 the
+ *    call does nothing and returns FA_OK.  B*H*N must be below 2^31.
+ *  - scale is finite and > 0 (1/sqrt(d) is the usual choice).
+ *  - block_mask (nullable) is uint8 [N/128][N/128] in device memory, row =
+ *    query tile, column = key tile, nonzero = keep; all (b, h) share it.
+ *  - kv_len (nullable) is int32 [B] in device memory: keys c >= kv_len[b]
+ *    are masked for every query of batch b.  Values must lie in [0, N];
+ *    the kernels clamp values outside that range into it.
+ *  - stream is a cudaStream_t (passed as void*; NULL = legacy default
+ *    stream).  Work is enqueued asynchronously; the return value covers
+ *    argument checks and launch errors only.  Device-side failures (a
+ *    pipeline wait that timed out) are reported by fa_get_device_status.
+ *  - The caller owns every buffer.  fa_fwd allocates nothing.  fa_bwd uses
+ *    only the caller's workspace.  Nothing is freed by the library.
+ *  - On any nonzero return, nothing was launched and no output was touched.
+ */
+#ifndef FA_B200_H
+#define FA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t fa_bf16; /* bfloat16 bit pattern */
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_NULL = -1,           /* a required pointer is NULL */
+    FA_ERR_ALIGN = -2,          /* a pointer breaks its alignment rule */
+    FA_ERR_SHAPE = -3,          /* negative size, N % 128 != 0, or B*H*N >= 2^31 */
+    FA_ERR_UNSUPPORTED_D = -4,  /* d not in {64, 128} */
+    FA_ERR_WORKSPACE = -5,      /* workspace NULL or smaller than fa_bwd_workspace_size */
+    FA_ERR_CUDA = -6,           /* a CUDA runtime/driver call failed */
+    FA_ERR_TIMEOUT = -7,        /* a device pipeline wait gave up (fa_get_device_status) */
+    FA_ERR_ARG = -8             /* scale not finite or not > 0, or phase not in 0..2 */
+} fa_status;
+
+/*
+ * Forward pass: writes O and LSE.  One persistent launch; each CTA takes
+ * (b, h, pair of 128-row query tiles) work units and streams the key/value
+ * tiles that hold at least one allowed entry (causal, key-padding and
+ * block-sparse tile skipping), with the online softmax (running row max and
+ * row sum, partial output rescaled as tiles arrive; opendecode.dev, "The
+ * key idea").
+ */
+int fa_fwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o, float* lse,
+           int B, int H, int N, int d, float scale, int causal,
+           const uint8_t* block_mask, const int32_t* kv_len, void* stream);
+
+/*
+ * fa_fwd plus a record of the tiles it computed: visited (device, uint8
+ * [B][H][N/128][N/128], zeroed by the caller) gets 1 at [b][h][i][j] for
+ * every (query tile i, key tile j) whose scores the kernel formed.  Same
+ * kernel as fa_fwd; intended for tests of the tile-skip logic.
+ */
+int fa_fwd_traced(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o, float* lse,
+                  int B, int H, int N, int d, float scale, int causal,
+                  const uint8_t* block_mask, const int32_t* kv_len, uint8_t* visited,
+                  void* stream);
+
+/*
+ * Bytes of device workspace fa_bwd needs: 4*B*H*N (D) + 4*B*H*N (LSE in
+ * base 2) + 4*B*H*N*d (float32 dQ accumulator), each region 256-byte
+ * aligned.  Returns 0 for an empty or invalid shape.
+ */
+size_t fa_bwd_workspace_size(int B, int H, int N, int d);
+
+/*
+ * Backward pass: from Q, K, V, O, LSE (as written by fa_fwd with the same
+ * mask arguments) and dO, writes dQ, dK, dV.  Three launches on `stream`:
+ * a preprocess kernel (D = rowsum(dO o O), zero the dQ accumulator), the
+ * main kernel (one CTA per (b, h, 128-key tile): recompute S and P,
+ * accumulate dK and dV on chip, add dQ partials into the float32
+ * accumulator), and a kernel that writes dQ = bf16(scale * accumulator).
+ * workspace must be 256-byte aligned and hold fa_bwd_workspace_size bytes;
+ * its contents on entry do not matter and on exit are unspecified.  Calls
+ * that share a workspace must not overlap on the device.
+ */
+int fa_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf16* o,
+           const float* lse, const fa_bf16* dout, fa_bf16* dq, fa_bf16* dk, fa_bf16* dv,
+           int B, int H, int N, int d, float scale, int causal,
+           const uint8_t* block_mask, const int32_t* kv_len,
+           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * fa_bwd plus a record of the tiles the main kernel computed: visited
+ * (device, uint8 [B][H][N/128][N/128], zeroed by the caller) gets 1 at
+ * [b][h][i][j] for every (query tile i, key tile j) it recomputed.
+ */
+int fa_bwd_traced(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf16* o,
+                  const float* lse, const fa_bf16* dout, fa_bf16* dq, fa_bf16* dk, fa_bf16* dv,
+                  int B, int H, int N, int d, float scale, int causal,
+                  const uint8_t* block_mask, const int32_t* kv_len,
+                  void* workspace, size_t workspace_bytes, uint8_t* visited, void* stream);
+
+/*
+ * One of the three launches of fa_bwd, for callers that schedule or time them
+ * separately: phase 0 = preprocess (D, base-2 LSE, zeroed dQ accumulator in
+ * the workspace), 1 = main kernel (dK, dV; dQ partials into the
+ * accumulator), 2 = dQ = bf16(scale * accumulator).  Arguments as for
+ * fa_bwd.  Calling phases 0, 1, 2 in order on one stream with the same
+ * arguments and workspace is exactly fa_bwd; a phase reads what the earlier
+ * phases left in the workspace.
+ */
+int fa_bwd_phase(int phase, const fa_bf16* q, const fa_bf16* k, const fa_bf16* v,
+                 const fa_bf16* o, const float* lse, const fa_bf16* dout, fa_bf16* dq, fa_bf16* dk,
+                 fa_bf16* dv, int B, int H, int N, int d, float scale, int causal,
+                 const uint8_t* block_mask, const int32_t* kv_len, void* workspace,
+                 size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronises `stream`, then returns FA_OK if no kernel of this library
+ * has reported a device-side failure since the last call, FA_ERR_TIMEOUT
+ * if a pipeline wait gave up (the kernel then skipped the rest of its work
+ * and its outputs are incomplete), or FA_ERR_CUDA if synchronising failed.
+ * Clears the recorded state.  The state is per process and per device.
+ */
+int fa_get_device_status(void* stream);
+
+/* Static, NUL-terminated description of a status code. */
+const char* fa_status_string(int status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_H */

@@ -18,8 +18,17 @@ Functions (all arrays contiguous, float64 unless stated):
   ``(o, lse)`` for q, k, v of shape [B, H, N, d].
 * ``attention_backward(q, k, v, dout, scale, causal, block_mask, kv_len)`` ->
   ``(dq, dk, dv, delta)`` by the chain rule on sum(O * dO).
+* ``attention_forward_band`` / ``attention_backward_band``: the same for query
+  rows [r_begin, r_end) of every head (dK, dV then hold those rows' share);
+  used to time bounded samples of large workloads.
 * ``attention_forward_rows(q_rows, rows, k, v, scale, causal, block_mask,
   kv_len_b)`` -> ``(o_rows, lse_rows)`` for chosen query rows of one head.
+* ``attention_backward_dq_rows(q_rows, dout_rows, rows, k, v, scale, causal,
+  block_mask, kv_len_b)`` -> ``(dq_rows, delta_rows)``: the row-local part of
+  the backward pass (dQ_r and D_r) for chosen query rows of one head.
+* ``attention_backward_kv_cols(q, k, v, dout, cols, scale, causal, block_mask,
+  kv_len_b)`` -> ``(dk_cols, dv_cols)``: dK and dV of chosen key columns of
+  one head (a full pass over the head's rows).
 * ``tile_visits(B, N, causal, block_mask, kv_len, T=128, i_begin=0,
   i_end=None)`` -> uint8 [B, i_end - i_begin, N // T]: 1 where a
   (query tile, key tile) pair holds at least one allowed (row, key).
@@ -68,14 +77,31 @@ def _load():
             lib.oracle_attention_backward.argtypes = [
                 _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                 ctypes.c_int, ctypes.c_double, ctypes.c_int, _u8p, _i32p, ctypes.c_int]
+            lib.oracle_attention_forward_band.argtypes = [
+                _dp, _dp, _dp, _dp, _dp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                ctypes.c_double, ctypes.c_int, _u8p, _i32p, ctypes.c_int, ctypes.c_int,
+                ctypes.c_int]
+            lib.oracle_attention_backward_band.argtypes = [
+                _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                ctypes.c_int, ctypes.c_double, ctypes.c_int, _u8p, _i32p, ctypes.c_int,
+                ctypes.c_int, ctypes.c_int]
             lib.oracle_attention_forward_rows.argtypes = [
                 _dp, _i64p, ctypes.c_int, _dp, _dp, _dp, _dp, ctypes.c_int, ctypes.c_int,
                 ctypes.c_double, ctypes.c_int, _u8p, ctypes.c_int]
+            lib.oracle_attention_backward_dq_rows.argtypes = [
+                _dp, _dp, _i64p, ctypes.c_int, _dp, _dp, _dp, _dp, ctypes.c_int, ctypes.c_int,
+                ctypes.c_double, ctypes.c_int, _u8p, ctypes.c_int]
+            lib.oracle_attention_backward_kv_cols.argtypes = [
+                _dp, _dp, _dp, _dp, _i64p, ctypes.c_int, _dp, _dp, ctypes.c_int, ctypes.c_int,
+                ctypes.c_double, ctypes.c_int, _u8p, ctypes.c_int, ctypes.c_int]
             lib.oracle_tile_visits.argtypes = [
                 _u8p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _u8p, _i32p,
                 ctypes.c_int, ctypes.c_int]
             for fn in (lib.oracle_attention_forward, lib.oracle_attention_backward,
-                       lib.oracle_attention_forward_rows, lib.oracle_tile_visits):
+                       lib.oracle_attention_forward_rows, lib.oracle_tile_visits,
+                       lib.oracle_attention_backward_dq_rows,
+                       lib.oracle_attention_backward_kv_cols, lib.oracle_attention_forward_band,
+                       lib.oracle_attention_backward_band):
                 fn.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -130,6 +156,42 @@ def attention_backward(q, k, v, dout, scale, causal=False, block_mask=None, kv_l
     return dq, dk, dv, delta
 
 
+def attention_forward_band(q, k, v, scale, causal=False, block_mask=None, kv_len=None,
+                           r_begin=0, r_end=None, nthreads=None):
+    """O and LSE for query rows [r_begin, r_end) of every head (other rows are 0)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, N, d = q.shape
+    r_end = N if r_end is None else r_end
+    bm, kl = _mask_args(block_mask, kv_len)
+    o = np.zeros_like(q)
+    lse = np.zeros((B, H, N), np.float64)
+    rc = _load().oracle_attention_forward_band(
+        _ptr(q, _dp), _ptr(k, _dp), _ptr(v, _dp), _ptr(o, _dp), _ptr(lse, _dp), B, H, N, d,
+        float(scale), int(bool(causal)), _ptr(bm, _u8p), _ptr(kl, _i32p), int(r_begin),
+        int(r_end), _threads(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attention_forward_band failed: {rc}")
+    return o, lse
+
+
+def attention_backward_band(q, k, v, dout, scale, causal=False, block_mask=None, kv_len=None,
+                            r_begin=0, r_end=None, nthreads=None):
+    """dQ rows [r_begin, r_end) and those rows' contributions to dK, dV, for every head."""
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, H, N, d = q.shape
+    r_end = N if r_end is None else r_end
+    bm, kl = _mask_args(block_mask, kv_len)
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(q), np.zeros_like(q)
+    delta = np.zeros((B, H, N), np.float64)
+    rc = _load().oracle_attention_backward_band(
+        _ptr(q, _dp), _ptr(k, _dp), _ptr(v, _dp), _ptr(dout, _dp), _ptr(dq, _dp), _ptr(dk, _dp),
+        _ptr(dv, _dp), _ptr(delta, _dp), B, H, N, d, float(scale), int(bool(causal)),
+        _ptr(bm, _u8p), _ptr(kl, _i32p), int(r_begin), int(r_end), _threads(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attention_backward_band failed: {rc}")
+    return dq, dk, dv, delta
+
+
 def attention_forward_rows(q_rows, rows, k, v, scale, causal=False, block_mask=None,
                            kv_len_b=None):
     """Forward for query rows ``rows`` (int array) of one head; q_rows is [R, d]."""
@@ -147,6 +209,44 @@ def attention_forward_rows(q_rows, rows, k, v, scale, causal=False, block_mask=N
     if rc != 0:
         raise RuntimeError(f"oracle_attention_forward_rows failed: {rc}")
     return o, lse
+
+
+def attention_backward_dq_rows(q_rows, dout_rows, rows, k, v, scale, causal=False,
+                               block_mask=None, kv_len_b=None):
+    """dQ_r and D_r for query rows ``rows`` of one head; q_rows, dout_rows are [R, d]."""
+    q_rows, dout_rows, k, v = _f64(q_rows), _f64(dout_rows), _f64(k), _f64(v)
+    rows = np.ascontiguousarray(np.asarray(rows, np.int64))
+    R, d = q_rows.shape
+    N = k.shape[0]
+    bm, _ = _mask_args(block_mask, None)
+    dq = np.empty((R, d), np.float64)
+    delta = np.empty((R,), np.float64)
+    rc = _load().oracle_attention_backward_dq_rows(
+        _ptr(q_rows, _dp), _ptr(dout_rows, _dp), _ptr(rows, _i64p), R, _ptr(k, _dp),
+        _ptr(v, _dp), _ptr(dq, _dp), _ptr(delta, _dp), N, d, float(scale), int(bool(causal)),
+        _ptr(bm, _u8p), -1 if kv_len_b is None else int(kv_len_b))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attention_backward_dq_rows failed: {rc}")
+    return dq, delta
+
+
+def attention_backward_kv_cols(q, k, v, dout, cols, scale, causal=False, block_mask=None,
+                               kv_len_b=None, nthreads=None):
+    """dK_c and dV_c for key columns ``cols`` of one head; q, k, v, dout are [N, d]."""
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    cols = np.ascontiguousarray(np.asarray(cols, np.int64))
+    N, d = q.shape
+    C = len(cols)
+    bm, _ = _mask_args(block_mask, None)
+    dk = np.empty((C, d), np.float64)
+    dv = np.empty((C, d), np.float64)
+    rc = _load().oracle_attention_backward_kv_cols(
+        _ptr(q, _dp), _ptr(k, _dp), _ptr(v, _dp), _ptr(dout, _dp), _ptr(cols, _i64p), C,
+        _ptr(dk, _dp), _ptr(dv, _dp), N, d, float(scale), int(bool(causal)), _ptr(bm, _u8p),
+        -1 if kv_len_b is None else int(kv_len_b), _threads(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attention_backward_kv_cols failed: {rc}")
+    return dk, dv
 
 
 def tile_visits(B, N, causal=False, block_mask=None, kv_len=None, T=128, i_begin=0, i_end=None):

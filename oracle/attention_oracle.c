@@ -51,6 +51,7 @@ typedef struct {
     const uint8_t *block_mask;
     const int32_t *kv_len;
     int backward;
+    int r_begin, r_end;     /* query rows computed in every head */
     int next_head;          /* shared work counter, guarded by lock */
     pthread_mutex_t lock;
 } oracle_job;
@@ -112,7 +113,7 @@ static void forward_head(const oracle_job *job, int bh, double *p)
     double *O = job->o + off;
     double *lse = job->lse + (size_t)bh * N;
     const int L = job->kv_len ? job->kv_len[b] : -1;
-    for (int r = 0; r < N; ++r) {
+    for (int r = job->r_begin; r < job->r_end; ++r) {
         double m, l;
         int count = softmax_row(Q + (size_t)r * d, r, K, N, d, job->scale, job->causal,
                                 job->block_mask, L, p, &m, &l);
@@ -141,7 +142,7 @@ static void backward_head(const oracle_job *job, int bh, double *p, double *dp)
     const int L = job->kv_len ? job->kv_len[b] : -1;
     memset(dK, 0, sizeof(double) * (size_t)N * d);
     memset(dV, 0, sizeof(double) * (size_t)N * d);
-    for (int r = 0; r < N; ++r) {
+    for (int r = job->r_begin; r < job->r_end; ++r) {
         const double *qr = Q + (size_t)r * d;
         const double *dor = dO + (size_t)r * d;
         double *dqr = dQ + (size_t)r * d;
@@ -228,16 +229,51 @@ static int run_job(oracle_job *job, int nthreads)
     return rc;
 }
 
-int oracle_attention_forward(const double *q, const double *k, const double *v, double *o,
-                             double *lse, int B, int H, int N, int d, double scale, int causal,
-                             const uint8_t *block_mask, const int32_t *kv_len, int nthreads)
+/*
+ * Forward (or backward) for query rows [r_begin, r_end) of every head.  The
+ * backward's dK and dV then hold the contributions of those rows only, and
+ * dQ, O and LSE rows outside the band are left untouched.  The *_band forms
+ * exist to time bounded samples of a large workload; the plain forms are the
+ * band [0, N).
+ */
+int oracle_attention_forward_band(const double *q, const double *k, const double *v, double *o,
+                                  double *lse, int B, int H, int N, int d, double scale,
+                                  int causal, const uint8_t *block_mask, const int32_t *kv_len,
+                                  int r_begin, int r_end, int nthreads)
 {
+    if (r_begin < 0 || r_end > N || r_begin > r_end) return -3;
     oracle_job job;
     memset(&job, 0, sizeof(job));
     job.q = q; job.k = k; job.v = v; job.o = o; job.lse = lse;
     job.B = B; job.H = H; job.N = N; job.d = d; job.scale = scale; job.causal = causal;
     job.block_mask = block_mask; job.kv_len = kv_len; job.backward = 0;
+    job.r_begin = r_begin; job.r_end = r_end;
     return run_job(&job, nthreads);
+}
+
+int oracle_attention_backward_band(const double *q, const double *k, const double *v,
+                                   const double *dout, double *dq, double *dk, double *dv,
+                                   double *delta, int B, int H, int N, int d, double scale,
+                                   int causal, const uint8_t *block_mask, const int32_t *kv_len,
+                                   int r_begin, int r_end, int nthreads)
+{
+    if (r_begin < 0 || r_end > N || r_begin > r_end) return -3;
+    oracle_job job;
+    memset(&job, 0, sizeof(job));
+    job.q = q; job.k = k; job.v = v; job.dout = dout;
+    job.dq = dq; job.dk = dk; job.dv = dv; job.delta = delta;
+    job.B = B; job.H = H; job.N = N; job.d = d; job.scale = scale; job.causal = causal;
+    job.block_mask = block_mask; job.kv_len = kv_len; job.backward = 1;
+    job.r_begin = r_begin; job.r_end = r_end;
+    return run_job(&job, nthreads);
+}
+
+int oracle_attention_forward(const double *q, const double *k, const double *v, double *o,
+                             double *lse, int B, int H, int N, int d, double scale, int causal,
+                             const uint8_t *block_mask, const int32_t *kv_len, int nthreads)
+{
+    return oracle_attention_forward_band(q, k, v, o, lse, B, H, N, d, scale, causal, block_mask,
+                                         kv_len, 0, N, nthreads);
 }
 
 int oracle_attention_backward(const double *q, const double *k, const double *v,
@@ -245,13 +281,8 @@ int oracle_attention_backward(const double *q, const double *k, const double *v,
                               double *delta, int B, int H, int N, int d, double scale, int causal,
                               const uint8_t *block_mask, const int32_t *kv_len, int nthreads)
 {
-    oracle_job job;
-    memset(&job, 0, sizeof(job));
-    job.q = q; job.k = k; job.v = v; job.dout = dout;
-    job.dq = dq; job.dk = dk; job.dv = dv; job.delta = delta;
-    job.B = B; job.H = H; job.N = N; job.d = d; job.scale = scale; job.causal = causal;
-    job.block_mask = block_mask; job.kv_len = kv_len; job.backward = 1;
-    return run_job(&job, nthreads);
+    return oracle_attention_backward_band(q, k, v, dout, dq, dk, dv, delta, B, H, N, d, scale,
+                                          causal, block_mask, kv_len, 0, N, nthreads);
 }
 
 /*
@@ -286,6 +317,176 @@ int oracle_attention_forward_rows(const double *q_rows, const int64_t *rows, int
     }
     free(p);
     return 0;
+}
+
+/*
+ * Backward quantities that depend on one query row only, for a chosen subset
+ * of rows of ONE head: dQ_r = scale sum_c dS_rc K_c and D_r = sum_c P_rc dP_rc
+ * (same computation as in oracle_attention_backward, row by row).  q_rows and
+ * dout_rows are [R][d]; K and V are the head's [N][d].
+ */
+int oracle_attention_backward_dq_rows(const double *q_rows, const double *dout_rows,
+                                      const int64_t *rows, int R, const double *k,
+                                      const double *v, double *dq_rows, double *delta_rows,
+                                      int N, int d, double scale, int causal,
+                                      const uint8_t *block_mask, int kv_len_b)
+{
+    if (R < 0 || N <= 0 || d <= 0) return -3;
+    double *p = (double *)malloc(sizeof(double) * (size_t)N);
+    double *dp = (double *)malloc(sizeof(double) * (size_t)N);
+    if (!p || !dp) { free(p); free(dp); return -6; }
+    for (int i = 0; i < R; ++i) {
+        const int r = (int)rows[i];
+        const double *qr = q_rows + (size_t)i * d;
+        const double *dor = dout_rows + (size_t)i * d;
+        double *dqr = dq_rows + (size_t)i * d;
+        double m, l;
+        int count = softmax_row(qr, r, k, N, d, scale, causal, block_mask, kv_len_b, p, &m, &l);
+        for (int x = 0; x < d; ++x) dqr[x] = 0.0;
+        delta_rows[i] = 0.0;
+        if (count == 0) continue;
+        double D = 0.0;
+        for (int c = 0; c < N; ++c) {
+            if (p[c] == 0.0) { dp[c] = 0.0; continue; }
+            const double *vc = v + (size_t)c * d;
+            double s = 0.0;
+            for (int x = 0; x < d; ++x) s += dor[x] * vc[x];
+            dp[c] = s;
+            D += p[c] * s;
+        }
+        delta_rows[i] = D;
+        for (int c = 0; c < N; ++c) {
+            if (p[c] == 0.0) continue;
+            const double ds = p[c] * (dp[c] - D);
+            const double *kc = k + (size_t)c * d;
+            for (int x = 0; x < d; ++x) dqr[x] += scale * ds * kc[x];
+        }
+    }
+    free(p);
+    free(dp);
+    return 0;
+}
+
+/*
+ * dK and dV for a chosen subset of key columns of ONE head:
+ *   dV_c = sum_r P_rc dO_r,  dK_c = scale sum_r P_rc (dP_rc - D_r) Q_r
+ * for c in cols[0..C).  Every row r still needs its full softmax row and D_r,
+ * so this costs a full pass over the head; rows are split into fixed chunks
+ * of 256 handled by worker threads, and the per-chunk partial sums are added
+ * in chunk order, so the result does not depend on the thread count.
+ * q, k, v, dout are the head's [N][d]; dk_cols, dv_cols are [C][d].
+ */
+typedef struct {
+    const double *q, *k, *v, *dout;
+    const int64_t *cols;
+    int C, N, d;
+    double scale;
+    int causal;
+    const uint8_t *block_mask;
+    int L;
+    double *partial; /* [nchunks][2][C][d] */
+    int nchunks;
+    int next_chunk;
+    pthread_mutex_t lock;
+} kvcols_job;
+
+#define KVCOLS_CHUNK 256
+
+static void *kvcols_worker(void *arg)
+{
+    kvcols_job *job = (kvcols_job *)arg;
+    const int N = job->N, d = job->d, C = job->C;
+    double *p = (double *)malloc(sizeof(double) * (size_t)N);
+    double *dp = (double *)malloc(sizeof(double) * (size_t)N);
+    if (!p || !dp) { free(p); free(dp); return (void *)1; }
+    for (;;) {
+        pthread_mutex_lock(&job->lock);
+        int ch = job->next_chunk++;
+        pthread_mutex_unlock(&job->lock);
+        if (ch >= job->nchunks) break;
+        double *dk = job->partial + (size_t)ch * 2 * C * d;
+        double *dv = dk + (size_t)C * d;
+        memset(dk, 0, sizeof(double) * 2 * (size_t)C * d);
+        const int r_end = (ch + 1) * KVCOLS_CHUNK < N ? (ch + 1) * KVCOLS_CHUNK : N;
+        for (int r = ch * KVCOLS_CHUNK; r < r_end; ++r) {
+            const double *qr = job->q + (size_t)r * d;
+            const double *dor = job->dout + (size_t)r * d;
+            double m, l;
+            int count = softmax_row(qr, r, job->k, N, d, job->scale, job->causal,
+                                    job->block_mask, job->L, p, &m, &l);
+            if (count == 0) continue;
+            double D = 0.0;
+            for (int c = 0; c < N; ++c) {
+                if (p[c] == 0.0) { dp[c] = 0.0; continue; }
+                const double *vc = job->v + (size_t)c * d;
+                double s = 0.0;
+                for (int x = 0; x < d; ++x) s += dor[x] * vc[x];
+                dp[c] = s;
+                D += p[c] * s;
+            }
+            for (int i = 0; i < C; ++i) {
+                const int c = (int)job->cols[i];
+                if (p[c] == 0.0) continue;
+                const double ds = p[c] * (dp[c] - D);
+                for (int x = 0; x < d; ++x) {
+                    dk[(size_t)i * d + x] += job->scale * ds * qr[x];
+                    dv[(size_t)i * d + x] += p[c] * dor[x];
+                }
+            }
+        }
+    }
+    free(p);
+    free(dp);
+    return NULL;
+}
+
+int oracle_attention_backward_kv_cols(const double *q, const double *k, const double *v,
+                                      const double *dout, const int64_t *cols, int C,
+                                      double *dk_cols, double *dv_cols, int N, int d,
+                                      double scale, int causal, const uint8_t *block_mask,
+                                      int kv_len_b, int nthreads)
+{
+    if (C < 0 || N <= 0 || d <= 0) return -3;
+    for (int i = 0; i < C; ++i)
+        if (cols[i] < 0 || cols[i] >= N) return -3;
+    kvcols_job job;
+    memset(&job, 0, sizeof(job));
+    job.q = q; job.k = k; job.v = v; job.dout = dout; job.cols = cols; job.C = C;
+    job.N = N; job.d = d; job.scale = scale; job.causal = causal;
+    job.block_mask = block_mask; job.L = kv_len_b;
+    job.nchunks = (N + KVCOLS_CHUNK - 1) / KVCOLS_CHUNK;
+    job.partial = (double *)malloc(sizeof(double) * (size_t)job.nchunks * 2 * C * d + 1);
+    if (!job.partial) return -6;
+    pthread_mutex_init(&job.lock, NULL);
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > job.nchunks) nthreads = job.nchunks;
+    pthread_t *tids = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    int rc = 0, started = 0;
+    for (int t = 0; t < nthreads; ++t) {
+        if (pthread_create(&tids[t], NULL, kvcols_worker, &job) != 0) { rc = -6; break; }
+        ++started;
+    }
+    for (int t = 0; t < started; ++t) {
+        void *ret = NULL;
+        pthread_join(tids[t], &ret);
+        if (ret) rc = -6;
+    }
+    free(tids);
+    pthread_mutex_destroy(&job.lock);
+    if (rc == 0) {
+        memset(dk_cols, 0, sizeof(double) * (size_t)C * d);
+        memset(dv_cols, 0, sizeof(double) * (size_t)C * d);
+        for (int ch = 0; ch < job.nchunks; ++ch) {
+            const double *pk = job.partial + (size_t)ch * 2 * C * d;
+            const double *pv = pk + (size_t)C * d;
+            for (size_t e = 0; e < (size_t)C * d; ++e) {
+                dk_cols[e] += pk[e];
+                dv_cols[e] += pv[e];
+            }
+        }
+    }
+    free(job.partial);
+    return rc;
 }
 
 /*

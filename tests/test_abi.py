@@ -1,0 +1,135 @@
+"""The C-ABI library loads on a machine without a GPU, exports every function that
+include/fa.h declares, and rejects bad arguments on the host before any CUDA call."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from exact_io_aware_63_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[A-Za-z_0-9]+\s*\*?\s*(fa_[a-z_0-9]+)\s*\(",
+                                 text, flags=re.M)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ["fa_fwd", "fa_fwd_traced", "fa_bwd", "fa_bwd_traced", "fa_bwd_phase",
+              "fa_bwd_workspace_size",
+              "fa_get_device_status", "fa_status_string", "fa_version"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(binding.library_path() if os.path.exists(binding.library_path())
+                      else binding.load()._name)
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+
+
+def test_version_and_status_strings():
+    assert binding.fa_version() == 10000
+    for code in [0, -1, -2, -3, -4, -5, -6, -7, -8]:
+        assert binding.fa_status_string(code) != "unknown status"
+    assert binding.fa_status_string(12345) == "unknown status"
+
+
+def test_workspace_size():
+    B, H, N, d = 16, 16, 512, 64
+    R = B * H * N
+    ws = binding.fa_bwd_workspace_size(B, H, N, d)
+    assert ws >= 4 * R + 4 * R + 4 * R * d
+    assert ws % 256 == 0
+    assert binding.fa_bwd_workspace_size(1, 1, 100, 64) == 0      # N % 128
+    assert binding.fa_bwd_workspace_size(1, 1, 128, 96) == 0      # d
+    assert binding.fa_bwd_workspace_size(0, 1, 128, 64) == 0      # empty
+
+
+# Fake, well-aligned device addresses: validation fails before they are touched.
+P = 1 << 40
+
+
+def fwd(**kw):
+    a = dict(q=P, k=P, v=P, o=P, lse=P, B=1, H=1, N=128, d=64, scale=0.125, causal=0,
+             block_mask=None, kv_len=None)
+    a.update(kw)
+    lib = binding.load()
+    return lib.fa_fwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"], a["N"], a["d"],
+                      a["scale"], a["causal"], a["block_mask"], a["kv_len"], None)
+
+
+def bwd(**kw):
+    a = dict(q=P, k=P, v=P, o=P, lse=P, dout=P, dq=P, dk=P, dv=P, B=1, H=1, N=128, d=64,
+             scale=0.125, causal=0, block_mask=None, kv_len=None, ws=P, ws_bytes=1 << 30)
+    a.update(kw)
+    lib = binding.load()
+    return lib.fa_bwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["dout"], a["dq"], a["dk"],
+                      a["dv"], a["B"], a["H"], a["N"], a["d"], a["scale"], a["causal"],
+                      a["block_mask"], a["kv_len"], a["ws"], a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("call", [fwd, bwd])
+def test_shape_errors(call):
+    assert call(N=100) == -3
+    assert call(N=-128) == -3
+    assert call(B=-1) == -3
+    assert call(B=1 << 16, H=1 << 8, N=1 << 8) == -3   # B*H*N >= 2^31
+    assert call(d=96) == -4
+    assert call(d=32) == -4
+
+
+@pytest.mark.parametrize("call", [fwd, bwd])
+def test_empty_problems_are_no_ops(call):
+    assert call(B=0) == 0
+    assert call(H=0) == 0
+    assert call(N=0) == 0
+    # nothing is dereferenced for an empty problem, not even NULL pointers
+    assert call(B=0, q=None, k=None) == 0
+
+
+@pytest.mark.parametrize("call", [fwd, bwd])
+def test_null_and_alignment(call):
+    assert call(q=None) == -1
+    assert call(o=None) == -1 if call is fwd else call(dq=None) == -1
+    assert call(k=P + 8) == -2
+    assert call(lse=P + 2) == -2
+    assert call(kv_len=P + 1) == -2
+
+
+@pytest.mark.parametrize("call", [fwd, bwd])
+def test_scale_errors(call):
+    assert call(scale=0.0) == -8
+    assert call(scale=-1.0) == -8
+    assert call(scale=float("inf")) == -8
+    assert call(scale=float("nan")) == -8
+
+
+def test_backward_workspace_errors():
+    assert bwd(ws=None) == -5
+    assert bwd(ws_bytes=16) == -5
+    assert bwd(ws=P + 16) == -2
+
+
+def test_traced_variants_need_the_visit_buffer():
+    lib = binding.load()
+    rc = lib.fa_fwd_traced(P, P, P, P, P, 1, 1, 128, 64, 0.125, 0, None, None, None, None)
+    assert rc == -1
+    rc = lib.fa_bwd_traced(P, P, P, P, P, P, P, P, P, 1, 1, 128, 64, 0.125, 0, None, None, P,
+                           1 << 30, None, None)
+    assert rc == -1
+
+
+def test_backward_phase_number_is_checked():
+    lib = binding.load()
+    for ph in (-1, 3):
+        rc = lib.fa_bwd_phase(ph, P, P, P, P, P, P, P, P, P, 1, 1, 128, 64, 0.125, 0, None, None, P,
+                              1 << 30, None)
+        assert rc == -8

@@ -336,3 +336,56 @@ def test_tile_visits_agree_with_value_identity_probabilities():
         for j in range(3):
             blk = p[0, 0, i * 128:(i + 1) * 128, j * 128:(j + 1) * 128]
             assert bool(vis[i, j]) == bool(np.any(blk > 0)), (i, j)
+
+
+def test_backward_dq_rows_match_full_backward():
+    N, d = 384, 16
+    q, k, v, do = (rand((1, 1, N, d), t) for t in (39, 40, 41, 42))
+    bm = np.array([[1, 0, 1], [1, 1, 0], [0, 1, 1]], np.uint8)
+    rows = np.array([0, 7, 128, 200, 383])
+    for causal, kv in [(False, None), (True, 250)]:
+        kvl = None if kv is None else np.array([kv], np.int32)
+        dq, _, _, delta = oracle.attention_backward(q, k, v, do, 0.3, causal=causal,
+                                                    block_mask=bm, kv_len=kvl)
+        dqr, dr = oracle.attention_backward_dq_rows(q[0, 0, rows], do[0, 0, rows], rows, k[0, 0],
+                                                    v[0, 0], 0.3, causal=causal, block_mask=bm,
+                                                    kv_len_b=kv)
+        np.testing.assert_allclose(dqr, dq[0, 0, rows], atol=1e-13)
+        np.testing.assert_allclose(dr, delta[0, 0, rows], atol=1e-13)
+
+
+def test_backward_kv_cols_match_full_backward():
+    N, d = 640, 16
+    q, k, v, do = (rand((1, 1, N, d), t) for t in (43, 44, 45, 46))
+    bm = np.array([[1, 0, 1, 0, 1], [1, 1, 0, 0, 1], [0, 1, 1, 1, 0], [1, 0, 0, 1, 1],
+                   [0, 1, 1, 0, 1]], np.uint8)
+    cols = np.array([0, 5, 127, 128, 300, 511, 639])
+    for causal, kv in [(False, None), (True, 500)]:
+        kvl = None if kv is None else np.array([kv], np.int32)
+        _, dk, dv, _ = oracle.attention_backward(q, k, v, do, 0.3, causal=causal, block_mask=bm,
+                                                 kv_len=kvl)
+        for nt in (1, 3):
+            dkc, dvc = oracle.attention_backward_kv_cols(q[0, 0], k[0, 0], v[0, 0], do[0, 0], cols,
+                                                         0.3, causal=causal, block_mask=bm,
+                                                         kv_len_b=kv, nthreads=nt)
+            np.testing.assert_allclose(dkc, dk[0, 0, cols], atol=1e-12)
+            np.testing.assert_allclose(dvc, dv[0, 0, cols], atol=1e-12)
+
+
+def test_row_bands_partition_the_full_result():
+    N, d = 384, 8
+    q, k, v, do = (rand((1, 2, N, d), t) for t in (47, 48, 49, 50))
+    kvl = np.array([300], np.int32)
+    o, l = oracle.attention_forward(q, k, v, 0.4, causal=True, kv_len=kvl)
+    dq, dk, dv, _ = oracle.attention_backward(q, k, v, do, 0.4, causal=True, kv_len=kvl)
+    o1, l1 = oracle.attention_forward_band(q, k, v, 0.4, True, None, kvl, 0, 150)
+    o2, l2 = oracle.attention_forward_band(q, k, v, 0.4, True, None, kvl, 150, N)
+    np.testing.assert_array_equal(o1[:, :, :150], o[:, :, :150])
+    np.testing.assert_array_equal(o2[:, :, 150:], o[:, :, 150:])
+    np.testing.assert_array_equal(l2[:, :, 150:], l[:, :, 150:])
+    g1 = oracle.attention_backward_band(q, k, v, do, 0.4, True, None, kvl, 0, 150)
+    g2 = oracle.attention_backward_band(q, k, v, do, 0.4, True, None, kvl, 150, N)
+    np.testing.assert_array_equal(g1[0][:, :, :150], dq[:, :, :150])
+    np.testing.assert_array_equal(g2[0][:, :, 150:], dq[:, :, 150:])
+    np.testing.assert_allclose(g1[1] + g2[1], dk, atol=1e-13)
+    np.testing.assert_allclose(g1[2] + g2[2], dv, atol=1e-13)
