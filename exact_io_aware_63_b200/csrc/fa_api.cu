@@ -49,6 +49,21 @@ bool make_tmap(CUtensorMap* m, const void* base, long long rows, int d) {
   return r == CUDA_SUCCESS;
 }
 
+// [rows][d] float32 accumulator, boxes of 32 rows x 32 columns (128 bytes),
+// 128-byte swizzle: the target of the dQ TMA reduce-adds.
+bool make_tmap_f32_acc(CUtensorMap* m, const void* base, long long rows, int d) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 4};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 // Shape checks shared by every entry point.  Returns FA_OK, an error, or 1
@@ -153,9 +168,9 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
   float* delta = reinterpret_cast<float*>(ws + wl.delta);
   float* lse2 = reinterpret_cast<float*>(ws + wl.lse2);
   float* dq_acc = reinterpret_cast<float*>(ws + wl.dq_acc);
-  CUtensorMap tq, tk, tv, tdo;
+  CUtensorMap tq, tk, tv, tdo, tdq;
   if (!make_tmap(&tq, q, rows, D) || !make_tmap(&tk, k, rows, D) || !make_tmap(&tv, v, rows, D) ||
-      !make_tmap(&tdo, dout, rows, D))
+      !make_tmap(&tdo, dout, rows, D) || !make_tmap_f32_acc(&tdq, dq_acc, rows, D))
     return FA_ERR_CUDA;
   static bool smem_set = false;
   if (!smem_set) {
@@ -192,7 +207,7 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
     p.scale = scale;
     p.scale_log2 = scale * fa::kLog2e;
     const int grid = p.num_units < num_sms ? p.num_units : num_sms;
-    fa::fa_bwd_kernel<D><<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(tq, tk, tv, tdo, p);
+    fa::fa_bwd_kernel<D><<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdq, p);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   // dQ

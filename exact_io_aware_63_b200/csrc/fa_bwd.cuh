@@ -20,13 +20,15 @@
 //   warps 4-7   "dS" group, one key row per thread (TMEM lane): P^T, dS^T,
 //               and the dK / dV epilogue of each unit
 //   warps 8-11  "dQ" group, one query row per thread: drains dQ partials from
-//               TMEM and adds them into the float32 accumulator in HBM
+//               TMEM through shared memory into the float32 accumulator in
+//               HBM with TMA reduce-adds
 // Per visited query tile i the MMA thread issues, all accumulating in TMEM:
 //   S^T  = K_j Q_i^T          (cols   0..127)
 //   dP^T = V_j dO_i^T         (cols 128..255)
 //   dV  += P^T dO_i           (A = P^T bf16 in TMEM over S^T's first 64 cols)
 //   dK  += dS^T Q_i           (A = dS^T bf16 in TMEM over dP^T's first 64 cols)
-//   dQ   = dS K_j             (A = dS from shared memory; result over cols 0..D-1)
+//   dQ   = dS K_j             (A = dS from shared memory; result in cols 384..447
+//                             for D = 64, over S^T's cols 0..127 for D = 128)
 // dK and dV accumulate in cols 256..256+2D-1 for the whole unit.
 #pragma once
 
@@ -121,6 +123,10 @@ struct BwdParams {
 template <int D>
 struct BwdCfg {
   static constexpr int kThreads = 384;
+  // registers per thread: 168 at launch (384 x 168 = 64512); the producer /
+  // MMA warpgroup gives back 80 each, the two math warpgroups take 40 more:
+  // 128 x 88 + 256 x 208 = 64512.
+  static constexpr uint32_t kRegsLaunch = 168, kRegsLow = 88, kRegsHigh = 208;
   static constexpr int kTileBytes = kTile * D * 2;
   static constexpr int kBoxes = D / 64;
   static constexpr int kStages = (D == 64) ? 4 : 2;
@@ -128,7 +134,9 @@ struct BwdCfg {
   static constexpr int kOffV = kOffK + kTileBytes;
   static constexpr int kOffQ = kOffV + kTileBytes;
   static constexpr int kOffDO = kOffQ + kStages * kTileBytes;
-  static constexpr int kOffDS = kOffDO + kStages * kTileBytes;  // 128 x 128 bf16
+  // 128 x 128 bf16 dS tile for the dQ MMA; once that MMA has read it, the dQ
+  // group reuses it to stage float32 dQ partials for the TMA reduce-add.
+  static constexpr int kOffDS = kOffDO + kStages * kTileBytes;
   static constexpr int kOffBar = kOffDS + kTile * kTile * 2;
   // kv_full, kv_empty, qdo_full[S], qdo_empty[S], s_full, dp_full, p_full, ds_full,
   // ds_smem_empty, dq_full, dq_empty, dkv_full, drain
@@ -136,10 +144,16 @@ struct BwdCfg {
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kColS = 0;      // S^T, then P^T (bf16), then dQ
+  static constexpr uint32_t kColS = 0;      // S^T, then P^T (bf16)
   static constexpr uint32_t kColDP = 128;   // dP^T, then dS^T (bf16)
   static constexpr uint32_t kColDK = 256;
   static constexpr uint32_t kColDV = 256 + D;
+  // dQ = dS K_j: its own columns when they fit (D = 64), else over S^T
+  static constexpr uint32_t kColDQ = (D == 64) ? 384 : 0;
+  static constexpr bool kDqAliasesS = (kColDQ == kColS);
+  // dQ staging: each dQ warp owns 8 KB of the dS tile = two 32 x 32 float32 boxes
+  static constexpr int kDqBoxesPerRound = 2;
+  static constexpr int kDqRounds = D / 64;
 };
 
 struct BwdUnit {
@@ -179,17 +193,12 @@ __device__ __forceinline__ BwdUnit bwd_decode(const BwdParams& p, int u) {
   return w;
 }
 
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
-               "f"(c), "f"(d)
-               : "memory");
-}
 
 template <int D>
 __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                  const BwdParams p) {
+                  const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
   using Cfg = BwdCfg<D>;
   constexpr int S = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -221,7 +230,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     mbar_init(dp_full, 1);
     mbar_init(p_full, 128);
     mbar_init(ds_full, 128);
-    mbar_init(ds_smem_empty, 1);
+    mbar_init(ds_smem_empty, 4);  // one arrival per dQ warp
     mbar_init(dq_full, 1);
     mbar_init(dq_empty, 128);
     mbar_init(dkv_full, 1);
@@ -232,6 +241,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
     prefetch_tmap(&tm_do);
+    prefetch_tmap(&tm_dq);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_base_slot), Cfg::kTmemCols);
@@ -242,9 +252,12 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_base_slot;
   const int G = gridDim.x;
+  static_assert(Cfg::kRegsLow * 128 + Cfg::kRegsHigh * 256 <= Cfg::kRegsLaunch * Cfg::kThreads,
+                "register split exceeds the launch allocation");
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    setmaxnreg_dec<Cfg::kRegsLow>();
     if (lane == 0) {
       uint32_t kv_cnt = 0, qdo_cnt = 0;
       bool ok = true;
@@ -283,6 +296,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    setmaxnreg_dec<Cfg::kRegsLow>();
     if (lane == 0) {
       constexpr uint32_t idesc_kk = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T
       constexpr uint32_t idesc_tn = idesc_bf16_f32(128, D, 0, 1);    // dV, dK (A in TMEM)
@@ -304,8 +318,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
           const int s = qdo_cnt % S;
           ok = mbar_wait(qdo_full(s), (qdo_cnt / S) & 1);
           if (!ok) break;
-          ok = mbar_wait(dq_empty, (dq_cnt & 1) ^ 1);
-          if (!ok) break;
+          if (Cfg::kDqAliasesS) {  // S^T overwrites the previous dQ: wait for its drain
+            ok = mbar_wait(dq_empty, (dq_cnt & 1) ^ 1);
+            if (!ok) break;
+          }
           tc_fence_after();
           const uint32_t qa = sbase + Cfg::kOffQ + s * Cfg::kTileBytes;
           const uint32_t doa = sbase + Cfg::kOffDO + s * Cfg::kTileBytes;
@@ -340,6 +356,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
           ok = mbar_wait(ds_full, ds_cnt & 1);
           ++ds_cnt;
           if (!ok) break;
+          if (!Cfg::kDqAliasesS) {  // dQ columns must have been drained
+            ok = mbar_wait(dq_empty, (dq_cnt & 1) ^ 1);
+            if (!ok) break;
+          }
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
@@ -348,12 +368,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
                     (t > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
-            umma_ss(tmem + Cfg::kColS, sw128_desc(dsa + kk * 2048, 16384, 1024),
+            umma_ss(tmem + Cfg::kColDQ, sw128_desc(dsa + kk * 2048, 16384, 1024),
                     sw128_desc(ka + kk * 2048, 16384, 1024), idesc_dq, kk > 0 ? 1u : 0u);
           umma_commit(dq_full);
           ++dq_cnt;
           umma_commit(qdo_empty(s));
-          umma_commit(ds_smem_empty);
           ++qdo_cnt;
           if (*abort_flag) ok = false;
         }
@@ -366,8 +385,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       mbar_wait(drain_bar, 0);
     }
     __syncwarp();
-  } else if (warp >= 4 && warp < 8) {
+  } else if (warp < 4) {
+    setmaxnreg_dec<Cfg::kRegsLow>();  // idle warps of the first warpgroup
+  } else if (warp < 8) {
     // ------------------------------------------------------------ dS group
+    setmaxnreg_inc<Cfg::kRegsHigh>();
     const int quarter = warp & 3;
     const int kr = quarter * 32 + lane;  // key row within the tile
     const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
@@ -392,40 +414,41 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       }
       const bool key_valid = c_key < w.L;
       for (int i = bwd_next(p, w, w.i_begin); i < p.n_t; i = bwd_next(p, w, i + 1)) {
-        const float* lse2_t = p.lse2 + (size_t)w.bh * p.N + i * kTile;
-        const float* dl_t = p.delta + (size_t)w.bh * p.N + i * kTile;
+        const float4* lse2_t = reinterpret_cast<const float4*>(p.lse2 + (size_t)w.bh * p.N + i * kTile);
+        const float4* dl_t = reinterpret_cast<const float4*>(p.delta + (size_t)w.bh * p.N + i * kTile);
         const bool diag = p.causal && (i == w.j);
         ok = __all_sync(0xffffffffu, mbar_wait(s_full, s_cnt & 1));
         ++s_cnt;
         if (!ok) break;
         tc_fence_after();
-        // P^T row: p[q] = exp2(S^T[kr][q] * scale*log2e - lse2[q]), masked -> 0
-        uint32_t ppk[64];
-        {
-          uint32_t r[4][32];
+        // P^T row: p[q] = exp2(S^T[kr][q] * scale*log2e - lse2[q]); masked -> 0.
+        // Written as bf16 over the first 64 columns of S^T (A operand of dV).
 #pragma unroll
-          for (int c = 0; c < 4; ++c) tmem_ld32(t_lane + Cfg::kColS + c * 32, r[c]);
+        for (int h = 0; h < 2; ++h) {
+          uint32_t r[2][32];
+          tmem_ld32(t_lane + Cfg::kColS + h * 64, r[0]);
+          tmem_ld32(t_lane + Cfg::kColS + h * 64 + 32, r[1]);
           tmem_wait_ld();
+          reg_fence32(r[0]);
+          reg_fence32(r[1]);
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            reg_fence32(r[c]);
-            float lz[32];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const float4 v4 = __ldg(reinterpret_cast<const float4*>(lse2_t + c * 32) + e);
-              lz[4 * e] = v4.x; lz[4 * e + 1] = v4.y; lz[4 * e + 2] = v4.z; lz[4 * e + 3] = v4.w;
-            }
+          for (int cc = 0; cc < 2; ++cc) {
+            const int c = 2 * h + cc;
             uint32_t pk[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int q0 = c * 32 + 2 * e;
-              float p0 = ex2_approx(fmaf(__uint_as_float(r[c][2 * e]), p.scale_log2, -lz[2 * e]));
-              float p1 =
-                  ex2_approx(fmaf(__uint_as_float(r[c][2 * e + 1]), p.scale_log2, -lz[2 * e + 1]));
+            for (int e4 = 0; e4 < 8; ++e4) {
+              const float4 lz = __ldg(lse2_t + c * 8 + e4);
+              const int q0 = c * 32 + 4 * e4;
+              float p0 = ex2_approx(fmaf(__uint_as_float(r[cc][4 * e4]), p.scale_log2, -lz.x));
+              float p1 = ex2_approx(fmaf(__uint_as_float(r[cc][4 * e4 + 1]), p.scale_log2, -lz.y));
+              float p2 = ex2_approx(fmaf(__uint_as_float(r[cc][4 * e4 + 2]), p.scale_log2, -lz.z));
+              float p3 = ex2_approx(fmaf(__uint_as_float(r[cc][4 * e4 + 3]), p.scale_log2, -lz.w));
               if (!key_valid || (diag && kr > q0)) p0 = 0.f;
               if (!key_valid || (diag && kr > q0 + 1)) p1 = 0.f;
-              pk[e] = pack_bf16x2(p0, p1);
-              ppk[c * 16 + e] = pk[e];
+              if (!key_valid || (diag && kr > q0 + 2)) p2 = 0.f;
+              if (!key_valid || (diag && kr > q0 + 3)) p3 = 0.f;
+              pk[2 * e4] = pack_bf16x2(p0, p1);
+              pk[2 * e4 + 1] = pack_bf16x2(p2, p3);
             }
             tmem_st16(t_lane + Cfg::kColS + c * 16, pk);
           }
@@ -433,7 +456,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(p_full);
-        // dS^T row: ds[q] = p[q] * (dP^T[kr][q] - D[q])
+        // dS^T row: ds[q] = p[q] * (dP^T[kr][q] - D[q]), p read back (bf16) from TMEM
         ok = __all_sync(0xffffffffu, mbar_wait(dp_full, dp_cnt & 1));
         ++dp_cnt;
         if (!ok) break;
@@ -444,23 +467,24 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t r[32];
+          uint32_t pp[16];
           tmem_ld32(t_lane + Cfg::kColDP + c * 32, r);
+          tmem_ld16(t_lane + Cfg::kColS + c * 16, pp);
           tmem_wait_ld();
           reg_fence32(r);
-          float dz[32];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float4 v4 = __ldg(reinterpret_cast<const float4*>(dl_t + c * 32) + e);
-            dz[4 * e] = v4.x; dz[4 * e + 1] = v4.y; dz[4 * e + 2] = v4.z; dz[4 * e + 3] = v4.w;
-          }
+          reg_fence16(pp);
           uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float2 pp =
-                __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ppk[c * 16 + e]));
-            const float ds0 = pp.x * (__uint_as_float(r[2 * e]) - dz[2 * e]);
-            const float ds1 = pp.y * (__uint_as_float(r[2 * e + 1]) - dz[2 * e + 1]);
-            pk[e] = pack_bf16x2(ds0, ds1);
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const float4 dz = __ldg(dl_t + c * 8 + e4);
+            const float2 pa =
+                __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pp[2 * e4]));
+            const float2 pb =
+                __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pp[2 * e4 + 1]));
+            pk[2 * e4] = pack_bf16x2(pa.x * (__uint_as_float(r[4 * e4]) - dz.x),
+                                     pa.y * (__uint_as_float(r[4 * e4 + 1]) - dz.y));
+            pk[2 * e4 + 1] = pack_bf16x2(pb.x * (__uint_as_float(r[4 * e4 + 2]) - dz.z),
+                                         pb.y * (__uint_as_float(r[4 * e4 + 3]) - dz.w));
           }
           tmem_st16(t_lane + Cfg::kColDP + c * 16, pk);
           // shared-memory copy for the dQ MMA: [key][query], 64-query chunks 16 KB
@@ -512,11 +536,16 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       tc_fence_before();
     }
     if (!ok) *abort_flag = 1;
-  } else if (warp >= 8) {
+  } else {
     // ------------------------------------------------------------ dQ group
-    const int quarter = warp & 3;
-    const int qr = quarter * 32 + lane;  // query row within the tile
+    setmaxnreg_inc<Cfg::kRegsHigh>();
+    // Drains dQ partials: TMEM -> registers -> shared memory (the dS tile,
+    // free once the dQ MMA has read it) -> TMA reduce-add into the float32
+    // accumulator, in 32 x 32 boxes (128-byte swizzled rows).
+    const int quarter = warp & 3;  // rows quarter*32 .. +31 of the query tile
     const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
+    uint8_t* stage = smem + Cfg::kOffDS + quarter * (Cfg::kDqBoxesPerRound * 4096);
+    const uint32_t stage_u32 = smem_u32(stage);
     uint32_t dq_cnt = 0;
     bool ok = true;
     for (int round = 0; ok; ++round) {
@@ -531,23 +560,42 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         tc_fence_after();
         uint32_t r[D / 32][32];
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) tmem_ld32(t_lane + Cfg::kColS + c * 32, r[c]);
+        for (int c = 0; c < D / 32; ++c) tmem_ld32(t_lane + Cfg::kColDQ + c * 32, r[c]);
         tmem_wait_ld();
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) reg_fence32(r[c]);
         tc_fence_before();
         mbar_arrive(dq_empty);
-        float* dst = p.dq_acc + ((size_t)w.bh * p.N + i * kTile + qr) * D;
+        const int y = w.bh * p.N + i * kTile + quarter * 32;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c)
+        for (int rd = 0; rd < Cfg::kDqRounds; ++rd) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            red_add_v4(dst + c * 32 + 4 * e, __uint_as_float(r[c][4 * e]),
-                       __uint_as_float(r[c][4 * e + 1]), __uint_as_float(r[c][4 * e + 2]),
-                       __uint_as_float(r[c][4 * e + 3]));
+          for (int bxi = 0; bxi < Cfg::kDqBoxesPerRound; ++bxi) {
+            const int c = rd * Cfg::kDqBoxesPerRound + bxi;
+            uint8_t* rowp = stage + bxi * 4096 + lane * 128;
+#pragma unroll
+            for (int g = 0; g < 8; ++g)
+              *reinterpret_cast<uint4*>(rowp + ((g ^ (lane & 7)) << 4)) =
+                  make_uint4(r[c][4 * g], r[c][4 * g + 1], r[c][4 * g + 2], r[c][4 * g + 3]);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+#pragma unroll
+            for (int bxi = 0; bxi < Cfg::kDqBoxesPerRound; ++bxi)
+              tma_reduce_add_2d(&tm_dq, (rd * Cfg::kDqBoxesPerRound + bxi) * 32, y,
+                                stage_u32 + bxi * 4096);
+            bulk_commit_group();
+            bulk_wait_group_read0();
+          }
+          __syncwarp();
+        }
+        if (lane == 0) mbar_arrive(ds_smem_empty);
         if (*abort_flag) { ok = false; break; }
       }
     }
+    if (lane == 0) bulk_wait_group0();
+    __syncwarp();
     if (!ok) *abort_flag = 1;
   }
 

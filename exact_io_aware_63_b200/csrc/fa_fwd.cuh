@@ -60,6 +60,10 @@ struct FwdParams {
 template <int D>
 struct FwdCfg {
   static constexpr int kThreads = 384;
+  // registers per thread: 168 at launch (384 x 168 = 64512); the producer /
+  // MMA warpgroup gives back 64 each, the two softmax warpgroups take 32 more:
+  // 128 x 104 + 256 x 200 = 64512.
+  static constexpr uint32_t kRegsLaunch = 168, kRegsLow = 104, kRegsHigh = 200;
   static constexpr int kTileBytes = kTile * D * 2;  // one 128 x D bf16 tile
   static constexpr int kBoxes = D / 64;             // 64-column TMA boxes per tile
   static constexpr int kStages = (D == 64) ? 4 : 2;
@@ -195,9 +199,12 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_base_slot;
   const int G = gridDim.x;
+  static_assert(Cfg::kRegsLow * 128 + Cfg::kRegsHigh * 256 <= Cfg::kRegsLaunch * Cfg::kThreads,
+                "register split exceeds the launch allocation");
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    setmaxnreg_dec<Cfg::kRegsLow>();
     if (lane == 0) {
       uint32_t q_cnt[2] = {0, 0};
       uint32_t kv_cnt = 0;
@@ -243,6 +250,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    setmaxnreg_dec<Cfg::kRegsLow>();
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
@@ -251,23 +259,28 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
       uint32_t kv_cnt = 0;
       bool ok = true;
 
+      // Descriptors: one base per tile; the start-address field (bits 0..13,
+      // address >> 4) is advanced by adding (byte offset >> 4).  Tiles lie in
+      // the first 256 KB of shared memory, so the field never carries over.
+      const uint64_t desc_q0 = sw128_desc(sbase + Cfg::kOffQ, 16, 1024);
+      const uint64_t desc_k0 = sw128_desc(sbase + Cfg::kOffK, 16, 1024);
+      const uint64_t desc_v0 = sw128_desc(sbase + Cfg::kOffV, 16384, 1024);
       auto issue_s = [&](int x, int s) {
-        const uint32_t qa = sbase + Cfg::kOffQ + x * Cfg::kTileBytes;
-        const uint32_t ka = sbase + Cfg::kOffK + s * Cfg::kTileBytes;
+        const uint64_t dq = desc_q0 + ((x * Cfg::kTileBytes) >> 4);
+        const uint64_t dk = desc_k0 + ((s * Cfg::kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_ss(tmem + Cfg::col_s(x), sw128_desc(qa + off, 16, 1024),
-                  sw128_desc(ka + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+          umma_ss(tmem + Cfg::col_s(x), dq + off, dk + off, idesc_s, kk > 0 ? 1u : 0u);
         }
         umma_commit(s_full(x));
       };
       auto issue_pv = [&](int x, int s, uint32_t acc) {
-        const uint32_t va = sbase + Cfg::kOffV + s * Cfg::kTileBytes;
+        const uint64_t dv = desc_v0 + ((s * Cfg::kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk) {
-          umma_ts(tmem + Cfg::col_o(x), tmem + Cfg::col_s(x) + kk * 8,
-                  sw128_desc(va + kk * 2048, 16384, 1024), idesc_pv, (kk > 0 || acc) ? 1u : 0u);
+          umma_ts(tmem + Cfg::col_o(x), tmem + Cfg::col_s(x) + kk * 8, dv + ((kk * 2048) >> 4),
+                  idesc_pv, (kk > 0 || acc) ? 1u : 0u);
         }
       };
 
@@ -351,8 +364,11 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
       mbar_wait(drain_bar, 0);
     }
     __syncwarp();
-  } else if (warp >= 4) {
+  } else if (warp < 4) {
+    setmaxnreg_dec<Cfg::kRegsLow>();  // idle warps of the first warpgroup
+  } else {
     // ------------------------------------------------------------ softmax
+    setmaxnreg_inc<Cfg::kRegsHigh>();
     const int x = (warp >= 8) ? 1 : 0;
     const int quarter = warp & 3;
     const int r_local = quarter * 32 + lane;  // row within the query tile = TMEM lane
