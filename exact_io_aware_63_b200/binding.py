@@ -8,6 +8,7 @@ import of a function raises.
 Raw entry points (same argument order as the C ABI; tensors are passed as
 torch tensors or None, the stream as a torch.cuda.Stream or None = current):
 ``fa_fwd``, ``fa_fwd_traced``, ``fa_bwd``, ``fa_bwd_traced``, ``fa_bwd_phase``,
+``fa_bwd_noalloc``,
 ``fa_bwd_workspace_size``, ``fa_get_device_status``, ``fa_status_string``,
 ``fa_version``.
 
@@ -38,6 +39,7 @@ _SIGS = {
     "fa_bwd": (_i, [_vp] * 9 + [_i, _i, _i, _i, _f, _i, _vp, _vp, _vp, _sz, _vp]),
     "fa_bwd_traced": (_i, [_vp] * 9 + [_i, _i, _i, _i, _f, _i, _vp, _vp, _vp, _sz, _vp, _vp]),
     "fa_bwd_phase": (_i, [_i] + [_vp] * 9 + [_i, _i, _i, _i, _f, _i, _vp, _vp, _vp, _sz, _vp]),
+    "fa_bwd_noalloc": (_i, [_vp] * 9 + [_i, _i, _i, _i, _f, _i, _vp, _vp, _vp]),
     "fa_get_device_status": (_i, [_vp]),
     "fa_status_string": (ctypes.c_char_p, [_i]),
     "fa_version": (_i, []),
@@ -46,7 +48,10 @@ _SIGS = {
 FA_OK = 0
 STATUS_NAMES = {0: "FA_OK", -1: "FA_ERR_NULL", -2: "FA_ERR_ALIGN", -3: "FA_ERR_SHAPE",
                 -4: "FA_ERR_UNSUPPORTED_D", -5: "FA_ERR_WORKSPACE", -6: "FA_ERR_CUDA",
-                -7: "FA_ERR_TIMEOUT", -8: "FA_ERR_ARG"}
+                -7: "FA_ERR_TIMEOUT", -8: "FA_ERR_ARG", -9: "FA_ERR_SCRATCH_LIMIT"}
+
+# size of the library's built-in scratch for fa_bwd_noalloc (FA_BWD_NOALLOC_SCRATCH_BYTES)
+BWD_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 class FAError(RuntimeError):
@@ -140,6 +145,16 @@ def fa_bwd_phase(phase, q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, ca
                                _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, float(scale),
                                int(bool(causal)), _ptr(block_mask), _ptr(kv_len), _ptr(workspace),
                                int(workspace_bytes), _stream(stream))
+
+
+def fa_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, block_mask,
+                   kv_len, stream=None):
+    """fa_bwd without a workspace argument: the library's built-in static scratch is used
+    (for callers that cannot allocate device memory; see include/fa.h)."""
+    return load().fa_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
+                                 _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, float(scale),
+                                 int(bool(causal)), _ptr(block_mask), _ptr(kv_len),
+                                 _stream(stream))
 
 
 def fa_get_device_status(stream=None):

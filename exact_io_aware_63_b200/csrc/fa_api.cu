@@ -348,6 +348,8 @@ const char* fa_status_string(int status) {
     case FA_ERR_CUDA: return "a CUDA runtime or driver call failed";
     case FA_ERR_TIMEOUT: return "a device pipeline wait timed out; outputs are incomplete";
     case FA_ERR_ARG: return "invalid argument (scale not finite or not > 0, or unknown phase)";
+    case FA_ERR_SCRATCH_LIMIT:
+      return "shape needs more backward scratch than the built-in FA_BWD_NOALLOC_SCRATCH_BYTES";
     default: return "unknown status";
   }
 }
@@ -355,3 +357,59 @@ const char* fa_status_string(int status) {
 int fa_version(void) { return kVersion; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// fa_bwd_noalloc: the backward pass with its scratch in a static device array,
+// for callers that cannot allocate device memory.  The array is the whole
+// workspace of fa_bwd (same layout); kernels receive its device address as
+// an ordinary pointer.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char fa_bwd_noalloc_scratch[FA_BWD_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of fa_bwd_noalloc_scratch on the current device `dev`, looked
+// up once per device and cached.  In host code the array's name is only a
+// host-side handle, never a usable device address.
+int noalloc_scratch(int dev, void** out) {
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+  std::lock_guard<std::mutex> guard(g_noalloc_mutex);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, fa_bwd_noalloc_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return FA_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" int fa_bwd_noalloc(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v,
+                              const fa_bf16* o, const float* lse, const fa_bf16* dout,
+                              fa_bf16* dq, fa_bf16* dk, fa_bf16* dv, int B, int H, int N, int d,
+                              float scale, int causal, const uint8_t* block_mask,
+                              const int32_t* kv_len, void* stream) {
+  int rc = check_shape(B, H, N, d);
+  if (rc == 1) return FA_OK;
+  if (rc != FA_OK) return rc;
+  const size_t need = ws_layout(B, H, N, d).total;
+  if (need > static_cast<size_t>(FA_BWD_NOALLOC_SCRATCH_BYTES)) return FA_ERR_SCRATCH_LIMIT;
+  if (!q) return FA_ERR_NULL;
+  if (!aligned(q, 16)) return FA_ERR_ALIGN;
+  if (select_device(q) <= 0) return FA_ERR_CUDA;  // makes q's device current
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  void* scratch = nullptr;
+  rc = noalloc_scratch(dev, &scratch);
+  if (rc != FA_OK) return rc;
+  return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, block_mask, kv_len,
+                  scratch, static_cast<size_t>(FA_BWD_NOALLOC_SCRATCH_BYTES), nullptr, stream);
+}

@@ -62,7 +62,9 @@ typedef enum {
     FA_ERR_WORKSPACE = -5,      /* workspace NULL or smaller than fa_bwd_workspace_size */
     FA_ERR_CUDA = -6,           /* a CUDA runtime/driver call failed */
     FA_ERR_TIMEOUT = -7,        /* a device pipeline wait gave up (fa_get_device_status) */
-    FA_ERR_ARG = -8             /* scale not finite or not > 0, or phase not in 0..2 */
+    FA_ERR_ARG = -8,            /* scale not finite or not > 0, or phase not in 0..2 */
+    FA_ERR_SCRATCH_LIMIT = -9   /* fa_bwd_noalloc: the shape needs more scratch than
+                                   FA_BWD_NOALLOC_SCRATCH_BYTES */
 } fa_status;
 
 /*
@@ -137,6 +139,41 @@ int fa_bwd_phase(int phase, const fa_bf16* q, const fa_bf16* k, const fa_bf16* v
                  fa_bf16* dv, int B, int H, int N, int d, float scale, int causal,
                  const uint8_t* block_mask, const int32_t* kv_len, void* workspace,
                  size_t workspace_bytes, void* stream);
+
+/*
+ * Size in bytes of the library's built-in backward scratch buffer (64 MiB),
+ * used only by fa_bwd_noalloc.
+ */
+#define FA_BWD_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+/*
+ * fa_bwd without a caller-provided workspace, for callers that cannot
+ * allocate device memory themselves: code that runs where the host side owns
+ * no device allocator (a plugin handed only input and output buffers by its
+ * host application), or deployments that forbid device allocations after
+ * start-up.  The paper has no counterpart; this is an interface convenience.
+ *
+ * Same arguments and results as fa_bwd, minus the workspace.  The scratch
+ * (D, base-2 LSE and the float32 dQ accumulator) lives in one static device
+ * array of FA_BWD_NOALLOC_SCRATCH_BYTES inside the library, which every GPU
+ * that loads the library holds until the process exits.  The call allocates
+ * and frees nothing.
+ *  - Shapes whose scratch (fa_bwd_workspace_size) exceeds that size return
+ *    FA_ERR_SCRATCH_LIMIT and launch nothing.  With d = 64 that admits
+ *    B*H*N up to about 254K rows; with d = 128 about 129K rows.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current) and caches it; make
+ *    that first call before any stream capture.
+ *  - Every call on a device shares the one array.  Each call overwrites what
+ *    it reads (the accumulator is zeroed by the call's first kernel), so the
+ *    contents a previous call left behind do not matter, but calls whose
+ *    kernels overlap on the device (two streams, or two host threads) race
+ *    on the array and give wrong results: serialise them.
+ */
+int fa_bwd_noalloc(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf16* o,
+                   const float* lse, const fa_bf16* dout, fa_bf16* dq, fa_bf16* dk, fa_bf16* dv,
+                   int B, int H, int N, int d, float scale, int causal,
+                   const uint8_t* block_mask, const int32_t* kv_len, void* stream);
 
 /*
  * Synchronises `stream`, then returns FA_OK if no kernel of this library
