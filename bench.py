@@ -184,6 +184,19 @@ class ClockSampler:
                 "samples": len(window)}
 
 
+def workload_or_shape(args):
+    """The named workload, or (with --shape B,H,N,d) the same kind of inputs at another
+    size (used for profiling captures on a smaller case)."""
+    from exact_io_aware_63_b200 import inputs
+    if not args.shape:
+        return inputs.workload_inputs(args.workload)
+    w = inputs.WORKLOADS[args.workload]
+    B, H, N, d = (int(t) for t in args.shape.split(","))
+    return inputs.make_inputs(B, H, N, d, scale=w.scale if d == w.d else None, causal=w.causal,
+                              seed=w.seed, key_padding=(N // 2, N) if w.key_padding else None,
+                              block_keep=(1.0 / 16.0) if w.block_sparse else None)
+
+
 # ----------------------------------------------------------------------------
 # our arm
 # ----------------------------------------------------------------------------
@@ -206,7 +219,7 @@ def run_ours(args):
     binding.load(build_if_missing=False)
 
     w = inputs.WORKLOADS[args.workload]
-    x = inputs.workload_inputs(args.workload)
+    x = workload_or_shape(args)
     B, H, N, d = x.q.shape
     q, k, v, do = (t.to(dev) for t in (x.q, x.k, x.v, x.dout))
     bm = None if x.block_mask is None else x.block_mask.to(dev)
@@ -350,7 +363,8 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_t, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": args.workload, "description": w.description,
+        "config": {"workload": args.workload + (f" at shape {args.shape}" if args.shape else ""),
+                   "description": w.description,
                    "B": B, "H": H, "N": N, "d": d, "causal": causal,
                    "key_padding": x.kv_len is not None, "block_sparse": x.block_mask is not None,
                    "flop_density": density(x), "seed": w.seed,
@@ -487,7 +501,8 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": args.workload, "description": w.description, "B": B, "H": H,
+            "config": {"workload": args.workload + (f" at shape {args.shape}" if args.shape else ""),
+                   "description": w.description, "B": B, "H": H,
                        "N": N, "d": d, "parallelism": "cpu threads"},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": used, "kind": "oracle",
                              "sample": sample},
@@ -503,6 +518,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="bert")
+    ap.add_argument("--shape", default="",
+                    help="B,H,N,d: the workload's kind of inputs at another size (profiling)")
     ap.add_argument("--clock-window", type=float, default=1.5,
                     help="seconds of untimed load before timing, sampled for clocks")
     ap.add_argument("--cpu-budget", type=float, default=20.0,

@@ -108,6 +108,14 @@ bool set_smem(Kernel k, int bytes) {
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Heads per work-unit group: as many as keep `bytes_per_head` of re-read data
+// within a 48 MB share of the 126 MB L2.
+int heads_per_group(int BH, double bytes_per_head) {
+  const double budget = 48.0 * 1024 * 1024;
+  int g = static_cast<int>(budget / bytes_per_head);
+  return g < 1 ? 1 : (g > BH ? BH : g);
+}
+
 struct WsLayout {
   size_t delta, lse2, dq_acc, total;
 };
@@ -146,8 +154,8 @@ int launch_fwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o,
   p.H = H;
   p.N = N;
   p.n_t = N / fa::kTile;
-  p.num_pairs = (p.n_t + 1) / 2;
-  p.num_units = B * H * p.num_pairs;
+  p.num_units = B * H * p.n_t;
+  p.heads_per_group = heads_per_group(B * H, 4.0 * N * D);  // K and V
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * fa::kLog2e;
   const int grid = p.num_units < num_sms ? p.num_units : num_sms;
@@ -203,6 +211,7 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
     p.N = N;
     p.n_t = N / fa::kTile;
     p.num_units = B * H * p.n_t;
+    p.heads_per_group = heads_per_group(B * H, 8.0 * N * D);  // Q, dO, f32 dQ accumulator
     p.causal = causal ? 1 : 0;
     p.scale = scale;
     p.scale_log2 = scale * fa::kLog2e;
@@ -332,7 +341,7 @@ int fa_get_device_status(void* stream) {
   if (v != 0) {
     const unsigned int z = 0;
     if (cudaMemcpyToSymbol(fa::g_device_status, &z, sizeof(z)) != cudaSuccess) return FA_ERR_CUDA;
-    return FA_ERR_TIMEOUT;
+    return (v & fa::FA_DEV_TIMEOUT) ? FA_ERR_TIMEOUT : FA_ERR_CUDA;
   }
   return FA_OK;
 }

@@ -13,13 +13,15 @@
 //   fa_bwd_kernel        one CTA per (b, h, 128-key tile j), persistent
 //   fa_bwd_dq_kernel     dQ = bf16(scale * accumulator)
 //
-// fa_bwd_kernel roles (12 warps):
-//   warp 0      TMA producer: K_j, V_j once per unit; Q_i, dO_i per visited
-//               query tile through a kStages-deep ring
+// fa_bwd_kernel roles (16 warps):
+//   warp 0      TMA producer: K_j, V_j once per unit; Q_i, dO_i and the
+//               tile's LSE*log2(e) and D rows per visited query tile through a
+//               kStages-deep ring
 //   warp 1      MMA issuer (one thread), TMEM owner
-//   warps 4-7   "dS" group, one key row per thread (TMEM lane): P^T, dS^T,
-//               and the dK / dV epilogue of each unit
-//   warps 8-11  "dQ" group, one query row per thread: drains dQ partials from
+//   warps 4-11  two "dS" warpgroups, one key row per thread (TMEM lane), each
+//               on half of the 128 query columns: P^T, dS^T, and the dK (first
+//               warpgroup) / dV (second) epilogue of each unit
+//   warps 12-15 "dQ" group, one query row per thread: drains dQ partials from
 //               TMEM through shared memory into the float32 accumulator in
 //               HBM with TMA reduce-adds
 // Per visited query tile i the MMA thread issues, all accumulating in TMEM:
@@ -115,6 +117,7 @@ struct BwdParams {
   uint8_t* visited;
   int B, H, N, n_t;
   int num_units;
+  int heads_per_group;  // unit order: see bwd_decode
   int causal;
   float scale;
   float scale_log2;
@@ -122,11 +125,15 @@ struct BwdParams {
 
 template <int D>
 struct BwdCfg {
-  static constexpr int kThreads = 384;
-  // registers per thread: 168 at launch (384 x 168 = 64512); the producer /
-  // MMA warpgroup gives back 80 each, the two math warpgroups take 40 more:
-  // 128 x 88 + 256 x 208 = 64512.
-  static constexpr uint32_t kRegsLaunch = 168, kRegsLow = 88, kRegsHigh = 208;
+  static constexpr int kThreads = 512;
+  // registers per thread: 128 at launch (512 x 128 = 65536); the producer /
+  // MMA warpgroup drops to 88 and the rest is shared by the two dS
+  // warpgroups and the dQ warpgroup (which holds a whole float32 dQ row):
+  // D = 64:  128 x 88 + 256 x 136 + 128 x 120 = 61440
+  // D = 128: 128 x 88 + 256 x 128 + 128 x 168 = 65536
+  static constexpr uint32_t kRegsLaunch = 128, kRegsLow = 88;
+  static constexpr uint32_t kRegsDs = (D == 64) ? 136 : 128;
+  static constexpr uint32_t kRegsDq = (D == 64) ? 120 : 168;
   static constexpr int kTileBytes = kTile * D * 2;
   static constexpr int kBoxes = D / 64;
   static constexpr int kStages = (D == 64) ? 4 : 2;
@@ -137,15 +144,23 @@ struct BwdCfg {
   // 128 x 128 bf16 dS tile for the dQ MMA; once that MMA has read it, the dQ
   // group reuses it to stage float32 dQ partials for the TMA reduce-add.
   static constexpr int kOffDS = kOffDO + kStages * kTileBytes;
-  static constexpr int kOffBar = kOffDS + kTile * kTile * 2;
+  // per stage: LSE*log2(e) and D of the stage's 128 query rows
+  static constexpr int kOffRow = kOffDS + kTile * kTile * 2;
+  static constexpr int kRowBytes = kTile * 4;
+  static constexpr int kOffBar = kOffRow + 2 * kStages * kRowBytes;
   // kv_full, kv_empty, qdo_full[S], qdo_empty[S], s_full, dp_full, p_full, ds_full,
   // ds_smem_empty, dq_full, dq_empty, dkv_full, drain
   static constexpr int kNumBars = 2 + 2 * kStages + 9;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+  static constexpr int kSmemBytes = kOffMisc + 16;
+  static_assert(kSmemBytes <= 232448, "shared memory over the per-block limit");
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kColS = 0;      // S^T, then P^T (bf16)
-  static constexpr uint32_t kColDP = 128;   // dP^T, then dS^T (bf16)
+  // S^T fp32 in cols 0..127; the two math warpgroups each own 64 of them
+  // (queries 0..63 and 64..127) and write their P^T (bf16, 32 packed cols)
+  // over the start of their own 64: P^T for queries 16k..16k+15 sits at
+  // kColS + (k / 4) * 64 + (k % 4) * 8.  The same for dP^T / dS^T at kColDP.
+  static constexpr uint32_t kColS = 0;
+  static constexpr uint32_t kColDP = 128;
   static constexpr uint32_t kColDK = 256;
   static constexpr uint32_t kColDV = 256 + D;
   // dQ = dS K_j: its own columns when they fit (D = 64), else over S^T
@@ -154,6 +169,10 @@ struct BwdCfg {
   // dQ staging: each dQ warp owns 8 KB of the dS tile = two 32 x 32 float32 boxes
   static constexpr int kDqBoxesPerRound = 2;
   static constexpr int kDqRounds = D / 64;
+  // TMEM column of the bf16 operand for K-step kk (16 queries) of the dV / dK MMAs
+  __device__ static constexpr uint32_t packed_col(uint32_t base, int kk) {
+    return base + (kk >> 2) * 64 + (kk & 3) * 8;
+  }
 };
 
 struct BwdUnit {
@@ -176,12 +195,11 @@ __device__ __forceinline__ int bwd_next(const BwdParams& p, const BwdUnit& w, in
 }
 
 __device__ __forceinline__ BwdUnit bwd_decode(const BwdParams& p, int u) {
+  // heads in groups whose Q, dO and dQ accumulator fit in a share of L2; inside
+  // a group key tile 0 first (for causal masks it sees the most queries)
   BwdUnit w;
-  const int BH = p.B * p.H;
-  const int rank = u / BH;  // key tile; for causal masks tile 0 sees the most queries
-  w.bh = u - rank * BH;
+  group_order(u, p.n_t, p.B * p.H, p.heads_per_group, w.bh, w.j);
   w.b = w.bh / p.H;
-  w.j = rank;
   int L = p.N;
   if (p.kv_len) {
     L = __ldg(p.kv_len + w.b);
@@ -201,9 +219,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
                   const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
   using Cfg = BwdCfg<D>;
   constexpr int S = Cfg::kStages;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if (!smem_aligned_1024(smem)) return;
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + Cfg::kOffBar;
   const uint32_t kv_full = bar0, kv_empty = bar0 + 8;
@@ -215,6 +232,12 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
   const uint32_t dkv_full = s_full + 56, drain_bar = s_full + 64;
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kOffMisc + 4);
+  auto lse2_smem = [&](int s) {
+    return reinterpret_cast<const float4*>(smem + Cfg::kOffRow + s * Cfg::kRowBytes);
+  };
+  auto delta_smem = [&](int s) {
+    return reinterpret_cast<const float4*>(smem + Cfg::kOffRow + (S + s) * Cfg::kRowBytes);
+  };
 
   const int warp = warp_id();
   const int lane = lane_id();
@@ -228,8 +251,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
-    mbar_init(p_full, 128);
-    mbar_init(ds_full, 128);
+    mbar_init(p_full, 256);
+    mbar_init(ds_full, 256);
     mbar_init(ds_smem_empty, 4);  // one arrival per dQ warp
     mbar_init(dq_full, 1);
     mbar_init(dq_empty, 128);
@@ -252,7 +275,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_base_slot;
   const int G = gridDim.x;
-  static_assert(Cfg::kRegsLow * 128 + Cfg::kRegsHigh * 256 <= Cfg::kRegsLaunch * Cfg::kThreads,
+  static_assert(Cfg::kRegsLow * 128 + Cfg::kRegsDs * 256 + Cfg::kRegsDq * 128 <=
+                    Cfg::kRegsLaunch * Cfg::kThreads,
                 "register split exceeds the launch allocation");
 
   if (warp == 0) {
@@ -280,13 +304,17 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
           ok = mbar_wait(qdo_empty(s), ((qdo_cnt / S) & 1) ^ 1);
           if (!ok) break;
           const int qrow = w.bh * p.N + i * kTile;
-          mbar_arrive_expect_tx(qdo_full(s), 2 * Cfg::kTileBytes);
+          mbar_arrive_expect_tx(qdo_full(s), 2 * Cfg::kTileBytes + 2 * Cfg::kRowBytes);
           for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
             tma_load_2d(sbase + Cfg::kOffQ + s * Cfg::kTileBytes + bx * 16384, &tm_q, bx * 64, qrow,
                         qdo_full(s));
             tma_load_2d(sbase + Cfg::kOffDO + s * Cfg::kTileBytes + bx * 16384, &tm_do, bx * 64,
                         qrow, qdo_full(s));
           }
+          bulk_load(sbase + Cfg::kOffRow + s * Cfg::kRowBytes, p.lse2 + qrow, Cfg::kRowBytes,
+                    qdo_full(s));
+          bulk_load(sbase + Cfg::kOffRow + (S + s) * Cfg::kRowBytes, p.delta + qrow,
+                    Cfg::kRowBytes, qdo_full(s));
           ++qdo_cnt;
         }
         if (*abort_flag) ok = false;
@@ -303,8 +331,15 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       constexpr uint32_t idesc_dq = idesc_bf16_f32(128, D, 1, 1);    // dQ (both MN-major)
       uint32_t kv_cnt = 0, qdo_cnt = 0, p_cnt = 0, ds_cnt = 0, dq_cnt = 0;
       bool ok = true;
-      const uint32_t ka = sbase + Cfg::kOffK, va = sbase + Cfg::kOffV;
-      const uint32_t dsa = sbase + Cfg::kOffDS;
+      // one descriptor base per operand; offsets are added to the start-address field
+      const uint64_t dk_k = sw128_desc(sbase + Cfg::kOffK, 16, 1024);     // K_j, K-major
+      const uint64_t dv_k = sw128_desc(sbase + Cfg::kOffV, 16, 1024);     // V_j, K-major
+      const uint64_t dq_k0 = sw128_desc(sbase + Cfg::kOffQ, 16, 1024);    // Q_i, K-major
+      const uint64_t ddo_k0 = sw128_desc(sbase + Cfg::kOffDO, 16, 1024);  // dO_i, K-major
+      const uint64_t dq_m0 = sw128_desc(sbase + Cfg::kOffQ, 16384, 1024);    // Q_i, MN-major
+      const uint64_t ddo_m0 = sw128_desc(sbase + Cfg::kOffDO, 16384, 1024);  // dO_i, MN-major
+      const uint64_t dk_m = sw128_desc(sbase + Cfg::kOffK, 16384, 1024);     // K_j, MN-major
+      const uint64_t dds_m = sw128_desc(sbase + Cfg::kOffDS, 16384, 1024);   // dS, MN-major
       for (int round = 0; ok; ++round) {
         const int u = unit_for_round(round, blockIdx.x, G);
         if (u >= p.num_units) break;
@@ -323,23 +358,21 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
             if (!ok) break;
           }
           tc_fence_after();
-          const uint32_t qa = sbase + Cfg::kOffQ + s * Cfg::kTileBytes;
-          const uint32_t doa = sbase + Cfg::kOffDO + s * Cfg::kTileBytes;
-          // S^T = K_j Q_i^T
+          const uint32_t stage_off = (s * Cfg::kTileBytes) >> 4;
+          // S^T = K_j Q_i^T ; dP^T = V_j dO_i^T
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            umma_ss(tmem + Cfg::kColS, sw128_desc(ka + off, 16, 1024),
-                    sw128_desc(qa + off, 16, 1024), idesc_kk, kk > 0 ? 1u : 0u);
+            const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+            umma_ss(tmem + Cfg::kColS, dk_k + off, dq_k0 + stage_off + off, idesc_kk,
+                    kk > 0 ? 1u : 0u);
           }
           umma_commit(s_full);
           if (p.visited) p.visited[((size_t)w.bh * p.n_t + i) * p.n_t + w.j] = 1;
-          // dP^T = V_j dO_i^T
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            umma_ss(tmem + Cfg::kColDP, sw128_desc(va + off, 16, 1024),
-                    sw128_desc(doa + off, 16, 1024), idesc_kk, kk > 0 ? 1u : 0u);
+            const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+            umma_ss(tmem + Cfg::kColDP, dv_k + off, ddo_k0 + stage_off + off, idesc_kk,
+                    kk > 0 ? 1u : 0u);
           }
           umma_commit(dp_full);
           // dV += P^T dO_i
@@ -349,8 +382,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
-            umma_ts(tmem + Cfg::kColDV, tmem + Cfg::kColS + kk * 8,
-                    sw128_desc(doa + kk * 2048, 16384, 1024), idesc_tn,
+            umma_ts(tmem + Cfg::kColDV, tmem + Cfg::packed_col(Cfg::kColS, kk),
+                    ddo_m0 + stage_off + ((kk * 2048) >> 4), idesc_tn,
                     (t > 0 || kk > 0) ? 1u : 0u);
           // dK += dS^T Q_i ; dQ = dS K_j
           ok = mbar_wait(ds_full, ds_cnt & 1);
@@ -363,13 +396,13 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
-            umma_ts(tmem + Cfg::kColDK, tmem + Cfg::kColDP + kk * 8,
-                    sw128_desc(qa + kk * 2048, 16384, 1024), idesc_tn,
+            umma_ts(tmem + Cfg::kColDK, tmem + Cfg::packed_col(Cfg::kColDP, kk),
+                    dq_m0 + stage_off + ((kk * 2048) >> 4), idesc_tn,
                     (t > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
-            umma_ss(tmem + Cfg::kColDQ, sw128_desc(dsa + kk * 2048, 16384, 1024),
-                    sw128_desc(ka + kk * 2048, 16384, 1024), idesc_dq, kk > 0 ? 1u : 0u);
+            umma_ss(tmem + Cfg::kColDQ, dds_m + ((kk * 2048) >> 4), dk_m + ((kk * 2048) >> 4),
+                    idesc_dq, kk > 0 ? 1u : 0u);
           umma_commit(dq_full);
           ++dq_cnt;
           umma_commit(qdo_empty(s));
@@ -387,14 +420,19 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     __syncwarp();
   } else if (warp < 4) {
     setmaxnreg_dec<Cfg::kRegsLow>();  // idle warps of the first warpgroup
-  } else if (warp < 8) {
-    // ------------------------------------------------------------ dS group
-    setmaxnreg_inc<Cfg::kRegsHigh>();
+  } else if (warp < 12) {
+    // ------------------------------------------------------------ dS groups
+    // Warpgroup h (warps 4-7: h = 0, warps 8-11: h = 1) handles queries
+    // 64h..64h+63 of every key row; one key row per thread (TMEM lane).
+    if constexpr (Cfg::kRegsDs > Cfg::kRegsLaunch) setmaxnreg_inc<Cfg::kRegsDs>();
+    const int h = (warp >= 8) ? 1 : 0;
     const int quarter = warp & 3;
     const int kr = quarter * 32 + lane;  // key row within the tile
     const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
-    uint8_t* ds_smem = smem + Cfg::kOffDS;
-    uint32_t s_cnt = 0, dp_cnt = 0, dsm_cnt = 0, dkv_cnt = 0;
+    const uint32_t tS = t_lane + Cfg::kColS + h * 64;    // this half's S^T / P^T columns
+    const uint32_t tDP = t_lane + Cfg::kColDP + h * 64;  // this half's dP^T / dS^T columns
+    uint8_t* ds_rowp = smem + Cfg::kOffDS + h * 16384 + kr * 128;
+    uint32_t s_cnt = 0, dp_cnt = 0, dsm_cnt = 0, dkv_cnt = 0, qdo_cnt = 0;
     bool ok = true;
     for (int round = 0; ok; ++round) {
       const int u = unit_for_round(round, blockIdx.x, G);
@@ -402,47 +440,43 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       const BwdUnit w = bwd_decode(p, u);
       const int c_key = w.j * kTile + kr;  // key index within the head
       const size_t krow = (size_t)w.bh * p.N + c_key;
-      uint4* dk_row = reinterpret_cast<uint4*>(p.dk + krow * D);
-      uint4* dv_row = reinterpret_cast<uint4*>(p.dv + krow * D);
+      // warpgroup 0 writes the dK row, warpgroup 1 the dV row
+      uint4* out_row = reinterpret_cast<uint4*>((h ? p.dv : p.dk) + krow * D);
       if (!w.any) {
 #pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
-          dk_row[c] = make_uint4(0, 0, 0, 0);
-          dv_row[c] = make_uint4(0, 0, 0, 0);
-        }
+        for (int c = 0; c < D / 8; ++c) out_row[c] = make_uint4(0, 0, 0, 0);
         continue;
       }
       const bool key_valid = c_key < w.L;
       for (int i = bwd_next(p, w, w.i_begin); i < p.n_t; i = bwd_next(p, w, i + 1)) {
-        const float4* lse2_t = reinterpret_cast<const float4*>(p.lse2 + (size_t)w.bh * p.N + i * kTile);
-        const float4* dl_t = reinterpret_cast<const float4*>(p.delta + (size_t)w.bh * p.N + i * kTile);
+        const int s = qdo_cnt % S;
+        ++qdo_cnt;
+        const float4* lz4 = lse2_smem(s) + h * 16;
+        const float4* dz4 = delta_smem(s) + h * 16;
         const bool diag = p.causal && (i == w.j);
         ok = __all_sync(0xffffffffu, mbar_wait(s_full, s_cnt & 1));
         ++s_cnt;
         if (!ok) break;
         tc_fence_after();
-        // P^T row: p[q] = exp2(S^T[kr][q] * scale*log2e - lse2[q]); masked -> 0.
-        // Written as bf16 over the first 64 columns of S^T (A operand of dV).
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        // P^T: p[q] = exp2(S^T[kr][q] * scale*log2e - lse2[q]); masked -> 0
+        {
           uint32_t r[2][32];
-          tmem_ld32(t_lane + Cfg::kColS + h * 64, r[0]);
-          tmem_ld32(t_lane + Cfg::kColS + h * 64 + 32, r[1]);
+          tmem_ld32(tS, r[0]);
+          tmem_ld32(tS + 32, r[1]);
           tmem_wait_ld();
           reg_fence32(r[0]);
           reg_fence32(r[1]);
 #pragma unroll
-          for (int cc = 0; cc < 2; ++cc) {
-            const int c = 2 * h + cc;
+          for (int c = 0; c < 2; ++c) {
             uint32_t pk[16];
 #pragma unroll
             for (int e4 = 0; e4 < 8; ++e4) {
-              const float4 lz = __ldg(lse2_t + c * 8 + e4);
-              const int q0 = c * 32 + 4 * e4;
-              float p0 = ex2_approx(fmaf(__uint_as_float(r[cc][4 * e4]), p.scale_log2, -lz.x));
-              float p1 = ex2_approx(fmaf(__uint_as_float(r[cc][4 * e4 + 1]), p.scale_log2, -lz.y));
-              float p2 = ex2_approx(fmaf(__uint_as_float(r[cc][4 * e4 + 2]), p.scale_log2, -lz.z));
-              float p3 = ex2_approx(fmaf(__uint_as_float(r[cc][4 * e4 + 3]), p.scale_log2, -lz.w));
+              const float4 lz = lz4[c * 8 + e4];
+              const int q0 = h * 64 + c * 32 + 4 * e4;  // query within the tile
+              float p0 = ex2_approx(fmaf(__uint_as_float(r[c][4 * e4]), p.scale_log2, -lz.x));
+              float p1 = ex2_approx(fmaf(__uint_as_float(r[c][4 * e4 + 1]), p.scale_log2, -lz.y));
+              float p2 = ex2_approx(fmaf(__uint_as_float(r[c][4 * e4 + 2]), p.scale_log2, -lz.z));
+              float p3 = ex2_approx(fmaf(__uint_as_float(r[c][4 * e4 + 3]), p.scale_log2, -lz.w));
               if (!key_valid || (diag && kr > q0)) p0 = 0.f;
               if (!key_valid || (diag && kr > q0 + 1)) p1 = 0.f;
               if (!key_valid || (diag && kr > q0 + 2)) p2 = 0.f;
@@ -450,13 +484,13 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
               pk[2 * e4] = pack_bf16x2(p0, p1);
               pk[2 * e4 + 1] = pack_bf16x2(p2, p3);
             }
-            tmem_st16(t_lane + Cfg::kColS + c * 16, pk);
+            tmem_st16(tS + c * 16, pk);
           }
         }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(p_full);
-        // dS^T row: ds[q] = p[q] * (dP^T[kr][q] - D[q]), p read back (bf16) from TMEM
+        // dS^T: ds[q] = p[q] * (dP^T[kr][q] - D[q]), p read back (bf16) from TMEM
         ok = __all_sync(0xffffffffu, mbar_wait(dp_full, dp_cnt & 1));
         ++dp_cnt;
         if (!ok) break;
@@ -464,37 +498,40 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         ++dsm_cnt;
         if (!ok) break;
         tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          uint32_t pp[16];
-          tmem_ld32(t_lane + Cfg::kColDP + c * 32, r);
-          tmem_ld16(t_lane + Cfg::kColS + c * 16, pp);
+        {
+          uint32_t r[2][32];
+          uint32_t pp[32];
+          tmem_ld32(tDP, r[0]);
+          tmem_ld32(tDP + 32, r[1]);
+          tmem_ld32(tS, pp);  // both halves' P: 32 packed columns
           tmem_wait_ld();
-          reg_fence32(r);
-          reg_fence16(pp);
-          uint32_t pk[16];
+          reg_fence32(r[0]);
+          reg_fence32(r[1]);
+          reg_fence32(pp);
 #pragma unroll
-          for (int e4 = 0; e4 < 8; ++e4) {
-            const float4 dz = __ldg(dl_t + c * 8 + e4);
-            const float2 pa =
-                __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pp[2 * e4]));
-            const float2 pb =
-                __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pp[2 * e4 + 1]));
-            pk[2 * e4] = pack_bf16x2(pa.x * (__uint_as_float(r[4 * e4]) - dz.x),
-                                     pa.y * (__uint_as_float(r[4 * e4 + 1]) - dz.y));
-            pk[2 * e4 + 1] = pack_bf16x2(pb.x * (__uint_as_float(r[4 * e4 + 2]) - dz.z),
-                                         pb.y * (__uint_as_float(r[4 * e4 + 3]) - dz.w));
-          }
-          tmem_st16(t_lane + Cfg::kColDP + c * 16, pk);
-          // shared-memory copy for the dQ MMA: [key][query], 64-query chunks 16 KB
-          // apart, 128-byte rows, 16-byte granules swizzled by (key & 7)
-          uint8_t* rowp = ds_smem + (c >> 1) * 16384 + kr * 128;
+          for (int c = 0; c < 2; ++c) {
+            uint32_t pk[16];
 #pragma unroll
-          for (int g4 = 0; g4 < 4; ++g4) {
-            const int g = (c & 1) * 4 + g4;
-            *reinterpret_cast<uint4*>(rowp + ((g ^ (kr & 7)) << 4)) =
-                make_uint4(pk[4 * g4], pk[4 * g4 + 1], pk[4 * g4 + 2], pk[4 * g4 + 3]);
+            for (int e4 = 0; e4 < 8; ++e4) {
+              const float4 dz = dz4[c * 8 + e4];
+              const float2 pa =
+                  __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pp[c * 16 + 2 * e4]));
+              const float2 pb = __bfloat1622float2(
+                  *reinterpret_cast<const __nv_bfloat162*>(&pp[c * 16 + 2 * e4 + 1]));
+              pk[2 * e4] = pack_bf16x2(pa.x * (__uint_as_float(r[c][4 * e4]) - dz.x),
+                                       pa.y * (__uint_as_float(r[c][4 * e4 + 1]) - dz.y));
+              pk[2 * e4 + 1] = pack_bf16x2(pb.x * (__uint_as_float(r[c][4 * e4 + 2]) - dz.z),
+                                           pb.y * (__uint_as_float(r[c][4 * e4 + 3]) - dz.w));
+            }
+            tmem_st16(tDP + c * 16, pk);
+            // shared-memory copy for the dQ MMA: [key][query], this half's 64-query
+            // chunk, 128-byte rows, 16-byte granules swizzled by (key & 7)
+#pragma unroll
+            for (int g4 = 0; g4 < 4; ++g4) {
+              const int g = c * 4 + g4;
+              *reinterpret_cast<uint4*>(ds_rowp + ((g ^ (kr & 7)) << 4)) =
+                  make_uint4(pk[4 * g4], pk[4 * g4 + 1], pk[4 * g4 + 2], pk[4 * g4 + 3]);
+            }
           }
         }
         fence_proxy_async_smem();
@@ -504,44 +541,39 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         if (*abort_flag) { ok = false; break; }
       }
       if (!ok) break;
-      // ---------------------------------------------- dK, dV epilogue
+      // ---------------------------------------------- dK (h = 0) / dV (h = 1) epilogue
       ok = __all_sync(0xffffffffu, mbar_wait(dkv_full, dkv_cnt & 1));
       ++dkv_cnt;
       if (!ok) break;
       tc_fence_after();
+      const float mul = h ? 1.f : p.scale;
+      const uint32_t tAcc = t_lane + (h ? Cfg::kColDV : Cfg::kColDK);
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t r[32];
-        tmem_ld32(t_lane + Cfg::kColDK + c * 32, r);
+        tmem_ld32(tAcc + c * 32, r);
         tmem_wait_ld();
         reg_fence32(r);
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e)
-          pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * p.scale,
-                              __uint_as_float(r[2 * e + 1]) * p.scale);
+          pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * mul, __uint_as_float(r[2 * e + 1]) * mul);
 #pragma unroll
         for (int v4 = 0; v4 < 4; ++v4)
-          dk_row[c * 4 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
-        tmem_ld32(t_lane + Cfg::kColDV + c * 32, r);
-        tmem_wait_ld();
-        reg_fence32(r);
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-          pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
-#pragma unroll
-        for (int v4 = 0; v4 < 4; ++v4)
-          dv_row[c * 4 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+          out_row[c * 4 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
       }
       tc_fence_before();
     }
     if (!ok) *abort_flag = 1;
   } else {
     // ------------------------------------------------------------ dQ group
-    setmaxnreg_inc<Cfg::kRegsHigh>();
     // Drains dQ partials: TMEM -> registers -> shared memory (the dS tile,
     // free once the dQ MMA has read it) -> TMA reduce-add into the float32
     // accumulator, in 32 x 32 boxes (128-byte swizzled rows).
+    if constexpr (Cfg::kRegsDq > Cfg::kRegsLaunch)
+      setmaxnreg_inc<Cfg::kRegsDq>();
+    else if constexpr (Cfg::kRegsDq < Cfg::kRegsLaunch)
+      setmaxnreg_dec<Cfg::kRegsDq>();
     const int quarter = warp & 3;  // rows quarter*32 .. +31 of the query tile
     const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
     uint8_t* stage = smem + Cfg::kOffDS + quarter * (Cfg::kDqBoxesPerRound * 4096);

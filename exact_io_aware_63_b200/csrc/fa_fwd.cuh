@@ -10,18 +10,21 @@
 // score tile lives in on-chip memory only.
 //
 // B200 mapping (one persistent CTA per SM, 12 warps):
-//   warp 0      TMA producer: Q tiles of the unit, then the K/V tiles it
-//               visits, through a kStages-deep mbarrier ring.
+//   warp 0      TMA producer: the unit's Q tile (double-buffered across
+//               units), then the K/V tiles it visits, through a kStages-deep
+//               mbarrier ring
 //   warp 1      MMA issuer (one thread): S = Q K^T and O += P V as tcgen05
-//               MMAs accumulating in tensor memory.  Also owns the TMEM
-//               allocation.
-//   warps 4-7   softmax for query tile A (TMEM lanes 0-127, one row each)
-//   warps 8-11  softmax for query tile B
-// A work unit is (b, h, pair of 128-row query tiles A = 2p, B = 2p+1).  The
-// two tiles share every K/V tile load and alternate on the tensor core, so
-// one tile's softmax runs while the other tile's MMAs execute.
+//               MMAs accumulating in tensor memory; owns the TMEM allocation
+//   warps 4-7   softmax warpgroup 0 (TMEM lanes 0-127, one query row each)
+//   warps 8-11  softmax warpgroup 1
+// A work unit is (b, h, one 128-row query tile).  The unit's visited key
+// tiles are dealt alternately to the two softmax warpgroups: warpgroup x
+// owns S_x, O_x in TMEM and its own running (m, l) for every row, so one
+// warpgroup's softmax runs while the tensor core works for the other.  At
+// the end of the unit the two partial results are merged (the same
+// rescaling rule as the online softmax, applied once more).
 //
-// TMEM columns: S_A [0,128), S_B [128,256), O_A [256,256+D), O_B after it.
+// TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 after it.
 // P (bf16) is written over the first 64 columns of its S tile and read from
 // there by the P V MMA.  tcgen05 MMAs issued by one thread execute in issue
 // order, which makes this aliasing safe: the next S MMA into the same
@@ -34,6 +37,8 @@
 // float32.  Any reference max gives the same O / l and LSE in exact
 // arithmetic, because O and l are always scaled by the same factor.
 #pragma once
+
+#include <type_traits>
 
 #include "sm100.cuh"
 
@@ -51,8 +56,8 @@ struct FwdParams {
   const int32_t* kv_len;
   uint8_t* visited;
   int B, H, N, n_t;
-  int num_pairs;
   int num_units;
+  int heads_per_group;  // unit order: see fwd_decode
   int causal;
   float scale_log2;  // scale * log2(e)
 };
@@ -66,79 +71,76 @@ struct FwdCfg {
   static constexpr uint32_t kRegsLaunch = 168, kRegsLow = 104, kRegsHigh = 200;
   static constexpr int kTileBytes = kTile * D * 2;  // one 128 x D bf16 tile
   static constexpr int kBoxes = D / 64;             // 64-column TMA boxes per tile
-  static constexpr int kStages = (D == 64) ? 4 : 2;
-  static constexpr int kOffQ = 0;  // Q_A, Q_B
+  static constexpr int kStages = (D == 64) ? 5 : 2;
+  static constexpr int kOffQ = 0;  // two Q buffers (consecutive units)
   static constexpr int kOffK = kOffQ + 2 * kTileBytes;
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
-  static constexpr int kOffBar = kOffV + kStages * kTileBytes;
+  static constexpr int kOffML = kOffV + kStages * kTileBytes;  // [2 warpgroups][128 rows] (m, l)
+  static constexpr int kOffBar = kOffML + 2 * kTile * 8;
   // barriers: q_full[2], q_empty[2], k_full[S], k_empty[S], v_full[S], v_empty[S],
-  //           s_full[2], p_full[2], o_full[2], drain
-  static constexpr int kNumBars = 4 + 4 * kStages + 6 + 1;
+  //           s_full[2], p_full[2], o_full[2], drain, ml_ready, merged
+  static constexpr int kNumBars = 4 + 4 * kStages + 6 + 3;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
+  static constexpr int kSmemBytes = kOffMisc + 16;
+  static_assert(kSmemBytes <= 232448, "shared memory over the per-block limit");
   static constexpr uint32_t kTmemCols = 512;
+  // pairs (of every 8) whose exponentials ex2_poly2 computes on interior tiles
+  static constexpr int kPolyPer8 = (D == 64) ? 3 : 1;
   __device__ static constexpr uint32_t col_s(int x) { return x ? 128u : 0u; }
   __device__ static constexpr uint32_t col_o(int x) { return x ? 256u + D : 256u; }
 };
 
-// Work-unit order: longest units first (for causal masks the last query
-// tiles see the most keys), then snake order over CTAs so that the sum of
-// lengths per CTA evens out.
+// Work-unit order: heads are taken in groups whose K and V fit in a share of
+// L2 (the units running at the same time then re-read K and V from L2, not
+// HBM); inside a group the longest units come first (for causal masks the
+// last query tiles see the most keys), and units go to CTAs in snake order so
+// that the sum of lengths per CTA evens out.
 __device__ __forceinline__ int unit_for_round(int round, int cta, int G) {
   return round * G + ((round & 1) ? (G - 1 - cta) : cta);
 }
 
 struct FwdUnit {
-  int bh, b, iA, iB, has_b, L, j_end;
+  int bh, b, i, L, j_end;
 };
+
+// Unit u -> (head group g, rank within the group, head): ranks are
+// interleaved over the group's heads, rank 0 (longest) first.
+__device__ __forceinline__ void group_order(int u, int n_t, int BH, int G, int& bh, int& rank) {
+  const int per_group = G * n_t;
+  const int g = u / per_group;
+  const int r = u - g * per_group;
+  const int h0 = g * G;
+  const int gh = min(G, BH - h0);
+  rank = r / gh;
+  bh = h0 + (r - rank * gh);
+}
 
 __device__ __forceinline__ FwdUnit fwd_decode(const FwdParams& p, int u) {
   FwdUnit w;
-  const int BH = p.B * p.H;
-  const int rank = u / BH;  // 0 = longest
-  w.bh = u - rank * BH;
+  int rank;  // 0 = longest
+  group_order(u, p.n_t, p.B * p.H, p.heads_per_group, w.bh, rank);
   w.b = w.bh / p.H;
-  const int pair = p.causal ? (p.num_pairs - 1 - rank) : rank;
-  w.iA = 2 * pair;
-  w.iB = 2 * pair + 1;
-  w.has_b = w.iB < p.n_t;
+  w.i = p.causal ? (p.n_t - 1 - rank) : rank;
   int L = p.N;
   if (p.kv_len) {
     L = __ldg(p.kv_len + w.b);
     L = L < 0 ? 0 : (L > p.N ? p.N : L);
   }
   w.L = L;
-  int j_end = (L + kTile - 1) / kTile;
-  if (p.causal) {
-    const int last = w.has_b ? w.iB : w.iA;
-    j_end = min(j_end, last + 1);
-  }
+  int j_end = (L + kTile - 1) / kTile;   // key tiles holding a key c < L
+  if (p.causal) j_end = min(j_end, w.i + 1);
   w.j_end = j_end;
   return w;
 }
 
-// Is key tile j visited by query tile i?  (Some (r, c) in the tile pair is
-// allowed.)  Causal: j <= i.  Key padding: j*128 < L.  Block mask: nonzero.
-__device__ __forceinline__ bool fwd_tile_on(const FwdParams& p, const FwdUnit& w, int i, int j) {
-  if (p.causal && j > i) return false;
-  if (j * kTile >= w.L) return false;
-  if (p.block_mask && __ldg(p.block_mask + (size_t)i * p.n_t + j) == 0) return false;
-  return true;
-}
-
-__device__ __forceinline__ int fwd_flags(const FwdParams& p, const FwdUnit& w, int j) {
-  int f = fwd_tile_on(p, w, w.iA, j) ? 1 : 0;
-  if (w.has_b && fwd_tile_on(p, w, w.iB, j)) f |= 2;
-  return f;
-}
-
-// First visited key tile >= j (or j_end).
-__device__ __forceinline__ int fwd_next(const FwdParams& p, const FwdUnit& w, int j, int& flags) {
-  for (; j < w.j_end; ++j) {
-    flags = fwd_flags(p, w, j);
-    if (flags) return j;
-  }
-  flags = 0;
+// First key tile >= j that query tile w.i visits (or j_end): tiles below
+// j_end hold an allowed key for causal and key-padding masks; the block mask
+// is the only test left.
+__device__ __forceinline__ int fwd_next(const FwdParams& p, const FwdUnit& w, int j) {
+  if (!p.block_mask) return j < w.j_end ? j : w.j_end;
+  const uint8_t* row = p.block_mask + (size_t)w.i * p.n_t;
+  for (; j < w.j_end; ++j)
+    if (__ldg(row + j)) return j;
   return w.j_end;
 }
 
@@ -148,9 +150,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
                   const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   using Cfg = FwdCfg<D>;
   constexpr int S = Cfg::kStages;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if (!smem_aligned_1024(smem)) return;
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + Cfg::kOffBar;
   auto q_full = [&](int x) { return bar0 + 8 * x; };
@@ -163,8 +164,13 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
   auto p_full = [&](int x) { return bar0 + 8 * (6 + 4 * S + x); };
   auto o_full = [&](int x) { return bar0 + 8 * (8 + 4 * S + x); };
   const uint32_t drain_bar = bar0 + 8 * (10 + 4 * S);
+  // the two softmax warpgroups meet twice per unit in the merge: (m, l)
+  // published, and both partial outputs read (bounded waits, 256 arrivals)
+  const uint32_t ml_ready = bar0 + 8 * (11 + 4 * S);
+  const uint32_t merged = bar0 + 8 * (12 + 4 * S);
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kOffMisc + 4);
+  float2* ml_smem = reinterpret_cast<float2*>(smem + Cfg::kOffML);  // [2][128] (m, l)
 
   const int warp = warp_id();
   const int lane = lane_id();
@@ -184,6 +190,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
       mbar_init(v_empty(s), 1);
     }
     mbar_init(drain_bar, 1);
+    mbar_init(ml_ready, 256);
+    mbar_init(merged, 256);
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tmap(&tm_q);
@@ -206,26 +214,21 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
     // ------------------------------------------------------------ producer
     setmaxnreg_dec<Cfg::kRegsLow>();
     if (lane == 0) {
-      uint32_t q_cnt[2] = {0, 0};
-      uint32_t kv_cnt = 0;
+      uint32_t q_cnt = 0, kv_cnt = 0;
       bool ok = true;
       for (int round = 0; ok; ++round) {
         const int u = unit_for_round(round, blockIdx.x, G);
         if (u >= p.num_units) break;
         const FwdUnit w = fwd_decode(p, u);
-        const int nq = w.has_b ? 2 : 1;
-        for (int x = 0; x < nq && ok; ++x) {
-          ok = mbar_wait(q_empty(x), (q_cnt[x] & 1) ^ 1);
-          if (!ok) break;
-          const int row = w.bh * p.N + (x ? w.iB : w.iA) * kTile;
-          mbar_arrive_expect_tx(q_full(x), Cfg::kTileBytes);
-          for (int bx = 0; bx < Cfg::kBoxes; ++bx)
-            tma_load_2d(sbase + Cfg::kOffQ + x * Cfg::kTileBytes + bx * 16384, &tm_q, bx * 64, row,
-                        q_full(x));
-          ++q_cnt[x];
-        }
-        int fl;
-        for (int j = fwd_next(p, w, 0, fl); j < w.j_end && ok; j = fwd_next(p, w, j + 1, fl)) {
+        const int qb = q_cnt & 1;
+        ok = mbar_wait(q_empty(qb), ((q_cnt >> 1) & 1) ^ 1);
+        if (!ok) break;
+        ++q_cnt;
+        mbar_arrive_expect_tx(q_full(qb), Cfg::kTileBytes);
+        for (int bx = 0; bx < Cfg::kBoxes; ++bx)
+          tma_load_2d(sbase + Cfg::kOffQ + qb * Cfg::kTileBytes + bx * 16384, &tm_q, bx * 64,
+                      w.bh * p.N + w.i * kTile, q_full(qb));
+        for (int j = fwd_next(p, w, 0); j < w.j_end && ok; j = fwd_next(p, w, j + 1)) {
           const int s = kv_cnt % S;
           const uint32_t ph = (kv_cnt / S) & 1;
           const int row = w.bh * p.N + j * kTile;
@@ -254,109 +257,75 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
-      uint32_t q_cnt[2] = {0, 0};
-      uint32_t p_cnt[2] = {0, 0};
-      uint32_t kv_cnt = 0;
-      bool ok = true;
-
-      // Descriptors: one base per tile; the start-address field (bits 0..13,
+      // Descriptors: one base per operand; the start-address field (bits 0..13,
       // address >> 4) is advanced by adding (byte offset >> 4).  Tiles lie in
       // the first 256 KB of shared memory, so the field never carries over.
       const uint64_t desc_q0 = sw128_desc(sbase + Cfg::kOffQ, 16, 1024);
       const uint64_t desc_k0 = sw128_desc(sbase + Cfg::kOffK, 16, 1024);
       const uint64_t desc_v0 = sw128_desc(sbase + Cfg::kOffV, 16384, 1024);
-      auto issue_s = [&](int x, int s) {
-        const uint64_t dq = desc_q0 + ((x * Cfg::kTileBytes) >> 4);
-        const uint64_t dk = desc_k0 + ((s * Cfg::kTileBytes) >> 4);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
-          umma_ss(tmem + Cfg::col_s(x), dq + off, dk + off, idesc_s, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(s_full(x));
-      };
-      auto issue_pv = [&](int x, int s, uint32_t acc) {
-        const uint64_t dv = desc_v0 + ((s * Cfg::kTileBytes) >> 4);
-#pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk) {
-          umma_ts(tmem + Cfg::col_o(x), tmem + Cfg::col_s(x) + kk * 8, dv + ((kk * 2048) >> 4),
-                  idesc_pv, (kk > 0 || acc) ? 1u : 0u);
-        }
-      };
-
+      uint32_t q_cnt = 0, kv_cnt = 0;
+      uint32_t p_cnt[2] = {0, 0};
+      bool ok = true;
       for (int round = 0; ok; ++round) {
         const int u = unit_for_round(round, blockIdx.x, G);
         if (u >= p.num_units) break;
         const FwdUnit w = fwd_decode(p, u);
-        const int nq = w.has_b ? 2 : 1;
-        for (int x = 0; x < nq && ok; ++x) {
-          ok = mbar_wait(q_full(x), q_cnt[x] & 1);
-          ++q_cnt[x];
-        }
+        const int qb = q_cnt & 1;
+        ok = mbar_wait(q_full(qb), (q_cnt >> 1) & 1);
+        ++q_cnt;
         if (!ok) break;
-        tc_fence_after();
-        int started[2] = {0, 0};
-        int fl = 0;
-        int j = fwd_next(p, w, 0, fl);
-        if (j < w.j_end) {
-          const int s = kv_cnt % S;
-          ok = mbar_wait(k_full(s), (kv_cnt / S) & 1);
+        const uint64_t dq = desc_q0 + ((qb * Cfg::kTileBytes) >> 4);
+        // S(k) for the k-th visited key tile j, into warpgroup (k & 1)'s S columns
+        auto issue_s = [&](int k, int j) -> bool {
+          const uint32_t c = kv_cnt + k;
+          const int s = c % S;
+          if (!mbar_wait(k_full(s), (c / S) & 1)) return false;
+          tc_fence_after();
+          const uint64_t dk = desc_k0 + ((s * Cfg::kTileBytes) >> 4);
+          const int x = k & 1;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+            umma_ss(tmem + Cfg::col_s(x), dq + off, dk + off, idesc_s, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(s_full(x));
+          umma_commit(k_empty(s));
+          if (p.visited) p.visited[((size_t)w.bh * p.n_t + w.i) * p.n_t + j] = 1;
+          return true;
+        };
+        int jk = fwd_next(p, w, 0);                                   // tile of visit k
+        int jk1 = (jk < w.j_end) ? fwd_next(p, w, jk + 1) : w.j_end;  // visit k + 1
+        if (jk < w.j_end) ok = issue_s(0, jk);
+        if (ok && jk1 < w.j_end) ok = issue_s(1, jk1);
+        int k = 0;
+        while (ok && jk < w.j_end) {
+          const int x = k & 1;
+          const uint32_t c = kv_cnt + k;
+          const int s = c % S;
+          const int jk2 = (jk1 < w.j_end) ? fwd_next(p, w, jk1 + 1) : w.j_end;
+          ok = mbar_wait(p_full(x), p_cnt[x] & 1);
+          ++p_cnt[x];
+          if (!ok) break;
+          ok = mbar_wait(v_full(s), (c / S) & 1);
           if (!ok) break;
           tc_fence_after();
-          for (int x = 0; x < 2; ++x)
-            if (fl & (1 << x)) {
-              issue_s(x, s);
-              if (p.visited)
-                p.visited[((size_t)w.bh * p.n_t + (x ? w.iB : w.iA)) * p.n_t + j] = 1;
-            }
-          umma_commit(k_empty(s));
-        }
-        while (j < w.j_end && ok) {
-          const int s = kv_cnt % S;
-          int fln = 0;
-          const int jn = fwd_next(p, w, j + 1, fln);
-          const uint32_t cn = kv_cnt + 1;
-          const int sn = cn % S;
-          bool v_ready = false, k_next_ready = false;
-          for (int x = 0; x < 2 && ok; ++x) {
-            if (fl & (1 << x)) {
-              ok = mbar_wait(p_full(x), p_cnt[x] & 1);
-              ++p_cnt[x];
-              if (!ok) break;
-              if (!v_ready) {
-                ok = mbar_wait(v_full(s), (kv_cnt / S) & 1);
-                if (!ok) break;
-                v_ready = true;
-              }
-              tc_fence_after();
-              issue_pv(x, s, started[x]);
-              started[x] = 1;
-            }
-            if (x == 1) umma_commit(v_empty(s));
-            if (jn < w.j_end && (fln & (1 << x))) {
-              if (!k_next_ready) {
-                ok = mbar_wait(k_full(sn), (cn / S) & 1);
-                if (!ok) break;
-                tc_fence_after();
-                k_next_ready = true;
-              }
-              issue_s(x, sn);
-              if (p.visited)
-                p.visited[((size_t)w.bh * p.n_t + (x ? w.iB : w.iA)) * p.n_t + jn] = 1;
-            }
-          }
-          if (!ok) break;
-          if (jn < w.j_end) umma_commit(k_empty(sn));
-          kv_cnt = cn;
-          j = jn;
-          fl = fln;
+          const uint64_t dv = desc_v0 + ((s * Cfg::kTileBytes) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            umma_ts(tmem + Cfg::col_o(x), tmem + Cfg::col_s(x) + kk * 8, dv + ((kk * 2048) >> 4),
+                    idesc_pv, (kk > 0 || k >= 2) ? 1u : 0u);
+          umma_commit(v_empty(s));
+          if (jk2 < w.j_end) ok = issue_s(k + 2, jk2);
+          jk = jk1;
+          jk1 = jk2;
+          ++k;
           if (*abort_flag) ok = false;
         }
         if (!ok) break;
-        for (int x = 0; x < nq; ++x) {
-          if (started[x]) umma_commit(o_full(x));
-          umma_commit(q_empty(x));
-        }
+        if (k >= 1) umma_commit(o_full(0));
+        if (k >= 2) umma_commit(o_full(1));
+        umma_commit(q_empty(qb));
+        kv_cnt += k;
       }
       if (!ok) *abort_flag = 1;
       // all issued MMAs complete before TMEM is released
@@ -369,27 +338,27 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
   } else {
     // ------------------------------------------------------------ softmax
     setmaxnreg_inc<Cfg::kRegsHigh>();
+    constexpr int kPolyPer8 = Cfg::kPolyPer8;
     const int x = (warp >= 8) ? 1 : 0;
     const int quarter = warp & 3;
     const int r_local = quarter * 32 + lane;  // row within the query tile = TMEM lane
     const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
     const uint32_t tS = t_lane + Cfg::col_s(x);
     const uint32_t tO = t_lane + Cfg::col_o(x);
-    uint32_t s_cnt = 0, o_cnt = 0;
+    uint32_t s_cnt = 0, unit_cnt = 0;
+    uint32_t o_cnt[2] = {0, 0};
     bool ok = true;
     for (int round = 0; ok; ++round) {
       const int u = unit_for_round(round, blockIdx.x, G);
       if (u >= p.num_units) break;
       const FwdUnit w = fwd_decode(p, u);
-      if (x == 1 && !w.has_b) continue;
-      const int i = x ? w.iB : w.iA;
-      const int row = i * kTile + r_local;  // query index within the head
+      const int row = w.i * kTile + r_local;  // query index within the head
       float m_used = -INFINITY;              // log2 domain, scale folded in
       float l = 0.f;
-      int cnt = 0;
-      int fl = 0;
-      for (int j = fwd_next(p, w, 0, fl); j < w.j_end; j = fwd_next(p, w, j + 1, fl)) {
-        if (!(fl & (1 << x))) continue;
+      int cnt = 0;   // tiles this warpgroup processed
+      int k = 0;     // visit index over both warpgroups
+      for (int j = fwd_next(p, w, 0); j < w.j_end; j = fwd_next(p, w, j + 1), ++k) {
+        if ((k & 1) != x) continue;
         ok = __all_sync(0xffffffffu, mbar_wait(s_full(x), s_cnt & 1));
         ++s_cnt;
         if (!ok) break;
@@ -408,17 +377,25 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
           }
         }
         // element masks on boundary tiles only
-        const bool diag = p.causal && (j == i);
+        const bool diag = p.causal && (j == w.i);
         const int kv_lim = w.L - j * kTile;  // keys c >= kv_lim are padding
-        if (diag || kv_lim < kTile) {
+        const bool boundary = diag || kv_lim < kTile;
+        if (boundary) {
           const int lim = diag ? min(r_local + 1, kv_lim) : kv_lim;
 #pragma unroll
           for (int c = 0; c < kTile; ++c)
             if (c >= lim) sv[c] = -INFINITY;
         }
-        float mx = sv[0];
+        // row max: eight independent chains of 3-input max, then combined
+        float mx8[8];
 #pragma unroll
-        for (int c = 1; c < kTile; ++c) mx = fmaxf(mx, sv[c]);
+        for (int t = 0; t < 8; ++t) mx8[t] = fmaxf(sv[t], sv[t + 8]);
+#pragma unroll
+        for (int c = 16; c < kTile; c += 16)
+#pragma unroll
+          for (int t = 0; t < 8; ++t) mx8[t] = fmax3(mx8[t], sv[c + t], sv[c + 8 + t]);
+        const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                               fmaxf(mx8[6], mx8[7]));
         const float m_new = mx * p.scale_log2;  // -inf if the whole row is masked here
         float alpha = 1.f;
         bool rescale = false;
@@ -430,6 +407,49 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
           l *= alpha;
           rescale = true;
         }
+        const float m_sub = (m_used == -INFINITY) ? 0.f : m_used;
+        // P = 2^(s * scale * log2 e - m), two elements per packed FMA.  On
+        // interior tiles kPolyPer8 of every 8 pairs use ex2_poly2 on the FMA pipe
+        // to offload the MUFU unit; boundary tiles (which hold -inf) use the
+        // hardware exp2 throughout.
+        const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
+        const uint64_t negm2 = f2_pack(-m_sub, -m_sub);
+        uint64_t ls4[4] = {0, 0, 0, 0};  // packed partial row sums (0.0f bit pattern)
+        auto make_p = [&](auto soft_tag) {
+          constexpr bool kSoft = decltype(soft_tag)::value;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const uint64_t xx =
+                  f2_fma(f2_pack(sv[c * 32 + 2 * e], sv[c * 32 + 2 * e + 1]), scale2, negm2);
+              float x0, x1, p0, p1;
+              f2_unpack(xx, x0, x1);
+              if (kSoft && (e & 7) < kPolyPer8) {
+                ex2_poly2(x0, x1, p0, p1);
+              } else {
+                p0 = ex2_approx(x0);
+                p1 = ex2_approx(x1);
+              }
+              ls4[e & 3] = f2_add(ls4[e & 3], f2_pack(p0, p1));
+              pk[e] = pack_bf16x2(p0, p1);
+            }
+            tmem_st16(tS + c * 16, pk);
+          }
+        };
+        if (boundary)
+          make_p(std::false_type{});
+        else
+          make_p(std::true_type{});
+        {
+          const uint64_t s2 = f2_add(f2_add(ls4[0], ls4[1]), f2_add(ls4[2], ls4[3]));
+          float s_lo, s_hi;
+          f2_unpack(s2, s_lo, s_hi);
+          l += s_lo + s_hi;
+        }
+        // O rescale (rare: the row max grew by more than 2^8) after P is out of
+        // registers; it completes before p_full, so before the next P V MMA
         if (__any_sync(0xffffffffu, rescale)) {
           uint32_t r[32];
 #pragma unroll
@@ -442,21 +462,6 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
             tmem_st32(tO + c * 32, r);
           }
         }
-        const float m_sub = (m_used == -INFINITY) ? 0.f : m_used;
-        float lsum = 0.f;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float p0 = ex2_approx(fmaf(sv[c * 32 + 2 * e], p.scale_log2, -m_sub));
-            const float p1 = ex2_approx(fmaf(sv[c * 32 + 2 * e + 1], p.scale_log2, -m_sub));
-            lsum += p0 + p1;
-            pk[e] = pack_bf16x2(p0, p1);
-          }
-          tmem_st16(tS + c * 16, pk);
-        }
-        l += lsum;
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(p_full(x));
@@ -464,37 +469,68 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
         if (*abort_flag) { ok = false; break; }
       }
       if (!ok) break;
-      // ---------------------------------------------------- epilogue
-      const size_t grow = (size_t)w.bh * p.N + row;
-      uint4* orow = reinterpret_cast<uint4*>(p.o + grow * D);
-      if (cnt > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(o_full(x), o_cnt & 1));
-        ++o_cnt;
-        if (!ok) break;
-        tc_fence_after();
-        const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tO + c * 32, r);
-          tmem_wait_ld();
-          reg_fence32(r);
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e)
-            pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv_l,
-                                __uint_as_float(r[2 * e + 1]) * inv_l);
-#pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4)
-            orow[c * 4 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
-        }
-        tc_fence_before();
-        p.lse[grow] = (l > 0.f) ? (m_used + log2f(l)) * kLn2 : -INFINITY;
-      } else {
-#pragma unroll
-        for (int c = 0; c < D / 8; ++c) orow[c] = make_uint4(0, 0, 0, 0);
-        p.lse[grow] = -INFINITY;
+      // ---------------------------------------------------- merge + epilogue
+      // k = visits of the unit: warpgroup 0 processed ceil(k/2), warpgroup 1
+      // floor(k/2).  Both warpgroups read both partial outputs: warpgroup x
+      // finishes columns [x*D/2, (x+1)*D/2) of every row.
+      const int n0 = (k + 1) / 2, n1 = k / 2;
+      if (n0 > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(o_full(0), o_cnt[0] & 1));
+        ++o_cnt[0];
       }
+      if (ok && n1 > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(o_full(1), o_cnt[1] & 1));
+        ++o_cnt[1];
+      }
+      if (!ok) break;
+      tc_fence_after();
+      ml_smem[x * kTile + r_local] = make_float2(m_used, cnt > 0 ? l : 0.f);
+      mbar_arrive(ml_ready);
+      ok = __all_sync(0xffffffffu, mbar_wait(ml_ready, unit_cnt & 1));
+      if (!ok) break;
+      const float2 ml0 = ml_smem[r_local];
+      const float2 ml1 = ml_smem[kTile + r_local];
+      const float m = fmaxf(ml0.x, ml1.x);
+      const float a0 = (ml0.y > 0.f) ? ex2_approx(ml0.x - m) : 0.f;
+      const float a1 = (ml1.y > 0.f) ? ex2_approx(ml1.x - m) : 0.f;
+      const float lt = ml0.y * a0 + ml1.y * a1;
+      const float inv_l = (lt > 0.f) ? 1.f / lt : 0.f;
+      const float f0 = a0 * inv_l, f1 = a1 * inv_l;
+      const size_t grow = (size_t)w.bh * p.N + row;
+      uint4* orow = reinterpret_cast<uint4*>(p.o + grow * D + x * (D / 2));
+      // A warpgroup that processed no tile left its O unwritten: its factor is 0
+      // and its values are dropped by a select (never multiplied, in case the
+      // unwritten columns hold a NaN pattern).
+      const bool use0 = n0 > 0, use1 = n1 > 0;
+#pragma unroll 1
+      for (int c = 0; c < D / 64; ++c) {
+        const uint32_t col = x * (D / 2) + c * 32;
+        uint32_t r0[32], r1[32];
+        tmem_ld32(t_lane + Cfg::col_o(0) + col, r0);
+        tmem_ld32(t_lane + Cfg::col_o(1) + col, r1);
+        tmem_wait_ld();
+        reg_fence32(r0);
+        reg_fence32(r1);
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float a = use0 ? __uint_as_float(r0[2 * e]) * f0 : 0.f;
+          const float b = use0 ? __uint_as_float(r0[2 * e + 1]) * f0 : 0.f;
+          const float c2 = use1 ? __uint_as_float(r1[2 * e]) * f1 : 0.f;
+          const float d2 = use1 ? __uint_as_float(r1[2 * e + 1]) * f1 : 0.f;
+          pk[e] = pack_bf16x2(a + c2, b + d2);
+        }
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4)
+          orow[c * 4 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+      }
+      if (x == 0) p.lse[grow] = (lt > 0.f) ? (m + log2f(lt)) * kLn2 : -INFINITY;
+      tc_fence_before();
+      // neither warpgroup starts the next unit (whose first P V overwrites an O)
+      // before both have read both partial outputs
+      mbar_arrive(merged);
+      ok = __all_sync(0xffffffffu, mbar_wait(merged, unit_cnt & 1));
+      ++unit_cnt;
     }
     if (!ok) *abort_flag = 1;
   }

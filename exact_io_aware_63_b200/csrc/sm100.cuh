@@ -17,7 +17,10 @@ namespace fa {
 // ---------------------------------------------------------------------------
 // device status word (read and cleared by fa_get_device_status)
 // ---------------------------------------------------------------------------
-enum : unsigned { FA_DEV_TIMEOUT = 1u };
+enum : unsigned {
+  FA_DEV_TIMEOUT = 1u,     // a bounded wait gave up
+  FA_DEV_SMEM_ALIGN = 2u,  // dynamic shared memory not 1024-byte aligned (kernel did nothing)
+};
 // One word per translation unit that includes this header (internal linkage).
 static __device__ unsigned int g_device_status = 0;
 
@@ -31,6 +34,15 @@ __device__ __forceinline__ unsigned long long globaltimer_ns() {
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// Dynamic shared memory must start on a 1024-byte boundary (the 128-byte
+// swizzle repeats every 1024 bytes).  Returns false, and records the fact,
+// when it does not; every thread sees the same answer.
+__device__ __forceinline__ bool smem_aligned_1024(const void* p) {
+  if ((__cvta_generic_to_shared(p) & 1023u) == 0) return true;
+  if (threadIdx.x == 0) atomicOr(&g_device_status, FA_DEV_SMEM_ALIGN);
+  return false;
 }
 
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31u; }
@@ -320,6 +332,75 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// 2^x evaluated on the FMA pipe instead of the MUFU unit, for -126 <= x <= 126
+// (smaller x is clamped to -126; the result is then ~1e-38, i.e. zero for our
+// purposes).  x = n + f with n = round(x) (obtained by adding 1.5 * 2^23, which
+// leaves round(x) in the low mantissa bits) and f in [-1/2, 1/2]; 2^f is a
+// degree-3 polynomial whose coefficients are the minimax (Remez exchange) fit
+// of 2^f on [-1/2, 1/2] for relative error (max relative error 7.5e-5, i.e.
+// 13.7 bits: more than the 8 bits a bfloat16 probability keeps); 2^n is added
+// to the exponent field.
+__device__ __forceinline__ float ex2_poly(float x) {
+  constexpr float kC0 = 0.99992805719375610f;
+  constexpr float kC1 = 0.69326096773147583f;
+  constexpr float kC2 = 0.24261112511157990f;
+  constexpr float kC3 = 0.05517166852951050f;
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  x = fmaxf(x, -126.0f);
+  const float t = x + kRound;
+  const float f = x - (t - kRound);
+  const float p = fmaf(fmaf(fmaf(kC3, f, kC2), f, kC1), f, kC0);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// ---------------------------------------------------------------------------
+// packed float32 pairs (one instruction for two values on sm_100)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// ex2_poly on a pair (same polynomial and range as ex2_poly).
+__device__ __forceinline__ void ex2_poly2(float x0, float x1, float& y0, float& y1) {
+  constexpr float kC0 = 0.99992805719375610f;
+  constexpr float kC1 = 0.69326096773147583f;
+  constexpr float kC2 = 0.24261112511157990f;
+  constexpr float kC3 = 0.05517166852951050f;
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  const uint64_t x = f2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
+  const uint64_t t = f2_add(x, f2_pack(kRound, kRound));
+  const uint64_t n = f2_add(t, f2_pack(-kRound, -kRound));
+  const uint64_t f = f2_fma(n, f2_pack(-1.0f, -1.0f), x);
+  uint64_t q = f2_fma(f, f2_pack(kC3, kC3), f2_pack(kC2, kC2));
+  q = f2_fma(q, f, f2_pack(kC1, kC1));
+  q = f2_fma(q, f, f2_pack(kC0, kC0));
+  float q0, q1, t0, t1;
+  f2_unpack(q, q0, q1);
+  f2_unpack(t, t0, t1);
+  y0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -337,9 +418,5 @@ __device__ __forceinline__ void setmaxnreg_inc() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
-// Named barrier over `nthreads` threads (a multiple of 32) with id `id` (1..15).
-__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
 
 }  // namespace fa
