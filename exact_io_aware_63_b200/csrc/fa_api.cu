@@ -130,20 +130,33 @@ WsLayout ws_layout(int B, int H, int N, int d) {
   return w;
 }
 
+template <int D, bool kPair>
+int launch_fwd_mode(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                    fa::FwdParams& p, cudaStream_t stream, int num_sms) {
+  using Cfg = fa::FwdCfg<D, kPair>;
+  static bool smem_set = false;
+  if (!smem_set) {
+    if (!set_smem(fa::fa_fwd_kernel<D, kPair>, Cfg::kSmemBytes)) return FA_ERR_CUDA;
+    smem_set = true;
+  }
+  const int per_head = kPair ? (p.n_t + 1) / 2 : p.n_t;
+  p.num_units = p.B * p.H * per_head;
+  const int grid = p.num_units < num_sms ? p.num_units : num_sms;
+  fa::fa_fwd_kernel<D, kPair><<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// Pair mode (two query tiles share each K/V tile) unless a block mask is
+// given: random tile masks give two query tiles few key tiles in common, and
+// split mode keeps both softmax warpgroups busy on one query tile instead.
 template <int D>
 int launch_fwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o, float* lse, int B,
                int H, int N, float scale, int causal, const uint8_t* block_mask,
                const int32_t* kv_len, uint8_t* visited, cudaStream_t stream, int num_sms) {
-  using Cfg = fa::FwdCfg<D>;
   const long long rows = static_cast<long long>(B) * H * N;
   CUtensorMap tq, tk, tv;
   if (!make_tmap(&tq, q, rows, D) || !make_tmap(&tk, k, rows, D) || !make_tmap(&tv, v, rows, D))
     return FA_ERR_CUDA;
-  static bool smem_set = false;
-  if (!smem_set) {
-    if (!set_smem(fa::fa_fwd_kernel<D>, Cfg::kSmemBytes)) return FA_ERR_CUDA;
-    smem_set = true;
-  }
   fa::FwdParams p;
   p.o = o;
   p.lse = lse;
@@ -154,13 +167,11 @@ int launch_fwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o,
   p.H = H;
   p.N = N;
   p.n_t = N / fa::kTile;
-  p.num_units = B * H * p.n_t;
   p.heads_per_group = heads_per_group(B * H, 4.0 * N * D);  // K and V
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * fa::kLog2e;
-  const int grid = p.num_units < num_sms ? p.num_units : num_sms;
-  fa::fa_fwd_kernel<D><<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(tq, tk, tv, p);
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  if (block_mask) return launch_fwd_mode<D, false>(tq, tk, tv, p, stream, num_sms);
+  return launch_fwd_mode<D, true>(tq, tk, tv, p, stream, num_sms);
 }
 
 template <int D>

@@ -14,9 +14,9 @@
 //   fa_bwd_dq_kernel     dQ = bf16(scale * accumulator)
 //
 // fa_bwd_kernel roles (16 warps):
-//   warp 0      TMA producer: K_j, V_j once per unit; Q_i, dO_i and the
-//               tile's LSE*log2(e) and D rows per visited query tile through a
-//               kStages-deep ring
+//   warp 0      TMA producer: K_j, V_j once per unit; per visited query tile
+//               Q_i with the tile's LSE*log2(e) and D rows (one ring) and
+//               dO_i (a second ring)
 //   warp 1      MMA issuer (one thread), TMEM owner
 //   warps 4-11  two "dS" warpgroups, one key row per thread (TMEM lane), each
 //               on half of the 128 query columns: P^T, dS^T, and the dK (first
@@ -39,9 +39,9 @@
 namespace fa {
 
 // ---------------------------------------------------------------------------
-// preprocess: D_r = sum_x dO_rx O_rx (f32), lse2_r = LSE_r * log2(e)
-// (+inf for rows with no allowed key, so that exp2(s - lse2) = 0), and zero
-// the dQ accumulator.
+// preprocess: D_r = sum_x dO_rx O_rx (f32) and LSE_r * log2(e) (+inf for rows
+// with no allowed key, so that exp2(s - LSE2) = 0), both stored NEGATED (the
+// main kernel adds them), and zero the dQ accumulator.
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const uint16_t* __restrict__ o,
@@ -78,9 +78,9 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const uint16_t* __restr
     for (int off = kLanesPerRow / 2; off > 0; off >>= 1)
       acc += __shfl_xor_sync(0xffffffffu, acc, off);
     if (r < rows && part == 0) {
-      delta[r] = acc;
+      delta[r] = -acc;
       const float l = lse[r];
-      lse2[r] = (l == -INFINITY) ? INFINITY : l * kLog2e;
+      lse2[r] = (l == -INFINITY) ? -INFINITY : -l * kLog2e;
     }
   }
   const long long n4 = rows * (D / 4);
@@ -108,8 +108,8 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const float4* __restrict
 // ---------------------------------------------------------------------------
 struct BwdParams {
   float* dq_acc;
-  const float* delta;
-  const float* lse2;
+  const float* delta;  // -D per row
+  const float* lse2;   // -LSE * log2(e) per row (-inf: row with no key)
   uint16_t* dk;
   uint16_t* dv;
   const uint8_t* block_mask;
@@ -127,30 +127,36 @@ template <int D>
 struct BwdCfg {
   static constexpr int kThreads = 512;
   // registers per thread: 128 at launch (512 x 128 = 65536); the producer /
-  // MMA warpgroup drops to 88 and the rest is shared by the two dS
-  // warpgroups and the dQ warpgroup (which holds a whole float32 dQ row):
-  // D = 64:  128 x 88 + 256 x 136 + 128 x 120 = 61440
+  // MMA warpgroup drops to 96 (D = 64) or 88 (D = 128) and the rest is shared
+  // by the two dS warpgroups and the dQ warpgroup (which holds a whole
+  // float32 dQ row):
+  // D = 64:  128 x 96 + 256 x 136 + 128 x 120 = 62464
   // D = 128: 128 x 88 + 256 x 128 + 128 x 168 = 65536
-  static constexpr uint32_t kRegsLaunch = 128, kRegsLow = 88;
+  static constexpr uint32_t kRegsLaunch = 128, kRegsLow = (D == 64) ? 96 : 88;
   static constexpr uint32_t kRegsDs = (D == 64) ? 136 : 128;
   static constexpr uint32_t kRegsDq = (D == 64) ? 120 : 168;
   static constexpr int kTileBytes = kTile * D * 2;
   static constexpr int kBoxes = D / 64;
-  static constexpr int kStages = (D == 64) ? 4 : 2;
+  // Q_i (with the tile's -LSE2 and -D rows) and dO_i come through separate
+  // rings: dO_i is released after the dV MMA, Q_i after the dK MMA.
+  static constexpr int kQStages = (D == 64) ? 3 : 2;
+  static constexpr int kDoStages = (D == 64) ? 3 : 1;
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kOffK + kTileBytes;
   static constexpr int kOffQ = kOffV + kTileBytes;
-  static constexpr int kOffDO = kOffQ + kStages * kTileBytes;
-  // 128 x 128 bf16 dS tile for the dQ MMA; once that MMA has read it, the dQ
-  // group reuses it to stage float32 dQ partials for the TMA reduce-add.
-  static constexpr int kOffDS = kOffDO + kStages * kTileBytes;
-  // per stage: LSE*log2(e) and D of the stage's 128 query rows
-  static constexpr int kOffRow = kOffDS + kTile * kTile * 2;
+  static constexpr int kOffDO = kOffQ + kQStages * kTileBytes;
+  // 128 x 128 bf16 dS tile: A operand of the dQ MMA
+  static constexpr int kOffDS = kOffDO + kDoStages * kTileBytes;
+  // float32 dQ partials staged for the TMA reduce-add: 8 KB per dQ warp
+  static constexpr int kOffDQ = kOffDS + kTile * kTile * 2;
+  static constexpr int kDqStageBytes = 4 * 8192;
+  // per Q stage: -LSE*log2(e) and -D of the stage's 128 query rows
+  static constexpr int kOffRow = kOffDQ + kDqStageBytes;
   static constexpr int kRowBytes = kTile * 4;
-  static constexpr int kOffBar = kOffRow + 2 * kStages * kRowBytes;
-  // kv_full, kv_empty, qdo_full[S], qdo_empty[S], s_full, dp_full, p_full, ds_full,
-  // ds_smem_empty, dq_full, dq_empty, dkv_full, drain
-  static constexpr int kNumBars = 2 + 2 * kStages + 9;
+  static constexpr int kOffBar = kOffRow + 2 * kQStages * kRowBytes;
+  // kv_full, kv_empty, q_full[QS], q_empty[QS], do_full[DS], do_empty[DS], s_full,
+  // dp_full, p_full, ds_full, ds_smem_empty, dq_full, dq_empty, dkv_full, drain
+  static constexpr int kNumBars = 2 + 2 * kQStages + 2 * kDoStages + 9;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16;
   static_assert(kSmemBytes <= 232448, "shared memory over the per-block limit");
@@ -166,9 +172,11 @@ struct BwdCfg {
   // dQ = dS K_j: its own columns when they fit (D = 64), else over S^T
   static constexpr uint32_t kColDQ = (D == 64) ? 384 : 0;
   static constexpr bool kDqAliasesS = (kColDQ == kColS);
-  // dQ staging: each dQ warp owns 8 KB of the dS tile = two 32 x 32 float32 boxes
+  // dQ staging: each dQ warp owns 8 KB = two 32 x 32 float32 boxes
   static constexpr int kDqBoxesPerRound = 2;
   static constexpr int kDqRounds = D / 64;
+  // pairs (of every 4) whose exponentials ex2_poly2 computes, off the diagonal
+  static constexpr int kPolyPer4 = 1;
   // TMEM column of the bf16 operand for K-step kk (16 queries) of the dV / dK MMAs
   __device__ static constexpr uint32_t packed_col(uint32_t base, int kk) {
     return base + (kk >> 2) * 64 + (kk & 3) * 8;
@@ -218,15 +226,17 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                   const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
   using Cfg = BwdCfg<D>;
-  constexpr int S = Cfg::kStages;
+  constexpr int QS = Cfg::kQStages, DOS = Cfg::kDoStages;
   extern __shared__ __align__(1024) uint8_t smem[];
   if (!smem_aligned_1024(smem)) return;
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + Cfg::kOffBar;
   const uint32_t kv_full = bar0, kv_empty = bar0 + 8;
-  auto qdo_full = [&](int s) { return bar0 + 8 * (2 + s); };
-  auto qdo_empty = [&](int s) { return bar0 + 8 * (2 + S + s); };
-  const uint32_t s_full = bar0 + 8 * (2 + 2 * S);
+  auto q_full = [&](int s) { return bar0 + 8 * (2 + s); };
+  auto q_empty = [&](int s) { return bar0 + 8 * (2 + QS + s); };
+  auto do_full = [&](int s) { return bar0 + 8 * (2 + 2 * QS + s); };
+  auto do_empty = [&](int s) { return bar0 + 8 * (2 + 2 * QS + DOS + s); };
+  const uint32_t s_full = bar0 + 8 * (2 + 2 * QS + 2 * DOS);
   const uint32_t dp_full = s_full + 8, p_full = s_full + 16, ds_full = s_full + 24;
   const uint32_t ds_smem_empty = s_full + 32, dq_full = s_full + 40, dq_empty = s_full + 48;
   const uint32_t dkv_full = s_full + 56, drain_bar = s_full + 64;
@@ -236,7 +246,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     return reinterpret_cast<const float4*>(smem + Cfg::kOffRow + s * Cfg::kRowBytes);
   };
   auto delta_smem = [&](int s) {
-    return reinterpret_cast<const float4*>(smem + Cfg::kOffRow + (S + s) * Cfg::kRowBytes);
+    return reinterpret_cast<const float4*>(smem + Cfg::kOffRow + (QS + s) * Cfg::kRowBytes);
   };
 
   const int warp = warp_id();
@@ -245,15 +255,19 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
     mbar_init(kv_empty, 1);
-    for (int s = 0; s < S; ++s) {
-      mbar_init(qdo_full(s), 1);
-      mbar_init(qdo_empty(s), 1);
+    for (int s = 0; s < QS; ++s) {
+      mbar_init(q_full(s), 1);
+      mbar_init(q_empty(s), 1);
+    }
+    for (int s = 0; s < DOS; ++s) {
+      mbar_init(do_full(s), 1);
+      mbar_init(do_empty(s), 1);
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
     mbar_init(p_full, 256);
     mbar_init(ds_full, 256);
-    mbar_init(ds_smem_empty, 4);  // one arrival per dQ warp
+    mbar_init(ds_smem_empty, 1);
     mbar_init(dq_full, 1);
     mbar_init(dq_empty, 128);
     mbar_init(dkv_full, 1);
@@ -283,7 +297,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     // ------------------------------------------------------------ producer
     setmaxnreg_dec<Cfg::kRegsLow>();
     if (lane == 0) {
-      uint32_t kv_cnt = 0, qdo_cnt = 0;
+      uint32_t kv_cnt = 0, q_cnt = 0, do_cnt = 0;
       bool ok = true;
       for (int round = 0; ok; ++round) {
         const int u = unit_for_round(round, blockIdx.x, G);
@@ -300,22 +314,27 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
           tma_load_2d(sbase + Cfg::kOffV + bx * 16384, &tm_v, bx * 64, krow, kv_full);
         }
         for (int i = bwd_next(p, w, w.i_begin); i < p.n_t && ok; i = bwd_next(p, w, i + 1)) {
-          const int s = qdo_cnt % S;
-          ok = mbar_wait(qdo_empty(s), ((qdo_cnt / S) & 1) ^ 1);
-          if (!ok) break;
           const int qrow = w.bh * p.N + i * kTile;
-          mbar_arrive_expect_tx(qdo_full(s), 2 * Cfg::kTileBytes + 2 * Cfg::kRowBytes);
-          for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
-            tma_load_2d(sbase + Cfg::kOffQ + s * Cfg::kTileBytes + bx * 16384, &tm_q, bx * 64, qrow,
-                        qdo_full(s));
-            tma_load_2d(sbase + Cfg::kOffDO + s * Cfg::kTileBytes + bx * 16384, &tm_do, bx * 64,
-                        qrow, qdo_full(s));
-          }
-          bulk_load(sbase + Cfg::kOffRow + s * Cfg::kRowBytes, p.lse2 + qrow, Cfg::kRowBytes,
-                    qdo_full(s));
-          bulk_load(sbase + Cfg::kOffRow + (S + s) * Cfg::kRowBytes, p.delta + qrow,
-                    Cfg::kRowBytes, qdo_full(s));
-          ++qdo_cnt;
+          const int sq = q_cnt % QS;
+          ok = mbar_wait(q_empty(sq), ((q_cnt / QS) & 1) ^ 1);
+          if (!ok) break;
+          mbar_arrive_expect_tx(q_full(sq), Cfg::kTileBytes + 2 * Cfg::kRowBytes);
+          for (int bx = 0; bx < Cfg::kBoxes; ++bx)
+            tma_load_2d(sbase + Cfg::kOffQ + sq * Cfg::kTileBytes + bx * 16384, &tm_q, bx * 64,
+                        qrow, q_full(sq));
+          bulk_load(sbase + Cfg::kOffRow + sq * Cfg::kRowBytes, p.lse2 + qrow, Cfg::kRowBytes,
+                    q_full(sq));
+          bulk_load(sbase + Cfg::kOffRow + (QS + sq) * Cfg::kRowBytes, p.delta + qrow,
+                    Cfg::kRowBytes, q_full(sq));
+          ++q_cnt;
+          const int so = do_cnt % DOS;
+          ok = mbar_wait(do_empty(so), ((do_cnt / DOS) & 1) ^ 1);
+          if (!ok) break;
+          mbar_arrive_expect_tx(do_full(so), Cfg::kTileBytes);
+          for (int bx = 0; bx < Cfg::kBoxes; ++bx)
+            tma_load_2d(sbase + Cfg::kOffDO + so * Cfg::kTileBytes + bx * 16384, &tm_do, bx * 64,
+                        qrow, do_full(so));
+          ++do_cnt;
         }
         if (*abort_flag) ok = false;
       }
@@ -329,7 +348,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       constexpr uint32_t idesc_kk = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T
       constexpr uint32_t idesc_tn = idesc_bf16_f32(128, D, 0, 1);    // dV, dK (A in TMEM)
       constexpr uint32_t idesc_dq = idesc_bf16_f32(128, D, 1, 1);    // dQ (both MN-major)
-      uint32_t kv_cnt = 0, qdo_cnt = 0, p_cnt = 0, ds_cnt = 0, dq_cnt = 0;
+      uint32_t kv_cnt = 0, q_cnt = 0, do_cnt = 0, p_cnt = 0, ds_cnt = 0, dq_cnt = 0;
       bool ok = true;
       // one descriptor base per operand; offsets are added to the start-address field
       const uint64_t dk_k = sw128_desc(sbase + Cfg::kOffK, 16, 1024);     // K_j, K-major
@@ -350,20 +369,23 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         if (!ok) break;
         int t = 0;
         for (int i = bwd_next(p, w, w.i_begin); i < p.n_t && ok; i = bwd_next(p, w, i + 1), ++t) {
-          const int s = qdo_cnt % S;
-          ok = mbar_wait(qdo_full(s), (qdo_cnt / S) & 1);
+          const int sq = q_cnt % QS, so = do_cnt % DOS;
+          ok = mbar_wait(q_full(sq), (q_cnt / QS) & 1);
+          if (!ok) break;
+          ok = mbar_wait(do_full(so), (do_cnt / DOS) & 1);
           if (!ok) break;
           if (Cfg::kDqAliasesS) {  // S^T overwrites the previous dQ: wait for its drain
             ok = mbar_wait(dq_empty, (dq_cnt & 1) ^ 1);
             if (!ok) break;
           }
           tc_fence_after();
-          const uint32_t stage_off = (s * Cfg::kTileBytes) >> 4;
+          const uint32_t q_off = (sq * Cfg::kTileBytes) >> 4;
+          const uint32_t do_off = (so * Cfg::kTileBytes) >> 4;
           // S^T = K_j Q_i^T ; dP^T = V_j dO_i^T
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
-            umma_ss(tmem + Cfg::kColS, dk_k + off, dq_k0 + stage_off + off, idesc_kk,
+            umma_ss(tmem + Cfg::kColS, dk_k + off, dq_k0 + q_off + off, idesc_kk,
                     kk > 0 ? 1u : 0u);
           }
           umma_commit(s_full);
@@ -371,7 +393,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
-            umma_ss(tmem + Cfg::kColDP, dv_k + off, ddo_k0 + stage_off + off, idesc_kk,
+            umma_ss(tmem + Cfg::kColDP, dv_k + off, ddo_k0 + do_off + off, idesc_kk,
                     kk > 0 ? 1u : 0u);
           }
           umma_commit(dp_full);
@@ -383,8 +405,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
             umma_ts(tmem + Cfg::kColDV, tmem + Cfg::packed_col(Cfg::kColS, kk),
-                    ddo_m0 + stage_off + ((kk * 2048) >> 4), idesc_tn,
+                    ddo_m0 + do_off + ((kk * 2048) >> 4), idesc_tn,
                     (t > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(do_empty(so));
+          ++do_cnt;
           // dK += dS^T Q_i ; dQ = dS K_j
           ok = mbar_wait(ds_full, ds_cnt & 1);
           ++ds_cnt;
@@ -397,16 +421,17 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
             umma_ts(tmem + Cfg::kColDK, tmem + Cfg::packed_col(Cfg::kColDP, kk),
-                    dq_m0 + stage_off + ((kk * 2048) >> 4), idesc_tn,
+                    dq_m0 + q_off + ((kk * 2048) >> 4), idesc_tn,
                     (t > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(q_empty(sq));
+          ++q_cnt;
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
             umma_ss(tmem + Cfg::kColDQ, dds_m + ((kk * 2048) >> 4), dk_m + ((kk * 2048) >> 4),
                     idesc_dq, kk > 0 ? 1u : 0u);
           umma_commit(dq_full);
+          umma_commit(ds_smem_empty);
           ++dq_cnt;
-          umma_commit(qdo_empty(s));
-          ++qdo_cnt;
           if (*abort_flag) ok = false;
         }
         if (!ok) break;
@@ -425,6 +450,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     // Warpgroup h (warps 4-7: h = 0, warps 8-11: h = 1) handles queries
     // 64h..64h+63 of every key row; one key row per thread (TMEM lane).
     if constexpr (Cfg::kRegsDs > Cfg::kRegsLaunch) setmaxnreg_inc<Cfg::kRegsDs>();
+    constexpr int kPolyPer4 = Cfg::kPolyPer4;
     const int h = (warp >= 8) ? 1 : 0;
     const int quarter = warp & 3;
     const int kr = quarter * 32 + lane;  // key row within the tile
@@ -432,7 +458,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     const uint32_t tS = t_lane + Cfg::kColS + h * 64;    // this half's S^T / P^T columns
     const uint32_t tDP = t_lane + Cfg::kColDP + h * 64;  // this half's dP^T / dS^T columns
     uint8_t* ds_rowp = smem + Cfg::kOffDS + h * 16384 + kr * 128;
-    uint32_t s_cnt = 0, dp_cnt = 0, dsm_cnt = 0, dkv_cnt = 0, qdo_cnt = 0;
+    uint32_t s_cnt = 0, dp_cnt = 0, dsm_cnt = 0, dkv_cnt = 0, q_cnt = 0;
     bool ok = true;
     for (int round = 0; ok; ++round) {
       const int u = unit_for_round(round, blockIdx.x, G);
@@ -449,16 +475,19 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       }
       const bool key_valid = c_key < w.L;
       for (int i = bwd_next(p, w, w.i_begin); i < p.n_t; i = bwd_next(p, w, i + 1)) {
-        const int s = qdo_cnt % S;
-        ++qdo_cnt;
-        const float4* lz4 = lse2_smem(s) + h * 16;
-        const float4* dz4 = delta_smem(s) + h * 16;
+        const int sq = q_cnt % QS;
+        ++q_cnt;
+        const float4* lz4 = lse2_smem(sq) + h * 16;   // -LSE2
+        const float4* dz4 = delta_smem(sq) + h * 16;  // -D
         const bool diag = p.causal && (i == w.j);
         ok = __all_sync(0xffffffffu, mbar_wait(s_full, s_cnt & 1));
         ++s_cnt;
         if (!ok) break;
         tc_fence_after();
-        // P^T: p[q] = exp2(S^T[kr][q] * scale*log2e - lse2[q]); masked -> 0
+        // P^T: p[q] = exp2(S^T[kr][q] * scale*log2e - LSE2[q]); masked -> 0.
+        // Three kinds of row: a key beyond kv_len (all zero, no exponentials),
+        // the causal diagonal tile (element mask), and the rest (no mask; part
+        // of the exponentials on the FMA pipe through ex2_poly2).
         {
           uint32_t r[2][32];
           tmem_ld32(tS, r[0]);
@@ -466,24 +495,54 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
           tmem_wait_ld();
           reg_fence32(r[0]);
           reg_fence32(r[1]);
+          const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             uint32_t pk[16];
+            // kind: 0 = no mask (part of the exponentials through ex2_poly2),
+            //       1 = causal diagonal tile (element mask)
+            auto make_p = [&](auto kind_tag) {
+              constexpr int kKind = decltype(kind_tag)::value;
 #pragma unroll
-            for (int e4 = 0; e4 < 8; ++e4) {
-              const float4 lz = lz4[c * 8 + e4];
-              const int q0 = h * 64 + c * 32 + 4 * e4;  // query within the tile
-              float p0 = ex2_approx(fmaf(__uint_as_float(r[c][4 * e4]), p.scale_log2, -lz.x));
-              float p1 = ex2_approx(fmaf(__uint_as_float(r[c][4 * e4 + 1]), p.scale_log2, -lz.y));
-              float p2 = ex2_approx(fmaf(__uint_as_float(r[c][4 * e4 + 2]), p.scale_log2, -lz.z));
-              float p3 = ex2_approx(fmaf(__uint_as_float(r[c][4 * e4 + 3]), p.scale_log2, -lz.w));
-              if (!key_valid || (diag && kr > q0)) p0 = 0.f;
-              if (!key_valid || (diag && kr > q0 + 1)) p1 = 0.f;
-              if (!key_valid || (diag && kr > q0 + 2)) p2 = 0.f;
-              if (!key_valid || (diag && kr > q0 + 3)) p3 = 0.f;
-              pk[2 * e4] = pack_bf16x2(p0, p1);
-              pk[2 * e4 + 1] = pack_bf16x2(p2, p3);
+              for (int e4 = 0; e4 < 8; ++e4) {
+                const float4 nl = lz4[c * 8 + e4];  // -LSE2 of 4 queries
+                const uint64_t xa = f2_fma(
+                    f2_pack(__uint_as_float(r[c][4 * e4]), __uint_as_float(r[c][4 * e4 + 1])),
+                    scale2, f2_pack(nl.x, nl.y));
+                const uint64_t xb = f2_fma(
+                    f2_pack(__uint_as_float(r[c][4 * e4 + 2]), __uint_as_float(r[c][4 * e4 + 3])),
+                    scale2, f2_pack(nl.z, nl.w));
+                float x0, x1, x2, x3, p0, p1, p2, p3;
+                f2_unpack(xa, x0, x1);
+                f2_unpack(xb, x2, x3);
+                if (kKind == 0 && (e4 & 3) < kPolyPer4) {
+                  ex2_poly2(x0, x1, p0, p1);
+                } else {
+                  p0 = ex2_approx(x0);
+                  p1 = ex2_approx(x1);
+                }
+                p2 = ex2_approx(x2);
+                p3 = ex2_approx(x3);
+                if (kKind == 1) {
+                  const int q0 = h * 64 + c * 32 + 4 * e4;  // query within the tile
+                  p0 = (kr > q0) ? 0.f : p0;
+                  p1 = (kr > q0 + 1) ? 0.f : p1;
+                  p2 = (kr > q0 + 2) ? 0.f : p2;
+                  p3 = (kr > q0 + 3) ? 0.f : p3;
+                }
+                pk[2 * e4] = pack_bf16x2(p0, p1);
+                pk[2 * e4 + 1] = pack_bf16x2(p2, p3);
+              }
+            };
+            if (!key_valid) {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) pk[e] = 0u;
+            } else if (diag) {
+              make_p(std::integral_constant<int, 1>{});
+            } else {
+              make_p(std::integral_constant<int, 0>{});
             }
+            __syncwarp();
             tmem_st16(tS + c * 16, pk);
           }
         }
@@ -491,6 +550,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         tc_fence_before();
         mbar_arrive(p_full);
         // dS^T: ds[q] = p[q] * (dP^T[kr][q] - D[q]), p read back (bf16) from TMEM
+        // (rows beyond kv_len have p = 0, hence ds = 0)
         ok = __all_sync(0xffffffffu, mbar_wait(dp_full, dp_cnt & 1));
         ++dp_cnt;
         if (!ok) break;
@@ -513,15 +573,18 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
             uint32_t pk[16];
 #pragma unroll
             for (int e4 = 0; e4 < 8; ++e4) {
-              const float4 dz = dz4[c * 8 + e4];
-              const float2 pa =
-                  __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pp[c * 16 + 2 * e4]));
-              const float2 pb = __bfloat1622float2(
-                  *reinterpret_cast<const __nv_bfloat162*>(&pp[c * 16 + 2 * e4 + 1]));
-              pk[2 * e4] = pack_bf16x2(pa.x * (__uint_as_float(r[c][4 * e4]) - dz.x),
-                                       pa.y * (__uint_as_float(r[c][4 * e4 + 1]) - dz.y));
-              pk[2 * e4 + 1] = pack_bf16x2(pb.x * (__uint_as_float(r[c][4 * e4 + 2]) - dz.z),
-                                           pb.y * (__uint_as_float(r[c][4 * e4 + 3]) - dz.w));
+              const float4 nd = dz4[c * 8 + e4];  // -D of 4 queries
+              const uint64_t ta = f2_add(
+                  f2_pack(__uint_as_float(r[c][4 * e4]), __uint_as_float(r[c][4 * e4 + 1])),
+                  f2_pack(nd.x, nd.y));
+              const uint64_t tb = f2_add(
+                  f2_pack(__uint_as_float(r[c][4 * e4 + 2]), __uint_as_float(r[c][4 * e4 + 3])),
+                  f2_pack(nd.z, nd.w));
+              float d0, d1, d2, d3;
+              f2_unpack(f2_mul(ta, bf16x2_to_f2(pp[c * 16 + 2 * e4])), d0, d1);
+              f2_unpack(f2_mul(tb, bf16x2_to_f2(pp[c * 16 + 2 * e4 + 1])), d2, d3);
+              pk[2 * e4] = pack_bf16x2(d0, d1);
+              pk[2 * e4 + 1] = pack_bf16x2(d2, d3);
             }
             tmem_st16(tDP + c * 16, pk);
             // shared-memory copy for the dQ MMA: [key][query], this half's 64-query
@@ -567,16 +630,16 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     if (!ok) *abort_flag = 1;
   } else {
     // ------------------------------------------------------------ dQ group
-    // Drains dQ partials: TMEM -> registers -> shared memory (the dS tile,
-    // free once the dQ MMA has read it) -> TMA reduce-add into the float32
-    // accumulator, in 32 x 32 boxes (128-byte swizzled rows).
+    // Drains dQ partials: TMEM -> registers -> its own shared-memory staging
+    // area -> TMA reduce-add into the float32 accumulator, in 32 x 32 boxes
+    // (128-byte swizzled rows).
     if constexpr (Cfg::kRegsDq > Cfg::kRegsLaunch)
       setmaxnreg_inc<Cfg::kRegsDq>();
     else if constexpr (Cfg::kRegsDq < Cfg::kRegsLaunch)
       setmaxnreg_dec<Cfg::kRegsDq>();
     const int quarter = warp & 3;  // rows quarter*32 .. +31 of the query tile
     const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
-    uint8_t* stage = smem + Cfg::kOffDS + quarter * (Cfg::kDqBoxesPerRound * 4096);
+    uint8_t* stage = smem + Cfg::kOffDQ + quarter * (Cfg::kDqBoxesPerRound * 4096);
     const uint32_t stage_u32 = smem_u32(stage);
     uint32_t dq_cnt = 0;
     bool ok = true;
@@ -622,7 +685,6 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
           }
           __syncwarp();
         }
-        if (lane == 0) mbar_arrive(ds_smem_empty);
         if (*abort_flag) { ok = false; break; }
       }
     }

@@ -17,12 +17,19 @@
 //               MMAs accumulating in tensor memory; owns the TMEM allocation
 //   warps 4-7   softmax warpgroup 0 (TMEM lanes 0-127, one query row each)
 //   warps 8-11  softmax warpgroup 1
-// A work unit is (b, h, one 128-row query tile).  The unit's visited key
-// tiles are dealt alternately to the two softmax warpgroups: warpgroup x
-// owns S_x, O_x in TMEM and its own running (m, l) for every row, so one
-// warpgroup's softmax runs while the tensor core works for the other.  At
-// the end of the unit the two partial results are merged (the same
-// rescaling rule as the online softmax, applied once more).
+// Two ways of filling a work unit, chosen per launch:
+//  * pair mode (no block mask): the unit is (b, h, query tiles 2p and 2p+1).
+//    Both tiles visit the same key tiles (up to the causal diagonal), so
+//    every K/V tile is loaded once for 256 query rows; softmax warpgroup x
+//    owns query tile 2p+x outright.
+//  * split mode (block mask): the unit is (b, h, one query tile), whose
+//    visited key tiles are dealt alternately to the two warpgroups; each
+//    keeps its own running (m, l) and O, and the two partial results are
+//    merged at the end of the unit (the online-softmax rescaling applied
+//    once more).  Random masks give two query tiles few key tiles in common,
+//    so pairing them would leave one warpgroup idle.
+// Either way one warpgroup's softmax runs while the tensor core works for
+// the other.
 //
 // TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 after it.
 // P (bf16) is written over the first 64 columns of its S tile and read from
@@ -62,7 +69,7 @@ struct FwdParams {
   float scale_log2;  // scale * log2(e)
 };
 
-template <int D>
+template <int D, bool kPair>
 struct FwdCfg {
   static constexpr int kThreads = 384;
   // registers per thread: 168 at launch (384 x 168 = 64512); the producer /
@@ -72,8 +79,13 @@ struct FwdCfg {
   static constexpr int kTileBytes = kTile * D * 2;  // one 128 x D bf16 tile
   static constexpr int kBoxes = D / 64;             // 64-column TMA boxes per tile
   static constexpr int kStages = (D == 64) ? 5 : 2;
-  static constexpr int kOffQ = 0;  // two Q buffers (consecutive units)
-  static constexpr int kOffK = kOffQ + 2 * kTileBytes;
+  // Q slots: one per unit in flight (double-buffered across units except for
+  // pair mode at D = 128, where shared memory holds only one); a slot holds
+  // one query tile (split) or two (pair)
+  static constexpr int kQPerSlot = kPair ? 2 : 1;
+  static constexpr int kQSlots = (kPair && D == 128) ? 1 : 2;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kOffQ + kQSlots * kQPerSlot * kTileBytes;
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
   static constexpr int kOffML = kOffV + kStages * kTileBytes;  // [2 warpgroups][128 rows] (m, l)
   static constexpr int kOffBar = kOffML + 2 * kTile * 8;
@@ -100,7 +112,12 @@ __device__ __forceinline__ int unit_for_round(int round, int cta, int G) {
 }
 
 struct FwdUnit {
-  int bh, b, i, L, j_end;
+  int bh, b;
+  int i0, i1;           // query tile of warpgroup 0 / 1 (split mode: the same tile)
+  int has1;             // pair mode: query tile i1 exists
+  int L;                // keys c < L are not padding
+  int j_end0, j_end1;   // key tiles below j_end_x may hold an allowed key for tile i_x
+  int j_end;            // the unit's key tiles lie below j_end
 };
 
 // Unit u -> (head group g, rank within the group, head): ranks are
@@ -115,41 +132,54 @@ __device__ __forceinline__ void group_order(int u, int n_t, int BH, int G, int& 
   bh = h0 + (r - rank * gh);
 }
 
+template <bool kPair>
 __device__ __forceinline__ FwdUnit fwd_decode(const FwdParams& p, int u) {
   FwdUnit w;
+  const int per_head = kPair ? (p.n_t + 1) / 2 : p.n_t;
   int rank;  // 0 = longest
-  group_order(u, p.n_t, p.B * p.H, p.heads_per_group, w.bh, rank);
+  group_order(u, per_head, p.B * p.H, p.heads_per_group, w.bh, rank);
   w.b = w.bh / p.H;
-  w.i = p.causal ? (p.n_t - 1 - rank) : rank;
+  const int slot = p.causal ? (per_head - 1 - rank) : rank;
   int L = p.N;
   if (p.kv_len) {
     L = __ldg(p.kv_len + w.b);
     L = L < 0 ? 0 : (L > p.N ? p.N : L);
   }
   w.L = L;
-  int j_end = (L + kTile - 1) / kTile;   // key tiles holding a key c < L
-  if (p.causal) j_end = min(j_end, w.i + 1);
-  w.j_end = j_end;
+  const int j_kv = (L + kTile - 1) / kTile;  // key tiles holding a key c < L
+  if (kPair) {
+    w.i0 = 2 * slot;
+    w.i1 = 2 * slot + 1;
+    w.has1 = w.i1 < p.n_t;
+  } else {
+    w.i0 = w.i1 = slot;
+    w.has1 = 0;
+  }
+  w.j_end0 = p.causal ? min(j_kv, w.i0 + 1) : j_kv;
+  w.j_end1 = (kPair && !w.has1) ? 0 : (p.causal ? min(j_kv, w.i1 + 1) : j_kv);
+  w.j_end = max(w.j_end0, w.j_end1);
   return w;
 }
 
-// First key tile >= j that query tile w.i visits (or j_end): tiles below
-// j_end hold an allowed key for causal and key-padding masks; the block mask
-// is the only test left.
+// Split mode: first key tile >= j that query tile w.i0 visits (or j_end):
+// tiles below j_end hold an allowed key for causal and key-padding masks; the
+// block mask is the only test left.  (Pair mode has no block mask: its tiles
+// are all of [0, j_end_x).)
 __device__ __forceinline__ int fwd_next(const FwdParams& p, const FwdUnit& w, int j) {
   if (!p.block_mask) return j < w.j_end ? j : w.j_end;
-  const uint8_t* row = p.block_mask + (size_t)w.i * p.n_t;
+  const uint8_t* row = p.block_mask + (size_t)w.i0 * p.n_t;
   for (; j < w.j_end; ++j)
     if (__ldg(row + j)) return j;
   return w.j_end;
 }
 
-template <int D>
-__global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
+template <int D, bool kPair>
+__global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using Cfg = FwdCfg<D>;
+  using Cfg = FwdCfg<D, kPair>;
   constexpr int S = Cfg::kStages;
+  constexpr int QSLOTS = Cfg::kQSlots;
   extern __shared__ __align__(1024) uint8_t smem[];
   if (!smem_aligned_1024(smem)) return;
   const uint32_t sbase = smem_u32(smem);
@@ -164,13 +194,17 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
   auto p_full = [&](int x) { return bar0 + 8 * (6 + 4 * S + x); };
   auto o_full = [&](int x) { return bar0 + 8 * (8 + 4 * S + x); };
   const uint32_t drain_bar = bar0 + 8 * (10 + 4 * S);
-  // the two softmax warpgroups meet twice per unit in the merge: (m, l)
-  // published, and both partial outputs read (bounded waits, 256 arrivals)
+  // split mode: the two softmax warpgroups meet twice per unit in the merge:
+  // (m, l) published, and both partial outputs read (bounded waits, 256 arrivals)
   const uint32_t ml_ready = bar0 + 8 * (11 + 4 * S);
   const uint32_t merged = bar0 + 8 * (12 + 4 * S);
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kOffMisc + 4);
   float2* ml_smem = reinterpret_cast<float2*>(smem + Cfg::kOffML);  // [2][128] (m, l)
+  // shared-memory address of query tile x (0 / 1) of Q slot q
+  auto q_tile = [&](int q, int x) {
+    return sbase + Cfg::kOffQ + (q * Cfg::kQPerSlot + (kPair ? x : 0)) * Cfg::kTileBytes;
+  };
 
   const int warp = warp_id();
   const int lane = lane_id();
@@ -219,15 +253,17 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
       for (int round = 0; ok; ++round) {
         const int u = unit_for_round(round, blockIdx.x, G);
         if (u >= p.num_units) break;
-        const FwdUnit w = fwd_decode(p, u);
-        const int qb = q_cnt & 1;
-        ok = mbar_wait(q_empty(qb), ((q_cnt >> 1) & 1) ^ 1);
+        const FwdUnit w = fwd_decode<kPair>(p, u);
+        const int qs = q_cnt % QSLOTS;
+        ok = mbar_wait(q_empty(qs), ((q_cnt / QSLOTS) & 1) ^ 1);
         if (!ok) break;
         ++q_cnt;
-        mbar_arrive_expect_tx(q_full(qb), Cfg::kTileBytes);
-        for (int bx = 0; bx < Cfg::kBoxes; ++bx)
-          tma_load_2d(sbase + Cfg::kOffQ + qb * Cfg::kTileBytes + bx * 16384, &tm_q, bx * 64,
-                      w.bh * p.N + w.i * kTile, q_full(qb));
+        const int nq = (kPair && w.has1) ? 2 : 1;
+        mbar_arrive_expect_tx(q_full(qs), nq * Cfg::kTileBytes);
+        for (int x = 0; x < nq; ++x)
+          for (int bx = 0; bx < Cfg::kBoxes; ++bx)
+            tma_load_2d(q_tile(qs, x) + bx * 16384, &tm_q, bx * 64,
+                        w.bh * p.N + (x ? w.i1 : w.i0) * kTile, q_full(qs));
         for (int j = fwd_next(p, w, 0); j < w.j_end && ok; j = fwd_next(p, w, j + 1)) {
           const int s = kv_cnt % S;
           const uint32_t ph = (kv_cnt / S) & 1;
@@ -269,63 +305,127 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
       for (int round = 0; ok; ++round) {
         const int u = unit_for_round(round, blockIdx.x, G);
         if (u >= p.num_units) break;
-        const FwdUnit w = fwd_decode(p, u);
-        const int qb = q_cnt & 1;
-        ok = mbar_wait(q_full(qb), (q_cnt >> 1) & 1);
+        const FwdUnit w = fwd_decode<kPair>(p, u);
+        const int qs = q_cnt % QSLOTS;
+        ok = mbar_wait(q_full(qs), (q_cnt / QSLOTS) & 1);
         ++q_cnt;
         if (!ok) break;
-        const uint64_t dq = desc_q0 + ((qb * Cfg::kTileBytes) >> 4);
-        // S(k) for the k-th visited key tile j, into warpgroup (k & 1)'s S columns
-        auto issue_s = [&](int k, int j) -> bool {
-          const uint32_t c = kv_cnt + k;
+        // S_x = Q_x K^T for key tile j held in stage c % S, into warpgroup x's S columns
+        auto issue_s = [&](int x, uint32_t c, int j) {
           const int s = c % S;
-          if (!mbar_wait(k_full(s), (c / S) & 1)) return false;
-          tc_fence_after();
+          const uint64_t dq = desc_q0 + ((q_tile(qs, x) - (sbase + Cfg::kOffQ)) >> 4);
           const uint64_t dk = desc_k0 + ((s * Cfg::kTileBytes) >> 4);
-          const int x = k & 1;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
             umma_ss(tmem + Cfg::col_s(x), dq + off, dk + off, idesc_s, kk > 0 ? 1u : 0u);
           }
           umma_commit(s_full(x));
-          umma_commit(k_empty(s));
-          if (p.visited) p.visited[((size_t)w.bh * p.n_t + w.i) * p.n_t + j] = 1;
-          return true;
+          if (p.visited)
+            p.visited[((size_t)w.bh * p.n_t + (x ? w.i1 : w.i0)) * p.n_t + j] = 1;
         };
-        int jk = fwd_next(p, w, 0);                                   // tile of visit k
-        int jk1 = (jk < w.j_end) ? fwd_next(p, w, jk + 1) : w.j_end;  // visit k + 1
-        if (jk < w.j_end) ok = issue_s(0, jk);
-        if (ok && jk1 < w.j_end) ok = issue_s(1, jk1);
-        int k = 0;
-        while (ok && jk < w.j_end) {
-          const int x = k & 1;
-          const uint32_t c = kv_cnt + k;
+        // O_x += P_x V for the stage c % S
+        auto issue_pv = [&](int x, uint32_t c, uint32_t acc) {
           const int s = c % S;
-          const int jk2 = (jk1 < w.j_end) ? fwd_next(p, w, jk1 + 1) : w.j_end;
-          ok = mbar_wait(p_full(x), p_cnt[x] & 1);
-          ++p_cnt[x];
-          if (!ok) break;
-          ok = mbar_wait(v_full(s), (c / S) & 1);
-          if (!ok) break;
-          tc_fence_after();
           const uint64_t dv = desc_v0 + ((s * Cfg::kTileBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
             umma_ts(tmem + Cfg::col_o(x), tmem + Cfg::col_s(x) + kk * 8, dv + ((kk * 2048) >> 4),
-                    idesc_pv, (kk > 0 || k >= 2) ? 1u : 0u);
-          umma_commit(v_empty(s));
-          if (jk2 < w.j_end) ok = issue_s(k + 2, jk2);
-          jk = jk1;
-          jk1 = jk2;
-          ++k;
-          if (*abort_flag) ok = false;
+                    idesc_pv, (kk > 0 || acc) ? 1u : 0u);
+        };
+        int n_items = 0;  // key tiles consumed by this unit
+        if constexpr (kPair) {
+          // Both tiles walk key tiles 0 .. j_end - 1; tile x takes those below
+          // j_end_x.  Per key tile: PV_0, S_0(next), PV_1, S_1(next), so that
+          // each warpgroup's next S follows its own P V immediately.
+          const int j_end = w.j_end;
+          if (j_end > 0) {
+            ok = mbar_wait(k_full(kv_cnt % S), (kv_cnt / S) & 1);
+            if (ok) {
+              tc_fence_after();
+              if (w.j_end0 > 0) issue_s(0, kv_cnt, 0);
+              if (w.j_end1 > 0) issue_s(1, kv_cnt, 0);
+              umma_commit(k_empty(kv_cnt % S));
+            }
+          }
+          for (int j = 0; j < j_end && ok; ++j) {
+            const uint32_t c = kv_cnt + j;
+            const bool next = j + 1 < j_end;
+            bool v_ready = false, k_next = false;
+            for (int x = 0; x < 2 && ok; ++x) {
+              const int je = x ? w.j_end1 : w.j_end0;
+              if (j < je) {
+                ok = mbar_wait(p_full(x), p_cnt[x] & 1);
+                ++p_cnt[x];
+                if (!ok) break;
+                if (!v_ready) {
+                  ok = mbar_wait(v_full(c % S), (c / S) & 1);
+                  if (!ok) break;
+                  v_ready = true;
+                }
+                tc_fence_after();
+                issue_pv(x, c, j > 0);
+              }
+              if (x == 1) umma_commit(v_empty(c % S));
+              if (next && j + 1 < je) {
+                if (!k_next) {
+                  ok = mbar_wait(k_full((c + 1) % S), ((c + 1) / S) & 1);
+                  if (!ok) break;
+                  tc_fence_after();
+                  k_next = true;
+                }
+                issue_s(x, c + 1, j + 1);
+              }
+            }
+            if (ok && next) umma_commit(k_empty((c + 1) % S));
+            if (*abort_flag) ok = false;
+          }
+          if (!ok) break;
+          n_items = j_end;
+          if (w.j_end0 > 0) umma_commit(o_full(0));
+          if (w.j_end1 > 0) umma_commit(o_full(1));
+        } else {
+          // k-th visited key tile goes to warpgroup k & 1: S(k), S(k + 1) first,
+          // then per k: P V(k), S(k + 2) (same warpgroup, its S columns are free
+          // once P V(k) has read P(k) - tcgen05 MMAs execute in issue order)
+          auto issue_s_k = [&](int k, int j) -> bool {
+            const uint32_t c = kv_cnt + k;
+            if (!mbar_wait(k_full(c % S), (c / S) & 1)) return false;
+            tc_fence_after();
+            issue_s(k & 1, c, j);
+            umma_commit(k_empty(c % S));
+            return true;
+          };
+          int jk = fwd_next(p, w, 0);                                   // tile of visit k
+          int jk1 = (jk < w.j_end) ? fwd_next(p, w, jk + 1) : w.j_end;  // visit k + 1
+          if (jk < w.j_end) ok = issue_s_k(0, jk);
+          if (ok && jk1 < w.j_end) ok = issue_s_k(1, jk1);
+          int k = 0;
+          while (ok && jk < w.j_end) {
+            const int x = k & 1;
+            const uint32_t c = kv_cnt + k;
+            const int jk2 = (jk1 < w.j_end) ? fwd_next(p, w, jk1 + 1) : w.j_end;
+            ok = mbar_wait(p_full(x), p_cnt[x] & 1);
+            ++p_cnt[x];
+            if (!ok) break;
+            ok = mbar_wait(v_full(c % S), (c / S) & 1);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv(x, c, k >= 2);
+            umma_commit(v_empty(c % S));
+            if (jk2 < w.j_end) ok = issue_s_k(k + 2, jk2);
+            jk = jk1;
+            jk1 = jk2;
+            ++k;
+            if (*abort_flag) ok = false;
+          }
+          if (!ok) break;
+          n_items = k;
+          if (k >= 1) umma_commit(o_full(0));
+          if (k >= 2) umma_commit(o_full(1));
         }
-        if (!ok) break;
-        if (k >= 1) umma_commit(o_full(0));
-        if (k >= 2) umma_commit(o_full(1));
-        umma_commit(q_empty(qb));
-        kv_cnt += k;
+        umma_commit(q_empty(qs));
+        kv_cnt += n_items;
       }
       if (!ok) *abort_flag = 1;
       // all issued MMAs complete before TMEM is released
@@ -351,14 +451,18 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
     for (int round = 0; ok; ++round) {
       const int u = unit_for_round(round, blockIdx.x, G);
       if (u >= p.num_units) break;
-      const FwdUnit w = fwd_decode(p, u);
-      const int row = w.i * kTile + r_local;  // query index within the head
-      float m_used = -INFINITY;              // log2 domain, scale folded in
+      const FwdUnit w = fwd_decode<kPair>(p, u);
+      if (kPair && x == 1 && !w.has1) continue;  // pair with no second tile
+      const int i_me = x ? w.i1 : w.i0;           // this warpgroup's query tile
+      const int j_end_me = x ? w.j_end1 : w.j_end0;
+      const int row = i_me * kTile + r_local;     // query index within the head
+      float m_used = -INFINITY;                   // log2 domain, scale folded in
       float l = 0.f;
-      int cnt = 0;   // tiles this warpgroup processed
-      int k = 0;     // visit index over both warpgroups
-      for (int j = fwd_next(p, w, 0); j < w.j_end; j = fwd_next(p, w, j + 1), ++k) {
-        if ((k & 1) != x) continue;
+      int cnt = 0;  // tiles this warpgroup processed
+      int k = 0;    // split mode: visit index over both warpgroups
+      for (int j = kPair ? 0 : fwd_next(p, w, 0); j < (kPair ? j_end_me : w.j_end);
+           j = kPair ? j + 1 : fwd_next(p, w, j + 1), ++k) {
+        if (!kPair && (k & 1) != x) continue;
         ok = __all_sync(0xffffffffu, mbar_wait(s_full(x), s_cnt & 1));
         ++s_cnt;
         if (!ok) break;
@@ -377,7 +481,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
           }
         }
         // element masks on boundary tiles only
-        const bool diag = p.causal && (j == w.i);
+        const bool diag = p.causal && (j == i_me);
         const int kv_lim = w.L - j * kTile;  // keys c >= kv_lim are padding
         const bool boundary = diag || kv_lim < kTile;
         if (boundary) {
@@ -469,68 +573,102 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
         if (*abort_flag) { ok = false; break; }
       }
       if (!ok) break;
-      // ---------------------------------------------------- merge + epilogue
-      // k = visits of the unit: warpgroup 0 processed ceil(k/2), warpgroup 1
-      // floor(k/2).  Both warpgroups read both partial outputs: warpgroup x
-      // finishes columns [x*D/2, (x+1)*D/2) of every row.
-      const int n0 = (k + 1) / 2, n1 = k / 2;
-      if (n0 > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(o_full(0), o_cnt[0] & 1));
-        ++o_cnt[0];
-      }
-      if (ok && n1 > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(o_full(1), o_cnt[1] & 1));
-        ++o_cnt[1];
-      }
-      if (!ok) break;
-      tc_fence_after();
-      ml_smem[x * kTile + r_local] = make_float2(m_used, cnt > 0 ? l : 0.f);
-      mbar_arrive(ml_ready);
-      ok = __all_sync(0xffffffffu, mbar_wait(ml_ready, unit_cnt & 1));
-      if (!ok) break;
-      const float2 ml0 = ml_smem[r_local];
-      const float2 ml1 = ml_smem[kTile + r_local];
-      const float m = fmaxf(ml0.x, ml1.x);
-      const float a0 = (ml0.y > 0.f) ? ex2_approx(ml0.x - m) : 0.f;
-      const float a1 = (ml1.y > 0.f) ? ex2_approx(ml1.x - m) : 0.f;
-      const float lt = ml0.y * a0 + ml1.y * a1;
-      const float inv_l = (lt > 0.f) ? 1.f / lt : 0.f;
-      const float f0 = a0 * inv_l, f1 = a1 * inv_l;
       const size_t grow = (size_t)w.bh * p.N + row;
-      uint4* orow = reinterpret_cast<uint4*>(p.o + grow * D + x * (D / 2));
-      // A warpgroup that processed no tile left its O unwritten: its factor is 0
-      // and its values are dropped by a select (never multiplied, in case the
-      // unwritten columns hold a NaN pattern).
-      const bool use0 = n0 > 0, use1 = n1 > 0;
+      if constexpr (kPair) {
+        // ---------------------------------------------------- epilogue (own tile)
+        uint4* orow = reinterpret_cast<uint4*>(p.o + grow * D);
+        if (cnt > 0) {
+          ok = __all_sync(0xffffffffu, mbar_wait(o_full(x), o_cnt[x] & 1));
+          ++o_cnt[x];
+          if (!ok) break;
+          tc_fence_after();
+          const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
 #pragma unroll 1
-      for (int c = 0; c < D / 64; ++c) {
-        const uint32_t col = x * (D / 2) + c * 32;
-        uint32_t r0[32], r1[32];
-        tmem_ld32(t_lane + Cfg::col_o(0) + col, r0);
-        tmem_ld32(t_lane + Cfg::col_o(1) + col, r1);
-        tmem_wait_ld();
-        reg_fence32(r0);
-        reg_fence32(r1);
-        uint32_t pk[16];
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32(tO + c * 32, r);
+            tmem_wait_ld();
+            reg_fence32(r);
+            uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float a = use0 ? __uint_as_float(r0[2 * e]) * f0 : 0.f;
-          const float b = use0 ? __uint_as_float(r0[2 * e + 1]) * f0 : 0.f;
-          const float c2 = use1 ? __uint_as_float(r1[2 * e]) * f1 : 0.f;
-          const float d2 = use1 ? __uint_as_float(r1[2 * e + 1]) * f1 : 0.f;
-          pk[e] = pack_bf16x2(a + c2, b + d2);
+            for (int e = 0; e < 16; ++e)
+              pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv_l,
+                                  __uint_as_float(r[2 * e + 1]) * inv_l);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              orow[c * 4 + v4] =
+                  make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+          }
+          tc_fence_before();
+          p.lse[grow] = (l > 0.f) ? (m_used + log2f(l)) * kLn2 : -INFINITY;
+        } else {
+#pragma unroll
+          for (int c = 0; c < D / 8; ++c) orow[c] = make_uint4(0, 0, 0, 0);
+          p.lse[grow] = -INFINITY;
         }
+      } else {
+        // ---------------------------------------------------- merge + epilogue
+        // k = visits of the unit: warpgroup 0 processed ceil(k/2), warpgroup 1
+        // floor(k/2).  Both warpgroups read both partial outputs: warpgroup x
+        // finishes columns [x*D/2, (x+1)*D/2) of every row.
+        const int n0 = (k + 1) / 2, n1 = k / 2;
+        if (n0 > 0) {
+          ok = __all_sync(0xffffffffu, mbar_wait(o_full(0), o_cnt[0] & 1));
+          ++o_cnt[0];
+        }
+        if (ok && n1 > 0) {
+          ok = __all_sync(0xffffffffu, mbar_wait(o_full(1), o_cnt[1] & 1));
+          ++o_cnt[1];
+        }
+        if (!ok) break;
+        tc_fence_after();
+        ml_smem[x * kTile + r_local] = make_float2(m_used, cnt > 0 ? l : 0.f);
+        mbar_arrive(ml_ready);
+        ok = __all_sync(0xffffffffu, mbar_wait(ml_ready, unit_cnt & 1));
+        if (!ok) break;
+        const float2 ml0 = ml_smem[r_local];
+        const float2 ml1 = ml_smem[kTile + r_local];
+        const float m = fmaxf(ml0.x, ml1.x);
+        const float a0 = (ml0.y > 0.f) ? ex2_approx(ml0.x - m) : 0.f;
+        const float a1 = (ml1.y > 0.f) ? ex2_approx(ml1.x - m) : 0.f;
+        const float lt = ml0.y * a0 + ml1.y * a1;
+        const float inv_l = (lt > 0.f) ? 1.f / lt : 0.f;
+        const float f0 = a0 * inv_l, f1 = a1 * inv_l;
+        uint4* orow = reinterpret_cast<uint4*>(p.o + grow * D + x * (D / 2));
+        // A warpgroup that processed no tile left its O unwritten: its factor is 0
+        // and its values are dropped by a select (never multiplied, in case the
+        // unwritten columns hold a NaN pattern).
+        const bool use0 = n0 > 0, use1 = n1 > 0;
+#pragma unroll 1
+        for (int c = 0; c < D / 64; ++c) {
+          const uint32_t col = x * (D / 2) + c * 32;
+          uint32_t r0[32], r1[32];
+          tmem_ld32(t_lane + Cfg::col_o(0) + col, r0);
+          tmem_ld32(t_lane + Cfg::col_o(1) + col, r1);
+          tmem_wait_ld();
+          reg_fence32(r0);
+          reg_fence32(r1);
+          uint32_t pk[16];
 #pragma unroll
-        for (int v4 = 0; v4 < 4; ++v4)
-          orow[c * 4 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+          for (int e = 0; e < 16; ++e) {
+            const float a = use0 ? __uint_as_float(r0[2 * e]) * f0 : 0.f;
+            const float b = use0 ? __uint_as_float(r0[2 * e + 1]) * f0 : 0.f;
+            const float c2 = use1 ? __uint_as_float(r1[2 * e]) * f1 : 0.f;
+            const float d2 = use1 ? __uint_as_float(r1[2 * e + 1]) * f1 : 0.f;
+            pk[e] = pack_bf16x2(a + c2, b + d2);
+          }
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            orow[c * 4 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+        }
+        if (x == 0) p.lse[grow] = (lt > 0.f) ? (m + log2f(lt)) * kLn2 : -INFINITY;
+        tc_fence_before();
+        // neither warpgroup starts the next unit (whose first P V overwrites an O)
+        // before both have read both partial outputs
+        mbar_arrive(merged);
+        ok = __all_sync(0xffffffffu, mbar_wait(merged, unit_cnt & 1));
+        ++unit_cnt;
       }
-      if (x == 0) p.lse[grow] = (lt > 0.f) ? (m + log2f(lt)) * kLn2 : -INFINITY;
-      tc_fence_before();
-      // neither warpgroup starts the next unit (whose first P V overwrites an O)
-      // before both have read both partial outputs
-      mbar_arrive(merged);
-      ok = __all_sync(0xffffffffu, mbar_wait(merged, unit_cnt & 1));
-      ++unit_cnt;
     }
     if (!ok) *abort_flag = 1;
   }
