@@ -30,7 +30,7 @@
 //   dV  += P^T dO_i           (A = P^T bf16 in TMEM over S^T's first 64 cols)
 //   dK  += dS^T Q_i           (A = dS^T bf16 in TMEM over dP^T's first 64 cols)
 //   dQ   = dS K_j             (A = dS from shared memory; result in cols 384..447
-//                             for D = 64, over S^T's cols 0..127 for D = 128)
+//                             for D = 64, over dP^T's cols 128..255 for D = 128)
 // dK and dV accumulate in cols 256..256+2D-1 for the whole unit.
 #pragma once
 
@@ -126,15 +126,14 @@ struct BwdParams {
 template <int D>
 struct BwdCfg {
   static constexpr int kThreads = 512;
-  // registers per thread: 128 at launch (512 x 128 = 65536); the producer /
-  // MMA warpgroup drops to 96 (D = 64) or 88 (D = 128) and the rest is shared
-  // by the two dS warpgroups and the dQ warpgroup (which holds a whole
-  // float32 dQ row):
-  // D = 64:  128 x 96 + 256 x 136 + 128 x 120 = 62464
-  // D = 128: 128 x 88 + 256 x 128 + 128 x 168 = 65536
-  static constexpr uint32_t kRegsLaunch = 128, kRegsLow = (D == 64) ? 96 : 88;
+  // registers per thread: 128 at launch (512 x 128 = 65536), redistributed:
+  //          producer/MMA   two dS warpgroups   dQ warpgroup
+  // D = 64:  128 x 104   +  256 x 136        +  128 x 112  = 62464
+  // D = 128: 128 x 96    +  256 x 128        +  128 x 160  = 65536
+  // (the dQ warpgroup holds a whole float32 dQ row)
+  static constexpr uint32_t kRegsLaunch = 128, kRegsLow = (D == 64) ? 104 : 96;
   static constexpr uint32_t kRegsDs = (D == 64) ? 136 : 128;
-  static constexpr uint32_t kRegsDq = (D == 64) ? 120 : 168;
+  static constexpr uint32_t kRegsDq = (D == 64) ? 112 : 160;
   static constexpr int kTileBytes = kTile * D * 2;
   static constexpr int kBoxes = D / 64;
   // Q_i (with the tile's -LSE2 and -D rows) and dO_i come through separate
@@ -169,9 +168,10 @@ struct BwdCfg {
   static constexpr uint32_t kColDP = 128;
   static constexpr uint32_t kColDK = 256;
   static constexpr uint32_t kColDV = 256 + D;
-  // dQ = dS K_j: its own columns when they fit (D = 64), else over S^T
-  static constexpr uint32_t kColDQ = (D == 64) ? 384 : 0;
-  static constexpr bool kDqAliasesS = (kColDQ == kColS);
+  // dQ = dS K_j: its own columns when they fit (D = 64), else over dP^T
+  // (after the dK MMA has read dS^T there; the next dP^T waits for the drain)
+  static constexpr uint32_t kColDQ = (D == 64) ? 384 : 128;
+  static constexpr bool kDqAliasesDP = (kColDQ == kColDP);
   // dQ staging: each dQ warp owns 8 KB = two 32 x 32 float32 boxes
   static constexpr int kDqBoxesPerRound = 2;
   static constexpr int kDqRounds = D / 64;
@@ -348,7 +348,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       constexpr uint32_t idesc_kk = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T
       constexpr uint32_t idesc_tn = idesc_bf16_f32(128, D, 0, 1);    // dV, dK (A in TMEM)
       constexpr uint32_t idesc_dq = idesc_bf16_f32(128, D, 1, 1);    // dQ (both MN-major)
-      uint32_t kv_cnt = 0, q_cnt = 0, do_cnt = 0, p_cnt = 0, ds_cnt = 0, dq_cnt = 0;
+      uint32_t kv_cnt = 0, q_cnt = 0, do_cnt = 0, p_cnt = 0, ds_cnt = 0;
+      uint32_t dq_cnt = 0, dq_drained = 0;  // dQ MMAs issued / drained by the dQ group
       bool ok = true;
       // one descriptor base per operand; offsets are added to the start-address field
       const uint64_t dk_k = sw128_desc(sbase + Cfg::kOffK, 16, 1024);     // K_j, K-major
@@ -359,6 +360,45 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       const uint64_t ddo_m0 = sw128_desc(sbase + Cfg::kOffDO, 16384, 1024);  // dO_i, MN-major
       const uint64_t dk_m = sw128_desc(sbase + Cfg::kOffK, 16384, 1024);     // K_j, MN-major
       const uint64_t dds_m = sw128_desc(sbase + Cfg::kOffDS, 16384, 1024);   // dS, MN-major
+      // waits until every issued dQ has been read out of TMEM by the dQ group
+      auto drain_dq = [&]() -> bool {
+        while (dq_drained < dq_cnt) {
+          if (!mbar_wait(dq_empty, dq_drained & 1)) return false;
+          ++dq_drained;
+        }
+        return true;
+      };
+      // S^T = K_j Q_i^T for the Q tile in ring slot c
+      auto issue_st = [&](uint32_t c, const BwdUnit& w, int i) -> bool {
+        const int sq = c % QS;
+        if (!mbar_wait(q_full(sq), (c / QS) & 1)) return false;
+        tc_fence_after();
+        const uint32_t q_off = (sq * Cfg::kTileBytes) >> 4;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+          umma_ss(tmem + Cfg::kColS, dk_k + off, dq_k0 + q_off + off, idesc_kk, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(s_full);
+        if (p.visited) p.visited[((size_t)w.bh * p.n_t + i) * p.n_t + w.j] = 1;
+        return true;
+      };
+      // dP^T = V_j dO_i^T for the dO tile in ring slot c
+      auto issue_dpt = [&](uint32_t c) -> bool {
+        const int so = c % DOS;
+        if (!mbar_wait(do_full(so), (c / DOS) & 1)) return false;
+        if (Cfg::kDqAliasesDP && !drain_dq()) return false;  // dP^T overwrites the last dQ
+        tc_fence_after();
+        const uint32_t do_off = (so * Cfg::kTileBytes) >> 4;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+          umma_ss(tmem + Cfg::kColDP, dv_k + off, ddo_k0 + do_off + off, idesc_kk,
+                  kk > 0 ? 1u : 0u);
+        }
+        umma_commit(dp_full);
+        return true;
+      };
       for (int round = 0; ok; ++round) {
         const int u = unit_for_round(round, blockIdx.x, G);
         if (u >= p.num_units) break;
@@ -367,36 +407,19 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         ok = mbar_wait(kv_full, kv_cnt & 1);
         ++kv_cnt;
         if (!ok) break;
-        int t = 0;
-        for (int i = bwd_next(p, w, w.i_begin); i < p.n_t && ok; i = bwd_next(p, w, i + 1), ++t) {
+        // Per query tile t the issue order is
+        //   dV(t) | S^T(t+1) dK(t) dQ(t) dP^T(t+1)
+        // so that the P phase of tile t+1 overlaps the dK / dQ MMAs of tile t:
+        // S^T's columns are free once dS(t) is ready (its P^T has been read by
+        // the dV MMA and by the dS warps), and dP^T(t+1) follows dK(t), which
+        // reads dS^T(t) from the dP^T columns.
+        int i = bwd_next(p, w, w.i_begin);
+        ok = issue_st(q_cnt, w, i) && issue_dpt(do_cnt);
+        for (int t = 0; ok && i < p.n_t; ++t) {
+          const int inext = bwd_next(p, w, i + 1);
           const int sq = q_cnt % QS, so = do_cnt % DOS;
-          ok = mbar_wait(q_full(sq), (q_cnt / QS) & 1);
-          if (!ok) break;
-          ok = mbar_wait(do_full(so), (do_cnt / DOS) & 1);
-          if (!ok) break;
-          if (Cfg::kDqAliasesS) {  // S^T overwrites the previous dQ: wait for its drain
-            ok = mbar_wait(dq_empty, (dq_cnt & 1) ^ 1);
-            if (!ok) break;
-          }
-          tc_fence_after();
           const uint32_t q_off = (sq * Cfg::kTileBytes) >> 4;
           const uint32_t do_off = (so * Cfg::kTileBytes) >> 4;
-          // S^T = K_j Q_i^T ; dP^T = V_j dO_i^T
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
-            umma_ss(tmem + Cfg::kColS, dk_k + off, dq_k0 + q_off + off, idesc_kk,
-                    kk > 0 ? 1u : 0u);
-          }
-          umma_commit(s_full);
-          if (p.visited) p.visited[((size_t)w.bh * p.n_t + i) * p.n_t + w.j] = 1;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
-            umma_ss(tmem + Cfg::kColDP, dv_k + off, ddo_k0 + do_off + off, idesc_kk,
-                    kk > 0 ? 1u : 0u);
-          }
-          umma_commit(dp_full);
           // dV += P^T dO_i
           ok = mbar_wait(p_full, p_cnt & 1);
           ++p_cnt;
@@ -409,15 +432,15 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
                     (t > 0 || kk > 0) ? 1u : 0u);
           umma_commit(do_empty(so));
           ++do_cnt;
-          // dK += dS^T Q_i ; dQ = dS K_j
           ok = mbar_wait(ds_full, ds_cnt & 1);
           ++ds_cnt;
           if (!ok) break;
-          if (!Cfg::kDqAliasesS) {  // dQ columns must have been drained
-            ok = mbar_wait(dq_empty, (dq_cnt & 1) ^ 1);
+          if (inext < p.n_t) {
+            ok = issue_st(q_cnt + 1, w, inext);
             if (!ok) break;
           }
           tc_fence_after();
+          // dK += dS^T Q_i
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
             umma_ts(tmem + Cfg::kColDK, tmem + Cfg::packed_col(Cfg::kColDP, kk),
@@ -425,6 +448,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
                     (t > 0 || kk > 0) ? 1u : 0u);
           umma_commit(q_empty(sq));
           ++q_cnt;
+          // dQ = dS K_j
+          if (!Cfg::kDqAliasesDP && !drain_dq()) { ok = false; break; }
+          tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
             umma_ss(tmem + Cfg::kColDQ, dds_m + ((kk * 2048) >> 4), dk_m + ((kk * 2048) >> 4),
@@ -432,6 +458,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
           umma_commit(dq_full);
           umma_commit(ds_smem_empty);
           ++dq_cnt;
+          if (inext < p.n_t) {
+            ok = issue_dpt(do_cnt);
+            if (!ok) break;
+          }
+          i = inext;
           if (*abort_flag) ok = false;
         }
         if (!ok) break;
