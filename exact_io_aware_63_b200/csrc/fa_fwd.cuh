@@ -97,7 +97,7 @@ struct FwdCfg {
   static_assert(kSmemBytes <= 232448, "shared memory over the per-block limit");
   static constexpr uint32_t kTmemCols = 512;
   // pairs (of every 8) whose exponentials ex2_poly2 computes on interior tiles
-  static constexpr int kPolyPer8 = (D == 64) ? 3 : 1;
+  static constexpr int kPolyPer8 = (D == 64) ? 2 : 1;
   __device__ static constexpr uint32_t col_s(int x) { return x ? 128u : 0u; }
   __device__ static constexpr uint32_t col_o(int x) { return x ? 256u + D : 256u; }
 };
@@ -338,14 +338,15 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
           // Both tiles walk key tiles 0 .. j_end - 1; tile x takes those below
           // j_end_x.  Per key tile: PV_0, S_0(next), PV_1, S_1(next), so that
           // each warpgroup's next S follows its own P V immediately.
+          // Warpgroup 1 starts one step behind warpgroup 0 (its first S is
+          // issued after P V_0(0)), so that one warpgroup's softmax overlaps
+          // the other's MMAs instead of competing with it for issue slots.
           const int j_end = w.j_end;
           if (j_end > 0) {
             ok = mbar_wait(k_full(kv_cnt % S), (kv_cnt / S) & 1);
             if (ok) {
               tc_fence_after();
               if (w.j_end0 > 0) issue_s(0, kv_cnt, 0);
-              if (w.j_end1 > 0) issue_s(1, kv_cnt, 0);
-              umma_commit(k_empty(kv_cnt % S));
             }
           }
           for (int j = 0; j < j_end && ok; ++j) {
@@ -376,6 +377,10 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
                 }
                 issue_s(x, c + 1, j + 1);
               }
+              if (x == 0 && j == 0) {  // the delayed first S of warpgroup 1
+                if (w.j_end1 > 0) issue_s(1, c, 0);
+                umma_commit(k_empty(c % S));
+              }
             }
             if (ok && next) umma_commit(k_empty((c + 1) % S));
             if (*abort_flag) ok = false;
@@ -385,9 +390,10 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
           if (w.j_end0 > 0) umma_commit(o_full(0));
           if (w.j_end1 > 0) umma_commit(o_full(1));
         } else {
-          // k-th visited key tile goes to warpgroup k & 1: S(k), S(k + 1) first,
-          // then per k: P V(k), S(k + 2) (same warpgroup, its S columns are free
-          // once P V(k) has read P(k) - tcgen05 MMAs execute in issue order)
+          // k-th visited key tile goes to warpgroup k & 1: S(0) first, then per
+          // k: P V(k), S(k + 2) (same warpgroup, its S columns are free once
+          // P V(k) has read P(k) - tcgen05 MMAs execute in issue order), with
+          // S(1) issued right after P V(0)
           auto issue_s_k = [&](int k, int j) -> bool {
             const uint32_t c = kv_cnt + k;
             if (!mbar_wait(k_full(c % S), (c / S) & 1)) return false;
@@ -398,8 +404,8 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
           };
           int jk = fwd_next(p, w, 0);                                   // tile of visit k
           int jk1 = (jk < w.j_end) ? fwd_next(p, w, jk + 1) : w.j_end;  // visit k + 1
+          // warpgroup 1's first S (visit 1) is issued after P V(0): see pair mode
           if (jk < w.j_end) ok = issue_s_k(0, jk);
-          if (ok && jk1 < w.j_end) ok = issue_s_k(1, jk1);
           int k = 0;
           while (ok && jk < w.j_end) {
             const int x = k & 1;
@@ -413,7 +419,8 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
             tc_fence_after();
             issue_pv(x, c, k >= 2);
             umma_commit(v_empty(c % S));
-            if (jk2 < w.j_end) ok = issue_s_k(k + 2, jk2);
+            if (k == 0 && jk1 < w.j_end) ok = issue_s_k(1, jk1);
+            if (ok && jk2 < w.j_end) ok = issue_s_k(k + 2, jk2);
             jk = jk1;
             jk1 = jk2;
             ++k;
