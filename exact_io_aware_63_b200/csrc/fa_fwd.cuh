@@ -302,18 +302,27 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
       uint32_t q_cnt = 0, kv_cnt = 0;
       uint32_t p_cnt[2] = {0, 0};
       bool ok = true;
+      // Pair mode with two Q slots looks one unit ahead: warpgroup x's first S
+      // of the next unit is issued right after its last P V of this one, so
+      // its epilogue overlaps that MMA and the one-step offset between the two
+      // warpgroups carries over from unit to unit.
+      constexpr bool kLook = kPair && QSLOTS == 2;
+      uint32_t pre = 0;      // bit x: S_x of this unit's first key tile already issued
+      bool pre_q = false;    // this unit's Q already waited for
+      bool pre_k = false;    // this unit's first K tile already waited for
       for (int round = 0; ok; ++round) {
         const int u = unit_for_round(round, blockIdx.x, G);
         if (u >= p.num_units) break;
         const FwdUnit w = fwd_decode<kPair>(p, u);
         const int qs = q_cnt % QSLOTS;
-        ok = mbar_wait(q_full(qs), (q_cnt / QSLOTS) & 1);
+        if (!pre_q) ok = mbar_wait(q_full(qs), (q_cnt / QSLOTS) & 1);
         ++q_cnt;
         if (!ok) break;
-        // S_x = Q_x K^T for key tile j held in stage c % S, into warpgroup x's S columns
-        auto issue_s = [&](int x, uint32_t c, int j) {
+        // S_x = Q_x K^T of unit w's key tile j, Q from slot q, K from stage c % S,
+        // into warpgroup x's S columns
+        auto issue_s_of = [&](const FwdUnit& wu, int q, int x, uint32_t c, int j) {
           const int s = c % S;
-          const uint64_t dq = desc_q0 + ((q_tile(qs, x) - (sbase + Cfg::kOffQ)) >> 4);
+          const uint64_t dq = desc_q0 + ((q_tile(q, x) - (sbase + Cfg::kOffQ)) >> 4);
           const uint64_t dk = desc_k0 + ((s * Cfg::kTileBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
@@ -322,8 +331,9 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
           }
           umma_commit(s_full(x));
           if (p.visited)
-            p.visited[((size_t)w.bh * p.n_t + (x ? w.i1 : w.i0)) * p.n_t + j] = 1;
+            p.visited[((size_t)wu.bh * p.n_t + (x ? wu.i1 : wu.i0)) * p.n_t + j] = 1;
         };
+        auto issue_s = [&](int x, uint32_t c, int j) { issue_s_of(w, qs, x, c, j); };
         // O_x += P_x V for the stage c % S
         auto issue_pv = [&](int x, uint32_t c, uint32_t acc) {
           const int s = c % S;
@@ -336,17 +346,27 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
         int n_items = 0;  // key tiles consumed by this unit
         if constexpr (kPair) {
           // Both tiles walk key tiles 0 .. j_end - 1; tile x takes those below
-          // j_end_x.  Per key tile: PV_0, S_0(next), PV_1, S_1(next), so that
-          // each warpgroup's next S follows its own P V immediately.
-          // Warpgroup 1 starts one step behind warpgroup 0 (its first S is
-          // issued after P V_0(0)), so that one warpgroup's softmax overlaps
-          // the other's MMAs instead of competing with it for issue slots.
+          // j_end_x (j_end_0 >= 1 whenever j_end >= 1).  Per key tile: PV_0,
+          // S_0(next), PV_1, S_1(next), so that each warpgroup's next S follows
+          // its own P V immediately.  In the first unit warpgroup 1 starts one
+          // step behind warpgroup 0 (its first S is issued after P V_0(0)), so
+          // that one warpgroup's softmax overlaps the other's MMAs instead of
+          // competing with it for issue slots.
           const int j_end = w.j_end;
-          if (j_end > 0) {
-            ok = mbar_wait(k_full(kv_cnt % S), (kv_cnt / S) & 1);
+          // the next unit (look-ahead)
+          const int un = unit_for_round(round + 1, blockIdx.x, G);
+          const bool has_next = kLook && un < p.num_units;
+          FwdUnit wn = w;
+          if (has_next) wn = fwd_decode<kPair>(p, un);
+          const int qsn = q_cnt % QSLOTS;
+          const uint32_t cn = kv_cnt + j_end;  // ring index of the next unit's first tile
+          uint32_t pre_next = 0;
+          bool q_next = false, k_next0 = false;
+          if (j_end > 0 && !(pre & 1)) {
+            if (!pre_k) ok = mbar_wait(k_full(kv_cnt % S), (kv_cnt / S) & 1);
             if (ok) {
               tc_fence_after();
-              if (w.j_end0 > 0) issue_s(0, kv_cnt, 0);
+              issue_s(0, kv_cnt, 0);
             }
           }
           for (int j = 0; j < j_end && ok; ++j) {
@@ -366,6 +386,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
                 }
                 tc_fence_after();
                 issue_pv(x, c, j > 0);
+                if (j == je - 1) umma_commit(o_full(x));
               }
               if (x == 1) umma_commit(v_empty(c % S));
               if (next && j + 1 < je) {
@@ -376,9 +397,26 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
                   k_next = true;
                 }
                 issue_s(x, c + 1, j + 1);
+              } else if (has_next && j == je - 1 && (x ? wn.j_end1 : wn.j_end0) > 0) {
+                // warpgroup x is done with this unit: its first S of the next one
+                if (!q_next) {
+                  ok = mbar_wait(q_full(qsn), (q_cnt / QSLOTS) & 1);
+                  if (!ok) break;
+                  q_next = true;
+                }
+                if (!k_next0) {
+                  ok = mbar_wait(k_full(cn % S), (cn / S) & 1);
+                  if (!ok) break;
+                  k_next0 = true;
+                }
+                tc_fence_after();
+                issue_s_of(wn, qsn, x, cn, 0);
+                pre_next |= 1u << x;
               }
-              if (x == 0 && j == 0) {  // the delayed first S of warpgroup 1
-                if (w.j_end1 > 0) issue_s(1, c, 0);
+              if (x == 0 && j == 0) {
+                // warpgroup 1's first S of this unit, unless issued already;
+                // then K of tile 0 has both its readers
+                if (w.j_end1 > 0 && !(pre & 2)) issue_s(1, c, 0);
                 umma_commit(k_empty(c % S));
               }
             }
@@ -387,8 +425,9 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
           }
           if (!ok) break;
           n_items = j_end;
-          if (w.j_end0 > 0) umma_commit(o_full(0));
-          if (w.j_end1 > 0) umma_commit(o_full(1));
+          pre = pre_next;
+          pre_q = q_next;
+          pre_k = k_next0;
         } else {
           // k-th visited key tile goes to warpgroup k & 1: S(0) first, then per
           // k: P V(k), S(k + 2) (same warpgroup, its S columns are free once
