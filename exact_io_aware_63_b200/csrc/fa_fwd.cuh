@@ -90,16 +90,24 @@ struct FwdCfg {
   static constexpr int kOffML = kOffV + kStages * kTileBytes;  // [2 warpgroups][128 rows] (m, l)
   static constexpr int kOffBar = kOffML + 2 * kTile * 8;
   // barriers: q_full[2], q_empty[2], k_full[S], k_empty[S], v_full[S], v_empty[S],
-  //           s_full[2], p_full[2], o_full[2], drain, ml_ready, merged
-  static constexpr int kNumBars = 4 + 4 * kStages + 6 + 3;
+  //           s_full[2], p_full[2], o_full[2], drain[2], ml_ready, merged, s_free[2],
+  //           p_free[2]
+  static constexpr int kNumBars = 18 + 4 * kStages;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16;
   static_assert(kSmemBytes <= 232448, "shared memory over the per-block limit");
   static constexpr uint32_t kTmemCols = 512;
   // pairs (of every 8) whose exponentials ex2_poly2 computes on interior tiles
   static constexpr int kPolyPer8 = (D == 64) ? 2 : 1;
+  // D = 64 leaves 128 TMEM columns after S_0, S_1, O_0, O_1: P gets its own
+  // 64 columns per warpgroup, so the next S can be issued as soon as the
+  // softmax has read the current one, and each warpgroup has its own MMA
+  // issuer.  D = 128 fills TMEM with S and O; P is then written over the first
+  // 64 columns of its S tile and one thread issues all MMAs.
+  static constexpr bool kSepP = (D == 64);
   __device__ static constexpr uint32_t col_s(int x) { return x ? 128u : 0u; }
   __device__ static constexpr uint32_t col_o(int x) { return x ? 256u + D : 256u; }
+  __device__ static constexpr uint32_t col_p(int x) { return kSepP ? 384u + 64u * x : col_s(x); }
 };
 
 // Work-unit order: heads are taken in groups whose K and V fit in a share of
@@ -194,10 +202,15 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
   auto p_full = [&](int x) { return bar0 + 8 * (6 + 4 * S + x); };
   auto o_full = [&](int x) { return bar0 + 8 * (8 + 4 * S + x); };
   const uint32_t drain_bar = bar0 + 8 * (10 + 4 * S);
+  auto drain = [&](int x) { return x ? bar0 + 8 * (17 + 4 * S) : drain_bar; };
   // split mode: the two softmax warpgroups meet twice per unit in the merge:
   // (m, l) published, and both partial outputs read (bounded waits, 256 arrivals)
   const uint32_t ml_ready = bar0 + 8 * (11 + 4 * S);
   const uint32_t merged = bar0 + 8 * (12 + 4 * S);
+  // separate-P layout: warpgroup x has read S_x (128 arrivals) / P V_x has read P_x
+  auto s_free = [&](int x) { return bar0 + 8 * (13 + 4 * S + x); };
+  auto p_free = [&](int x) { return bar0 + 8 * (15 + 4 * S + x); };
+  static_assert(Cfg::kNumBars == 18 + 4 * S, "barrier layout");
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kOffMisc + 4);
   float2* ml_smem = reinterpret_cast<float2*>(smem + Cfg::kOffML);  // [2][128] (m, l)
@@ -212,18 +225,23 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
   if (threadIdx.x == 0) {
     for (int x = 0; x < 2; ++x) {
       mbar_init(q_full(x), 1);
-      mbar_init(q_empty(x), 1);
+      // separate-P layout: both warpgroups' issuers arrive
+      mbar_init(q_empty(x), Cfg::kSepP ? 2 : 1);
       mbar_init(s_full(x), 1);
       mbar_init(p_full(x), 128);
       mbar_init(o_full(x), 1);
+      mbar_init(s_free(x), 128);
+      mbar_init(p_free(x), 1);
     }
     for (int s = 0; s < S; ++s) {
       mbar_init(k_full(s), 1);
-      mbar_init(k_empty(s), 1);
+      // separate-P pair mode: both issuers arrive for every tile of the unit
+      mbar_init(k_empty(s), (Cfg::kSepP && kPair) ? 2 : 1);
       mbar_init(v_full(s), 1);
-      mbar_init(v_empty(s), 1);
+      mbar_init(v_empty(s), (Cfg::kSepP && kPair) ? 2 : 1);
     }
     mbar_init(drain_bar, 1);
+    mbar_init(drain(1), 1);
     mbar_init(ml_ready, 256);
     mbar_init(merged, 256);
     *abort_flag = 0;
@@ -287,8 +305,8 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
       if (!ok) *abort_flag = 1;
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 && !Cfg::kSepP) {
+    // ------------------------------------------------- MMA issuer (D = 128)
     setmaxnreg_dec<Cfg::kRegsLow>();
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
@@ -479,6 +497,178 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
       mbar_wait(drain_bar, 0);
     }
     __syncwarp();
+  } else if (Cfg::kSepP && (warp == 1 || warp == 2)) {
+    // -------------------------- MMA issuers, one per softmax warpgroup (D = 64)
+    setmaxnreg_dec<Cfg::kRegsLow>();
+    if (lane == 0) {
+      const int x = warp - 1;  // the warpgroup this thread issues for
+      // pair mode with two Q slots: the warpgroup's first S of the next unit is
+      // issued right after its last S of this one, so its epilogue overlaps it
+      constexpr bool kLook = kPair && QSLOTS == 2;
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+      const uint64_t desc_q0 = sw128_desc(sbase + Cfg::kOffQ, 16, 1024);
+      const uint64_t desc_k0 = sw128_desc(sbase + Cfg::kOffK, 16, 1024);
+      const uint64_t desc_v0 = sw128_desc(sbase + Cfg::kOffV, 16384, 1024);
+      // S_x = Q (slot q) K^T, K from ring index c; the k_empty commit releases K
+      auto issue_s = [&](int q, uint32_t c) {
+        const int s = c % S;
+        const uint64_t dq = desc_q0 + ((q_tile(q, x) - (sbase + Cfg::kOffQ)) >> 4);
+        const uint64_t dk = desc_k0 + ((s * Cfg::kTileBytes) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+          umma_ss(tmem + Cfg::col_s(x), dq + off, dk + off, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(s_full(x));
+        umma_commit(k_empty(s));
+      };
+      // O_x (+)= P_x V, V from ring index c; p_free and v_empty release P_x and V
+      auto issue_pv = [&](uint32_t c, uint32_t acc) {
+        const int s = c % S;
+        const uint64_t dv = desc_v0 + ((s * Cfg::kTileBytes) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          umma_ts(tmem + Cfg::col_o(x), tmem + Cfg::col_p(x) + kk * 8, dv + ((kk * 2048) >> 4),
+                  idesc_pv, (kk > 0 || acc) ? 1u : 0u);
+        umma_commit(p_free(x));
+        umma_commit(v_empty(s));
+      };
+      auto mark = [&](const FwdUnit& wu, int j) {
+        if (p.visited) p.visited[((size_t)wu.bh * p.n_t + (x ? wu.i1 : wu.i0)) * p.n_t + j] = 1;
+      };
+      // Own visits of a unit.  Pair mode: key tiles 0 .. je - 1, ring index =
+      // unit base + tile.  Split mode: visits k = x, x + 2, ... of the unit's
+      // visited key tiles, ring index = unit base + k.  nvis counts the unit's
+      // visits (both warpgroups) seen so far; after the last own visit it is
+      // the unit's total.
+      auto own_first = [&](const FwdUnit& wu, int& j, int& nvis) {
+        if constexpr (kPair) {
+          j = 0;
+          nvis = 0;
+        } else {
+          j = fwd_next(p, wu, 0);
+          nvis = (j < wu.j_end) ? 1 : 0;
+          if (x == 1 && j < wu.j_end) {
+            j = fwd_next(p, wu, j + 1);
+            nvis += (j < wu.j_end) ? 1 : 0;
+          }
+        }
+      };
+      auto own_next = [&](const FwdUnit& wu, int j, int& nvis) -> int {
+        if constexpr (kPair) {
+          return j + 1;
+        } else {
+          const int j1 = fwd_next(p, wu, j + 1);  // the other warpgroup's visit
+          if (j1 >= wu.j_end) return wu.j_end;
+          ++nvis;
+          const int j2 = fwd_next(p, wu, j1 + 1);
+          if (j2 < wu.j_end) ++nvis;
+          return j2;
+        }
+      };
+      uint32_t q_cnt = 0, kv_cnt = 0;  // units started; ring index of the unit's first tile
+      uint32_t t_cnt = 0;              // tiles of this warpgroup (s_free / p_full phases)
+      bool pre = false;                // this unit's Q awaited and first own S issued
+      bool ok = true;
+      for (int round = 0; ok; ++round) {
+        const int u = unit_for_round(round, blockIdx.x, G);
+        if (u >= p.num_units) break;
+        const FwdUnit w = fwd_decode<kPair>(p, u);
+        const int qs = q_cnt % QSLOTS;
+        const uint32_t q_par = (q_cnt / QSLOTS) & 1;
+        ++q_cnt;
+        const int je = kPair ? (x ? w.j_end1 : w.j_end0) : w.j_end;  // own visits lie below je
+        int nvis = 0, j = 0;
+        own_first(w, j, nvis);
+        bool pre_next = false;
+        // Q is awaited even without an own visit, so that the q_empty arrival
+        // cannot complete the slot's previous phase
+        if (!pre) ok = mbar_wait(q_full(qs), q_par);
+        if (ok && j < je && !pre) {
+          const uint32_t c = kv_cnt + (kPair ? j : x);
+          ok = mbar_wait(k_full(c % S), (c / S) & 1);
+          if (ok) {
+            tc_fence_after();
+            issue_s(qs, c);
+            mark(w, j);
+          }
+        }
+        if (ok && j >= je) umma_commit(q_empty(qs));  // no own visit: done with Q
+        if (!ok) break;
+        int cnt = 0;
+        while (j < je) {
+          const uint32_t c = kv_cnt + (kPair ? j : x + 2 * cnt);
+          const int j2 = own_next(w, j, nvis);
+          const uint32_t c2 = kv_cnt + (kPair ? j2 : x + 2 * (cnt + 1));
+          // the warpgroup has S(j) in registers: the next S
+          ok = mbar_wait(s_free(x), t_cnt & 1);
+          if (!ok) break;
+          if (j2 < je) {
+            ok = mbar_wait(k_full(c2 % S), (c2 / S) & 1);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(qs, c2);
+            mark(w, j2);
+          } else {
+            umma_commit(q_empty(qs));  // this warpgroup's last S on this Q is issued
+            if constexpr (kLook) {
+              const int un = unit_for_round(round + 1, blockIdx.x, G);
+              if (un < p.num_units) {
+                const FwdUnit wn = fwd_decode<kPair>(p, un);
+                if ((x ? wn.j_end1 : wn.j_end0) > 0) {
+                  const int qsn = q_cnt % QSLOTS;
+                  const uint32_t cn = kv_cnt + w.j_end;
+                  ok = mbar_wait(q_full(qsn), (q_cnt / QSLOTS) & 1) &&
+                       mbar_wait(k_full(cn % S), (cn / S) & 1);
+                  if (!ok) break;
+                  tc_fence_after();
+                  issue_s(qsn, cn);
+                  mark(wn, 0);
+                  pre_next = true;
+                }
+              }
+            }
+          }
+          // P(j) is in TMEM: O += P V
+          ok = mbar_wait(p_full(x), t_cnt & 1) && mbar_wait(v_full(c % S), (c / S) & 1);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(c, cnt > 0 ? 1u : 0u);
+          if (j2 >= je) umma_commit(o_full(x));
+          ++t_cnt;
+          ++cnt;
+          j = j2;
+          if (*abort_flag) {
+            ok = false;
+            break;
+          }
+        }
+        if (!ok) break;
+        // pair mode: the unit's key tiles this warpgroup does not read (the last
+        // one of the even query tile under a causal mask; all of them for a
+        // missing odd tile): arrive for them on the ring, each after its load
+        // has landed, so that the arrival counts for this use of the stage
+        if constexpr (kPair) {
+          for (int jj = je; jj < w.j_end && ok; ++jj) {
+            const uint32_t cc = kv_cnt + jj;
+            ok = mbar_wait(k_full(cc % S), (cc / S) & 1) && mbar_wait(v_full(cc % S), (cc / S) & 1);
+            if (ok) {
+              umma_commit(k_empty(cc % S));
+              umma_commit(v_empty(cc % S));
+            }
+          }
+          if (!ok) break;
+        }
+        kv_cnt += kPair ? w.j_end : nvis;
+        pre = pre_next;
+      }
+      if (!ok) *abort_flag = 1;
+      // all issued MMAs complete before TMEM is released
+      umma_commit(drain(x));
+      mbar_wait(drain(x), 0);
+    }
+    __syncwarp();
   } else if (warp < 4) {
     setmaxnreg_dec<Cfg::kRegsLow>();  // idle warps of the first warpgroup
   } else {
@@ -491,6 +681,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
     const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
     const uint32_t tS = t_lane + Cfg::col_s(x);
     const uint32_t tO = t_lane + Cfg::col_o(x);
+    const uint32_t tP = t_lane + Cfg::col_p(x);
     uint32_t s_cnt = 0, unit_cnt = 0;
     uint32_t o_cnt[2] = {0, 0};
     bool ok = true;
@@ -525,6 +716,11 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 32; ++e) sv[c * 32 + e] = __uint_as_float(r[c][e]);
           }
+        }
+        if constexpr (Cfg::kSepP) {
+          // S_x is in registers: the issuer may overwrite it with the next S
+          tc_fence_before();
+          mbar_arrive(s_free(x));
         }
         // element masks on boundary tiles only
         const bool diag = p.causal && (j == i_me);
@@ -585,9 +781,18 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
               ls4[e & 3] = f2_add(ls4[e & 3], f2_pack(p0, p1));
               pk[e] = pack_bf16x2(p0, p1);
             }
-            tmem_st16(tS + c * 16, pk);
+            tmem_st16(tP + c * 16, pk);
           }
         };
+        if constexpr (Cfg::kSepP) {
+          // P_x is overwritten below: the previous P V of this warpgroup must
+          // have read it (and finished its O update before any rescale of O)
+          if (s_cnt >= 2) {
+            ok = __all_sync(0xffffffffu, mbar_wait(p_free(x), (s_cnt - 2) & 1));
+            if (!ok) break;
+          }
+          tc_fence_after();
+        }
         if (boundary)
           make_p(std::false_type{});
         else
