@@ -17,7 +17,8 @@
 //   warp 0      TMA producer: K_j, V_j once per unit; per visited query tile
 //               Q_i with the tile's LSE*log2(e) and D rows (one ring) and
 //               dO_i (a second ring)
-//   warp 1      MMA issuer (one thread), TMEM owner
+//   warp 1      TMEM owner; MMA issuer (one thread).  D = 64: warps 1-3 each
+//               issue one share of the MMAs (S^T and dV / dP^T and dK / dQ)
 //   warps 4-11  two "dS" warpgroups, one key row per thread (TMEM lane), each
 //               on half of the 128 query columns: P^T, dS^T, and the dK (first
 //               warpgroup) / dV (second) epilogue of each unit
@@ -154,8 +155,8 @@ struct BwdCfg {
   static constexpr int kRowBytes = kTile * 4;
   static constexpr int kOffBar = kOffRow + 2 * kQStages * kRowBytes;
   // kv_full, kv_empty, q_full[QS], q_empty[QS], do_full[DS], do_empty[DS], s_full,
-  // dp_full, p_full, ds_full, ds_smem_empty, dq_full, dq_empty, dkv_full, drain
-  static constexpr int kNumBars = 2 + 2 * kQStages + 2 * kDoStages + 9;
+  // dp_full, p_full, ds_full, ds_smem_empty, dq_full, dq_empty, dkv_full, drain[3]
+  static constexpr int kNumBars = 2 + 2 * kQStages + 2 * kDoStages + 11;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16;
   static_assert(kSmemBytes <= 232448, "shared memory over the per-block limit");
@@ -172,6 +173,10 @@ struct BwdCfg {
   // (after the dK MMA has read dS^T there; the next dP^T waits for the drain)
   static constexpr uint32_t kColDQ = (D == 64) ? 384 : 128;
   static constexpr bool kDqAliasesDP = (kColDQ == kColDP);
+  // With dQ in its own columns the MMAs split into three independent issue
+  // streams (warps 1-3): one issuing thread beside twelve busy math warps is
+  // starved of issue slots.  D = 128 (dQ over dP^T) keeps one issuer.
+  static constexpr bool kMultiIssue = !kDqAliasesDP;
   // dQ staging: each dQ warp owns 8 KB = two 32 x 32 float32 boxes
   static constexpr int kDqBoxesPerRound = 2;
   static constexpr int kDqRounds = D / 64;
@@ -240,6 +245,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
   const uint32_t dp_full = s_full + 8, p_full = s_full + 16, ds_full = s_full + 24;
   const uint32_t ds_smem_empty = s_full + 32, dq_full = s_full + 40, dq_empty = s_full + 48;
   const uint32_t dkv_full = s_full + 56, drain_bar = s_full + 64;
+  auto drain = [&](int r) { return drain_bar + 8 * r; };
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kOffMisc + 4);
   auto lse2_smem = [&](int s) {
@@ -254,14 +260,16 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
-    mbar_init(kv_empty, 1);
+    // three issuers: K and V are read by all three, Q and dO by two each
+    constexpr uint32_t kIssuers = Cfg::kMultiIssue ? 3 : 1;
+    mbar_init(kv_empty, kIssuers);
     for (int s = 0; s < QS; ++s) {
       mbar_init(q_full(s), 1);
-      mbar_init(q_empty(s), 1);
+      mbar_init(q_empty(s), Cfg::kMultiIssue ? 2 : 1);
     }
     for (int s = 0; s < DOS; ++s) {
       mbar_init(do_full(s), 1);
-      mbar_init(do_empty(s), 1);
+      mbar_init(do_empty(s), Cfg::kMultiIssue ? 2 : 1);
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
@@ -270,8 +278,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     mbar_init(ds_smem_empty, 1);
     mbar_init(dq_full, 1);
     mbar_init(dq_empty, 128);
-    mbar_init(dkv_full, 1);
-    mbar_init(drain_bar, 1);
+    mbar_init(dkv_full, Cfg::kMultiIssue ? 2 : 1);  // dV and dK issuers
+    for (int r = 0; r < 3; ++r) mbar_init(drain(r), 1);
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tmap(&tm_q);
@@ -341,8 +349,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       if (!ok) *abort_flag = 1;
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 && !Cfg::kMultiIssue) {
+    // ------------------------------------------------- MMA issuer (D = 128)
     setmaxnreg_dec<Cfg::kRegsLow>();
     if (lane == 0) {
       constexpr uint32_t idesc_kk = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T
@@ -472,6 +480,145 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       if (!ok) *abort_flag = 1;
       umma_commit(drain_bar);
       mbar_wait(drain_bar, 0);
+    }
+    __syncwarp();
+  } else if (Cfg::kMultiIssue && warp <= 3) {
+    // ------------------------------- MMA issuers, three warps (D = 64)
+    // role 0: S^T and dV (the P^T columns); role 1: dP^T and dK (the dS^T
+    // columns); role 2: dQ (its own columns).  Each role keeps its TMEM
+    // columns' read-before-overwrite order in its own issue order; what one
+    // role needs from another comes through the math groups' barriers.
+    setmaxnreg_dec<Cfg::kRegsLow>();
+    if (lane == 0) {
+      const int role = warp - 1;
+      constexpr uint32_t idesc_kk = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T
+      constexpr uint32_t idesc_tn = idesc_bf16_f32(128, D, 0, 1);    // dV, dK (A in TMEM)
+      constexpr uint32_t idesc_dq = idesc_bf16_f32(128, D, 1, 1);    // dQ (both MN-major)
+      const uint64_t dk_k = sw128_desc(sbase + Cfg::kOffK, 16, 1024);     // K_j, K-major
+      const uint64_t dv_k = sw128_desc(sbase + Cfg::kOffV, 16, 1024);     // V_j, K-major
+      const uint64_t dq_k0 = sw128_desc(sbase + Cfg::kOffQ, 16, 1024);    // Q_i, K-major
+      const uint64_t ddo_k0 = sw128_desc(sbase + Cfg::kOffDO, 16, 1024);  // dO_i, K-major
+      const uint64_t dq_m0 = sw128_desc(sbase + Cfg::kOffQ, 16384, 1024);    // Q_i, MN-major
+      const uint64_t ddo_m0 = sw128_desc(sbase + Cfg::kOffDO, 16384, 1024);  // dO_i, MN-major
+      const uint64_t dk_m = sw128_desc(sbase + Cfg::kOffK, 16384, 1024);     // K_j, MN-major
+      const uint64_t dds_m = sw128_desc(sbase + Cfg::kOffDS, 16384, 1024);   // dS, MN-major
+      uint32_t kv_cnt = 0, q_cnt = 0, do_cnt = 0, p_cnt = 0, ds_cnt = 0;
+      uint32_t dq_cnt = 0;  // role 2: dQ MMAs issued (= dq_empty phases to await)
+      bool ok = true;
+      // role 0: S^T = K_j Q_i^T for the Q tile of ring index c; Q is released
+      // for this role as soon as the MMA has read it
+      auto issue_st = [&](uint32_t c, const BwdUnit& w, int i) -> bool {
+        const int sq = c % QS;
+        if (!mbar_wait(q_full(sq), (c / QS) & 1)) return false;
+        tc_fence_after();
+        const uint32_t q_off = (sq * Cfg::kTileBytes) >> 4;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+          umma_ss(tmem + Cfg::kColS, dk_k + off, dq_k0 + q_off + off, idesc_kk, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(s_full);
+        umma_commit(q_empty(sq));
+        if (p.visited) p.visited[((size_t)w.bh * p.n_t + i) * p.n_t + w.j] = 1;
+        return true;
+      };
+      // role 1: dP^T = V_j dO_i^T for the dO tile of ring index c; dO is
+      // released for this role as soon as the MMA has read it
+      auto issue_dpt = [&](uint32_t c) -> bool {
+        const int so = c % DOS;
+        if (!mbar_wait(do_full(so), (c / DOS) & 1)) return false;
+        tc_fence_after();
+        const uint32_t do_off = (so * Cfg::kTileBytes) >> 4;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+          umma_ss(tmem + Cfg::kColDP, dv_k + off, ddo_k0 + do_off + off, idesc_kk,
+                  kk > 0 ? 1u : 0u);
+        }
+        umma_commit(dp_full);
+        umma_commit(do_empty(so));
+        return true;
+      };
+      for (int round = 0; ok; ++round) {
+        const int u = unit_for_round(round, blockIdx.x, G);
+        if (u >= p.num_units) break;
+        const BwdUnit w = bwd_decode(p, u);
+        if (!w.any) continue;
+        ok = mbar_wait(kv_full, kv_cnt & 1);
+        ++kv_cnt;
+        if (!ok) break;
+        int i = bwd_next(p, w, w.i_begin);
+        if (role == 0) ok = issue_st(q_cnt, w, i);
+        if (role == 1) ok = issue_dpt(do_cnt);
+        for (int t = 0; ok && i < p.n_t; ++t) {
+          const int inext = bwd_next(p, w, i + 1);
+          const int sq = q_cnt % QS, so = do_cnt % DOS;
+          if (role == 0) {
+            // dV += P^T dO_i, once P^T is in TMEM (dO_i was awaited by role 1
+            // for dP^T; awaited here too, since the roles run independently)
+            ok = mbar_wait(p_full, p_cnt & 1) && mbar_wait(do_full(so), (do_cnt / DOS) & 1);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t do_off = (so * Cfg::kTileBytes) >> 4;
+#pragma unroll
+            for (int kk = 0; kk < kTile / 16; ++kk)
+              umma_ts(tmem + Cfg::kColDV, tmem + Cfg::packed_col(Cfg::kColS, kk),
+                      ddo_m0 + do_off + ((kk * 2048) >> 4), idesc_tn,
+                      (t > 0 || kk > 0) ? 1u : 0u);
+            umma_commit(do_empty(so));
+            // S^T(t+1) over P^T(t): after dV(t) (issue order) and after the
+            // math groups are done with P(t) (ds_full)
+            ok = mbar_wait(ds_full, ds_cnt & 1);
+            if (!ok) break;
+            if (inext < p.n_t) {
+              ok = issue_st(q_cnt + 1, w, inext);
+              if (!ok) break;
+            }
+          } else if (role == 1) {
+            // dK += dS^T Q_i, then dP^T(t+1) over dS^T(t) (issue order)
+            ok = mbar_wait(ds_full, ds_cnt & 1) && mbar_wait(q_full(sq), (q_cnt / QS) & 1);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t q_off = (sq * Cfg::kTileBytes) >> 4;
+#pragma unroll
+            for (int kk = 0; kk < kTile / 16; ++kk)
+              umma_ts(tmem + Cfg::kColDK, tmem + Cfg::packed_col(Cfg::kColDP, kk),
+                      dq_m0 + q_off + ((kk * 2048) >> 4), idesc_tn,
+                      (t > 0 || kk > 0) ? 1u : 0u);
+            umma_commit(q_empty(sq));
+            if (inext < p.n_t) {
+              ok = issue_dpt(do_cnt + 1);
+              if (!ok) break;
+            }
+          } else {
+            // dQ = dS K_j once dS is in shared memory and the previous dQ has
+            // been drained from its columns
+            ok = mbar_wait(ds_full, ds_cnt & 1);
+            if (ok && dq_cnt > 0) ok = mbar_wait(dq_empty, (dq_cnt - 1) & 1);
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < kTile / 16; ++kk)
+              umma_ss(tmem + Cfg::kColDQ, dds_m + ((kk * 2048) >> 4), dk_m + ((kk * 2048) >> 4),
+                      idesc_dq, kk > 0 ? 1u : 0u);
+            umma_commit(dq_full);
+            umma_commit(ds_smem_empty);
+            ++dq_cnt;
+          }
+          ++p_cnt;
+          ++ds_cnt;
+          ++q_cnt;
+          ++do_cnt;
+          i = inext;
+          if (*abort_flag) ok = false;
+        }
+        if (!ok) break;
+        umma_commit(kv_empty);
+        if (role < 2) umma_commit(dkv_full);
+      }
+      if (!ok) *abort_flag = 1;
+      umma_commit(drain(role));
+      mbar_wait(drain(role), 0);
     }
     __syncwarp();
   } else if (warp < 4) {
