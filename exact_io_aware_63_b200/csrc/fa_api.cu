@@ -187,9 +187,10 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
   float* delta = reinterpret_cast<float*>(ws + wl.delta);
   float* lse2 = reinterpret_cast<float*>(ws + wl.lse2);
   float* dq_acc = reinterpret_cast<float*>(ws + wl.dq_acc);
-  CUtensorMap tq, tk, tv, tdo, tdq;
+  CUtensorMap tq, tk, tv, tdo, tdq, tdk, tdv;
   if (!make_tmap(&tq, q, rows, D) || !make_tmap(&tk, k, rows, D) || !make_tmap(&tv, v, rows, D) ||
-      !make_tmap(&tdo, dout, rows, D) || !make_tmap_f32_acc(&tdq, dq_acc, rows, D))
+      !make_tmap(&tdo, dout, rows, D) || !make_tmap_f32_acc(&tdq, dq_acc, rows, D) ||
+      !make_tmap(&tdk, dk, rows, D) || !make_tmap(&tdv, dv, rows, D))
     return FA_ERR_CUDA;
   static bool smem_set = false;
   if (!smem_set) {
@@ -227,7 +228,8 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
     p.scale = scale;
     p.scale_log2 = scale * fa::kLog2e;
     const int grid = p.num_units < num_sms ? p.num_units : num_sms;
-    fa::fa_bwd_kernel<D><<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdq, p);
+    fa::fa_bwd_kernel<D>
+        <<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdq, tdk, tdv, p);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   // dQ

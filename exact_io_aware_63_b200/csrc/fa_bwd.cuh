@@ -139,11 +139,17 @@ struct BwdCfg {
   static constexpr int kBoxes = D / 64;
   // Q_i (with the tile's -LSE2 and -D rows) and dO_i come through separate
   // rings: dO_i is released after the dV MMA, Q_i after the dK MMA.
-  static constexpr int kQStages = (D == 64) ? 3 : 2;
-  static constexpr int kDoStages = (D == 64) ? 3 : 1;
+  // D = 64: K/V double-buffered across units (the next unit's K and V load
+  // while this one runs), two-stage Q and dO rings.  D = 128: one K/V buffer.
+  static constexpr bool kSmallD = (D == 64);
+  static constexpr int kKvStages = kSmallD ? 2 : 1;
+  static constexpr int kQStages = 2;
+  static constexpr int kDoStages = kSmallD ? 2 : 1;
+  // K/V slot s: K at kOffK + s * kKvSlotBytes, V right after it
+  static constexpr int kKvSlotBytes = 2 * kTileBytes;
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kOffK + kTileBytes;
-  static constexpr int kOffQ = kOffV + kTileBytes;
+  static constexpr int kOffQ = kOffK + kKvStages * kKvSlotBytes;
   static constexpr int kOffDO = kOffQ + kQStages * kTileBytes;
   // 128 x 128 bf16 dS tile: A operand of the dQ MMA
   static constexpr int kOffDS = kOffDO + kDoStages * kTileBytes;
@@ -151,12 +157,25 @@ struct BwdCfg {
   static constexpr int kOffDQ = kOffDS + kTile * kTile * 2;
   static constexpr int kDqStageBytes = 4 * 8192;
   // per Q stage: -LSE*log2(e) and -D of the stage's 128 query rows
-  static constexpr int kOffRow = kOffDQ + kDqStageBytes;
+  // D = 64: the dK and dV tiles of a unit are staged here (128-byte swizzled
+  // rows, the TMA box layout; 1024-byte aligned like every tile) and written
+  // with one TMA store each; D = 128 has no room and stores rows directly
+  static constexpr bool kEpiTma = kSmallD;
+  static constexpr int kOffEpi = kOffDQ + kDqStageBytes;
+  static constexpr int kEpiBytes = kEpiTma ? 2 * kTileBytes : 0;
+  static constexpr int kOffRow = kOffEpi + kEpiBytes;
   static constexpr int kRowBytes = kTile * 4;
-  static constexpr int kOffBar = kOffRow + 2 * kQStages * kRowBytes;
-  // kv_full, kv_empty, q_full[QS], q_empty[QS], do_full[DS], do_empty[DS], s_full,
-  // dp_full, p_full, ds_full, ds_smem_empty, dq_full, dq_empty, dkv_full, drain[3]
-  static constexpr int kNumBars = 2 + 2 * kQStages + 2 * kDoStages + 11;
+  // unit records: the producer decodes each work unit once and publishes it
+  // here (kUnitRing slots of two int4) for the other roles
+  static constexpr int kUnitRing = 4;
+  static constexpr int kOffUnit = kOffRow + 2 * kQStages * kRowBytes;
+  static constexpr int kOffBar = kOffUnit + kUnitRing * 32;
+  static_assert(kOffEpi % 1024 == 0, "staging tiles must be 1024-byte aligned");
+  // kv_full[KVS], kv_empty[KVS], q_full[QS], q_empty[QS], do_full[DS], do_empty[DS],
+  // s_full, dp_full, p_full, ds_full, ds_smem_empty, dq_full, dq_empty, dkv_full,
+  // drain[3], s_free, p_free, unit_full[UR], unit_empty[UR], epi_ready[2]
+  static constexpr int kNumBars =
+      2 * kKvStages + 2 * kQStages + 2 * kDoStages + 15 + 2 * kUnitRing;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16;
   static_assert(kSmemBytes <= 232448, "shared memory over the per-block limit");
@@ -186,10 +205,18 @@ struct BwdCfg {
   __device__ static constexpr uint32_t packed_col(uint32_t base, int kk) {
     return base + (kk >> 2) * 64 + (kk & 3) * 8;
   }
+  // P^T: D = 64 keeps it in the last 64 columns (32 per warpgroup half), so
+  // that the next S^T may be issued once S^T is in the math warps' registers;
+  // D = 128 writes it over S^T as described above
+  static constexpr uint32_t kColP = kSmallD ? 448 : kColS;
+  static constexpr uint32_t kPHalf = kSmallD ? 32 : 64;  // columns between the halves' P^T
+  __device__ static constexpr uint32_t p_col(int kk) {
+    return kColP + (kk >> 2) * kPHalf + (kk & 3) * 8;
+  }
 };
 
 struct BwdUnit {
-  int bh, b, j, L, i_begin, any;
+  int bh, b, j, L, i_begin, any, i_first;  // i_first: first visited query tile
 };
 
 __device__ __forceinline__ bool bwd_tile_on(const BwdParams& p, const BwdUnit& w, int i) {
@@ -220,7 +247,8 @@ __device__ __forceinline__ BwdUnit bwd_decode(const BwdParams& p, int u) {
   }
   w.L = L;
   w.i_begin = p.causal ? w.j : 0;
-  w.any = bwd_next(p, w, w.i_begin) < p.n_t;
+  w.i_first = bwd_next(p, w, w.i_begin);
+  w.any = w.i_first < p.n_t;
   return w;
 }
 
@@ -229,23 +257,66 @@ template <int D>
 __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                  const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
+                  const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ CUtensorMap tm_dk,
+                  const __grid_constant__ CUtensorMap tm_dv, const BwdParams p) {
   using Cfg = BwdCfg<D>;
-  constexpr int QS = Cfg::kQStages, DOS = Cfg::kDoStages;
+  constexpr int QS = Cfg::kQStages, DOS = Cfg::kDoStages, KVS = Cfg::kKvStages;
   extern __shared__ __align__(1024) uint8_t smem[];
   if (!smem_aligned_1024(smem)) return;
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + Cfg::kOffBar;
-  const uint32_t kv_full = bar0, kv_empty = bar0 + 8;
-  auto q_full = [&](int s) { return bar0 + 8 * (2 + s); };
-  auto q_empty = [&](int s) { return bar0 + 8 * (2 + QS + s); };
-  auto do_full = [&](int s) { return bar0 + 8 * (2 + 2 * QS + s); };
-  auto do_empty = [&](int s) { return bar0 + 8 * (2 + 2 * QS + DOS + s); };
-  const uint32_t s_full = bar0 + 8 * (2 + 2 * QS + 2 * DOS);
+  auto kv_full = [&](int s) { return bar0 + 8 * s; };
+  auto kv_empty = [&](int s) { return bar0 + 8 * (KVS + s); };
+  const uint32_t bar1 = bar0 + 8 * 2 * KVS;
+  auto q_full = [&](int s) { return bar1 + 8 * s; };
+  auto q_empty = [&](int s) { return bar1 + 8 * (QS + s); };
+  auto do_full = [&](int s) { return bar1 + 8 * (2 * QS + s); };
+  auto do_empty = [&](int s) { return bar1 + 8 * (2 * QS + DOS + s); };
+  const uint32_t s_full = bar1 + 8 * (2 * QS + 2 * DOS);
   const uint32_t dp_full = s_full + 8, p_full = s_full + 16, ds_full = s_full + 24;
   const uint32_t ds_smem_empty = s_full + 32, dq_full = s_full + 40, dq_empty = s_full + 48;
   const uint32_t dkv_full = s_full + 56, drain_bar = s_full + 64;
   auto drain = [&](int r) { return drain_bar + 8 * r; };
+  // D = 64: the math groups have S^T in registers (256 arrivals) / dV has read P^T
+  const uint32_t s_free = drain_bar + 24, p_free = drain_bar + 32;
+  constexpr int UR = Cfg::kUnitRing;
+  auto unit_full = [&](int s) { return drain_bar + 40 + 8 * s; };
+  auto unit_empty = [&](int s) { return drain_bar + 40 + 8 * (UR + s); };
+  // D = 64 epilogue: all 128 rows of warpgroup h's dK / dV tile are staged
+  auto epi_ready = [&](int h) { return drain_bar + 40 + 8 * (2 * UR + h); };
+  static_assert((2 * KVS + 2 * QS + 2 * DOS + 15 + 2 * UR) == Cfg::kNumBars, "barrier layout");
+  int4* unit_rec = reinterpret_cast<int4*>(smem + Cfg::kOffUnit);  // [UR][2]
+  // the warps that read each unit record: the MMA issuer(s), 8 dS and 4 dQ warps
+  constexpr uint32_t kUnitReaders = (Cfg::kMultiIssue ? 3 : 1) + 12;
+  auto load_unit = [&](int s) {
+    const int4 a = unit_rec[2 * s], b = unit_rec[2 * s + 1];
+    BwdUnit w;
+    w.bh = a.x;
+    w.b = a.y;
+    w.j = a.z;
+    w.L = a.w;
+    w.i_begin = b.x;
+    w.any = b.y;
+    w.i_first = b.z;
+    return w;
+  };
+  // one thread's read of round r's unit record (it releases the slot)
+  auto fetch_one = [&](int r, BwdUnit& w) -> bool {
+    const int s = r % UR;
+    if (!mbar_wait(unit_full(s), (r / UR) & 1)) return false;
+    w = load_unit(s);
+    mbar_arrive(unit_empty(s));
+    return true;
+  };
+  // a whole warp's read (all 32 lanes; lane 0 releases the slot)
+  auto fetch_warp = [&](int r, BwdUnit& w) -> bool {
+    const int s = r % UR;
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(unit_full(s), (r / UR) & 1));
+    if (ok) w = load_unit(s);
+    __syncwarp();
+    if (ok && lane_id() == 0) mbar_arrive(unit_empty(s));
+    return ok;
+  };
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kOffMisc + 4);
   auto lse2_smem = [&](int s) {
@@ -259,10 +330,12 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
   const int lane = lane_id();
 
   if (threadIdx.x == 0) {
-    mbar_init(kv_full, 1);
     // three issuers: K and V are read by all three, Q and dO by two each
     constexpr uint32_t kIssuers = Cfg::kMultiIssue ? 3 : 1;
-    mbar_init(kv_empty, kIssuers);
+    for (int s = 0; s < KVS; ++s) {
+      mbar_init(kv_full(s), 1);
+      mbar_init(kv_empty(s), kIssuers);
+    }
     for (int s = 0; s < QS; ++s) {
       mbar_init(q_full(s), 1);
       mbar_init(q_empty(s), Cfg::kMultiIssue ? 2 : 1);
@@ -280,6 +353,14 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     mbar_init(dq_empty, 128);
     mbar_init(dkv_full, Cfg::kMultiIssue ? 2 : 1);  // dV and dK issuers
     for (int r = 0; r < 3; ++r) mbar_init(drain(r), 1);
+    mbar_init(s_free, 256);
+    mbar_init(p_free, 1);
+    for (int s = 0; s < UR; ++s) {
+      mbar_init(unit_full(s), 1);
+      mbar_init(unit_empty(s), kUnitReaders);
+    }
+    mbar_init(epi_ready(0), 128);
+    mbar_init(epi_ready(1), 128);
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tmap(&tm_q);
@@ -287,6 +368,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     prefetch_tmap(&tm_v);
     prefetch_tmap(&tm_do);
     prefetch_tmap(&tm_dq);
+    if (Cfg::kEpiTma) {
+      prefetch_tmap(&tm_dk);
+      prefetch_tmap(&tm_dv);
+    }
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_base_slot), Cfg::kTmemCols);
@@ -307,21 +392,39 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     if (lane == 0) {
       uint32_t kv_cnt = 0, q_cnt = 0, do_cnt = 0;
       bool ok = true;
+      int published = 0;  // unit records written
       for (int round = 0; ok; ++round) {
         const int u = unit_for_round(round, blockIdx.x, G);
         if (u >= p.num_units) break;
-        const BwdUnit w = bwd_decode(p, u);
+        // publish this round's unit and the next one (the other roles read a
+        // unit's record before its first tile and the next one's at its last)
+        while (published <= round + 1) {
+          const int un = unit_for_round(published, blockIdx.x, G);
+          if (un >= p.num_units) break;
+          const BwdUnit wr = bwd_decode(p, un);
+          const int s = published % UR;
+          ok = mbar_wait(unit_empty(s), ((published / UR) & 1) ^ 1);
+          if (!ok) break;
+          unit_rec[2 * s] = make_int4(wr.bh, wr.b, wr.j, wr.L);
+          unit_rec[2 * s + 1] = make_int4(wr.i_begin, wr.any, wr.i_first, 0);
+          mbar_arrive(unit_full(s));
+          ++published;
+        }
+        if (!ok) break;
+        const BwdUnit w = load_unit(round % UR);
         if (!w.any) continue;
-        ok = mbar_wait(kv_empty, (kv_cnt & 1) ^ 1);
+        const int skv = kv_cnt % KVS;
+        ok = mbar_wait(kv_empty(skv), ((kv_cnt / KVS) & 1) ^ 1);
         if (!ok) break;
         ++kv_cnt;
         const int krow = w.bh * p.N + w.j * kTile;
-        mbar_arrive_expect_tx(kv_full, 2 * Cfg::kTileBytes);
+        const uint32_t kv_off = skv * Cfg::kKvSlotBytes;
+        mbar_arrive_expect_tx(kv_full(skv), 2 * Cfg::kTileBytes);
         for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
-          tma_load_2d(sbase + Cfg::kOffK + bx * 16384, &tm_k, bx * 64, krow, kv_full);
-          tma_load_2d(sbase + Cfg::kOffV + bx * 16384, &tm_v, bx * 64, krow, kv_full);
+          tma_load_2d(sbase + Cfg::kOffK + kv_off + bx * 16384, &tm_k, bx * 64, krow, kv_full(skv));
+          tma_load_2d(sbase + Cfg::kOffV + kv_off + bx * 16384, &tm_v, bx * 64, krow, kv_full(skv));
         }
-        for (int i = bwd_next(p, w, w.i_begin); i < p.n_t && ok; i = bwd_next(p, w, i + 1)) {
+        for (int i = w.i_first; i < p.n_t && ok; i = bwd_next(p, w, i + 1)) {
           const int qrow = w.bh * p.N + i * kTile;
           const int sq = q_cnt % QS;
           ok = mbar_wait(q_empty(sq), ((q_cnt / QS) & 1) ^ 1);
@@ -410,9 +513,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       for (int round = 0; ok; ++round) {
         const int u = unit_for_round(round, blockIdx.x, G);
         if (u >= p.num_units) break;
-        const BwdUnit w = bwd_decode(p, u);
+        BwdUnit w;
+        ok = fetch_one(round, w);
+        if (!ok) break;
         if (!w.any) continue;
-        ok = mbar_wait(kv_full, kv_cnt & 1);
+        ok = mbar_wait(kv_full(0), kv_cnt & 1);
         ++kv_cnt;
         if (!ok) break;
         // Per query tile t the issue order is
@@ -421,7 +526,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         // S^T's columns are free once dS(t) is ready (its P^T has been read by
         // the dV MMA and by the dS warps), and dP^T(t+1) follows dK(t), which
         // reads dS^T(t) from the dP^T columns.
-        int i = bwd_next(p, w, w.i_begin);
+        int i = w.i_first;
         ok = issue_st(q_cnt, w, i) && issue_dpt(do_cnt);
         for (int t = 0; ok && i < p.n_t; ++t) {
           const int inext = bwd_next(p, w, i + 1);
@@ -435,7 +540,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
-            umma_ts(tmem + Cfg::kColDV, tmem + Cfg::packed_col(Cfg::kColS, kk),
+            umma_ts(tmem + Cfg::kColDV, tmem + Cfg::p_col(kk),
                     ddo_m0 + do_off + ((kk * 2048) >> 4), idesc_tn,
                     (t > 0 || kk > 0) ? 1u : 0u);
           umma_commit(do_empty(so));
@@ -474,7 +579,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
           if (*abort_flag) ok = false;
         }
         if (!ok) break;
-        umma_commit(kv_empty);
+        umma_commit(kv_empty(0));
         umma_commit(dkv_full);
       }
       if (!ok) *abort_flag = 1;
@@ -484,99 +589,142 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     __syncwarp();
   } else if (Cfg::kMultiIssue && warp <= 3) {
     // ------------------------------- MMA issuers, three warps (D = 64)
-    // role 0: S^T and dV (the P^T columns); role 1: dP^T and dK (the dS^T
-    // columns); role 2: dQ (its own columns).  Each role keeps its TMEM
-    // columns' read-before-overwrite order in its own issue order; what one
-    // role needs from another comes through the math groups' barriers.
+    // role 0: S^T and dV; role 1: dP^T and dK; role 2: dQ.  Each role keeps
+    // the read-before-overwrite order of its own TMEM columns in its issue
+    // order; what it needs from the other roles comes through the math
+    // groups' barriers.  S^T(t+1) follows the math groups' read of S^T(t)
+    // (s_free) and dP^T(t+1) follows dK(t), also across the boundary to the
+    // next unit, whose K and V are already loaded in the other K/V slot.
     setmaxnreg_dec<Cfg::kRegsLow>();
     if (lane == 0) {
       const int role = warp - 1;
       constexpr uint32_t idesc_kk = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T
       constexpr uint32_t idesc_tn = idesc_bf16_f32(128, D, 0, 1);    // dV, dK (A in TMEM)
       constexpr uint32_t idesc_dq = idesc_bf16_f32(128, D, 1, 1);    // dQ (both MN-major)
-      const uint64_t dk_k = sw128_desc(sbase + Cfg::kOffK, 16, 1024);     // K_j, K-major
-      const uint64_t dv_k = sw128_desc(sbase + Cfg::kOffV, 16, 1024);     // V_j, K-major
+      const uint64_t dk_k0 = sw128_desc(sbase + Cfg::kOffK, 16, 1024);    // K_j, K-major
+      const uint64_t dv_k0 = sw128_desc(sbase + Cfg::kOffV, 16, 1024);    // V_j, K-major
       const uint64_t dq_k0 = sw128_desc(sbase + Cfg::kOffQ, 16, 1024);    // Q_i, K-major
       const uint64_t ddo_k0 = sw128_desc(sbase + Cfg::kOffDO, 16, 1024);  // dO_i, K-major
       const uint64_t dq_m0 = sw128_desc(sbase + Cfg::kOffQ, 16384, 1024);    // Q_i, MN-major
       const uint64_t ddo_m0 = sw128_desc(sbase + Cfg::kOffDO, 16384, 1024);  // dO_i, MN-major
-      const uint64_t dk_m = sw128_desc(sbase + Cfg::kOffK, 16384, 1024);     // K_j, MN-major
+      const uint64_t dk_m0 = sw128_desc(sbase + Cfg::kOffK, 16384, 1024);    // K_j, MN-major
       const uint64_t dds_m = sw128_desc(sbase + Cfg::kOffDS, 16384, 1024);   // dS, MN-major
-      uint32_t kv_cnt = 0, q_cnt = 0, do_cnt = 0, p_cnt = 0, ds_cnt = 0;
-      uint32_t dq_cnt = 0;  // role 2: dQ MMAs issued (= dq_empty phases to await)
+      uint32_t kv_cnt = 0, q_cnt = 0, do_cnt = 0, t_cnt = 0;  // t_cnt: tiles (barrier phases)
       bool ok = true;
-      // role 0: S^T = K_j Q_i^T for the Q tile of ring index c; Q is released
-      // for this role as soon as the MMA has read it
-      auto issue_st = [&](uint32_t c, const BwdUnit& w, int i) -> bool {
+      // role 0: S^T = K Q_i^T, K from K/V slot skv, Q of ring index c
+      auto issue_st = [&](uint32_t c, int skv, const BwdUnit& w, int i) -> bool {
         const int sq = c % QS;
         if (!mbar_wait(q_full(sq), (c / QS) & 1)) return false;
         tc_fence_after();
         const uint32_t q_off = (sq * Cfg::kTileBytes) >> 4;
+        const uint32_t k_off = (skv * Cfg::kKvSlotBytes) >> 4;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
-          umma_ss(tmem + Cfg::kColS, dk_k + off, dq_k0 + q_off + off, idesc_kk, kk > 0 ? 1u : 0u);
+          umma_ss(tmem + Cfg::kColS, dk_k0 + k_off + off, dq_k0 + q_off + off, idesc_kk,
+                  kk > 0 ? 1u : 0u);
         }
         umma_commit(s_full);
-        umma_commit(q_empty(sq));
+        umma_commit(q_empty(sq));  // this role's use of Q_i
         if (p.visited) p.visited[((size_t)w.bh * p.n_t + i) * p.n_t + w.j] = 1;
         return true;
       };
-      // role 1: dP^T = V_j dO_i^T for the dO tile of ring index c; dO is
-      // released for this role as soon as the MMA has read it
-      auto issue_dpt = [&](uint32_t c) -> bool {
+      // role 1: dP^T = V dO_i^T, V from K/V slot skv, dO of ring index c
+      auto issue_dpt = [&](uint32_t c, int skv) -> bool {
         const int so = c % DOS;
         if (!mbar_wait(do_full(so), (c / DOS) & 1)) return false;
         tc_fence_after();
         const uint32_t do_off = (so * Cfg::kTileBytes) >> 4;
+        const uint32_t v_off = (skv * Cfg::kKvSlotBytes) >> 4;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
-          umma_ss(tmem + Cfg::kColDP, dv_k + off, ddo_k0 + do_off + off, idesc_kk,
+          umma_ss(tmem + Cfg::kColDP, dv_k0 + v_off + off, ddo_k0 + do_off + off, idesc_kk,
                   kk > 0 ? 1u : 0u);
         }
         umma_commit(dp_full);
-        umma_commit(do_empty(so));
+        umma_commit(do_empty(so));  // this role's use of dO_i
         return true;
       };
+      bool pre = false;  // roles 0 / 1: this unit's first S^T / dP^T already issued
+      bool have_next = false;  // the next round's record was read at the look-ahead
+      BwdUnit w_next;
       for (int round = 0; ok; ++round) {
         const int u = unit_for_round(round, blockIdx.x, G);
         if (u >= p.num_units) break;
-        const BwdUnit w = bwd_decode(p, u);
+        BwdUnit w;
+        if (have_next) {
+          w = w_next;
+          have_next = false;
+        } else {
+          ok = fetch_one(round, w);
+          if (!ok) break;
+        }
         if (!w.any) continue;
-        ok = mbar_wait(kv_full, kv_cnt & 1);
+        const int skv = kv_cnt % KVS;
+        if (!pre) ok = mbar_wait(kv_full(skv), (kv_cnt / KVS) & 1);
         ++kv_cnt;
         if (!ok) break;
-        int i = bwd_next(p, w, w.i_begin);
-        if (role == 0) ok = issue_st(q_cnt, w, i);
-        if (role == 1) ok = issue_dpt(do_cnt);
+        const uint32_t k_off = (skv * Cfg::kKvSlotBytes) >> 4;
+        int i = w.i_first;
+        if (!pre) {
+          if (role == 0) ok = issue_st(q_cnt, skv, w, i);
+          if (role == 1) ok = issue_dpt(do_cnt, skv);
+          if (!ok) break;
+        }
+        bool pre_next = false;
+        // the first tile of the next unit, for the look-ahead at the last tile
+        auto next_unit_first = [&](BwdUnit& wn, int& in) -> bool {
+          const int un = unit_for_round(round + 1, blockIdx.x, G);
+          if (un >= p.num_units) return false;
+          if (!fetch_one(round + 1, w_next)) {
+            ok = false;
+            return false;
+          }
+          have_next = true;
+          wn = w_next;
+          if (!wn.any) return false;
+          in = wn.i_first;
+          if (!mbar_wait(kv_full(kv_cnt % KVS), (kv_cnt / KVS) & 1)) {
+            ok = false;
+            return false;
+          }
+          return true;
+        };
         for (int t = 0; ok && i < p.n_t; ++t) {
           const int inext = bwd_next(p, w, i + 1);
           const int sq = q_cnt % QS, so = do_cnt % DOS;
           if (role == 0) {
-            // dV += P^T dO_i, once P^T is in TMEM (dO_i was awaited by role 1
-            // for dP^T; awaited here too, since the roles run independently)
-            ok = mbar_wait(p_full, p_cnt & 1) && mbar_wait(do_full(so), (do_cnt / DOS) & 1);
+            // S^T(t+1) once the math groups hold S^T(t) in registers
+            ok = mbar_wait(s_free, t_cnt & 1);
+            if (!ok) break;
+            if (inext < p.n_t) {
+              ok = issue_st(q_cnt + 1, skv, w, inext);
+            } else {
+              BwdUnit wn;
+              int in;
+              if (next_unit_first(wn, in)) {
+                ok = issue_st(q_cnt + 1, kv_cnt % KVS, wn, in);
+                pre_next = true;
+              }
+            }
+            if (!ok) break;
+            // dV += P^T dO_i once P^T is in TMEM (dO_i awaited here as well:
+            // the roles run independently)
+            ok = mbar_wait(p_full, t_cnt & 1) && mbar_wait(do_full(so), (do_cnt / DOS) & 1);
             if (!ok) break;
             tc_fence_after();
             const uint32_t do_off = (so * Cfg::kTileBytes) >> 4;
 #pragma unroll
             for (int kk = 0; kk < kTile / 16; ++kk)
-              umma_ts(tmem + Cfg::kColDV, tmem + Cfg::packed_col(Cfg::kColS, kk),
+              umma_ts(tmem + Cfg::kColDV, tmem + Cfg::p_col(kk),
                       ddo_m0 + do_off + ((kk * 2048) >> 4), idesc_tn,
                       (t > 0 || kk > 0) ? 1u : 0u);
+            umma_commit(p_free);
             umma_commit(do_empty(so));
-            // S^T(t+1) over P^T(t): after dV(t) (issue order) and after the
-            // math groups are done with P(t) (ds_full)
-            ok = mbar_wait(ds_full, ds_cnt & 1);
-            if (!ok) break;
-            if (inext < p.n_t) {
-              ok = issue_st(q_cnt + 1, w, inext);
-              if (!ok) break;
-            }
           } else if (role == 1) {
             // dK += dS^T Q_i, then dP^T(t+1) over dS^T(t) (issue order)
-            ok = mbar_wait(ds_full, ds_cnt & 1) && mbar_wait(q_full(sq), (q_cnt / QS) & 1);
+            ok = mbar_wait(ds_full, t_cnt & 1) && mbar_wait(q_full(sq), (q_cnt / QS) & 1);
             if (!ok) break;
             tc_fence_after();
             const uint32_t q_off = (sq * Cfg::kTileBytes) >> 4;
@@ -587,34 +735,41 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
                       (t > 0 || kk > 0) ? 1u : 0u);
             umma_commit(q_empty(sq));
             if (inext < p.n_t) {
-              ok = issue_dpt(do_cnt + 1);
-              if (!ok) break;
+              ok = issue_dpt(do_cnt + 1, skv);
+            } else {
+              umma_commit(dkv_full);  // dK of the unit complete (with role 0's dV)
+              BwdUnit wn;
+              int in;
+              if (next_unit_first(wn, in)) {
+                ok = issue_dpt(do_cnt + 1, kv_cnt % KVS);
+                pre_next = true;
+              }
             }
+            if (!ok) break;
           } else {
-            // dQ = dS K_j once dS is in shared memory and the previous dQ has
+            // dQ = dS K once dS is in shared memory and the previous dQ has
             // been drained from its columns
-            ok = mbar_wait(ds_full, ds_cnt & 1);
-            if (ok && dq_cnt > 0) ok = mbar_wait(dq_empty, (dq_cnt - 1) & 1);
+            ok = mbar_wait(ds_full, t_cnt & 1);
+            if (ok && t_cnt > 0) ok = mbar_wait(dq_empty, (t_cnt - 1) & 1);
             if (!ok) break;
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < kTile / 16; ++kk)
-              umma_ss(tmem + Cfg::kColDQ, dds_m + ((kk * 2048) >> 4), dk_m + ((kk * 2048) >> 4),
-                      idesc_dq, kk > 0 ? 1u : 0u);
+              umma_ss(tmem + Cfg::kColDQ, dds_m + ((kk * 2048) >> 4),
+                      dk_m0 + k_off + ((kk * 2048) >> 4), idesc_dq, kk > 0 ? 1u : 0u);
             umma_commit(dq_full);
             umma_commit(ds_smem_empty);
-            ++dq_cnt;
           }
-          ++p_cnt;
-          ++ds_cnt;
+          ++t_cnt;
           ++q_cnt;
           ++do_cnt;
           i = inext;
           if (*abort_flag) ok = false;
         }
         if (!ok) break;
-        umma_commit(kv_empty);
-        if (role < 2) umma_commit(dkv_full);
+        if (role == 0) umma_commit(dkv_full);  // dV of the unit complete
+        umma_commit(kv_empty(skv));            // this role's use of the unit's K/V
+        pre = pre_next;
       }
       if (!ok) *abort_flag = 1;
       umma_commit(drain(role));
@@ -633,15 +788,18 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     const int quarter = warp & 3;
     const int kr = quarter * 32 + lane;  // key row within the tile
     const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
-    const uint32_t tS = t_lane + Cfg::kColS + h * 64;    // this half's S^T / P^T columns
+    const uint32_t tS = t_lane + Cfg::kColS + h * 64;    // this half's S^T columns
+    const uint32_t tP = t_lane + Cfg::kColP + h * Cfg::kPHalf;  // this half's P^T (bf16)
     const uint32_t tDP = t_lane + Cfg::kColDP + h * 64;  // this half's dP^T / dS^T columns
     uint8_t* ds_rowp = smem + Cfg::kOffDS + h * 16384 + kr * 128;
-    uint32_t s_cnt = 0, dp_cnt = 0, dsm_cnt = 0, dkv_cnt = 0, q_cnt = 0;
+    uint32_t s_cnt = 0, dp_cnt = 0, dsm_cnt = 0, dkv_cnt = 0, q_cnt = 0, epi_cnt = 0;
     bool ok = true;
     for (int round = 0; ok; ++round) {
       const int u = unit_for_round(round, blockIdx.x, G);
       if (u >= p.num_units) break;
-      const BwdUnit w = bwd_decode(p, u);
+      BwdUnit w;
+      ok = fetch_warp(round, w);
+      if (!ok) break;
       const int c_key = w.j * kTile + kr;  // key index within the head
       const size_t krow = (size_t)w.bh * p.N + c_key;
       // warpgroup 0 writes the dK row, warpgroup 1 the dV row
@@ -652,7 +810,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         continue;
       }
       const bool key_valid = c_key < w.L;
-      for (int i = bwd_next(p, w, w.i_begin); i < p.n_t; i = bwd_next(p, w, i + 1)) {
+      for (int i = w.i_first; i < p.n_t; i = bwd_next(p, w, i + 1)) {
         const int sq = q_cnt % QS;
         ++q_cnt;
         const float4* lz4 = lse2_smem(sq) + h * 16;   // -LSE2
@@ -673,6 +831,16 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
           tmem_wait_ld();
           reg_fence32(r[0]);
           reg_fence32(r[1]);
+          bool wait_ok = true;
+          if constexpr (Cfg::kSmallD) {
+            // S^T is in registers: the next S^T may be issued over it.  P^T is
+            // written below: the previous dV must have read it.
+            tc_fence_before();
+            mbar_arrive(s_free);
+            if (s_cnt >= 2) wait_ok = mbar_wait(p_free, (s_cnt - 2) & 1);
+            tc_fence_after();
+          }
+          ok = __all_sync(0xffffffffu, wait_ok);
           const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
@@ -721,9 +889,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
               make_p(std::integral_constant<int, 0>{});
             }
             __syncwarp();
-            tmem_st16(tS + c * 16, pk);
+            tmem_st16(tP + c * 16, pk);
           }
         }
+        if (!ok) break;
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(p_full);
@@ -741,7 +910,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
           uint32_t pp[32];
           tmem_ld32(tDP, r[0]);
           tmem_ld32(tDP + 32, r[1]);
-          tmem_ld32(tS, pp);  // both halves' P: 32 packed columns
+          tmem_ld32(tP, pp);  // this half's P: 32 packed columns
           tmem_wait_ld();
           reg_fence32(r[0]);
           reg_fence32(r[1]);
@@ -789,6 +958,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       tc_fence_after();
       const float mul = h ? 1.f : p.scale;
       const uint32_t tAcc = t_lane + (h ? Cfg::kColDV : Cfg::kColDK);
+      uint8_t* epi_row = smem + Cfg::kOffEpi + h * Cfg::kTileBytes + kr * 128;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t r[32];
@@ -800,12 +970,40 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         for (int e = 0; e < 16; ++e)
           pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * mul, __uint_as_float(r[2 * e + 1]) * mul);
 #pragma unroll
-        for (int v4 = 0; v4 < 4; ++v4)
-          out_row[c * 4 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+        for (int v4 = 0; v4 < 4; ++v4) {
+          const uint4 val = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+          if constexpr (Cfg::kEpiTma) {
+            const int g = c * 4 + v4;  // 16-byte granule of the 128-byte row
+            *reinterpret_cast<uint4*>(epi_row + ((g ^ (kr & 7)) << 4)) = val;
+          } else {
+            out_row[c * 4 + v4] = val;
+          }
+        }
       }
       tc_fence_before();
+      if constexpr (Cfg::kEpiTma) {
+        // the whole tile is staged: one thread of the warpgroup stores it.
+        // The staging area is written again only in the next unit's epilogue,
+        // after dkv_full, which needs this thread's arrivals of that unit,
+        // made after the store below has read the tile.
+        fence_proxy_async_smem();
+        mbar_arrive(epi_ready(h));
+        if (kr == 0) {
+          ok = mbar_wait(epi_ready(h), epi_cnt & 1);
+          if (ok) {
+            tma_store_2d(h ? &tm_dv : &tm_dk, 0, w.bh * p.N + w.j * kTile,
+                         smem_u32(smem + Cfg::kOffEpi + h * Cfg::kTileBytes));
+            bulk_commit_group();
+            bulk_wait_group_read0();
+          }
+        }
+        ++epi_cnt;
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+      }
     }
     if (!ok) *abort_flag = 1;
+    if (Cfg::kEpiTma && kr == 0) bulk_wait_group0();  // stores complete before exit
   } else {
     // ------------------------------------------------------------ dQ group
     // Drains dQ partials: TMEM -> registers -> its own shared-memory staging
@@ -824,9 +1022,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     for (int round = 0; ok; ++round) {
       const int u = unit_for_round(round, blockIdx.x, G);
       if (u >= p.num_units) break;
-      const BwdUnit w = bwd_decode(p, u);
+      BwdUnit w;
+      ok = fetch_warp(round, w);
+      if (!ok) break;
       if (!w.any) continue;
-      for (int i = bwd_next(p, w, w.i_begin); i < p.n_t; i = bwd_next(p, w, i + 1)) {
+      for (int i = w.i_first; i < p.n_t; i = bwd_next(p, w, i + 1)) {
         ok = __all_sync(0xffffffffu, mbar_wait(dq_full, dq_cnt & 1));
         ++dq_cnt;
         if (!ok) break;

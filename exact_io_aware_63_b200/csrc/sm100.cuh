@@ -135,6 +135,15 @@ __device__ __forceinline__ void tma_reduce_add_2d(const void* tmap, int x, int y
       "r"(x), "r"(y), "r"(src)
       : "memory");
 }
+// 2-D tiled TMA store of a shared-memory box to global memory at (x, y).
+// Tracked by bulk groups.
+__device__ __forceinline__ void tma_store_2d(const void* tmap, int x, int y, uint32_t src) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+          reinterpret_cast<uint64_t>(tmap)),
+      "r"(x), "r"(y), "r"(src)
+      : "memory");
+}
 __device__ __forceinline__ void bulk_commit_group() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
