@@ -117,7 +117,7 @@ int heads_per_group(int BH, double bytes_per_head) {
 }
 
 struct WsLayout {
-  size_t delta, lse2, dq_acc, total;
+  size_t delta, lse2, dq_acc, counter, total;
 };
 
 WsLayout ws_layout(int B, int H, int N, int d) {
@@ -126,7 +126,8 @@ WsLayout ws_layout(int B, int H, int N, int d) {
   w.delta = 0;
   w.lse2 = round_up(w.delta + 4 * R, 256);
   w.dq_acc = round_up(w.lse2 + 4 * R, 256);
-  w.total = round_up(w.dq_acc + 4 * R * d, 256);
+  w.counter = round_up(w.dq_acc + 4 * R * d, 256);
+  w.total = w.counter + 256;
   return w;
 }
 
@@ -187,6 +188,7 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
   float* delta = reinterpret_cast<float*>(ws + wl.delta);
   float* lse2 = reinterpret_cast<float*>(ws + wl.lse2);
   float* dq_acc = reinterpret_cast<float*>(ws + wl.dq_acc);
+  int* counter = reinterpret_cast<int*>(ws + wl.counter);
   CUtensorMap tq, tk, tv, tdo, tdq, tdk, tdv;
   if (!make_tmap(&tq, q, rows, D) || !make_tmap(&tk, k, rows, D) || !make_tmap(&tv, v, rows, D) ||
       !make_tmap(&tdo, dout, rows, D) || !make_tmap_f32_acc(&tdq, dq_acc, rows, D) ||
@@ -204,7 +206,7 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
     const long long cap = static_cast<long long>(num_sms) * 8;
     if (blocks > cap) blocks = cap;
     fa::fa_bwd_pre_kernel<D><<<static_cast<int>(blocks), threads, 0, stream>>>(
-        o, dout, lse, delta, lse2, reinterpret_cast<float4*>(dq_acc), rows);
+        o, dout, lse, delta, lse2, reinterpret_cast<float4*>(dq_acc), counter, rows);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   // main
@@ -224,6 +226,7 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
     p.n_t = N / fa::kTile;
     p.num_units = B * H * p.n_t;
     p.heads_per_group = heads_per_group(B * H, 8.0 * N * D);  // Q, dO, f32 dQ accumulator
+    p.work_counter = counter;
     p.causal = causal ? 1 : 0;
     p.scale = scale;
     p.scale_log2 = scale * fa::kLog2e;

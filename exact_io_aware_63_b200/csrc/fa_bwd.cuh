@@ -51,7 +51,10 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const uint16_t* __restr
                                                          float* __restrict__ delta,
                                                          float* __restrict__ lse2,
                                                          float4* __restrict__ dq_acc,
+                                                         int* __restrict__ work_counter,
                                                          long long rows) {
+  // the main kernel's CTAs take work units from this counter
+  if (blockIdx.x == 0 && threadIdx.x == 0) *work_counter = 0;
   constexpr int kLanesPerRow = D / 8;  // one 16-byte chunk (8 bf16) per lane
   constexpr int kRowsPerWarp = 32 / kLanesPerRow;
   const long long warp_global = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5;
@@ -119,6 +122,7 @@ struct BwdParams {
   int B, H, N, n_t;
   int num_units;
   int heads_per_group;  // unit order: see bwd_decode
+  int* work_counter;    // next unit to take (zeroed by fa_bwd_pre_kernel)
   int causal;
   float scale;
   float scale_log2;
@@ -130,11 +134,11 @@ struct BwdCfg {
   // registers per thread: 128 at launch (512 x 128 = 65536), redistributed:
   //          producer/MMA   two dS warpgroups   dQ warpgroup
   // D = 64:  128 x 104   +  256 x 136        +  128 x 112  = 62464
-  // D = 128: 128 x 96    +  256 x 128        +  128 x 160  = 65536
+  // D = 128: 128 x 112   +  256 x 128        +  128 x 144  = 65536
   // (the dQ warpgroup holds a whole float32 dQ row)
-  static constexpr uint32_t kRegsLaunch = 128, kRegsLow = (D == 64) ? 104 : 96;
+  static constexpr uint32_t kRegsLaunch = 128, kRegsLow = (D == 64) ? 104 : 112;
   static constexpr uint32_t kRegsDs = (D == 64) ? 136 : 128;
-  static constexpr uint32_t kRegsDq = (D == 64) ? 112 : 160;
+  static constexpr uint32_t kRegsDq = (D == 64) ? 112 : 144;
   static constexpr int kTileBytes = kTile * D * 2;
   static constexpr int kBoxes = D / 64;
   // Q_i (with the tile's -LSE2 and -D rows) and dO_i come through separate
@@ -217,6 +221,7 @@ struct BwdCfg {
 
 struct BwdUnit {
   int bh, b, j, L, i_begin, any, i_first;  // i_first: first visited query tile
+  int valid;                                // 0: no unit left (end of the work)
 };
 
 __device__ __forceinline__ bool bwd_tile_on(const BwdParams& p, const BwdUnit& w, int i) {
@@ -249,6 +254,7 @@ __device__ __forceinline__ BwdUnit bwd_decode(const BwdParams& p, int u) {
   w.i_begin = p.causal ? w.j : 0;
   w.i_first = bwd_next(p, w, w.i_begin);
   w.any = w.i_first < p.n_t;
+  w.valid = 1;
   return w;
 }
 
@@ -298,6 +304,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     w.i_begin = b.x;
     w.any = b.y;
     w.i_first = b.z;
+    w.valid = b.w;
     return w;
   };
   // one thread's read of round r's unit record (it releases the slot)
@@ -381,7 +388,6 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_base_slot;
-  const int G = gridDim.x;
   static_assert(Cfg::kRegsLow * 128 + Cfg::kRegsDs * 256 + Cfg::kRegsDq * 128 <=
                     Cfg::kRegsLaunch * Cfg::kThreads,
                 "register split exceeds the launch allocation");
@@ -392,26 +398,35 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     if (lane == 0) {
       uint32_t kv_cnt = 0, q_cnt = 0, do_cnt = 0;
       bool ok = true;
+      // Units are taken from a counter shared by all CTAs (reset by the
+      // preprocess kernel), in the order bwd_decode gives them (longest
+      // first), so that the CTAs finish together whatever the unit lengths.
+      // This round's unit and the next one are published (the other roles
+      // read a unit's record before its first tile and the next one's at its
+      // last); after the work runs out, one record marks the end.
       int published = 0;  // unit records written
+      bool ended = false;
       for (int round = 0; ok; ++round) {
-        const int u = unit_for_round(round, blockIdx.x, G);
-        if (u >= p.num_units) break;
-        // publish this round's unit and the next one (the other roles read a
-        // unit's record before its first tile and the next one's at its last)
-        while (published <= round + 1) {
-          const int un = unit_for_round(published, blockIdx.x, G);
-          if (un >= p.num_units) break;
-          const BwdUnit wr = bwd_decode(p, un);
+        while (!ended && published <= round + 1) {
+          const int un = atomicAdd(p.work_counter, 1);
+          BwdUnit wr;
+          if (un < p.num_units) wr = bwd_decode(p, un);
           const int s = published % UR;
           ok = mbar_wait(unit_empty(s), ((published / UR) & 1) ^ 1);
           if (!ok) break;
-          unit_rec[2 * s] = make_int4(wr.bh, wr.b, wr.j, wr.L);
-          unit_rec[2 * s + 1] = make_int4(wr.i_begin, wr.any, wr.i_first, 0);
+          if (un < p.num_units) {
+            unit_rec[2 * s] = make_int4(wr.bh, wr.b, wr.j, wr.L);
+            unit_rec[2 * s + 1] = make_int4(wr.i_begin, wr.any, wr.i_first, 1);
+          } else {
+            unit_rec[2 * s + 1] = make_int4(0, 0, p.n_t, 0);
+            ended = true;
+          }
           mbar_arrive(unit_full(s));
           ++published;
         }
         if (!ok) break;
         const BwdUnit w = load_unit(round % UR);
+        if (!w.valid) break;
         if (!w.any) continue;
         const int skv = kv_cnt % KVS;
         ok = mbar_wait(kv_empty(skv), ((kv_cnt / KVS) & 1) ^ 1);
@@ -511,11 +526,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         return true;
       };
       for (int round = 0; ok; ++round) {
-        const int u = unit_for_round(round, blockIdx.x, G);
-        if (u >= p.num_units) break;
         BwdUnit w;
         ok = fetch_one(round, w);
-        if (!ok) break;
+        if (!ok || !w.valid) break;
         if (!w.any) continue;
         ok = mbar_wait(kv_full(0), kv_cnt & 1);
         ++kv_cnt;
@@ -650,8 +663,6 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       bool have_next = false;  // the next round's record was read at the look-ahead
       BwdUnit w_next;
       for (int round = 0; ok; ++round) {
-        const int u = unit_for_round(round, blockIdx.x, G);
-        if (u >= p.num_units) break;
         BwdUnit w;
         if (have_next) {
           w = w_next;
@@ -660,6 +671,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
           ok = fetch_one(round, w);
           if (!ok) break;
         }
+        if (!w.valid) break;
         if (!w.any) continue;
         const int skv = kv_cnt % KVS;
         if (!pre) ok = mbar_wait(kv_full(skv), (kv_cnt / KVS) & 1);
@@ -675,15 +687,13 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         bool pre_next = false;
         // the first tile of the next unit, for the look-ahead at the last tile
         auto next_unit_first = [&](BwdUnit& wn, int& in) -> bool {
-          const int un = unit_for_round(round + 1, blockIdx.x, G);
-          if (un >= p.num_units) return false;
           if (!fetch_one(round + 1, w_next)) {
             ok = false;
             return false;
           }
           have_next = true;
           wn = w_next;
-          if (!wn.any) return false;
+          if (!wn.valid || !wn.any) return false;
           in = wn.i_first;
           if (!mbar_wait(kv_full(kv_cnt % KVS), (kv_cnt / KVS) & 1)) {
             ok = false;
@@ -795,11 +805,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     uint32_t s_cnt = 0, dp_cnt = 0, dsm_cnt = 0, dkv_cnt = 0, q_cnt = 0, epi_cnt = 0;
     bool ok = true;
     for (int round = 0; ok; ++round) {
-      const int u = unit_for_round(round, blockIdx.x, G);
-      if (u >= p.num_units) break;
       BwdUnit w;
       ok = fetch_warp(round, w);
-      if (!ok) break;
+      if (!ok || !w.valid) break;
       const int c_key = w.j * kTile + kr;  // key index within the head
       const size_t krow = (size_t)w.bh * p.N + c_key;
       // warpgroup 0 writes the dK row, warpgroup 1 the dV row
@@ -1020,11 +1028,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     uint32_t dq_cnt = 0;
     bool ok = true;
     for (int round = 0; ok; ++round) {
-      const int u = unit_for_round(round, blockIdx.x, G);
-      if (u >= p.num_units) break;
       BwdUnit w;
       ok = fetch_warp(round, w);
-      if (!ok) break;
+      if (!ok || !w.valid) break;
       if (!w.any) continue;
       for (int i = w.i_first; i < p.n_t; i = bwd_next(p, w, i + 1)) {
         ok = __all_sync(0xffffffffu, mbar_wait(dq_full, dq_cnt & 1));

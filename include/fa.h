@@ -92,8 +92,9 @@ int fa_fwd_traced(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16*
 
 /*
  * Bytes of device workspace fa_bwd needs: 4*B*H*N (D) + 4*B*H*N (LSE in
- * base 2) + 4*B*H*N*d (float32 dQ accumulator), each region 256-byte
- * aligned.  Returns 0 for an empty or invalid shape.
+ * base 2) + 4*B*H*N*d (float32 dQ accumulator) + 256 (the counter from which
+ * the main kernel's CTAs take work units), each region 256-byte aligned.
+ * Returns 0 for an empty or invalid shape.
  */
 size_t fa_bwd_workspace_size(int B, int H, int N, int d);
 
@@ -127,9 +128,10 @@ int fa_bwd_traced(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa
 
 /*
  * One of the three launches of fa_bwd, for callers that schedule or time them
- * separately: phase 0 = preprocess (D, base-2 LSE, zeroed dQ accumulator in
- * the workspace), 1 = main kernel (dK, dV; dQ partials into the
- * accumulator), 2 = dQ = bf16(scale * accumulator).  Arguments as for
+ * separately: phase 0 = preprocess (D, base-2 LSE, zeroed dQ accumulator and
+ * work-unit counter in the workspace), 1 = main kernel (dK, dV; dQ partials
+ * into the accumulator; takes its work units from the counter, so each
+ * phase 1 needs a phase 0 before it), 2 = dQ = bf16(scale * accumulator).  Arguments as for
  * fa_bwd.  Calling phases 0, 1, 2 in order on one stream with the same
  * arguments and workspace is exactly fa_bwd; a phase reads what the earlier
  * phases left in the workspace.
