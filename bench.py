@@ -82,16 +82,19 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+# the headers the benchmarked kernels are compiled from
+BENCHED_KERNEL_SOURCES = ("fa_bwd.cuh", "fa_fwd.cuh", "sm100.cuh")
+
+
 def kernel_source_hash():
-    """Hash of the device-code sources (the kernel headers); host-side ABI code is
-    left out because it does not change what a kernel does."""
+    """Hash of the device-code sources of the benchmarked kernels; host-side ABI code
+    is left out because it does not change what a kernel does."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "exact_io_aware_63_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith(".cuh"):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode())
-                h.update(f.read())
+    for name in BENCHED_KERNEL_SOURCES:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
@@ -511,6 +514,121 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+
+# ----------------------------------------------------------------------------
+# comparison with standard attention (materialised score matrix)
+# ----------------------------------------------------------------------------
+
+def standard_allowed(x, dev):
+    """Boolean [B or 1, 1, N, N] mask of allowed (query, key) pairs, the same
+    definition the library and the oracle use."""
+    import torch
+    B, H, N, d = x.q.shape
+    r = torch.arange(N, device=dev)
+    allowed = torch.ones((1, 1, N, N), dtype=torch.bool, device=dev)
+    if x.causal:
+        allowed = allowed & (r[None, None, None, :] <= r[None, None, :, None])
+    if x.block_mask is not None:
+        bm = x.block_mask.to(dev).bool()
+        allowed = allowed & bm.repeat_interleave(128, 0).repeat_interleave(128, 1)[None, None]
+    if x.kv_len is not None:
+        kl = x.kv_len.to(dev)
+        allowed = allowed & (r[None, None, None, :] < kl[:, None, None, None])
+    return allowed
+
+
+def run_vs_standard(args):
+    """Times fwd+bwd of standard attention written with plain PyTorch ops (S and P
+    materialised in HBM, softmax in float32, autograd for the backward; "Standard
+    Attention Algorithm" of the FlashAttention pages) against this library on the
+    same inputs, and reports the ratio of step times and of the extra device memory
+    each needs beyond inputs and outputs."""
+    import torch
+    from exact_io_aware_63_b200 import binding
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    binding.load(build_if_missing=False)
+    x = workload_or_shape(args)
+    B, H, N, d = x.q.shape
+    # S (f32), P (bf16) and their gradients: skip sizes whose score matrices do not fit
+    score_bytes = B * H * N * N * (4 + 2 + 4 + 2)
+    line = {"metric": "fwd+bwd step time and extra device memory: standard attention vs this library",
+            "workload": args.workload if not args.shape else args.shape,
+            "config": {"B": B, "H": H, "N": N, "d": d, "causal": bool(x.causal),
+                       "key_padding": x.kv_len is not None, "block_sparse": x.block_mask is not None},
+            "pages_claim": "2-4x faster than standard attention; memory linear instead of quadratic in N"}
+    if score_bytes > 100e9:
+        line["standard"] = f"skipped: score matrices would need {score_bytes / 1e9:.0f} GB"
+        print(json.dumps(line))
+        return
+    q, k, v, do = (t.to(dev) for t in (x.q, x.k, x.v, x.dout))
+    bm = None if x.block_mask is None else x.block_mask.to(dev)
+    kl = None if x.kv_len is None else x.kv_len.to(dev)
+    allowed = standard_allowed(x, dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def std_step():
+        qq, kk, vv = (t.detach().requires_grad_() for t in (q, k, v))
+        s = torch.matmul(qq, kk.transpose(-1, -2)).float() * x.scale
+        s = s.masked_fill(~allowed, float("-inf"))
+        pm = torch.softmax(s, dim=-1).to(torch.bfloat16)
+        out = torch.matmul(pm, vv)
+        out.backward(do)
+        return out, qq.grad, kk.grad, vv.grad
+
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    ws_bytes = binding.fa_bwd_workspace_size(B, H, N, d)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+
+    def our_step():
+        for rc in (binding.fa_fwd(q, k, v, o, lse, B, H, N, d, x.scale, x.causal, bm, kl,
+                                  stream.cuda_stream),
+                   binding.fa_bwd(q, k, v, o, lse, do, dq, dk, dv, B, H, N, d, x.scale, x.causal,
+                                  bm, kl, ws, ws_bytes, stream.cuda_stream)):
+            if rc != 0:
+                raise RuntimeError(binding.fa_status_string(rc))
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(args.steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        ts.sort()
+        return ts[len(ts) // 2]
+
+    ours_ms = timed(our_step)
+    std_ms = timed(lambda: std_step())
+    # extra memory beyond inputs and outputs: ours = LSE + backward workspace;
+    # standard = peak of one step above what was allocated before it, minus its outputs
+    torch.cuda.synchronize()
+    torch.cuda.reset_peak_memory_stats(dev)
+    base = torch.cuda.memory_allocated(dev)
+    res = std_step()
+    torch.cuda.synchronize()
+    out_bytes = sum(t.numel() * t.element_size() for t in res)
+    std_extra = torch.cuda.max_memory_allocated(dev) - base - out_bytes
+    our_extra = lse.numel() * 4 + ws_bytes
+    o_std = res[0].detach().float()
+    has_key = allowed.expand(B, H, N, N).any(-1)[..., None]  # rows with an allowed key
+    o_diff = float((o.float() - o_std).abs().masked_fill(~has_key, 0.0).max())
+    line.update({"ours_ms": ours_ms, "standard_ms": std_ms, "speedup": std_ms / ours_ms,
+                 "ours_extra_bytes": our_extra, "standard_extra_bytes": int(std_extra),
+                 "memory_ratio": std_extra / our_extra, "max_abs_diff_O": o_diff,
+                 "l2": "flushed between timed steps", "timing": "median of steps, CUDA events"})
+    print(json.dumps(line))
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -526,11 +644,16 @@ def main():
                     help="CPU-seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--vs-standard", action="store_true",
+                    help="instead of the benchmark line, compare one step with standard "
+                         "attention (S and P materialised) on the same inputs")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("note: warm-up raised to 3 steps", file=sys.stderr)
         args.warmup = 3
-    if args.impl == "reference":
+    if args.vs_standard:
+        run_vs_standard(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)
