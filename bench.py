@@ -247,11 +247,12 @@ def run_ours(args):
         check(binding.fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, bm, kl, S), "fa_fwd")
         if ev is not None:
             ev[1].record(stream)
-        for ph in range(3):
+        # fa_bwd is phases 0, 1, 2; fa_bwd_deterministic is 0, 1, 3
+        for i, ph in enumerate((0, 1, 3) if args.deterministic else (0, 1, 2)):
             check(binding.fa_bwd_phase(ph, q, k, v, o, lse, do, dq, dk, dv, B, H, N, d, scale,
                                        causal, bm, kl, ws, ws_bytes, S), "fa_bwd_phase")
             if ev is not None:
-                ev[2 + ph].record(stream)
+                ev[2 + i].record(stream)
 
     def barrier():
         if dist is not None:
@@ -323,8 +324,9 @@ def run_ours(args):
             v.copy_(hv, non_blocking=True)
             do.copy_(hdo, non_blocking=True)
             check(binding.fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, bm, kl, S), "fa_fwd")
-            check(binding.fa_bwd(q, k, v, o, lse, do, dq, dk, dv, B, H, N, d, scale, causal, bm, kl,
-                                 ws, ws_bytes, S), "fa_bwd")
+            bwd = binding.fa_bwd_deterministic if args.deterministic else binding.fa_bwd
+            check(bwd(q, k, v, o, lse, do, dq, dk, dv, B, H, N, d, scale, causal, bm, kl,
+                      ws, ws_bytes, S), "fa_bwd")
             ho.copy_(o, non_blocking=True)
             hlse.copy_(lse, non_blocking=True)
             hdq.copy_(dq, non_blocking=True)
@@ -358,7 +360,7 @@ def run_ours(args):
                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": achieved / peaks["bf16_tflops"],
                 "peak_source": f"{peak_kind} bf16_tflops (burst)",
-                "traffic": ncu_traffic(dom, args.workload),
+                "traffic": ncu_traffic(dom, args.workload + (f"@{args.shape}" if args.shape else "")),
                 "algorithmic_bytes": dom_bytes,
                 "algorithmic_flops": dom_flops,
                 "ms_per_launch": dom_t}
@@ -372,7 +374,8 @@ def run_ours(args):
                    "key_padding": x.kv_len is not None, "block_sparse": x.block_mask is not None,
                    "flop_density": density(x), "seed": w.seed,
                    "l2": "flushed between timed steps (256 MiB write)",
-                   "parallelism": f"replica x{world}"},
+                   "parallelism": f"replica x{world}",
+                   "backward": "fa_bwd_deterministic" if args.deterministic else "fa_bwd"},
         "fwd_tflops": fwd_tflops,
         "bwd_tflops": bwd_tflops,
         "fwd_bwd_pct_of_peak": per_gpu / peaks["bf16_tflops"],
@@ -644,6 +647,8 @@ def main():
                     help="CPU-seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--deterministic", action="store_true",
+                    help="time fa_bwd_deterministic (ordered dQ kernel) instead of fa_bwd")
     ap.add_argument("--vs-standard", action="store_true",
                     help="instead of the benchmark line, compare one step with standard "
                          "attention (S and P materialised) on the same inputs")

@@ -8,7 +8,7 @@ import of a function raises.
 Raw entry points (same argument order as the C ABI; tensors are passed as
 torch tensors or None, the stream as a torch.cuda.Stream or None = current):
 ``fa_fwd``, ``fa_fwd_traced``, ``fa_bwd``, ``fa_bwd_traced``, ``fa_bwd_phase``,
-``fa_bwd_noalloc``,
+``fa_bwd_deterministic``, ``fa_bwd_noalloc``,
 ``fa_bwd_workspace_size``, ``fa_get_device_status``, ``fa_status_string``,
 ``fa_version``.
 
@@ -40,6 +40,7 @@ _SIGS = {
     "fa_bwd_traced": (_i, [_vp] * 9 + [_i, _i, _i, _i, _f, _i, _vp, _vp, _vp, _sz, _vp, _vp]),
     "fa_bwd_phase": (_i, [_i] + [_vp] * 9 + [_i, _i, _i, _i, _f, _i, _vp, _vp, _vp, _sz, _vp]),
     "fa_bwd_noalloc": (_i, [_vp] * 9 + [_i, _i, _i, _i, _f, _i, _vp, _vp, _vp]),
+    "fa_bwd_deterministic": (_i, [_vp] * 9 + [_i, _i, _i, _i, _f, _i, _vp, _vp, _vp, _sz, _vp]),
     "fa_get_device_status": (_i, [_vp]),
     "fa_status_string": (ctypes.c_char_p, [_i]),
     "fa_version": (_i, []),
@@ -147,6 +148,15 @@ def fa_bwd_phase(phase, q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, ca
                                int(workspace_bytes), _stream(stream))
 
 
+def fa_bwd_deterministic(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal,
+                         block_mask, kv_len, workspace, workspace_bytes, stream=None):
+    """fa_bwd with a bitwise-reproducible dQ (ordered per-query-tile kernel)."""
+    return load().fa_bwd_deterministic(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
+                                       _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, float(scale),
+                                       int(bool(causal)), _ptr(block_mask), _ptr(kv_len),
+                                       _ptr(workspace), int(workspace_bytes), _stream(stream))
+
+
 def fa_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, block_mask,
                    kv_len, stream=None):
     """fa_bwd without a workspace argument: the library's built-in static scratch is used
@@ -195,15 +205,21 @@ def attention_forward(q, k, v, scale, causal=False, block_mask=None, kv_len=None
 
 
 def attention_backward(q, k, v, o, lse, dout, scale, causal=False, block_mask=None, kv_len=None,
-                       workspace=None, visited=None, stream=None):
-    """dQ, dK, dV for the forward that produced (o, lse)."""
+                       workspace=None, visited=None, stream=None, deterministic=False):
+    """dQ, dK, dV for the forward that produced (o, lse).  ``deterministic`` selects
+    fa_bwd_deterministic (bitwise-reproducible dQ)."""
     import torch
     B, H, N, d = q.shape
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws_bytes = fa_bwd_workspace_size(B, H, N, d)
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
-    if visited is None:
+    if deterministic:
+        if visited is not None:
+            raise ValueError("the deterministic backward has no traced variant")
+        rc = fa_bwd_deterministic(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal,
+                                  block_mask, kv_len, workspace, workspace.numel(), stream)
+    elif visited is None:
         rc = fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, block_mask,
                     kv_len, workspace, workspace.numel(), stream)
     else:

@@ -12,6 +12,7 @@
 
 #include "fa.h"
 #include "fa_bwd.cuh"
+#include "fa_bwd_det.cuh"
 #include "fa_fwd.cuh"
 
 namespace {
@@ -246,6 +247,38 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
         reinterpret_cast<const float4*>(dq_acc), reinterpret_cast<uint4*>(dq), scale, n8);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
+  // dQ without atomics: one CTA walks each query tile's key tiles in order
+  if (phases & 8u) {
+    using DCfg = fa::DetCfg<D>;
+    static bool det_smem_set = false;
+    if (!det_smem_set) {
+      if (!set_smem(fa::fa_bwd_dq_det_kernel<D>, DCfg::kSmemBytes)) return FA_ERR_CUDA;
+      det_smem_set = true;
+    }
+    fa::DetParams dp;
+    fa::FwdParams& sp = dp.sched;
+    sp.o = nullptr;
+    sp.lse = nullptr;
+    sp.block_mask = block_mask;
+    sp.kv_len = kv_len;
+    sp.visited = nullptr;
+    sp.B = B;
+    sp.H = H;
+    sp.N = N;
+    sp.n_t = N / fa::kTile;
+    sp.num_units = B * H * sp.n_t;
+    sp.heads_per_group = heads_per_group(B * H, 4.0 * N * D);  // K and V
+    sp.causal = causal ? 1 : 0;
+    sp.scale_log2 = scale * fa::kLog2e;
+    dp.delta = delta;
+    dp.lse2 = lse2;
+    dp.dq = dq;
+    dp.scale = scale;
+    const int grid = sp.num_units < num_sms ? sp.num_units : num_sms;
+    fa::fa_bwd_dq_det_kernel<D><<<grid, DCfg::kThreads, DCfg::kSmemBytes, stream>>>(tq, tk, tv,
+                                                                                    tdo, dp);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
   return FA_OK;
 }
 
@@ -345,9 +378,19 @@ int fa_bwd_phase(int phase, const fa_bf16* q, const fa_bf16* k, const fa_bf16* v
                  fa_bf16* dv, int B, int H, int N, int d, float scale, int causal,
                  const uint8_t* block_mask, const int32_t* kv_len, void* workspace,
                  size_t workspace_bytes, void* stream) {
-  if (phase < 0 || phase > 2) return FA_ERR_ARG;
+  if (phase < 0 || phase > 3) return FA_ERR_ARG;
   return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, block_mask, kv_len,
                   workspace, workspace_bytes, nullptr, stream, 1u << phase);
+}
+
+int fa_bwd_deterministic(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf16* o,
+                         const float* lse, const fa_bf16* dout, fa_bf16* dq, fa_bf16* dk,
+                         fa_bf16* dv, int B, int H, int N, int d, float scale, int causal,
+                         const uint8_t* block_mask, const int32_t* kv_len, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  // preprocess, main kernel (its dK and dV), then dQ by the ordered kernel
+  return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, block_mask, kv_len,
+                  workspace, workspace_bytes, nullptr, stream, 1u | 2u | 8u);
 }
 
 int fa_get_device_status(void* stream) {

@@ -62,7 +62,7 @@ typedef enum {
     FA_ERR_WORKSPACE = -5,      /* workspace NULL or smaller than fa_bwd_workspace_size */
     FA_ERR_CUDA = -6,           /* a CUDA runtime/driver call failed */
     FA_ERR_TIMEOUT = -7,        /* a device pipeline wait gave up (fa_get_device_status) */
-    FA_ERR_ARG = -8,            /* scale not finite or not > 0, or phase not in 0..2 */
+    FA_ERR_ARG = -8,            /* scale not finite or not > 0, or phase not in 0..3 */
     FA_ERR_SCRATCH_LIMIT = -9   /* fa_bwd_noalloc: the shape needs more scratch than
                                    FA_BWD_NOALLOC_SCRATCH_BYTES */
 } fa_status;
@@ -127,20 +127,41 @@ int fa_bwd_traced(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa
                   void* workspace, size_t workspace_bytes, uint8_t* visited, void* stream);
 
 /*
- * One of the three launches of fa_bwd, for callers that schedule or time them
- * separately: phase 0 = preprocess (D, base-2 LSE, zeroed dQ accumulator and
- * work-unit counter in the workspace), 1 = main kernel (dK, dV; dQ partials
- * into the accumulator; takes its work units from the counter, so each
- * phase 1 needs a phase 0 before it), 2 = dQ = bf16(scale * accumulator).  Arguments as for
+ * One launch of fa_bwd or fa_bwd_deterministic, for callers that schedule or
+ * time them separately: phase 0 = preprocess (D, base-2 LSE, zeroed dQ
+ * accumulator and work-unit counter in the workspace), 1 = main kernel (dK,
+ * dV; dQ partials into the accumulator; takes its work units from the
+ * counter, so each phase 1 needs a phase 0 before it), 2 = dQ = bf16(scale *
+ * accumulator), 3 = dQ by the ordered kernel of fa_bwd_deterministic (reads
+ * only what phase 0 wrote).  Arguments as for
  * fa_bwd.  Calling phases 0, 1, 2 in order on one stream with the same
- * arguments and workspace is exactly fa_bwd; a phase reads what the earlier
- * phases left in the workspace.
+ * arguments and workspace is exactly fa_bwd, and 0, 1, 3 is exactly
+ * fa_bwd_deterministic; a phase reads what the earlier phases left in the
+ * workspace.
  */
 int fa_bwd_phase(int phase, const fa_bf16* q, const fa_bf16* k, const fa_bf16* v,
                  const fa_bf16* o, const float* lse, const fa_bf16* dout, fa_bf16* dq, fa_bf16* dk,
                  fa_bf16* dv, int B, int H, int N, int d, float scale, int causal,
                  const uint8_t* block_mask, const int32_t* kv_len, void* workspace,
                  size_t workspace_bytes, void* stream);
+
+/*
+ * fa_bwd with a bitwise-reproducible result: the same arguments and
+ * workspace, the same outputs within rounding, and on every run on the same
+ * device the same bits.  fa_bwd's dQ sums the key tiles' contributions with
+ * reduce-adds whose order varies between runs; here one CTA owns each query
+ * tile and adds its visited key tiles' dS K_j products in increasing j, on
+ * chip (recomputing S, P and dP for the purpose), and writes dQ once.  The
+ * backward pass of the pages recomputes the score tiles instead of storing
+ * them ("FlashAttention, Decoded", "The Hardware Picture"); the order of the
+ * sums is this library's choice.  Costs about 60% more tensor-core work than
+ * fa_bwd.  Three launches: preprocess, main kernel (dK, dV), ordered dQ.
+ */
+int fa_bwd_deterministic(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf16* o,
+                         const float* lse, const fa_bf16* dout, fa_bf16* dq, fa_bf16* dk,
+                         fa_bf16* dv, int B, int H, int N, int d, float scale, int causal,
+                         const uint8_t* block_mask, const int32_t* kv_len, void* workspace,
+                         size_t workspace_bytes, void* stream);
 
 /*
  * Size in bytes of the library's built-in backward scratch buffer (64 MiB),

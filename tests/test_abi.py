@@ -23,7 +23,7 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ["fa_fwd", "fa_fwd_traced", "fa_bwd", "fa_bwd_traced", "fa_bwd_phase",
-              "fa_bwd_workspace_size",
+              "fa_bwd_deterministic", "fa_bwd_workspace_size",
               "fa_get_device_status", "fa_status_string", "fa_version"]:
         assert n in names
 
@@ -76,7 +76,18 @@ def bwd(**kw):
                       a["block_mask"], a["kv_len"], a["ws"], a["ws_bytes"], None)
 
 
-@pytest.mark.parametrize("call", [fwd, bwd])
+def bwd_det(**kw):
+    a = dict(q=P, k=P, v=P, o=P, lse=P, dout=P, dq=P, dk=P, dv=P, B=1, H=1, N=128, d=64,
+             scale=0.125, causal=0, block_mask=None, kv_len=None, ws=P, ws_bytes=1 << 30)
+    a.update(kw)
+    lib = binding.load()
+    return lib.fa_bwd_deterministic(a["q"], a["k"], a["v"], a["o"], a["lse"], a["dout"], a["dq"],
+                                    a["dk"], a["dv"], a["B"], a["H"], a["N"], a["d"], a["scale"],
+                                    a["causal"], a["block_mask"], a["kv_len"], a["ws"],
+                                    a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("call", [fwd, bwd, bwd_det])
 def test_shape_errors(call):
     assert call(N=100) == -3
     assert call(N=-128) == -3
@@ -86,7 +97,7 @@ def test_shape_errors(call):
     assert call(d=32) == -4
 
 
-@pytest.mark.parametrize("call", [fwd, bwd])
+@pytest.mark.parametrize("call", [fwd, bwd, bwd_det])
 def test_empty_problems_are_no_ops(call):
     assert call(B=0) == 0
     assert call(H=0) == 0
@@ -95,7 +106,7 @@ def test_empty_problems_are_no_ops(call):
     assert call(B=0, q=None, k=None) == 0
 
 
-@pytest.mark.parametrize("call", [fwd, bwd])
+@pytest.mark.parametrize("call", [fwd, bwd, bwd_det])
 def test_null_and_alignment(call):
     assert call(q=None) == -1
     assert call(o=None) == -1 if call is fwd else call(dq=None) == -1
@@ -104,7 +115,7 @@ def test_null_and_alignment(call):
     assert call(kv_len=P + 1) == -2
 
 
-@pytest.mark.parametrize("call", [fwd, bwd])
+@pytest.mark.parametrize("call", [fwd, bwd, bwd_det])
 def test_scale_errors(call):
     assert call(scale=0.0) == -8
     assert call(scale=-1.0) == -8
@@ -112,10 +123,11 @@ def test_scale_errors(call):
     assert call(scale=float("nan")) == -8
 
 
-def test_backward_workspace_errors():
-    assert bwd(ws=None) == -5
-    assert bwd(ws_bytes=16) == -5
-    assert bwd(ws=P + 16) == -2
+@pytest.mark.parametrize("call", [bwd, bwd_det])
+def test_backward_workspace_errors(call):
+    assert call(ws=None) == -5
+    assert call(ws_bytes=16) == -5
+    assert call(ws=P + 16) == -2
 
 
 def test_traced_variants_need_the_visit_buffer():
@@ -129,7 +141,7 @@ def test_traced_variants_need_the_visit_buffer():
 
 def test_backward_phase_number_is_checked():
     lib = binding.load()
-    for ph in (-1, 3):
+    for ph in (-1, 4):
         rc = lib.fa_bwd_phase(ph, P, P, P, P, P, P, P, P, P, 1, 1, 128, 64, 0.125, 0, None, None, P,
                               1 << 30, None)
         assert rc == -8
