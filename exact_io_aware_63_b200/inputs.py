@@ -79,7 +79,7 @@ class Inputs:
     scale: float
     causal: bool
     kv_len: Optional[torch.Tensor]      # int32 [B] or None
-    block_mask: Optional[torch.Tensor]  # uint8 [N/128, N/128] or None
+    block_mask: Optional[torch.Tensor]  # uint8 [ceil(N/128), ceil(N/128)] or None
 
     @property
     def shape(self):
@@ -130,7 +130,7 @@ def make_inputs(B: int, H: int, N: int, d: int, *, scale: Optional[float] = None
     if kv_len is None and key_padding is not None:
         kv_len = draw_kv_len(B, N, key_padding[0], key_padding[1], gen)
     if block_mask is None and block_keep is not None:
-        block_mask = draw_block_mask(N // TILE, block_keep, gen)
+        block_mask = draw_block_mask(-(-N // TILE), block_keep, gen)  # ceil(N / 128) tiles
     if kv_len is not None:
         kv_len = torch.as_tensor(kv_len, dtype=torch.int32).contiguous()
     if block_mask is not None:

@@ -30,7 +30,7 @@ Functions (all arrays contiguous, float64 unless stated):
   kv_len_b)`` -> ``(dk_cols, dv_cols)``: dK and dV of chosen key columns of
   one head (a full pass over the head's rows).
 * ``tile_visits(B, N, causal, block_mask, kv_len, T=128, i_begin=0,
-  i_end=None)`` -> uint8 [B, i_end - i_begin, N // T]: 1 where a
+  i_end=None)`` -> uint8 [B, i_end - i_begin, ceil(N / T)]: 1 where a
   (query tile, key tile) pair holds at least one allowed (row, key).
 """
 
@@ -250,7 +250,7 @@ def attention_backward_kv_cols(q, k, v, dout, cols, scale, causal=False, block_m
 
 
 def tile_visits(B, N, causal=False, block_mask=None, kv_len=None, T=128, i_begin=0, i_end=None):
-    nt = N // T
+    nt = -(-N // T)  # ceil(N / T): a last, partial tile holds the remaining positions
     i_end = nt if i_end is None else i_end
     bm, kl = _mask_args(block_mask, kv_len)
     out = np.zeros((B, i_end - i_begin, nt), np.uint8)

@@ -14,7 +14,8 @@
  * out one query row at a time:
  *
  *   M(r,c) = (!causal || c <= r) && (kv_len == NULL || c < kv_len[b])
- *            && (block_mask == NULL || block_mask[(r/128)*(N/128) + c/128] != 0)
+ *            && (block_mask == NULL || block_mask[(r/128)*nt + c/128] != 0)
+ *            with nt = ceil(N / 128) (a last, partial tile holds the rest)
  *   S_rc   = scale * sum_k Q_rk K_ck          if M(r,c), else -inf
  *   m_r    = max_c S_rc,  l_r = sum_c exp(S_rc - m_r)
  *   P_rc   = exp(S_rc - m_r) / l_r,  LSE_r = m_r + ln l_r  (natural log)
@@ -62,7 +63,8 @@ static int allowed(int r, int c, int N, int causal, const uint8_t *block_mask, i
     if (causal && c > r) return 0;
     if (L >= 0 && c >= L) return 0;
     if (block_mask) {
-        int nt = N / ORACLE_MASK_TILE;
+        /* nt = ceil(N / 128): a last, partial tile holds the remaining positions */
+        int nt = (N + ORACLE_MASK_TILE - 1) / ORACLE_MASK_TILE;
         if (!block_mask[(size_t)(r / ORACLE_MASK_TILE) * nt + (c / ORACLE_MASK_TILE)]) return 0;
     }
     return 1;
@@ -208,7 +210,6 @@ static void *worker(void *arg)
 static int run_job(oracle_job *job, int nthreads)
 {
     if (job->B <= 0 || job->H <= 0 || job->N <= 0 || job->d <= 0) return -3;
-    if (job->block_mask && job->N % ORACLE_MASK_TILE != 0) return -3;
     if (nthreads < 1) nthreads = 1;
     if (nthreads > job->B * job->H) nthreads = job->B * job->H;
     pthread_mutex_init(&job->lock, NULL);
@@ -491,17 +492,18 @@ int oracle_attention_backward_kv_cols(const double *q, const double *k, const do
 
 /*
  * Which (query tile, key tile) pairs hold at least one allowed (r, c).
- * visits is [B][i_end - i_begin][n_t] with n_t = N / T: the entry for query
- * tile i (i_begin <= i < i_end) and key tile j is 1 when some r in tile i and
- * some c in tile j have M(r,c), else 0.  Brute force over the entries of each
+ * visits is [B][i_end - i_begin][n_t] with n_t = ceil(N / T) (a last, partial
+ * tile holds the remaining positions): the entry for query tile i
+ * (i_begin <= i < i_end) and key tile j is 1 when some r < N in tile i and
+ * some c < N in tile j have M(r,c), else 0.  Brute force over the entries of each
  * tile pair (stopping at the first allowed one), straight from the
  * definition of M; heads share the mask, so only b matters.
  */
 int oracle_tile_visits(uint8_t *visits, int B, int N, int T, int causal,
                        const uint8_t *block_mask, const int32_t *kv_len, int i_begin, int i_end)
 {
-    if (T <= 0 || N % T != 0 || (block_mask && N % ORACLE_MASK_TILE != 0)) return -3;
-    const int nt = N / T;
+    if (T <= 0 || N <= 0) return -3;
+    const int nt = (N + T - 1) / T;
     if (i_begin < 0 || i_end > nt || i_begin > i_end) return -3;
     const int ni = i_end - i_begin;
     for (int b = 0; b < B; ++b) {
@@ -509,8 +511,8 @@ int oracle_tile_visits(uint8_t *visits, int B, int N, int T, int causal,
         for (int i = i_begin; i < i_end; ++i)
             for (int j = 0; j < nt; ++j) {
                 int any = 0;
-                for (int r = i * T; r < (i + 1) * T && !any; ++r)
-                    for (int c = j * T; c < (j + 1) * T; ++c)
+                for (int r = i * T; r < (i + 1) * T && r < N && !any; ++r)
+                    for (int c = j * T; c < (j + 1) * T && c < N; ++c)
                         if (allowed(r, c, N, causal, block_mask, L)) { any = 1; break; }
                 visits[((size_t)b * ni + (i - i_begin)) * nt + j] = (uint8_t)any;
             }

@@ -87,6 +87,26 @@ def test_zero_query_gives_mean_of_allowed_values(causal, kv, use_bm):
             assert abs(lse[0, h, r] - math.log(cnt)) < 1e-13
 
 
+@pytest.mark.parametrize("causal,kv", [(False, None), (True, None), (False, 290), (True, 260)])
+def test_zero_query_partial_last_tile(causal, kv):
+    # N = 300: tiles 0..127, 128..255 and a partial tile 256..299; the block mask
+    # has ceil(300 / 128) = 3 rows and columns, its last ones covering the rest
+    B, H, N, d = 1, 1, 300, 8
+    q = np.zeros((B, H, N, d))
+    k, v = rand((B, H, N, d), 11), rand((B, H, N, d), 12)
+    bm = np.array([[1, 0, 1], [0, 1, 0], [1, 1, 1]], np.uint8)
+    kvl = None if kv is None else np.array([kv], np.int32)
+    o, lse = oracle.attention_forward(q, k, v, 0.5, causal=causal, block_mask=bm, kv_len=kvl)
+    for r in [0, 5, 127, 128, 255, 256, 270, 299]:
+        keys = [c for c in range(N)
+                if (not causal or c <= r) and (kv is None or c < kv) and bm[r // 128, c // 128]]
+        if not keys:
+            assert np.all(o[0, 0, r] == 0) and lse[0, 0, r] == -np.inf
+            continue
+        np.testing.assert_allclose(o[0, 0, r], v[0, 0, keys].mean(axis=0), atol=1e-13)
+        assert abs(lse[0, 0, r] - math.log(len(keys))) < 1e-13
+
+
 def test_dominant_score_selects_one_value_row():
     N, d = 64, 64
     rng = np.random.default_rng(3)
@@ -321,6 +341,21 @@ def test_tile_visits_hand_enumerated():
     assert masked.tolist() == [[1, 0, 0, 0], [0, 1, 0, 0], [1, 0, 0, 0], [0, 0, 1, 1]]
     part = oracle.tile_visits(1, 512, causal=True, block_mask=bm, i_begin=2, i_end=4)[0]
     assert part.tolist() == masked[2:].tolist()
+
+
+def test_tile_visits_partial_last_tile_hand_enumerated():
+    # N = 300 -> tiles 0..127, 128..255, 256..299.  Written out by hand.
+    assert oracle.tile_visits(1, 300, causal=True)[0].tolist() == [[1, 0, 0], [1, 1, 0],
+                                                                    [1, 1, 1]]
+    # keys < 256 end exactly at the second tile; keys < 257 reach the partial one
+    kv = oracle.tile_visits(2, 300, kv_len=np.array([256, 257], np.int32))
+    assert kv[0].tolist() == [[1, 1, 0]] * 3
+    assert kv[1].tolist() == [[1, 1, 1]] * 3
+    bm = np.array([[1, 0, 1], [0, 1, 0], [0, 1, 1]], np.uint8)
+    assert oracle.tile_visits(1, 300, block_mask=bm)[0].tolist() == bm.tolist()
+    # N = 100: a single partial tile
+    assert oracle.tile_visits(1, 100, causal=True)[0].tolist() == [[1]]
+    assert oracle.tile_visits(1, 100, kv_len=np.array([0], np.int32))[0].tolist() == [[0]]
 
 
 def test_tile_visits_agree_with_value_identity_probabilities():
