@@ -36,30 +36,35 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [rows][d] bf16 tensor, boxes of 128 rows x 64 columns, 128-byte swizzle.
-bool make_tmap(CUtensorMap* m, const void* base, long long rows, int d) {
+// [B*H][N][d] bf16 tensor viewed per head (x = column, y = row within the
+// head, z = head), boxes of 128 rows x 64 columns, 128-byte swizzle.  Rows of
+// a box beyond N are zero-filled on loads and dropped on stores, so a partial
+// last tile never touches the next head.
+bool make_tmap(CUtensorMap* m, const void* base, int BH, int N, int d) {
   auto fn = encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
-  cuuint32_t box[2] = {64, 128};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
-// [rows][d] float32 accumulator, boxes of 32 rows x 32 columns (128 bytes),
-// 128-byte swizzle: the target of the dQ TMA reduce-adds.
-bool make_tmap_f32_acc(CUtensorMap* m, const void* base, long long rows, int d) {
+// [B*H][N][d] float32 accumulator viewed per head, boxes of 32 rows x 32
+// columns (128 bytes), 128-byte swizzle: the target of the dQ TMA reduce-adds.
+bool make_tmap_f32_acc(CUtensorMap* m, const void* base, int BH, int N, int d) {
   auto fn = encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 4};
-  cuuint32_t box[2] = {32, 32};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides,
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 4, static_cast<cuuint64_t>(N) * d * 4};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -72,7 +77,6 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 int check_shape(int B, int H, int N, int d) {
   if (B < 0 || H < 0 || N < 0) return FA_ERR_SHAPE;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED_D;
-  if (N % fa::kTile != 0) return FA_ERR_SHAPE;
   if (B == 0 || H == 0 || N == 0) return 1;
   const long long rows = static_cast<long long>(B) * H * N;
   if (rows >= (1LL << 31)) return FA_ERR_SHAPE;
@@ -121,12 +125,16 @@ struct WsLayout {
   size_t delta, lse2, dq_acc, counter, total;
 };
 
+// D and LSE2 are kept per head in N rounded up to 128 rows (Rp rows in all),
+// so that each 128-row tile of them is one aligned 512-byte block
 WsLayout ws_layout(int B, int H, int N, int d) {
   const size_t R = static_cast<size_t>(B) * H * N;
+  const size_t Np = (static_cast<size_t>(N) + fa::kTile - 1) / fa::kTile * fa::kTile;
+  const size_t Rp = static_cast<size_t>(B) * H * Np;
   WsLayout w;
   w.delta = 0;
-  w.lse2 = round_up(w.delta + 4 * R, 256);
-  w.dq_acc = round_up(w.lse2 + 4 * R, 256);
+  w.lse2 = round_up(w.delta + 4 * Rp, 256);
+  w.dq_acc = round_up(w.lse2 + 4 * Rp, 256);
   w.counter = round_up(w.dq_acc + 4 * R * d, 256);
   w.total = w.counter + 256;
   return w;
@@ -155,9 +163,9 @@ template <int D>
 int launch_fwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o, float* lse, int B,
                int H, int N, float scale, int causal, const uint8_t* block_mask,
                const int32_t* kv_len, uint8_t* visited, cudaStream_t stream, int num_sms) {
-  const long long rows = static_cast<long long>(B) * H * N;
   CUtensorMap tq, tk, tv;
-  if (!make_tmap(&tq, q, rows, D) || !make_tmap(&tk, k, rows, D) || !make_tmap(&tv, v, rows, D))
+  if (!make_tmap(&tq, q, B * H, N, D) || !make_tmap(&tk, k, B * H, N, D) ||
+      !make_tmap(&tv, v, B * H, N, D))
     return FA_ERR_CUDA;
   fa::FwdParams p;
   p.o = o;
@@ -168,7 +176,7 @@ int launch_fwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o,
   p.B = B;
   p.H = H;
   p.N = N;
-  p.n_t = N / fa::kTile;
+  p.n_t = (N + fa::kTile - 1) / fa::kTile;
   p.heads_per_group = heads_per_group(B * H, 4.0 * N * D);  // K and V
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * fa::kLog2e;
@@ -191,9 +199,10 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
   float* dq_acc = reinterpret_cast<float*>(ws + wl.dq_acc);
   int* counter = reinterpret_cast<int*>(ws + wl.counter);
   CUtensorMap tq, tk, tv, tdo, tdq, tdk, tdv;
-  if (!make_tmap(&tq, q, rows, D) || !make_tmap(&tk, k, rows, D) || !make_tmap(&tv, v, rows, D) ||
-      !make_tmap(&tdo, dout, rows, D) || !make_tmap_f32_acc(&tdq, dq_acc, rows, D) ||
-      !make_tmap(&tdk, dk, rows, D) || !make_tmap(&tdv, dv, rows, D))
+  const int BH = B * H;
+  if (!make_tmap(&tq, q, BH, N, D) || !make_tmap(&tk, k, BH, N, D) || !make_tmap(&tv, v, BH, N, D) ||
+      !make_tmap(&tdo, dout, BH, N, D) || !make_tmap_f32_acc(&tdq, dq_acc, BH, N, D) ||
+      !make_tmap(&tdk, dk, BH, N, D) || !make_tmap(&tdv, dv, BH, N, D))
     return FA_ERR_CUDA;
   static bool smem_set = false;
   if (!smem_set) {
@@ -203,11 +212,14 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
   // preprocess
   if (phases & 1u) {
     const int threads = 256;
+    const int Np = (N + fa::kTile - 1) / fa::kTile * fa::kTile;
+    const long long rows_p = static_cast<long long>(B) * H * Np;
     long long blocks = (rows * (D / 4) + threads - 1) / threads;
     const long long cap = static_cast<long long>(num_sms) * 8;
     if (blocks > cap) blocks = cap;
     fa::fa_bwd_pre_kernel<D><<<static_cast<int>(blocks), threads, 0, stream>>>(
-        o, dout, lse, delta, lse2, reinterpret_cast<float4*>(dq_acc), counter, rows);
+        o, dout, lse, delta, lse2, reinterpret_cast<float4*>(dq_acc), counter, N, Np, rows_p,
+        rows);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   // main
@@ -224,7 +236,7 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
     p.B = B;
     p.H = H;
     p.N = N;
-    p.n_t = N / fa::kTile;
+    p.n_t = (N + fa::kTile - 1) / fa::kTile;
     p.num_units = B * H * p.n_t;
     p.heads_per_group = heads_per_group(B * H, 8.0 * N * D);  // Q, dO, f32 dQ accumulator
     p.work_counter = counter;
@@ -265,7 +277,7 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
     sp.B = B;
     sp.H = H;
     sp.N = N;
-    sp.n_t = N / fa::kTile;
+    sp.n_t = (N + fa::kTile - 1) / fa::kTile;
     sp.num_units = B * H * sp.n_t;
     sp.heads_per_group = heads_per_group(B * H, 4.0 * N * D);  // K and V
     sp.causal = causal ? 1 : 0;

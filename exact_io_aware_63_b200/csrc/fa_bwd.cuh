@@ -52,6 +52,7 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const uint16_t* __restr
                                                          float* __restrict__ lse2,
                                                          float4* __restrict__ dq_acc,
                                                          int* __restrict__ work_counter,
+                                                         int N, int Np, long long rows_p,
                                                          long long rows) {
   // the main kernel's CTAs take work units from this counter
   if (blockIdx.x == 0 && threadIdx.x == 0) *work_counter = 0;
@@ -62,10 +63,17 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const uint16_t* __restr
   const int lane = threadIdx.x & 31;
   const int sub = lane / kLanesPerRow;
   const int part = lane % kLanesPerRow;
-  for (long long r0 = warp_global * kRowsPerWarp; r0 < rows; r0 += nwarps * kRowsPerWarp) {
-    const long long r = r0 + sub;
+  // D and LSE2 go to a per-head padded layout (Np = N rounded up to 128 rows
+  // per head) so that every 128-row tile of them starts 512-byte aligned;
+  // padding rows get -LSE2 = -inf (P = 0) and -D = 0
+  for (long long r0 = warp_global * kRowsPerWarp; r0 < rows_p; r0 += nwarps * kRowsPerWarp) {
+    const long long pr = r0 + sub;
+    const long long bh = pr / Np;
+    const int rr = static_cast<int>(pr - bh * Np);
+    const bool valid = pr < rows_p && rr < N;
+    const long long r = bh * N + rr;
     float acc = 0.f;
-    if (r < rows) {
+    if (valid) {
       const uint4 a = __ldg(reinterpret_cast<const uint4*>(o + r * D) + part);
       const uint4 b = __ldg(reinterpret_cast<const uint4*>(dout + r * D) + part);
       const uint32_t av[4] = {a.x, a.y, a.z, a.w};
@@ -81,10 +89,10 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const uint16_t* __restr
 #pragma unroll
     for (int off = kLanesPerRow / 2; off > 0; off >>= 1)
       acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (r < rows && part == 0) {
-      delta[r] = -acc;
-      const float l = lse[r];
-      lse2[r] = (l == -INFINITY) ? -INFINITY : -l * kLog2e;
+    if (pr < rows_p && part == 0) {
+      delta[pr] = valid ? -acc : 0.f;
+      const float l = valid ? lse[r] : -INFINITY;
+      lse2[pr] = (l == -INFINITY) ? -INFINITY : -l * kLog2e;
     }
   }
   const long long n4 = rows * (D / 4);
@@ -133,11 +141,11 @@ struct BwdCfg {
   static constexpr int kThreads = 512;
   // registers per thread: 128 at launch (512 x 128 = 65536), redistributed:
   //          producer/MMA   two dS warpgroups   dQ warpgroup
-  // D = 64:  128 x 104   +  256 x 136        +  128 x 112  = 62464
+  // D = 64:  128 x 104   +  256 x 144        +  128 x 112  = 64512
   // D = 128: 128 x 112   +  256 x 128        +  128 x 144  = 65536
   // (the dQ warpgroup holds a whole float32 dQ row)
   static constexpr uint32_t kRegsLaunch = 128, kRegsLow = (D == 64) ? 104 : 112;
-  static constexpr uint32_t kRegsDs = (D == 64) ? 136 : 128;
+  static constexpr uint32_t kRegsDs = (D == 64) ? 144 : 128;
   static constexpr uint32_t kRegsDq = (D == 64) ? 112 : 144;
   static constexpr int kTileBytes = kTile * D * 2;
   static constexpr int kBoxes = D / 64;
@@ -432,22 +440,26 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         ok = mbar_wait(kv_empty(skv), ((kv_cnt / KVS) & 1) ^ 1);
         if (!ok) break;
         ++kv_cnt;
-        const int krow = w.bh * p.N + w.j * kTile;
+        const int krow = w.j * kTile;  // within head w.bh
         const uint32_t kv_off = skv * Cfg::kKvSlotBytes;
         mbar_arrive_expect_tx(kv_full(skv), 2 * Cfg::kTileBytes);
         for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
-          tma_load_2d(sbase + Cfg::kOffK + kv_off + bx * 16384, &tm_k, bx * 64, krow, kv_full(skv));
-          tma_load_2d(sbase + Cfg::kOffV + kv_off + bx * 16384, &tm_v, bx * 64, krow, kv_full(skv));
+          tma_load_3d(sbase + Cfg::kOffK + kv_off + bx * 16384, &tm_k, bx * 64, krow, w.bh,
+                      kv_full(skv));
+          tma_load_3d(sbase + Cfg::kOffV + kv_off + bx * 16384, &tm_v, bx * 64, krow, w.bh,
+                      kv_full(skv));
         }
         for (int i = w.i_first; i < p.n_t && ok; i = bwd_next(p, w, i + 1)) {
-          const int qrow = w.bh * p.N + i * kTile;
+          // the tile's -LSE2 and -D rows (per-head padded layout: n_t * 128 rows
+          // per head, so the 512-byte block is aligned and stays in the head)
+          const long long qrow = (long long)w.bh * p.n_t * kTile + i * kTile;
           const int sq = q_cnt % QS;
           ok = mbar_wait(q_empty(sq), ((q_cnt / QS) & 1) ^ 1);
           if (!ok) break;
           mbar_arrive_expect_tx(q_full(sq), Cfg::kTileBytes + 2 * Cfg::kRowBytes);
           for (int bx = 0; bx < Cfg::kBoxes; ++bx)
-            tma_load_2d(sbase + Cfg::kOffQ + sq * Cfg::kTileBytes + bx * 16384, &tm_q, bx * 64,
-                        qrow, q_full(sq));
+            tma_load_3d(sbase + Cfg::kOffQ + sq * Cfg::kTileBytes + bx * 16384, &tm_q, bx * 64,
+                        i * kTile, w.bh, q_full(sq));
           bulk_load(sbase + Cfg::kOffRow + sq * Cfg::kRowBytes, p.lse2 + qrow, Cfg::kRowBytes,
                     q_full(sq));
           bulk_load(sbase + Cfg::kOffRow + (QS + sq) * Cfg::kRowBytes, p.delta + qrow,
@@ -458,8 +470,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
           if (!ok) break;
           mbar_arrive_expect_tx(do_full(so), Cfg::kTileBytes);
           for (int bx = 0; bx < Cfg::kBoxes; ++bx)
-            tma_load_2d(sbase + Cfg::kOffDO + so * Cfg::kTileBytes + bx * 16384, &tm_do, bx * 64,
-                        qrow, do_full(so));
+            tma_load_3d(sbase + Cfg::kOffDO + so * Cfg::kTileBytes + bx * 16384, &tm_do, bx * 64,
+                        i * kTile, w.bh, do_full(so));
           ++do_cnt;
         }
         if (*abort_flag) ok = false;
@@ -812,9 +824,12 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       const size_t krow = (size_t)w.bh * p.N + c_key;
       // warpgroup 0 writes the dK row, warpgroup 1 the dV row
       uint4* out_row = reinterpret_cast<uint4*>((h ? p.dv : p.dk) + krow * D);
+      // key rows of a partial last tile beyond N belong to no output
+      const bool key_row_ok = c_key < p.N;
       if (!w.any) {
 #pragma unroll
-        for (int c = 0; c < D / 8; ++c) out_row[c] = make_uint4(0, 0, 0, 0);
+        for (int c = 0; c < D / 8; ++c)
+          if (key_row_ok) out_row[c] = make_uint4(0, 0, 0, 0);
         continue;
       }
       const bool key_valid = c_key < w.L;
@@ -824,6 +839,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         const float4* lz4 = lse2_smem(sq) + h * 16;   // -LSE2
         const float4* dz4 = delta_smem(sq) + h * 16;  // -D
         const bool diag = p.causal && (i == w.j);
+        // a partial last query tile: queries >= q_lim lie beyond N (their Q and
+        // dO rows read as zero, their -LSE2 and -D entries are not theirs) and
+        // get P = dS = 0 by selection
+        const int q_lim = p.N - i * kTile;
+        const bool qtail = q_lim < kTile;
         ok = __all_sync(0xffffffffu, mbar_wait(s_full, s_cnt & 1));
         ++s_cnt;
         if (!ok) break;
@@ -878,11 +898,13 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
                 p2 = ex2_approx(x2);
                 p3 = ex2_approx(x3);
                 if (kKind == 1) {
+                  // allowed: the causal diagonal's c <= r (key kr, query q) and q < N
                   const int q0 = h * 64 + c * 32 + 4 * e4;  // query within the tile
-                  p0 = (kr > q0) ? 0.f : p0;
-                  p1 = (kr > q0 + 1) ? 0.f : p1;
-                  p2 = (kr > q0 + 2) ? 0.f : p2;
-                  p3 = (kr > q0 + 3) ? 0.f : p3;
+                  auto keep = [&](int q) { return (!diag || kr <= q) && q < q_lim; };
+                  p0 = keep(q0) ? p0 : 0.f;
+                  p1 = keep(q0 + 1) ? p1 : 0.f;
+                  p2 = keep(q0 + 2) ? p2 : 0.f;
+                  p3 = keep(q0 + 3) ? p3 : 0.f;
                 }
                 pk[2 * e4] = pack_bf16x2(p0, p1);
                 pk[2 * e4 + 1] = pack_bf16x2(p2, p3);
@@ -891,7 +913,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
             if (!key_valid) {
 #pragma unroll
               for (int e = 0; e < 16; ++e) pk[e] = 0u;
-            } else if (diag) {
+            } else if (diag || qtail) {
               make_p(std::integral_constant<int, 1>{});
             } else {
               make_p(std::integral_constant<int, 0>{});
@@ -938,6 +960,14 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
               float d0, d1, d2, d3;
               f2_unpack(f2_mul(ta, bf16x2_to_f2(pp[c * 16 + 2 * e4])), d0, d1);
               f2_unpack(f2_mul(tb, bf16x2_to_f2(pp[c * 16 + 2 * e4 + 1])), d2, d3);
+              if (qtail) {
+                // p = 0 there, but -D beyond N may be infinite: select, not multiply
+                const int q0 = h * 64 + c * 32 + 4 * e4;
+                d0 = (q0 < q_lim) ? d0 : 0.f;
+                d1 = (q0 + 1 < q_lim) ? d1 : 0.f;
+                d2 = (q0 + 2 < q_lim) ? d2 : 0.f;
+                d3 = (q0 + 3 < q_lim) ? d3 : 0.f;
+              }
               pk[2 * e4] = pack_bf16x2(d0, d1);
               pk[2 * e4 + 1] = pack_bf16x2(d2, d3);
             }
@@ -983,7 +1013,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
           if constexpr (Cfg::kEpiTma) {
             const int g = c * 4 + v4;  // 16-byte granule of the 128-byte row
             *reinterpret_cast<uint4*>(epi_row + ((g ^ (kr & 7)) << 4)) = val;
-          } else {
+          } else if (key_row_ok) {
             out_row[c * 4 + v4] = val;
           }
         }
@@ -999,7 +1029,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         if (kr == 0) {
           ok = mbar_wait(epi_ready(h), epi_cnt & 1);
           if (ok) {
-            tma_store_2d(h ? &tm_dv : &tm_dk, 0, w.bh * p.N + w.j * kTile,
+            tma_store_3d(h ? &tm_dv : &tm_dk, 0, w.j * kTile, w.bh,
                          smem_u32(smem + Cfg::kOffEpi + h * Cfg::kTileBytes));
             bulk_commit_group();
             bulk_wait_group_read0();
@@ -1045,7 +1075,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         for (int c = 0; c < D / 32; ++c) reg_fence32(r[c]);
         tc_fence_before();
         mbar_arrive(dq_empty);
-        const int y = w.bh * p.N + i * kTile + quarter * 32;
+        const int y = i * kTile + quarter * 32;  // row within head w.bh
 #pragma unroll
         for (int rd = 0; rd < Cfg::kDqRounds; ++rd) {
 #pragma unroll
@@ -1062,7 +1092,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
           if (lane == 0) {
 #pragma unroll
             for (int bxi = 0; bxi < Cfg::kDqBoxesPerRound; ++bxi)
-              tma_reduce_add_2d(&tm_dq, (rd * Cfg::kDqBoxesPerRound + bxi) * 32, y,
+              tma_reduce_add_3d(&tm_dq, (rd * Cfg::kDqBoxesPerRound + bxi) * 32, y, w.bh,
                                 stage_u32 + bxi * 4096);
             bulk_commit_group();
             bulk_wait_group_read0();

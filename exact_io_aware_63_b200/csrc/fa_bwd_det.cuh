@@ -141,28 +141,29 @@ __global__ void __launch_bounds__(DetCfg<D>::kThreads, 1)
         ok = mbar_wait(q_empty(qs), ((q_cnt / QS) & 1) ^ 1);
         if (!ok) break;
         ++q_cnt;
-        const int qrow = w.bh * p.N + w.i0 * kTile;
+        // the tile's -LSE2 and -D rows (per-head padded layout of the workspace)
+        const long long qrow = (long long)w.bh * p.n_t * kTile + w.i0 * kTile;
         mbar_arrive_expect_tx(q_full(qs), 2 * Cfg::kTileBytes + 2 * Cfg::kRowBytes);
         for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
-          tma_load_2d(q_tile(qs) + bx * 16384, &tm_q, bx * 64, qrow, q_full(qs));
-          tma_load_2d(do_tile(qs) + bx * 16384, &tm_do, bx * 64, qrow, q_full(qs));
+          tma_load_3d(q_tile(qs) + bx * 16384, &tm_q, bx * 64, w.i0 * kTile, w.bh, q_full(qs));
+          tma_load_3d(do_tile(qs) + bx * 16384, &tm_do, bx * 64, w.i0 * kTile, w.bh, q_full(qs));
         }
         bulk_load(rows_of(qs), dp.lse2 + qrow, Cfg::kRowBytes, q_full(qs));
         bulk_load(rows_of(qs) + Cfg::kRowBytes, dp.delta + qrow, Cfg::kRowBytes, q_full(qs));
         for (int j = fwd_next(p, w, 0); j < w.j_end && ok; j = fwd_next(p, w, j + 1)) {
           const int s = kv_cnt % S;
           const uint32_t ph = (kv_cnt / S) & 1;
-          const int krow = w.bh * p.N + j * kTile;
+          const int krow = j * kTile;  // within head w.bh
           ok = mbar_wait(k_empty(s), ph ^ 1);
           if (!ok) break;
           mbar_arrive_expect_tx(k_full(s), Cfg::kTileBytes);
           for (int bx = 0; bx < Cfg::kBoxes; ++bx)
-            tma_load_2d(k_tile(s) + bx * 16384, &tm_k, bx * 64, krow, k_full(s));
+            tma_load_3d(k_tile(s) + bx * 16384, &tm_k, bx * 64, krow, w.bh, k_full(s));
           ok = mbar_wait(v_empty(s), ph ^ 1);
           if (!ok) break;
           mbar_arrive_expect_tx(v_full(s), Cfg::kTileBytes);
           for (int bx = 0; bx < Cfg::kBoxes; ++bx)
-            tma_load_2d(v_tile(s) + bx * 16384, &tm_v, bx * 64, krow, v_full(s));
+            tma_load_3d(v_tile(s) + bx * 16384, &tm_v, bx * 64, krow, w.bh, v_full(s));
           ++kv_cnt;
         }
         if (*abort_flag) ok = false;
@@ -276,11 +277,13 @@ __global__ void __launch_bounds__(DetCfg<D>::kThreads, 1)
       ++q_cnt;
       const int row = w.i0 * kTile + r_local;  // query index within the head
       uint4* out_row = reinterpret_cast<uint4*>(dp.dq + ((size_t)w.bh * p.N + row) * D);
+      const bool row_ok = row < p.N;  // rows of a partial last tile beyond N: no output
       int j = fwd_next(p, w, 0);
       if (j >= w.j_end) {
         // no key visible to this query tile: dQ = 0 (Q and the rows are not read)
 #pragma unroll
-        for (int c = 0; c < D / 8; ++c) out_row[c] = make_uint4(0, 0, 0, 0);
+        for (int c = 0; c < D / 8; ++c)
+          if (row_ok) out_row[c] = make_uint4(0, 0, 0, 0);
         continue;
       }
       // this row's -LSE2 and -D (the slot is refilled only after the unit's
@@ -378,7 +381,9 @@ __global__ void __launch_bounds__(DetCfg<D>::kThreads, 1)
                               __uint_as_float(r[2 * e + 1]) * dp.scale);
 #pragma unroll
         for (int v4 = 0; v4 < 4; ++v4)
-          out_row[c * 4 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+          if (row_ok)
+            out_row[c * 4 + v4] =
+                make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
       }
       tc_fence_before();
     }

@@ -280,24 +280,24 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
         mbar_arrive_expect_tx(q_full(qs), nq * Cfg::kTileBytes);
         for (int x = 0; x < nq; ++x)
           for (int bx = 0; bx < Cfg::kBoxes; ++bx)
-            tma_load_2d(q_tile(qs, x) + bx * 16384, &tm_q, bx * 64,
-                        w.bh * p.N + (x ? w.i1 : w.i0) * kTile, q_full(qs));
+            tma_load_3d(q_tile(qs, x) + bx * 16384, &tm_q, bx * 64, (x ? w.i1 : w.i0) * kTile,
+                        w.bh, q_full(qs));
         for (int j = fwd_next(p, w, 0); j < w.j_end && ok; j = fwd_next(p, w, j + 1)) {
           const int s = kv_cnt % S;
           const uint32_t ph = (kv_cnt / S) & 1;
-          const int row = w.bh * p.N + j * kTile;
+          const int row = j * kTile;  // within head w.bh
           ok = mbar_wait(k_empty(s), ph ^ 1);
           if (!ok) break;
           mbar_arrive_expect_tx(k_full(s), Cfg::kTileBytes);
           for (int bx = 0; bx < Cfg::kBoxes; ++bx)
-            tma_load_2d(sbase + Cfg::kOffK + s * Cfg::kTileBytes + bx * 16384, &tm_k, bx * 64, row,
-                        k_full(s));
+            tma_load_3d(sbase + Cfg::kOffK + s * Cfg::kTileBytes + bx * 16384, &tm_k, bx * 64, row,
+                        w.bh, k_full(s));
           ok = mbar_wait(v_empty(s), ph ^ 1);
           if (!ok) break;
           mbar_arrive_expect_tx(v_full(s), Cfg::kTileBytes);
           for (int bx = 0; bx < Cfg::kBoxes; ++bx)
-            tma_load_2d(sbase + Cfg::kOffV + s * Cfg::kTileBytes + bx * 16384, &tm_v, bx * 64, row,
-                        v_full(s));
+            tma_load_3d(sbase + Cfg::kOffV + s * Cfg::kTileBytes + bx * 16384, &tm_v, bx * 64, row,
+                        w.bh, v_full(s));
           ++kv_cnt;
         }
         if (*abort_flag) ok = false;
@@ -825,6 +825,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
       }
       if (!ok) break;
       const size_t grow = (size_t)w.bh * p.N + row;
+      const bool row_ok = row < p.N;  // rows of a partial last tile beyond N are not output
       if constexpr (kPair) {
         // ---------------------------------------------------- epilogue (own tile)
         uint4* orow = reinterpret_cast<uint4*>(p.o + grow * D);
@@ -847,15 +848,17 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
                                   __uint_as_float(r[2 * e + 1]) * inv_l);
 #pragma unroll
             for (int v4 = 0; v4 < 4; ++v4)
-              orow[c * 4 + v4] =
-                  make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+              if (row_ok)
+                orow[c * 4 + v4] =
+                    make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
           }
           tc_fence_before();
-          p.lse[grow] = (l > 0.f) ? (m_used + log2f(l)) * kLn2 : -INFINITY;
+          if (row_ok) p.lse[grow] = (l > 0.f) ? (m_used + log2f(l)) * kLn2 : -INFINITY;
         } else {
 #pragma unroll
-          for (int c = 0; c < D / 8; ++c) orow[c] = make_uint4(0, 0, 0, 0);
-          p.lse[grow] = -INFINITY;
+          for (int c = 0; c < D / 8; ++c)
+            if (row_ok) orow[c] = make_uint4(0, 0, 0, 0);
+          if (row_ok) p.lse[grow] = -INFINITY;
         }
       } else {
         // ---------------------------------------------------- merge + epilogue
@@ -910,9 +913,11 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
           }
 #pragma unroll
           for (int v4 = 0; v4 < 4; ++v4)
-            orow[c * 4 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+            if (row_ok)
+              orow[c * 4 + v4] =
+                  make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
         }
-        if (x == 0) p.lse[grow] = (lt > 0.f) ? (m + log2f(lt)) * kLn2 : -INFINITY;
+        if (x == 0 && row_ok) p.lse[grow] = (lt > 0.f) ? (m + log2f(lt)) * kLn2 : -INFINITY;
         tc_fence_before();
         // neither warpgroup starts the next unit (whose first P V overwrites an O)
         // before both have read both partial outputs

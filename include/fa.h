@@ -10,7 +10,7 @@
  * every batch b and head h, with row r and key c:
  *
  *   allowed(r,c) = (!causal || c <= r) && (kv_len == NULL || c < kv_len[b])
- *                  && (block_mask == NULL || block_mask[(r/128)*(N/128) + c/128] != 0)
+ *                  && (block_mask == NULL || block_mask[(r/128)*nt + c/128] != 0)
  *   S_rc  = scale * <Q_r, K_c>  (allowed), -inf (otherwise)
  *   P_rc  = exp(S_rc - LSE_r),  LSE_r = ln sum_c exp(S_rc)
  *   O_r   = sum_c P_rc V_c
@@ -25,11 +25,13 @@
  *  - Tensors Q, K, V, O, dO, dQ, dK, dV are bfloat16 (raw 16-bit patterns,
  *    type fa_bf16), contiguous [B][H][N][d] in device memory, base address
  *    16-byte aligned.  LSE is float32 [B][H][N] (natural log), 4-byte aligned.
- *  - d is 64 or 128.  N is a multiple of 128.  B, H, N >= 0; if any is 0 the
+ *  - d is 64 or 128.  N is any length: tiles are 128 long, and when 128 does
+ *    not divide N the last tile is partial.  B, H, N >= 0; if any is 0 the
  *    call does nothing and returns FA_OK.  B*H*N must be below 2^31.
  *  - scale is finite and > 0 (1/sqrt(d) is the usual choice).
- *  - block_mask (nullable) is uint8 [N/128][N/128] in device memory, row =
- *    query tile, column = key tile, nonzero = keep; all (b, h) share it.
+ *  - block_mask (nullable) is uint8 [nt][nt] with nt = ceil(N/128), in device
+ *    memory, row = query tile, column = key tile, nonzero = keep; all (b, h)
+ *    share it; a last, partial tile's row and column cover its positions.
  *  - kv_len (nullable) is int32 [B] in device memory: keys c >= kv_len[b]
  *    are masked for every query of batch b.  Values must lie in [0, N];
  *    the kernels clamp values outside that range into it.
@@ -57,7 +59,7 @@ typedef enum {
     FA_OK = 0,
     FA_ERR_NULL = -1,           /* a required pointer is NULL */
     FA_ERR_ALIGN = -2,          /* a pointer breaks its alignment rule */
-    FA_ERR_SHAPE = -3,          /* negative size, N % 128 != 0, or B*H*N >= 2^31 */
+    FA_ERR_SHAPE = -3,          /* negative size, or B*H*N >= 2^31 */
     FA_ERR_UNSUPPORTED_D = -4,  /* d not in {64, 128} */
     FA_ERR_WORKSPACE = -5,      /* workspace NULL or smaller than fa_bwd_workspace_size */
     FA_ERR_CUDA = -6,           /* a CUDA runtime/driver call failed */
@@ -81,7 +83,7 @@ int fa_fwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o, flo
 
 /*
  * fa_fwd plus a record of the tiles it computed: visited (device, uint8
- * [B][H][N/128][N/128], zeroed by the caller) gets 1 at [b][h][i][j] for
+ * [B][H][nt][nt] (nt = ceil(N/128)), zeroed by the caller) gets 1 at [b][h][i][j] for
  * every (query tile i, key tile j) whose scores the kernel formed.  Same
  * kernel as fa_fwd; intended for tests of the tile-skip logic.
  */
@@ -91,9 +93,10 @@ int fa_fwd_traced(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16*
                   void* stream);
 
 /*
- * Bytes of device workspace fa_bwd needs: 4*B*H*N (D) + 4*B*H*N (LSE in
+ * Bytes of device workspace fa_bwd needs: 4*B*H*Np (D) + 4*B*H*Np (LSE in
  * base 2) + 4*B*H*N*d (float32 dQ accumulator) + 256 (the counter from which
- * the main kernel's CTAs take work units), each region 256-byte aligned.
+ * the main kernel's CTAs take work units), each region 256-byte aligned,
+ * where Np is N rounded up to a multiple of 128.
  * Returns 0 for an empty or invalid shape.
  */
 size_t fa_bwd_workspace_size(int B, int H, int N, int d);
@@ -117,7 +120,7 @@ int fa_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf16* 
 
 /*
  * fa_bwd plus a record of the tiles the main kernel computed: visited
- * (device, uint8 [B][H][N/128][N/128], zeroed by the caller) gets 1 at
+ * (device, uint8 [B][H][nt][nt] (nt = ceil(N/128)), zeroed by the caller) gets 1 at
  * [b][h][i][j] for every (query tile i, key tile j) it recomputed.
  */
 int fa_bwd_traced(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf16* o,

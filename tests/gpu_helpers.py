@@ -30,7 +30,7 @@ def to_dev(x):
 def run_gpu(x, backward=True, traced=False):
     q, k, v, do, bm, kl = to_dev(x)
     B, H, N, d = q.shape
-    n_t = N // 128
+    n_t = -(-N // 128)  # ceil: a last, partial tile counts
     out = {}
     vis_f = torch.zeros((B, H, n_t, n_t), dtype=torch.uint8, device=q.device) if traced else None
     o, lse = binding.attention_forward(q, k, v, x.scale, x.causal, bm, kl, visited=vis_f)

@@ -48,7 +48,8 @@ def test_workspace_size():
     ws = binding.fa_bwd_workspace_size(B, H, N, d)
     assert ws >= 4 * R + 4 * R + 4 * R * d
     assert ws % 256 == 0
-    assert binding.fa_bwd_workspace_size(1, 1, 100, 64) == 0      # N % 128
+    assert binding.fa_bwd_workspace_size(1, 1, 100, 64) >= 4 * 100 * 66   # any N >= 1
+    assert binding.fa_bwd_workspace_size(1, 1, -128, 64) == 0     # negative
     assert binding.fa_bwd_workspace_size(1, 1, 128, 96) == 0      # d
     assert binding.fa_bwd_workspace_size(0, 1, 128, 64) == 0      # empty
 
@@ -89,8 +90,8 @@ def bwd_det(**kw):
 
 @pytest.mark.parametrize("call", [fwd, bwd, bwd_det])
 def test_shape_errors(call):
-    assert call(N=100) == -3
     assert call(N=-128) == -3
+    assert call(N=-1) == -3
     assert call(B=-1) == -3
     assert call(B=1 << 16, H=1 << 8, N=1 << 8) == -3   # B*H*N >= 2^31
     assert call(d=96) == -4

@@ -48,6 +48,11 @@ def test_key_padding_against_oracle(cuda_device, d):
     _check_against_oracle(x)
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_partial_last_tile_against_oracle(cuda_device, d):
+    _check_against_oracle(inputs.make_inputs(2, 2, 300, d, causal=True, seed=330 + d))
+
+
 def test_block_mask_against_oracle(cuda_device):
     x = inputs.make_inputs(1, 2, 1024, 64, seed=320, block_keep=0.25)
     _check_against_oracle(x)

@@ -114,3 +114,29 @@ def test_large_scores(cuda_device):
     dq, dk, dv, _ = oracle.attention_backward(q, k, v, do, x.scale, x.causal, bm, kl)
     compare_grads({n: np.stack([f64(out[n][b, h]) for b, h in heads])[:, None]
                    for n in ("dq", "dk", "dv")}, {"dq": dq, "dk": dk, "dv": dv}, "large scores")
+
+
+# ---------------------------------------------------------------------------
+# sequence lengths that 128 does not divide: a last, partial tile
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1, 100, 200, 383])
+def test_partial_last_tile(cuda_device, d, causal, N):
+    # B * H > 1 so that a partial tile of one head sits next to the next head's rows
+    x = inputs.make_inputs(2, 2, N, d, causal=causal, seed=500 + N + d + int(causal))
+    check_all_heads(x)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_partial_last_tile_with_key_padding(cuda_device, d):
+    x = inputs.make_inputs(3, 2, 300, d, causal=True, seed=540 + d,
+                           kv_len=torch.tensor([300, 257, 129], dtype=torch.int32))
+    check_all_heads(x)
+
+
+def test_partial_last_tile_with_block_mask(cuda_device):
+    bm = torch.tensor([[1, 0, 1], [0, 1, 0], [1, 1, 1]], dtype=torch.uint8)
+    x = inputs.make_inputs(1, 3, 300, 64, seed=550, block_mask=bm)
+    check_all_heads(x)

@@ -43,6 +43,14 @@ def test_masks_small(cuda_device, causal):
     check(x)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_masks_partial_last_tile(cuda_device, causal):
+    # N = 700: five full tiles and a partial sixth
+    x = inputs.make_inputs(3, 2, 700, 64, causal=causal, seed=33, block_keep=0.3,
+                           kv_len=torch.tensor([1, 641, 700], dtype=torch.int32))
+    check(x)
+
+
 @pytest.mark.parametrize("name", ["bert", "gpt2"])
 def test_workloads(cuda_device, name):
     check(inputs.workload_inputs(name))
