@@ -68,10 +68,14 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const uint16_t* __restr
   // padding rows get -LSE2 = -inf (P = 0) and -D = 0
   for (long long r0 = warp_global * kRowsPerWarp; r0 < rows_p; r0 += nwarps * kRowsPerWarp) {
     const long long pr = r0 + sub;
-    const long long bh = pr / Np;
-    const int rr = static_cast<int>(pr - bh * Np);
-    const bool valid = pr < rows_p && rr < N;
-    const long long r = bh * N + rr;
+    long long r = pr;  // when 128 divides N the two layouts coincide
+    bool valid = pr < rows_p;
+    if (Np != N) {
+      const long long bh = pr / Np;
+      const int rr = static_cast<int>(pr - bh * Np);
+      valid = valid && rr < N;
+      r = bh * N + rr;
+    }
     float acc = 0.f;
     if (valid) {
       const uint4 a = __ldg(reinterpret_cast<const uint4*>(o + r * D) + part);
@@ -839,11 +843,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         const float4* lz4 = lse2_smem(sq) + h * 16;   // -LSE2
         const float4* dz4 = delta_smem(sq) + h * 16;  // -D
         const bool diag = p.causal && (i == w.j);
-        // a partial last query tile: queries >= q_lim lie beyond N (their Q and
-        // dO rows read as zero, their -LSE2 and -D entries are not theirs) and
-        // get P = dS = 0 by selection
-        const int q_lim = p.N - i * kTile;
-        const bool qtail = q_lim < kTile;
+        // A partial last query tile needs no mask: a query beyond N has Q and dO
+        // rows read as zero (so S = dP = 0) and padding entries -LSE2 = -inf,
+        // -D = 0, so P is 0 (or, on the polynomial path, clamped to about
+        // 2^-126) and dS = P * 0 = 0; its contributions P dO, dS Q and dS K are
+        // exactly zero and nothing in them can be infinite or NaN.
         ok = __all_sync(0xffffffffu, mbar_wait(s_full, s_cnt & 1));
         ++s_cnt;
         if (!ok) break;
@@ -898,13 +902,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
                 p2 = ex2_approx(x2);
                 p3 = ex2_approx(x3);
                 if (kKind == 1) {
-                  // allowed: the causal diagonal's c <= r (key kr, query q) and q < N
                   const int q0 = h * 64 + c * 32 + 4 * e4;  // query within the tile
-                  auto keep = [&](int q) { return (!diag || kr <= q) && q < q_lim; };
-                  p0 = keep(q0) ? p0 : 0.f;
-                  p1 = keep(q0 + 1) ? p1 : 0.f;
-                  p2 = keep(q0 + 2) ? p2 : 0.f;
-                  p3 = keep(q0 + 3) ? p3 : 0.f;
+                  p0 = (kr > q0) ? 0.f : p0;
+                  p1 = (kr > q0 + 1) ? 0.f : p1;
+                  p2 = (kr > q0 + 2) ? 0.f : p2;
+                  p3 = (kr > q0 + 3) ? 0.f : p3;
                 }
                 pk[2 * e4] = pack_bf16x2(p0, p1);
                 pk[2 * e4 + 1] = pack_bf16x2(p2, p3);
@@ -913,7 +915,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
             if (!key_valid) {
 #pragma unroll
               for (int e = 0; e < 16; ++e) pk[e] = 0u;
-            } else if (diag || qtail) {
+            } else if (diag) {
               make_p(std::integral_constant<int, 1>{});
             } else {
               make_p(std::integral_constant<int, 0>{});
@@ -960,14 +962,6 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
               float d0, d1, d2, d3;
               f2_unpack(f2_mul(ta, bf16x2_to_f2(pp[c * 16 + 2 * e4])), d0, d1);
               f2_unpack(f2_mul(tb, bf16x2_to_f2(pp[c * 16 + 2 * e4 + 1])), d2, d3);
-              if (qtail) {
-                // p = 0 there, but -D beyond N may be infinite: select, not multiply
-                const int q0 = h * 64 + c * 32 + 4 * e4;
-                d0 = (q0 < q_lim) ? d0 : 0.f;
-                d1 = (q0 + 1 < q_lim) ? d1 : 0.f;
-                d2 = (q0 + 2 < q_lim) ? d2 : 0.f;
-                d3 = (q0 + 3 < q_lim) ? d3 : 0.f;
-              }
               pk[2 * e4] = pack_bf16x2(d0, d1);
               pk[2 * e4 + 1] = pack_bf16x2(d2, d3);
             }
