@@ -9,14 +9,18 @@
 //   dQ = scale * dS K,  dK = scale * dS^T Q.
 //
 // Three launches:
-//   fa_bwd_pre_kernel    D and LSE*log2(e) per row; zero the f32 dQ accumulator
-//   fa_bwd_kernel        one CTA per (b, h, 128-key tile j), persistent
+//   fa_bwd_pre_kernel    -D and -LSE*log2(e) per row (per-head padded layout),
+//                        zero the f32 dQ accumulator and the work counter
+//   fa_bwd_kernel        persistent; a unit is (b, h, 128-key tile j)
 //   fa_bwd_dq_kernel     dQ = bf16(scale * accumulator)
 //
 // fa_bwd_kernel roles (16 warps):
-//   warp 0      TMA producer: K_j, V_j once per unit; per visited query tile
-//               Q_i with the tile's LSE*log2(e) and D rows (one ring) and
-//               dO_i (a second ring)
+//   warp 0      TMA producer: takes units from a counter shared by all CTAs,
+//               decodes each once and publishes it in a shared-memory ring
+//               for the other roles; loads K_j, V_j once per unit
+//               (double-buffered across units for D = 64) and per visited
+//               query tile Q_i with the tile's -LSE2 and -D rows (one ring)
+//               and dO_i (a second ring)
 //   warp 1      TMEM owner; MMA issuer (one thread).  D = 64: warps 1-3 each
 //               issue one share of the MMAs (S^T and dV / dP^T and dK / dQ)
 //   warps 4-11  two "dS" warpgroups, one key row per thread (TMEM lane), each
@@ -25,10 +29,11 @@
 //   warps 12-15 "dQ" group, one query row per thread: drains dQ partials from
 //               TMEM through shared memory into the float32 accumulator in
 //               HBM with TMA reduce-adds
-// Per visited query tile i the MMA thread issues, all accumulating in TMEM:
+// Per visited query tile i, all accumulating in TMEM:
 //   S^T  = K_j Q_i^T          (cols   0..127)
 //   dP^T = V_j dO_i^T         (cols 128..255)
-//   dV  += P^T dO_i           (A = P^T bf16 in TMEM over S^T's first 64 cols)
+//   dV  += P^T dO_i           (A = P^T bf16 in TMEM: its own cols 448..511 for
+//                             D = 64, over S^T's first 64 cols for D = 128)
 //   dK  += dS^T Q_i           (A = dS^T bf16 in TMEM over dP^T's first 64 cols)
 //   dQ   = dS K_j             (A = dS from shared memory; result in cols 384..447
 //                             for D = 64, over dP^T's cols 128..255 for D = 128)
@@ -44,8 +49,10 @@ namespace fa {
 // with no allowed key, so that exp2(s - LSE2) = 0), both stored NEGATED (the
 // main kernel adds them), and zero the dQ accumulator.
 // ---------------------------------------------------------------------------
+// Memory-bound: eight resident blocks per SM (at most 32 registers a thread)
+// keep enough loads in flight.
 template <int D>
-__global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const uint16_t* __restrict__ o,
+__global__ void __launch_bounds__(256, 8) fa_bwd_pre_kernel(const uint16_t* __restrict__ o,
                                                          const uint16_t* __restrict__ dout,
                                                          const float* __restrict__ lse,
                                                          float* __restrict__ delta,

@@ -10,13 +10,17 @@
 // score tile lives in on-chip memory only.
 //
 // B200 mapping (one persistent CTA per SM, 12 warps):
-//   warp 0      TMA producer: the unit's Q tile (double-buffered across
-//               units), then the K/V tiles it visits, through a kStages-deep
-//               mbarrier ring
-//   warp 1      MMA issuer (one thread): S = Q K^T and O += P V as tcgen05
-//               MMAs accumulating in tensor memory; owns the TMEM allocation
+//   warp 0      TMA producer: the unit's Q tile(s) (double-buffered across
+//               units where shared memory allows), then the K/V tiles it
+//               visits, through a kStages-deep mbarrier ring
+//   warp 1      owns the TMEM allocation; issues MMAs (one thread): for both
+//               warpgroups at D = 128, for warpgroup 0 at D = 64
+//   warp 2      D = 64: issues warpgroup 1's MMAs
 //   warps 4-7   softmax warpgroup 0 (TMEM lanes 0-127, one query row each)
 //   warps 8-11  softmax warpgroup 1
+// A single MMA-issuing thread beside eight busy softmax warps gets too few
+// issue slots to keep the tensor core fed, hence one issuer per warpgroup
+// where the layout allows it (D = 64).
 // Two ways of filling a work unit, chosen per launch:
 //  * pair mode (no block mask): the unit is (b, h, query tiles 2p and 2p+1).
 //    Both tiles visit the same key tiles (up to the causal diagonal), so
@@ -32,10 +36,16 @@
 // the other.
 //
 // TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 after it.
-// P (bf16) is written over the first 64 columns of its S tile and read from
-// there by the P V MMA.  tcgen05 MMAs issued by one thread execute in issue
-// order, which makes this aliasing safe: the next S MMA into the same
-// columns is issued after the P V MMA that reads them.
+// D = 64: P_0 [384,448), P_1 [448,512) (bf16, two per column).  Once all of
+// warpgroup x holds S_x in registers (s_free) its issuer issues the next
+// S_x, so S_x(j+1) runs while softmax(j) runs; the P V MMA signals p_free
+// once it has read P_x.  D = 128: no room for P, which is written over the
+// first 64 columns of its S tile; tcgen05 MMAs issued by one thread execute
+// in issue order, which makes this aliasing safe: the next S MMA into the
+// same columns is issued after the P V MMA that reads them.
+//
+// Rows of a partial last query tile beyond N are computed (their Q rows
+// load as zero) but not stored; keys beyond N are masked like key padding.
 //
 // Online softmax state per row (thread): m (running max, in units of
 // log2, scale folded in), l (running sum).  O is rescaled only when the row
