@@ -29,6 +29,10 @@ Functions (all arrays contiguous, float64 unless stated):
 * ``attention_backward_kv_cols(q, k, v, dout, cols, scale, causal, block_mask,
   kv_len_b)`` -> ``(dk_cols, dv_cols)``: dK and dV of chosen key columns of
   one head (a full pass over the head's rows).
+* ``attention_forward_dropout`` / ``attention_backward_dropout`` (extra
+  arguments ``p_drop, seed, offset``): the same with dropout on P; the mask is
+  ``dropout_keep(BH, N, p_drop, seed, offset)``, cut from Philox-4x32-10 draws
+  (``philox4x32_10(counter, key)``).
 * ``tile_visits(B, N, causal, block_mask, kv_len, T=128, i_begin=0,
   i_end=None)`` -> uint8 [B, i_end - i_begin, ceil(N / T)]: 1 where a
   (query tile, key tile) pair holds at least one allowed (row, key).
@@ -97,6 +101,25 @@ def _load():
             lib.oracle_tile_visits.argtypes = [
                 _u8p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _u8p, _i32p,
                 ctypes.c_int, ctypes.c_int]
+            _f = ctypes.c_float
+            lib.oracle_attention_forward_dropout.argtypes = [
+                _dp, _dp, _dp, _dp, _dp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                ctypes.c_double, ctypes.c_int, _u8p, _i32p, _f, ctypes.c_uint64, ctypes.c_uint32,
+                ctypes.c_int]
+            lib.oracle_attention_backward_dropout.argtypes = [
+                _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                ctypes.c_int, ctypes.c_double, ctypes.c_int, _u8p, _i32p, _f, ctypes.c_uint64,
+                ctypes.c_uint32, ctypes.c_int]
+            lib.oracle_dropout_keep.argtypes = [
+                _u8p, ctypes.POINTER(ctypes.c_uint16), ctypes.c_int, ctypes.c_int, _f,
+                ctypes.c_uint64, ctypes.c_uint32]
+            lib.oracle_philox4x32_10.argtypes = [
+                ctypes.POINTER(ctypes.c_uint32), ctypes.c_uint32, ctypes.c_uint32,
+                ctypes.POINTER(ctypes.c_uint32)]
+            lib.oracle_philox4x32_10.restype = None
+            for fn in (lib.oracle_attention_forward_dropout, lib.oracle_attention_backward_dropout,
+                       lib.oracle_dropout_keep):
+                fn.restype = ctypes.c_int
             for fn in (lib.oracle_attention_forward, lib.oracle_attention_backward,
                        lib.oracle_attention_forward_rows, lib.oracle_tile_visits,
                        lib.oracle_attention_backward_dq_rows,
@@ -154,6 +177,64 @@ def attention_backward(q, k, v, dout, scale, causal=False, block_mask=None, kv_l
     if rc != 0:
         raise RuntimeError(f"oracle_attention_backward failed: {rc}")
     return dq, dk, dv, delta
+
+
+def attention_forward_dropout(q, k, v, scale, p_drop, seed, offset=0, causal=False,
+                              block_mask=None, kv_len=None, nthreads=None):
+    """(o, lse) with dropout on P (keep mask from dropout_keep, kept entries scaled by
+    65536 / (65536 - floor(p_drop * 65536)))."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, N, d = q.shape
+    bm, kl = _mask_args(block_mask, kv_len)
+    o = np.empty_like(q)
+    lse = np.empty((B, H, N), np.float64)
+    rc = _load().oracle_attention_forward_dropout(
+        _ptr(q, _dp), _ptr(k, _dp), _ptr(v, _dp), _ptr(o, _dp), _ptr(lse, _dp), B, H, N, d,
+        float(scale), int(bool(causal)), _ptr(bm, _u8p), _ptr(kl, _i32p), float(p_drop),
+        int(seed), int(offset), _threads(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attention_forward_dropout failed: {rc}")
+    return o, lse
+
+
+def attention_backward_dropout(q, k, v, dout, scale, p_drop, seed, offset=0, causal=False,
+                               block_mask=None, kv_len=None, nthreads=None):
+    """(dq, dk, dv, delta) of sum(O * dO) for the dropout forward with the same mask."""
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, H, N, d = q.shape
+    bm, kl = _mask_args(block_mask, kv_len)
+    dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
+    delta = np.empty((B, H, N), np.float64)
+    rc = _load().oracle_attention_backward_dropout(
+        _ptr(q, _dp), _ptr(k, _dp), _ptr(v, _dp), _ptr(dout, _dp), _ptr(dq, _dp), _ptr(dk, _dp),
+        _ptr(dv, _dp), _ptr(delta, _dp), B, H, N, d, float(scale), int(bool(causal)),
+        _ptr(bm, _u8p), _ptr(kl, _i32p), float(p_drop), int(seed), int(offset),
+        _threads(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attention_backward_dropout failed: {rc}")
+    return dq, dk, dv, delta
+
+
+def dropout_keep(BH, N, p_drop, seed, offset=0):
+    """(keep uint8 [BH, N, N], draws uint16 [BH, N, N]): the dropout mask and the
+    16-bit draws it is cut from."""
+    keep = np.empty((BH, N, N), np.uint8)
+    draws = np.empty((BH, N, N), np.uint16)
+    rc = _load().oracle_dropout_keep(_ptr(keep, _u8p),
+                                     draws.ctypes.data_as(ctypes.POINTER(ctypes.c_uint16)),
+                                     BH, N, float(p_drop), int(seed), int(offset))
+    if rc != 0:
+        raise RuntimeError(f"oracle_dropout_keep failed: {rc}")
+    return keep, draws
+
+
+def philox4x32_10(counter, key):
+    """The four 32-bit output words of Philox-4x32-10 for a counter of four words and a
+    key of two."""
+    ctr = (ctypes.c_uint32 * 4)(*[int(c) & 0xFFFFFFFF for c in counter])
+    out = (ctypes.c_uint32 * 4)()
+    _load().oracle_philox4x32_10(ctr, int(key[0]) & 0xFFFFFFFF, int(key[1]) & 0xFFFFFFFF, out)
+    return [int(x) for x in out]
 
 
 def attention_forward_band(q, k, v, scale, causal=False, block_mask=None, kv_len=None,

@@ -52,10 +52,63 @@ typedef struct {
     const uint8_t *block_mask;
     const int32_t *kv_len;
     int backward;
+    int dropout;            /* keep mask Z and scale below apply (see dropout_keep) */
+    uint32_t drop_t;        /* drop when the element's 16-bit draw is below drop_t */
+    double drop_scale;      /* 65536 / (65536 - drop_t) */
+    uint32_t seed_lo, seed_hi, offset;
     int r_begin, r_end;     /* query rows computed in every head */
     int next_head;          /* shared work counter, guarded by lock */
     pthread_mutex_t lock;
 } oracle_job;
+
+/*
+ * Philox-4x32-10, the counter-based generator of Salmon, Moraes, Dror and
+ * Shaw, "Parallel Random Numbers: As Easy as 1, 2, 3" (SC 2011): ten rounds,
+ * each multiplying counter words 0 and 2 by the two round constants into
+ * 64-bit products and mixing their halves with words 1 and 3 and the key,
+ * the key being advanced by the two Weyl constants between rounds.
+ */
+static void philox4x32_10(const uint32_t ctr_in[4], uint32_t k0, uint32_t k1, uint32_t out[4])
+{
+    uint32_t c0 = ctr_in[0], c1 = ctr_in[1], c2 = ctr_in[2], c3 = ctr_in[3];
+    for (int round = 0; round < 10; ++round) {
+        const uint64_t p0 = (uint64_t)0xD2511F53u * c0;
+        const uint64_t p1 = (uint64_t)0xCD9E8D57u * c2;
+        const uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+        const uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+        const uint32_t n0 = hi1 ^ c1 ^ k0;
+        const uint32_t n2 = hi0 ^ c3 ^ k1;
+        c0 = n0; c1 = lo1; c2 = n2; c3 = lo0;
+        k0 += 0x9E3779B9u;
+        k1 += 0xBB67AE85u;
+    }
+    out[0] = c0; out[1] = c1; out[2] = c2; out[3] = c3;
+}
+
+/*
+ * Dropout draw for element (head bh, query r, key c): Philox-4x32-10 with
+ * counter (c / 8, r, bh, offset) and key (seed_lo, seed_hi) gives eight
+ * 16-bit values, for keys 8*(c/8) .. 8*(c/8)+7 in order (value k is the low
+ * half of word k/2 for even k, the high half for odd k).  The element is kept
+ * when its value is at least drop_t = floor(p * 65536).
+ */
+static uint32_t dropout_u16(int bh, int r, int c, uint32_t seed_lo, uint32_t seed_hi,
+                            uint32_t offset)
+{
+    const uint32_t ctr[4] = {(uint32_t)c >> 3, (uint32_t)r, (uint32_t)bh, offset};
+    uint32_t w[4];
+    philox4x32_10(ctr, seed_lo, seed_hi, w);
+    const int kk = c & 7;
+    return (w[kk >> 1] >> (16 * (kk & 1))) & 0xFFFFu;
+}
+
+/* Z_rc * scale for the job's dropout (1 without dropout). */
+static double dropout_weight(const oracle_job *job, int bh, int r, int c)
+{
+    if (!job->dropout) return 1.0;
+    const uint32_t u = dropout_u16(bh, r, c, job->seed_lo, job->seed_hi, job->offset);
+    return u >= job->drop_t ? job->drop_scale : 0.0;
+}
 
 /* The mask M(r,c) exactly as defined above. */
 static int allowed(int r, int c, int N, int causal, const uint8_t *block_mask, int L)
@@ -128,7 +181,8 @@ static void forward_head(const oracle_job *job, int bh, double *p)
         for (int c = 0; c < N; ++c) {
             if (p[c] == 0.0) continue;
             const double *vc = V + (size_t)c * d;
-            for (int x = 0; x < d; ++x) orow[x] += p[c] * vc[x];
+            const double pw = p[c] * dropout_weight(job, bh, r, c);
+            for (int x = 0; x < d; ++x) orow[x] += pw * vc[x];
         }
         lse[r] = m + log(l);
     }
@@ -156,27 +210,30 @@ static void backward_head(const oracle_job *job, int bh, double *p, double *dp)
             if (job->delta) job->delta[(size_t)bh * N + r] = 0.0;
             continue;
         }
-        /* dP_rc = dO_r . V_c and D_r = sum_c P_rc dP_rc */
+        /* With dropout O_r = sum_c P_rc W_rc V_c, W = Z * scale: by the chain rule
+           the gradient reaching P_rc is W_rc dP_rc with dP_rc = dO_r . V_c, and
+           D_r = sum_c P_rc W_rc dP_rc (= dO_r . O_r); without dropout W = 1. */
         double D = 0.0;
         for (int c = 0; c < N; ++c) {
             if (p[c] == 0.0) { dp[c] = 0.0; continue; }
             const double *vc = V + (size_t)c * d;
             double s = 0.0;
             for (int x = 0; x < d; ++x) s += dor[x] * vc[x];
-            dp[c] = s;
-            D += p[c] * s;
+            dp[c] = s * dropout_weight(job, bh, r, c);
+            D += p[c] * dp[c];
         }
         if (job->delta) job->delta[(size_t)bh * N + r] = D;
         for (int c = 0; c < N; ++c) {
             if (p[c] == 0.0) continue;
             const double ds = p[c] * (dp[c] - D);
+            const double pw = p[c] * dropout_weight(job, bh, r, c);
             const double *kc = K + (size_t)c * d;
             double *dkc = dK + (size_t)c * d;
             double *dvc = dV + (size_t)c * d;
             for (int x = 0; x < d; ++x) {
                 dqr[x] += job->scale * ds * kc[x];
                 dkc[x] += job->scale * ds * qr[x];
-                dvc[x] += p[c] * dor[x];
+                dvc[x] += pw * dor[x];
             }
         }
     }
@@ -284,6 +341,86 @@ int oracle_attention_backward(const double *q, const double *k, const double *v,
 {
     return oracle_attention_backward_band(q, k, v, dout, dq, dk, dv, delta, B, H, N, d, scale,
                                           causal, block_mask, kv_len, 0, N, nthreads);
+}
+
+/*
+ * Dropout (applied to P before P V, as the pages' fused operation lists
+ * dropout among the steps standard attention runs separately: [HF] "Standard
+ * Attention Algorithm"): the threshold is drop_t = floor(p_drop * 65536) taken
+ * in single precision (p_drop * 65536 is exact there), an element is kept when
+ * its 16-bit draw (dropout_u16) is >= drop_t, and kept entries are scaled by
+ * 65536 / (65536 - drop_t), which makes the expectation of P Z exactly P.
+ * LSE is the softmax's, unaffected by dropout.
+ */
+static int set_dropout(oracle_job *job, float p_drop, uint64_t seed, uint32_t offset)
+{
+    if (!(p_drop >= 0.0f && p_drop < 1.0f)) return -8;
+    job->dropout = 1;
+    job->drop_t = (uint32_t)(p_drop * 65536.0f);
+    job->drop_scale = 65536.0 / (65536.0 - (double)job->drop_t);
+    job->seed_lo = (uint32_t)seed;
+    job->seed_hi = (uint32_t)(seed >> 32);
+    job->offset = offset;
+    return 0;
+}
+
+int oracle_attention_forward_dropout(const double *q, const double *k, const double *v,
+                                     double *o, double *lse, int B, int H, int N, int d,
+                                     double scale, int causal, const uint8_t *block_mask,
+                                     const int32_t *kv_len, float p_drop, uint64_t seed,
+                                     uint32_t offset, int nthreads)
+{
+    oracle_job job;
+    memset(&job, 0, sizeof(job));
+    job.q = q; job.k = k; job.v = v; job.o = o; job.lse = lse;
+    job.B = B; job.H = H; job.N = N; job.d = d; job.scale = scale; job.causal = causal;
+    job.block_mask = block_mask; job.kv_len = kv_len; job.backward = 0;
+    job.r_begin = 0; job.r_end = N;
+    int rc = set_dropout(&job, p_drop, seed, offset);
+    return rc ? rc : run_job(&job, nthreads);
+}
+
+int oracle_attention_backward_dropout(const double *q, const double *k, const double *v,
+                                      const double *dout, double *dq, double *dk, double *dv,
+                                      double *delta, int B, int H, int N, int d, double scale,
+                                      int causal, const uint8_t *block_mask,
+                                      const int32_t *kv_len, float p_drop, uint64_t seed,
+                                      uint32_t offset, int nthreads)
+{
+    oracle_job job;
+    memset(&job, 0, sizeof(job));
+    job.q = q; job.k = k; job.v = v; job.dout = dout;
+    job.dq = dq; job.dk = dk; job.dv = dv; job.delta = delta;
+    job.B = B; job.H = H; job.N = N; job.d = d; job.scale = scale; job.causal = causal;
+    job.block_mask = block_mask; job.kv_len = kv_len; job.backward = 1;
+    job.r_begin = 0; job.r_end = N;
+    int rc = set_dropout(&job, p_drop, seed, offset);
+    return rc ? rc : run_job(&job, nthreads);
+}
+
+/* The dropout keep mask Z as uint8 [BH][N][N] (1 = kept), and raw 16-bit draws
+   as uint16 [BH][N][N] when draws is not NULL. */
+int oracle_dropout_keep(uint8_t *keep, uint16_t *draws, int BH, int N, float p_drop,
+                        uint64_t seed, uint32_t offset)
+{
+    oracle_job job;
+    memset(&job, 0, sizeof(job));
+    if (set_dropout(&job, p_drop, seed, offset)) return -8;
+    for (int bh = 0; bh < BH; ++bh)
+        for (int r = 0; r < N; ++r)
+            for (int c = 0; c < N; ++c) {
+                const uint32_t u = dropout_u16(bh, r, c, job.seed_lo, job.seed_hi, offset);
+                const size_t i = ((size_t)bh * N + r) * N + c;
+                keep[i] = (uint8_t)(u >= job.drop_t);
+                if (draws) draws[i] = (uint16_t)u;
+            }
+    return 0;
+}
+
+/* Philox-4x32-10 itself, for the tests: out = philox(counter, key). */
+void oracle_philox4x32_10(const uint32_t counter[4], uint32_t k0, uint32_t k1, uint32_t out[4])
+{
+    philox4x32_10(counter, k0, k1, out);
 }
 
 /*

@@ -424,3 +424,111 @@ def test_row_bands_partition_the_full_result():
     np.testing.assert_array_equal(g2[0][:, :, 150:], dq[:, :, 150:])
     np.testing.assert_allclose(g1[1] + g2[1], dk, atol=1e-13)
     np.testing.assert_allclose(g1[2] + g2[2], dv, atol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# dropout (the pages list dropout among the steps the fused kernel absorbs:
+# [HF] "Standard Attention Algorithm"); the mask comes from Philox-4x32-10
+# ---------------------------------------------------------------------------
+
+def test_dropout_with_zero_probability_is_plain_attention():
+    q, k, v, do = (rand((1, 2, 96, 8), t) for t in (60, 61, 62, 63))
+    kvl = np.array([70], np.int32)
+    o, l = oracle.attention_forward(q, k, v, 0.3, causal=True, kv_len=kvl)
+    od, ld = oracle.attention_forward_dropout(q, k, v, 0.3, 0.0, seed=5, causal=True, kv_len=kvl)
+    assert np.array_equal(o, od) and np.array_equal(l, ld)
+    g = oracle.attention_backward(q, k, v, do, 0.3, causal=True, kv_len=kvl)
+    gd = oracle.attention_backward_dropout(q, k, v, do, 0.3, 0.0, seed=5, causal=True, kv_len=kvl)
+    for a, b in zip(g, gd):
+        assert np.array_equal(a, b)
+
+
+def test_philox_is_a_bijection_of_the_counter():
+    # each round is invertible for a fixed key, so distinct counters never collide
+    outs = {tuple(oracle.philox4x32_10([i, i >> 3, 7, 1], [11, 13])) for i in range(4096)}
+    assert len(outs) == 4096
+
+
+def test_dropout_draws_are_uniform_16_bit_values():
+    _, u = oracle.dropout_keep(4, 256, 0.0, seed=0x1234567890ABCDEF, offset=3)
+    x = u.astype(np.float64).ravel()
+    n = x.size
+    mu, sd = 32767.5, 65536 / math.sqrt(12)
+    assert abs(x.mean() - mu) < 5 * sd / math.sqrt(n)
+    assert abs(x.std() - sd) < 0.01 * sd
+    # top bytes: chi-square with 255 degrees of freedom, far inside 5 standard deviations
+    counts = np.bincount((u.ravel() >> 8).astype(np.int64), minlength=256)
+    e = n / 256
+    chi2 = float(((counts - e) ** 2 / e).sum())
+    assert abs(chi2 - 255) < 5 * math.sqrt(2 * 255)
+    # neighbours along keys and along queries are uncorrelated
+    for a, b in ((u[:, :, :-1], u[:, :, 1:]), (u[:, :-1, :], u[:, 1:, :])):
+        r = np.corrcoef(a.ravel().astype(np.float64), b.ravel().astype(np.float64))[0, 1]
+        assert abs(r) < 5 / math.sqrt(a.size)
+
+
+@pytest.mark.parametrize("p", [0.1, 0.5, 0.9])
+def test_dropout_keep_fraction(p):
+    keep, u = oracle.dropout_keep(2, 256, p, seed=99)
+    t = int(np.float32(p) * np.float32(65536.0))
+    assert np.array_equal(keep, (u >= t).astype(np.uint8))
+    n = keep.size
+    q_keep = 1 - t / 65536
+    assert abs(keep.mean() - q_keep) < 5 * math.sqrt(q_keep * (1 - q_keep) / n)
+    # another seed or offset draws another mask: disagreement 2 q (1 - q) on average
+    k2, _ = oracle.dropout_keep(2, 256, p, seed=100)
+    k3, _ = oracle.dropout_keep(2, 256, p, seed=99, offset=1)
+    for other in (k2, k3):
+        dis = (keep != other).mean()
+        exp = 2 * q_keep * (1 - q_keep)
+        assert abs(dis - exp) < 5 * math.sqrt(exp * (1 - exp) / n)
+
+
+def test_dropout_zero_query_closed_form():
+    # Q = 0: P is uniform over the allowed keys, so O_r = w / count * sum of kept V rows
+    B, H, N, d, p = 1, 2, 200, 8, 0.3
+    q = np.zeros((B, H, N, d))
+    k, v = rand((B, H, N, d), 64), rand((B, H, N, d), 65)
+    kvl = np.array([150], np.int32)
+    o, l = oracle.attention_forward_dropout(q, k, v, 0.5, p, seed=21, offset=4, causal=True,
+                                            kv_len=kvl)
+    keep, _ = oracle.dropout_keep(B * H, N, p, seed=21, offset=4)
+    t = int(np.float32(p) * np.float32(65536.0))
+    w = 65536.0 / (65536.0 - t)
+    for h in range(H):
+        for r in [0, 1, 77, 149, 150, 199]:
+            keys = [c for c in range(N) if c <= r and c < 150]
+            kept = [c for c in keys if keep[h, r, c]]
+            want = w * v[0, h, kept].sum(axis=0) / len(keys)
+            np.testing.assert_allclose(o[0, h, r], want, atol=1e-13)
+            assert abs(l[0, h, r] - math.log(len(keys))) < 1e-13
+
+
+@pytest.mark.parametrize("causal,kv", [(False, None), (True, 11)])
+def test_dropout_finite_difference_gradients(causal, kv):
+    # the mask depends on (seed, offset, head, row, key) only, so L = sum(O * dO) is a
+    # smooth function of q, k, v and its central differences give the gradients
+    B, H, N, d, scale, p = 1, 1, 16, 8, 0.4, 0.35
+    q, k, v, do = (rand((B, H, N, d), t) for t in (70, 71, 72, 73))
+    kvl = None if kv is None else np.array([kv], np.int32)
+    dq, dk, dv, _ = oracle.attention_backward_dropout(q, k, v, do, scale, p, seed=3,
+                                                      causal=causal, kv_len=kvl)
+
+    def loss(qq, kk, vv):
+        o, _ = oracle.attention_forward_dropout(qq, kk, vv, scale, p, seed=3, causal=causal,
+                                                kv_len=kvl)
+        return float((o * do).sum())
+
+    h = 1e-6
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args = {"q": (q, k, v), "k": (q, k, v), "v": (q, k, v)}[name]
+            a_p = [xp if n == name else t for n, t in zip("qkv", args)]
+            a_m = [xm if n == name else t for n, t in zip("qkv", args)]
+            num[idx] = (loss(*a_p) - loss(*a_m)) / (2 * h)
+        err = np.linalg.norm(num - g) / np.linalg.norm(g)
+        assert err < 1e-7, (name, err)
