@@ -241,12 +241,38 @@ def run_ours(args):
         if rc != 0:
             raise RuntimeError(f"{what}: {binding.fa_status_string(rc)}")
 
+    drop = args.dropout
+    seed, offset = 0x5EED, 0
+
+    def fwd_call():
+        if drop > 0:
+            return binding.fa_fwd_dropout(q, k, v, o, lse, B, H, N, d, scale, causal, bm, kl, drop,
+                                          seed, offset, S)
+        return binding.fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, bm, kl, S)
+
+    def bwd_call():
+        if drop > 0:
+            return binding.fa_bwd_dropout(q, k, v, o, lse, do, dq, dk, dv, B, H, N, d, scale,
+                                          causal, bm, kl, drop, seed, offset, ws, ws_bytes, S)
+        bwd = binding.fa_bwd_deterministic if args.deterministic else binding.fa_bwd
+        return bwd(q, k, v, o, lse, do, dq, dk, dv, B, H, N, d, scale, causal, bm, kl, ws,
+                   ws_bytes, S)
+
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        check(binding.fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, bm, kl, S), "fa_fwd")
+        check(fwd_call(), "forward")
         if ev is not None:
             ev[1].record(stream)
+        if drop > 0:
+            # one call, three kernels: timed together as the "main" interval
+            if ev is not None:
+                ev[2].record(stream)
+            check(bwd_call(), "fa_bwd_dropout")
+            if ev is not None:
+                ev[3].record(stream)
+                ev[4].record(stream)
+            return
         # fa_bwd is phases 0, 1, 2; fa_bwd_deterministic is 0, 1, 3
         for i, ph in enumerate((0, 1, 3) if args.deterministic else (0, 1, 2)):
             check(binding.fa_bwd_phase(ph, q, k, v, o, lse, do, dq, dk, dv, B, H, N, d, scale,
@@ -323,10 +349,8 @@ def run_ours(args):
             k.copy_(hk, non_blocking=True)
             v.copy_(hv, non_blocking=True)
             do.copy_(hdo, non_blocking=True)
-            check(binding.fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, bm, kl, S), "fa_fwd")
-            bwd = binding.fa_bwd_deterministic if args.deterministic else binding.fa_bwd
-            check(bwd(q, k, v, o, lse, do, dq, dk, dv, B, H, N, d, scale, causal, bm, kl,
-                      ws, ws_bytes, S), "fa_bwd")
+            check(fwd_call(), "forward")
+            check(bwd_call(), "backward")
             ho.copy_(o, non_blocking=True)
             hlse.copy_(lse, non_blocking=True)
             hdq.copy_(dq, non_blocking=True)
@@ -375,7 +399,10 @@ def run_ours(args):
                    "flop_density": density(x), "seed": w.seed,
                    "l2": "flushed between timed steps (256 MiB write)",
                    "parallelism": f"replica x{world}",
-                   "backward": "fa_bwd_deterministic" if args.deterministic else "fa_bwd"},
+                   "backward": ("fa_bwd_dropout (its three kernels timed together as bwd_main)"
+                                if drop > 0 else "fa_bwd_deterministic" if args.deterministic
+                                else "fa_bwd"),
+                   "dropout": drop},
         "fwd_tflops": fwd_tflops,
         "bwd_tflops": bwd_tflops,
         "fwd_bwd_pct_of_peak": per_gpu / peaks["bf16_tflops"],
@@ -389,7 +416,7 @@ def run_ours(args):
         "gpu_launches": 4 * args.steps,
         "clocks": clocks,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and drop == 0:
         line["cpu_baseline"] = cpu_baseline(x, budget_s=args.cpu_budget)
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -649,6 +676,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--deterministic", action="store_true",
                     help="time fa_bwd_deterministic (ordered dQ kernel) instead of fa_bwd")
+    ap.add_argument("--dropout", type=float, default=0.0,
+                    help="time fa_fwd_dropout / fa_bwd_dropout with this probability")
     ap.add_argument("--vs-standard", action="store_true",
                     help="instead of the benchmark line, compare one step with standard "
                          "attention (S and P materialised) on the same inputs")

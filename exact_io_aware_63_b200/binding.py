@@ -31,6 +31,8 @@ _vp = ctypes.c_void_p
 _i = ctypes.c_int
 _f = ctypes.c_float
 _sz = ctypes.c_size_t
+_u64 = ctypes.c_uint64
+_u32 = ctypes.c_uint32
 
 _SIGS = {
     "fa_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _vp, _vp]),
@@ -41,6 +43,9 @@ _SIGS = {
     "fa_bwd_phase": (_i, [_i] + [_vp] * 9 + [_i, _i, _i, _i, _f, _i, _vp, _vp, _vp, _sz, _vp]),
     "fa_bwd_noalloc": (_i, [_vp] * 9 + [_i, _i, _i, _i, _f, _i, _vp, _vp, _vp]),
     "fa_bwd_deterministic": (_i, [_vp] * 9 + [_i, _i, _i, _i, _f, _i, _vp, _vp, _vp, _sz, _vp]),
+    "fa_fwd_dropout": (_i, [_vp] * 5 + [_i, _i, _i, _i, _f, _i, _vp, _vp, _f, _u64, _u32, _vp]),
+    "fa_bwd_dropout": (_i, [_vp] * 9 + [_i, _i, _i, _i, _f, _i, _vp, _vp, _f, _u64, _u32, _vp,
+                                        _sz, _vp]),
     "fa_get_device_status": (_i, [_vp]),
     "fa_status_string": (ctypes.c_char_p, [_i]),
     "fa_version": (_i, []),
@@ -167,6 +172,24 @@ def fa_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal,
                                  _stream(stream))
 
 
+def fa_fwd_dropout(q, k, v, o, lse, B, H, N, d, scale, causal, block_mask, kv_len, p_drop, seed,
+                   offset, stream=None):
+    """fa_fwd with dropout of probability p_drop on P (Philox keep mask, include/fa.h)."""
+    return load().fa_fwd_dropout(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
+                                 float(scale), int(bool(causal)), _ptr(block_mask), _ptr(kv_len),
+                                 float(p_drop), int(seed), int(offset), _stream(stream))
+
+
+def fa_bwd_dropout(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, block_mask,
+                   kv_len, p_drop, seed, offset, workspace, workspace_bytes, stream=None):
+    """fa_bwd for the output of fa_fwd_dropout with the same p_drop, seed and offset."""
+    return load().fa_bwd_dropout(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
+                                 _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, float(scale),
+                                 int(bool(causal)), _ptr(block_mask), _ptr(kv_len),
+                                 float(p_drop), int(seed), int(offset), _ptr(workspace),
+                                 int(workspace_bytes), _stream(stream))
+
+
 def fa_get_device_status(stream=None):
     return load().fa_get_device_status(_stream(stream))
 
@@ -189,13 +212,20 @@ def _check(rc, what):
 
 
 def attention_forward(q, k, v, scale, causal=False, block_mask=None, kv_len=None, visited=None,
-                      stream=None):
-    """O, LSE for bf16 CUDA tensors q, k, v of shape [B, H, N, d]."""
+                      stream=None, dropout=None):
+    """O, LSE for bf16 CUDA tensors q, k, v of shape [B, H, N, d].  ``dropout`` is None or
+    (p_drop, seed, offset) and selects fa_fwd_dropout."""
     import torch
     B, H, N, d = q.shape
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    if visited is None:
+    if dropout is not None:
+        if visited is not None:
+            raise ValueError("the dropout forward has no traced variant")
+        p_drop, seed, offset = dropout
+        rc = fa_fwd_dropout(q, k, v, o, lse, B, H, N, d, scale, causal, block_mask, kv_len,
+                            p_drop, seed, offset, stream)
+    elif visited is None:
         rc = fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, block_mask, kv_len, stream)
     else:
         rc = fa_fwd_traced(q, k, v, o, lse, B, H, N, d, scale, causal, block_mask, kv_len,
@@ -205,16 +235,25 @@ def attention_forward(q, k, v, scale, causal=False, block_mask=None, kv_len=None
 
 
 def attention_backward(q, k, v, o, lse, dout, scale, causal=False, block_mask=None, kv_len=None,
-                       workspace=None, visited=None, stream=None, deterministic=False):
+                       workspace=None, visited=None, stream=None, deterministic=False,
+                       dropout=None):
     """dQ, dK, dV for the forward that produced (o, lse).  ``deterministic`` selects
-    fa_bwd_deterministic (bitwise-reproducible dQ)."""
+    fa_bwd_deterministic (bitwise-reproducible dQ); ``dropout`` = (p_drop, seed, offset),
+    the forward's, selects fa_bwd_dropout."""
     import torch
     B, H, N, d = q.shape
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws_bytes = fa_bwd_workspace_size(B, H, N, d)
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
-    if deterministic:
+    if dropout is not None:
+        if visited is not None or deterministic:
+            raise ValueError("the dropout backward has no traced or deterministic variant")
+        p_drop, seed, offset = dropout
+        rc = fa_bwd_dropout(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal,
+                            block_mask, kv_len, p_drop, seed, offset, workspace,
+                            workspace.numel(), stream)
+    elif deterministic:
         if visited is not None:
             raise ValueError("the deterministic backward has no traced variant")
         rc = fa_bwd_deterministic(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal,

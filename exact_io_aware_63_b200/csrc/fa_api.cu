@@ -140,19 +140,49 @@ WsLayout ws_layout(int B, int H, int N, int d) {
   return w;
 }
 
-template <int D, bool kPair>
+// Dropout arguments after validation: the threshold on the 16-bit draws and
+// the weight of kept entries (see FwdParams).
+struct DropArgs {
+  bool on = false;
+  uint32_t t = 0;
+  float w = 1.f;
+  uint32_t seed_lo = 0, seed_hi = 0, offset = 0;
+};
+
+int make_drop(float p_drop, uint64_t seed, uint32_t offset, DropArgs* d) {
+  if (!(p_drop >= 0.f && p_drop < 1.f)) return FA_ERR_ARG;
+  d->on = true;
+  d->t = static_cast<uint32_t>(p_drop * 65536.0f);  // exact product, truncated
+  d->w = 65536.0f / (65536.0f - static_cast<float>(d->t));
+  d->seed_lo = static_cast<uint32_t>(seed);
+  d->seed_hi = static_cast<uint32_t>(seed >> 32);
+  d->offset = offset;
+  return FA_OK;
+}
+
+template <typename P>
+void set_drop(P& p, const DropArgs& dr) {
+  p.drop_t = dr.t;
+  p.drop_w = dr.w;
+  p.seed_lo = dr.seed_lo;
+  p.seed_hi = dr.seed_hi;
+  p.drop_offset = dr.offset;
+}
+
+template <int D, bool kPair, bool kDrop>
 int launch_fwd_mode(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                     fa::FwdParams& p, cudaStream_t stream, int num_sms) {
   using Cfg = fa::FwdCfg<D, kPair>;
   static bool smem_set = false;
   if (!smem_set) {
-    if (!set_smem(fa::fa_fwd_kernel<D, kPair>, Cfg::kSmemBytes)) return FA_ERR_CUDA;
+    if (!set_smem(fa::fa_fwd_kernel<D, kPair, kDrop>, Cfg::kSmemBytes)) return FA_ERR_CUDA;
     smem_set = true;
   }
   const int per_head = kPair ? (p.n_t + 1) / 2 : p.n_t;
   p.num_units = p.B * p.H * per_head;
   const int grid = p.num_units < num_sms ? p.num_units : num_sms;
-  fa::fa_fwd_kernel<D, kPair><<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(tq, tk, tv, p);
+  fa::fa_fwd_kernel<D, kPair, kDrop>
+      <<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -162,7 +192,8 @@ int launch_fwd_mode(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensor
 template <int D>
 int launch_fwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o, float* lse, int B,
                int H, int N, float scale, int causal, const uint8_t* block_mask,
-               const int32_t* kv_len, uint8_t* visited, cudaStream_t stream, int num_sms) {
+               const int32_t* kv_len, uint8_t* visited, cudaStream_t stream, int num_sms,
+               const DropArgs& dr) {
   CUtensorMap tq, tk, tv;
   if (!make_tmap(&tq, q, B * H, N, D) || !make_tmap(&tk, k, B * H, N, D) ||
       !make_tmap(&tv, v, B * H, N, D))
@@ -180,8 +211,13 @@ int launch_fwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o,
   p.heads_per_group = heads_per_group(B * H, 4.0 * N * D);  // K and V
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * fa::kLog2e;
-  if (block_mask) return launch_fwd_mode<D, false>(tq, tk, tv, p, stream, num_sms);
-  return launch_fwd_mode<D, true>(tq, tk, tv, p, stream, num_sms);
+  set_drop(p, dr);
+  if (dr.on) {
+    if (block_mask) return launch_fwd_mode<D, false, true>(tq, tk, tv, p, stream, num_sms);
+    return launch_fwd_mode<D, true, true>(tq, tk, tv, p, stream, num_sms);
+  }
+  if (block_mask) return launch_fwd_mode<D, false, false>(tq, tk, tv, p, stream, num_sms);
+  return launch_fwd_mode<D, true, false>(tq, tk, tv, p, stream, num_sms);
 }
 
 template <int D>
@@ -189,7 +225,7 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
                const float* lse, const fa_bf16* dout, fa_bf16* dq, fa_bf16* dk, fa_bf16* dv, int B,
                int H, int N, float scale, int causal, const uint8_t* block_mask,
                const int32_t* kv_len, void* workspace, uint8_t* visited, cudaStream_t stream,
-               int num_sms, unsigned phases) {
+               int num_sms, unsigned phases, const DropArgs& dr) {
   using Cfg = fa::BwdCfg<D>;
   const long long rows = static_cast<long long>(B) * H * N;
   const WsLayout wl = ws_layout(B, H, N, D);
@@ -206,7 +242,9 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
     return FA_ERR_CUDA;
   static bool smem_set = false;
   if (!smem_set) {
-    if (!set_smem(fa::fa_bwd_kernel<D>, Cfg::kSmemBytes)) return FA_ERR_CUDA;
+    if (!set_smem(fa::fa_bwd_kernel<D, false>, Cfg::kSmemBytes) ||
+        !set_smem(fa::fa_bwd_kernel<D, true>, Cfg::kSmemBytes))
+      return FA_ERR_CUDA;
     smem_set = true;
   }
   // preprocess
@@ -243,9 +281,14 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
     p.causal = causal ? 1 : 0;
     p.scale = scale;
     p.scale_log2 = scale * fa::kLog2e;
+    set_drop(p, dr);
     const int grid = p.num_units < num_sms ? p.num_units : num_sms;
-    fa::fa_bwd_kernel<D>
-        <<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdq, tdk, tdv, p);
+    if (dr.on)
+      fa::fa_bwd_kernel<D, true>
+          <<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdq, tdk, tdv, p);
+    else
+      fa::fa_bwd_kernel<D, false>
+          <<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdq, tdk, tdv, p);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   // dQ
@@ -296,7 +339,8 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
 
 int fwd_impl(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o, float* lse, int B,
              int H, int N, int d, float scale, int causal, const uint8_t* block_mask,
-             const int32_t* kv_len, uint8_t* visited, void* stream) {
+             const int32_t* kv_len, uint8_t* visited, void* stream,
+             const DropArgs& dr = DropArgs()) {
   int rc = check_shape(B, H, N, d);
   if (rc == 1) return FA_OK;
   if (rc != FA_OK) return rc;
@@ -311,16 +355,16 @@ int fwd_impl(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o, f
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (d == 64)
     return launch_fwd<64>(q, k, v, o, lse, B, H, N, scale, causal, block_mask, kv_len, visited, s,
-                          sms);
+                          sms, dr);
   return launch_fwd<128>(q, k, v, o, lse, B, H, N, scale, causal, block_mask, kv_len, visited, s,
-                         sms);
+                         sms, dr);
 }
 
 int bwd_impl(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf16* o,
              const float* lse, const fa_bf16* dout, fa_bf16* dq, fa_bf16* dk, fa_bf16* dv, int B,
              int H, int N, int d, float scale, int causal, const uint8_t* block_mask,
              const int32_t* kv_len, void* workspace, size_t workspace_bytes, uint8_t* visited,
-             void* stream, unsigned phases = 7u) {
+             void* stream, unsigned phases = 7u, const DropArgs& dr = DropArgs()) {
   int rc = check_shape(B, H, N, d);
   if (rc == 1) return FA_OK;
   if (rc != FA_OK) return rc;
@@ -339,9 +383,9 @@ int bwd_impl(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf16
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (d == 64)
     return launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, scale, causal, block_mask,
-                          kv_len, workspace, visited, s, sms, phases);
+                          kv_len, workspace, visited, s, sms, phases, dr);
   return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, scale, causal, block_mask,
-                         kv_len, workspace, visited, s, sms, phases);
+                         kv_len, workspace, visited, s, sms, phases, dr);
 }
 
 }  // namespace
@@ -405,6 +449,29 @@ int fa_bwd_deterministic(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, c
                   workspace, workspace_bytes, nullptr, stream, 1u | 2u | 8u);
 }
 
+int fa_fwd_dropout(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o, float* lse,
+                   int B, int H, int N, int d, float scale, int causal, const uint8_t* block_mask,
+                   const int32_t* kv_len, float p_drop, uint64_t seed, uint32_t offset,
+                   void* stream) {
+  DropArgs dr;
+  const int rc = make_drop(p_drop, seed, offset, &dr);
+  if (rc != FA_OK) return rc;
+  return fwd_impl(q, k, v, o, lse, B, H, N, d, scale, causal, block_mask, kv_len, nullptr, stream,
+                  dr);
+}
+
+int fa_bwd_dropout(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf16* o,
+                   const float* lse, const fa_bf16* dout, fa_bf16* dq, fa_bf16* dk, fa_bf16* dv,
+                   int B, int H, int N, int d, float scale, int causal, const uint8_t* block_mask,
+                   const int32_t* kv_len, float p_drop, uint64_t seed, uint32_t offset,
+                   void* workspace, size_t workspace_bytes, void* stream) {
+  DropArgs dr;
+  const int rc = make_drop(p_drop, seed, offset, &dr);
+  if (rc != FA_OK) return rc;
+  return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, block_mask, kv_len,
+                  workspace, workspace_bytes, nullptr, stream, 7u, dr);
+}
+
 int fa_get_device_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
   unsigned int v = 0;
@@ -422,12 +489,14 @@ const char* fa_status_string(int status) {
     case FA_OK: return "ok";
     case FA_ERR_NULL: return "a required pointer is NULL";
     case FA_ERR_ALIGN: return "a pointer is not aligned as required";
-    case FA_ERR_SHAPE: return "unsupported shape (negative size, N % 128 != 0, or B*H*N >= 2^31)";
+    case FA_ERR_SHAPE: return "unsupported shape (negative size, or B*H*N >= 2^31)";
     case FA_ERR_UNSUPPORTED_D: return "head dimension d must be 64 or 128";
     case FA_ERR_WORKSPACE: return "workspace missing or smaller than fa_bwd_workspace_size()";
     case FA_ERR_CUDA: return "a CUDA runtime or driver call failed";
     case FA_ERR_TIMEOUT: return "a device pipeline wait timed out; outputs are incomplete";
-    case FA_ERR_ARG: return "invalid argument (scale not finite or not > 0, or unknown phase)";
+    case FA_ERR_ARG:
+      return "invalid argument (scale not finite or not > 0, unknown phase, or dropout "
+             "probability outside [0, 1))";
     case FA_ERR_SCRATCH_LIMIT:
       return "shape needs more backward scratch than the built-in FA_BWD_NOALLOC_SCRATCH_BYTES";
     default: return "unknown status";

@@ -142,6 +142,10 @@ struct BwdParams {
   int num_units;
   int heads_per_group;  // unit order: see bwd_decode
   int* work_counter;    // next unit to take (zeroed by fa_bwd_pre_kernel)
+  // dropout (kernels instantiated with kDrop): the forward's mask, see FwdParams
+  uint32_t drop_t;
+  float drop_w;
+  uint32_t seed_lo, seed_hi, drop_offset;
   int causal;
   float scale;
   float scale_log2;
@@ -278,7 +282,7 @@ __device__ __forceinline__ BwdUnit bwd_decode(const BwdParams& p, int u) {
 }
 
 
-template <int D>
+template <int D, bool kDrop = false>
 __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -855,6 +859,42 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         // -D = 0, so P is 0 (or, on the polynomial path, clamped to about
         // 2^-126) and dS = P * 0 = 0; its contributions P dO, dS Q and dS K are
         // exactly zero and nothing in them can be infinite or NaN.
+        // dropout: this key's keep bits for the half's 64 queries, drawn while
+        // the S^T MMA runs.  The eight lanes of a key group split each 32-query
+        // chunk (lane slot s takes queries s, s + 8, s + 16, s + 24), then each
+        // lane gathers its own key's draw of every query from the lane that made
+        // it (all 32 lanes take part: this sits outside the per-lane branches).
+        uint32_t kb[2] = {0u, 0u};
+        if constexpr (kDrop) {
+          const int slot = lane & 7;
+          const int src0 = lane & ~7;
+          const int widx = (kr & 7) >> 1;
+          const int hsh = (kr & 1) * 16;
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            uint4 mine[4];
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+              mine[t] = philox4x32_10(static_cast<uint32_t>(c_key >> 3),
+                                      static_cast<uint32_t>(i * kTile + h * 64 + c * 32 + slot +
+                                                            8 * t),
+                                      static_cast<uint32_t>(w.bh), p.drop_offset, p.seed_lo,
+                                      p.seed_hi);
+            uint32_t bits = 0;
+#pragma unroll
+            for (int qq = 0; qq < 32; ++qq) {
+              const int src = src0 | (qq & 7);
+              const uint4 m = mine[qq >> 3];
+              const uint32_t w0 = __shfl_sync(0xffffffffu, m.x, src);
+              const uint32_t w1 = __shfl_sync(0xffffffffu, m.y, src);
+              const uint32_t w2 = __shfl_sync(0xffffffffu, m.z, src);
+              const uint32_t w3 = __shfl_sync(0xffffffffu, m.w, src);
+              const uint32_t word = widx == 0 ? w0 : widx == 1 ? w1 : widx == 2 ? w2 : w3;
+              bits |= static_cast<uint32_t>(((word >> hsh) & 0xFFFFu) >= p.drop_t) << qq;
+            }
+            kb[c] = bits;
+          }
+        }
         ok = __all_sync(0xffffffffu, mbar_wait(s_full, s_cnt & 1));
         ++s_cnt;
         if (!ok) break;
@@ -863,6 +903,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         // Three kinds of row: a key beyond kv_len (all zero, no exponentials),
         // the causal diagonal tile (element mask), and the rest (no mask; part
         // of the exponentials on the FMA pipe through ex2_poly2).
+        // dropout: the undropped P (packed bf16) stays in registers for the dS
+        // phase; TMEM gets the kept, scaled P^T for the dV MMA
+        [[maybe_unused]] uint32_t pu[2][16];
         {
           uint32_t r[2][32];
           tmem_ld32(tS, r[0]);
@@ -915,13 +958,25 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
                   p2 = (kr > q0 + 2) ? 0.f : p2;
                   p3 = (kr > q0 + 3) ? 0.f : p3;
                 }
+                if constexpr (kDrop) {
+                  pu[c][2 * e4] = pack_bf16x2(p0, p1);
+                  pu[c][2 * e4 + 1] = pack_bf16x2(p2, p3);
+                  const uint32_t b4 = kb[c] >> (4 * e4);
+                  p0 = (b4 & 1u) ? p0 * p.drop_w : 0.f;
+                  p1 = (b4 & 2u) ? p1 * p.drop_w : 0.f;
+                  p2 = (b4 & 4u) ? p2 * p.drop_w : 0.f;
+                  p3 = (b4 & 8u) ? p3 * p.drop_w : 0.f;
+                }
                 pk[2 * e4] = pack_bf16x2(p0, p1);
                 pk[2 * e4 + 1] = pack_bf16x2(p2, p3);
               }
             };
             if (!key_valid) {
 #pragma unroll
-              for (int e = 0; e < 16; ++e) pk[e] = 0u;
+              for (int e = 0; e < 16; ++e) {
+                pk[e] = 0u;
+                if constexpr (kDrop) pu[c][e] = 0u;
+              }
             } else if (diag) {
               make_p(std::integral_constant<int, 1>{});
             } else {
@@ -945,30 +1000,60 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         {
+          // dropout: the P kept in registers, one 32-query chunk of dP^T at a time
+          // (fewer registers live next to it); otherwise both chunks and P^T at once
           uint32_t r[2][32];
-          uint32_t pp[32];
-          tmem_ld32(tDP, r[0]);
-          tmem_ld32(tDP + 32, r[1]);
-          tmem_ld32(tP, pp);  // this half's P: 32 packed columns
-          tmem_wait_ld();
-          reg_fence32(r[0]);
-          reg_fence32(r[1]);
-          reg_fence32(pp);
+          [[maybe_unused]] uint32_t pp[32];
+          if constexpr (kDrop) {
+            tmem_ld32(tDP, r[0]);
+          } else {
+            tmem_ld32(tDP, r[0]);
+            tmem_ld32(tDP + 32, r[1]);
+            tmem_ld32(tP, pp);  // this half's P: 32 packed columns
+            tmem_wait_ld();
+            reg_fence32(r[0]);
+            reg_fence32(r[1]);
+            reg_fence32(pp);
+          }
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
+            if constexpr (kDrop) {
+              if (c == 1) tmem_ld32(tDP + 32, r[1]);
+              tmem_wait_ld();
+              reg_fence32(r[c]);
+            }
             uint32_t pk[16];
 #pragma unroll
             for (int e4 = 0; e4 < 8; ++e4) {
               const float4 nd = dz4[c * 8 + e4];  // -D of 4 queries
-              const uint64_t ta = f2_add(
-                  f2_pack(__uint_as_float(r[c][4 * e4]), __uint_as_float(r[c][4 * e4 + 1])),
-                  f2_pack(nd.x, nd.y));
-              const uint64_t tb = f2_add(
-                  f2_pack(__uint_as_float(r[c][4 * e4 + 2]), __uint_as_float(r[c][4 * e4 + 3])),
-                  f2_pack(nd.z, nd.w));
+              uint64_t ta, tb;
+              uint32_t pa, pb;
+              if constexpr (kDrop) {
+                // dropout: the gradient reaching P is dP * Z * w
+                const uint32_t b4 = kb[c] >> (4 * e4);
+                const float z0 = (b4 & 1u) ? p.drop_w : 0.f, z1 = (b4 & 2u) ? p.drop_w : 0.f;
+                const float z2 = (b4 & 4u) ? p.drop_w : 0.f, z3 = (b4 & 8u) ? p.drop_w : 0.f;
+                ta = f2_fma(
+                    f2_pack(__uint_as_float(r[c][4 * e4]), __uint_as_float(r[c][4 * e4 + 1])),
+                    f2_pack(z0, z1), f2_pack(nd.x, nd.y));
+                tb = f2_fma(
+                    f2_pack(__uint_as_float(r[c][4 * e4 + 2]), __uint_as_float(r[c][4 * e4 + 3])),
+                    f2_pack(z2, z3), f2_pack(nd.z, nd.w));
+                pa = pu[c][2 * e4];  // the undropped P
+                pb = pu[c][2 * e4 + 1];
+              } else {
+                ta = f2_add(
+                    f2_pack(__uint_as_float(r[c][4 * e4]), __uint_as_float(r[c][4 * e4 + 1])),
+                    f2_pack(nd.x, nd.y));
+                tb = f2_add(
+                    f2_pack(__uint_as_float(r[c][4 * e4 + 2]), __uint_as_float(r[c][4 * e4 + 3])),
+                    f2_pack(nd.z, nd.w));
+                pa = pp[c * 16 + 2 * e4];
+                pb = pp[c * 16 + 2 * e4 + 1];
+              }
               float d0, d1, d2, d3;
-              f2_unpack(f2_mul(ta, bf16x2_to_f2(pp[c * 16 + 2 * e4])), d0, d1);
-              f2_unpack(f2_mul(tb, bf16x2_to_f2(pp[c * 16 + 2 * e4 + 1])), d2, d3);
+              f2_unpack(f2_mul(ta, bf16x2_to_f2(pa)), d0, d1);
+              f2_unpack(f2_mul(tb, bf16x2_to_f2(pb)), d2, d3);
               pk[2 * e4] = pack_bf16x2(d0, d1);
               pk[2 * e4 + 1] = pack_bf16x2(d2, d3);
             }

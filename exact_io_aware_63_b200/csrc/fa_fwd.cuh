@@ -77,6 +77,13 @@ struct FwdParams {
   int heads_per_group;  // unit order: see fwd_decode
   int causal;
   float scale_log2;  // scale * log2(e)
+  // dropout (kernels instantiated with kDrop): element (head bh, query r, key
+  // c) is kept when its 16-bit Philox-4x32-10 draw (counter (c / 8, r, bh,
+  // drop_offset), key (seed_lo, seed_hi); draw c % 8 of the call) is at least
+  // drop_t; kept entries of P are scaled by drop_w = 65536 / (65536 - drop_t)
+  uint32_t drop_t;
+  float drop_w;
+  uint32_t seed_lo, seed_hi, drop_offset;
 };
 
 template <int D, bool kPair>
@@ -191,7 +198,7 @@ __device__ __forceinline__ int fwd_next(const FwdParams& p, const FwdUnit& w, in
   return w.j_end;
 }
 
-template <int D, bool kPair>
+template <int D, bool kPair, bool kDrop = false>
 __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -710,6 +717,30 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
       for (int j = kPair ? 0 : fwd_next(p, w, 0); j < (kPair ? j_end_me : w.j_end);
            j = kPair ? j + 1 : fwd_next(p, w, j + 1), ++k) {
         if (!kPair && (k & 1) != x) continue;
+        // dropout: the row's keep bits for the tile's 128 keys (bit e of kbits[c]
+        // is key j*128 + c*32 + e), drawn while the S MMA runs; one draw covers
+        // eight keys
+        [[maybe_unused]] uint32_t kbits[4];
+        if constexpr (kDrop) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t bits = 0;
+#pragma unroll 1
+            for (int g = 0; g < 4; ++g) {
+              const uint4 d4 = philox4x32_10(static_cast<uint32_t>(j * (kTile / 8) + c * 4 + g),
+                                             static_cast<uint32_t>(row),
+                                             static_cast<uint32_t>(w.bh), p.drop_offset,
+                                             p.seed_lo, p.seed_hi);
+              const uint32_t wd[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+              for (int v = 0; v < 4; ++v) {
+                bits |= static_cast<uint32_t>((wd[v] & 0xFFFFu) >= p.drop_t) << (g * 8 + 2 * v);
+                bits |= static_cast<uint32_t>((wd[v] >> 16) >= p.drop_t) << (g * 8 + 2 * v + 1);
+              }
+            }
+            kbits[c] = bits;
+          }
+        }
         ok = __all_sync(0xffffffffu, mbar_wait(s_full(x), s_cnt & 1));
         ++s_cnt;
         if (!ok) break;
@@ -789,6 +820,11 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
                 p1 = ex2_approx(x1);
               }
               ls4[e & 3] = f2_add(ls4[e & 3], f2_pack(p0, p1));
+              if constexpr (kDrop) {
+                // the row sum above is the softmax's; P V gets the kept, scaled P
+                p0 = ((kbits[c] >> (2 * e)) & 1u) ? p0 * p.drop_w : 0.f;
+                p1 = ((kbits[c] >> (2 * e + 1)) & 1u) ? p1 * p.drop_w : 0.f;
+              }
               pk[e] = pack_bf16x2(p0, p1);
             }
             tmem_st16(tP + c * 16, pk);

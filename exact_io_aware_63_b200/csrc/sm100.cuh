@@ -372,6 +372,29 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// Philox-4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As
+// Easy as 1, 2, 3", SC 2011): ten rounds; each forms the 64-bit products of
+// counter words 0 and 2 with two fixed multipliers, makes the new words 0 and
+// 2 from their high halves XORed with words 1 and 3 and the key, the new words
+// 1 and 3 from their low halves, then advances the key by two Weyl constants.
+__device__ __forceinline__ uint4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3,
+                                               uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int round = 0; round < 10; ++round) {
+    const uint32_t lo0 = 0xD2511F53u * c0, hi0 = __umulhi(0xD2511F53u, c0);
+    const uint32_t lo1 = 0xCD9E8D57u * c2, hi1 = __umulhi(0xCD9E8D57u, c2);
+    const uint32_t n0 = hi1 ^ c1 ^ k0;
+    const uint32_t n2 = hi0 ^ c3 ^ k1;
+    c0 = n0;
+    c1 = lo1;
+    c2 = n2;
+    c3 = lo0;
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
+  return make_uint4(c0, c1, c2, c3);
+}
+
 // 2^x evaluated on the FMA pipe instead of the MUFU unit, for -126 <= x <= 126
 // (smaller x is clamped to -126; the result is then ~1e-38, i.e. zero for our
 // purposes).  x = n + f with n = round(x) (obtained by adding 1.5 * 2^23, which

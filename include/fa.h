@@ -64,7 +64,8 @@ typedef enum {
     FA_ERR_WORKSPACE = -5,      /* workspace NULL or smaller than fa_bwd_workspace_size */
     FA_ERR_CUDA = -6,           /* a CUDA runtime/driver call failed */
     FA_ERR_TIMEOUT = -7,        /* a device pipeline wait gave up (fa_get_device_status) */
-    FA_ERR_ARG = -8,            /* scale not finite or not > 0, or phase not in 0..3 */
+    FA_ERR_ARG = -8,            /* scale not finite or not > 0, phase not in 0..3, or
+                                   p_drop outside [0, 1) */
     FA_ERR_SCRATCH_LIMIT = -9   /* fa_bwd_noalloc: the shape needs more scratch than
                                    FA_BWD_NOALLOC_SCRATCH_BYTES */
 } fa_status;
@@ -165,6 +166,46 @@ int fa_bwd_deterministic(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, c
                          fa_bf16* dv, int B, int H, int N, int d, float scale, int causal,
                          const uint8_t* block_mask, const int32_t* kv_len, void* workspace,
                          size_t workspace_bytes, void* stream);
+
+/*
+ * Forward and backward passes with dropout on the attention probabilities,
+ * fused into the same kernels.  Standard attention runs masking, softmax and
+ * dropout as separate memory-bound passes over the N x N matrix ("FlashAttention:
+ * A Novel Attention Algorithm with IO Awareness, Fast and Memory-Efficient",
+ * "Standard Attention Algorithm", the GPT-2 time breakdown); here the keep
+ * mask is drawn on chip and never stored.  The backward pass draws the same
+ * mask again from the same counters.
+ *
+ *   O_r  = sum_c P_rc Z_rc V_c,  Z_rc = w * keep(b*H + h, r, c) with
+ *   w = 65536 / (65536 - t),  t = floor(p_drop * 65536) (single precision,
+ *   where that product is exact), keep = (16-bit draw >= t).
+ *   The draw for (head index bh = b*H + h, query r, key c) is value c % 8 of
+ *   Philox-4x32-10 (Salmon et al., SC 2011) with counter
+ *   (c / 8, r, bh, offset) and key (seed low 32 bits, seed high 32 bits):
+ *   value k is the low 16 bits of output word k/2 for even k, the high 16
+ *   bits for odd k.
+ *   LSE is the softmax's and does not depend on the mask.  The backward pass
+ *   returns the gradients of that O: dV = (P o Z)^T dO,
+ *   dS = P o (Z o (dO V^T) - D) with D_r = sum_x dO_rx O_rx (O the dropped
+ *   output), dQ = scale * dS K, dK = scale * dS^T Q.
+ *
+ * p_drop must lie in [0, 1) (FA_ERR_ARG otherwise); p_drop = 0 keeps every
+ * entry and gives fa_fwd's and fa_bwd's results.  Pass the same p_drop, seed
+ * and offset to both passes; callers advance offset (or seed) between
+ * layers or steps that must draw independent masks.  All other arguments,
+ * layouts and error codes are those of fa_fwd and fa_bwd.  There is no
+ * deterministic-dQ variant with dropout.
+ */
+int fa_fwd_dropout(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o, float* lse,
+                   int B, int H, int N, int d, float scale, int causal, const uint8_t* block_mask,
+                   const int32_t* kv_len, float p_drop, uint64_t seed, uint32_t offset,
+                   void* stream);
+
+int fa_bwd_dropout(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf16* o,
+                   const float* lse, const fa_bf16* dout, fa_bf16* dq, fa_bf16* dk, fa_bf16* dv,
+                   int B, int H, int N, int d, float scale, int causal, const uint8_t* block_mask,
+                   const int32_t* kv_len, float p_drop, uint64_t seed, uint32_t offset,
+                   void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Size in bytes of the library's built-in backward scratch buffer (64 MiB),

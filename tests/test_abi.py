@@ -23,7 +23,8 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ["fa_fwd", "fa_fwd_traced", "fa_bwd", "fa_bwd_traced", "fa_bwd_phase",
-              "fa_bwd_deterministic", "fa_bwd_workspace_size",
+              "fa_bwd_deterministic", "fa_fwd_dropout", "fa_bwd_dropout",
+              "fa_bwd_workspace_size",
               "fa_get_device_status", "fa_status_string", "fa_version"]:
         assert n in names
 
@@ -88,7 +89,33 @@ def bwd_det(**kw):
                                     a["ws_bytes"], None)
 
 
-@pytest.mark.parametrize("call", [fwd, bwd, bwd_det])
+def fwd_drop(**kw):
+    a = dict(q=P, k=P, v=P, o=P, lse=P, B=1, H=1, N=128, d=64, scale=0.125, causal=0,
+             block_mask=None, kv_len=None, p_drop=0.1, seed=1, offset=0)
+    a.update(kw)
+    lib = binding.load()
+    return lib.fa_fwd_dropout(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"], a["N"],
+                              a["d"], a["scale"], a["causal"], a["block_mask"], a["kv_len"],
+                              a["p_drop"], a["seed"], a["offset"], None)
+
+
+def bwd_drop(**kw):
+    a = dict(q=P, k=P, v=P, o=P, lse=P, dout=P, dq=P, dk=P, dv=P, B=1, H=1, N=128, d=64,
+             scale=0.125, causal=0, block_mask=None, kv_len=None, p_drop=0.1, seed=1, offset=0,
+             ws=P, ws_bytes=1 << 30)
+    a.update(kw)
+    lib = binding.load()
+    return lib.fa_bwd_dropout(a["q"], a["k"], a["v"], a["o"], a["lse"], a["dout"], a["dq"],
+                              a["dk"], a["dv"], a["B"], a["H"], a["N"], a["d"], a["scale"],
+                              a["causal"], a["block_mask"], a["kv_len"], a["p_drop"], a["seed"],
+                              a["offset"], a["ws"], a["ws_bytes"], None)
+
+
+ALL_CALLS = [fwd, bwd, bwd_det, fwd_drop, bwd_drop]
+FWD_CALLS = (fwd, fwd_drop)
+
+
+@pytest.mark.parametrize("call", ALL_CALLS)
 def test_shape_errors(call):
     assert call(N=-128) == -3
     assert call(N=-1) == -3
@@ -98,7 +125,7 @@ def test_shape_errors(call):
     assert call(d=32) == -4
 
 
-@pytest.mark.parametrize("call", [fwd, bwd, bwd_det])
+@pytest.mark.parametrize("call", ALL_CALLS)
 def test_empty_problems_are_no_ops(call):
     assert call(B=0) == 0
     assert call(H=0) == 0
@@ -107,16 +134,16 @@ def test_empty_problems_are_no_ops(call):
     assert call(B=0, q=None, k=None) == 0
 
 
-@pytest.mark.parametrize("call", [fwd, bwd, bwd_det])
+@pytest.mark.parametrize("call", ALL_CALLS)
 def test_null_and_alignment(call):
     assert call(q=None) == -1
-    assert call(o=None) == -1 if call is fwd else call(dq=None) == -1
+    assert call(o=None) == -1 if call in FWD_CALLS else call(dq=None) == -1
     assert call(k=P + 8) == -2
     assert call(lse=P + 2) == -2
     assert call(kv_len=P + 1) == -2
 
 
-@pytest.mark.parametrize("call", [fwd, bwd, bwd_det])
+@pytest.mark.parametrize("call", ALL_CALLS)
 def test_scale_errors(call):
     assert call(scale=0.0) == -8
     assert call(scale=-1.0) == -8
@@ -124,7 +151,7 @@ def test_scale_errors(call):
     assert call(scale=float("nan")) == -8
 
 
-@pytest.mark.parametrize("call", [bwd, bwd_det])
+@pytest.mark.parametrize("call", [bwd, bwd_det, bwd_drop])
 def test_backward_workspace_errors(call):
     assert call(ws=None) == -5
     assert call(ws_bytes=16) == -5
@@ -146,3 +173,14 @@ def test_backward_phase_number_is_checked():
         rc = lib.fa_bwd_phase(ph, P, P, P, P, P, P, P, P, P, 1, 1, 128, 64, 0.125, 0, None, None, P,
                               1 << 30, None)
         assert rc == -8
+
+
+@pytest.mark.parametrize("call", [fwd_drop, bwd_drop])
+def test_dropout_probability_is_checked(call):
+    for bad in (-0.1, 1.0, 1.5, float("nan"), float("inf")):
+        assert call(p_drop=bad) == -8
+    # checked before anything else, even for an empty problem
+    assert call(p_drop=1.0, B=0) == -8
+    # valid probabilities pass the dropout check and reach the shape checks
+    for good in (0.0, 0.1, 0.5, 0.999):
+        assert call(p_drop=good, d=96) == -4
