@@ -144,29 +144,31 @@ WsLayout ws_layout(int B, int H, int N, int d) {
 // the weight of kept entries (see FwdParams).
 struct DropArgs {
   bool on = false;
-  uint32_t t = 0;
-  float w = 1.f;
-  uint32_t seed_lo = 0, seed_hi = 0, offset = 0;
+  fa::DropoutParams dp = {};
 };
 
 int make_drop(float p_drop, uint64_t seed, uint32_t offset, DropArgs* d) {
   if (!(p_drop >= 0.f && p_drop < 1.f)) return FA_ERR_ARG;
   d->on = true;
-  d->t = static_cast<uint32_t>(p_drop * 65536.0f);  // exact product, truncated
-  d->w = 65536.0f / (65536.0f - static_cast<float>(d->t));
-  d->seed_lo = static_cast<uint32_t>(seed);
-  d->seed_hi = static_cast<uint32_t>(seed >> 32);
-  d->offset = offset;
+  const uint32_t t = static_cast<uint32_t>(p_drop * 65536.0f);  // exact product, truncated
+  d->dp.t_hi = t << 16;
+  d->dp.w = 65536.0f / (65536.0f - static_cast<float>(t));
+  d->dp.offset = offset;
+  // Philox-4x32-10 round keys: the key (low, high word of seed) bumped by the
+  // Weyl constants once per round
+  uint32_t k0 = static_cast<uint32_t>(seed), k1 = static_cast<uint32_t>(seed >> 32);
+  for (int r = 0; r < 10; ++r) {
+    d->dp.rk[2 * r] = k0;
+    d->dp.rk[2 * r + 1] = k1;
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
   return FA_OK;
 }
 
 template <typename P>
 void set_drop(P& p, const DropArgs& dr) {
-  p.drop_t = dr.t;
-  p.drop_w = dr.w;
-  p.seed_lo = dr.seed_lo;
-  p.seed_hi = dr.seed_hi;
-  p.drop_offset = dr.offset;
+  p.drop = dr.dp;
 }
 
 template <int D, bool kPair, bool kDrop>

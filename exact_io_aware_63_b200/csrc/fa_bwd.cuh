@@ -142,13 +142,10 @@ struct BwdParams {
   int num_units;
   int heads_per_group;  // unit order: see bwd_decode
   int* work_counter;    // next unit to take (zeroed by fa_bwd_pre_kernel)
-  // dropout (kernels instantiated with kDrop): the forward's mask, see FwdParams
-  uint32_t drop_t;
-  float drop_w;
-  uint32_t seed_lo, seed_hi, drop_offset;
   int causal;
   float scale;
   float scale_log2;
+  DropoutParams drop;   // the forward's mask (kernels instantiated with kDrop)
 };
 
 template <int D>
@@ -820,7 +817,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     // Warpgroup h (warps 4-7: h = 0, warps 8-11: h = 1) handles queries
     // 64h..64h+63 of every key row; one key row per thread (TMEM lane).
     if constexpr (Cfg::kRegsDs > Cfg::kRegsLaunch) setmaxnreg_inc<Cfg::kRegsDs>();
-    constexpr int kPolyPer4 = Cfg::kPolyPer4;
+    // with dropout the generator's integer multiplies load the FMA pipe:
+    // every exponential goes to the MUFU unit
+    constexpr int kPolyPer4 = kDrop ? 0 : Cfg::kPolyPer4;
     const int h = (warp >= 8) ? 1 : 0;
     const int quarter = warp & 3;
     const int kr = quarter * 32 + lane;  // key row within the tile
@@ -859,38 +858,34 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         // -D = 0, so P is 0 (or, on the polynomial path, clamped to about
         // 2^-126) and dS = P * 0 = 0; its contributions P dO, dS Q and dS K are
         // exactly zero and nothing in them can be infinite or NaN.
-        // dropout: this key's keep bits for the half's 64 queries, drawn while
-        // the S^T MMA runs.  The eight lanes of a key group split each 32-query
-        // chunk (lane slot s takes queries s, s + 8, s + 16, s + 24), then each
-        // lane gathers its own key's draw of every query from the lane that made
-        // it (all 32 lanes take part: this sits outside the per-lane branches).
+        // dropout: this key's keep bits for the half's 64 queries (bit q of kb[c]
+        // is query i*128 + h*64 + c*32 + q), drawn while the S^T MMA runs.  A
+        // draw covers eight keys of one query, so the eight lanes of a key group
+        // share the work: lane slot s draws queries s + 8t (t < 4) and packs the
+        // keep bits into R (bit 8t + k = key k of the group, query s + 8t); each
+        // lane then reads R from the group's eight lanes and keeps its own key's
+        // bits.  All 32 lanes take part: this sits outside the per-lane branches.
         uint32_t kb[2] = {0u, 0u};
         if constexpr (kDrop) {
           const int slot = lane & 7;
           const int src0 = lane & ~7;
-          const int widx = (kr & 7) >> 1;
-          const int hsh = (kr & 1) * 16;
+          const int kk = kr & 7;  // this lane's key within its group of eight
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
-            uint4 mine[4];
+            uint32_t R = 0;
 #pragma unroll
-            for (int t = 0; t < 4; ++t)
-              mine[t] = philox4x32_10(static_cast<uint32_t>(c_key >> 3),
-                                      static_cast<uint32_t>(i * kTile + h * 64 + c * 32 + slot +
-                                                            8 * t),
-                                      static_cast<uint32_t>(w.bh), p.drop_offset, p.seed_lo,
-                                      p.seed_hi);
+            for (int t = 0; t < 4; ++t) {
+              const uint4 d4 = philox4x32_10_rk(
+                  static_cast<uint32_t>(c_key >> 3),
+                  static_cast<uint32_t>(i * kTile + h * 64 + c * 32 + slot + 8 * t),
+                  static_cast<uint32_t>(w.bh), p.drop.offset, p.drop.rk);
+              R |= keep_bits8(d4, p.drop.t_hi) << (8 * t);
+            }
             uint32_t bits = 0;
 #pragma unroll
-            for (int qq = 0; qq < 32; ++qq) {
-              const int src = src0 | (qq & 7);
-              const uint4 m = mine[qq >> 3];
-              const uint32_t w0 = __shfl_sync(0xffffffffu, m.x, src);
-              const uint32_t w1 = __shfl_sync(0xffffffffu, m.y, src);
-              const uint32_t w2 = __shfl_sync(0xffffffffu, m.z, src);
-              const uint32_t w3 = __shfl_sync(0xffffffffu, m.w, src);
-              const uint32_t word = widx == 0 ? w0 : widx == 1 ? w1 : widx == 2 ? w2 : w3;
-              bits |= static_cast<uint32_t>(((word >> hsh) & 0xFFFFu) >= p.drop_t) << qq;
+            for (int s8 = 0; s8 < 8; ++s8) {
+              const uint32_t Rs = __shfl_sync(0xffffffffu, R, src0 | s8);
+              bits |= ((Rs >> kk) & 0x01010101u) << s8;  // queries s8 + 8t
             }
             kb[c] = bits;
           }
@@ -959,13 +954,14 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
                   p3 = (kr > q0 + 3) ? 0.f : p3;
                 }
                 if constexpr (kDrop) {
+                  // dV gets the kept P (w is applied in its epilogue); dS the whole P
                   pu[c][2 * e4] = pack_bf16x2(p0, p1);
                   pu[c][2 * e4 + 1] = pack_bf16x2(p2, p3);
                   const uint32_t b4 = kb[c] >> (4 * e4);
-                  p0 = (b4 & 1u) ? p0 * p.drop_w : 0.f;
-                  p1 = (b4 & 2u) ? p1 * p.drop_w : 0.f;
-                  p2 = (b4 & 4u) ? p2 * p.drop_w : 0.f;
-                  p3 = (b4 & 8u) ? p3 * p.drop_w : 0.f;
+                  p0 = (b4 & 1u) ? p0 : 0.f;
+                  p1 = (b4 & 2u) ? p1 : 0.f;
+                  p2 = (b4 & 4u) ? p2 : 0.f;
+                  p3 = (b4 & 8u) ? p3 : 0.f;
                 }
                 pk[2 * e4] = pack_bf16x2(p0, p1);
                 pk[2 * e4 + 1] = pack_bf16x2(p2, p3);
@@ -1031,8 +1027,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
               if constexpr (kDrop) {
                 // dropout: the gradient reaching P is dP * Z * w
                 const uint32_t b4 = kb[c] >> (4 * e4);
-                const float z0 = (b4 & 1u) ? p.drop_w : 0.f, z1 = (b4 & 2u) ? p.drop_w : 0.f;
-                const float z2 = (b4 & 4u) ? p.drop_w : 0.f, z3 = (b4 & 8u) ? p.drop_w : 0.f;
+                const float z0 = (b4 & 1u) ? p.drop.w : 0.f, z1 = (b4 & 2u) ? p.drop.w : 0.f;
+                const float z2 = (b4 & 4u) ? p.drop.w : 0.f, z3 = (b4 & 8u) ? p.drop.w : 0.f;
                 ta = f2_fma(
                     f2_pack(__uint_as_float(r[c][4 * e4]), __uint_as_float(r[c][4 * e4 + 1])),
                     f2_pack(z0, z1), f2_pack(nd.x, nd.y));
@@ -1080,7 +1076,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       ++dkv_cnt;
       if (!ok) break;
       tc_fence_after();
-      const float mul = h ? 1.f : p.scale;
+      const float mul = h ? (kDrop ? p.drop.w : 1.f) : p.scale;  // dV: dropout weight
       const uint32_t tAcc = t_lane + (h ? Cfg::kColDV : Cfg::kColDK);
       uint8_t* epi_row = smem + Cfg::kOffEpi + h * Cfg::kTileBytes + kr * 128;
 #pragma unroll

@@ -66,6 +66,30 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleLog2 = 8.0f;
 
+// Dropout on P.  Element (head bh, query r, key c) is kept when its 16-bit
+// draw is at least t: the draw is value c % 8 of Philox-4x32-10 with counter
+// (c / 8, r, bh, offset) and key (seed_lo, seed_hi), value k being the low
+// (even k) or high (odd k) half of output word k / 2.  Kept entries weigh
+// w = 65536 / (65536 - t), dropped ones 0.
+struct DropoutParams {
+  uint32_t t_hi;     // t << 16: low half kept iff (word << 16) >= t_hi, high iff word >= t_hi
+  float w;
+  uint32_t offset;
+  uint32_t rk[20];   // the key's round keys, see philox4x32_10_rk
+};
+
+// keep bits of one draw's eight values (bit k = value k)
+__device__ __forceinline__ uint32_t keep_bits8(const uint4 d, uint32_t t_hi) {
+  const uint32_t wd[4] = {d.x, d.y, d.z, d.w};
+  uint32_t b = 0;
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    b |= static_cast<uint32_t>((wd[v] << 16) >= t_hi) << (2 * v);
+    b |= static_cast<uint32_t>(wd[v] >= t_hi) << (2 * v + 1);
+  }
+  return b;
+}
+
 struct FwdParams {
   uint16_t* o;
   float* lse;
@@ -77,13 +101,7 @@ struct FwdParams {
   int heads_per_group;  // unit order: see fwd_decode
   int causal;
   float scale_log2;  // scale * log2(e)
-  // dropout (kernels instantiated with kDrop): element (head bh, query r, key
-  // c) is kept when its 16-bit Philox-4x32-10 draw (counter (c / 8, r, bh,
-  // drop_offset), key (seed_lo, seed_hi); draw c % 8 of the call) is at least
-  // drop_t; kept entries of P are scaled by drop_w = 65536 / (65536 - drop_t)
-  uint32_t drop_t;
-  float drop_w;
-  uint32_t seed_lo, seed_hi, drop_offset;
+  DropoutParams drop;  // read by kernels instantiated with kDrop only
 };
 
 template <int D, bool kPair>
@@ -691,6 +709,8 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
   } else {
     // ------------------------------------------------------------ softmax
     setmaxnreg_inc<Cfg::kRegsHigh>();
+    // with dropout the generator's integer multiplies load the FMA pipe:
+    // every exponential goes to the MUFU unit
     constexpr int kPolyPer8 = Cfg::kPolyPer8;
     const int x = (warp >= 8) ? 1 : 0;
     const int quarter = warp & 3;
@@ -717,30 +737,6 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
       for (int j = kPair ? 0 : fwd_next(p, w, 0); j < (kPair ? j_end_me : w.j_end);
            j = kPair ? j + 1 : fwd_next(p, w, j + 1), ++k) {
         if (!kPair && (k & 1) != x) continue;
-        // dropout: the row's keep bits for the tile's 128 keys (bit e of kbits[c]
-        // is key j*128 + c*32 + e), drawn while the S MMA runs; one draw covers
-        // eight keys
-        [[maybe_unused]] uint32_t kbits[4];
-        if constexpr (kDrop) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t bits = 0;
-#pragma unroll 1
-            for (int g = 0; g < 4; ++g) {
-              const uint4 d4 = philox4x32_10(static_cast<uint32_t>(j * (kTile / 8) + c * 4 + g),
-                                             static_cast<uint32_t>(row),
-                                             static_cast<uint32_t>(w.bh), p.drop_offset,
-                                             p.seed_lo, p.seed_hi);
-              const uint32_t wd[4] = {d4.x, d4.y, d4.z, d4.w};
-#pragma unroll
-              for (int v = 0; v < 4; ++v) {
-                bits |= static_cast<uint32_t>((wd[v] & 0xFFFFu) >= p.drop_t) << (g * 8 + 2 * v);
-                bits |= static_cast<uint32_t>((wd[v] >> 16) >= p.drop_t) << (g * 8 + 2 * v + 1);
-              }
-            }
-            kbits[c] = bits;
-          }
-        }
         ok = __all_sync(0xffffffffu, mbar_wait(s_full(x), s_cnt & 1));
         ++s_cnt;
         if (!ok) break;
@@ -807,8 +803,18 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             uint32_t pk[16];
+            [[maybe_unused]] uint4 d4;
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
+              if constexpr (kDrop) {
+                // one draw per eight keys: keys c*32 + 8*(e/4) .. +7 of the tile
+                // (inline, so that the generator's integer work interleaves with
+                // the exponentials)
+                if ((e & 3) == 0)
+                  d4 = philox4x32_10_rk(static_cast<uint32_t>(j * (kTile / 8) + c * 4 + (e >> 2)),
+                                        static_cast<uint32_t>(row), static_cast<uint32_t>(w.bh),
+                                        p.drop.offset, p.drop.rk);
+              }
               const uint64_t xx =
                   f2_fma(f2_pack(sv[c * 32 + 2 * e], sv[c * 32 + 2 * e + 1]), scale2, negm2);
               float x0, x1, p0, p1;
@@ -821,9 +827,12 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
               }
               ls4[e & 3] = f2_add(ls4[e & 3], f2_pack(p0, p1));
               if constexpr (kDrop) {
-                // the row sum above is the softmax's; P V gets the kept, scaled P
-                p0 = ((kbits[c] >> (2 * e)) & 1u) ? p0 * p.drop_w : 0.f;
-                p1 = ((kbits[c] >> (2 * e + 1)) & 1u) ? p1 * p.drop_w : 0.f;
+                // the row sum above is the softmax's; P V gets the kept P, and
+                // the weight w of kept entries is applied with 1 / l at the end
+                const uint32_t word = (e & 3) == 0 ? d4.x : (e & 3) == 1 ? d4.y
+                                    : (e & 3) == 2 ? d4.z : d4.w;
+                p0 = ((word << 16) >= p.drop.t_hi) ? p0 : 0.f;
+                p1 = (word >= p.drop.t_hi) ? p1 : 0.f;
               }
               pk[e] = pack_bf16x2(p0, p1);
             }
@@ -880,7 +889,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
           ++o_cnt[x];
           if (!ok) break;
           tc_fence_after();
-          const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+          const float inv_l = (l > 0.f) ? (kDrop ? p.drop.w : 1.f) / l : 0.f;
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
             uint32_t r[32];
@@ -932,7 +941,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
         const float a0 = (ml0.y > 0.f) ? ex2_approx(ml0.x - m) : 0.f;
         const float a1 = (ml1.y > 0.f) ? ex2_approx(ml1.x - m) : 0.f;
         const float lt = ml0.y * a0 + ml1.y * a1;
-        const float inv_l = (lt > 0.f) ? 1.f / lt : 0.f;
+        const float inv_l = (lt > 0.f) ? (kDrop ? p.drop.w : 1.f) / lt : 0.f;
         const float f0 = a0 * inv_l, f1 = a1 * inv_l;
         uint4* orow = reinterpret_cast<uint4*>(p.o + grow * D + x * (D / 2));
         // A warpgroup that processed no tile left its O unwritten: its factor is 0

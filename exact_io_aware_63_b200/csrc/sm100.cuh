@@ -395,6 +395,29 @@ __device__ __forceinline__ uint4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_
   return make_uint4(c0, c1, c2, c3);
 }
 
+// The same generator with its ten round keys given: rk[2r] and rk[2r + 1] are
+// the key words of round r (k0 + r * 0x9E3779B9, k1 + r * 0xBB67AE85).  With rk
+// in kernel parameters every key enters its XOR straight from the constant
+// bank, so a call costs the multiplies and XORs of its rounds only.
+__device__ __forceinline__ uint4 philox4x32_10_rk(uint32_t c0, uint32_t c1, uint32_t c2,
+                                                  uint32_t c3, const uint32_t (&rk)[20]) {
+#pragma unroll
+  for (int round = 0; round < 10; ++round) {
+    // one 32 x 32 -> 64-bit multiply per product (its high and low words)
+    const uint64_t m0 = static_cast<uint64_t>(0xD2511F53u) * c0;
+    const uint64_t m1 = static_cast<uint64_t>(0xCD9E8D57u) * c2;
+    const uint32_t lo0 = static_cast<uint32_t>(m0), hi0 = static_cast<uint32_t>(m0 >> 32);
+    const uint32_t lo1 = static_cast<uint32_t>(m1), hi1 = static_cast<uint32_t>(m1 >> 32);
+    const uint32_t n0 = hi1 ^ c1 ^ rk[2 * round];
+    const uint32_t n2 = hi0 ^ c3 ^ rk[2 * round + 1];
+    c0 = n0;
+    c1 = lo1;
+    c2 = n2;
+    c3 = lo0;
+  }
+  return make_uint4(c0, c1, c2, c3);
+}
+
 // 2^x evaluated on the FMA pipe instead of the MUFU unit, for -126 <= x <= 126
 // (smaller x is clamped to -126; the result is then ~1e-38, i.e. zero for our
 // purposes).  x = n + f with n = round(x) (obtained by adding 1.5 * 2^23, which
