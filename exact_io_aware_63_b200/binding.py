@@ -46,6 +46,7 @@ _SIGS = {
     "fa_fwd_dropout": (_i, [_vp] * 5 + [_i, _i, _i, _i, _f, _i, _vp, _vp, _f, _u64, _u32, _vp]),
     "fa_bwd_dropout": (_i, [_vp] * 9 + [_i, _i, _i, _i, _f, _i, _vp, _vp, _f, _u64, _u32, _vp,
                                         _sz, _vp]),
+    "fa_selftest_wait_timeout": (_i, [_i, ctypes.c_uint, _vp, _vp]),
     "fa_get_device_status": (_i, [_vp]),
     "fa_status_string": (ctypes.c_char_p, [_i]),
     "fa_version": (_i, []),
@@ -188,6 +189,12 @@ def fa_bwd_dropout(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal,
                                  int(bool(causal)), _ptr(block_mask), _ptr(kv_len),
                                  float(p_drop), int(seed), int(offset), _ptr(workspace),
                                  int(workspace_bytes), _stream(stream))
+
+
+def fa_selftest_wait_timeout(arrive, limit_us, result, stream=None):
+    """One warp waits on a barrier for at most limit_us; see include/fa.h."""
+    return load().fa_selftest_wait_timeout(int(arrive), int(limit_us), _ptr(result),
+                                           _stream(stream))
 
 
 def fa_get_device_status(stream=None):

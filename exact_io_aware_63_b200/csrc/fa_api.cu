@@ -15,6 +15,30 @@
 #include "fa_bwd_det.cuh"
 #include "fa_fwd.cuh"
 
+namespace fa {
+
+// Check of the bounded-wait machinery every kernel relies on: one warp waits
+// on a shared-memory mbarrier with the given limit.  With arrive = 0 nothing
+// completes the barrier's phase, so the wait must give up, record
+// FA_DEV_TIMEOUT in the status word and return; with arrive = 1 the warp
+// arrives first and the wait succeeds at once.  Either way the kernel ends.
+__global__ void __launch_bounds__(32, 1)
+    fa_selftest_wait_kernel(int arrive, unsigned long long limit_ns, int* result) {
+  __shared__ __align__(8) unsigned long long bar_storage;
+  const uint32_t bar = smem_u32(&bar_storage);
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+  if (arrive && threadIdx.x == 0) mbar_arrive(bar);
+  __syncwarp();
+  const bool ok = mbar_wait_for(bar, 0, limit_ns);
+  if (threadIdx.x == 0) *result = ok ? 1 : 0;
+}
+
+}  // namespace fa
+
 namespace {
 
 constexpr int kVersion = 10000;  // 1.0.0
@@ -472,6 +496,15 @@ int fa_bwd_dropout(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const f
   if (rc != FA_OK) return rc;
   return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, block_mask, kv_len,
                   workspace, workspace_bytes, nullptr, stream, 7u, dr);
+}
+
+int fa_selftest_wait_timeout(int arrive, unsigned int limit_us, int* result, void* stream) {
+  if (!result) return FA_ERR_NULL;
+  if (!aligned(result, 4)) return FA_ERR_ALIGN;
+  if (limit_us == 0 || limit_us > 2000000u) return FA_ERR_ARG;
+  fa::fa_selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      arrive ? 1 : 0, 1000ull * limit_us, result);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 int fa_get_device_status(void* stream) {

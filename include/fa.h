@@ -208,6 +208,21 @@ int fa_bwd_dropout(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const f
                    void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Self-test of the failure path every kernel relies on.  Each pipeline wait
+ * in the kernels is bounded in time; when a wait gives up, the kernel records
+ * a timeout in a device status word, winds down and exits, and
+ * fa_get_device_status then returns FA_ERR_TIMEOUT (and clears the word).
+ * This call launches one warp that waits on a shared-memory barrier for at
+ * most limit_us microseconds (1 .. 2,000,000, else FA_ERR_ARG).  With
+ * arrive = 0 nothing completes the barrier, so the wait must give up and
+ * record the timeout; with arrive != 0 the warp arrives first and the wait
+ * succeeds.  *result (device memory, int, 4-byte aligned) is set to 1 if the
+ * wait succeeded, 0 if it gave up.  No fault, trap or unbounded wait is
+ * involved: the kernel always ends, and the context stays usable.
+ */
+int fa_selftest_wait_timeout(int arrive, unsigned int limit_us, int* result, void* stream);
+
+/*
  * Size in bytes of the library's built-in backward scratch buffer (64 MiB),
  * used only by fa_bwd_noalloc.
  */

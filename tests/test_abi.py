@@ -24,6 +24,7 @@ def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ["fa_fwd", "fa_fwd_traced", "fa_bwd", "fa_bwd_traced", "fa_bwd_phase",
               "fa_bwd_deterministic", "fa_fwd_dropout", "fa_bwd_dropout",
+              "fa_selftest_wait_timeout",
               "fa_bwd_workspace_size",
               "fa_get_device_status", "fa_status_string", "fa_version"]:
         assert n in names
@@ -184,3 +185,11 @@ def test_dropout_probability_is_checked(call):
     # valid probabilities pass the dropout check and reach the shape checks
     for good in (0.0, 0.1, 0.5, 0.999):
         assert call(p_drop=good, d=96) == -4
+
+
+def test_selftest_arguments_are_checked():
+    lib = binding.load()
+    assert lib.fa_selftest_wait_timeout(0, 1000, None, None) == -1
+    assert lib.fa_selftest_wait_timeout(0, 1000, P + 2, None) == -2
+    assert lib.fa_selftest_wait_timeout(0, 0, P, None) == -8
+    assert lib.fa_selftest_wait_timeout(0, 2_000_001, P, None) == -8
