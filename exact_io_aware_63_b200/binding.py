@@ -46,6 +46,9 @@ _SIGS = {
     "fa_fwd_dropout": (_i, [_vp] * 5 + [_i, _i, _i, _i, _f, _i, _vp, _vp, _f, _u64, _u32, _vp]),
     "fa_bwd_dropout": (_i, [_vp] * 9 + [_i, _i, _i, _i, _f, _i, _vp, _vp, _f, _u64, _u32, _vp,
                                         _sz, _vp]),
+    "fa_fwd_varlen": (_i, [_vp] * 6 + [_i, _i, _i, _i, _i, _f, _i, _f, _u64, _u32, _vp]),
+    "fa_bwd_varlen": (_i, [_vp] * 10 + [_i, _i, _i, _i, _i, _f, _i, _f, _u64, _u32, _vp, _sz,
+                                         _vp]),
     "fa_selftest_wait_timeout": (_i, [_i, ctypes.c_uint, _vp, _vp]),
     "fa_get_device_status": (_i, [_vp]),
     "fa_status_string": (ctypes.c_char_p, [_i]),
@@ -191,6 +194,27 @@ def fa_bwd_dropout(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal,
                                  int(workspace_bytes), _stream(stream))
 
 
+def fa_fwd_varlen(q, k, v, o, lse, cu_seqlens, B, H, max_seqlen, total_tokens, d, scale, causal,
+                  p_drop=0.0, seed=0, offset=0, stream=None):
+    """Forward pass of a packed variable-length batch ([T, H, d] tensors, LSE [H, T])."""
+    return load().fa_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_seqlens),
+                                B, H, max_seqlen, total_tokens, d, float(scale),
+                                int(bool(causal)), float(p_drop), int(seed), int(offset),
+                                _stream(stream))
+
+
+def fa_bwd_varlen(q, k, v, o, lse, dout, dq, dk, dv, cu_seqlens, B, H, max_seqlen, total_tokens,
+                  d, scale, causal, p_drop, seed, offset, workspace, workspace_bytes,
+                  stream=None):
+    """Backward pass of a packed variable-length batch; workspace of
+    fa_bwd_workspace_size(B, H, max_seqlen, d) bytes."""
+    return load().fa_bwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
+                                _ptr(dq), _ptr(dk), _ptr(dv), _ptr(cu_seqlens), B, H, max_seqlen,
+                                total_tokens, d, float(scale), int(bool(causal)), float(p_drop),
+                                int(seed), int(offset), _ptr(workspace), int(workspace_bytes),
+                                _stream(stream))
+
+
 def fa_selftest_wait_timeout(arrive, limit_us, result, stream=None):
     """One warp waits on a barrier for at most limit_us; see include/fa.h."""
     return load().fa_selftest_wait_timeout(int(arrive), int(limit_us), _ptr(result),
@@ -272,4 +296,37 @@ def attention_backward(q, k, v, o, lse, dout, scale, causal=False, block_mask=No
         rc = fa_bwd_traced(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal,
                            block_mask, kv_len, workspace, workspace.numel(), visited, stream)
     _check(rc, "fa_bwd")
+    return dq, dk, dv
+
+
+def attention_forward_varlen(q, k, v, cu_seqlens, max_seqlen, scale, causal=False, dropout=None,
+                             stream=None):
+    """O [T, H, d] and LSE [H, T] for a packed batch: bf16 CUDA tensors [T, H, d] and
+    int32 CUDA cu_seqlens [B + 1]; ``dropout`` = None or (p_drop, seed, offset)."""
+    import torch
+    T, H, d = q.shape
+    B = cu_seqlens.numel() - 1
+    o = torch.empty_like(q)
+    lse = torch.empty((H, T), dtype=torch.float32, device=q.device)
+    p_drop, seed, offset = dropout if dropout is not None else (0.0, 0, 0)
+    rc = fa_fwd_varlen(q, k, v, o, lse, cu_seqlens, B, H, max_seqlen, T, d, scale, causal, p_drop,
+                       seed, offset, stream)
+    _check(rc, "fa_fwd_varlen")
+    return o, lse
+
+
+def attention_backward_varlen(q, k, v, o, lse, dout, cu_seqlens, max_seqlen, scale, causal=False,
+                              dropout=None, workspace=None, stream=None):
+    """dQ, dK, dV [T, H, d] for the packed forward that produced (o, lse)."""
+    import torch
+    T, H, d = q.shape
+    B = cu_seqlens.numel() - 1
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws_bytes = fa_bwd_workspace_size(B, H, max_seqlen, d)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    p_drop, seed, offset = dropout if dropout is not None else (0.0, 0, 0)
+    rc = fa_bwd_varlen(q, k, v, o, lse, dout, dq, dk, dv, cu_seqlens, B, H, max_seqlen, T, d,
+                       scale, causal, p_drop, seed, offset, workspace, workspace.numel(), stream)
+    _check(rc, "fa_bwd_varlen")
     return dq, dk, dv

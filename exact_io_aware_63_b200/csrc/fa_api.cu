@@ -94,6 +94,51 @@ bool make_tmap_f32_acc(CUtensorMap* m, const void* base, int BH, int N, int d) {
   return r == CUDA_SUCCESS;
 }
 
+// Packed [T][H][d] tensors (variable-length batches) mapped as (d, H, T), so
+// that the strides increase: box (64, 1, 128) is a 128-token tile of one head,
+// laid out in shared memory exactly like the (64, 128, 1) box of make_tmap.
+bool make_tmap_packed(CUtensorMap* m, const void* base, int H, int T, int d) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
+                        static_cast<cuuint64_t>(T)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(H) * d * 2};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// The float32 [T][H][d] dQ accumulator of a packed batch: boxes of 32 tokens x
+// 32 columns of one head.
+bool make_tmap_f32_acc_packed(CUtensorMap* m, const void* base, int H, int T, int d) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
+                        static_cast<cuuint64_t>(T)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 4, static_cast<cuuint64_t>(H) * d * 4};
+  cuuint32_t box[3] = {32, 1, 32};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Geometry of a packed variable-length batch (cu == nullptr: the [B][H][N][d]
+// layout).  N passed alongside is the longest sequence.
+struct Packed {
+  const int32_t* cu = nullptr;
+  int T = 0;
+};
+
+// Tensor map of a bf16 operand in either layout.
+bool make_tmap_any(CUtensorMap* m, const void* base, int B, int H, int N, int d, const Packed& pk) {
+  return pk.cu ? make_tmap_packed(m, base, H, pk.T, d) : make_tmap(m, base, B * H, N, d);
+}
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 // Shape checks shared by every entry point.  Returns FA_OK, an error, or 1
@@ -104,6 +149,20 @@ int check_shape(int B, int H, int N, int d) {
   if (B == 0 || H == 0 || N == 0) return 1;
   const long long rows = static_cast<long long>(B) * H * N;
   if (rows >= (1LL << 31)) return FA_ERR_SHAPE;
+  return FA_OK;
+}
+
+// Checks of a packed variable-length batch (before check_shape, which then
+// sees B, H and max_seqlen): FA_OK, an error, or 1 for "nothing to do".
+int check_packed(const int32_t* cu, int B, int H, int max_seqlen, int T, int d) {
+  if (B < 0 || H < 0 || max_seqlen < 0 || T < 0) return FA_ERR_SHAPE;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED_D;
+  if (B == 0 || H == 0 || max_seqlen == 0 || T == 0) return 1;
+  // B sequences of at most max_seqlen tokens: the workspace and the unit grid
+  // are sized for B * max_seqlen rows per head
+  if (static_cast<long long>(T) > static_cast<long long>(B) * max_seqlen) return FA_ERR_SHAPE;
+  if (!cu) return FA_ERR_NULL;
+  if (!aligned(cu, 4)) return FA_ERR_ALIGN;
   return FA_OK;
 }
 
@@ -195,19 +254,20 @@ void set_drop(P& p, const DropArgs& dr) {
   p.drop = dr.dp;
 }
 
-template <int D, bool kPair, bool kDrop>
+template <int D, bool kPair, bool kDrop, bool kPacked = false>
 int launch_fwd_mode(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                     fa::FwdParams& p, cudaStream_t stream, int num_sms) {
   using Cfg = fa::FwdCfg<D, kPair>;
   static bool smem_set = false;
   if (!smem_set) {
-    if (!set_smem(fa::fa_fwd_kernel<D, kPair, kDrop>, Cfg::kSmemBytes)) return FA_ERR_CUDA;
+    if (!set_smem(fa::fa_fwd_kernel<D, kPair, kDrop, kPacked>, Cfg::kSmemBytes))
+      return FA_ERR_CUDA;
     smem_set = true;
   }
   const int per_head = kPair ? (p.n_t + 1) / 2 : p.n_t;
   p.num_units = p.B * p.H * per_head;
   const int grid = p.num_units < num_sms ? p.num_units : num_sms;
-  fa::fa_fwd_kernel<D, kPair, kDrop>
+  fa::fa_fwd_kernel<D, kPair, kDrop, kPacked>
       <<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -219,10 +279,10 @@ template <int D>
 int launch_fwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o, float* lse, int B,
                int H, int N, float scale, int causal, const uint8_t* block_mask,
                const int32_t* kv_len, uint8_t* visited, cudaStream_t stream, int num_sms,
-               const DropArgs& dr) {
+               const DropArgs& dr, const Packed& pk) {
   CUtensorMap tq, tk, tv;
-  if (!make_tmap(&tq, q, B * H, N, D) || !make_tmap(&tk, k, B * H, N, D) ||
-      !make_tmap(&tv, v, B * H, N, D))
+  if (!make_tmap_any(&tq, q, B, H, N, D, pk) || !make_tmap_any(&tk, k, B, H, N, D, pk) ||
+      !make_tmap_any(&tv, v, B, H, N, D, pk))
     return FA_ERR_CUDA;
   fa::FwdParams p;
   p.o = o;
@@ -230,6 +290,9 @@ int launch_fwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o,
   p.block_mask = block_mask;
   p.kv_len = kv_len;
   p.visited = visited;
+  p.cu_seqlens = pk.cu;
+  p.T = pk.T;
+  p.o_stride = pk.cu ? static_cast<long long>(H) * D : D;
   p.B = B;
   p.H = H;
   p.N = N;
@@ -238,6 +301,10 @@ int launch_fwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o,
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * fa::kLog2e;
   set_drop(p, dr);
+  if (pk.cu) {  // packed batches have no block mask: pair mode
+    if (dr.on) return launch_fwd_mode<D, true, true, true>(tq, tk, tv, p, stream, num_sms);
+    return launch_fwd_mode<D, true, false, true>(tq, tk, tv, p, stream, num_sms);
+  }
   if (dr.on) {
     if (block_mask) return launch_fwd_mode<D, false, true>(tq, tk, tv, p, stream, num_sms);
     return launch_fwd_mode<D, true, true>(tq, tk, tv, p, stream, num_sms);
@@ -251,9 +318,10 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
                const float* lse, const fa_bf16* dout, fa_bf16* dq, fa_bf16* dk, fa_bf16* dv, int B,
                int H, int N, float scale, int causal, const uint8_t* block_mask,
                const int32_t* kv_len, void* workspace, uint8_t* visited, cudaStream_t stream,
-               int num_sms, unsigned phases, const DropArgs& dr) {
+               int num_sms, unsigned phases, const DropArgs& dr, const Packed& pk) {
   using Cfg = fa::BwdCfg<D>;
-  const long long rows = static_cast<long long>(B) * H * N;
+  // rows of the dQ accumulator and of dQ (packed: tokens x heads)
+  const long long rows = pk.cu ? static_cast<long long>(pk.T) * H : static_cast<long long>(B) * H * N;
   const WsLayout wl = ws_layout(B, H, N, D);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* delta = reinterpret_cast<float*>(ws + wl.delta);
@@ -262,14 +330,19 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
   int* counter = reinterpret_cast<int*>(ws + wl.counter);
   CUtensorMap tq, tk, tv, tdo, tdq, tdk, tdv;
   const int BH = B * H;
-  if (!make_tmap(&tq, q, BH, N, D) || !make_tmap(&tk, k, BH, N, D) || !make_tmap(&tv, v, BH, N, D) ||
-      !make_tmap(&tdo, dout, BH, N, D) || !make_tmap_f32_acc(&tdq, dq_acc, BH, N, D) ||
-      !make_tmap(&tdk, dk, BH, N, D) || !make_tmap(&tdv, dv, BH, N, D))
+  const bool acc_ok = pk.cu ? make_tmap_f32_acc_packed(&tdq, dq_acc, H, pk.T, D)
+                            : make_tmap_f32_acc(&tdq, dq_acc, BH, N, D);
+  if (!make_tmap_any(&tq, q, B, H, N, D, pk) || !make_tmap_any(&tk, k, B, H, N, D, pk) ||
+      !make_tmap_any(&tv, v, B, H, N, D, pk) || !make_tmap_any(&tdo, dout, B, H, N, D, pk) ||
+      !acc_ok || !make_tmap_any(&tdk, dk, B, H, N, D, pk) ||
+      !make_tmap_any(&tdv, dv, B, H, N, D, pk))
     return FA_ERR_CUDA;
   static bool smem_set = false;
   if (!smem_set) {
-    if (!set_smem(fa::fa_bwd_kernel<D, false>, Cfg::kSmemBytes) ||
-        !set_smem(fa::fa_bwd_kernel<D, true>, Cfg::kSmemBytes))
+    if (!set_smem(fa::fa_bwd_kernel<D, false, false>, Cfg::kSmemBytes) ||
+        !set_smem(fa::fa_bwd_kernel<D, true, false>, Cfg::kSmemBytes) ||
+        !set_smem(fa::fa_bwd_kernel<D, false, true>, Cfg::kSmemBytes) ||
+        !set_smem(fa::fa_bwd_kernel<D, true, true>, Cfg::kSmemBytes))
       return FA_ERR_CUDA;
     smem_set = true;
   }
@@ -278,12 +351,18 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
     const int threads = 256;
     const int Np = (N + fa::kTile - 1) / fa::kTile * fa::kTile;
     const long long rows_p = static_cast<long long>(B) * H * Np;
-    long long blocks = (rows * (D / 4) + threads - 1) / threads;
+    const long long work = (rows > rows_p ? rows : rows_p) * (D / 4);
+    long long blocks = (work + threads - 1) / threads;
     const long long cap = static_cast<long long>(num_sms) * 8;
     if (blocks > cap) blocks = cap;
-    fa::fa_bwd_pre_kernel<D><<<static_cast<int>(blocks), threads, 0, stream>>>(
-        o, dout, lse, delta, lse2, reinterpret_cast<float4*>(dq_acc), counter, N, Np, rows_p,
-        rows);
+    if (pk.cu)
+      fa::fa_bwd_pre_packed_kernel<D><<<static_cast<int>(blocks), threads, 0, stream>>>(
+          o, dout, lse, delta, lse2, reinterpret_cast<float4*>(dq_acc), counter, pk.cu, H, N, Np,
+          pk.T, rows_p, rows);
+    else
+      fa::fa_bwd_pre_kernel<D><<<static_cast<int>(blocks), threads, 0, stream>>>(
+          o, dout, lse, delta, lse2, reinterpret_cast<float4*>(dq_acc), counter, N, Np, rows_p,
+          rows);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   // main
@@ -297,6 +376,9 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
     p.block_mask = block_mask;
     p.kv_len = kv_len;
     p.visited = visited;
+    p.cu_seqlens = pk.cu;
+    p.T = pk.T;
+    p.o_stride = pk.cu ? static_cast<long long>(H) * D : D;
     p.B = B;
     p.H = H;
     p.N = N;
@@ -309,11 +391,17 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
     p.scale_log2 = scale * fa::kLog2e;
     set_drop(p, dr);
     const int grid = p.num_units < num_sms ? p.num_units : num_sms;
-    if (dr.on)
-      fa::fa_bwd_kernel<D, true>
+    if (pk.cu && dr.on)
+      fa::fa_bwd_kernel<D, true, true>
+          <<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdq, tdk, tdv, p);
+    else if (pk.cu)
+      fa::fa_bwd_kernel<D, false, true>
+          <<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdq, tdk, tdv, p);
+    else if (dr.on)
+      fa::fa_bwd_kernel<D, true, false>
           <<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdq, tdk, tdv, p);
     else
-      fa::fa_bwd_kernel<D, false>
+      fa::fa_bwd_kernel<D, false, false>
           <<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdq, tdk, tdv, p);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
@@ -343,6 +431,9 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
     sp.block_mask = block_mask;
     sp.kv_len = kv_len;
     sp.visited = nullptr;
+    sp.cu_seqlens = nullptr;  // the ordered dQ kernel takes the [B][H][N][d] layout only
+    sp.T = 0;
+    sp.o_stride = D;
     sp.B = B;
     sp.H = H;
     sp.N = N;
@@ -366,7 +457,7 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
 int fwd_impl(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o, float* lse, int B,
              int H, int N, int d, float scale, int causal, const uint8_t* block_mask,
              const int32_t* kv_len, uint8_t* visited, void* stream,
-             const DropArgs& dr = DropArgs()) {
+             const DropArgs& dr = DropArgs(), const Packed& pk = Packed()) {
   int rc = check_shape(B, H, N, d);
   if (rc == 1) return FA_OK;
   if (rc != FA_OK) return rc;
@@ -381,16 +472,17 @@ int fwd_impl(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o, f
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (d == 64)
     return launch_fwd<64>(q, k, v, o, lse, B, H, N, scale, causal, block_mask, kv_len, visited, s,
-                          sms, dr);
+                          sms, dr, pk);
   return launch_fwd<128>(q, k, v, o, lse, B, H, N, scale, causal, block_mask, kv_len, visited, s,
-                         sms, dr);
+                         sms, dr, pk);
 }
 
 int bwd_impl(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf16* o,
              const float* lse, const fa_bf16* dout, fa_bf16* dq, fa_bf16* dk, fa_bf16* dv, int B,
              int H, int N, int d, float scale, int causal, const uint8_t* block_mask,
              const int32_t* kv_len, void* workspace, size_t workspace_bytes, uint8_t* visited,
-             void* stream, unsigned phases = 7u, const DropArgs& dr = DropArgs()) {
+             void* stream, unsigned phases = 7u, const DropArgs& dr = DropArgs(),
+             const Packed& pk = Packed()) {
   int rc = check_shape(B, H, N, d);
   if (rc == 1) return FA_OK;
   if (rc != FA_OK) return rc;
@@ -409,9 +501,9 @@ int bwd_impl(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf16
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (d == 64)
     return launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, scale, causal, block_mask,
-                          kv_len, workspace, visited, s, sms, phases, dr);
+                          kv_len, workspace, visited, s, sms, phases, dr, pk);
   return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, scale, causal, block_mask,
-                         kv_len, workspace, visited, s, sms, phases, dr);
+                         kv_len, workspace, visited, s, sms, phases, dr, pk);
 }
 
 }  // namespace
@@ -505,6 +597,43 @@ int fa_selftest_wait_timeout(int arrive, unsigned int limit_us, int* result, voi
   fa::fa_selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
       arrive ? 1 : 0, 1000ull * limit_us, result);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int fa_fwd_varlen(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o, float* lse,
+                  const int32_t* cu_seqlens, int B, int H, int max_seqlen, int total_tokens, int d,
+                  float scale, int causal, float p_drop, uint64_t seed, uint32_t offset,
+                  void* stream) {
+  DropArgs dr;
+  int rc = make_drop(p_drop, seed, offset, &dr);
+  if (rc != FA_OK) return rc;
+  if (p_drop == 0.f) dr = DropArgs();  // keep-all: the kernels without dropout
+  rc = check_packed(cu_seqlens, B, H, max_seqlen, total_tokens, d);
+  if (rc == 1) return FA_OK;
+  if (rc != FA_OK) return rc;
+  Packed pk;
+  pk.cu = cu_seqlens;
+  pk.T = total_tokens;
+  return fwd_impl(q, k, v, o, lse, B, H, max_seqlen, d, scale, causal, nullptr, nullptr, nullptr,
+                  stream, dr, pk);
+}
+
+int fa_bwd_varlen(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf16* o,
+                  const float* lse, const fa_bf16* dout, fa_bf16* dq, fa_bf16* dk, fa_bf16* dv,
+                  const int32_t* cu_seqlens, int B, int H, int max_seqlen, int total_tokens, int d,
+                  float scale, int causal, float p_drop, uint64_t seed, uint32_t offset,
+                  void* workspace, size_t workspace_bytes, void* stream) {
+  DropArgs dr;
+  int rc = make_drop(p_drop, seed, offset, &dr);
+  if (rc != FA_OK) return rc;
+  if (p_drop == 0.f) dr = DropArgs();
+  rc = check_packed(cu_seqlens, B, H, max_seqlen, total_tokens, d);
+  if (rc == 1) return FA_OK;
+  if (rc != FA_OK) return rc;
+  Packed pk;
+  pk.cu = cu_seqlens;
+  pk.T = total_tokens;
+  return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, B, H, max_seqlen, d, scale, causal, nullptr,
+                  nullptr, workspace, workspace_bytes, nullptr, stream, 7u, dr, pk);
 }
 
 int fa_get_device_status(void* stream) {

@@ -113,6 +113,68 @@ __global__ void __launch_bounds__(256, 8) fa_bwd_pre_kernel(const uint16_t* __re
     dq_acc[e] = z;
 }
 
+// The same for packed variable-length batches: O, dO [T][H][d], LSE [H][T];
+// D and LSE2 in the per-head padded layout of the unit grid ([B*H][Np], Np =
+// the longest sequence rounded up to 128), rows past a sequence's end as
+// padding; the accumulator is [T][H][d] (acc_rows = T * H rows).
+template <int D>
+__global__ void __launch_bounds__(256, 8) fa_bwd_pre_packed_kernel(
+    const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
+    const float* __restrict__ lse, float* __restrict__ delta, float* __restrict__ lse2,
+    float4* __restrict__ dq_acc, int* __restrict__ work_counter,
+    const int32_t* __restrict__ cu_seqlens, int H, int N, int Np, int T, long long rows_p,
+    long long acc_rows) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) *work_counter = 0;
+  constexpr int kLanesPerRow = D / 8;
+  constexpr int kRowsPerWarp = 32 / kLanesPerRow;
+  const long long warp_global = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5;
+  const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int sub = lane / kLanesPerRow;
+  const int part = lane % kLanesPerRow;
+  for (long long r0 = warp_global * kRowsPerWarp; r0 < rows_p; r0 += nwarps * kRowsPerWarp) {
+    const long long pr = r0 + sub;
+    bool valid = pr < rows_p;
+    long long orow = 0, lrow = 0;  // O / dO row (of T * H) and LSE index
+    if (valid) {
+      const int bh = static_cast<int>(pr / Np);
+      const int rr = static_cast<int>(pr - static_cast<long long>(bh) * Np);
+      const int b = bh / H, h = bh - b * H;
+      const SeqSpan sp = seq_span(cu_seqlens, b, N, T);
+      valid = rr < sp.len;
+      orow = (static_cast<long long>(sp.start) + rr) * H + h;
+      lrow = static_cast<long long>(h) * T + sp.start + rr;
+    }
+    float acc = 0.f;
+    if (valid) {
+      const uint4 a = __ldg(reinterpret_cast<const uint4*>(o + orow * D) + part);
+      const uint4 b = __ldg(reinterpret_cast<const uint4*>(dout + orow * D) + part);
+      const uint32_t av[4] = {a.x, a.y, a.z, a.w};
+      const uint32_t bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 fa2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&av[e]));
+        const float2 fb2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bv[e]));
+        acc = fmaf(fa2.x, fb2.x, acc);
+        acc = fmaf(fa2.y, fb2.y, acc);
+      }
+    }
+#pragma unroll
+    for (int off = kLanesPerRow / 2; off > 0; off >>= 1)
+      acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (pr < rows_p && part == 0) {
+      delta[pr] = valid ? -acc : 0.f;
+      const float l = valid ? lse[lrow] : -INFINITY;
+      lse2[pr] = (l == -INFINITY) ? -INFINITY : -l * kLog2e;
+    }
+  }
+  const long long n4 = acc_rows * (D / 4);
+  const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n4;
+       e += (long long)gridDim.x * blockDim.x)
+    dq_acc[e] = z;
+}
+
 // dQ = bf16(scale * accumulator), 8 elements per thread per step.
 __global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const float4* __restrict__ dq_acc,
                                                         uint4* __restrict__ dq, float scale,
@@ -141,6 +203,12 @@ struct BwdParams {
   int B, H, N, n_t;
   int num_units;
   int heads_per_group;  // unit order: see bwd_decode
+  // packed variable-length batches (null: the [B][H][N][d] layout), as in
+  // FwdParams; o_stride = elements between consecutive rows of one head's
+  // dK / dV
+  const int32_t* cu_seqlens;
+  int T;
+  long long o_stride;
   int* work_counter;    // next unit to take (zeroed by fa_bwd_pre_kernel)
   int causal;
   float scale;
@@ -193,7 +261,7 @@ struct BwdCfg {
   // here (kUnitRing slots of two int4) for the other roles
   static constexpr int kUnitRing = 4;
   static constexpr int kOffUnit = kOffRow + 2 * kQStages * kRowBytes;
-  static constexpr int kOffBar = kOffUnit + kUnitRing * 32;
+  static constexpr int kOffBar = kOffUnit + kUnitRing * 48;  // records of three int4
   static_assert(kOffEpi % 1024 == 0, "staging tiles must be 1024-byte aligned");
   // kv_full[KVS], kv_empty[KVS], q_full[QS], q_empty[QS], do_full[DS], do_empty[DS],
   // s_full, dp_full, p_full, ds_full, ds_smem_empty, dq_full, dq_empty, dkv_full,
@@ -242,6 +310,10 @@ struct BwdCfg {
 struct BwdUnit {
   int bh, b, j, L, i_begin, any, i_first;  // i_first: first visited query tile
   int valid;                                // 0: no unit left (end of the work)
+  int tok_base;  // row c of dK / dV is row tok_base + c of the [rows][o_stride] arrays
+  int tz;        // TMA third coordinate (the head; packed: h, at column h * d)
+  int nq;        // rows of this head (N, or the sequence's length)
+  int n_tq;      // query tiles of this head
 };
 
 __device__ __forceinline__ bool bwd_tile_on(const BwdParams& p, const BwdUnit& w, int i) {
@@ -251,14 +323,15 @@ __device__ __forceinline__ bool bwd_tile_on(const BwdParams& p, const BwdUnit& w
   return true;
 }
 
-// First visited query tile >= i (or n_t).
+// First visited query tile >= i (or n_tq).
 __device__ __forceinline__ int bwd_next(const BwdParams& p, const BwdUnit& w, int i) {
-  if (w.j * kTile >= w.L) return p.n_t;
-  for (; i < p.n_t; ++i)
+  if (w.j * kTile >= w.L) return w.n_tq;
+  for (; i < w.n_tq; ++i)
     if (bwd_tile_on(p, w, i)) return i;
-  return p.n_t;
+  return w.n_tq;
 }
 
+template <bool kPacked = false>
 __device__ __forceinline__ BwdUnit bwd_decode(const BwdParams& p, int u) {
   // heads in groups whose Q, dO and dQ accumulator fit in a share of L2; inside
   // a group key tile 0 first (for causal masks it sees the most queries)
@@ -266,20 +339,33 @@ __device__ __forceinline__ BwdUnit bwd_decode(const BwdParams& p, int u) {
   group_order(u, p.n_t, p.B * p.H, p.heads_per_group, w.bh, w.j);
   w.b = w.bh / p.H;
   int L = p.N;
-  if (p.kv_len) {
-    L = __ldg(p.kv_len + w.b);
-    L = L < 0 ? 0 : (L > p.N ? p.N : L);
+  if constexpr (kPacked) {
+    const SeqSpan sp = seq_span(p.cu_seqlens, w.b, p.N, p.T);
+    L = sp.len;
+    w.tok_base = sp.start;
+    w.tz = w.bh - w.b * p.H;
+    w.nq = sp.len;
+    w.n_tq = (sp.len + kTile - 1) / kTile;
+  } else {
+    if (p.kv_len) {
+      L = __ldg(p.kv_len + w.b);
+      L = L < 0 ? 0 : (L > p.N ? p.N : L);
+    }
+    w.tok_base = w.bh * p.N;
+    w.tz = w.bh;
+    w.nq = p.N;
+    w.n_tq = p.n_t;
   }
   w.L = L;
   w.i_begin = p.causal ? w.j : 0;
   w.i_first = bwd_next(p, w, w.i_begin);
-  w.any = w.i_first < p.n_t;
+  w.any = w.i_first < w.n_tq;
   w.valid = 1;
   return w;
 }
 
 
-template <int D, bool kDrop = false>
+template <int D, bool kDrop = false, bool kPacked = false>
 __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -311,12 +397,24 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
   // D = 64 epilogue: all 128 rows of warpgroup h's dK / dV tile are staged
   auto epi_ready = [&](int h) { return drain_bar + 40 + 8 * (2 * UR + h); };
   static_assert((2 * KVS + 2 * QS + 2 * DOS + 15 + 2 * UR) == Cfg::kNumBars, "barrier layout");
-  int4* unit_rec = reinterpret_cast<int4*>(smem + Cfg::kOffUnit);  // [UR][2]
+  int4* unit_rec = reinterpret_cast<int4*>(smem + Cfg::kOffUnit);  // [UR][3]
   // the warps that read each unit record: the MMA issuer(s), 8 dS and 4 dQ warps
   constexpr uint32_t kUnitReaders = (Cfg::kMultiIssue ? 3 : 1) + 12;
   auto load_unit = [&](int s) {
-    const int4 a = unit_rec[2 * s], b = unit_rec[2 * s + 1];
+    const int4 a = unit_rec[3 * s], b = unit_rec[3 * s + 1];
     BwdUnit w;
+    if constexpr (kPacked) {
+      const int4 c = unit_rec[3 * s + 2];
+      w.tok_base = c.x;
+      w.tz = c.y;
+      w.nq = c.z;
+      w.n_tq = c.w;
+    } else {
+      w.tok_base = a.x * p.N;
+      w.tz = a.x;
+      w.nq = p.N;
+      w.n_tq = p.n_t;
+    }
     w.bh = a.x;
     w.b = a.y;
     w.j = a.z;
@@ -430,15 +528,21 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         while (!ended && published <= round + 1) {
           const int un = atomicAdd(p.work_counter, 1);
           BwdUnit wr;
-          if (un < p.num_units) wr = bwd_decode(p, un);
+          if (un < p.num_units) {
+            wr = bwd_decode<kPacked>(p, un);
+            // packed batches: key tiles beyond a shorter sequence's end have
+            // no rows at all (nothing to compute or write): not published
+            if (kPacked && wr.j >= wr.n_tq) continue;
+          }
           const int s = published % UR;
           ok = mbar_wait(unit_empty(s), ((published / UR) & 1) ^ 1);
           if (!ok) break;
           if (un < p.num_units) {
-            unit_rec[2 * s] = make_int4(wr.bh, wr.b, wr.j, wr.L);
-            unit_rec[2 * s + 1] = make_int4(wr.i_begin, wr.any, wr.i_first, 1);
+            unit_rec[3 * s] = make_int4(wr.bh, wr.b, wr.j, wr.L);
+            unit_rec[3 * s + 1] = make_int4(wr.i_begin, wr.any, wr.i_first, 1);
+            if constexpr (kPacked) unit_rec[3 * s + 2] = make_int4(wr.tok_base, wr.tz, wr.nq, wr.n_tq);
           } else {
-            unit_rec[2 * s + 1] = make_int4(0, 0, p.n_t, 0);
+            unit_rec[3 * s + 1] = make_int4(0, 0, 0, 0);
             ended = true;
           }
           mbar_arrive(unit_full(s));
@@ -452,26 +556,31 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         ok = mbar_wait(kv_empty(skv), ((kv_cnt / KVS) & 1) ^ 1);
         if (!ok) break;
         ++kv_cnt;
-        const int krow = w.j * kTile;  // within head w.bh
+        // TMA rows: packed batches address the sequence's tokens (rows past its
+        // end belong to the next sequence: masked keys, queries whose
+        // contributions vanish through the padding -LSE2 = -inf)
+        const int trow0 = kPacked ? w.tok_base : 0;
+        const int2 kyz = tile_yz(kPacked, trow0 + w.j * kTile, w.tz);
         const uint32_t kv_off = skv * Cfg::kKvSlotBytes;
         mbar_arrive_expect_tx(kv_full(skv), 2 * Cfg::kTileBytes);
         for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
-          tma_load_3d(sbase + Cfg::kOffK + kv_off + bx * 16384, &tm_k, bx * 64, krow, w.bh,
+          tma_load_3d(sbase + Cfg::kOffK + kv_off + bx * 16384, &tm_k, bx * 64, kyz.x, kyz.y,
                       kv_full(skv));
-          tma_load_3d(sbase + Cfg::kOffV + kv_off + bx * 16384, &tm_v, bx * 64, krow, w.bh,
+          tma_load_3d(sbase + Cfg::kOffV + kv_off + bx * 16384, &tm_v, bx * 64, kyz.x, kyz.y,
                       kv_full(skv));
         }
-        for (int i = w.i_first; i < p.n_t && ok; i = bwd_next(p, w, i + 1)) {
+        for (int i = w.i_first; i < w.n_tq && ok; i = bwd_next(p, w, i + 1)) {
           // the tile's -LSE2 and -D rows (per-head padded layout: n_t * 128 rows
           // per head, so the 512-byte block is aligned and stays in the head)
           const long long qrow = (long long)w.bh * p.n_t * kTile + i * kTile;
+          const int2 qyz = tile_yz(kPacked, trow0 + i * kTile, w.tz);
           const int sq = q_cnt % QS;
           ok = mbar_wait(q_empty(sq), ((q_cnt / QS) & 1) ^ 1);
           if (!ok) break;
           mbar_arrive_expect_tx(q_full(sq), Cfg::kTileBytes + 2 * Cfg::kRowBytes);
           for (int bx = 0; bx < Cfg::kBoxes; ++bx)
             tma_load_3d(sbase + Cfg::kOffQ + sq * Cfg::kTileBytes + bx * 16384, &tm_q, bx * 64,
-                        i * kTile, w.bh, q_full(sq));
+                        qyz.x, qyz.y, q_full(sq));
           bulk_load(sbase + Cfg::kOffRow + sq * Cfg::kRowBytes, p.lse2 + qrow, Cfg::kRowBytes,
                     q_full(sq));
           bulk_load(sbase + Cfg::kOffRow + (QS + sq) * Cfg::kRowBytes, p.delta + qrow,
@@ -483,7 +592,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
           mbar_arrive_expect_tx(do_full(so), Cfg::kTileBytes);
           for (int bx = 0; bx < Cfg::kBoxes; ++bx)
             tma_load_3d(sbase + Cfg::kOffDO + so * Cfg::kTileBytes + bx * 16384, &tm_do, bx * 64,
-                        i * kTile, w.bh, do_full(so));
+                        qyz.x, qyz.y, do_full(so));
           ++do_cnt;
         }
         if (*abort_flag) ok = false;
@@ -565,7 +674,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         // reads dS^T(t) from the dP^T columns.
         int i = w.i_first;
         ok = issue_st(q_cnt, w, i) && issue_dpt(do_cnt);
-        for (int t = 0; ok && i < p.n_t; ++t) {
+        for (int t = 0; ok && i < w.n_tq; ++t) {
           const int inext = bwd_next(p, w, i + 1);
           const int sq = q_cnt % QS, so = do_cnt % DOS;
           const uint32_t q_off = (sq * Cfg::kTileBytes) >> 4;
@@ -585,7 +694,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
           ok = mbar_wait(ds_full, ds_cnt & 1);
           ++ds_cnt;
           if (!ok) break;
-          if (inext < p.n_t) {
+          if (inext < w.n_tq) {
             ok = issue_st(q_cnt + 1, w, inext);
             if (!ok) break;
           }
@@ -608,7 +717,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
           umma_commit(dq_full);
           umma_commit(ds_smem_empty);
           ++dq_cnt;
-          if (inext < p.n_t) {
+          if (inext < w.n_tq) {
             ok = issue_dpt(do_cnt);
             if (!ok) break;
           }
@@ -725,14 +834,14 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
           }
           return true;
         };
-        for (int t = 0; ok && i < p.n_t; ++t) {
+        for (int t = 0; ok && i < w.n_tq; ++t) {
           const int inext = bwd_next(p, w, i + 1);
           const int sq = q_cnt % QS, so = do_cnt % DOS;
           if (role == 0) {
             // S^T(t+1) once the math groups hold S^T(t) in registers
             ok = mbar_wait(s_free, t_cnt & 1);
             if (!ok) break;
-            if (inext < p.n_t) {
+            if (inext < w.n_tq) {
               ok = issue_st(q_cnt + 1, skv, w, inext);
             } else {
               BwdUnit wn;
@@ -768,7 +877,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
                       dq_m0 + q_off + ((kk * 2048) >> 4), idesc_tn,
                       (t > 0 || kk > 0) ? 1u : 0u);
             umma_commit(q_empty(sq));
-            if (inext < p.n_t) {
+            if (inext < w.n_tq) {
               ok = issue_dpt(do_cnt + 1, skv);
             } else {
               umma_commit(dkv_full);  // dK of the unit complete (with role 0's dV)
@@ -835,11 +944,19 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       ok = fetch_warp(round, w);
       if (!ok || !w.valid) break;
       const int c_key = w.j * kTile + kr;  // key index within the head
-      const size_t krow = (size_t)w.bh * p.N + c_key;
+      const long long krow = static_cast<long long>(w.tok_base) + c_key;
+      const int hcol = kPacked ? w.tz : 0;
       // warpgroup 0 writes the dK row, warpgroup 1 the dV row
-      uint4* out_row = reinterpret_cast<uint4*>((h ? p.dv : p.dk) + krow * D);
-      // key rows of a partial last tile beyond N belong to no output
-      const bool key_row_ok = c_key < p.N;
+      uint4* out_row = reinterpret_cast<uint4*>(
+          (h ? p.dv : p.dk) + krow * (kPacked ? p.o_stride : static_cast<long long>(D)) +
+          static_cast<long long>(hcol) * D);
+      // key rows of a partial last tile beyond N (packed: beyond the sequence)
+      // belong to no output
+      const bool key_row_ok = c_key < w.nq;
+      // The TMA store writes all 128 rows of the tile; the 3-D tensor map
+      // clips them at N, but in a packed batch rows past the sequence's end
+      // belong to the next sequence: such a tile is written row by row.
+      const bool epi_tma = Cfg::kEpiTma && !(kPacked && (w.j + 1) * kTile > w.nq);
       if (!w.any) {
 #pragma unroll
         for (int c = 0; c < D / 8; ++c)
@@ -847,7 +964,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         continue;
       }
       const bool key_valid = c_key < w.L;
-      for (int i = w.i_first; i < p.n_t; i = bwd_next(p, w, i + 1)) {
+      for (int i = w.i_first; i < w.n_tq; i = bwd_next(p, w, i + 1)) {
         const int sq = q_cnt % QS;
         ++q_cnt;
         const float4* lz4 = lse2_smem(sq) + h * 16;   // -LSE2
@@ -1092,7 +1209,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
 #pragma unroll
         for (int v4 = 0; v4 < 4; ++v4) {
           const uint4 val = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
-          if constexpr (Cfg::kEpiTma) {
+          if (epi_tma) {
             const int g = c * 4 + v4;  // 16-byte granule of the 128-byte row
             *reinterpret_cast<uint4*>(epi_row + ((g ^ (kr & 7)) << 4)) = val;
           } else if (key_row_ok) {
@@ -1101,7 +1218,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         }
       }
       tc_fence_before();
-      if constexpr (Cfg::kEpiTma) {
+      if (epi_tma) {
         // the whole tile is staged: one thread of the warpgroup stores it.
         // The staging area is written again only in the next unit's epilogue,
         // after dkv_full, which needs this thread's arrivals of that unit,
@@ -1111,7 +1228,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         if (kr == 0) {
           ok = mbar_wait(epi_ready(h), epi_cnt & 1);
           if (ok) {
-            tma_store_3d(h ? &tm_dv : &tm_dk, 0, w.j * kTile, w.bh,
+            const int2 yz = tile_yz(kPacked, (kPacked ? w.tok_base : 0) + w.j * kTile, w.tz);
+            tma_store_3d(h ? &tm_dv : &tm_dk, 0, yz.x, yz.y,
                          smem_u32(smem + Cfg::kOffEpi + h * Cfg::kTileBytes));
             bulk_commit_group();
             bulk_wait_group_read0();
@@ -1144,7 +1262,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       ok = fetch_warp(round, w);
       if (!ok || !w.valid) break;
       if (!w.any) continue;
-      for (int i = w.i_first; i < p.n_t; i = bwd_next(p, w, i + 1)) {
+      for (int i = w.i_first; i < w.n_tq; i = bwd_next(p, w, i + 1)) {
         ok = __all_sync(0xffffffffu, mbar_wait(dq_full, dq_cnt & 1));
         ++dq_cnt;
         if (!ok) break;
@@ -1157,7 +1275,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         for (int c = 0; c < D / 32; ++c) reg_fence32(r[c]);
         tc_fence_before();
         mbar_arrive(dq_empty);
-        const int y = i * kTile + quarter * 32;  // row within head w.bh
+        // row of the accumulator's tensor map (packed: token row; rows past the
+        // sequence's end receive exact or ~1e-38-scaled zeros, see above)
+        const int2 yz = tile_yz(kPacked, (kPacked ? w.tok_base : 0) + i * kTile + quarter * 32, w.tz);
 #pragma unroll
         for (int rd = 0; rd < Cfg::kDqRounds; ++rd) {
 #pragma unroll
@@ -1174,7 +1294,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
           if (lane == 0) {
 #pragma unroll
             for (int bxi = 0; bxi < Cfg::kDqBoxesPerRound; ++bxi)
-              tma_reduce_add_3d(&tm_dq, (rd * Cfg::kDqBoxesPerRound + bxi) * 32, y, w.bh,
+              tma_reduce_add_3d(&tm_dq, (rd * Cfg::kDqBoxesPerRound + bxi) * 32, yz.x, yz.y,
                                 stage_u32 + bxi * 4096);
             bulk_commit_group();
             bulk_wait_group_read0();

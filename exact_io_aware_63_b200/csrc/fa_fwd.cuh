@@ -90,12 +90,38 @@ __device__ __forceinline__ uint32_t keep_bits8(const uint4 d, uint32_t t_hi) {
   return b;
 }
 
+// Packed variable-length batches: sequence b holds tokens cu_seqlens[b] ..
+// cu_seqlens[b+1] - 1 of [T][H][d] tensors.  The values are clamped so that
+// every row index stays inside [0, T): the start into [0, T], the length into
+// [0, min(N, T - start)] (N = the longest sequence, the unit grid's size).
+struct SeqSpan {
+  int start, len;
+};
+__device__ __forceinline__ SeqSpan seq_span(const int32_t* cu, int b, int N, int T) {
+  const long long s = min(max(static_cast<long long>(__ldg(cu + b)), 0ll), static_cast<long long>(T));
+  const long long len = static_cast<long long>(__ldg(cu + b + 1)) - s;
+  const long long cap = min(static_cast<long long>(N), static_cast<long long>(T) - s);
+  return {static_cast<int>(s), static_cast<int>(max(0ll, min(len, cap)))};
+}
+
+// A 128-row tile of one head: [B*H][N][d] tensors are mapped as (d, N, B*H)
+// and packed [T][H][d] tensors as (d, H, T) (strides increasing in both), so
+// the tile's (row, head) are the map's (y, z), or (z, y) when packed.
+__device__ __forceinline__ int2 tile_yz(bool packed, int row, int head) {
+  return packed ? make_int2(head, row) : make_int2(row, head);
+}
+
 struct FwdParams {
   uint16_t* o;
   float* lse;
   const uint8_t* block_mask;
   const int32_t* kv_len;
   uint8_t* visited;
+  // packed variable-length batches (null: the [B][H][N][d] layout); N is then
+  // the longest sequence and T the number of tokens
+  const int32_t* cu_seqlens;
+  int T;
+  long long o_stride;  // elements between consecutive rows of one head's O (d, or H*d packed)
   int B, H, N, n_t;
   int num_units;
   int heads_per_group;  // unit order: see fwd_decode
@@ -156,6 +182,10 @@ __device__ __forceinline__ int unit_for_round(int round, int cta, int G) {
 
 struct FwdUnit {
   int bh, b;
+  int nq;        // query rows (N, or the sequence's length)
+  int tok_base;  // first row of this head: B*H*N rows (b*H+h)*N, or the sequence's first token
+  int tz;        // the head's TMA coordinate: b*H+h, or h (packed)
+  bool empty;    // packed: the unit's query tiles lie beyond its sequence
   int i0, i1;           // query tile of warpgroup 0 / 1 (split mode: the same tile)
   int has1;             // pair mode: query tile i1 exists
   int L;                // keys c < L are not padding
@@ -175,7 +205,7 @@ __device__ __forceinline__ void group_order(int u, int n_t, int BH, int G, int& 
   bh = h0 + (r - rank * gh);
 }
 
-template <bool kPair>
+template <bool kPair, bool kPacked = false>
 __device__ __forceinline__ FwdUnit fwd_decode(const FwdParams& p, int u) {
   FwdUnit w;
   const int per_head = kPair ? (p.n_t + 1) / 2 : p.n_t;
@@ -184,24 +214,54 @@ __device__ __forceinline__ FwdUnit fwd_decode(const FwdParams& p, int u) {
   w.b = w.bh / p.H;
   const int slot = p.causal ? (per_head - 1 - rank) : rank;
   int L = p.N;
-  if (p.kv_len) {
-    L = __ldg(p.kv_len + w.b);
-    L = L < 0 ? 0 : (L > p.N ? p.N : L);
+  int n_tq = p.n_t;  // query tiles of this head
+  if constexpr (kPacked) {
+    const SeqSpan sp = seq_span(p.cu_seqlens, w.b, p.N, p.T);
+    const int h = w.bh - w.b * p.H;
+    L = sp.len;
+    n_tq = (sp.len + kTile - 1) / kTile;
+    w.nq = sp.len;
+    w.tok_base = sp.start;
+    w.tz = h;
+  } else {
+    if (p.kv_len) {
+      L = __ldg(p.kv_len + w.b);
+      L = L < 0 ? 0 : (L > p.N ? p.N : L);
+    }
+    w.nq = p.N;
+    w.tok_base = w.bh * p.N;
+    w.tz = w.bh;
   }
   w.L = L;
   const int j_kv = (L + kTile - 1) / kTile;  // key tiles holding a key c < L
   if (kPair) {
     w.i0 = 2 * slot;
     w.i1 = 2 * slot + 1;
-    w.has1 = w.i1 < p.n_t;
+    w.has1 = w.i1 < n_tq;
   } else {
     w.i0 = w.i1 = slot;
     w.has1 = 0;
   }
+  w.empty = w.i0 >= n_tq;
   w.j_end0 = p.causal ? min(j_kv, w.i0 + 1) : j_kv;
   w.j_end1 = (kPair && !w.has1) ? 0 : (p.causal ? min(j_kv, w.i1 + 1) : j_kv);
   w.j_end = max(w.j_end0, w.j_end1);
   return w;
+}
+
+// The first round >= r whose unit has work, or one whose unit is past the
+// last (every role walks the same sequence).  Only packed batches have units
+// without work: query tiles beyond a shorter sequence's end.
+template <bool kPair, bool kPacked>
+__device__ __forceinline__ int live_round(const FwdParams& p, int r, int cta, int G) {
+  if constexpr (!kPacked) {
+    return r;
+  } else {
+    for (;; ++r) {
+      const int u = unit_for_round(r, cta, G);
+      if (u >= p.num_units || !fwd_decode<kPair, true>(p, u).empty) return r;
+    }
+  }
 }
 
 // Split mode: first key tile >= j that query tile w.i0 visits (or j_end):
@@ -216,7 +276,7 @@ __device__ __forceinline__ int fwd_next(const FwdParams& p, const FwdUnit& w, in
   return w.j_end;
 }
 
-template <int D, bool kPair, bool kDrop = false>
+template <int D, bool kPair, bool kDrop = false, bool kPacked = false>
 __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -303,36 +363,42 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
     if (lane == 0) {
       uint32_t q_cnt = 0, kv_cnt = 0;
       bool ok = true;
-      for (int round = 0; ok; ++round) {
+      for (int round = live_round<kPair, kPacked>(p, 0, blockIdx.x, G); ok;
+           round = live_round<kPair, kPacked>(p, round + 1, blockIdx.x, G)) {
         const int u = unit_for_round(round, blockIdx.x, G);
         if (u >= p.num_units) break;
-        const FwdUnit w = fwd_decode<kPair>(p, u);
+        const FwdUnit w = fwd_decode<kPair, kPacked>(p, u);
         const int qs = q_cnt % QSLOTS;
         ok = mbar_wait(q_empty(qs), ((q_cnt / QSLOTS) & 1) ^ 1);
         if (!ok) break;
         ++q_cnt;
         const int nq = (kPair && w.has1) ? 2 : 1;
         mbar_arrive_expect_tx(q_full(qs), nq * Cfg::kTileBytes);
-        for (int x = 0; x < nq; ++x)
+        for (int x = 0; x < nq; ++x) {
+          const int2 yz =
+              tile_yz(kPacked, (kPacked ? w.tok_base : 0) + (x ? w.i1 : w.i0) * kTile, w.tz);
           for (int bx = 0; bx < Cfg::kBoxes; ++bx)
-            tma_load_3d(q_tile(qs, x) + bx * 16384, &tm_q, bx * 64, (x ? w.i1 : w.i0) * kTile,
-                        w.bh, q_full(qs));
+            tma_load_3d(q_tile(qs, x) + bx * 16384, &tm_q, bx * 64, yz.x, yz.y, q_full(qs));
+        }
         for (int j = fwd_next(p, w, 0); j < w.j_end && ok; j = fwd_next(p, w, j + 1)) {
           const int s = kv_cnt % S;
           const uint32_t ph = (kv_cnt / S) & 1;
-          const int row = j * kTile;  // within head w.bh
+          // packed batches: rows past the sequence's end belong to the next
+          // sequence; they are masked (keys) or not stored (queries)
+          const int2 yz =
+              tile_yz(kPacked, (kPacked ? w.tok_base : 0) + j * kTile, w.tz);
           ok = mbar_wait(k_empty(s), ph ^ 1);
           if (!ok) break;
           mbar_arrive_expect_tx(k_full(s), Cfg::kTileBytes);
           for (int bx = 0; bx < Cfg::kBoxes; ++bx)
-            tma_load_3d(sbase + Cfg::kOffK + s * Cfg::kTileBytes + bx * 16384, &tm_k, bx * 64, row,
-                        w.bh, k_full(s));
+            tma_load_3d(sbase + Cfg::kOffK + s * Cfg::kTileBytes + bx * 16384, &tm_k, bx * 64,
+                        yz.x, yz.y, k_full(s));
           ok = mbar_wait(v_empty(s), ph ^ 1);
           if (!ok) break;
           mbar_arrive_expect_tx(v_full(s), Cfg::kTileBytes);
           for (int bx = 0; bx < Cfg::kBoxes; ++bx)
-            tma_load_3d(sbase + Cfg::kOffV + s * Cfg::kTileBytes + bx * 16384, &tm_v, bx * 64, row,
-                        w.bh, v_full(s));
+            tma_load_3d(sbase + Cfg::kOffV + s * Cfg::kTileBytes + bx * 16384, &tm_v, bx * 64,
+                        yz.x, yz.y, v_full(s));
           ++kv_cnt;
         }
         if (*abort_flag) ok = false;
@@ -363,10 +429,11 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
       uint32_t pre = 0;      // bit x: S_x of this unit's first key tile already issued
       bool pre_q = false;    // this unit's Q already waited for
       bool pre_k = false;    // this unit's first K tile already waited for
-      for (int round = 0; ok; ++round) {
+      for (int round = live_round<kPair, kPacked>(p, 0, blockIdx.x, G); ok;
+           round = live_round<kPair, kPacked>(p, round + 1, blockIdx.x, G)) {
         const int u = unit_for_round(round, blockIdx.x, G);
         if (u >= p.num_units) break;
-        const FwdUnit w = fwd_decode<kPair>(p, u);
+        const FwdUnit w = fwd_decode<kPair, kPacked>(p, u);
         const int qs = q_cnt % QSLOTS;
         if (!pre_q) ok = mbar_wait(q_full(qs), (q_cnt / QSLOTS) & 1);
         ++q_cnt;
@@ -407,10 +474,12 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
           // competing with it for issue slots.
           const int j_end = w.j_end;
           // the next unit (look-ahead)
-          const int un = unit_for_round(round + 1, blockIdx.x, G);
+          const int un =
+              unit_for_round(live_round<kPair, kPacked>(p, round + 1, blockIdx.x, G), blockIdx.x,
+                             G);
           const bool has_next = kLook && un < p.num_units;
           FwdUnit wn = w;
-          if (has_next) wn = fwd_decode<kPair>(p, un);
+          if (has_next) wn = fwd_decode<kPair, kPacked>(p, un);
           const int qsn = q_cnt % QSLOTS;
           const uint32_t cn = kv_cnt + j_end;  // ring index of the next unit's first tile
           uint32_t pre_next = 0;
@@ -606,10 +675,11 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
       uint32_t t_cnt = 0;              // tiles of this warpgroup (s_free / p_full phases)
       bool pre = false;                // this unit's Q awaited and first own S issued
       bool ok = true;
-      for (int round = 0; ok; ++round) {
+      for (int round = live_round<kPair, kPacked>(p, 0, blockIdx.x, G); ok;
+           round = live_round<kPair, kPacked>(p, round + 1, blockIdx.x, G)) {
         const int u = unit_for_round(round, blockIdx.x, G);
         if (u >= p.num_units) break;
-        const FwdUnit w = fwd_decode<kPair>(p, u);
+        const FwdUnit w = fwd_decode<kPair, kPacked>(p, u);
         const int qs = q_cnt % QSLOTS;
         const uint32_t q_par = (q_cnt / QSLOTS) & 1;
         ++q_cnt;
@@ -648,9 +718,11 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
           } else {
             umma_commit(q_empty(qs));  // this warpgroup's last S on this Q is issued
             if constexpr (kLook) {
-              const int un = unit_for_round(round + 1, blockIdx.x, G);
+              const int un =
+              unit_for_round(live_round<kPair, kPacked>(p, round + 1, blockIdx.x, G), blockIdx.x,
+                             G);
               if (un < p.num_units) {
-                const FwdUnit wn = fwd_decode<kPair>(p, un);
+                const FwdUnit wn = fwd_decode<kPair, kPacked>(p, un);
                 if ((x ? wn.j_end1 : wn.j_end0) > 0) {
                   const int qsn = q_cnt % QSLOTS;
                   const uint32_t cn = kv_cnt + w.j_end;
@@ -722,10 +794,11 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
     uint32_t s_cnt = 0, unit_cnt = 0;
     uint32_t o_cnt[2] = {0, 0};
     bool ok = true;
-    for (int round = 0; ok; ++round) {
+    for (int round = live_round<kPair, kPacked>(p, 0, blockIdx.x, G); ok;
+           round = live_round<kPair, kPacked>(p, round + 1, blockIdx.x, G)) {
       const int u = unit_for_round(round, blockIdx.x, G);
       if (u >= p.num_units) break;
-      const FwdUnit w = fwd_decode<kPair>(p, u);
+      const FwdUnit w = fwd_decode<kPair, kPacked>(p, u);
       if (kPair && x == 1 && !w.has1) continue;  // pair with no second tile
       const int i_me = x ? w.i1 : w.i0;           // this warpgroup's query tile
       const int j_end_me = x ? w.j_end1 : w.j_end0;
@@ -879,11 +952,18 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
         if (*abort_flag) { ok = false; break; }
       }
       if (!ok) break;
-      const size_t grow = (size_t)w.bh * p.N + row;
-      const bool row_ok = row < p.N;  // rows of a partial last tile beyond N are not output
+      // rows of a partial last tile beyond N (packed: beyond the sequence) are
+      // not output
+      const bool row_ok = row < w.nq;
+      // O row: [B*H*N][d], or [T][H][d] at column h*d; LSE: [B*H*N], or [H][T]
+      uint16_t* const o_row = p.o + (static_cast<long long>(w.tok_base) + row) *
+                                        (kPacked ? p.o_stride : static_cast<long long>(D)) +
+                              (kPacked ? static_cast<long long>(w.tz) * D : 0ll);
+      float* const lse_ptr = p.lse + (kPacked ? static_cast<long long>(w.tz) * p.T : 0ll) +
+                             w.tok_base + row;
       if constexpr (kPair) {
         // ---------------------------------------------------- epilogue (own tile)
-        uint4* orow = reinterpret_cast<uint4*>(p.o + grow * D);
+        uint4* orow = reinterpret_cast<uint4*>(o_row);
         if (cnt > 0) {
           ok = __all_sync(0xffffffffu, mbar_wait(o_full(x), o_cnt[x] & 1));
           ++o_cnt[x];
@@ -908,12 +988,12 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
                     make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
           }
           tc_fence_before();
-          if (row_ok) p.lse[grow] = (l > 0.f) ? (m_used + log2f(l)) * kLn2 : -INFINITY;
+          if (row_ok) *lse_ptr = (l > 0.f) ? (m_used + log2f(l)) * kLn2 : -INFINITY;
         } else {
 #pragma unroll
           for (int c = 0; c < D / 8; ++c)
             if (row_ok) orow[c] = make_uint4(0, 0, 0, 0);
-          if (row_ok) p.lse[grow] = -INFINITY;
+          if (row_ok) *lse_ptr = -INFINITY;
         }
       } else {
         // ---------------------------------------------------- merge + epilogue
@@ -943,7 +1023,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
         const float lt = ml0.y * a0 + ml1.y * a1;
         const float inv_l = (lt > 0.f) ? (kDrop ? p.drop.w : 1.f) / lt : 0.f;
         const float f0 = a0 * inv_l, f1 = a1 * inv_l;
-        uint4* orow = reinterpret_cast<uint4*>(p.o + grow * D + x * (D / 2));
+        uint4* orow = reinterpret_cast<uint4*>(o_row + x * (D / 2));
         // A warpgroup that processed no tile left its O unwritten: its factor is 0
         // and its values are dropped by a select (never multiplied, in case the
         // unwritten columns hold a NaN pattern).
@@ -972,7 +1052,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
               orow[c * 4 + v4] =
                   make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
         }
-        if (x == 0 && row_ok) p.lse[grow] = (lt > 0.f) ? (m + log2f(lt)) * kLn2 : -INFINITY;
+        if (x == 0 && row_ok) *lse_ptr = (lt > 0.f) ? (m + log2f(lt)) * kLn2 : -INFINITY;
         tc_fence_before();
         // neither warpgroup starts the next unit (whose first P V overwrites an O)
         // before both have read both partial outputs

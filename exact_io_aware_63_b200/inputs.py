@@ -144,3 +144,49 @@ def workload_inputs(name: str) -> Inputs:
     return make_inputs(w.B, w.H, w.N, w.d, scale=w.scale, causal=w.causal, seed=w.seed,
                        key_padding=(256, 512) if w.key_padding else None,
                        block_keep=(1.0 / 16.0) if w.block_sparse else None)
+
+
+@dataclasses.dataclass
+class PackedInputs:
+    """A packed variable-length batch on the host: q, k, v, dout bfloat16 [T, H, d];
+    sequence b is tokens cu_seqlens[b] .. cu_seqlens[b+1]-1."""
+    q: torch.Tensor
+    k: torch.Tensor
+    v: torch.Tensor
+    dout: torch.Tensor
+    cu_seqlens: torch.Tensor  # int32 [B + 1]
+    max_seqlen: int
+    scale: float
+    causal: bool
+
+    @property
+    def lengths(self):
+        return [int(self.cu_seqlens[b + 1] - self.cu_seqlens[b])
+                for b in range(len(self.cu_seqlens) - 1)]
+
+
+def make_packed_inputs(lengths, H: int, d: int, *, scale: Optional[float] = None,
+                       causal: bool = False, seed: int = 0) -> PackedInputs:
+    """q, k, v, dO ~ N(0,1) (float32 -> bfloat16) for sequences of the given lengths,
+    packed token by token ([T, H, d], T = sum of lengths), drawn in the order q, k, v, dO."""
+    lengths = [int(n) for n in lengths]
+    cu = torch.zeros(len(lengths) + 1, dtype=torch.int32)
+    if lengths:
+        cu[1:] = torch.cumsum(torch.tensor(lengths, dtype=torch.int64), 0).to(torch.int32)
+    T = int(cu[-1])
+    gen = torch.Generator().manual_seed(int(seed))
+    shape = (T, H, d)
+
+    def draw():
+        return torch.randn(shape, generator=gen, dtype=torch.float32).to(torch.bfloat16)
+
+    q, k, v, dout = draw(), draw(), draw(), draw()
+    return PackedInputs(q, k, v, dout, cu, max(lengths) if lengths else 0,
+                        float(scale if scale is not None else 1.0 / math.sqrt(d)), bool(causal))
+
+
+def draw_lengths(B: int, lo: int, hi: int, seed: int):
+    """B sequence lengths uniform on the integers lo..hi (inclusive), from ``seed``."""
+    gen = torch.Generator().manual_seed(int(seed))
+    u = torch.rand(B, generator=gen, dtype=torch.float64)
+    return [int(x) for x in (lo + torch.floor(u * (hi - lo + 1))).to(torch.int64)]

@@ -208,6 +208,43 @@ int fa_bwd_dropout(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const f
                    void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Packed variable-length batches: B sequences of different lengths stored
+ * token after token, with no padding.  Sequence b is tokens cu_seqlens[b] ..
+ * cu_seqlens[b+1] - 1, and each sequence is its own attention problem (the
+ * operation above with N = its length; causal masks are top-left aligned
+ * within the sequence).
+ *  - Q, K, V, O, dO, dQ, dK, dV: bfloat16 [T][H][d] (T = total_tokens =
+ *    cu_seqlens[B]), 16-byte aligned; LSE: float32 [H][T].
+ *  - cu_seqlens: int32 [B + 1] in device memory, 4-byte aligned, with
+ *    cu_seqlens[0] = 0, non-decreasing, cu_seqlens[B] = T, and every length at
+ *    most max_seqlen.  The kernels clamp each sequence into [0, T) and its
+ *    length into [0, max_seqlen], so inconsistent values give wrong results
+ *    for those sequences but never an access outside the tensors.
+ *  - Host checks: B, H, max_seqlen, total_tokens >= 0 (FA_ERR_SHAPE);
+ *    total_tokens <= B * max_seqlen (FA_ERR_SHAPE); B*H*max_seqlen < 2^31;
+ *    cu_seqlens non-NULL (FA_ERR_NULL) and 4-byte aligned (FA_ERR_ALIGN); d,
+ *    scale and p_drop as elsewhere.  If B, H, max_seqlen or total_tokens is 0
+ *    the call does nothing and returns FA_OK.
+ *  - p_drop, seed, offset: dropout as in fa_fwd_dropout (p_drop = 0: none);
+ *    the draws number heads b*H + h and rows and keys within the sequence.
+ *  - No block mask and no kv_len (a sequence's length is its key length).
+ *  - fa_bwd_varlen's workspace: fa_bwd_workspace_size(B, H, max_seqlen, d)
+ *    bytes, 256-byte aligned.
+ * Work is scheduled on the grid of B x H x ceil(max_seqlen / 128) tiles;
+ * tiles past a shorter sequence's end are skipped.
+ */
+int fa_fwd_varlen(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o, float* lse,
+                  const int32_t* cu_seqlens, int B, int H, int max_seqlen, int total_tokens, int d,
+                  float scale, int causal, float p_drop, uint64_t seed, uint32_t offset,
+                  void* stream);
+
+int fa_bwd_varlen(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf16* o,
+                  const float* lse, const fa_bf16* dout, fa_bf16* dq, fa_bf16* dk, fa_bf16* dv,
+                  const int32_t* cu_seqlens, int B, int H, int max_seqlen, int total_tokens, int d,
+                  float scale, int causal, float p_drop, uint64_t seed, uint32_t offset,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Self-test of the failure path every kernel relies on.  Each pipeline wait
  * in the kernels is bounded in time; when a wait gives up, the kernel records
  * a timeout in a device status word, winds down and exits, and

@@ -33,6 +33,13 @@ Functions (all arrays contiguous, float64 unless stated):
   arguments ``p_drop, seed, offset``): the same with dropout on P; the mask is
   ``dropout_keep(BH, N, p_drop, seed, offset)``, cut from Philox-4x32-10 draws
   (``philox4x32_10(counter, key)``).
+* ``attention_forward_varlen(q, k, v, cu_seqlens, scale, causal, dropout)`` /
+  ``attention_backward_varlen(q, k, v, dout, cu_seqlens, scale, causal,
+  dropout)``: packed variable-length batches (q, k, v, dout [T, H, d];
+  sequence b = tokens cu_seqlens[b] .. cu_seqlens[b+1]-1), each sequence its
+  own attention problem; computed through the functions above on the
+  zero-padded [B, H, N, d] problem with key lengths kv_len = the sequence
+  lengths, keeping each sequence's own rows.
 * ``tile_visits(B, N, causal, block_mask, kv_len, T=128, i_begin=0,
   i_end=None)`` -> uint8 [B, i_end - i_begin, ceil(N / T)]: 1 where a
   (query tile, key tile) pair holds at least one allowed (row, key).
@@ -340,3 +347,68 @@ def tile_visits(B, N, causal=False, block_mask=None, kv_len=None, T=128, i_begin
     if rc != 0:
         raise RuntimeError(f"oracle_tile_visits failed: {rc}")
     return out
+
+
+def _unpack_lengths(cu_seqlens):
+    cu = [int(c) for c in np.asarray(cu_seqlens)]
+    return cu, [cu[b + 1] - cu[b] for b in range(len(cu) - 1)]
+
+
+def _pad(x, cu, lens, N):
+    """[T, H, d] -> zero-padded [B, H, N, d]."""
+    T, H, d = x.shape
+    out = np.zeros((len(lens), H, N, d), np.float64)
+    for b, n in enumerate(lens):
+        out[b, :, :n] = np.transpose(x[cu[b]:cu[b] + n], (1, 0, 2))
+    return out
+
+
+def _unpad(x, cu, lens, T):
+    """[B, H, N, d] -> [T, H, d] (each sequence's own rows)."""
+    H, d = x.shape[1], x.shape[3]
+    out = np.zeros((T, H, d), np.float64)
+    for b, n in enumerate(lens):
+        out[cu[b]:cu[b] + n] = np.transpose(x[b, :, :n], (1, 0, 2))
+    return out
+
+
+def attention_forward_varlen(q, k, v, cu_seqlens, scale, causal=False, dropout=None,
+                             nthreads=None):
+    """(o [T, H, d], lse [H, T]) of a packed variable-length batch.  Sequence b is the
+    attention problem of its own tokens; as the zero-padded [B, H, N, d] problem with
+    kv_len = lengths its rows are unchanged (padded keys are masked).  ``dropout`` is
+    None or (p_drop, seed, offset); heads are numbered b*H + h, rows and keys within
+    the sequence."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    T, H, d = q.shape
+    cu, lens = _unpack_lengths(cu_seqlens)
+    N = max(lens) if lens else 0
+    kl = np.array(lens, np.int32)
+    qp, kp, vp = (_pad(x, cu, lens, N) for x in (q, k, v))
+    if dropout is None:
+        o, lse = attention_forward(qp, kp, vp, scale, causal, None, kl, nthreads)
+    else:
+        o, lse = attention_forward_dropout(qp, kp, vp, scale, dropout[0], dropout[1], dropout[2],
+                                           causal, None, kl, nthreads)
+    lse_p = np.full((H, T), -np.inf)
+    for b, n in enumerate(lens):
+        lse_p[:, cu[b]:cu[b] + n] = lse[b, :, :n]
+    return _unpad(o, cu, lens, T), lse_p
+
+
+def attention_backward_varlen(q, k, v, dout, cu_seqlens, scale, causal=False, dropout=None,
+                              nthreads=None):
+    """(dq, dk, dv) [T, H, d] of sum(O * dO) for the packed batch.  In the padded
+    problem the padded rows get dO = 0, so they add nothing to any gradient."""
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    T, H, d = q.shape
+    cu, lens = _unpack_lengths(cu_seqlens)
+    N = max(lens) if lens else 0
+    kl = np.array(lens, np.int32)
+    qp, kp, vp, dp = (_pad(x, cu, lens, N) for x in (q, k, v, dout))
+    if dropout is None:
+        dq, dk, dv, _ = attention_backward(qp, kp, vp, dp, scale, causal, None, kl, nthreads)
+    else:
+        dq, dk, dv, _ = attention_backward_dropout(qp, kp, vp, dp, scale, dropout[0], dropout[1],
+                                                   dropout[2], causal, None, kl, nthreads)
+    return tuple(_unpad(x, cu, lens, T) for x in (dq, dk, dv))

@@ -24,7 +24,7 @@ def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ["fa_fwd", "fa_fwd_traced", "fa_bwd", "fa_bwd_traced", "fa_bwd_phase",
               "fa_bwd_deterministic", "fa_fwd_dropout", "fa_bwd_dropout",
-              "fa_selftest_wait_timeout",
+              "fa_selftest_wait_timeout", "fa_fwd_varlen", "fa_bwd_varlen",
               "fa_bwd_workspace_size",
               "fa_get_device_status", "fa_status_string", "fa_version"]:
         assert n in names
@@ -193,3 +193,48 @@ def test_selftest_arguments_are_checked():
     assert lib.fa_selftest_wait_timeout(0, 1000, P + 2, None) == -2
     assert lib.fa_selftest_wait_timeout(0, 0, P, None) == -8
     assert lib.fa_selftest_wait_timeout(0, 2_000_001, P, None) == -8
+
+
+def fwd_varlen(**kw):
+    a = dict(q=P, k=P, v=P, o=P, lse=P, cu=P, B=2, H=1, max_seqlen=128, T=200, d=64, scale=0.125,
+             causal=0, p_drop=0.0)
+    a.update(kw)
+    return binding.load().fa_fwd_varlen(a["q"], a["k"], a["v"], a["o"], a["lse"], a["cu"], a["B"],
+                                        a["H"], a["max_seqlen"], a["T"], a["d"], a["scale"],
+                                        a["causal"], a["p_drop"], 0, 0, None)
+
+
+def bwd_varlen(**kw):
+    a = dict(q=P, k=P, v=P, o=P, lse=P, dout=P, dq=P, dk=P, dv=P, cu=P, B=2, H=1, max_seqlen=128,
+             T=200, d=64, scale=0.125, causal=0, p_drop=0.0, ws=P, ws_bytes=1 << 30)
+    a.update(kw)
+    return binding.load().fa_bwd_varlen(a["q"], a["k"], a["v"], a["o"], a["lse"], a["dout"],
+                                        a["dq"], a["dk"], a["dv"], a["cu"], a["B"], a["H"],
+                                        a["max_seqlen"], a["T"], a["d"], a["scale"], a["causal"],
+                                        a["p_drop"], 0, 0, a["ws"], a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("call", [fwd_varlen, bwd_varlen])
+def test_varlen_argument_checks(call):
+    assert call(B=-1) == -3
+    assert call(T=-5) == -3
+    assert call(max_seqlen=-1) == -3
+    assert call(T=300) == -3                   # more tokens than B * max_seqlen
+    assert call(d=96) == -4
+    assert call(cu=None) == -1
+    assert call(cu=P + 2) == -2
+    assert call(q=None) == -1
+    assert call(k=P + 8) == -2
+    assert call(scale=0.0) == -8
+    assert call(p_drop=1.0) == -8
+    # empty problems do nothing
+    assert call(B=0, cu=None) == 0
+    assert call(T=0, cu=None) == 0
+    assert call(max_seqlen=0, T=0, cu=None) == 0
+    assert call(H=0) == 0
+
+
+def test_varlen_backward_workspace_checks():
+    assert bwd_varlen(ws=None) == -5
+    assert bwd_varlen(ws_bytes=64) == -5
+    assert bwd_varlen(ws=P + 16) == -2

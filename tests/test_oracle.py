@@ -532,3 +532,51 @@ def test_dropout_finite_difference_gradients(causal, kv):
             num[idx] = (loss(*a_p) - loss(*a_m)) / (2 * h)
         err = np.linalg.norm(num - g) / np.linalg.norm(g)
         assert err < 1e-7, (name, err)
+
+
+# ---------------------------------------------------------------------------
+# packed variable-length batches: each sequence is its own attention problem
+# ---------------------------------------------------------------------------
+
+def _packed(lengths, H, d, seed):
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    T = int(cu[-1])
+    q, k, v, do = (rand((T, H, d), seed + t) for t in range(4))
+    return cu, q, k, v, do
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_sequences_are_independent_problems(causal):
+    lengths = [5, 1, 0, 13, 8]
+    H, d, scale = 2, 4, 0.6
+    cu, q, k, v, do = _packed(lengths, H, d, 80)
+    o, lse = oracle.attention_forward_varlen(q, k, v, cu, scale, causal)
+    dq, dk, dv = oracle.attention_backward_varlen(q, k, v, do, cu, scale, causal)
+    for b, n in enumerate(lengths):
+        if n == 0:
+            continue
+        sl = slice(cu[b], cu[b] + n)
+        one = lambda x: np.transpose(x[sl], (1, 0, 2))[None]  # [1, H, n, d]
+        o1, l1 = oracle.attention_forward(one(q), one(k), one(v), scale, causal)
+        g1 = oracle.attention_backward(one(q), one(k), one(v), one(do), scale, causal)
+        np.testing.assert_allclose(np.transpose(o[sl], (1, 0, 2)), o1[0], atol=1e-13)
+        np.testing.assert_allclose(lse[:, sl], l1[0], atol=1e-13)
+        for got, want in zip((dq, dk, dv), g1[:3]):
+            np.testing.assert_allclose(np.transpose(got[sl], (1, 0, 2)), want[0], atol=1e-12)
+
+
+def test_varlen_equal_lengths_is_the_batched_problem_with_dropout():
+    B, H, N, d, scale = 3, 2, 24, 4, 0.5
+    cu, q, k, v, do = _packed([N] * B, H, d, 90)
+    dense = lambda x: np.transpose(x.reshape(B, N, H, d), (0, 2, 1, 3))
+    drop = (0.3, 17, 2)
+    o, lse = oracle.attention_forward_varlen(q, k, v, cu, scale, True, dropout=drop)
+    od, ld = oracle.attention_forward_dropout(dense(q), dense(k), dense(v), scale, *drop,
+                                              causal=True)
+    np.testing.assert_allclose(dense(o), od, atol=1e-13)
+    np.testing.assert_allclose(lse.reshape(H, B, N).transpose(1, 0, 2), ld, atol=1e-13)
+    g = oracle.attention_backward_varlen(q, k, v, do, cu, scale, True, dropout=drop)
+    gd = oracle.attention_backward_dropout(dense(q), dense(k), dense(v), dense(do), scale, *drop,
+                                           causal=True)
+    for got, want in zip(g, gd[:3]):
+        np.testing.assert_allclose(dense(got), want, atol=1e-12)
