@@ -23,6 +23,7 @@ from __future__ import annotations
 import argparse
 import datetime
 import hashlib
+import itertools
 import json
 import os
 import statistics
@@ -63,10 +64,25 @@ def flops_fwd(x):
     return 4.0 * B * H * N * N * d * density(x)
 
 
-def ideal_bytes(x):
-    """Each input read once and each output written once (bytes)."""
+def packed_lengths(x):
+    """--varlen: the workload's sequences without padding (key lengths, else N)."""
     B, H, N, d = x.q.shape
-    E, R = B * H * N * d, B * H * N
+    return [int(l) for l in x.kv_len] if x.kv_len is not None else [N] * B
+
+
+def flops_fwd_packed(x):
+    """Forward FLOPs of the packed batch: each sequence its own L x L problem."""
+    B, H, N, d = x.q.shape
+    f = 0.5 if x.causal else 1.0
+    return sum(4.0 * H * L * L * d * f for L in packed_lengths(x))
+
+
+def ideal_bytes(x, rows=None):
+    """Each input read once and each output written once (bytes); ``rows`` = the rows of
+    every head together (default B*H*N; a packed batch has T*H)."""
+    B, H, N, d = x.q.shape
+    R = B * H * N if rows is None else rows
+    E = R * d
     fwd = 3 * 2 * E + 2 * E + 4 * R                    # Q, K, V in; O, LSE out
     bwd_main = 4 * 2 * E + 2 * 4 * R + 2 * 2 * E + 2 * 4 * E   # Q K V dO, lse2 D in; dK dV out; dQ acc
     return fwd, bwd_main
@@ -224,7 +240,21 @@ def run_ours(args):
     w = inputs.WORKLOADS[args.workload]
     x = workload_or_shape(args)
     B, H, N, d = x.q.shape
+    if args.varlen and (x.block_mask is not None or args.deterministic or args.dropout > 0):
+        raise SystemExit("--varlen runs the plain packed kernels (no block mask, dropout or "
+                         "deterministic dQ)")
     q, k, v, do = (t.to(dev) for t in (x.q, x.k, x.v, x.dout))
+    if args.varlen:
+        # the same tensors, each sequence's own rows packed token by token ([T, H, d])
+        lens = packed_lengths(x)
+        def pack(t):
+            return torch.cat([t[b, :, :lens[b]].transpose(0, 1) for b in range(B)]).contiguous()
+
+        pq, pkk, pv, pdo = (pack(t) for t in (q, k, v, do))
+        T = pq.shape[0]
+        cu = torch.tensor([0] + list(itertools.accumulate(lens)), dtype=torch.int32, device=dev)
+        po, pdq, pdk, pdv = (torch.empty_like(pq) for _ in range(4))
+        plse = torch.empty((H, T), dtype=torch.float32, device=dev)
     bm = None if x.block_mask is None else x.block_mask.to(dev)
     kl = None if x.kv_len is None else x.kv_len.to(dev)
     o = torch.empty_like(q)
@@ -245,12 +275,18 @@ def run_ours(args):
     seed, offset = 0x5EED, 0
 
     def fwd_call():
+        if args.varlen:
+            return binding.fa_fwd_varlen(pq, pkk, pv, po, plse, cu, B, H, N, T, d, scale, causal,
+                                         0.0, 0, 0, S)
         if drop > 0:
             return binding.fa_fwd_dropout(q, k, v, o, lse, B, H, N, d, scale, causal, bm, kl, drop,
                                           seed, offset, S)
         return binding.fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, bm, kl, S)
 
     def bwd_call():
+        if args.varlen:
+            return binding.fa_bwd_varlen(pq, pkk, pv, po, plse, pdo, pdq, pdk, pdv, cu, B, H, N, T,
+                                         d, scale, causal, 0.0, 0, 0, ws, ws_bytes, S)
         if drop > 0:
             return binding.fa_bwd_dropout(q, k, v, o, lse, do, dq, dk, dv, B, H, N, d, scale,
                                           causal, bm, kl, drop, seed, offset, ws, ws_bytes, S)
@@ -264,11 +300,11 @@ def run_ours(args):
         check(fwd_call(), "forward")
         if ev is not None:
             ev[1].record(stream)
-        if drop > 0:
+        if drop > 0 or args.varlen:
             # one call, three kernels: timed together as the "main" interval
             if ev is not None:
                 ev[2].record(stream)
-            check(bwd_call(), "fa_bwd_dropout")
+            check(bwd_call(), "backward")
             if ev is not None:
                 ev[3].record(stream)
                 ev[4].record(stream)
@@ -332,7 +368,7 @@ def run_ours(args):
 
     # ---------------------------------------------------------------- e2e
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not args.varlen:
         hq, hk, hv, hdo = (t.pin_memory() for t in (x.q, x.k, x.v, x.dout))
         ho, hdq, hdk, hdv = (torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
                              for _ in range(4))
@@ -367,7 +403,7 @@ def run_ours(args):
 
     # ---------------------------------------------------------------- report
     peaks, peak_kind = load_peaks()
-    ff = flops_fwd(x)
+    ff = flops_fwd_packed(x) if args.varlen else flops_fwd(x)
     fb = 2.5 * ff
     value = whole_job_tflops(3.5 * ff, world, step_t)
     fwd_tflops = ff / (fwd_t * 1e-3) / 1e12
@@ -375,16 +411,20 @@ def run_ours(args):
     bwd_tflops = fb / ((pre_t + main_t + post_t) * 1e-3) / 1e12
     per_gpu = value / world
     # dominant kernel by time: the backward main kernel or the forward kernel
+    ib = ideal_bytes(x, T * H if args.varlen else None)
     if main_t >= fwd_t:
-        dom, dom_t, dom_flops, dom_bytes = "fa_bwd_kernel", main_t, fb, ideal_bytes(x)[1]
+        dom, dom_t, dom_flops, dom_bytes = "fa_bwd_kernel", main_t, fb, ib[1]
     else:
-        dom, dom_t, dom_flops, dom_bytes = "fa_fwd_kernel", fwd_t, ff, ideal_bytes(x)[0]
+        dom, dom_t, dom_flops, dom_bytes = "fa_fwd_kernel", fwd_t, ff, ib[0]
+    # DRAM bytes were captured for the plain kernels on the [B][H][N][d] layout only
+    plain = not args.varlen and drop == 0
     achieved = dom_flops / (dom_t * 1e-3) / 1e12
     roofline = {"kernel": dom, "bound": "tensor", "achieved": achieved,
                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": achieved / peaks["bf16_tflops"],
                 "peak_source": f"{peak_kind} bf16_tflops (burst)",
-                "traffic": ncu_traffic(dom, args.workload + (f"@{args.shape}" if args.shape else "")),
+                "traffic": (ncu_traffic(dom, args.workload + (f"@{args.shape}" if args.shape else ""))
+                            if plain else None),
                 "algorithmic_bytes": dom_bytes,
                 "algorithmic_flops": dom_flops,
                 "ms_per_launch": dom_t}
@@ -400,9 +440,14 @@ def run_ours(args):
                    "l2": "flushed between timed steps (256 MiB write)",
                    "parallelism": f"replica x{world}",
                    "backward": ("fa_bwd_dropout (its three kernels timed together as bwd_main)"
-                                if drop > 0 else "fa_bwd_deterministic" if args.deterministic
+                                if drop > 0 else
+                                "fa_bwd_varlen (its three kernels timed together as bwd_main)"
+                                if args.varlen else "fa_bwd_deterministic" if args.deterministic
                                 else "fa_bwd"),
-                   "dropout": drop},
+                   "dropout": drop,
+                   "packed": ({"total_tokens": int(T), "max_seqlen": N,
+                               "flops": "4*H*d*sum(L_b^2) per forward, x1/2 causal"}
+                              if args.varlen else None)},
         "fwd_tflops": fwd_tflops,
         "bwd_tflops": bwd_tflops,
         "fwd_bwd_pct_of_peak": per_gpu / peaks["bf16_tflops"],
@@ -416,7 +461,7 @@ def run_ours(args):
         "gpu_launches": 4 * args.steps,
         "clocks": clocks,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and drop == 0:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and drop == 0 and not args.varlen:
         line["cpu_baseline"] = cpu_baseline(x, budget_s=args.cpu_budget)
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -676,6 +721,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--deterministic", action="store_true",
                     help="time fa_bwd_deterministic (ordered dQ kernel) instead of fa_bwd")
+    ap.add_argument("--varlen", action="store_true",
+                    help="time fa_fwd_varlen / fa_bwd_varlen on the workload's sequences packed "
+                         "without padding")
     ap.add_argument("--dropout", type=float, default=0.0,
                     help="time fa_fwd_dropout / fa_bwd_dropout with this probability")
     ap.add_argument("--vs-standard", action="store_true",
