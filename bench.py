@@ -294,10 +294,17 @@ def run_ours(args):
         return bwd(q, k, v, o, lse, do, dq, dk, dv, B, H, N, d, scale, causal, bm, kl, ws,
                    ws_bytes, S)
 
-    def step(ev=None):
+    def step(ev=None, inner=True):
+        """One forward + backward.  ev[0] / ev[4] bracket the step; with ``inner`` the
+        phases are bracketed as well (ev[1..3]), which serialises the kernels' launches."""
         if ev is not None:
             ev[0].record(stream)
         check(fwd_call(), "forward")
+        if not inner:
+            check(bwd_call(), "backward")
+            if ev is not None:
+                ev[4].record(stream)
+            return
         if ev is not None:
             ev[1].record(stream)
         if drop > 0 or args.varlen:
@@ -342,13 +349,22 @@ def run_ours(args):
         torch.cuda.synchronize()
 
     n_ev = 5
+    # timed steps: the whole step between two events (the library's kernels follow one
+    # another with programmatic dependent launch); then as many steps with every phase
+    # bracketed by events, for the per-kernel times and the roofline
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    evp = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
     t0 = time.time()
     for kk in range(args.steps):
         flush.zero_()                      # L2 flushed between timed steps
-        step(evs[kk])
+        step(evs[kk], inner=False)
+    torch.cuda.synchronize()
+    barrier()
+    for kk in range(args.steps):
+        flush.zero_()
+        step(evp[kk])
     torch.cuda.synchronize()
     barrier()
     t1 = time.time()
@@ -358,10 +374,10 @@ def run_ours(args):
         raise RuntimeError("device status after timing: " + binding.fa_status_string(st))
 
     step_ms = [e[0].elapsed_time(e[4]) for e in evs]
-    fwd_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    pre_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    main_ms = [e[2].elapsed_time(e[3]) for e in evs]
-    post_ms = [e[3].elapsed_time(e[4]) for e in evs]
+    fwd_ms = [e[0].elapsed_time(e[1]) for e in evp]
+    pre_ms = [e[1].elapsed_time(e[2]) for e in evp]
+    main_ms = [e[2].elapsed_time(e[3]) for e in evp]
+    post_ms = [e[3].elapsed_time(e[4]) for e in evp]
     mean = lambda a: sum(a) / len(a)
     step_t, fwd_t, pre_t, main_t, post_t = max_over_ranks(
         [mean(step_ms), mean(fwd_ms), mean(pre_ms), mean(main_ms), mean(post_ms)], dist, dev)
@@ -438,6 +454,8 @@ def run_ours(args):
                    "key_padding": x.kv_len is not None, "block_sparse": x.block_mask is not None,
                    "flop_density": density(x), "seed": w.seed,
                    "l2": "flushed between timed steps (256 MiB write)",
+                   "timing": ("value: K whole steps, CUDA events around each step; ms and "
+                              "roofline: K further steps with an event between kernels"),
                    "parallelism": f"replica x{world}",
                    "backward": ("fa_bwd_dropout (its three kernels timed together as bwd_main)"
                                 if drop > 0 else

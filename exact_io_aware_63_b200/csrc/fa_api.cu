@@ -139,6 +139,26 @@ bool make_tmap_any(CUtensorMap* m, const void* base, int B, int H, int N, int d,
   return pk.cu ? make_tmap_packed(m, base, H, pk.T, d) : make_tmap(m, base, B * H, N, d);
 }
 
+// Launches a kernel with programmatic stream serialization: it may be
+// scheduled while the previous kernel in the stream is finishing, and waits
+// (griddepcontrol.wait, in the kernel) before it touches global memory.  This
+// hides the launch gap between the library's back-to-back kernels.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 // Shape checks shared by every entry point.  Returns FA_OK, an error, or 1
@@ -267,9 +287,9 @@ int launch_fwd_mode(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensor
   const int per_head = kPair ? (p.n_t + 1) / 2 : p.n_t;
   p.num_units = p.B * p.H * per_head;
   const int grid = p.num_units < num_sms ? p.num_units : num_sms;
-  fa::fa_fwd_kernel<D, kPair, kDrop, kPacked>
-      <<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(tq, tk, tv, p);
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  const cudaError_t e = launch_pdl(fa::fa_fwd_kernel<D, kPair, kDrop, kPacked>, dim3(grid),
+                                   dim3(Cfg::kThreads), Cfg::kSmemBytes, stream, tq, tk, tv, p);
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 // Pair mode (two query tiles share each K/V tile) unless a block mask is
@@ -355,15 +375,17 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
     long long blocks = (work + threads - 1) / threads;
     const long long cap = static_cast<long long>(num_sms) * 8;
     if (blocks > cap) blocks = cap;
+    cudaError_t e;
     if (pk.cu)
-      fa::fa_bwd_pre_packed_kernel<D><<<static_cast<int>(blocks), threads, 0, stream>>>(
-          o, dout, lse, delta, lse2, reinterpret_cast<float4*>(dq_acc), counter, pk.cu, H, N, Np,
-          pk.T, rows_p, rows);
+      e = launch_pdl(fa::fa_bwd_pre_packed_kernel<D>, dim3(static_cast<int>(blocks)),
+                     dim3(threads), 0, stream, o, dout, lse, delta, lse2,
+                     reinterpret_cast<float4*>(dq_acc), counter, pk.cu, H, N, Np, pk.T, rows_p,
+                     rows);
     else
-      fa::fa_bwd_pre_kernel<D><<<static_cast<int>(blocks), threads, 0, stream>>>(
-          o, dout, lse, delta, lse2, reinterpret_cast<float4*>(dq_acc), counter, N, Np, rows_p,
-          rows);
-    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+      e = launch_pdl(fa::fa_bwd_pre_kernel<D>, dim3(static_cast<int>(blocks)), dim3(threads), 0,
+                     stream, o, dout, lse, delta, lse2, reinterpret_cast<float4*>(dq_acc), counter,
+                     N, Np, rows_p, rows);
+    if (e != cudaSuccess) return FA_ERR_CUDA;
   }
   // main
   if (phases & 2u) {
@@ -391,19 +413,12 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
     p.scale_log2 = scale * fa::kLog2e;
     set_drop(p, dr);
     const int grid = p.num_units < num_sms ? p.num_units : num_sms;
-    if (pk.cu && dr.on)
-      fa::fa_bwd_kernel<D, true, true>
-          <<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdq, tdk, tdv, p);
-    else if (pk.cu)
-      fa::fa_bwd_kernel<D, false, true>
-          <<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdq, tdk, tdv, p);
-    else if (dr.on)
-      fa::fa_bwd_kernel<D, true, false>
-          <<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdq, tdk, tdv, p);
-    else
-      fa::fa_bwd_kernel<D, false, false>
-          <<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdq, tdk, tdv, p);
-    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    auto kernel = pk.cu ? (dr.on ? fa::fa_bwd_kernel<D, true, true> : fa::fa_bwd_kernel<D, false, true>)
+                        : (dr.on ? fa::fa_bwd_kernel<D, true, false>
+                                 : fa::fa_bwd_kernel<D, false, false>);
+    if (launch_pdl(kernel, dim3(grid), dim3(Cfg::kThreads), Cfg::kSmemBytes, stream, tq, tk, tv,
+                   tdo, tdq, tdk, tdv, p) != cudaSuccess)
+      return FA_ERR_CUDA;
   }
   // dQ
   if (phases & 4u) {
@@ -412,9 +427,10 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
     long long blocks = (n8 + threads - 1) / threads;
     const long long cap = static_cast<long long>(num_sms) * 8;
     if (blocks > cap) blocks = cap;
-    fa::fa_bwd_dq_kernel<<<static_cast<int>(blocks), threads, 0, stream>>>(
-        reinterpret_cast<const float4*>(dq_acc), reinterpret_cast<uint4*>(dq), scale, n8);
-    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    if (launch_pdl(fa::fa_bwd_dq_kernel, dim3(static_cast<int>(blocks)), dim3(threads), 0, stream,
+                   reinterpret_cast<const float4*>(dq_acc), reinterpret_cast<uint4*>(dq), scale,
+                   n8) != cudaSuccess)
+      return FA_ERR_CUDA;
   }
   // dQ without atomics: one CTA walks each query tile's key tiles in order
   if (phases & 8u) {
@@ -447,9 +463,9 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
     dp.dq = dq;
     dp.scale = scale;
     const int grid = sp.num_units < num_sms ? sp.num_units : num_sms;
-    fa::fa_bwd_dq_det_kernel<D><<<grid, DCfg::kThreads, DCfg::kSmemBytes, stream>>>(tq, tk, tv,
-                                                                                    tdo, dp);
-    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    if (launch_pdl(fa::fa_bwd_dq_det_kernel<D>, dim3(grid), dim3(DCfg::kThreads),
+                   DCfg::kSmemBytes, stream, tq, tk, tv, tdo, dp) != cudaSuccess)
+      return FA_ERR_CUDA;
   }
   return FA_OK;
 }

@@ -61,6 +61,8 @@ __global__ void __launch_bounds__(256, 8) fa_bwd_pre_kernel(const uint16_t* __re
                                                          int* __restrict__ work_counter,
                                                          int N, int Np, long long rows_p,
                                                          long long rows) {
+  pdl_launch_dependents();
+  pdl_wait();
   // the main kernel's CTAs take work units from this counter
   if (blockIdx.x == 0 && threadIdx.x == 0) *work_counter = 0;
   constexpr int kLanesPerRow = D / 8;  // one 16-byte chunk (8 bf16) per lane
@@ -124,6 +126,8 @@ __global__ void __launch_bounds__(256, 8) fa_bwd_pre_packed_kernel(
     float4* __restrict__ dq_acc, int* __restrict__ work_counter,
     const int32_t* __restrict__ cu_seqlens, int H, int N, int Np, int T, long long rows_p,
     long long acc_rows) {
+  pdl_launch_dependents();
+  pdl_wait();
   if (blockIdx.x == 0 && threadIdx.x == 0) *work_counter = 0;
   constexpr int kLanesPerRow = D / 8;
   constexpr int kRowsPerWarp = 32 / kLanesPerRow;
@@ -179,6 +183,8 @@ __global__ void __launch_bounds__(256, 8) fa_bwd_pre_packed_kernel(
 __global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const float4* __restrict__ dq_acc,
                                                         uint4* __restrict__ dq, float scale,
                                                         long long n8) {
+  pdl_launch_dependents();
+  pdl_wait();
   for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n8;
        e += (long long)gridDim.x * blockDim.x) {
     const float4 a = __ldg(dq_acc + 2 * e);
@@ -374,6 +380,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
   using Cfg = BwdCfg<D>;
   constexpr int QS = Cfg::kQStages, DOS = Cfg::kDoStages, KVS = Cfg::kKvStages;
   extern __shared__ __align__(1024) uint8_t smem[];
+  pdl_launch_dependents();
   if (!smem_aligned_1024(smem)) return;
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + Cfg::kOffBar;
@@ -505,6 +512,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // the set-up above touches shared and tensor memory only; global memory
+  // waits for the previous kernel in the stream
+  pdl_wait();
   const uint32_t tmem = *tmem_base_slot;
   static_assert(Cfg::kRegsLow * 128 + Cfg::kRegsDs * 256 + Cfg::kRegsDq * 128 <=
                     Cfg::kRegsLaunch * Cfg::kThreads,

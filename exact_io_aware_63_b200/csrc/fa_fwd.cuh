@@ -284,6 +284,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
   constexpr int S = Cfg::kStages;
   constexpr int QSLOTS = Cfg::kQSlots;
   extern __shared__ __align__(1024) uint8_t smem[];
+  pdl_launch_dependents();
   if (!smem_aligned_1024(smem)) return;
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + Cfg::kOffBar;
@@ -352,6 +353,9 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // the set-up above touches shared and tensor memory only; global memory
+  // waits for the previous kernel in the stream
+  pdl_wait();
   const uint32_t tmem = *tmem_base_slot;
   const int G = gridDim.x;
   static_assert(Cfg::kRegsLow * 128 + Cfg::kRegsHigh * 256 <= Cfg::kRegsLaunch * Cfg::kThreads,

@@ -45,6 +45,17 @@ __device__ __forceinline__ bool smem_aligned_1024(const void* p) {
   return false;
 }
 
+// Programmatic dependent launch.  The library launches its kernels with
+// programmatic stream serialization: a kernel lets the next one in the stream
+// be scheduled as soon as all its CTAs are running (launch_dependents), and
+// waits before touching global memory until the previous kernel has finished
+// and its writes are visible (wait).  Launched without that attribute, both
+// are no-ops.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31u; }
 __device__ __forceinline__ uint32_t warp_id() { return threadIdx.x >> 5; }
 
