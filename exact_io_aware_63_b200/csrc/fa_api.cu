@@ -276,7 +276,7 @@ void set_drop(P& p, const DropArgs& dr) {
 
 template <int D, bool kPair, bool kDrop, bool kPacked = false>
 int launch_fwd_mode(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                    fa::FwdParams& p, cudaStream_t stream, int num_sms) {
+                    const CUtensorMap& to, fa::FwdParams& p, cudaStream_t stream, int num_sms) {
   using Cfg = fa::FwdCfg<D, kPair>;
   static bool smem_set = false;
   if (!smem_set) {
@@ -288,7 +288,8 @@ int launch_fwd_mode(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensor
   p.num_units = p.B * p.H * per_head;
   const int grid = p.num_units < num_sms ? p.num_units : num_sms;
   const cudaError_t e = launch_pdl(fa::fa_fwd_kernel<D, kPair, kDrop, kPacked>, dim3(grid),
-                                   dim3(Cfg::kThreads), Cfg::kSmemBytes, stream, tq, tk, tv, p);
+                                   dim3(Cfg::kThreads), Cfg::kSmemBytes, stream, tq, tk, tv, to,
+                                   p);
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -300,9 +301,9 @@ int launch_fwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o,
                int H, int N, float scale, int causal, const uint8_t* block_mask,
                const int32_t* kv_len, uint8_t* visited, cudaStream_t stream, int num_sms,
                const DropArgs& dr, const Packed& pk) {
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (!make_tmap_any(&tq, q, B, H, N, D, pk) || !make_tmap_any(&tk, k, B, H, N, D, pk) ||
-      !make_tmap_any(&tv, v, B, H, N, D, pk))
+      !make_tmap_any(&tv, v, B, H, N, D, pk) || !make_tmap_any(&to, o, B, H, N, D, pk))
     return FA_ERR_CUDA;
   fa::FwdParams p;
   p.o = o;
@@ -322,15 +323,15 @@ int launch_fwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o,
   p.scale_log2 = scale * fa::kLog2e;
   set_drop(p, dr);
   if (pk.cu) {  // packed batches have no block mask: pair mode
-    if (dr.on) return launch_fwd_mode<D, true, true, true>(tq, tk, tv, p, stream, num_sms);
-    return launch_fwd_mode<D, true, false, true>(tq, tk, tv, p, stream, num_sms);
+    if (dr.on) return launch_fwd_mode<D, true, true, true>(tq, tk, tv, to, p, stream, num_sms);
+    return launch_fwd_mode<D, true, false, true>(tq, tk, tv, to, p, stream, num_sms);
   }
   if (dr.on) {
-    if (block_mask) return launch_fwd_mode<D, false, true>(tq, tk, tv, p, stream, num_sms);
-    return launch_fwd_mode<D, true, true>(tq, tk, tv, p, stream, num_sms);
+    if (block_mask) return launch_fwd_mode<D, false, true>(tq, tk, tv, to, p, stream, num_sms);
+    return launch_fwd_mode<D, true, true>(tq, tk, tv, to, p, stream, num_sms);
   }
-  if (block_mask) return launch_fwd_mode<D, false, false>(tq, tk, tv, p, stream, num_sms);
-  return launch_fwd_mode<D, true, false>(tq, tk, tv, p, stream, num_sms);
+  if (block_mask) return launch_fwd_mode<D, false, false>(tq, tk, tv, to, p, stream, num_sms);
+  return launch_fwd_mode<D, true, false>(tq, tk, tv, to, p, stream, num_sms);
 }
 
 template <int D>

@@ -169,6 +169,11 @@ struct FwdCfg {
   __device__ static constexpr uint32_t col_s(int x) { return x ? 128u : 0u; }
   __device__ static constexpr uint32_t col_o(int x) { return x ? 256u + D : 256u; }
   __device__ static constexpr uint32_t col_p(int x) { return kSepP ? 384u + 64u * x : col_s(x); }
+  // Pair mode at D = 64: a warpgroup stages its O tile (bf16, 128-byte
+  // swizzled rows) in its own query tile's shared memory, which the unit's
+  // S MMAs have finished reading, and one thread writes it with a TMA store;
+  // the Q slot is released (q_empty) only after the store has read it.
+  static constexpr bool kEpiTma = kSepP && kPair;
 };
 
 // Work-unit order: heads are taken in groups whose K and V fit in a share of
@@ -279,7 +284,8 @@ __device__ __forceinline__ int fwd_next(const FwdParams& p, const FwdUnit& w, in
 template <int D, bool kPair, bool kDrop = false, bool kPacked = false>
 __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                  const FwdParams p) {
   using Cfg = FwdCfg<D, kPair>;
   constexpr int S = Cfg::kStages;
   constexpr int QSLOTS = Cfg::kQSlots;
@@ -322,7 +328,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
     for (int x = 0; x < 2; ++x) {
       mbar_init(q_full(x), 1);
       // separate-P layout: both warpgroups' issuers arrive
-      mbar_init(q_empty(x), Cfg::kSepP ? 2 : 1);
+      mbar_init(q_empty(x), (Cfg::kSepP ? 2 : 1) + (Cfg::kEpiTma ? 2 : 0));
       mbar_init(s_full(x), 1);
       mbar_init(p_full(x), 128);
       mbar_init(o_full(x), 1);
@@ -345,6 +351,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
+    if (Cfg::kEpiTma) prefetch_tmap(&tm_o);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_base_slot), Cfg::kTmemCols);
@@ -796,6 +803,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
     const uint32_t tO = t_lane + Cfg::col_o(x);
     const uint32_t tP = t_lane + Cfg::col_p(x);
     uint32_t s_cnt = 0, unit_cnt = 0;
+    uint32_t q_use = 0;  // units seen: ring index of their Q slot
     uint32_t o_cnt[2] = {0, 0};
     bool ok = true;
     for (int round = live_round<kPair, kPacked>(p, 0, blockIdx.x, G); ok;
@@ -803,7 +811,20 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
       const int u = unit_for_round(round, blockIdx.x, G);
       if (u >= p.num_units) break;
       const FwdUnit w = fwd_decode<kPair, kPacked>(p, u);
-      if (kPair && x == 1 && !w.has1) continue;  // pair with no second tile
+      const int qs_me = q_use % QSLOTS;
+      const uint32_t q_par = (q_use / QSLOTS) & 1;
+      ++q_use;
+      if (kPair && x == 1 && !w.has1) {
+        // pair with no second tile: nothing to compute or write.  The staged
+        // epilogue releases this warpgroup's share of the Q slot, once this
+        // unit's Q has landed (so that the arrival counts for this use).
+        if constexpr (Cfg::kEpiTma) {
+          ok = __all_sync(0xffffffffu, mbar_wait(q_full(qs_me), q_par));
+          if (!ok) break;
+          if (r_local == 0) mbar_arrive(q_empty(qs_me));
+        }
+        continue;
+      }
       const int i_me = x ? w.i1 : w.i0;           // this warpgroup's query tile
       const int j_end_me = x ? w.j_end1 : w.j_end0;
       const int row = i_me * kTile + r_local;     // query index within the head
@@ -968,36 +989,70 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
       if constexpr (kPair) {
         // ---------------------------------------------------- epilogue (own tile)
         uint4* orow = reinterpret_cast<uint4*>(o_row);
+        // Staged: the tile goes through shared memory to one TMA store (the
+        // tensor map clips rows beyond N).  A packed tile that crosses its
+        // sequence's end is written row by row instead (the rows past the end
+        // belong to the next sequence).
+        const bool staged = Cfg::kEpiTma && (!kPacked || (i_me + 1) * kTile <= w.nq);
         if (cnt > 0) {
           ok = __all_sync(0xffffffffu, mbar_wait(o_full(x), o_cnt[x] & 1));
           ++o_cnt[x];
           if (!ok) break;
           tc_fence_after();
-          const float inv_l = (l > 0.f) ? (kDrop ? p.drop.w : 1.f) / l : 0.f;
+        } else if (Cfg::kEpiTma) {
+          // no key tile: the zeros below may be staged over the Q tile only
+          // after its load has landed
+          ok = __all_sync(0xffffffffu, mbar_wait(q_full(qs_me), q_par));
+          if (!ok) break;
+        }
+        const float inv_l = (cnt > 0 && l > 0.f) ? (kDrop ? p.drop.w : 1.f) / l : 0.f;
+        uint8_t* const stage_row = smem + Cfg::kOffQ +
+                                   (qs_me * Cfg::kQPerSlot + x) * Cfg::kTileBytes + r_local * 128;
 #pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t pk[16];
+          if (cnt > 0) {
             uint32_t r[32];
             tmem_ld32(tO + c * 32, r);
             tmem_wait_ld();
             reg_fence32(r);
-            uint32_t pk[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e)
               pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv_l,
                                   __uint_as_float(r[2 * e + 1]) * inv_l);
+          } else {
 #pragma unroll
-            for (int v4 = 0; v4 < 4; ++v4)
-              if (row_ok)
-                orow[c * 4 + v4] =
-                    make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+            for (int e = 0; e < 16; ++e) pk[e] = 0u;
           }
-          tc_fence_before();
-          if (row_ok) *lse_ptr = (l > 0.f) ? (m_used + log2f(l)) * kLn2 : -INFINITY;
-        } else {
 #pragma unroll
-          for (int c = 0; c < D / 8; ++c)
-            if (row_ok) orow[c] = make_uint4(0, 0, 0, 0);
-          if (row_ok) *lse_ptr = -INFINITY;
+          for (int v4 = 0; v4 < 4; ++v4) {
+            const uint4 val = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+            if (staged) {
+              const int g = c * 4 + v4;  // 16-byte granule of the 128-byte row
+              *reinterpret_cast<uint4*>(stage_row + ((g ^ (r_local & 7)) << 4)) = val;
+            } else if (row_ok) {
+              orow[c * 4 + v4] = val;
+            }
+          }
+        }
+        if (cnt > 0) tc_fence_before();
+        if (row_ok)
+          *lse_ptr = (cnt > 0 && l > 0.f) ? (m_used + log2f(l)) * kLn2 : -INFINITY;
+        if constexpr (Cfg::kEpiTma) {
+          if (staged) {
+            fence_proxy_async_smem();
+            named_bar_sync(8 + x, 128);  // the warpgroup's 128 rows are staged
+          }
+          if (r_local == 0) {
+            if (staged) {
+              const int2 yz = tile_yz(kPacked, (kPacked ? w.tok_base : 0) + i_me * kTile, w.tz);
+              tma_store_3d(&tm_o, 0, yz.x, yz.y,
+                           sbase + Cfg::kOffQ + (qs_me * Cfg::kQPerSlot + x) * Cfg::kTileBytes);
+              bulk_commit_group();
+              bulk_wait_group_read0();
+            }
+            mbar_arrive(q_empty(qs_me));  // the Q slot may be loaded again
+          }
         }
       } else {
         // ---------------------------------------------------- merge + epilogue
@@ -1066,6 +1121,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
       }
     }
     if (!ok) *abort_flag = 1;
+    if (Cfg::kEpiTma && r_local == 0) bulk_wait_group0();  // O stores complete before exit
   }
 
   tc_fence_before();
