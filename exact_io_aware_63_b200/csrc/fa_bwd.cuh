@@ -1094,7 +1094,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
                 pk[2 * e4 + 1] = pack_bf16x2(p2, p3);
               }
             };
-            if (!key_valid) {
+            // no allowed entry: a padding key, or (diagonal tile) a query chunk
+            // that lies wholly before the warp's 32 keys
+            if (!key_valid || (diag && quarter > 2 * h + c)) {
 #pragma unroll
               for (int e = 0; e < 16; ++e) {
                 pk[e] = 0u;

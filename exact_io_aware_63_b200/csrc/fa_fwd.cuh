@@ -861,11 +861,22 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
         const bool diag = p.causal && (j == i_me);
         const int kv_lim = w.L - j * kTile;  // keys c >= kv_lim are padding
         const bool boundary = diag || kv_lim < kTile;
+        // Keys c >= lim are masked.  A 32-key chunk that is masked for every
+        // row of the warp (padding past kv_len, or above the diagonal block of
+        // the warp's 32 rows) needs no exponentials: bit c of `skip` (the same
+        // in all lanes).
+        uint32_t skip = 0;
         if (boundary) {
           const int lim = diag ? min(r_local + 1, kv_lim) : kv_lim;
 #pragma unroll
-          for (int c = 0; c < kTile; ++c)
-            if (c >= lim) sv[c] = -INFINITY;
+          for (int c4 = 0; c4 < kTile / 32; ++c4) {
+            if (__all_sync(0xffffffffu, lim <= c4 * 32)) skip |= 1u << c4;
+            if (!__all_sync(0xffffffffu, lim >= c4 * 32 + 32)) {
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                if (c4 * 32 + e >= lim) sv[c4 * 32 + e] = -INFINITY;
+            }
+          }
         }
         // row max: eight independent chains of 3-input max, then combined
         float mx8[8];
@@ -901,6 +912,15 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             uint32_t pk[16];
+            if constexpr (!kSoft) {  // boundary tiles only: interior ones keep one straight line
+              if (skip & (1u << c)) {
+                // every key of the chunk is masked for the whole warp: P = 0
+#pragma unroll
+                for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                tmem_st16(tP + c * 16, pk);
+                continue;
+              }
+            }
             [[maybe_unused]] uint4 d4;
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
