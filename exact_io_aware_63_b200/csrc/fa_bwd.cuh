@@ -271,9 +271,9 @@ struct BwdCfg {
   static_assert(kOffEpi % 1024 == 0, "staging tiles must be 1024-byte aligned");
   // kv_full[KVS], kv_empty[KVS], q_full[QS], q_empty[QS], do_full[DS], do_empty[DS],
   // s_full, dp_full, p_full, ds_full, ds_smem_empty, dq_full, dq_empty, dkv_full,
-  // drain[3], s_free, p_free, unit_full[UR], unit_empty[UR], epi_ready[2]
+  // drain[3], s_free, p_free, unit_full[UR], unit_empty[UR]
   static constexpr int kNumBars =
-      2 * kKvStages + 2 * kQStages + 2 * kDoStages + 15 + 2 * kUnitRing;
+      2 * kKvStages + 2 * kQStages + 2 * kDoStages + 13 + 2 * kUnitRing;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16;
   static_assert(kSmemBytes <= 232448, "shared memory over the per-block limit");
@@ -401,9 +401,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
   constexpr int UR = Cfg::kUnitRing;
   auto unit_full = [&](int s) { return drain_bar + 40 + 8 * s; };
   auto unit_empty = [&](int s) { return drain_bar + 40 + 8 * (UR + s); };
-  // D = 64 epilogue: all 128 rows of warpgroup h's dK / dV tile are staged
-  auto epi_ready = [&](int h) { return drain_bar + 40 + 8 * (2 * UR + h); };
-  static_assert((2 * KVS + 2 * QS + 2 * DOS + 15 + 2 * UR) == Cfg::kNumBars, "barrier layout");
+
+  static_assert((2 * KVS + 2 * QS + 2 * DOS + 13 + 2 * UR) == Cfg::kNumBars, "barrier layout");
   int4* unit_rec = reinterpret_cast<int4*>(smem + Cfg::kOffUnit);  // [UR][3]
   // the warps that read each unit record: the MMA issuer(s), 8 dS and 4 dQ warps
   constexpr uint32_t kUnitReaders = (Cfg::kMultiIssue ? 3 : 1) + 12;
@@ -491,8 +490,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       mbar_init(unit_full(s), 1);
       mbar_init(unit_empty(s), kUnitReaders);
     }
-    mbar_init(epi_ready(0), 128);
-    mbar_init(epi_ready(1), 128);
+
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tmap(&tm_q);
@@ -947,7 +945,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     const uint32_t tP = t_lane + Cfg::kColP + h * Cfg::kPHalf;  // this half's P^T (bf16)
     const uint32_t tDP = t_lane + Cfg::kColDP + h * 64;  // this half's dP^T / dS^T columns
     uint8_t* ds_rowp = smem + Cfg::kOffDS + h * 16384 + kr * 128;
-    uint32_t s_cnt = 0, dp_cnt = 0, dsm_cnt = 0, dkv_cnt = 0, q_cnt = 0, epi_cnt = 0;
+    uint32_t s_cnt = 0, dp_cnt = 0, dsm_cnt = 0, dkv_cnt = 0, q_cnt = 0;
     bool ok = true;
     for (int round = 0; ok; ++round) {
       BwdUnit w;
@@ -1205,6 +1203,12 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       ++dkv_cnt;
       if (!ok) break;
       tc_fence_after();
+      if (epi_tma) {
+        // the previous unit's TMA store (issued by this warpgroup's first
+        // thread, not awaited then) has read the staging area
+        if (kr == 0) bulk_wait_group_read0();
+        named_bar_sync(1 + h, 128);
+      }
       const float mul = h ? (kDrop ? p.drop.w : 1.f) : p.scale;  // dV: dropout weight
       const uint32_t tAcc = t_lane + (h ? Cfg::kColDV : Cfg::kColDK);
       uint8_t* epi_row = smem + Cfg::kOffEpi + h * Cfg::kTileBytes + kr * 128;
@@ -1231,25 +1235,16 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       }
       tc_fence_before();
       if (epi_tma) {
-        // the whole tile is staged: one thread of the warpgroup stores it.
-        // The staging area is written again only in the next unit's epilogue,
-        // after dkv_full, which needs this thread's arrivals of that unit,
-        // made after the store below has read the tile.
+        // the whole tile is staged: one thread of the warpgroup stores it
+        // (the next epilogue waits for the store's read of the staging area)
         fence_proxy_async_smem();
-        mbar_arrive(epi_ready(h));
+        named_bar_sync(1 + h, 128);
         if (kr == 0) {
-          ok = mbar_wait(epi_ready(h), epi_cnt & 1);
-          if (ok) {
-            const int2 yz = tile_yz(kPacked, (kPacked ? w.tok_base : 0) + w.j * kTile, w.tz);
-            tma_store_3d(h ? &tm_dv : &tm_dk, 0, yz.x, yz.y,
-                         smem_u32(smem + Cfg::kOffEpi + h * Cfg::kTileBytes));
-            bulk_commit_group();
-            bulk_wait_group_read0();
-          }
+          const int2 yz = tile_yz(kPacked, (kPacked ? w.tok_base : 0) + w.j * kTile, w.tz);
+          tma_store_3d(h ? &tm_dv : &tm_dk, 0, yz.x, yz.y,
+                       smem_u32(smem + Cfg::kOffEpi + h * Cfg::kTileBytes));
+          bulk_commit_group();
         }
-        ++epi_cnt;
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
       }
     }
     if (!ok) *abort_flag = 1;
