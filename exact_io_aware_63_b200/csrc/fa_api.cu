@@ -342,7 +342,8 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
                int num_sms, unsigned phases, const DropArgs& dr, const Packed& pk) {
   using Cfg = fa::BwdCfg<D>;
   // rows of the dQ accumulator and of dQ (packed: tokens x heads)
-  const long long rows = pk.cu ? static_cast<long long>(pk.T) * H : static_cast<long long>(B) * H * N;
+  const long long rows =
+      pk.cu ? static_cast<long long>(pk.T) * H : static_cast<long long>(B) * H * N;
   const WsLayout wl = ws_layout(B, H, N, D);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* delta = reinterpret_cast<float*>(ws + wl.delta);
@@ -414,7 +415,8 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
     p.scale_log2 = scale * fa::kLog2e;
     set_drop(p, dr);
     const int grid = p.num_units < num_sms ? p.num_units : num_sms;
-    auto kernel = pk.cu ? (dr.on ? fa::fa_bwd_kernel<D, true, true> : fa::fa_bwd_kernel<D, false, true>)
+    auto kernel = pk.cu ? (dr.on ? fa::fa_bwd_kernel<D, true, true>
+                                 : fa::fa_bwd_kernel<D, false, true>)
                         : (dr.on ? fa::fa_bwd_kernel<D, true, false>
                                  : fa::fa_bwd_kernel<D, false, false>);
     if (launch_pdl(kernel, dim3(grid), dim3(Cfg::kThreads), Cfg::kSmemBytes, stream, tq, tk, tv,

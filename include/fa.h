@@ -42,6 +42,11 @@
  *  - The caller owns every buffer.  fa_fwd allocates nothing.  fa_bwd uses
  *    only the caller's workspace.  Nothing is freed by the library.
  *  - On any nonzero return, nothing was launched and no output was touched.
+ *  - Kernels are launched with programmatic stream serialization: each may
+ *    be scheduled while the previous kernel in the stream is finishing and
+ *    waits, before it touches global memory, until that kernel's writes are
+ *    visible.  Stream order is kept; a caller's own kernel that follows on
+ *    the stream starts early only if it was launched that way itself.
  */
 #ifndef FA_B200_H
 #define FA_B200_H
