@@ -41,3 +41,42 @@ def test_standard_attention_mask_without_masks_is_all_true():
     x = inputs.make_inputs(1, 1, 128, 64, seed=3)
     got = bench.standard_allowed(x, torch.device("cpu"))
     assert bool(got.all())
+
+
+def _count_allowed(x):
+    return int(_allowed_by_definition(x).sum()) * x.q.shape[1]
+
+
+def test_metric_flops_count_the_allowed_products():
+    # 4 d FLOPs per allowed (row, key) pair of every head: causal counts half the
+    # matrix (the metric's convention, which includes the diagonal's half), key
+    # padding counts its kept keys for every row, block masks their kept tiles
+    x = inputs.make_inputs(2, 3, 256, 64, seed=5, key_padding=(100, 256))
+    assert bench.flops_fwd(x) == 4.0 * 64 * _count_allowed(x)
+    x = inputs.make_inputs(1, 2, 256, 64, seed=6, block_keep=0.5)
+    assert bench.flops_fwd(x) == 4.0 * 64 * _count_allowed(x)
+    x = inputs.make_inputs(1, 1, 256, 64, causal=True, seed=7)
+    assert bench.flops_fwd(x) == 4.0 * 64 * 256 * 256 / 2
+
+
+def test_packed_batch_flops_are_each_sequence_alone():
+    x = inputs.make_inputs(3, 2, 512, 64, seed=8, key_padding=(200, 512))
+    lens = bench.packed_lengths(x)
+    assert lens == [int(v) for v in x.kv_len]
+    assert bench.flops_fwd_packed(x) == sum(4.0 * 2 * 64 * L * L for L in lens)
+    # no key padding: every sequence has N tokens, and the packed count is the dense one
+    y = inputs.make_inputs(2, 2, 256, 64, seed=9)
+    assert bench.packed_lengths(y) == [256, 256]
+    assert bench.flops_fwd_packed(y) == bench.flops_fwd(y)
+
+
+def test_ideal_bytes_follow_the_rows():
+    # forward: Q, K, V read and O written once (bf16, 2E each) plus LSE (4R); main
+    # backward kernel: Q, K, V, dO read (8E), -LSE2 and -D read (8R), dK and dV
+    # written (4E), the float32 dQ accumulator read and written once by its
+    # reduce-adds (8E)
+    x = inputs.make_inputs(2, 3, 256, 64, seed=10)
+    for R in (2 * 3 * 256, 100):
+        E = R * 64
+        got = bench.ideal_bytes(x) if R == 2 * 3 * 256 else bench.ideal_bytes(x, rows=R)
+        assert got == (8 * E + 4 * R, 20 * E + 8 * R)
