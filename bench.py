@@ -240,9 +240,8 @@ def run_ours(args):
     w = inputs.WORKLOADS[args.workload]
     x = workload_or_shape(args)
     B, H, N, d = x.q.shape
-    if args.varlen and (x.block_mask is not None or args.deterministic or args.dropout > 0):
-        raise SystemExit("--varlen runs the plain packed kernels (no block mask, dropout or "
-                         "deterministic dQ)")
+    if args.varlen and x.block_mask is not None:
+        raise SystemExit("--varlen: packed batches take no block mask")
     q, k, v, do = (t.to(dev) for t in (x.q, x.k, x.v, x.dout))
     if args.varlen:
         # the same tensors, each sequence's own rows packed token by token ([T, H, d])
@@ -748,6 +747,12 @@ def main():
                     help="instead of the benchmark line, compare one step with standard "
                          "attention (S and P materialised) on the same inputs")
     args = ap.parse_args()
+    modes = [m for m, on in (("--deterministic", args.deterministic), ("--varlen", args.varlen),
+                             ("--dropout", args.dropout > 0)) if on]
+    if len(modes) > 1:
+        ap.error(" and ".join(modes) + " select different backward paths: give one")
+    if not 0.0 <= args.dropout < 1.0:
+        ap.error("--dropout must lie in [0, 1)")
     if args.warmup < 3 and args.impl == "ours":
         print("note: warm-up raised to 3 steps", file=sys.stderr)
         args.warmup = 3
