@@ -8,12 +8,15 @@ import of a function raises.
 Raw entry points (same argument order as the C ABI; tensors are passed as
 torch tensors or None, the stream as a torch.cuda.Stream or None = current):
 ``fa_fwd``, ``fa_fwd_traced``, ``fa_bwd``, ``fa_bwd_traced``, ``fa_bwd_phase``,
-``fa_bwd_deterministic``, ``fa_bwd_noalloc``,
-``fa_bwd_workspace_size``, ``fa_get_device_status``, ``fa_status_string``,
+``fa_bwd_deterministic``, ``fa_fwd_dropout``, ``fa_bwd_dropout``, ``fa_fwd_varlen``,
+``fa_bwd_varlen``, ``fa_bwd_noalloc``, ``fa_bwd_workspace_size``,
+``fa_selftest_wait_timeout``, ``fa_get_device_status``, ``fa_status_string``,
 ``fa_version``.
 
 Convenience wrappers that allocate outputs: ``attention_forward`` and
-``attention_backward``.
+``attention_backward`` (options ``dropout=(p, seed, offset)`` and, for the backward,
+``deterministic=True``), ``attention_forward_varlen`` and ``attention_backward_varlen``
+for packed batches.
 """
 
 from __future__ import annotations
