@@ -238,3 +238,11 @@ def test_varlen_backward_workspace_checks():
     assert bwd_varlen(ws=None) == -5
     assert bwd_varlen(ws_bytes=64) == -5
     assert bwd_varlen(ws=P + 16) == -2
+
+
+def test_binding_has_every_declared_function():
+    # the Python binding carries the C ABI under the same names, each with a wrapper
+    declared = set(declared_functions())
+    assert set(binding._SIGS) == declared
+    for name in declared:
+        assert callable(getattr(binding, name)), name
