@@ -163,9 +163,13 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 // Shape checks shared by every entry point.  Returns FA_OK, an error, or 1
 // for "empty problem: nothing to do".
+// Head dimensions: 64 and 128 natively; 32 and 96 run on the 64 / 128 kernels,
+// whose tensor maps read the missing columns as zeros and whose stores stop at d.
+bool supported_d(int d) { return d == 32 || d == 64 || d == 96 || d == 128; }
+
 int check_shape(int B, int H, int N, int d) {
   if (B < 0 || H < 0 || N < 0) return FA_ERR_SHAPE;
-  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED_D;
+  if (!supported_d(d)) return FA_ERR_UNSUPPORTED_D;
   if (B == 0 || H == 0 || N == 0) return 1;
   const long long rows = static_cast<long long>(B) * H * N;
   if (rows >= (1LL << 31)) return FA_ERR_SHAPE;
@@ -176,7 +180,7 @@ int check_shape(int B, int H, int N, int d) {
 // sees B, H and max_seqlen): FA_OK, an error, or 1 for "nothing to do".
 int check_packed(const int32_t* cu, int B, int H, int max_seqlen, int T, int d) {
   if (B < 0 || H < 0 || max_seqlen < 0 || T < 0) return FA_ERR_SHAPE;
-  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED_D;
+  if (!supported_d(d)) return FA_ERR_UNSUPPORTED_D;
   if (B == 0 || H == 0 || max_seqlen == 0 || T == 0) return 1;
   // B sequences of at most max_seqlen tokens: the workspace and the unit grid
   // are sized for B * max_seqlen rows per head
@@ -298,12 +302,12 @@ int launch_fwd_mode(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensor
 // split mode keeps both softmax warpgroups busy on one query tile instead.
 template <int D>
 int launch_fwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o, float* lse, int B,
-               int H, int N, float scale, int causal, const uint8_t* block_mask,
+               int H, int N, int d, float scale, int causal, const uint8_t* block_mask,
                const int32_t* kv_len, uint8_t* visited, cudaStream_t stream, int num_sms,
                const DropArgs& dr, const Packed& pk) {
   CUtensorMap tq, tk, tv, to;
-  if (!make_tmap_any(&tq, q, B, H, N, D, pk) || !make_tmap_any(&tk, k, B, H, N, D, pk) ||
-      !make_tmap_any(&tv, v, B, H, N, D, pk) || !make_tmap_any(&to, o, B, H, N, D, pk))
+  if (!make_tmap_any(&tq, q, B, H, N, d, pk) || !make_tmap_any(&tk, k, B, H, N, d, pk) ||
+      !make_tmap_any(&tv, v, B, H, N, d, pk) || !make_tmap_any(&to, o, B, H, N, d, pk))
     return FA_ERR_CUDA;
   fa::FwdParams p;
   p.o = o;
@@ -313,12 +317,13 @@ int launch_fwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o,
   p.visited = visited;
   p.cu_seqlens = pk.cu;
   p.T = pk.T;
-  p.o_stride = pk.cu ? static_cast<long long>(H) * D : D;
+  p.o_stride = pk.cu ? static_cast<long long>(H) * d : d;
+  p.dcols = d;
   p.B = B;
   p.H = H;
   p.N = N;
   p.n_t = (N + fa::kTile - 1) / fa::kTile;
-  p.heads_per_group = heads_per_group(B * H, 4.0 * N * D);  // K and V
+  p.heads_per_group = heads_per_group(B * H, 4.0 * N * d);  // K and V
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * fa::kLog2e;
   set_drop(p, dr);
@@ -337,14 +342,14 @@ int launch_fwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o,
 template <int D>
 int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf16* o,
                const float* lse, const fa_bf16* dout, fa_bf16* dq, fa_bf16* dk, fa_bf16* dv, int B,
-               int H, int N, float scale, int causal, const uint8_t* block_mask,
+               int H, int N, int d, float scale, int causal, const uint8_t* block_mask,
                const int32_t* kv_len, void* workspace, uint8_t* visited, cudaStream_t stream,
                int num_sms, unsigned phases, const DropArgs& dr, const Packed& pk) {
   using Cfg = fa::BwdCfg<D>;
   // rows of the dQ accumulator and of dQ (packed: tokens x heads)
   const long long rows =
       pk.cu ? static_cast<long long>(pk.T) * H : static_cast<long long>(B) * H * N;
-  const WsLayout wl = ws_layout(B, H, N, D);
+  const WsLayout wl = ws_layout(B, H, N, d);  // the caller's workspace, sized for d
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* delta = reinterpret_cast<float*>(ws + wl.delta);
   float* lse2 = reinterpret_cast<float*>(ws + wl.lse2);
@@ -352,12 +357,12 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
   int* counter = reinterpret_cast<int*>(ws + wl.counter);
   CUtensorMap tq, tk, tv, tdo, tdq, tdk, tdv;
   const int BH = B * H;
-  const bool acc_ok = pk.cu ? make_tmap_f32_acc_packed(&tdq, dq_acc, H, pk.T, D)
-                            : make_tmap_f32_acc(&tdq, dq_acc, BH, N, D);
-  if (!make_tmap_any(&tq, q, B, H, N, D, pk) || !make_tmap_any(&tk, k, B, H, N, D, pk) ||
-      !make_tmap_any(&tv, v, B, H, N, D, pk) || !make_tmap_any(&tdo, dout, B, H, N, D, pk) ||
-      !acc_ok || !make_tmap_any(&tdk, dk, B, H, N, D, pk) ||
-      !make_tmap_any(&tdv, dv, B, H, N, D, pk))
+  const bool acc_ok = pk.cu ? make_tmap_f32_acc_packed(&tdq, dq_acc, H, pk.T, d)
+                            : make_tmap_f32_acc(&tdq, dq_acc, BH, N, d);
+  if (!make_tmap_any(&tq, q, B, H, N, d, pk) || !make_tmap_any(&tk, k, B, H, N, d, pk) ||
+      !make_tmap_any(&tv, v, B, H, N, d, pk) || !make_tmap_any(&tdo, dout, B, H, N, d, pk) ||
+      !acc_ok || !make_tmap_any(&tdk, dk, B, H, N, d, pk) ||
+      !make_tmap_any(&tdv, dv, B, H, N, d, pk))
     return FA_ERR_CUDA;
   static bool smem_set = false;
   if (!smem_set) {
@@ -373,7 +378,7 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
     const int threads = 256;
     const int Np = (N + fa::kTile - 1) / fa::kTile * fa::kTile;
     const long long rows_p = static_cast<long long>(B) * H * Np;
-    const long long work = (rows > rows_p ? rows : rows_p) * (D / 4);
+    const long long work = (rows > rows_p ? rows : rows_p) * (D / 4);  // lanes cover D columns
     long long blocks = (work + threads - 1) / threads;
     const long long cap = static_cast<long long>(num_sms) * 8;
     if (blocks > cap) blocks = cap;
@@ -382,11 +387,11 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
       e = launch_pdl(fa::fa_bwd_pre_packed_kernel<D>, dim3(static_cast<int>(blocks)),
                      dim3(threads), 0, stream, o, dout, lse, delta, lse2,
                      reinterpret_cast<float4*>(dq_acc), counter, pk.cu, H, N, Np, pk.T, rows_p,
-                     rows);
+                     rows, d);
     else
       e = launch_pdl(fa::fa_bwd_pre_kernel<D>, dim3(static_cast<int>(blocks)), dim3(threads), 0,
                      stream, o, dout, lse, delta, lse2, reinterpret_cast<float4*>(dq_acc), counter,
-                     N, Np, rows_p, rows);
+                     N, Np, rows_p, rows, d);
     if (e != cudaSuccess) return FA_ERR_CUDA;
   }
   // main
@@ -402,13 +407,14 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
     p.visited = visited;
     p.cu_seqlens = pk.cu;
     p.T = pk.T;
-    p.o_stride = pk.cu ? static_cast<long long>(H) * D : D;
+    p.o_stride = pk.cu ? static_cast<long long>(H) * d : d;
+    p.dcols = d;
     p.B = B;
     p.H = H;
     p.N = N;
     p.n_t = (N + fa::kTile - 1) / fa::kTile;
     p.num_units = B * H * p.n_t;
-    p.heads_per_group = heads_per_group(B * H, 8.0 * N * D);  // Q, dO, f32 dQ accumulator
+    p.heads_per_group = heads_per_group(B * H, 8.0 * N * d);  // Q, dO, f32 dQ accumulator
     p.work_counter = counter;
     p.causal = causal ? 1 : 0;
     p.scale = scale;
@@ -426,7 +432,7 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
   // dQ
   if (phases & 4u) {
     const int threads = 256;
-    const long long n8 = rows * D / 8;
+    const long long n8 = rows * d / 8;  // dQ is [rows][d]
     long long blocks = (n8 + threads - 1) / threads;
     const long long cap = static_cast<long long>(num_sms) * 8;
     if (blocks > cap) blocks = cap;
@@ -436,6 +442,7 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
       return FA_ERR_CUDA;
   }
   // dQ without atomics: one CTA walks each query tile's key tiles in order
+  // (head dimensions 64 and 128 only: bwd_impl checks it before any launch)
   if (phases & 8u) {
     using DCfg = fa::DetCfg<D>;
     static bool det_smem_set = false;
@@ -453,6 +460,7 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
     sp.cu_seqlens = nullptr;  // the ordered dQ kernel takes the [B][H][N][d] layout only
     sp.T = 0;
     sp.o_stride = D;
+    sp.dcols = D;
     sp.B = B;
     sp.H = H;
     sp.N = N;
@@ -489,11 +497,11 @@ int fwd_impl(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o, f
   const int sms = select_device(q);
   if (sms <= 0) return FA_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (d == 64)
-    return launch_fwd<64>(q, k, v, o, lse, B, H, N, scale, causal, block_mask, kv_len, visited, s,
-                          sms, dr, pk);
-  return launch_fwd<128>(q, k, v, o, lse, B, H, N, scale, causal, block_mask, kv_len, visited, s,
-                         sms, dr, pk);
+  if (d <= 64)
+    return launch_fwd<64>(q, k, v, o, lse, B, H, N, d, scale, causal, block_mask, kv_len, visited,
+                          s, sms, dr, pk);
+  return launch_fwd<128>(q, k, v, o, lse, B, H, N, d, scale, causal, block_mask, kv_len, visited,
+                         s, sms, dr, pk);
 }
 
 int bwd_impl(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf16* o,
@@ -505,6 +513,7 @@ int bwd_impl(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf16
   int rc = check_shape(B, H, N, d);
   if (rc == 1) return FA_OK;
   if (rc != FA_OK) return rc;
+  if ((phases & 8u) && d != 64 && d != 128) return FA_ERR_UNSUPPORTED_D;  // ordered dQ
   if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA_ERR_NULL;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
       !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
@@ -518,11 +527,11 @@ int bwd_impl(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf16
   const int sms = select_device(q);
   if (sms <= 0) return FA_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (d == 64)
-    return launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, scale, causal, block_mask,
-                          kv_len, workspace, visited, s, sms, phases, dr, pk);
-  return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, scale, causal, block_mask,
-                         kv_len, workspace, visited, s, sms, phases, dr, pk);
+  if (d <= 64)
+    return launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal,
+                          block_mask, kv_len, workspace, visited, s, sms, phases, dr, pk);
+  return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal,
+                         block_mask, kv_len, workspace, visited, s, sms, phases, dr, pk);
 }
 
 }  // namespace
@@ -673,7 +682,8 @@ const char* fa_status_string(int status) {
     case FA_ERR_NULL: return "a required pointer is NULL";
     case FA_ERR_ALIGN: return "a pointer is not aligned as required";
     case FA_ERR_SHAPE: return "unsupported shape (negative size, or B*H*N >= 2^31)";
-    case FA_ERR_UNSUPPORTED_D: return "head dimension d must be 64 or 128";
+    case FA_ERR_UNSUPPORTED_D:
+      return "head dimension d must be 32, 64, 96 or 128 (64 or 128 for the ordered dQ)";
     case FA_ERR_WORKSPACE: return "workspace missing or smaller than fa_bwd_workspace_size()";
     case FA_ERR_CUDA: return "a CUDA runtime or driver call failed";
     case FA_ERR_TIMEOUT: return "a device pipeline wait timed out; outputs are incomplete";

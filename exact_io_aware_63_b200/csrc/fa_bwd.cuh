@@ -60,7 +60,7 @@ __global__ void __launch_bounds__(256, 8) fa_bwd_pre_kernel(const uint16_t* __re
                                                          float4* __restrict__ dq_acc,
                                                          int* __restrict__ work_counter,
                                                          int N, int Np, long long rows_p,
-                                                         long long rows) {
+                                                         long long rows, int dcols) {
   pdl_launch_dependents();
   pdl_wait();
   // the main kernel's CTAs take work units from this counter
@@ -86,9 +86,9 @@ __global__ void __launch_bounds__(256, 8) fa_bwd_pre_kernel(const uint16_t* __re
       r = bh * N + rr;
     }
     float acc = 0.f;
-    if (valid) {
-      const uint4 a = __ldg(reinterpret_cast<const uint4*>(o + r * D) + part);
-      const uint4 b = __ldg(reinterpret_cast<const uint4*>(dout + r * D) + part);
+    if (valid && part * 8 < dcols) {  // rows of d = dcols columns (D / 8 lanes cover D)
+      const uint4 a = __ldg(reinterpret_cast<const uint4*>(o + r * dcols) + part);
+      const uint4 b = __ldg(reinterpret_cast<const uint4*>(dout + r * dcols) + part);
       const uint32_t av[4] = {a.x, a.y, a.z, a.w};
       const uint32_t bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
@@ -108,7 +108,7 @@ __global__ void __launch_bounds__(256, 8) fa_bwd_pre_kernel(const uint16_t* __re
       lse2[pr] = (l == -INFINITY) ? -INFINITY : -l * kLog2e;
     }
   }
-  const long long n4 = rows * (D / 4);
+  const long long n4 = rows * (dcols / 4);  // the accumulator is [rows][d] float32
   const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
   for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n4;
        e += (long long)gridDim.x * blockDim.x)
@@ -125,7 +125,7 @@ __global__ void __launch_bounds__(256, 8) fa_bwd_pre_packed_kernel(
     const float* __restrict__ lse, float* __restrict__ delta, float* __restrict__ lse2,
     float4* __restrict__ dq_acc, int* __restrict__ work_counter,
     const int32_t* __restrict__ cu_seqlens, int H, int N, int Np, int T, long long rows_p,
-    long long acc_rows) {
+    long long acc_rows, int dcols) {
   pdl_launch_dependents();
   pdl_wait();
   if (blockIdx.x == 0 && threadIdx.x == 0) *work_counter = 0;
@@ -150,9 +150,9 @@ __global__ void __launch_bounds__(256, 8) fa_bwd_pre_packed_kernel(
       lrow = static_cast<long long>(h) * T + sp.start + rr;
     }
     float acc = 0.f;
-    if (valid) {
-      const uint4 a = __ldg(reinterpret_cast<const uint4*>(o + orow * D) + part);
-      const uint4 b = __ldg(reinterpret_cast<const uint4*>(dout + orow * D) + part);
+    if (valid && part * 8 < dcols) {
+      const uint4 a = __ldg(reinterpret_cast<const uint4*>(o + orow * dcols) + part);
+      const uint4 b = __ldg(reinterpret_cast<const uint4*>(dout + orow * dcols) + part);
       const uint32_t av[4] = {a.x, a.y, a.z, a.w};
       const uint32_t bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
@@ -172,7 +172,7 @@ __global__ void __launch_bounds__(256, 8) fa_bwd_pre_packed_kernel(
       lse2[pr] = (l == -INFINITY) ? -INFINITY : -l * kLog2e;
     }
   }
-  const long long n4 = acc_rows * (D / 4);
+  const long long n4 = acc_rows * (dcols / 4);
   const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
   for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n4;
        e += (long long)gridDim.x * blockDim.x)
@@ -215,6 +215,7 @@ struct BwdParams {
   const int32_t* cu_seqlens;
   int T;
   long long o_stride;
+  int dcols;  // the tensors' head dimension d (<= D; columns D > d read as zeros)
   int* work_counter;    // next unit to take (zeroed by fa_bwd_pre_kernel)
   int causal;
   float scale;
@@ -955,9 +956,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       const long long krow = static_cast<long long>(w.tok_base) + c_key;
       const int hcol = kPacked ? w.tz : 0;
       // warpgroup 0 writes the dK row, warpgroup 1 the dV row
-      uint4* out_row = reinterpret_cast<uint4*>(
-          (h ? p.dv : p.dk) + krow * (kPacked ? p.o_stride : static_cast<long long>(D)) +
-          static_cast<long long>(hcol) * D);
+      uint4* out_row = reinterpret_cast<uint4*>((h ? p.dv : p.dk) + krow * p.o_stride +
+                                                static_cast<long long>(hcol) * p.dcols);
       // key rows of a partial last tile beyond N (packed: beyond the sequence)
       // belong to no output
       const bool key_row_ok = c_key < w.nq;
@@ -968,7 +968,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       if (!w.any) {
 #pragma unroll
         for (int c = 0; c < D / 8; ++c)
-          if (key_row_ok) out_row[c] = make_uint4(0, 0, 0, 0);
+          if (key_row_ok && c * 8 < p.dcols) out_row[c] = make_uint4(0, 0, 0, 0);
         continue;
       }
       const bool key_valid = c_key < w.L;
@@ -1228,7 +1228,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
           if (epi_tma) {
             const int g = c * 4 + v4;  // 16-byte granule of the 128-byte row
             *reinterpret_cast<uint4*>(epi_row + ((g ^ (kr & 7)) << 4)) = val;
-          } else if (key_row_ok) {
+          } else if (key_row_ok && c * 32 + v4 * 8 < p.dcols) {
             out_row[c * 4 + v4] = val;
           }
         }
@@ -1301,8 +1301,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
           if (lane == 0) {
 #pragma unroll
             for (int bxi = 0; bxi < Cfg::kDqBoxesPerRound; ++bxi)
-              tma_reduce_add_3d(&tm_dq, (rd * Cfg::kDqBoxesPerRound + bxi) * 32, yz.x, yz.y,
-                                stage_u32 + bxi * 4096);
+              // boxes of 32 columns; those wholly past d (D > d) are not sent
+              if ((rd * Cfg::kDqBoxesPerRound + bxi) * 32 < p.dcols)
+                tma_reduce_add_3d(&tm_dq, (rd * Cfg::kDqBoxesPerRound + bxi) * 32, yz.x, yz.y,
+                                  stage_u32 + bxi * 4096);
             bulk_commit_group();
             bulk_wait_group_read0();
           }

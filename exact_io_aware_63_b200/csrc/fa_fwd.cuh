@@ -122,6 +122,7 @@ struct FwdParams {
   const int32_t* cu_seqlens;
   int T;
   long long o_stride;  // elements between consecutive rows of one head's O (d, or H*d packed)
+  int dcols;           // the tensors' head dimension d (<= D; columns D > d read as zeros)
   int B, H, N, n_t;
   int num_units;
   int heads_per_group;  // unit order: see fwd_decode
@@ -1001,9 +1002,8 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
       // not output
       const bool row_ok = row < w.nq;
       // O row: [B*H*N][d], or [T][H][d] at column h*d; LSE: [B*H*N], or [H][T]
-      uint16_t* const o_row = p.o + (static_cast<long long>(w.tok_base) + row) *
-                                        (kPacked ? p.o_stride : static_cast<long long>(D)) +
-                              (kPacked ? static_cast<long long>(w.tz) * D : 0ll);
+      uint16_t* const o_row = p.o + (static_cast<long long>(w.tok_base) + row) * p.o_stride +
+                              (kPacked ? static_cast<long long>(w.tz) * p.dcols : 0ll);
       float* const lse_ptr = p.lse + (kPacked ? static_cast<long long>(w.tz) * p.T : 0ll) +
                              w.tok_base + row;
       if constexpr (kPair) {
@@ -1050,7 +1050,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
             if (staged) {
               const int g = c * 4 + v4;  // 16-byte granule of the 128-byte row
               *reinterpret_cast<uint4*>(stage_row + ((g ^ (r_local & 7)) << 4)) = val;
-            } else if (row_ok) {
+            } else if (row_ok && c * 32 + v4 * 8 < p.dcols) {
               orow[c * 4 + v4] = val;
             }
           }
@@ -1127,7 +1127,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
           }
 #pragma unroll
           for (int v4 = 0; v4 < 4; ++v4)
-            if (row_ok)
+            if (row_ok && static_cast<int>(col) + v4 * 8 < p.dcols)
               orow[c * 4 + v4] =
                   make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
         }

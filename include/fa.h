@@ -25,7 +25,10 @@
  *  - Tensors Q, K, V, O, dO, dQ, dK, dV are bfloat16 (raw 16-bit patterns,
  *    type fa_bf16), contiguous [B][H][N][d] in device memory, base address
  *    16-byte aligned.  LSE is float32 [B][H][N] (natural log), 4-byte aligned.
- *  - d is 64 or 128.  N is any length: tiles are 128 long, and when 128 does
+ *  - d is 32, 64, 96 or 128 (32 and 96 run on the 64- and 128-column kernels,
+ *    whose loads read the missing columns as zeros and whose stores stop at d;
+ *    the ordered dQ of fa_bwd_deterministic takes 64 and 128 only).
+ *    N is any length: tiles are 128 long, and when 128 does
  *    not divide N the last tile is partial.  B, H, N >= 0; if any is 0 the
  *    call does nothing and returns FA_OK.  B*H*N must be below 2^31.
  *  - scale is finite and > 0 (1/sqrt(d) is the usual choice).
@@ -65,7 +68,7 @@ typedef enum {
     FA_ERR_NULL = -1,           /* a required pointer is NULL */
     FA_ERR_ALIGN = -2,          /* a pointer breaks its alignment rule */
     FA_ERR_SHAPE = -3,          /* negative size, or B*H*N >= 2^31 */
-    FA_ERR_UNSUPPORTED_D = -4,  /* d not in {64, 128} */
+    FA_ERR_UNSUPPORTED_D = -4,  /* d not in {32, 64, 96, 128} ({64, 128} for the ordered dQ) */
     FA_ERR_WORKSPACE = -5,      /* workspace NULL or smaller than fa_bwd_workspace_size */
     FA_ERR_CUDA = -6,           /* a CUDA runtime/driver call failed */
     FA_ERR_TIMEOUT = -7,        /* a device pipeline wait gave up (fa_get_device_status) */

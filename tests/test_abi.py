@@ -52,7 +52,11 @@ def test_workspace_size():
     assert ws % 256 == 0
     assert binding.fa_bwd_workspace_size(1, 1, 100, 64) >= 4 * 100 * 66   # any N >= 1
     assert binding.fa_bwd_workspace_size(1, 1, -128, 64) == 0     # negative
-    assert binding.fa_bwd_workspace_size(1, 1, 128, 96) == 0      # d
+    assert binding.fa_bwd_workspace_size(1, 1, 128, 80) == 0      # d
+    # d = 32 and 96 run on the 64 / 128 kernels; their scratch is sized by d
+    assert binding.fa_bwd_workspace_size(1, 1, 128, 96) >= 4 * 128 * 96
+    assert binding.fa_bwd_workspace_size(1, 1, 128, 96) < binding.fa_bwd_workspace_size(
+        1, 1, 128, 128)
     assert binding.fa_bwd_workspace_size(0, 1, 128, 64) == 0      # empty
 
 
@@ -122,8 +126,9 @@ def test_shape_errors(call):
     assert call(N=-1) == -3
     assert call(B=-1) == -3
     assert call(B=1 << 16, H=1 << 8, N=1 << 8) == -3   # B*H*N >= 2^31
-    assert call(d=96) == -4
-    assert call(d=32) == -4
+    assert call(d=80) == -4
+    assert call(d=256) == -4
+    assert call(d=16) == -4
 
 
 @pytest.mark.parametrize("call", ALL_CALLS)
@@ -184,7 +189,7 @@ def test_dropout_probability_is_checked(call):
     assert call(p_drop=1.0, B=0) == -8
     # valid probabilities pass the dropout check and reach the shape checks
     for good in (0.0, 0.1, 0.5, 0.999):
-        assert call(p_drop=good, d=96) == -4
+        assert call(p_drop=good, d=80) == -4
 
 
 def test_selftest_arguments_are_checked():
@@ -220,7 +225,7 @@ def test_varlen_argument_checks(call):
     assert call(T=-5) == -3
     assert call(max_seqlen=-1) == -3
     assert call(T=300) == -3                   # more tokens than B * max_seqlen
-    assert call(d=96) == -4
+    assert call(d=80) == -4
     assert call(cu=None) == -1
     assert call(cu=P + 2) == -2
     assert call(q=None) == -1
@@ -246,3 +251,14 @@ def test_binding_has_every_declared_function():
     assert set(binding._SIGS) == declared
     for name in declared:
         assert callable(getattr(binding, name)), name
+
+
+def test_ordered_dq_takes_head_dimensions_64_and_128_only():
+    # d = 32 and 96 are accepted by fa_bwd but not by the ordered dQ kernel; the
+    # check comes before any launch
+    assert bwd_det(d=96) == -4
+    assert bwd_det(d=32) == -4
+    lib = binding.load()
+    rc = lib.fa_bwd_phase(3, P, P, P, P, P, P, P, P, P, 1, 1, 128, 96, 0.125, 0, None, None, P,
+                          1 << 30, None)
+    assert rc == -4

@@ -1,0 +1,70 @@
+"""Head dimensions 32 and 96: the 64- and 128-column kernels with tensor maps that read
+the missing columns as zeros and stores that stop at d, against the FP64 oracle."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from exact_io_aware_63_b200 import binding, inputs
+from gpu_helpers import BF16_U, GRAD_TOL, LSE_TOL, O_TOL, check_all_heads, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+DEV = torch.device("cuda", 0)
+
+
+@pytest.mark.parametrize("d", [32, 96])
+@pytest.mark.parametrize("causal", [False, True])
+def test_dense_with_partial_tile_and_key_padding(cuda_device, d, causal):
+    x = inputs.make_inputs(2, 2, 300, d, causal=causal, seed=800 + d,
+                           kv_len=torch.tensor([300, 133], dtype=torch.int32))
+    check_all_heads(x)
+
+
+@pytest.mark.parametrize("d", [32, 96])
+def test_block_mask(cuda_device, d):
+    check_all_heads(inputs.make_inputs(1, 2, 640, d, seed=810 + d, block_keep=0.5))
+
+
+@pytest.mark.parametrize("d", [32, 96])
+def test_packed_batch(cuda_device, d):
+    x = inputs.make_packed_inputs([1, 129, 300, 0, 64], 2, d, causal=True, seed=820 + d)
+    q, k, v, do = (t.to(DEV) for t in (x.q, x.k, x.v, x.dout))
+    cu = x.cu_seqlens.to(DEV)
+    o, lse = binding.attention_forward_varlen(q, k, v, cu, x.max_seqlen, x.scale, True)
+    dq, dk, dv = binding.attention_backward_varlen(q, k, v, o, lse, do, cu, x.max_seqlen,
+                                                   x.scale, True)
+    torch.cuda.synchronize()
+    assert binding.fa_get_device_status() == 0
+    f = lambda t: t.double().cpu().numpy()
+    qd, kd, vd, dod = (f(t) for t in (x.q, x.k, x.v, x.dout))
+    o_ref, lse_ref = oracle.attention_forward_varlen(qd, kd, vd, x.cu_seqlens.numpy(), x.scale,
+                                                     True)
+    assert float(np.abs(f(o) - o_ref).max()) <= O_TOL
+    fin = np.isfinite(lse_ref)
+    assert np.array_equal(np.isfinite(f(lse)), fin)
+    assert float(np.abs(f(lse)[fin] - lse_ref[fin]).max()) <= LSE_TOL
+    g = oracle.attention_backward_varlen(qd, kd, vd, dod, x.cu_seqlens.numpy(), x.scale, True)
+    for name, got, ref in zip(("dq", "dk", "dv"), (dq, dk, dv), g):
+        assert rel_l2(f(got), ref) <= GRAD_TOL, name
+
+
+@pytest.mark.parametrize("d", [32, 96])
+def test_dropout(cuda_device, d):
+    x = inputs.make_inputs(1, 2, 384, d, causal=True, seed=830 + d)
+    q, k, v, do = (t.to(DEV) for t in (x.q, x.k, x.v, x.dout))
+    drop = (0.2, 5, 1)
+    o, lse = binding.attention_forward(q, k, v, x.scale, True, dropout=drop)
+    dq, dk, dv = binding.attention_backward(q, k, v, o, lse, do, x.scale, True, dropout=drop)
+    torch.cuda.synchronize()
+    assert binding.fa_get_device_status() == 0
+    f = lambda t: t.double().cpu().numpy()
+    qd, kd, vd, dod = (f(t) for t in (x.q, x.k, x.v, x.dout))
+    o_ref, _ = oracle.attention_forward_dropout(qd, kd, vd, x.scale, *drop, causal=True)
+    pv, _ = oracle.attention_forward_dropout(qd, kd, np.abs(vd), x.scale, *drop, causal=True)
+    bound = np.maximum(O_TOL, BF16_U * pv + BF16_U * (1 + BF16_U) * np.abs(o_ref) + 1e-5)
+    assert np.all(np.abs(f(o) - o_ref) <= bound)
+    g = oracle.attention_backward_dropout(qd, kd, vd, dod, x.scale, *drop, causal=True)
+    for name, got, ref in zip(("dq", "dk", "dv"), (dq, dk, dv), g[:3]):
+        assert rel_l2(f(got), ref) <= GRAD_TOL, name
