@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -194,6 +195,8 @@ int check_scale(float scale) {
   return (std::isfinite(scale) && scale > 0.f) ? FA_OK : FA_ERR_ARG;
 }
 
+constexpr int kMaxDevices = 64;  // devices whose per-device state is cached
+
 // Makes the device that owns `ptr` current for this runtime instance and
 // returns its SM count (0 on failure).
 int select_device(const void* ptr) {
@@ -205,17 +208,29 @@ int select_device(const void* ptr) {
   int dev = attr.device;
   if (dev < 0) return 0;
   if (cudaSetDevice(dev) != cudaSuccess) return 0;
-  static int sm_count[64] = {0};
-  if (dev < 64 && sm_count[dev]) return sm_count[dev];
+  static std::atomic<int> sm_count[kMaxDevices];
+  if (dev < kMaxDevices) {
+    const int cached = sm_count[dev].load(std::memory_order_relaxed);
+    if (cached > 0) return cached;
+  }
   int n = 0;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  if (dev < 64) sm_count[dev] = n;
+  if (dev < kMaxDevices) sm_count[dev].store(n, std::memory_order_relaxed);
   return n;
 }
 
+// The opt-in to more than 48 KB of dynamic shared memory (cudaFuncSetAttribute)
+// holds for the current device only, so each kernel makes it once per device
+// of the process; `done` is that kernel's record, one flag per device.
 template <typename Kernel>
-bool set_smem(Kernel k, int bytes) {
-  return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+bool ensure_smem(Kernel k, int bytes, std::atomic<bool> (&done)[kMaxDevices]) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return false;
+  if (dev < kMaxDevices && done[dev].load(std::memory_order_acquire)) return true;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return false;
+  if (dev < kMaxDevices) done[dev].store(true, std::memory_order_release);
+  return true;
 }
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -282,12 +297,9 @@ template <int D, bool kPair, bool kDrop, bool kPacked = false>
 int launch_fwd_mode(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                     const CUtensorMap& to, fa::FwdParams& p, cudaStream_t stream, int num_sms) {
   using Cfg = fa::FwdCfg<D, kPair>;
-  static bool smem_set = false;
-  if (!smem_set) {
-    if (!set_smem(fa::fa_fwd_kernel<D, kPair, kDrop, kPacked>, Cfg::kSmemBytes))
-      return FA_ERR_CUDA;
-    smem_set = true;
-  }
+  static std::atomic<bool> smem_done[kMaxDevices];
+  if (!ensure_smem(fa::fa_fwd_kernel<D, kPair, kDrop, kPacked>, Cfg::kSmemBytes, smem_done))
+    return FA_ERR_CUDA;
   const int per_head = kPair ? (p.n_t + 1) / 2 : p.n_t;
   p.num_units = p.B * p.H * per_head;
   const int grid = p.num_units < num_sms ? p.num_units : num_sms;
@@ -364,15 +376,12 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
       !acc_ok || !make_tmap_any(&tdk, dk, B, H, N, d, pk) ||
       !make_tmap_any(&tdv, dv, B, H, N, d, pk))
     return FA_ERR_CUDA;
-  static bool smem_set = false;
-  if (!smem_set) {
-    if (!set_smem(fa::fa_bwd_kernel<D, false, false>, Cfg::kSmemBytes) ||
-        !set_smem(fa::fa_bwd_kernel<D, true, false>, Cfg::kSmemBytes) ||
-        !set_smem(fa::fa_bwd_kernel<D, false, true>, Cfg::kSmemBytes) ||
-        !set_smem(fa::fa_bwd_kernel<D, true, true>, Cfg::kSmemBytes))
-      return FA_ERR_CUDA;
-    smem_set = true;
-  }
+  static std::atomic<bool> smem_done[4][kMaxDevices];
+  if (!ensure_smem(fa::fa_bwd_kernel<D, false, false>, Cfg::kSmemBytes, smem_done[0]) ||
+      !ensure_smem(fa::fa_bwd_kernel<D, true, false>, Cfg::kSmemBytes, smem_done[1]) ||
+      !ensure_smem(fa::fa_bwd_kernel<D, false, true>, Cfg::kSmemBytes, smem_done[2]) ||
+      !ensure_smem(fa::fa_bwd_kernel<D, true, true>, Cfg::kSmemBytes, smem_done[3]))
+    return FA_ERR_CUDA;
   // preprocess
   if (phases & 1u) {
     const int threads = 256;
@@ -445,11 +454,9 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
   // (head dimensions 64 and 128 only: bwd_impl checks it before any launch)
   if (phases & 8u) {
     using DCfg = fa::DetCfg<D>;
-    static bool det_smem_set = false;
-    if (!det_smem_set) {
-      if (!set_smem(fa::fa_bwd_dq_det_kernel<D>, DCfg::kSmemBytes)) return FA_ERR_CUDA;
-      det_smem_set = true;
-    }
+    static std::atomic<bool> det_smem_done[kMaxDevices];
+    if (!ensure_smem(fa::fa_bwd_dq_det_kernel<D>, DCfg::kSmemBytes, det_smem_done))
+      return FA_ERR_CUDA;
     fa::DetParams dp;
     fa::FwdParams& sp = dp.sched;
     sp.o = nullptr;
@@ -710,7 +717,6 @@ static __device__ __align__(256) unsigned char fa_bwd_noalloc_scratch[FA_BWD_NOA
 
 namespace {
 
-constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mutex;
 void* g_noalloc_ptr[kMaxDevices] = {};
 

@@ -45,6 +45,10 @@
  *  - The caller owns every buffer.  fa_fwd allocates nothing.  fa_bwd uses
  *    only the caller's workspace.  Nothing is freed by the library.
  *  - On any nonzero return, nothing was launched and no output was touched.
+ *  - Each call makes the device that holds q current and launches there.
+ *    Calls may come from several host threads and target several devices
+ *    of one process; the library's per-device set-up (the kernels' shared
+ *    memory opt-in, the SM count) is made once per device.
  *  - Kernels are launched with programmatic stream serialization: each may
  *    be scheduled while the previous kernel in the stream is finishing and
  *    waits, before it touches global memory, until that kernel's writes are
@@ -278,7 +282,8 @@ int fa_selftest_wait_timeout(int arrive, unsigned int limit_us, int* result, voi
  * allocate device memory themselves: code that runs where the host side owns
  * no device allocator (a plugin handed only input and output buffers by its
  * host application), or deployments that forbid device allocations after
- * start-up.  The paper has no counterpart; this is an interface convenience.
+ * start-up.  The method itself has no counterpart: it is an interface
+ * convenience.
  *
  * Same arguments and results as fa_bwd, minus the workspace.  The scratch
  * (D, base-2 LSE and the float32 dQ accumulator) lives in one static device
