@@ -16,7 +16,9 @@ torch tensors or None, the stream as a torch.cuda.Stream or None = current):
 Convenience wrappers that allocate outputs: ``attention_forward`` and
 ``attention_backward`` (options ``dropout=(p, seed, offset)`` and, for the backward,
 ``deterministic=True``), ``attention_forward_varlen`` and ``attention_backward_varlen``
-for packed batches.
+for packed batches.  They check what the raw pointers cannot carry (dtype, shape,
+contiguity, one device for all tensors) and raise ValueError before any library call;
+they launch on the current stream of q's device unless given a stream.
 """
 
 from __future__ import annotations
@@ -245,12 +247,88 @@ def _check(rc, what):
         raise FAError(rc, what)
 
 
+def _expect(t, name, dtype, shape, device):
+    """Raise unless ``t`` is a contiguous tensor of ``dtype`` and ``shape`` on ``device``:
+    the C ABI sees raw pointers and cannot tell a wrong layout from a right one."""
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor, not {type(t).__name__}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device} (the device of q)")
+
+
+def _expect_workspace(ws, device):
+    import torch
+    if not isinstance(ws, torch.Tensor) or not ws.is_contiguous() or ws.device != device:
+        raise ValueError(f"workspace must be a contiguous tensor on {device}")
+
+
+def _expect_visited(visited, B, H, N, device):
+    import torch
+    nt = (N + 127) // 128
+    _expect(visited, "visited", torch.uint8, (B, H, nt, nt), device)
+
+
+def _expect_cuda(q, stream):
+    """Raise unless q is a CUDA tensor; return the stream to launch on (default: the current
+    stream of q's device, not of the current device)."""
+    import torch
+    if q.device.type != "cuda":
+        raise ValueError(f"the tensors must be CUDA tensors, q is on {q.device}")
+    return torch.cuda.current_stream(q.device) if stream is None else stream
+
+
+def _expect_dense(q, k, v, block_mask, kv_len, extra=()):
+    """Checks of a [B, H, N, d] call: q, k, v and ``extra`` (name, tensor, dtype, shape)."""
+    import torch
+    if not isinstance(q, torch.Tensor) or q.dim() != 4:
+        raise ValueError("q must be a 4-D tensor [B, H, N, d]")
+    B, H, N, d = q.shape
+    dev = q.device
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _expect(t, name, torch.bfloat16, (B, H, N, d), dev)
+    for name, t, dtype, shape in extra:
+        _expect(t, name, dtype, shape, dev)
+    nt = (N + 127) // 128
+    if block_mask is not None:
+        _expect(block_mask, "block_mask", torch.uint8, (nt, nt), dev)
+    if kv_len is not None:
+        _expect(kv_len, "kv_len", torch.int32, (B,), dev)
+    return B, H, N, d
+
+
+def _expect_packed(q, k, v, cu_seqlens, extra=()):
+    """Checks of a packed [T, H, d] call."""
+    import torch
+    if not isinstance(q, torch.Tensor) or q.dim() != 3:
+        raise ValueError("q must be a 3-D tensor [T, H, d]")
+    T, H, d = q.shape
+    dev = q.device
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _expect(t, name, torch.bfloat16, (T, H, d), dev)
+    if not isinstance(cu_seqlens, torch.Tensor) or cu_seqlens.dim() != 1 or cu_seqlens.numel() < 1:
+        raise ValueError("cu_seqlens must be a 1-D tensor [B + 1]")
+    _expect(cu_seqlens, "cu_seqlens", torch.int32, (cu_seqlens.numel(),), dev)
+    for name, t, dtype, shape in extra:
+        _expect(t, name, dtype, shape, dev)
+    return T, H, d
+
+
 def attention_forward(q, k, v, scale, causal=False, block_mask=None, kv_len=None, visited=None,
                       stream=None, dropout=None):
     """O, LSE for bf16 CUDA tensors q, k, v of shape [B, H, N, d].  ``dropout`` is None or
     (p_drop, seed, offset) and selects fa_fwd_dropout."""
     import torch
-    B, H, N, d = q.shape
+    B, H, N, d = _expect_dense(q, k, v, block_mask, kv_len)
+    if visited is not None:
+        _expect_visited(visited, B, H, N, q.device)
+    stream = _expect_cuda(q, stream)
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     if dropout is not None:
@@ -275,29 +353,36 @@ def attention_backward(q, k, v, o, lse, dout, scale, causal=False, block_mask=No
     fa_bwd_deterministic (bitwise-reproducible dQ); ``dropout`` = (p_drop, seed, offset),
     the forward's, selects fa_bwd_dropout."""
     import torch
-    B, H, N, d = q.shape
+    B, H, N, d = _expect_dense(q, k, v, block_mask, kv_len, extra=(
+        ("o", o, torch.bfloat16, q.shape), ("dout", dout, torch.bfloat16, q.shape),
+        ("lse", lse, torch.float32, q.shape[:3])))
+    if visited is not None:
+        _expect_visited(visited, B, H, N, q.device)
+    stream = _expect_cuda(q, stream)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws_bytes = fa_bwd_workspace_size(B, H, N, d)
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    else:
+        _expect_workspace(workspace, q.device)
     if dropout is not None:
         if visited is not None or deterministic:
             raise ValueError("the dropout backward has no traced or deterministic variant")
         p_drop, seed, offset = dropout
         rc = fa_bwd_dropout(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal,
                             block_mask, kv_len, p_drop, seed, offset, workspace,
-                            workspace.numel(), stream)
+                            workspace.nbytes, stream)
     elif deterministic:
         if visited is not None:
             raise ValueError("the deterministic backward has no traced variant")
         rc = fa_bwd_deterministic(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal,
-                                  block_mask, kv_len, workspace, workspace.numel(), stream)
+                                  block_mask, kv_len, workspace, workspace.nbytes, stream)
     elif visited is None:
         rc = fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, block_mask,
-                    kv_len, workspace, workspace.numel(), stream)
+                    kv_len, workspace, workspace.nbytes, stream)
     else:
         rc = fa_bwd_traced(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal,
-                           block_mask, kv_len, workspace, workspace.numel(), visited, stream)
+                           block_mask, kv_len, workspace, workspace.nbytes, visited, stream)
     _check(rc, "fa_bwd")
     return dq, dk, dv
 
@@ -307,7 +392,8 @@ def attention_forward_varlen(q, k, v, cu_seqlens, max_seqlen, scale, causal=Fals
     """O [T, H, d] and LSE [H, T] for a packed batch: bf16 CUDA tensors [T, H, d] and
     int32 CUDA cu_seqlens [B + 1]; ``dropout`` = None or (p_drop, seed, offset)."""
     import torch
-    T, H, d = q.shape
+    T, H, d = _expect_packed(q, k, v, cu_seqlens)
+    stream = _expect_cuda(q, stream)
     B = cu_seqlens.numel() - 1
     o = torch.empty_like(q)
     lse = torch.empty((H, T), dtype=torch.float32, device=q.device)
@@ -322,14 +408,19 @@ def attention_backward_varlen(q, k, v, o, lse, dout, cu_seqlens, max_seqlen, sca
                               dropout=None, workspace=None, stream=None):
     """dQ, dK, dV [T, H, d] for the packed forward that produced (o, lse)."""
     import torch
-    T, H, d = q.shape
+    T, H, d = _expect_packed(q, k, v, cu_seqlens, extra=(
+        ("o", o, torch.bfloat16, q.shape), ("dout", dout, torch.bfloat16, q.shape),
+        ("lse", lse, torch.float32, (q.shape[1], q.shape[0]))))
+    stream = _expect_cuda(q, stream)
     B = cu_seqlens.numel() - 1
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws_bytes = fa_bwd_workspace_size(B, H, max_seqlen, d)
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    else:
+        _expect_workspace(workspace, q.device)
     p_drop, seed, offset = dropout if dropout is not None else (0.0, 0, 0)
     rc = fa_bwd_varlen(q, k, v, o, lse, dout, dq, dk, dv, cu_seqlens, B, H, max_seqlen, T, d,
-                       scale, causal, p_drop, seed, offset, workspace, workspace.numel(), stream)
+                       scale, causal, p_drop, seed, offset, workspace, workspace.nbytes, stream)
     _check(rc, "fa_bwd_varlen")
     return dq, dk, dv
