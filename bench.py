@@ -576,7 +576,7 @@ def run_reference(args):
         return
     from exact_io_aware_63_b200 import inputs
     w = inputs.WORKLOADS[args.workload]
-    x = inputs.workload_inputs(args.workload)
+    x = workload_or_shape(args)
     threads = os.cpu_count() or 1
     B, H, N, d = x.q.shape
     n_heads, n_rows = sample_plan(x, threads)
@@ -597,14 +597,13 @@ def run_reference(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
             "config": {"workload": args.workload + (f" at shape {args.shape}" if args.shape else ""),
-                   "description": w.description, "B": B, "H": H,
-                       "N": N, "d": d, "parallelism": "cpu threads"},
+                       "description": w.description, "B": B, "H": H, "N": N, "d": d,
+                       "parallelism": "cpu threads"},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": used, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
-
 
 
 # ----------------------------------------------------------------------------

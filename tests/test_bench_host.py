@@ -80,3 +80,48 @@ def test_ideal_bytes_follow_the_rows():
         E = R * 64
         got = bench.ideal_bytes(x) if R == 2 * 3 * 256 else bench.ideal_bytes(x, rows=R)
         assert got == (8 * E + 4 * R, 20 * E + 8 * R)
+
+
+def test_oracle_sample_flops_cover_the_workload_when_the_sample_is_everything():
+    # the CPU baseline counts a sample's FLOPs as the metric counts the whole workload,
+    # pro rata to allowed entries: a sample of every head and row is the whole count
+    x = inputs.make_inputs(2, 2, 256, 64, causal=True, seed=11, key_padding=(100, 256))
+    _, flops, heads = bench.time_oracle(x, 4, 256, threads=2)
+    assert len(heads) == 4
+    assert abs(flops - 3.5 * bench.flops_fwd(x)) <= 1e-9 * flops
+    # half the heads (both of batch 0): batch 0's share of the allowed entries
+    _, half, heads = bench.time_oracle(x, 2, 256, threads=2)
+    assert heads == [(0, 0), (0, 1)]
+    share = bench.allowed_entries(x, range(256))
+    assert abs(half - 3.5 * bench.flops_fwd(x) * share[0] / share.sum()) <= 1e-9 * half
+
+
+def _bench(*argv, env=None):
+    import json
+    import subprocess
+    e = dict(os.environ)
+    e.update(env or {})
+    r = subprocess.run([sys.executable, os.path.join(os.path.dirname(bench.__file__), "bench.py"),
+                        *argv], capture_output=True, text=True, timeout=300, env=e)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    return [json.loads(l) for l in lines]
+
+
+def test_reference_arm_prints_one_contract_line():
+    (line,) = _bench("--impl", "reference", "--shape", "1,2,256,64", "--steps", "2",
+                     "--warmup", "1")
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC
+    assert line["unit"] == "TFLOP/s" and line["higher_is_better"] is True
+    assert line["n_gpus"] == 1 and line["steps"] == 2 and line["warmup"] == 1
+    assert line["value"] > 0 and line["dtype"] == "f64"
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1
+    assert line["e2e"] == {"value": line["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+    assert line["config"]["N"] == 256 and line["config"]["H"] == 2
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    assert _bench("--impl", "reference", "--shape", "1,1,128,64", "--steps", "1", "--warmup", "1",
+                  env={"RANK": "1", "WORLD_SIZE": "2"}) == []
