@@ -32,7 +32,8 @@ Functions (all arrays contiguous, float64 unless stated):
 * ``attention_forward_dropout`` / ``attention_backward_dropout`` (extra
   arguments ``p_drop, seed, offset``): the same with dropout on P; the mask is
   ``dropout_keep(BH, N, p_drop, seed, offset)``, cut from Philox-4x32-10 draws
-  (``philox4x32_10(counter, key)``).
+  (``philox4x32_10(counter, key)``, checked word for word against cuRAND's
+  host-side Philox-4x32-10 generator in the tests).
 * ``attention_forward_varlen(q, k, v, cu_seqlens, scale, causal, dropout)`` /
   ``attention_backward_varlen(q, k, v, dout, cu_seqlens, scale, causal,
   dropout)``: packed variable-length batches (q, k, v, dout [T, H, d];
