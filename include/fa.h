@@ -312,7 +312,10 @@ int fa_bwd_noalloc(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const f
  * has reported a device-side failure since the last call, FA_ERR_TIMEOUT
  * if a pipeline wait gave up (the kernel then skipped the rest of its work
  * and its outputs are incomplete), or FA_ERR_CUDA if synchronising failed.
- * Clears the recorded state.  The state is per process and per device.
+ * Clears the recorded state.  The state is per process and per device, and
+ * the call reads that of the calling thread's current device: the device of
+ * the last entry point this thread called (each call makes q's device
+ * current), so pass a stream of that device.
  */
 int fa_get_device_status(void* stream);
 
