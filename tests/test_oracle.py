@@ -580,3 +580,69 @@ def test_varlen_equal_lengths_is_the_batched_problem_with_dropout():
                                            causal=True)
     for got, want in zip(g, gd[:3]):
         np.testing.assert_allclose(dense(got), want, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# the backward against automatic differentiation at a multi-tile size
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("causal,kv,use_bm", [(False, None, False), (True, None, False),
+                                              (False, (150, 300), True), (True, (100, 260), True)])
+def test_backward_matches_automatic_differentiation(causal, kv, use_bm):
+    # The finite-difference pins run at N = 16; this one runs at N = 300 (two full tiles and
+    # a partial one), where the gradients come from torch's reverse-mode differentiation of
+    # L = sum(O * dO) in float64 rather than from the oracle's hand-derived chain rule.
+    import torch
+    B, H, N, d, s = 2, 2, 300, 32, 0.17
+    q, k, v, do = (rand((B, H, N, d), 900 + i) for i in range(4))
+    kvl = None if kv is None else np.array(kv, np.int32)
+    bm = None
+    if use_bm:
+        bm = np.zeros((3, 3), np.uint8)
+        bm[np.arange(3), np.arange(3)] = 1
+        bm[:, 0] = 1  # key 0 stays allowed, so no row is left without keys
+        bm[0, 2] = 1
+    dq, dk, dv, _ = oracle.attention_backward(q, k, v, do, s, causal, bm, kvl)
+
+    r = np.arange(N)[:, None]
+    c = np.arange(N)[None, :]
+    allowed = np.ones((B, 1, N, N), bool)
+    if causal:
+        allowed &= (c <= r)[None, None]
+    if kvl is not None:
+        allowed &= (c[None, None] < kvl[:, None, None, None])
+    if bm is not None:
+        allowed &= bm[r // 128, c // 128].astype(bool)[None, None]
+    tq, tk, tv = (torch.tensor(t, requires_grad=True) for t in (q, k, v))
+    scores = s * tq @ tk.transpose(-1, -2)
+    scores = scores.masked_fill(~torch.tensor(allowed), float("-inf"))
+    out = torch.softmax(scores, dim=-1) @ tv
+    (out * torch.tensor(do)).sum().backward()
+    for name, mine, ref in (("dq", dq, tq.grad), ("dk", dk, tk.grad), ("dv", dv, tv.grad)):
+        np.testing.assert_allclose(mine, ref.numpy(), rtol=0, atol=1e-11, err_msg=name)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_dropout_backward_matches_automatic_differentiation(causal):
+    # dropout's keep mask is an input to the arithmetic (drawn by dropout_keep); given it,
+    # O = w (P o Z) V and torch differentiates sum(O * dO) in float64 at N = 300
+    import torch
+    B, H, N, d, s = 1, 2, 300, 32, 0.2
+    p_drop, seed, offset = 0.3, 77, 5
+    q, k, v, do = (rand((B, H, N, d), 950 + i) for i in range(4))
+    kvl = np.array([230], np.int32)
+    dq, dk, dv, _ = oracle.attention_backward_dropout(q, k, v, do, s, p_drop, seed, offset,
+                                                      causal=causal, kv_len=kvl)
+    keep, _ = oracle.dropout_keep(B * H, N, p_drop, seed, offset)
+    t = math.floor(p_drop * 65536)
+    w = 65536.0 / (65536.0 - t)
+    r = np.arange(N)[:, None]
+    c = np.arange(N)[None, :]
+    allowed = (c < kvl[0]) & ((c <= r) if causal else True)
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    scores = (s * tq @ tk.transpose(-1, -2)).masked_fill(~torch.tensor(allowed), float("-inf"))
+    z = torch.tensor(keep.reshape(B, H, N, N).astype(np.float64))
+    out = (torch.softmax(scores, dim=-1) * z * w) @ tv
+    (out * torch.tensor(do)).sum().backward()
+    for name, mine, ref in (("dq", dq, tq.grad), ("dk", dk, tk.grad), ("dv", dv, tv.grad)):
+        np.testing.assert_allclose(mine, ref.numpy(), rtol=0, atol=1e-11, err_msg=name)
