@@ -262,3 +262,47 @@ def test_ordered_dq_takes_head_dimensions_64_and_128_only():
     rc = lib.fa_bwd_phase(3, P, P, P, P, P, P, P, P, P, 1, 1, 128, 96, 0.125, 0, None, None, P,
                           1 << 30, None)
     assert rc == -4
+
+
+C_CONSUMER = r"""
+#include <stdio.h>
+#include <string.h>
+#include "fa.h"
+
+int main(void) {
+    /* host-side paths only: no GPU is needed for any of these calls */
+    if (fa_version() <= 0) return 1;
+    if (strlen(fa_status_string(FA_ERR_SHAPE)) == 0) return 2;
+    if (fa_bwd_workspace_size(2, 3, 300, 64) == 0) return 3;
+    if (fa_bwd_workspace_size(-1, 3, 300, 64) != 0) return 4;
+    /* argument errors come back before any CUDA call */
+    if (fa_fwd(NULL, NULL, NULL, NULL, NULL, 1, 1, 128, 80, 0.125f, 0, NULL, NULL, NULL)
+        != FA_ERR_UNSUPPORTED_D) return 5;
+    if (fa_fwd(NULL, NULL, NULL, NULL, NULL, 1, 1, 128, 64, 0.125f, 0, NULL, NULL, NULL)
+        != FA_ERR_NULL) return 6;
+    if (fa_fwd(NULL, NULL, NULL, NULL, NULL, 0, 1, 128, 64, 0.125f, 0, NULL, NULL, NULL)
+        != FA_OK) return 7;
+    printf("ok %d\n", fa_version());
+    return 0;
+}
+"""
+
+
+def test_plain_c_program_links_and_calls_the_library(tmp_path):
+    # the boundary is a C ABI: a C99 program with no C++ or Python links against it
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not installed")
+    binding.load()  # builds the library if it is missing
+    lib_dir = os.path.dirname(binding.library_path())
+    src = tmp_path / "consumer.c"
+    src.write_text(C_CONSUMER)
+    exe = tmp_path / "consumer"
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.dirname(HEADER), str(src),
+                    "-L", lib_dir, "-lfa_b200", f"-Wl,-rpath,{lib_dir}", "-o", str(exe)],
+                   check=True, timeout=120)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, (r.returncode, r.stderr)
+    assert r.stdout.startswith("ok ")
