@@ -72,3 +72,32 @@ def test_packed_inputs_offsets_and_shapes():
     assert x.causal and abs(x.scale - 1 / math.sqrt(32)) < 1e-12
     assert inputs.draw_lengths(4, 10, 20, seed=7) == inputs.draw_lengths(4, 10, 20, seed=7)
     assert all(10 <= n <= 20 for n in inputs.draw_lengths(100, 10, 20, seed=8))
+
+
+def test_workload_table_matches_the_stated_configurations():
+    # (B, H, N, d), scale, causal, key padding, block-sparse for each named workload
+    want = {
+        "tiny": ((1, 1, 128, 64), 1 / 8, False, False, False),
+        "bert": ((16, 16, 512, 64), 1 / 8, False, True, False),
+        "gpt2": ((8, 12, 1024, 64), 1 / 8, True, False, False),
+        "long16k": ((1, 16, 16384, 128), 1 / math.sqrt(128), False, False, False),
+        "long16k_causal": ((1, 16, 16384, 128), 1 / math.sqrt(128), True, False, False),
+        "sparse64k": ((1, 8, 65536, 64), 1 / 8, False, False, True),
+    }
+    assert set(inputs.WORKLOADS) == set(want)
+    for name, (shape, scale, causal, padding, sparse) in want.items():
+        w = inputs.WORKLOADS[name]
+        assert (w.B, w.H, w.N, w.d) == shape, name
+        assert abs(w.scale - scale) < 1e-15 and w.causal == causal, name
+        assert w.key_padding == padding and w.block_sparse == sparse, name
+    # the two 16K workloads draw the same tensors; the others each have their own seed
+    assert inputs.WORKLOADS["long16k"].seed == inputs.WORKLOADS["long16k_causal"].seed
+    seeds = [w.seed for n, w in inputs.WORKLOADS.items() if n != "long16k_causal"]
+    assert len(set(seeds)) == len(seeds)
+
+
+def test_tiny_workload_tensors():
+    x = inputs.workload_inputs("tiny")
+    assert x.q.shape == (1, 1, 128, 64) and x.q.dtype == torch.bfloat16
+    assert x.kv_len is None and x.block_mask is None and not x.causal
+    assert abs(x.scale - 0.125) < 1e-15
