@@ -752,6 +752,11 @@ def main():
         ap.error(" and ".join(modes) + " select different backward paths: give one")
     if not 0.0 <= args.dropout < 1.0:
         ap.error("--dropout must lie in [0, 1)")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.impl == "ours" and not args.vs_standard and args.gpus != world:
+        ap.error(f"--gpus {args.gpus} with {world} process(es): launch one process per GPU, "
+                 f"e.g. python -m torch.distributed.run --nproc-per-node {args.gpus} bench.py "
+                 f"--gpus {args.gpus}")
     if args.warmup < 3 and args.impl == "ours":
         print("note: warm-up raised to 3 steps", file=sys.stderr)
         args.warmup = 3

@@ -125,3 +125,11 @@ def test_reference_arm_prints_one_contract_line():
 def test_reference_arm_runs_on_rank_zero_only():
     assert _bench("--impl", "reference", "--shape", "1,1,128,64", "--steps", "1", "--warmup", "1",
                   env={"RANK": "1", "WORLD_SIZE": "2"}) == []
+
+
+def test_gpu_count_must_match_the_launched_processes():
+    import subprocess
+    r = subprocess.run([sys.executable, os.path.join(os.path.dirname(bench.__file__), "bench.py"),
+                        "--gpus", "2", "--steps", "1"], capture_output=True, text=True, timeout=120,
+                       env={k: v for k, v in os.environ.items() if k != "WORLD_SIZE"})
+    assert r.returncode != 0 and "one process per GPU" in r.stderr
