@@ -133,3 +133,24 @@ def test_gpu_count_must_match_the_launched_processes():
                         "--gpus", "2", "--steps", "1"], capture_output=True, text=True, timeout=120,
                        env={k: v for k, v in os.environ.items() if k != "WORLD_SIZE"})
     assert r.returncode != 0 and "one process per GPU" in r.stderr
+
+
+def test_traffic_is_reported_only_for_the_sources_it_was_taken_on(tmp_path, monkeypatch):
+    # bench.py reports ncu DRAM bytes only while the benchmarked kernels' sources hash to
+    # the value recorded beside them; any change to those sources turns it into null
+    import json
+    csrc = tmp_path / "exact_io_aware_63_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for name in bench.BENCHED_KERNEL_SOURCES:
+        (csrc / name).write_text(f"// {name}\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h = bench.kernel_source_hash()
+    (tmp_path / "profiles").mkdir()
+    rec = {"bert": {"fa_bwd_kernel": {"dram_bytes_per_launch": 123, "source_hash": h}}}
+    (tmp_path / "profiles" / "ncu_traffic.json").write_text(json.dumps(rec))
+    assert bench.ncu_traffic("fa_bwd_kernel", "bert") == 123
+    assert bench.ncu_traffic("fa_fwd_kernel", "bert") is None
+    assert bench.ncu_traffic("fa_bwd_kernel", "gpt2") is None
+    (csrc / bench.BENCHED_KERNEL_SOURCES[0]).write_text("// changed\n")
+    assert bench.kernel_source_hash() != h
+    assert bench.ncu_traffic("fa_bwd_kernel", "bert") is None
