@@ -109,10 +109,14 @@ def _ptr(t):
     return t.data_ptr()
 
 
-def _stream(stream):
+def _stream(stream, like=None):
+    """The stream handle to pass: ``stream`` itself (a torch.cuda.Stream or a raw handle),
+    else the current stream of the device that holds ``like`` (else of the current
+    device)."""
     import torch
     if stream is None:
-        stream = torch.cuda.current_stream()
+        dev = like.device if isinstance(like, torch.Tensor) and like.is_cuda else None
+        stream = torch.cuda.current_stream(dev)
     if isinstance(stream, int):
         return stream
     return stream.cuda_stream
@@ -124,14 +128,14 @@ def _stream(stream):
 
 def fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, block_mask, kv_len, stream=None):
     return load().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, float(scale),
-                         int(bool(causal)), _ptr(block_mask), _ptr(kv_len), _stream(stream))
+                         int(bool(causal)), _ptr(block_mask), _ptr(kv_len), _stream(stream, q))
 
 
 def fa_fwd_traced(q, k, v, o, lse, B, H, N, d, scale, causal, block_mask, kv_len, visited,
                   stream=None):
     return load().fa_fwd_traced(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
                                 float(scale), int(bool(causal)), _ptr(block_mask), _ptr(kv_len),
-                                _ptr(visited), _stream(stream))
+                                _ptr(visited), _stream(stream, q))
 
 
 def fa_bwd_workspace_size(B, H, N, d):
@@ -143,7 +147,7 @@ def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, block_m
     return load().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq),
                          _ptr(dk), _ptr(dv), B, H, N, d, float(scale), int(bool(causal)),
                          _ptr(block_mask), _ptr(kv_len), _ptr(workspace), int(workspace_bytes),
-                         _stream(stream))
+                         _stream(stream, q))
 
 
 def fa_bwd_traced(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, block_mask, kv_len,
@@ -151,7 +155,7 @@ def fa_bwd_traced(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, 
     return load().fa_bwd_traced(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
                                 _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, float(scale),
                                 int(bool(causal)), _ptr(block_mask), _ptr(kv_len), _ptr(workspace),
-                                int(workspace_bytes), _ptr(visited), _stream(stream))
+                                int(workspace_bytes), _ptr(visited), _stream(stream, q))
 
 
 def fa_bwd_phase(phase, q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, block_mask,
@@ -159,7 +163,7 @@ def fa_bwd_phase(phase, q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, ca
     return load().fa_bwd_phase(int(phase), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
                                _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, float(scale),
                                int(bool(causal)), _ptr(block_mask), _ptr(kv_len), _ptr(workspace),
-                               int(workspace_bytes), _stream(stream))
+                               int(workspace_bytes), _stream(stream, q))
 
 
 def fa_bwd_deterministic(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal,
@@ -168,7 +172,7 @@ def fa_bwd_deterministic(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, c
     return load().fa_bwd_deterministic(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
                                        _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, float(scale),
                                        int(bool(causal)), _ptr(block_mask), _ptr(kv_len),
-                                       _ptr(workspace), int(workspace_bytes), _stream(stream))
+                                       _ptr(workspace), int(workspace_bytes), _stream(stream, q))
 
 
 def fa_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, block_mask,
@@ -178,7 +182,7 @@ def fa_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal,
     return load().fa_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
                                  _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, float(scale),
                                  int(bool(causal)), _ptr(block_mask), _ptr(kv_len),
-                                 _stream(stream))
+                                 _stream(stream, q))
 
 
 def fa_fwd_dropout(q, k, v, o, lse, B, H, N, d, scale, causal, block_mask, kv_len, p_drop, seed,
@@ -186,7 +190,7 @@ def fa_fwd_dropout(q, k, v, o, lse, B, H, N, d, scale, causal, block_mask, kv_le
     """fa_fwd with dropout of probability p_drop on P (Philox keep mask, include/fa.h)."""
     return load().fa_fwd_dropout(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
                                  float(scale), int(bool(causal)), _ptr(block_mask), _ptr(kv_len),
-                                 float(p_drop), int(seed), int(offset), _stream(stream))
+                                 float(p_drop), int(seed), int(offset), _stream(stream, q))
 
 
 def fa_bwd_dropout(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, block_mask,
@@ -196,7 +200,7 @@ def fa_bwd_dropout(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal,
                                  _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, float(scale),
                                  int(bool(causal)), _ptr(block_mask), _ptr(kv_len),
                                  float(p_drop), int(seed), int(offset), _ptr(workspace),
-                                 int(workspace_bytes), _stream(stream))
+                                 int(workspace_bytes), _stream(stream, q))
 
 
 def fa_fwd_varlen(q, k, v, o, lse, cu_seqlens, B, H, max_seqlen, total_tokens, d, scale, causal,
@@ -205,7 +209,7 @@ def fa_fwd_varlen(q, k, v, o, lse, cu_seqlens, B, H, max_seqlen, total_tokens, d
     return load().fa_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_seqlens),
                                 B, H, max_seqlen, total_tokens, d, float(scale),
                                 int(bool(causal)), float(p_drop), int(seed), int(offset),
-                                _stream(stream))
+                                _stream(stream, q))
 
 
 def fa_bwd_varlen(q, k, v, o, lse, dout, dq, dk, dv, cu_seqlens, B, H, max_seqlen, total_tokens,
@@ -217,13 +221,13 @@ def fa_bwd_varlen(q, k, v, o, lse, dout, dq, dk, dv, cu_seqlens, B, H, max_seqle
                                 _ptr(dq), _ptr(dk), _ptr(dv), _ptr(cu_seqlens), B, H, max_seqlen,
                                 total_tokens, d, float(scale), int(bool(causal)), float(p_drop),
                                 int(seed), int(offset), _ptr(workspace), int(workspace_bytes),
-                                _stream(stream))
+                                _stream(stream, q))
 
 
 def fa_selftest_wait_timeout(arrive, limit_us, result, stream=None):
     """One warp waits on a barrier for at most limit_us; see include/fa.h."""
     return load().fa_selftest_wait_timeout(int(arrive), int(limit_us), _ptr(result),
-                                           _stream(stream))
+                                           _stream(stream, result))
 
 
 def fa_get_device_status(stream=None):
