@@ -646,3 +646,38 @@ def test_dropout_backward_matches_automatic_differentiation(causal):
     (out * torch.tensor(do)).sum().backward()
     for name, mine, ref in (("dq", dq, tq.grad), ("dk", dk, tk.grad), ("dv", dv, tv.grad)):
         np.testing.assert_allclose(mine, ref.numpy(), rtol=0, atol=1e-11, err_msg=name)
+
+
+@pytest.mark.parametrize("causal,kv,use_bm", [(False, None, False), (True, None, False),
+                                              (True, (120, 300), True)])
+def test_forward_and_backward_match_torch_scaled_dot_product_attention(causal, kv, use_bm):
+    # torch's own attention routine (its float64 CPU path), with the mask as a boolean
+    # "may attend" matrix, is an independent implementation of the same definition
+    import torch
+    import torch.nn.functional as F
+    B, H, N, d, s = 2, 3, 300, 32, 0.21
+    q, k, v, do = (rand((B, H, N, d), 970 + i) for i in range(4))
+    kvl = None if kv is None else np.array(kv, np.int32)
+    bm = None
+    if use_bm:
+        bm = np.eye(3, dtype=np.uint8)
+        bm[2, 1] = 1
+        bm[:, 0] = 1  # key 0 stays allowed for every row
+    o, _ = oracle.attention_forward(q, k, v, s, causal, bm, kvl)
+    dq, dk, dv, _ = oracle.attention_backward(q, k, v, do, s, causal, bm, kvl)
+    r = np.arange(N)[:, None]
+    c = np.arange(N)[None, :]
+    allowed = np.ones((B, 1, N, N), bool)
+    if causal:
+        allowed &= (c <= r)[None, None]
+    if kvl is not None:
+        allowed &= (c[None, None] < kvl[:, None, None, None])
+    if bm is not None:
+        allowed &= bm[r // 128, c // 128].astype(bool)[None, None]
+    assert allowed.any(-1).all()  # every row keeps a key (the routine has no empty rows)
+    tq, tk, tv = (torch.tensor(t, requires_grad=True) for t in (q, k, v))
+    out = F.scaled_dot_product_attention(tq, tk, tv, attn_mask=torch.tensor(allowed), scale=s)
+    (out * torch.tensor(do)).sum().backward()
+    np.testing.assert_allclose(o, out.detach().numpy(), rtol=0, atol=1e-12)
+    for name, mine, ref in (("dq", dq, tq.grad), ("dk", dk, tk.grad), ("dv", dv, tv.grad)):
+        np.testing.assert_allclose(mine, ref.numpy(), rtol=0, atol=1e-11, err_msg=name)
