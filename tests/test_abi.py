@@ -306,3 +306,16 @@ def test_plain_c_program_links_and_calls_the_library(tmp_path):
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0, (r.returncode, r.stderr)
     assert r.stdout.startswith("ok ")
+
+
+def test_status_codes_agree_between_header_binding_and_library():
+    # every fa_status enumerator of the header: its value, the binding's name for it, and a
+    # distinct description from fa_status_string
+    text = open(HEADER).read()
+    body = re.search(r"typedef enum \{(.*?)\} fa_status;", text, flags=re.S).group(1)
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    codes = {name: int(val) for name, val in re.findall(r"(FA_[A-Z_]+)\s*=\s*(-?\d+)", body)}
+    assert codes["FA_OK"] == 0 and len(codes) == len(set(codes.values()))
+    assert {v: k for k, v in codes.items()} == binding.STATUS_NAMES
+    texts = [binding.fa_status_string(v) for v in codes.values()]
+    assert len(set(texts)) == len(texts) and "unknown status" not in texts
