@@ -319,3 +319,28 @@ def test_status_codes_agree_between_header_binding_and_library():
     assert {v: k for k, v in codes.items()} == binding.STATUS_NAMES
     texts = [binding.fa_status_string(v) for v in codes.values()]
     assert len(set(texts)) == len(texts) and "unknown status" not in texts
+
+
+def _c_type(param):
+    """ctypes type a C parameter declaration is marshalled as."""
+    p = re.sub(r"\bconst\b", "", param).strip()
+    if "*" in p:
+        return ctypes.c_void_p
+    base = " ".join(p.split()[:-1])  # drop the parameter name
+    return {"int": ctypes.c_int, "float": ctypes.c_float, "size_t": ctypes.c_size_t,
+            "uint64_t": ctypes.c_uint64, "uint32_t": ctypes.c_uint32,
+            "unsigned int": ctypes.c_uint}[base]
+
+
+def test_binding_signatures_match_the_header():
+    # a wrong count or kind of argtypes would shift every later argument silently
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    protos = dict(re.findall(r"\b(fa_[a-z_0-9]+)\s*\(([^()]*)\)\s*;", text))
+    assert set(protos) == set(binding._SIGS)
+    for name, params in protos.items():
+        params = [] if params.strip() in ("", "void") else [q.strip() for q in params.split(",")]
+        want = [_c_type(q) for q in params]
+        got = binding._SIGS[name][1]
+        assert len(got) == len(want), name
+        for i, (g, w) in enumerate(zip(got, want)):
+            assert ctypes.sizeof(g) == ctypes.sizeof(w) and g._type_ == w._type_, (name, i)
