@@ -344,3 +344,14 @@ def test_binding_signatures_match_the_header():
         assert len(got) == len(want), name
         for i, (g, w) in enumerate(zip(got, want)):
             assert ctypes.sizeof(g) == ctypes.sizeof(w) and g._type_ == w._type_, (name, i)
+
+
+def test_binding_return_types_match_the_header():
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    rets = dict((n, r.strip()) for r, n in
+                re.findall(r"^\s*((?:const\s+)?[a-z_0-9]+\s*\**)\s*(fa_[a-z_0-9]+)\s*\(", text,
+                           flags=re.M))
+    kinds = {"int": ctypes.c_int, "size_t": ctypes.c_size_t, "const char*": ctypes.c_char_p}
+    assert set(rets) == set(binding._SIGS)
+    for name, ret in rets.items():
+        assert binding._SIGS[name][0] is kinds[re.sub(r"\s*\*", "*", ret)], name
