@@ -681,3 +681,17 @@ def test_forward_and_backward_match_torch_scaled_dot_product_attention(causal, k
     np.testing.assert_allclose(o, out.detach().numpy(), rtol=0, atol=1e-12)
     for name, mine, ref in (("dq", dq, tq.grad), ("dk", dk, tk.grad), ("dv", dv, tv.grad)):
         np.testing.assert_allclose(mine, ref.numpy(), rtol=0, atol=1e-11, err_msg=name)
+
+
+def test_results_do_not_depend_on_the_thread_count():
+    # each head runs on one thread, in one fixed order of additions
+    q, k, v, do = (rand((2, 3, 200, 16), 990 + i) for i in range(4))
+    kvl = np.array([150, 200], np.int32)
+    outs = []
+    for nt in (1, 2, 5):
+        o, lse = oracle.attention_forward(q, k, v, 0.3, causal=True, kv_len=kvl, nthreads=nt)
+        g = oracle.attention_backward(q, k, v, do, 0.3, causal=True, kv_len=kvl, nthreads=nt)
+        outs.append((o, lse) + tuple(g))
+    for other in outs[1:]:
+        for a, b in zip(outs[0], other):
+            assert np.array_equal(a, b)
