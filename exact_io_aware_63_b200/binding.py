@@ -10,7 +10,7 @@ torch tensors or None, the stream as a torch.cuda.Stream or None = current):
 ``fa_fwd``, ``fa_fwd_traced``, ``fa_bwd``, ``fa_bwd_traced``, ``fa_bwd_phase``,
 ``fa_bwd_deterministic``, ``fa_fwd_dropout``, ``fa_bwd_dropout``, ``fa_fwd_varlen``,
 ``fa_bwd_varlen``, ``fa_bwd_noalloc``, ``fa_bwd_workspace_size``,
-``fa_selftest_wait_timeout``, ``fa_get_device_status``, ``fa_status_string``,
+``fa_selftest_wait_timeout``, ``fa_selftest_ex2``, ``fa_get_device_status``, ``fa_status_string``,
 ``fa_version``.
 
 Convenience wrappers that allocate outputs: ``attention_forward`` and
@@ -55,6 +55,7 @@ _SIGS = {
     "fa_bwd_varlen": (_i, [_vp] * 10 + [_i, _i, _i, _i, _i, _f, _i, _f, _u64, _u32, _vp, _sz,
                                          _vp]),
     "fa_selftest_wait_timeout": (_i, [_i, ctypes.c_uint, _vp, _vp]),
+    "fa_selftest_ex2": (_i, [_vp, _vp, _i, _i, _vp]),
     "fa_get_device_status": (_i, [_vp]),
     "fa_status_string": (ctypes.c_char_p, [_i]),
     "fa_version": (_i, []),
@@ -228,6 +229,12 @@ def fa_selftest_wait_timeout(arrive, limit_us, result, stream=None):
     """One warp waits on a barrier for at most limit_us; see include/fa.h."""
     return load().fa_selftest_wait_timeout(int(arrive), int(limit_us), _ptr(result),
                                            _stream(stream, result))
+
+
+def fa_selftest_ex2(x, y, n, pair, stream=None):
+    """y[i] = the kernels' FMA-pipe 2^x[i] for i < n (float32 device arrays); see
+    include/fa.h."""
+    return load().fa_selftest_ex2(_ptr(x), _ptr(y), int(n), int(bool(pair)), _stream(stream, x))
 
 
 def fa_get_device_status(stream=None):

@@ -38,6 +38,25 @@ __global__ void __launch_bounds__(32, 1)
   if (threadIdx.x == 0) *result = ok ? 1 : 0;
 }
 
+// The FMA-pipe exponential of the softmax (ex2_poly, and ex2_poly2 on
+// pairs) evaluated element by element, for tests of its error bound.
+__global__ void __launch_bounds__(256) fa_selftest_ex2_kernel(const float* __restrict__ x,
+                                                              float* __restrict__ y, int n,
+                                                              int pair) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (pair) {
+    const int i0 = 2 * i, i1 = 2 * i + 1;
+    if (i0 >= n) return;
+    const float x0 = x[i0], x1 = (i1 < n) ? x[i1] : 0.f;
+    float y0, y1;
+    ex2_poly2(x0, x1, y0, y1);
+    y[i0] = y0;
+    if (i1 < n) y[i1] = y1;
+  } else if (i < n) {
+    y[i] = ex2_poly(x[i]);
+  }
+}
+
 }  // namespace fa
 
 namespace {
@@ -634,6 +653,18 @@ int fa_selftest_wait_timeout(int arrive, unsigned int limit_us, int* result, voi
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+int fa_selftest_ex2(const float* x, float* y, int n, int pair, void* stream) {
+  if (n < 0) return FA_ERR_SHAPE;
+  if (n == 0) return FA_OK;
+  if (!x || !y) return FA_ERR_NULL;
+  if (!aligned(x, 4) || !aligned(y, 4)) return FA_ERR_ALIGN;
+  const long long threads = pair ? (static_cast<long long>(n) + 1) / 2 : n;
+  const int blocks = static_cast<int>((threads + 255) / 256);
+  fa::fa_selftest_ex2_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      x, y, n, pair ? 1 : 0);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 int fa_fwd_varlen(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o, float* lse,
                   const int32_t* cu_seqlens, int B, int H, int max_seqlen, int total_tokens, int d,
                   float scale, int causal, float p_drop, uint64_t seed, uint32_t offset,
@@ -719,20 +750,52 @@ namespace {
 
 std::mutex g_noalloc_mutex;
 void* g_noalloc_ptr[kMaxDevices] = {};
+unsigned long long g_noalloc_ctx[kMaxDevices] = {};  // context the address belongs to
+
+// Process-unique id of the calling thread's current CUDA context (0 if the
+// driver cannot tell).  A device reset replaces the context, and with it the
+// module and the array's address; the new context has a new id.
+unsigned long long current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(ptr);
+    ptr = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(ptr);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx ||
+      get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
 
 // Device address of fa_bwd_noalloc_scratch on the current device `dev`, looked
-// up once per device and cached.  In host code the array's name is only a
+// up once per device (again only if the device's context has been replaced,
+// as by cudaDeviceReset) and cached.  In host code the array's name is only a
 // host-side handle, never a usable device address.
 int noalloc_scratch(int dev, void** out) {
   if (dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+  // the caller has made `dev` current with cudaSetDevice, which also binds its
+  // primary context to this thread
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> guard(g_noalloc_mutex);
-  if (!g_noalloc_ptr[dev]) {
+  if (!g_noalloc_ptr[dev] || ctx == 0 || ctx != g_noalloc_ctx[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, fa_bwd_noalloc_scratch) != cudaSuccess || !p) {
       cudaGetLastError();
       return FA_ERR_CUDA;
     }
     g_noalloc_ptr[dev] = p;
+    g_noalloc_ctx[dev] = ctx;
   }
   *out = g_noalloc_ptr[dev];
   return FA_OK;

@@ -9,8 +9,9 @@
  * Decoded", gloss of abstract sentence 4 and "The Hardware Picture").  For
  * every batch b and head h, with row r and key c:
  *
- *   allowed(r,c) = (!causal || c <= r) && (kv_len == NULL || c < kv_len[b])
+ *   allowed(r,c) = (!causal || c <= r) && (kv_len == NULL || c < L_b)
  *                  && (block_mask == NULL || block_mask[(r/128)*nt + c/128] != 0)
+ *   with L_b = kv_len[b] clamped into [0, N]
  *   S_rc  = scale * <Q_r, K_c>  (allowed), -inf (otherwise)
  *   P_rc  = exp(S_rc - LSE_r),  LSE_r = ln sum_c exp(S_rc)
  *   O_r   = sum_c P_rc V_c
@@ -272,6 +273,20 @@ int fa_bwd_varlen(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa
 int fa_selftest_wait_timeout(int arrive, unsigned int limit_us, int* result, void* stream);
 
 /*
+ * Self-test of the softmax's exponential on the FMA pipe.  Part of the
+ * exponentials 2^x of the forward and backward kernels are computed without
+ * the special-function unit: x = n + f with n = round(x) and |f| <= 1/2, 2^f
+ * as a degree-3 polynomial (the minimax fit for relative error, at most
+ * 7.5e-5), and n added to the result's exponent field; x below -126 is taken
+ * as -126.  This call writes y[i] = that function of x[i] for i < n
+ * (pair = 0: the one-value form; pair != 0: the two-value form the kernels
+ * run on packed pairs, which must give the same results).  x and y are
+ * float32 arrays in device memory, 4-byte aligned.  n < 0 gives
+ * FA_ERR_SHAPE; n = 0 does nothing.  Asynchronous on `stream`.
+ */
+int fa_selftest_ex2(const float* x, float* y, int n, int pair, void* stream);
+
+/*
  * Size in bytes of the library's built-in backward scratch buffer (64 MiB),
  * used only by fa_bwd_noalloc.
  */
@@ -295,7 +310,9 @@ int fa_selftest_wait_timeout(int arrive, unsigned int limit_us, int* result, voi
  *    B*H*N up to about 254K rows; with d = 128 about 129K rows.
  *  - The first call on each device looks up the array's device address
  *    (cudaGetSymbolAddress, with that device current) and caches it; make
- *    that first call before any stream capture.
+ *    that first call before any stream capture.  The cache is tied to the
+ *    device's context: after cudaDeviceReset the next call looks the address
+ *    up again (so make that call, too, outside a capture).
  *  - Every call on a device shares the one array.  Each call overwrites what
  *    it reads (the accumulator is zeroed by the call's first kernel), so the
  *    contents a previous call left behind do not matter, but calls whose

@@ -99,13 +99,13 @@ def _load():
                 ctypes.c_int, ctypes.c_int]
             lib.oracle_attention_forward_rows.argtypes = [
                 _dp, _i64p, ctypes.c_int, _dp, _dp, _dp, _dp, ctypes.c_int, ctypes.c_int,
-                ctypes.c_double, ctypes.c_int, _u8p, ctypes.c_int]
+                ctypes.c_double, ctypes.c_int, _u8p, ctypes.c_int, ctypes.c_int]
             lib.oracle_attention_backward_dq_rows.argtypes = [
                 _dp, _dp, _i64p, ctypes.c_int, _dp, _dp, _dp, _dp, ctypes.c_int, ctypes.c_int,
-                ctypes.c_double, ctypes.c_int, _u8p, ctypes.c_int]
+                ctypes.c_double, ctypes.c_int, _u8p, ctypes.c_int, ctypes.c_int]
             lib.oracle_attention_backward_kv_cols.argtypes = [
                 _dp, _dp, _dp, _dp, _i64p, ctypes.c_int, _dp, _dp, ctypes.c_int, ctypes.c_int,
-                ctypes.c_double, ctypes.c_int, _u8p, ctypes.c_int, ctypes.c_int]
+                ctypes.c_double, ctypes.c_int, _u8p, ctypes.c_int, ctypes.c_int, ctypes.c_int]
             lib.oracle_tile_visits.argtypes = [
                 _u8p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _u8p, _i32p,
                 ctypes.c_int, ctypes.c_int]
@@ -294,7 +294,7 @@ def attention_forward_rows(q_rows, rows, k, v, scale, causal=False, block_mask=N
     rc = _load().oracle_attention_forward_rows(
         _ptr(q_rows, _dp), _ptr(rows, _i64p), R, _ptr(k, _dp), _ptr(v, _dp), _ptr(o, _dp),
         _ptr(lse, _dp), N, d, float(scale), int(bool(causal)), _ptr(bm, _u8p),
-        -1 if kv_len_b is None else int(kv_len_b))
+        int(kv_len_b is not None), 0 if kv_len_b is None else int(kv_len_b))
     if rc != 0:
         raise RuntimeError(f"oracle_attention_forward_rows failed: {rc}")
     return o, lse
@@ -313,7 +313,7 @@ def attention_backward_dq_rows(q_rows, dout_rows, rows, k, v, scale, causal=Fals
     rc = _load().oracle_attention_backward_dq_rows(
         _ptr(q_rows, _dp), _ptr(dout_rows, _dp), _ptr(rows, _i64p), R, _ptr(k, _dp),
         _ptr(v, _dp), _ptr(dq, _dp), _ptr(delta, _dp), N, d, float(scale), int(bool(causal)),
-        _ptr(bm, _u8p), -1 if kv_len_b is None else int(kv_len_b))
+        _ptr(bm, _u8p), int(kv_len_b is not None), 0 if kv_len_b is None else int(kv_len_b))
     if rc != 0:
         raise RuntimeError(f"oracle_attention_backward_dq_rows failed: {rc}")
     return dq, delta
@@ -332,7 +332,7 @@ def attention_backward_kv_cols(q, k, v, dout, cols, scale, causal=False, block_m
     rc = _load().oracle_attention_backward_kv_cols(
         _ptr(q, _dp), _ptr(k, _dp), _ptr(v, _dp), _ptr(dout, _dp), _ptr(cols, _i64p), C,
         _ptr(dk, _dp), _ptr(dv, _dp), N, d, float(scale), int(bool(causal)), _ptr(bm, _u8p),
-        -1 if kv_len_b is None else int(kv_len_b), _threads(nthreads))
+        int(kv_len_b is not None), 0 if kv_len_b is None else int(kv_len_b), _threads(nthreads))
     if rc != 0:
         raise RuntimeError(f"oracle_attention_backward_kv_cols failed: {rc}")
     return dk, dv

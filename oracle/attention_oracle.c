@@ -13,9 +13,10 @@
  * oracle is therefore the plain definition of standard attention, written
  * out one query row at a time:
  *
- *   M(r,c) = (!causal || c <= r) && (kv_len == NULL || c < kv_len[b])
+ *   M(r,c) = (!causal || c <= r) && (kv_len == NULL || c < L_b)
  *            && (block_mask == NULL || block_mask[(r/128)*nt + c/128] != 0)
- *            with nt = ceil(N / 128) (a last, partial tile holds the rest)
+ *            with L_b = kv_len[b] clamped into [0, N] and nt = ceil(N / 128)
+ *            (a last, partial tile holds the rest)
  *   S_rc   = scale * sum_k Q_rk K_ck          if M(r,c), else -inf
  *   m_r    = max_c S_rc,  l_r = sum_c exp(S_rc - m_r)
  *   P_rc   = exp(S_rc - m_r) / l_r,  LSE_r = m_r + ln l_r  (natural log)
@@ -110,11 +111,23 @@ static double dropout_weight(const oracle_job *job, int bh, int r, int c)
     return u >= job->drop_t ? job->drop_scale : 0.0;
 }
 
-/* The mask M(r,c) exactly as defined above. */
+/*
+ * Key limit L_b of the mask: keys c >= L_b are padding.  Without key lengths
+ * every key is allowed (L_b = N); a given length is taken clamped into
+ * [0, N], so a negative one allows no key and one above N allows them all
+ * (the contract of the library's kv_len argument).
+ */
+static int key_limit(int has_kv_len, int kv_len_b, int N)
+{
+    if (!has_kv_len) return N;
+    return kv_len_b < 0 ? 0 : (kv_len_b > N ? N : kv_len_b);
+}
+
+/* The mask M(r,c) exactly as defined above, with L = key_limit(...). */
 static int allowed(int r, int c, int N, int causal, const uint8_t *block_mask, int L)
 {
     if (causal && c > r) return 0;
-    if (L >= 0 && c >= L) return 0;
+    if (c >= L) return 0;
     if (block_mask) {
         /* nt = ceil(N / 128): a last, partial tile holds the remaining positions */
         int nt = (N + ORACLE_MASK_TILE - 1) / ORACLE_MASK_TILE;
@@ -167,7 +180,7 @@ static void forward_head(const oracle_job *job, int bh, double *p)
     const double *Q = job->q + off, *K = job->k + off, *V = job->v + off;
     double *O = job->o + off;
     double *lse = job->lse + (size_t)bh * N;
-    const int L = job->kv_len ? job->kv_len[b] : -1;
+    const int L = key_limit(job->kv_len != NULL, job->kv_len ? job->kv_len[b] : 0, N);
     for (int r = job->r_begin; r < job->r_end; ++r) {
         double m, l;
         int count = softmax_row(Q + (size_t)r * d, r, K, N, d, job->scale, job->causal,
@@ -195,7 +208,7 @@ static void backward_head(const oracle_job *job, int bh, double *p, double *dp)
     const size_t off = (size_t)bh * N * d;
     const double *Q = job->q + off, *K = job->k + off, *V = job->v + off, *dO = job->dout + off;
     double *dQ = job->dq + off, *dK = job->dk + off, *dV = job->dv + off;
-    const int L = job->kv_len ? job->kv_len[b] : -1;
+    const int L = key_limit(job->kv_len != NULL, job->kv_len ? job->kv_len[b] : 0, N);
     memset(dK, 0, sizeof(double) * (size_t)N * d);
     memset(dV, 0, sizeof(double) * (size_t)N * d);
     for (int r = job->r_begin; r < job->r_end; ++r) {
@@ -426,23 +439,25 @@ void oracle_philox4x32_10(const uint32_t counter[4], uint32_t k0, uint32_t k1, u
 /*
  * Forward for a chosen subset of query rows of ONE head.  q_rows is
  * [R][d] (row i holds query number rows[i]); K and V are the head's full
- * [N][d]; kv_len_b < 0 means no key padding.  Used to check sampled rows at
+ * [N][d]; has_kv_len = 0 means no key padding, else keys c >= kv_len_b
+ * (clamped into [0, N], see key_limit) are padding.  Used to check sampled rows at
  * sizes where the whole head is too slow on the CPU; each row is the same
  * computation as in oracle_attention_forward.
  */
 int oracle_attention_forward_rows(const double *q_rows, const int64_t *rows, int R,
                                   const double *k, const double *v, double *o_rows,
                                   double *lse_rows, int N, int d, double scale, int causal,
-                                  const uint8_t *block_mask, int kv_len_b)
+                                  const uint8_t *block_mask, int has_kv_len, int kv_len_b)
 {
     if (R < 0 || N <= 0 || d <= 0) return -3;
+    const int L = key_limit(has_kv_len, kv_len_b, N);
     double *p = (double *)malloc(sizeof(double) * (size_t)N);
     if (!p) return -6;
     for (int i = 0; i < R; ++i) {
         const int r = (int)rows[i];
         double m, l;
         int count = softmax_row(q_rows + (size_t)i * d, r, k, N, d, scale, causal, block_mask,
-                                kv_len_b, p, &m, &l);
+                                L, p, &m, &l);
         double *orow = o_rows + (size_t)i * d;
         for (int x = 0; x < d; ++x) orow[x] = 0.0;
         if (count == 0) { lse_rows[i] = -INFINITY; continue; }
@@ -467,9 +482,10 @@ int oracle_attention_backward_dq_rows(const double *q_rows, const double *dout_r
                                       const int64_t *rows, int R, const double *k,
                                       const double *v, double *dq_rows, double *delta_rows,
                                       int N, int d, double scale, int causal,
-                                      const uint8_t *block_mask, int kv_len_b)
+                                      const uint8_t *block_mask, int has_kv_len, int kv_len_b)
 {
     if (R < 0 || N <= 0 || d <= 0) return -3;
+    const int L = key_limit(has_kv_len, kv_len_b, N);
     double *p = (double *)malloc(sizeof(double) * (size_t)N);
     double *dp = (double *)malloc(sizeof(double) * (size_t)N);
     if (!p || !dp) { free(p); free(dp); return -6; }
@@ -479,7 +495,7 @@ int oracle_attention_backward_dq_rows(const double *q_rows, const double *dout_r
         const double *dor = dout_rows + (size_t)i * d;
         double *dqr = dq_rows + (size_t)i * d;
         double m, l;
-        int count = softmax_row(qr, r, k, N, d, scale, causal, block_mask, kv_len_b, p, &m, &l);
+        int count = softmax_row(qr, r, k, N, d, scale, causal, block_mask, L, p, &m, &l);
         for (int x = 0; x < d; ++x) dqr[x] = 0.0;
         delta_rows[i] = 0.0;
         if (count == 0) continue;
@@ -582,7 +598,7 @@ int oracle_attention_backward_kv_cols(const double *q, const double *k, const do
                                       const double *dout, const int64_t *cols, int C,
                                       double *dk_cols, double *dv_cols, int N, int d,
                                       double scale, int causal, const uint8_t *block_mask,
-                                      int kv_len_b, int nthreads)
+                                      int has_kv_len, int kv_len_b, int nthreads)
 {
     if (C < 0 || N <= 0 || d <= 0) return -3;
     for (int i = 0; i < C; ++i)
@@ -591,7 +607,7 @@ int oracle_attention_backward_kv_cols(const double *q, const double *k, const do
     memset(&job, 0, sizeof(job));
     job.q = q; job.k = k; job.v = v; job.dout = dout; job.cols = cols; job.C = C;
     job.N = N; job.d = d; job.scale = scale; job.causal = causal;
-    job.block_mask = block_mask; job.L = kv_len_b;
+    job.block_mask = block_mask; job.L = key_limit(has_kv_len, kv_len_b, N);
     job.nchunks = (N + KVCOLS_CHUNK - 1) / KVCOLS_CHUNK;
     job.partial = (double *)malloc(sizeof(double) * (size_t)job.nchunks * 2 * C * d + 1);
     if (!job.partial) return -6;
@@ -644,7 +660,7 @@ int oracle_tile_visits(uint8_t *visits, int B, int N, int T, int causal,
     if (i_begin < 0 || i_end > nt || i_begin > i_end) return -3;
     const int ni = i_end - i_begin;
     for (int b = 0; b < B; ++b) {
-        const int L = kv_len ? kv_len[b] : -1;
+        const int L = key_limit(kv_len != NULL, kv_len ? kv_len[b] : 0, N);
         for (int i = i_begin; i < i_end; ++i)
             for (int j = 0; j < nt; ++j) {
                 int any = 0;

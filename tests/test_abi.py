@@ -24,7 +24,7 @@ def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ["fa_fwd", "fa_fwd_traced", "fa_bwd", "fa_bwd_traced", "fa_bwd_phase",
               "fa_bwd_deterministic", "fa_fwd_dropout", "fa_bwd_dropout",
-              "fa_selftest_wait_timeout", "fa_fwd_varlen", "fa_bwd_varlen",
+              "fa_selftest_wait_timeout", "fa_selftest_ex2", "fa_fwd_varlen", "fa_bwd_varlen",
               "fa_bwd_workspace_size",
               "fa_get_device_status", "fa_status_string", "fa_version"]:
         assert n in names
@@ -198,6 +198,10 @@ def test_selftest_arguments_are_checked():
     assert lib.fa_selftest_wait_timeout(0, 1000, P + 2, None) == -2
     assert lib.fa_selftest_wait_timeout(0, 0, P, None) == -8
     assert lib.fa_selftest_wait_timeout(0, 2_000_001, P, None) == -8
+    assert lib.fa_selftest_ex2(P, P, -1, 0, None) == -3
+    assert lib.fa_selftest_ex2(None, None, 0, 0, None) == 0
+    assert lib.fa_selftest_ex2(None, P, 8, 1, None) == -1
+    assert lib.fa_selftest_ex2(P + 2, P, 8, 0, None) == -2
 
 
 def fwd_varlen(**kw):

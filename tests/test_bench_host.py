@@ -129,10 +129,30 @@ def test_reference_arm_runs_on_rank_zero_only():
 
 def test_gpu_count_must_match_the_launched_processes():
     import subprocess
+    env = dict(os.environ)
+    env.update({"WORLD_SIZE": "2", "RANK": "0"})
     r = subprocess.run([sys.executable, os.path.join(os.path.dirname(bench.__file__), "bench.py"),
-                        "--gpus", "2", "--steps", "1"], capture_output=True, text=True, timeout=120,
-                       env={k: v for k, v in os.environ.items() if k != "WORLD_SIZE"})
+                        "--gpus", "3", "--steps", "1"], capture_output=True, text=True, timeout=120,
+                       env=env)
     assert r.returncode != 0 and "one process per GPU" in r.stderr
+
+
+def test_gpus_without_a_launcher_start_one_rank_per_gpu():
+    # `--gpus 2` run as a plain command starts two ranks itself (torch.distributed.run,
+    # rendezvous on 127.0.0.1); the reference arm then runs on rank 0 alone and prints
+    # one line for the two-process job
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    import json
+    import subprocess
+    r = subprocess.run([sys.executable, os.path.join(os.path.dirname(bench.__file__), "bench.py"),
+                        "--gpus", "2", "--impl", "reference", "--shape", "1,1,128,64",
+                        "--steps", "1", "--warmup", "1"],
+                       capture_output=True, text=True, timeout=300, env=env)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(l) for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    assert lines[0]["impl"] == "reference" and lines[0]["n_gpus"] == 2
 
 
 def test_traffic_is_reported_only_for_the_sources_it_was_taken_on(tmp_path, monkeypatch):

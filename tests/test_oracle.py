@@ -235,6 +235,49 @@ def test_fully_masked_rows():
     assert np.all(np.isfinite(dk)) and np.all(np.isfinite(dv))
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_key_lengths_outside_zero_to_n_are_clamped(causal):
+    # The library's contract for kv_len: values are taken clamped into [0, N], so a
+    # negative length (or 0) leaves a batch with no key at all, and a length above N
+    # masks nothing.  Batch 0: kv_len = -3, batch 1: N + 5, batch 2: 0.
+    B, H, N, d = 3, 2, 200, 8
+    q, k, v, do = (rand((B, H, N, d), s) for s in (61, 62, 63, 64))
+    kvl = np.array([-3, N + 5, 0], np.int32)
+    o, lse = oracle.attention_forward(q, k, v, 0.3, causal=causal, kv_len=kvl)
+    dq, dk, dv, _ = oracle.attention_backward(q, k, v, do, 0.3, causal=causal, kv_len=kvl)
+    for b in (0, 2):  # no allowed key: the empty-row definition
+        assert np.all(o[b] == 0) and np.all(np.isneginf(lse[b]))
+        assert np.all(dq[b] == 0) and np.all(dk[b] == 0) and np.all(dv[b] == 0)
+    # batch 1 sees every key: the same values as without key lengths (Q = 0 closed form
+    # for the forward, and the unpadded call for the backward)
+    o0, lse0 = oracle.attention_forward(np.zeros_like(q[1:2]), k[1:2], v[1:2], 0.3,
+                                        causal=causal, kv_len=np.array([N + 5], np.int32))
+    for r in (0, 57, 199):
+        cnt = r + 1 if causal else N
+        np.testing.assert_allclose(o0[0, :, r], v[1, :, :cnt].mean(axis=1), atol=1e-13)
+        assert np.all(np.abs(lse0[0, :, r] - math.log(cnt)) < 1e-13)
+    o1, lse1 = oracle.attention_forward(q[1:2], k[1:2], v[1:2], 0.3, causal=causal)
+    dq1, dk1, dv1, _ = oracle.attention_backward(q[1:2], k[1:2], v[1:2], do[1:2], 0.3,
+                                                 causal=causal)
+    assert np.array_equal(o[1], o1[0]) and np.array_equal(lse[1], lse1[0])
+    assert np.array_equal(dq[1], dq1[0]) and np.array_equal(dk[1], dk1[0])
+    assert np.array_equal(dv[1], dv1[0])
+    # the one-head row and column functions follow the same rule
+    rows = np.array([0, 99, 199])
+    for kv_b, b in ((-3, 0), (N + 5, 1), (0, 2)):
+        orow, lrow = oracle.attention_forward_rows(q[b, 0, rows], rows, k[b, 0], v[b, 0], 0.3,
+                                                   causal=causal, kv_len_b=kv_b)
+        np.testing.assert_array_equal(orow, o[b, 0, rows])
+        np.testing.assert_array_equal(lrow, lse[b, 0, rows])
+        dqr, _ = oracle.attention_backward_dq_rows(q[b, 0, rows], do[b, 0, rows], rows, k[b, 0],
+                                                   v[b, 0], 0.3, causal=causal, kv_len_b=kv_b)
+        np.testing.assert_allclose(dqr, dq[b, 0, rows], rtol=0, atol=1e-12)
+        dkc, dvc = oracle.attention_backward_kv_cols(q[b, 0], k[b, 0], v[b, 0], do[b, 0], rows,
+                                                     0.3, causal=causal, kv_len_b=kv_b)
+        np.testing.assert_allclose(dkc, dk[b, 0, rows], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(dvc, dv[b, 0, rows], rtol=0, atol=1e-12)
+
+
 # ---------------------------------------------------------------------------
 # brute force: finite differences of L = sum(O * dO)
 # ---------------------------------------------------------------------------

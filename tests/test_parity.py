@@ -75,6 +75,20 @@ def test_rows_without_keys(cuda_device, d):
 
 
 @pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_key_lengths_outside_zero_to_n(cuda_device, d, causal):
+    # kv_len values are taken clamped into [0, N]: -3 leaves batch 0 without keys,
+    # N + 5 masks nothing in batch 1; the oracle follows the same contract
+    N = 384
+    x = inputs.make_inputs(2, 2, N, d, causal=causal, seed=31 + d + int(causal),
+                           kv_len=torch.tensor([-3, N + 5], dtype=torch.int32))
+    res, out = check_all_heads(x)
+    assert np.all(f64(out["o"])[0] == 0) and np.all(np.isneginf(f64(out["lse"])[0]))
+    for name in ("dq", "dk", "dv"):
+        assert np.all(f64(out[name])[0] == 0), name
+
+
+@pytest.mark.parametrize("d", [64, 128])
 def test_padded_keys_get_zero_gradients(cuda_device, d):
     x = inputs.make_inputs(2, 2, 512, d, seed=19 + d,
                            kv_len=torch.tensor([200, 333], dtype=torch.int32))

@@ -11,11 +11,18 @@ that shapes too large for the buffer are refused before anything runs.
 This file is named to be collected last.
 """
 
+import numpy as np
 import pytest
 import torch
 
+import oracle
 from exact_io_aware_63_b200 import binding, inputs
-from gpu_helpers import GRAD_TOL, rel_l2, f64, to_dev
+from gpu_helpers import compare_grads, f64, head_slices, rel_l2, to_dev
+
+# dK and dV come from the same kernels on the same inputs, each row accumulated by one
+# CTA in a fixed order: the same bits.  dQ is summed by reduce-adds whose order varies
+# from run to run: equal up to float32 reordering, far inside this bound.
+DQ_TOL = 2e-3
 
 
 def test_refuses_shapes_beyond_the_static_buffer():
@@ -53,6 +60,15 @@ def test_matches_fa_bwd_on_two_calls_in_a_row(cuda_device, name, shape, causal, 
         assert rc == 0, binding.fa_status_string(rc)
         torch.cuda.synchronize()
         assert binding.fa_get_device_status() == 0
-        for got, want, nm in zip((dq, dk, dv), ref, ("dq", "dk", "dv")):
-            e = rel_l2(f64(got), f64(want))
-            assert e <= GRAD_TOL, f"{name} call {call}: {nm} rel-L2 {e:.3e} vs fa_bwd"
+        assert torch.equal(dk, ref[1]), f"{name} call {call}: dK differs from fa_bwd's"
+        assert torch.equal(dv, ref[2]), f"{name} call {call}: dV differs from fa_bwd's"
+        e = rel_l2(f64(dq), f64(ref[0]))
+        assert e <= DQ_TOL, f"{name} call {call}: dQ rel-L2 {e:.3e} vs fa_bwd"
+    if shape is not None:
+        # the last call's gradients against the FP64 oracle, every head
+        heads = [(b, h) for b in range(B) for h in range(H)]
+        hq, hk, hv, hdo, hbm, hkl = head_slices(x, heads)
+        rdq, rdk, rdv, _ = oracle.attention_backward(hq, hk, hv, hdo, x.scale, x.causal, hbm, hkl)
+        pick = lambda t: np.stack([f64(t[b, h]) for b, h in heads])[:, None]
+        compare_grads({"dq": pick(dq), "dk": pick(dk), "dv": pick(dv)},
+                      {"dq": rdq, "dk": rdk, "dv": rdv}, f"{name} vs oracle")
