@@ -14,6 +14,7 @@
 #include "fa.h"
 #include "fa_bwd.cuh"
 #include "fa_bwd_det.cuh"
+#include "fa_d256.cuh"
 #include "fa_fwd.cuh"
 
 namespace fa {
@@ -84,13 +85,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // head, z = head), boxes of 128 rows x 64 columns, 128-byte swizzle.  Rows of
 // a box beyond N are zero-filled on loads and dropped on stores, so a partial
 // last tile never touches the next head.
-bool make_tmap(CUtensorMap* m, const void* base, int BH, int N, int d) {
+// box_rows = 32 gives the row-chunk boxes of the head-dimension-256 kernels.
+bool make_tmap(CUtensorMap* m, const void* base, int BH, int N, int d, int box_rows = 128) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
                         static_cast<cuuint64_t>(BH)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -183,9 +185,10 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 // Shape checks shared by every entry point.  Returns FA_OK, an error, or 1
 // for "empty problem: nothing to do".
-// Head dimensions: 64 and 128 natively; 32 and 96 run on the 64 / 128 kernels,
-// whose tensor maps read the missing columns as zeros and whose stores stop at d.
-bool supported_d(int d) { return d == 32 || d == 64 || d == 96 || d == 128; }
+// Head dimensions: 64, 128 and 256 natively; 32 and 96 run on the 64 / 128
+// kernels, whose tensor maps read the missing columns as zeros and whose stores
+// stop at d.
+bool supported_d(int d) { return d == 32 || d == 64 || d == 96 || d == 128 || d == 256; }
 
 int check_shape(int B, int H, int N, int d) {
   if (B < 0 || H < 0 || N < 0) return FA_ERR_SHAPE;
@@ -255,11 +258,16 @@ bool ensure_smem(Kernel k, int bytes, std::atomic<bool> (&done)[kMaxDevices]) {
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Heads per work-unit group: as many as keep `bytes_per_head` of re-read data
-// within a 48 MB share of the 126 MB L2.
+// within a 48 MB share of the 126 MB L2, with the heads spread evenly over the
+// groups (16 heads in groups of at most 5 become four groups of 4, not 5, 5,
+// 5, 1): a last group of few heads would leave its few longest units running
+// alone at the end of the launch.
 int heads_per_group(int BH, double bytes_per_head) {
   const double budget = 48.0 * 1024 * 1024;
   int g = static_cast<int>(budget / bytes_per_head);
-  return g < 1 ? 1 : (g > BH ? BH : g);
+  g = g < 1 ? 1 : (g > BH ? BH : g);
+  const int groups = (BH + g - 1) / g;
+  return (BH + groups - 1) / groups;
 }
 
 struct WsLayout {
@@ -276,7 +284,9 @@ WsLayout ws_layout(int B, int H, int N, int d) {
   w.delta = 0;
   w.lse2 = round_up(w.delta + 4 * Rp, 256);
   w.dq_acc = round_up(w.lse2 + 4 * Rp, 256);
-  w.counter = round_up(w.dq_acc + 4 * R * d, 256);
+  // head dimension 256 sums dQ on chip (no float32 accumulator in memory)
+  const size_t acc_bytes = (d == 256) ? 0 : 4 * R * d;
+  w.counter = round_up(w.dq_acc + acc_bytes, 256);
   w.total = w.counter + 256;
   return w;
 }
@@ -357,6 +367,10 @@ int launch_fwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o,
   p.heads_per_group = heads_per_group(B * H, 4.0 * N * d);  // K and V
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * fa::kLog2e;
+  // the launch's work counter: slots are handed out in turn (see g_fwd_work)
+  static std::atomic<unsigned int> ticket{0};
+  p.counter_slot = static_cast<int>(ticket.fetch_add(1u, std::memory_order_relaxed) %
+                                    static_cast<unsigned int>(fa::kFwdCounterSlots));
   set_drop(p, dr);
   if (pk.cu) {  // packed batches have no block mask: pair mode
     if (dr.on) return launch_fwd_mode<D, true, true, true>(tq, tk, tv, to, p, stream, num_sms);
@@ -495,6 +509,7 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
     sp.heads_per_group = heads_per_group(B * H, 4.0 * N * D);  // K and V
     sp.causal = causal ? 1 : 0;
     sp.scale_log2 = scale * fa::kLog2e;
+    sp.counter_slot = 0;  // the ordered dQ kernel deals its units statically
     dp.delta = delta;
     dp.lse2 = lse2;
     dp.dq = dq;
@@ -507,6 +522,137 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
   return FA_OK;
 }
 
+// Head dimension 256: one query tile per unit (see fa_d256.cuh).
+int launch_fwd256(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o, float* lse,
+                  int B, int H, int N, float scale, int causal, const uint8_t* block_mask,
+                  const int32_t* kv_len, uint8_t* visited, cudaStream_t stream, int num_sms) {
+  using Cfg = fa::Fwd256Cfg;
+  const int BH = B * H;
+  CUtensorMap tq, tk, tv, to;
+  if (!make_tmap(&tq, q, BH, N, 256) || !make_tmap(&tk, k, BH, N, 256) ||
+      !make_tmap(&tv, v, BH, N, 256, 32) || !make_tmap(&to, o, BH, N, 256))
+    return FA_ERR_CUDA;
+  fa::FwdParams p = {};
+  p.o = o;
+  p.lse = lse;
+  p.block_mask = block_mask;
+  p.kv_len = kv_len;
+  p.visited = visited;
+  p.o_stride = 256;
+  p.dcols = 256;
+  p.B = B;
+  p.H = H;
+  p.N = N;
+  p.n_t = (N + fa::kTile - 1) / fa::kTile;
+  p.num_units = BH * p.n_t;
+  p.heads_per_group = heads_per_group(BH, 4.0 * N * 256);  // K and V
+  p.causal = causal ? 1 : 0;
+  p.scale_log2 = scale * fa::kLog2e;
+  static std::atomic<bool> smem_done[kMaxDevices];
+  if (!ensure_smem(fa::fa_fwd256_kernel<false>, Cfg::kSmemBytes, smem_done)) return FA_ERR_CUDA;
+  const int grid = p.num_units < num_sms ? p.num_units : num_sms;
+  return launch_pdl(fa::fa_fwd256_kernel<false>, dim3(grid), dim3(Cfg::kThreads), Cfg::kSmemBytes,
+                    stream, tq, tk, tv, to, p) == cudaSuccess
+             ? FA_OK
+             : FA_ERR_CUDA;
+}
+
+// Head dimension 256 backward: preprocess (phase 0), the dK and dV passes
+// (phase 1), the dQ pass (phase 2, and phase 3: it is already ordered).
+int launch_bwd256(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf16* o,
+                  const float* lse, const fa_bf16* dout, fa_bf16* dq, fa_bf16* dk, fa_bf16* dv,
+                  int B, int H, int N, float scale, int causal, const uint8_t* block_mask,
+                  const int32_t* kv_len, void* workspace, uint8_t* visited, cudaStream_t stream,
+                  int num_sms, unsigned phases) {
+  using Cfg = fa::Bwd256Cfg;
+  constexpr int d = 256;
+  const int BH = B * H;
+  const WsLayout wl = ws_layout(B, H, N, d);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* delta = reinterpret_cast<float*>(ws + wl.delta);
+  float* lse2 = reinterpret_cast<float*>(ws + wl.lse2);
+  int* counter = reinterpret_cast<int*>(ws + wl.counter);
+  const int n_t = (N + fa::kTile - 1) / fa::kTile;
+  if (phases & 1u) {
+    const int threads = 256;
+    const long long rows_p = static_cast<long long>(BH) * n_t * fa::kTile;
+    long long blocks = (rows_p * (d / 4) + threads - 1) / threads;
+    const long long cap = static_cast<long long>(num_sms) * 8;
+    if (blocks > cap) blocks = cap;
+    // no dQ accumulator to zero (rows = 0)
+    if (launch_pdl(fa::fa_bwd_pre_kernel<256>, dim3(static_cast<int>(blocks)), dim3(threads), 0,
+                   stream, o, dout, lse, delta, lse2, static_cast<float4*>(nullptr), counter, N,
+                   n_t * fa::kTile, rows_p, 0ll, d) != cudaSuccess)
+      return FA_ERR_CUDA;
+  }
+  if (!(phases & 14u)) return FA_OK;
+  CUtensorMap tq, tk, tv, tdo, tq32, tk32, tdo32, tdq, tdk, tdv;
+  if (!make_tmap(&tq, q, BH, N, d) || !make_tmap(&tk, k, BH, N, d) ||
+      !make_tmap(&tv, v, BH, N, d) || !make_tmap(&tdo, dout, BH, N, d) ||
+      !make_tmap(&tq32, q, BH, N, d, 32) || !make_tmap(&tk32, k, BH, N, d, 32) ||
+      !make_tmap(&tdo32, dout, BH, N, d, 32) || !make_tmap(&tdq, dq, BH, N, d) ||
+      !make_tmap(&tdk, dk, BH, N, d) || !make_tmap(&tdv, dv, BH, N, d))
+    return FA_ERR_CUDA;
+  fa::Bwd256Params bp = {};
+  fa::FwdParams& pq = bp.q;
+  pq.block_mask = block_mask;
+  pq.kv_len = kv_len;
+  pq.visited = visited;
+  pq.o_stride = d;
+  pq.dcols = d;
+  pq.B = B;
+  pq.H = H;
+  pq.N = N;
+  pq.n_t = n_t;
+  pq.num_units = BH * n_t;
+  pq.heads_per_group = heads_per_group(BH, 4.0 * N * d);  // K and V
+  pq.causal = causal ? 1 : 0;
+  pq.scale_log2 = scale * fa::kLog2e;
+  fa::BwdParams& pk = bp.k;
+  pk.delta = delta;
+  pk.lse2 = lse2;
+  pk.dk = dk;
+  pk.dv = dv;
+  pk.block_mask = block_mask;
+  pk.kv_len = kv_len;
+  pk.visited = visited;
+  pk.o_stride = d;
+  pk.dcols = d;
+  pk.B = B;
+  pk.H = H;
+  pk.N = N;
+  pk.n_t = n_t;
+  pk.num_units = BH * n_t;
+  pk.heads_per_group = heads_per_group(BH, 4.0 * N * d);  // Q and dO
+  pk.work_counter = counter;
+  pk.causal = causal ? 1 : 0;
+  pk.scale = scale;
+  pk.scale_log2 = scale * fa::kLog2e;
+  bp.dq = dq;
+  static std::atomic<bool> smem_done[3][kMaxDevices];
+  if (!ensure_smem(fa::fa_bwd256_kernel<fa::kPassDQ>, Cfg::kSmemBytes, smem_done[0]) ||
+      !ensure_smem(fa::fa_bwd256_kernel<fa::kPassDK>, Cfg::kSmemBytes, smem_done[1]) ||
+      !ensure_smem(fa::fa_bwd256_kernel<fa::kPassDV>, Cfg::kSmemBytes, smem_done[2]))
+    return FA_ERR_CUDA;
+  const int grid = pk.num_units < num_sms ? pk.num_units : num_sms;
+  if (phases & 2u) {
+    if (launch_pdl(fa::fa_bwd256_kernel<fa::kPassDK>, dim3(grid), dim3(Cfg::kThreads),
+                   Cfg::kSmemBytes, stream, tq, tk, tv, tdo, tq32, tk32, tdo32, tdk, bp) !=
+            cudaSuccess ||
+        launch_pdl(fa::fa_bwd256_kernel<fa::kPassDV>, dim3(grid), dim3(Cfg::kThreads),
+                   Cfg::kSmemBytes, stream, tq, tk, tv, tdo, tq32, tk32, tdo32, tdv, bp) !=
+            cudaSuccess)
+      return FA_ERR_CUDA;
+  }
+  if (phases & 12u) {
+    if (launch_pdl(fa::fa_bwd256_kernel<fa::kPassDQ>, dim3(grid), dim3(Cfg::kThreads),
+                   Cfg::kSmemBytes, stream, tq, tk, tv, tdo, tq32, tk32, tdo32, tdq, bp) !=
+        cudaSuccess)
+      return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+
 int fwd_impl(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o, float* lse, int B,
              int H, int N, int d, float scale, int causal, const uint8_t* block_mask,
              const int32_t* kv_len, uint8_t* visited, void* stream,
@@ -514,6 +660,7 @@ int fwd_impl(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o, f
   int rc = check_shape(B, H, N, d);
   if (rc == 1) return FA_OK;
   if (rc != FA_OK) return rc;
+  if (d == 256 && (dr.on || pk.cu)) return FA_ERR_UNSUPPORTED_D;  // no dropout / packed form
   if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
     return FA_ERR_ALIGN;
@@ -523,6 +670,9 @@ int fwd_impl(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16* o, f
   const int sms = select_device(q);
   if (sms <= 0) return FA_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 256)
+    return launch_fwd256(q, k, v, o, lse, B, H, N, scale, causal, block_mask, kv_len, visited, s,
+                         sms);
   if (d <= 64)
     return launch_fwd<64>(q, k, v, o, lse, B, H, N, d, scale, causal, block_mask, kv_len, visited,
                           s, sms, dr, pk);
@@ -539,7 +689,8 @@ int bwd_impl(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf16
   int rc = check_shape(B, H, N, d);
   if (rc == 1) return FA_OK;
   if (rc != FA_OK) return rc;
-  if ((phases & 8u) && d != 64 && d != 128) return FA_ERR_UNSUPPORTED_D;  // ordered dQ
+  if ((phases & 8u) && d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED_D;  // ordered dQ
+  if (d == 256 && (dr.on || pk.cu)) return FA_ERR_UNSUPPORTED_D;  // no dropout / packed form
   if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA_ERR_NULL;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
       !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
@@ -553,6 +704,9 @@ int bwd_impl(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf16
   const int sms = select_device(q);
   if (sms <= 0) return FA_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 256)
+    return launch_bwd256(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, scale, causal, block_mask,
+                         kv_len, workspace, visited, s, sms, phases);
   if (d <= 64)
     return launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal,
                           block_mask, kv_len, workspace, visited, s, sms, phases, dr, pk);
@@ -721,7 +875,8 @@ const char* fa_status_string(int status) {
     case FA_ERR_ALIGN: return "a pointer is not aligned as required";
     case FA_ERR_SHAPE: return "unsupported shape (negative size, or B*H*N >= 2^31)";
     case FA_ERR_UNSUPPORTED_D:
-      return "head dimension d must be 32, 64, 96 or 128 (64 or 128 for the ordered dQ)";
+      return "head dimension d must be 32, 64, 96, 128 or 256 (64, 128 or 256 for the ordered "
+             "dQ; 256 has no dropout or packed form)";
     case FA_ERR_WORKSPACE: return "workspace missing or smaller than fa_bwd_workspace_size()";
     case FA_ERR_CUDA: return "a CUDA runtime or driver call failed";
     case FA_ERR_TIMEOUT: return "a device pipeline wait timed out; outputs are incomplete";

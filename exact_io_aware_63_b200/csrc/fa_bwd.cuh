@@ -676,11 +676,12 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         ++kv_cnt;
         if (!ok) break;
         // Per query tile t the issue order is
-        //   dV(t) | S^T(t+1) dK(t) dQ(t) dP^T(t+1)
-        // so that the P phase of tile t+1 overlaps the dK / dQ MMAs of tile t:
-        // S^T's columns are free once dS(t) is ready (its P^T has been read by
-        // the dV MMA and by the dS warps), and dP^T(t+1) follows dK(t), which
-        // reads dS^T(t) from the dP^T columns.
+        //   dV(t) S^T(t+1) | dK(t) dQ(t) dP^T(t+1)
+        // S^T's columns are free once the dV MMA has read P^T(t) from them (the
+        // math warps keep their own copy of P in registers for dS), so S^T(t+1)
+        // is computed while the math warps work on dS(t), and their P phase of
+        // tile t+1 overlaps the dK / dQ MMAs of tile t; dP^T(t+1) follows dK(t),
+        // which reads dS^T(t) from the dP^T columns, and the dQ drain.
         int i = w.i_first;
         ok = issue_st(q_cnt, w, i) && issue_dpt(do_cnt);
         for (int t = 0; ok && i < w.n_tq; ++t) {
@@ -700,13 +701,13 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
                     (t > 0 || kk > 0) ? 1u : 0u);
           umma_commit(do_empty(so));
           ++do_cnt;
-          ok = mbar_wait(ds_full, ds_cnt & 1);
-          ++ds_cnt;
-          if (!ok) break;
           if (inext < w.n_tq) {
             ok = issue_st(q_cnt + 1, w, inext);
             if (!ok) break;
           }
+          ok = mbar_wait(ds_full, ds_cnt & 1);
+          ++ds_cnt;
+          if (!ok) break;
           tc_fence_after();
           // dK += dS^T Q_i
 #pragma unroll
@@ -1023,9 +1024,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         // Three kinds of row: a key beyond kv_len (all zero, no exponentials),
         // the causal diagonal tile (element mask), and the rest (no mask; part
         // of the exponentials on the FMA pipe through ex2_poly2).
-        // dropout: the undropped P (packed bf16) stays in registers for the dS
-        // phase; TMEM gets the kept, scaled P^T for the dV MMA
-        [[maybe_unused]] uint32_t pu[2][16];
+        // P (packed bf16) stays in registers for the dS phase (with dropout the
+        // undropped P; TMEM gets the kept P^T for the dV MMA), so the dS phase
+        // does not read P^T back and, at D = 128, the next S^T may be written over
+        // P^T as soon as the dV MMA has read it
+        uint32_t pu[2][16];
         {
           uint32_t r[2][32];
           tmem_ld32(tS, r[0]);
@@ -1078,18 +1081,22 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
                   p2 = (kr > q0 + 2) ? 0.f : p2;
                   p3 = (kr > q0 + 3) ? 0.f : p3;
                 }
+                // dS gets the whole P; with dropout, dV the kept P (w is applied in
+                // its epilogue)
+                pu[c][2 * e4] = pack_bf16x2(p0, p1);
+                pu[c][2 * e4 + 1] = pack_bf16x2(p2, p3);
                 if constexpr (kDrop) {
-                  // dV gets the kept P (w is applied in its epilogue); dS the whole P
-                  pu[c][2 * e4] = pack_bf16x2(p0, p1);
-                  pu[c][2 * e4 + 1] = pack_bf16x2(p2, p3);
                   const uint32_t b4 = kb[c] >> (4 * e4);
                   p0 = (b4 & 1u) ? p0 : 0.f;
                   p1 = (b4 & 2u) ? p1 : 0.f;
                   p2 = (b4 & 4u) ? p2 : 0.f;
                   p3 = (b4 & 8u) ? p3 : 0.f;
+                  pk[2 * e4] = pack_bf16x2(p0, p1);
+                  pk[2 * e4 + 1] = pack_bf16x2(p2, p3);
+                } else {
+                  pk[2 * e4] = pu[c][2 * e4];
+                  pk[2 * e4 + 1] = pu[c][2 * e4 + 1];
                 }
-                pk[2 * e4] = pack_bf16x2(p0, p1);
-                pk[2 * e4 + 1] = pack_bf16x2(p2, p3);
               }
             };
             // no allowed entry: a padding key, or (diagonal tile) a query chunk
@@ -1098,7 +1105,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
 #pragma unroll
               for (int e = 0; e < 16; ++e) {
                 pk[e] = 0u;
-                if constexpr (kDrop) pu[c][e] = 0u;
+                pu[c][e] = 0u;
               }
             } else if (diag) {
               make_p(std::integral_constant<int, 1>{});
@@ -1123,20 +1130,17 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         {
-          // dropout: the P kept in registers, one 32-query chunk of dP^T at a time
-          // (fewer registers live next to it); otherwise both chunks and P^T at once
+          // dropout: one 32-query chunk of dP^T at a time (fewer registers live
+          // next to the keep bits); otherwise both chunks at once
           uint32_t r[2][32];
-          [[maybe_unused]] uint32_t pp[32];
           if constexpr (kDrop) {
             tmem_ld32(tDP, r[0]);
           } else {
             tmem_ld32(tDP, r[0]);
             tmem_ld32(tDP + 32, r[1]);
-            tmem_ld32(tP, pp);  // this half's P: 32 packed columns
             tmem_wait_ld();
             reg_fence32(r[0]);
             reg_fence32(r[1]);
-            reg_fence32(pp);
           }
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
@@ -1171,8 +1175,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
                 tb = f2_add(
                     f2_pack(__uint_as_float(r[c][4 * e4 + 2]), __uint_as_float(r[c][4 * e4 + 3])),
                     f2_pack(nd.z, nd.w));
-                pa = pp[c * 16 + 2 * e4];
-                pb = pp[c * 16 + 2 * e4 + 1];
+                pa = pu[c][2 * e4];
+                pb = pu[c][2 * e4 + 1];
               }
               float d0, d1, d2, d3;
               f2_unpack(f2_mul(ta, bf16x2_to_f2(pa)), d0, d1);

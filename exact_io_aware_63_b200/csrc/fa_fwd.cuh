@@ -10,9 +10,11 @@
 // score tile lives in on-chip memory only.
 //
 // B200 mapping (one persistent CTA per SM, 12 warps):
-//   warp 0      TMA producer: the unit's Q tile(s) (double-buffered across
-//               units where shared memory allows), then the K/V tiles it
-//               visits, through a kStages-deep mbarrier ring
+//   warp 0      TMA producer: takes work units from a counter shared by all
+//               CTAs and publishes them to the other roles through a
+//               shared-memory ring; loads the unit's Q tile(s) (double-
+//               buffered across units where shared memory allows), then the
+//               K/V tiles it visits, through a kStages-deep mbarrier ring
 //   warp 1      owns the TMEM allocation; issues MMAs (one thread): for both
 //               warpgroups at D = 128, for warpgroup 0 at D = 64
 //   warp 2      D = 64: issues warpgroup 1's MMAs
@@ -128,8 +130,34 @@ struct FwdParams {
   int heads_per_group;  // unit order: see fwd_decode
   int causal;
   float scale_log2;  // scale * log2(e)
+  int counter_slot;  // this launch's work counter: g_fwd_work[counter_slot]
   DropoutParams drop;  // read by kernels instantiated with kDrop only
 };
+
+// Work counters of the forward kernel, which has no workspace.  Launch t uses
+// slot t % kFwdCounterSlots (the host hands the slots out in turn): its CTAs
+// take units with atomicAdd on word 0 and count themselves out on word 1; the
+// last CTA to finish sets both back to zero for the launch that reuses the
+// slot.  Launches that are in flight together on one device (other streams)
+// therefore use different slots as long as fewer than kFwdCounterSlots of
+// them overlap.
+constexpr int kFwdCounterSlots = 1024;
+static __device__ unsigned int g_fwd_work[kFwdCounterSlots][2];
+
+// Called by one thread of each CTA once the CTA takes no more units: the last
+// CTA of the launch to get here sets the slot back to zero.
+__device__ __forceinline__ void fwd_count_out(int slot) {
+  __threadfence();
+  if (atomicAdd(&g_fwd_work[slot][1], 1u) == gridDim.x - 1) {
+    atomicExch(&g_fwd_work[slot][0], 0u);
+    atomicExch(&g_fwd_work[slot][1], 0u);
+  }
+}
+
+// Unit records: the producer takes each work unit from the launch's counter
+// and publishes its index in a ring of kUnitRing shared-memory slots for the
+// other roles; -1 marks the end of the work.
+constexpr int kUnitRing = 4;
 
 template <int D, bool kPair>
 struct FwdCfg {
@@ -153,10 +181,12 @@ struct FwdCfg {
   static constexpr int kOffBar = kOffML + 2 * kTile * 8;
   // barriers: q_full[2], q_empty[2], k_full[S], k_empty[S], v_full[S], v_empty[S],
   //           s_full[2], p_full[2], o_full[2], drain[2], ml_ready, merged, s_free[2],
-  //           p_free[2]
-  static constexpr int kNumBars = 18 + 4 * kStages;
+  //           p_free[2], unit_full[R], unit_empty[R]
+  static constexpr int kNumBars = 18 + 4 * kStages + 2 * kUnitRing;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kSmemBytes = kOffMisc + 16;
+  // misc: TMEM base address, abort flag, then the unit ring (kUnitRing ints)
+  static constexpr int kOffRing = kOffMisc + 16;
+  static constexpr int kSmemBytes = kOffRing + 4 * kUnitRing;
   static_assert(kSmemBytes <= 232448, "shared memory over the per-block limit");
   static constexpr uint32_t kTmemCols = 512;
   // pairs (of every 8) whose exponentials ex2_poly2 computes on interior tiles
@@ -180,8 +210,10 @@ struct FwdCfg {
 // Work-unit order: heads are taken in groups whose K and V fit in a share of
 // L2 (the units running at the same time then re-read K and V from L2, not
 // HBM); inside a group the longest units come first (for causal masks the
-// last query tiles see the most keys), and units go to CTAs in snake order so
-// that the sum of lengths per CTA evens out.
+// last query tiles see the most keys).  The forward kernel takes units in that
+// order from a counter shared by its CTAs; the ordered dQ kernel deals them to
+// CTAs in snake order instead (unit_for_round), so that the sum of lengths
+// per CTA evens out.
 __device__ __forceinline__ int unit_for_round(int round, int cta, int G) {
   return round * G + ((round & 1) ? (G - 1 - cta) : cta);
 }
@@ -255,21 +287,6 @@ __device__ __forceinline__ FwdUnit fwd_decode(const FwdParams& p, int u) {
   return w;
 }
 
-// The first round >= r whose unit has work, or one whose unit is past the
-// last (every role walks the same sequence).  Only packed batches have units
-// without work: query tiles beyond a shorter sequence's end.
-template <bool kPair, bool kPacked>
-__device__ __forceinline__ int live_round(const FwdParams& p, int r, int cta, int G) {
-  if constexpr (!kPacked) {
-    return r;
-  } else {
-    for (;; ++r) {
-      const int u = unit_for_round(r, cta, G);
-      if (u >= p.num_units || !fwd_decode<kPair, true>(p, u).empty) return r;
-    }
-  }
-}
-
 // Split mode: first key tile >= j that query tile w.i0 visits (or j_end):
 // tiles below j_end hold an allowed key for causal and key-padding masks; the
 // block mask is the only test left.  (Pair mode has no block mask: its tiles
@@ -292,7 +309,10 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
   constexpr int QSLOTS = Cfg::kQSlots;
   extern __shared__ __align__(1024) uint8_t smem[];
   pdl_launch_dependents();
-  if (!smem_aligned_1024(smem)) return;
+  if (!smem_aligned_1024(smem)) {
+    if (threadIdx.x == 0) fwd_count_out(p.counter_slot);
+    return;
+  }
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + Cfg::kOffBar;
   auto q_full = [&](int x) { return bar0 + 8 * x; };
@@ -313,9 +333,32 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
   // separate-P layout: warpgroup x has read S_x (128 arrivals) / P V_x has read P_x
   auto s_free = [&](int x) { return bar0 + 8 * (13 + 4 * S + x); };
   auto p_free = [&](int x) { return bar0 + 8 * (15 + 4 * S + x); };
-  static_assert(Cfg::kNumBars == 18 + 4 * S, "barrier layout");
+  constexpr int UR = kUnitRing;
+  auto unit_full = [&](int r) { return bar0 + 8 * (18 + 4 * S + r); };
+  auto unit_empty = [&](int r) { return bar0 + 8 * (18 + 4 * S + UR + r); };
+  static_assert(Cfg::kNumBars == 18 + 4 * S + 2 * UR, "barrier layout");
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kOffMisc + 4);
+  volatile int* unit_ring = reinterpret_cast<volatile int*>(smem + Cfg::kOffRing);
+  // the warps that read every unit record: the MMA issuer(s) and 8 softmax warps
+  constexpr uint32_t kUnitReaders = (Cfg::kSepP ? 2 : 1) + 8;
+  // one thread's read of round r's record (it releases the slot)
+  auto fetch_one = [&](int r, int& u) -> bool {
+    const int sl = r % UR;
+    if (!mbar_wait(unit_full(sl), (r / UR) & 1)) return false;
+    u = unit_ring[sl];
+    mbar_arrive(unit_empty(sl));
+    return true;
+  };
+  // a whole warp's read (lane 0 releases the slot)
+  auto fetch_warp = [&](int r, int& u) -> bool {
+    const int sl = r % UR;
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(unit_full(sl), (r / UR) & 1));
+    if (ok) u = unit_ring[sl];
+    __syncwarp();
+    if (ok && lane_id() == 0) mbar_arrive(unit_empty(sl));
+    return ok;
+  };
   float2* ml_smem = reinterpret_cast<float2*>(smem + Cfg::kOffML);  // [2][128] (m, l)
   // shared-memory address of query tile x (0 / 1) of Q slot q
   auto q_tile = [&](int q, int x) {
@@ -347,6 +390,10 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
     mbar_init(drain(1), 1);
     mbar_init(ml_ready, 256);
     mbar_init(merged, 256);
+    for (int r = 0; r < UR; ++r) {
+      mbar_init(unit_full(r), 1);
+      mbar_init(unit_empty(r), kUnitReaders);
+    }
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tmap(&tm_q);
@@ -365,7 +412,6 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
   // waits for the previous kernel in the stream
   pdl_wait();
   const uint32_t tmem = *tmem_base_slot;
-  const int G = gridDim.x;
   static_assert(Cfg::kRegsLow * 128 + Cfg::kRegsHigh * 256 <= Cfg::kRegsLaunch * Cfg::kThreads,
                 "register split exceeds the launch allocation");
 
@@ -375,10 +421,36 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
     if (lane == 0) {
       uint32_t q_cnt = 0, kv_cnt = 0;
       bool ok = true;
-      for (int round = live_round<kPair, kPacked>(p, 0, blockIdx.x, G); ok;
-           round = live_round<kPair, kPacked>(p, round + 1, blockIdx.x, G)) {
-        const int u = unit_for_round(round, blockIdx.x, G);
-        if (u >= p.num_units) break;
+      // Units come from the launch's counter, shared by all CTAs, in the order
+      // fwd_decode gives them (longest first within each head group), so that
+      // the CTAs finish together whatever the unit lengths.  Records are
+      // published one round ahead (the issuers read the next unit's record at
+      // the end of this one); after the work runs out, one record marks the end.
+      unsigned int* const work_next = &g_fwd_work[p.counter_slot][0];
+      int published = 0;
+      bool ended = false;
+      auto publish_through = [&](int upto) -> bool {
+        while (!ended && published <= upto) {
+          int un = static_cast<int>(atomicAdd(work_next, 1u));
+          if (un >= p.num_units) {
+            un = -1;
+          } else if (kPacked && fwd_decode<kPair, kPacked>(p, un).empty) {
+            continue;  // query tiles past a shorter sequence's end: no work
+          }
+          const int sl = published % UR;
+          if (!mbar_wait(unit_empty(sl), ((published / UR) & 1) ^ 1)) return false;
+          unit_ring[sl] = un;
+          mbar_arrive(unit_full(sl));
+          ++published;
+          if (un < 0) ended = true;
+        }
+        return true;
+      };
+      for (int round = 0; ok; ++round) {
+        ok = publish_through(round + 1);
+        if (!ok) break;
+        const int u = unit_ring[round % UR];
+        if (u < 0) break;
         const FwdUnit w = fwd_decode<kPair, kPacked>(p, u);
         const int qs = q_cnt % QSLOTS;
         ok = mbar_wait(q_empty(qs), ((q_cnt / QSLOTS) & 1) ^ 1);
@@ -441,10 +513,15 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
       uint32_t pre = 0;      // bit x: S_x of this unit's first key tile already issued
       bool pre_q = false;    // this unit's Q already waited for
       bool pre_k = false;    // this unit's first K tile already waited for
-      for (int round = live_round<kPair, kPacked>(p, 0, blockIdx.x, G); ok;
-           round = live_round<kPair, kPacked>(p, round + 1, blockIdx.x, G)) {
-        const int u = unit_for_round(round, blockIdx.x, G);
-        if (u >= p.num_units) break;
+      int u_ahead = -2;      // the next round's record when already read (-2: not read)
+      for (int round = 0; ok; ++round) {
+        int u = u_ahead;
+        u_ahead = -2;
+        if (u == -2 && !fetch_one(round, u)) {
+          ok = false;
+          break;
+        }
+        if (u < 0) break;
         const FwdUnit w = fwd_decode<kPair, kPacked>(p, u);
         const int qs = q_cnt % QSLOTS;
         if (!pre_q) ok = mbar_wait(q_full(qs), (q_cnt / QSLOTS) & 1);
@@ -486,10 +563,15 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
           // competing with it for issue slots.
           const int j_end = w.j_end;
           // the next unit (look-ahead)
-          const int un =
-              unit_for_round(live_round<kPair, kPacked>(p, round + 1, blockIdx.x, G), blockIdx.x,
-                             G);
-          const bool has_next = kLook && un < p.num_units;
+          int un = -1;
+          if (kLook) {
+            if (!fetch_one(round + 1, un)) {
+              ok = false;
+              break;
+            }
+            u_ahead = un;
+          }
+          const bool has_next = kLook && un >= 0;
           FwdUnit wn = w;
           if (has_next) wn = fwd_decode<kPair, kPacked>(p, un);
           const int qsn = q_cnt % QSLOTS;
@@ -687,10 +769,15 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
       uint32_t t_cnt = 0;              // tiles of this warpgroup (s_free / p_full phases)
       bool pre = false;                // this unit's Q awaited and first own S issued
       bool ok = true;
-      for (int round = live_round<kPair, kPacked>(p, 0, blockIdx.x, G); ok;
-           round = live_round<kPair, kPacked>(p, round + 1, blockIdx.x, G)) {
-        const int u = unit_for_round(round, blockIdx.x, G);
-        if (u >= p.num_units) break;
+      int u_ahead = -2;  // the next round's record when already read (-2: not read)
+      for (int round = 0; ok; ++round) {
+        int u = u_ahead;
+        u_ahead = -2;
+        if (u == -2 && !fetch_one(round, u)) {
+          ok = false;
+          break;
+        }
+        if (u < 0) break;
         const FwdUnit w = fwd_decode<kPair, kPacked>(p, u);
         const int qs = q_cnt % QSLOTS;
         const uint32_t q_par = (q_cnt / QSLOTS) & 1;
@@ -730,10 +817,13 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
           } else {
             umma_commit(q_empty(qs));  // this warpgroup's last S on this Q is issued
             if constexpr (kLook) {
-              const int un =
-              unit_for_round(live_round<kPair, kPacked>(p, round + 1, blockIdx.x, G), blockIdx.x,
-                             G);
-              if (un < p.num_units) {
+              int un = -1;
+              if (!fetch_one(round + 1, un)) {
+                ok = false;
+                break;
+              }
+              u_ahead = un;
+              if (un >= 0) {
                 const FwdUnit wn = fwd_decode<kPair, kPacked>(p, un);
                 if ((x ? wn.j_end1 : wn.j_end0) > 0) {
                   const int qsn = q_cnt % QSLOTS;
@@ -807,10 +897,10 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
     uint32_t q_use = 0;  // units seen: ring index of their Q slot
     uint32_t o_cnt[2] = {0, 0};
     bool ok = true;
-    for (int round = live_round<kPair, kPacked>(p, 0, blockIdx.x, G); ok;
-           round = live_round<kPair, kPacked>(p, round + 1, blockIdx.x, G)) {
-      const int u = unit_for_round(round, blockIdx.x, G);
-      if (u >= p.num_units) break;
+    for (int round = 0; ok; ++round) {
+      int u = -1;
+      ok = fetch_warp(round, u);
+      if (!ok || u < 0) break;
       const FwdUnit w = fwd_decode<kPair, kPacked>(p, u);
       const int qs_me = q_use % QSLOTS;
       const uint32_t q_par = (q_use / QSLOTS) & 1;
@@ -1148,6 +1238,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, Cfg::kTmemCols);
+  if (threadIdx.x == 0) fwd_count_out(p.counter_slot);
 }
 
 }  // namespace fa

@@ -26,9 +26,11 @@
  *  - Tensors Q, K, V, O, dO, dQ, dK, dV are bfloat16 (raw 16-bit patterns,
  *    type fa_bf16), contiguous [B][H][N][d] in device memory, base address
  *    16-byte aligned.  LSE is float32 [B][H][N] (natural log), 4-byte aligned.
- *  - d is 32, 64, 96 or 128 (32 and 96 run on the 64- and 128-column kernels,
- *    whose loads read the missing columns as zeros and whose stores stop at d;
- *    the ordered dQ of fa_bwd_deterministic takes 64 and 128 only).
+ *  - d is 32, 64, 96, 128 or 256 (32 and 96 run on the 64- and 128-column
+ *    kernels, whose loads read the missing columns as zeros and whose stores
+ *    stop at d; the ordered dQ of fa_bwd_deterministic takes 64, 128 and 256;
+ *    256 has kernels of its own, described at fa_bwd, and no dropout or
+ *    packed variable-length form: those calls return FA_ERR_UNSUPPORTED_D).
  *    N is any length: tiles are 128 long, and when 128 does
  *    not divide N the last tile is partial.  B, H, N >= 0; if any is 0 the
  *    call does nothing and returns FA_OK.  B*H*N must be below 2^31.
@@ -73,7 +75,8 @@ typedef enum {
     FA_ERR_NULL = -1,           /* a required pointer is NULL */
     FA_ERR_ALIGN = -2,          /* a pointer breaks its alignment rule */
     FA_ERR_SHAPE = -3,          /* negative size, or B*H*N >= 2^31 */
-    FA_ERR_UNSUPPORTED_D = -4,  /* d not in {32, 64, 96, 128} ({64, 128} for the ordered dQ) */
+    FA_ERR_UNSUPPORTED_D = -4,  /* d not in {32, 64, 96, 128, 256} ({64, 128, 256} for the
+                                   ordered dQ; 256 with dropout or packed batches) */
     FA_ERR_WORKSPACE = -5,      /* workspace NULL or smaller than fa_bwd_workspace_size */
     FA_ERR_CUDA = -6,           /* a CUDA runtime/driver call failed */
     FA_ERR_TIMEOUT = -7,        /* a device pipeline wait gave up (fa_get_device_status) */
@@ -108,9 +111,9 @@ int fa_fwd_traced(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, fa_bf16*
 
 /*
  * Bytes of device workspace fa_bwd needs: 4*B*H*Np (D) + 4*B*H*Np (LSE in
- * base 2) + 4*B*H*N*d (float32 dQ accumulator) + 256 (the counter from which
- * the main kernel's CTAs take work units), each region 256-byte aligned,
- * where Np is N rounded up to a multiple of 128.
+ * base 2) + 4*B*H*N*d (float32 dQ accumulator; none at d = 256) + 256 (the
+ * counter from which the main kernel's CTAs take work units), each region
+ * 256-byte aligned, where Np is N rounded up to a multiple of 128.
  * Returns 0 for an empty or invalid shape.
  */
 size_t fa_bwd_workspace_size(int B, int H, int N, int d);
@@ -122,6 +125,11 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d);
  * main kernel (one CTA per (b, h, 128-key tile): recompute S and P,
  * accumulate dK and dV on chip, add dQ partials into the float32
  * accumulator), and a kernel that writes dQ = bf16(scale * accumulator).
+ * At d = 256 a 128-key tile's float32 dK and dV would fill tensor memory, so
+ * the work after the preprocess kernel is three passes instead, each
+ * recomputing the score tile it needs: dK per key tile, dV per key tile, and
+ * dQ per query tile summed on chip in a fixed order (no accumulator in the
+ * workspace; the result is bitwise reproducible).
  * workspace must be 256-byte aligned and hold fa_bwd_workspace_size bytes;
  * its contents on entry do not matter and on exit are unspecified.  Calls
  * that share a workspace must not overlap on the device.
@@ -150,7 +158,8 @@ int fa_bwd_traced(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa
  * dV; dQ partials into the accumulator; takes its work units from the
  * counter, so each phase 1 needs a phase 0 before it), 2 = dQ = bf16(scale *
  * accumulator), 3 = dQ by the ordered kernel of fa_bwd_deterministic (reads
- * only what phase 0 wrote).  Arguments as for
+ * only what phase 0 wrote).  At d = 256: phase 1 = the dK and dV passes,
+ * phases 2 and 3 = the dQ pass.  Arguments as for
  * fa_bwd.  Calling phases 0, 1, 2 in order on one stream with the same
  * arguments and workspace is exactly fa_bwd, and 0, 1, 3 is exactly
  * fa_bwd_deterministic; a phase reads what the earlier phases left in the

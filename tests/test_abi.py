@@ -127,7 +127,7 @@ def test_shape_errors(call):
     assert call(B=-1) == -3
     assert call(B=1 << 16, H=1 << 8, N=1 << 8) == -3   # B*H*N >= 2^31
     assert call(d=80) == -4
-    assert call(d=256) == -4
+    assert call(d=192) == -4
     assert call(d=16) == -4
 
 
@@ -359,3 +359,19 @@ def test_binding_return_types_match_the_header():
     assert set(rets) == set(binding._SIGS)
     for name, ret in rets.items():
         assert binding._SIGS[name][0] is kinds[re.sub(r"\s*\*", "*", ret)], name
+
+
+def test_head_dimension_256_has_no_dropout_or_packed_form():
+    lib = binding.load()
+    # dropout at d = 256 is refused before any pointer is looked at
+    assert lib.fa_fwd_dropout(P, P, P, P, P, 1, 1, 128, 256, 0.0625, 0, None, None, 0.1, 1, 0,
+                              None) == -4
+    assert lib.fa_bwd_dropout(P, P, P, P, P, P, P, P, P, 1, 1, 128, 256, 0.0625, 0, None, None,
+                              0.1, 1, 0, P, 1 << 30, None) == -4
+    assert fwd_varlen(d=256) == -4
+    assert bwd_varlen(d=256) == -4
+    # the plain passes accept it: their next check is the NULL pointer
+    assert lib.fa_fwd(None, P, P, P, P, 1, 1, 128, 256, 0.0625, 0, None, None, None) == -1
+    # no float32 dQ accumulator at d = 256: -D and -LSE2 (4 bytes each per row, rows
+    # padded to 384) and the 256-byte counter only
+    assert binding.fa_bwd_workspace_size(1, 1, 300, 256) == 4 * 384 + 4 * 384 + 256

@@ -1,5 +1,9 @@
-"""Head dimensions 32 and 96: the 64- and 128-column kernels with tensor maps that read
-the missing columns as zeros and stores that stop at d, against the FP64 oracle."""
+"""Head dimensions other than 64 and 128, against the FP64 oracle.
+
+32 and 96 run on the 64- and 128-column kernels with tensor maps that read the missing
+columns as zeros and stores that stop at d.  256 has kernels of its own: a forward kernel
+with one query tile per unit, and a backward pass in three passes (dQ, dK, dV), each
+recomputing the score tile it needs."""
 
 import numpy as np
 import pytest
@@ -68,3 +72,59 @@ def test_dropout(cuda_device, d):
     g = oracle.attention_backward_dropout(qd, kd, vd, dod, x.scale, *drop, causal=True)
     for name, got, ref in zip(("dq", "dk", "dv"), (dq, dk, dv), g[:3]):
         assert rel_l2(f(got), ref) <= GRAD_TOL, name
+
+
+# ---------------------------------------------------------------------------
+# head dimension 256
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [128, 384, 640])
+def test_d256_dense(cuda_device, causal, N):
+    check_all_heads(inputs.make_inputs(2, 2, N, 256, causal=causal, seed=900 + N + int(causal)))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_d256_partial_tile_and_key_padding(cuda_device, causal):
+    # lengths inside a tile, on a tile edge, a single key, out of range
+    x = inputs.make_inputs(4, 2, 300, 256, causal=causal, seed=910 + int(causal),
+                           kv_len=torch.tensor([300, 128, 1, 77], dtype=torch.int32))
+    check_all_heads(x)
+
+
+def test_d256_block_mask_and_rows_without_keys(cuda_device):
+    bm = inputs.draw_block_mask(5, 0.3, torch.Generator().manual_seed(920))
+    bm[1, :] = 0  # query tile 1 sees no key tile
+    x = inputs.make_inputs(2, 2, 600, 256, causal=True, seed=921, block_mask=bm,
+                           kv_len=torch.tensor([600, 0], dtype=torch.int32))
+    res, out = check_all_heads(x)
+    from gpu_helpers import f64
+    assert np.all(f64(out["o"])[:, :, 128:256] == 0)
+    assert np.all(f64(out["o"])[1] == 0) and np.all(np.isneginf(f64(out["lse"])[1]))
+
+
+def test_d256_tile_visits_match_the_mask(cuda_device):
+    from gpu_helpers import run_gpu
+    x = inputs.make_inputs(2, 1, 700, 256, causal=True, seed=930, block_keep=0.4,
+                           kv_len=torch.tensor([700, 250], dtype=torch.int32))
+    out = run_gpu(x, backward=True, traced=True)
+    want = oracle.tile_visits(2, 700, True, x.block_mask.numpy(), x.kv_len.numpy())
+    for name in ("vis_f", "vis_b"):
+        got = out[name].cpu().numpy()[:, 0]
+        assert np.array_equal(got, want), name
+
+
+def test_d256_backward_is_bitwise_reproducible(cuda_device):
+    # every gradient is summed in a fixed order on chip: fa_bwd repeats itself bit for
+    # bit and equals fa_bwd_deterministic
+    from gpu_helpers import to_dev
+    x = inputs.make_inputs(1, 3, 512, 256, causal=True, seed=940)
+    q, k, v, do, bm, kl = to_dev(x)
+    o, lse = binding.attention_forward(q, k, v, x.scale, True)
+    a = binding.attention_backward(q, k, v, o, lse, do, x.scale, True)
+    b = binding.attention_backward(q, k, v, o, lse, do, x.scale, True)
+    c = binding.attention_backward(q, k, v, o, lse, do, x.scale, True, deterministic=True)
+    torch.cuda.synchronize()
+    assert binding.fa_get_device_status() == 0
+    for ta, tb, tc in zip(a, b, c):
+        assert torch.equal(ta, tb) and torch.equal(ta, tc)
