@@ -119,13 +119,13 @@ bool make_tmap_f32_acc(CUtensorMap* m, const void* base, int BH, int N, int d) {
 // Packed [T][H][d] tensors (variable-length batches) mapped as (d, H, T), so
 // that the strides increase: box (64, 1, 128) is a 128-token tile of one head,
 // laid out in shared memory exactly like the (64, 128, 1) box of make_tmap.
-bool make_tmap_packed(CUtensorMap* m, const void* base, int H, int T, int d) {
+bool make_tmap_packed(CUtensorMap* m, const void* base, int H, int T, int d, int box_rows = 128) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
                         static_cast<cuuint64_t>(T)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(H) * d * 2};
-  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -157,8 +157,10 @@ struct Packed {
 };
 
 // Tensor map of a bf16 operand in either layout.
-bool make_tmap_any(CUtensorMap* m, const void* base, int B, int H, int N, int d, const Packed& pk) {
-  return pk.cu ? make_tmap_packed(m, base, H, pk.T, d) : make_tmap(m, base, B * H, N, d);
+bool make_tmap_any(CUtensorMap* m, const void* base, int B, int H, int N, int d, const Packed& pk,
+                   int box_rows = 128) {
+  return pk.cu ? make_tmap_packed(m, base, H, pk.T, d, box_rows)
+               : make_tmap(m, base, B * H, N, d, box_rows);
 }
 
 // Launches a kernel with programmatic stream serialization: it may be
@@ -406,8 +408,8 @@ int launch_bwd(const fa_bf16* q, const fa_bf16* k, const fa_bf16* v, const fa_bf
                             : make_tmap_f32_acc(&tdq, dq_acc, BH, N, d);
   if (!make_tmap_any(&tq, q, B, H, N, d, pk) || !make_tmap_any(&tk, k, B, H, N, d, pk) ||
       !make_tmap_any(&tv, v, B, H, N, d, pk) || !make_tmap_any(&tdo, dout, B, H, N, d, pk) ||
-      !acc_ok || !make_tmap_any(&tdk, dk, B, H, N, d, pk) ||
-      !make_tmap_any(&tdv, dv, B, H, N, d, pk))
+      !acc_ok || !make_tmap_any(&tdk, dk, B, H, N, d, pk, 32) ||
+      !make_tmap_any(&tdv, dv, B, H, N, d, pk, 32))  // dK / dV: 32-row boxes, one per warp
     return FA_ERR_CUDA;
   static std::atomic<bool> smem_done[4][kMaxDevices];
   if (!ensure_smem(fa::fa_bwd_kernel<D, false, false>, Cfg::kSmemBytes, smem_done[0]) ||

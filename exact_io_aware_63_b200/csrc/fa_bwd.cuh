@@ -1208,10 +1208,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       if (epi_tma) {
-        // the previous unit's TMA store (issued by this warpgroup's first
-        // thread, not awaited then) has read the staging area
-        if (kr == 0) bulk_wait_group_read0();
-        named_bar_sync(1 + h, 128);
+        // this warp's previous TMA store (issued by its first lane, not awaited
+        // then) has read the warp's 32 staged rows
+        if (lane == 0) bulk_wait_group_read0();
+        __syncwarp();
       }
       const float mul = h ? (kDrop ? p.drop.w : 1.f) : p.scale;  // dV: dropout weight
       const uint32_t tAcc = t_lane + (h ? Cfg::kColDV : Cfg::kColDK);
@@ -1239,20 +1239,22 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       }
       tc_fence_before();
       if (epi_tma) {
-        // the whole tile is staged: one thread of the warpgroup stores it
-        // (the next epilogue waits for the store's read of the staging area)
+        // the warp's 32 rows are staged: its first lane stores them as one
+        // 32-row box (the next epilogue waits for the store's read of them),
+        // so no warp waits for another
         fence_proxy_async_smem();
-        named_bar_sync(1 + h, 128);
-        if (kr == 0) {
-          const int2 yz = tile_yz(kPacked, (kPacked ? w.tok_base : 0) + w.j * kTile, w.tz);
+        __syncwarp();
+        if (lane == 0) {
+          const int2 yz =
+              tile_yz(kPacked, (kPacked ? w.tok_base : 0) + w.j * kTile + quarter * 32, w.tz);
           tma_store_3d(h ? &tm_dv : &tm_dk, 0, yz.x, yz.y,
-                       smem_u32(smem + Cfg::kOffEpi + h * Cfg::kTileBytes));
+                       smem_u32(smem + Cfg::kOffEpi + h * Cfg::kTileBytes + quarter * 4096));
           bulk_commit_group();
         }
       }
     }
     if (!ok) *abort_flag = 1;
-    if (Cfg::kEpiTma && kr == 0) bulk_wait_group0();  // stores complete before exit
+    if (Cfg::kEpiTma && lane == 0) bulk_wait_group0();  // stores complete before exit
   } else {
     // ------------------------------------------------------------ dQ group
     // Drains dQ partials: TMEM -> registers -> its own shared-memory staging
