@@ -260,12 +260,14 @@ bool ensure_smem(Kernel k, int bytes, std::atomic<bool> (&done)[kMaxDevices]) {
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Heads per work-unit group: as many as keep `bytes_per_head` of re-read data
-// within a 48 MB share of the 126 MB L2, with the heads spread evenly over the
+// within a 96 MB share of the 126 MB L2, with the heads spread evenly over the
 // groups (16 heads in groups of at most 5 become four groups of 4, not 5, 5,
-// 5, 1): a last group of few heads would leave its few longest units running
-// alone at the end of the launch.
+// 5, 1).  Large groups matter for causal masks: the longest unit of the last
+// group runs alone at the end of the launch unless the group's work per SM
+// exceeds it (a 48 MB share left the SMs idle for 14-20% of a causal 8K
+// launch).
 int heads_per_group(int BH, double bytes_per_head) {
-  const double budget = 48.0 * 1024 * 1024;
+  const double budget = 96.0 * 1024 * 1024;
   int g = static_cast<int>(budget / bytes_per_head);
   g = g < 1 ? 1 : (g > BH ? BH : g);
   const int groups = (BH + g - 1) / g;
