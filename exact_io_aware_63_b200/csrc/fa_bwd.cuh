@@ -298,8 +298,6 @@ struct BwdCfg {
   // dQ staging: each dQ warp owns 8 KB = two 32 x 32 float32 boxes
   static constexpr int kDqBoxesPerRound = 2;
   static constexpr int kDqRounds = D / 64;
-  // pairs (of every 4) whose exponentials ex2_poly2 computes, off the diagonal
-  static constexpr int kPolyPer4 = 1;
   // TMEM column of the bf16 operand for K-step kk (16 queries) of the dV / dK MMAs
   __device__ static constexpr uint32_t packed_col(uint32_t base, int kk) {
     return base + (kk >> 2) * 64 + (kk & 3) * 8;
@@ -936,9 +934,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     // Warpgroup h (warps 4-7: h = 0, warps 8-11: h = 1) handles queries
     // 64h..64h+63 of every key row; one key row per thread (TMEM lane).
     if constexpr (Cfg::kRegsDs > Cfg::kRegsLaunch) setmaxnreg_inc<Cfg::kRegsDs>();
-    // with dropout the generator's integer multiplies load the FMA pipe:
-    // every exponential goes to the MUFU unit
-    constexpr int kPolyPer4 = kDrop ? 0 : Cfg::kPolyPer4;
+    // every exponential of the backward pass goes to the MUFU unit: moving a
+    // quarter of them to the FMA pipe (ex2_poly2, as the forward pass does)
+    // was 3% slower at D = 64 and no faster at D = 128
     const int h = (warp >= 8) ? 1 : 0;
     const int quarter = warp & 3;
     const int kr = quarter * 32 + lane;  // key row within the tile
@@ -1022,8 +1020,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         tc_fence_after();
         // P^T: p[q] = exp2(S^T[kr][q] * scale*log2e - LSE2[q]); masked -> 0.
         // Three kinds of row: a key beyond kv_len (all zero, no exponentials),
-        // the causal diagonal tile (element mask), and the rest (no mask; part
-        // of the exponentials on the FMA pipe through ex2_poly2).
+        // the causal diagonal tile (element mask), and the rest (no mask).
         // P (packed bf16) stays in registers for the dS phase (with dropout the
         // undropped P; TMEM gets the kept P^T for the dV MMA), so the dS phase
         // does not read P^T back and, at D = 128, the next S^T may be written over
@@ -1050,8 +1047,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             uint32_t pk[16];
-            // kind: 0 = no mask (part of the exponentials through ex2_poly2),
-            //       1 = causal diagonal tile (element mask)
+            // kind: 0 = no mask, 1 = causal diagonal tile (element mask)
             auto make_p = [&](auto kind_tag) {
               constexpr int kKind = decltype(kind_tag)::value;
 #pragma unroll
@@ -1066,12 +1062,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
                 float x0, x1, x2, x3, p0, p1, p2, p3;
                 f2_unpack(xa, x0, x1);
                 f2_unpack(xb, x2, x3);
-                if (kKind == 0 && (e4 & 3) < kPolyPer4) {
-                  ex2_poly2(x0, x1, p0, p1);
-                } else {
-                  p0 = ex2_approx(x0);
-                  p1 = ex2_approx(x1);
-                }
+                p0 = ex2_approx(x0);
+                p1 = ex2_approx(x1);
                 p2 = ex2_approx(x2);
                 p3 = ex2_approx(x3);
                 if (kKind == 1) {
