@@ -102,7 +102,7 @@ def load_peaks():
 
 # the sources the benchmarked kernels and their launches are compiled from (fa_api.cu
 # sets grid sizes and the unit order, which move DRAM traffic too)
-BENCHED_KERNEL_SOURCES = ("fa_api.cu", "fa_bwd.cuh", "fa_fwd.cuh", "sm100.cuh")
+BENCHED_KERNEL_SOURCES = ("fa_api.cu", "fa_bwd.cuh", "fa_d256.cuh", "fa_fwd.cuh", "sm100.cuh")
 
 
 def kernel_source_hash():
@@ -562,19 +562,28 @@ def oracle_sample(x, n_heads, n_rows):
     return heads, sel(x.q), sel(x.k), sel(x.v), sel(x.dout), kl
 
 
+def sample_band(N, n_rows):
+    """Query rows [r0, r1) of a sample: the middle n_rows rows of N.  Under a causal mask a
+    middle row has about N/2 keys, the mean over all rows; the first rows have almost none,
+    and a sample of them would time mostly the oracle's fixed cost per head."""
+    r0 = (N - n_rows) // 2
+    return r0, r0 + n_rows
+
+
 def time_oracle(x, n_heads, n_rows, threads):
     import numpy as np
     import oracle
     heads, q, k, v, do, kl = oracle_sample(x, n_heads, n_rows)
     bm = None if x.block_mask is None else x.block_mask.numpy()
     kl = None if kl is None else np.array(kl, np.int32)
+    B, H, N, d = x.q.shape
+    r0, r1 = sample_band(N, n_rows)
     t0 = time.perf_counter()
-    oracle.attention_forward_band(q, k, v, x.scale, x.causal, bm, kl, 0, n_rows, threads)
-    oracle.attention_backward_band(q, k, v, do, x.scale, x.causal, bm, kl, 0, n_rows, threads)
+    oracle.attention_forward_band(q, k, v, x.scale, x.causal, bm, kl, r0, r1, threads)
+    oracle.attention_backward_band(q, k, v, do, x.scale, x.causal, bm, kl, r0, r1, threads)
     dt = time.perf_counter() - t0
     # metric FLOPs of the sample: the workload's per-entry rate times the sample's entries
-    B, H, N, d = x.q.shape
-    per_b = allowed_entries(x, range(n_rows))
+    per_b = allowed_entries(x, range(r0, r1))
     entries = sum(per_b[b] for b, _ in heads)
     all_entries = allowed_entries(x, range(N)).sum() * H
     flops = 3.5 * flops_fwd(x) * entries / all_entries
@@ -588,25 +597,38 @@ def sample_plan(x, threads):
     return n_heads, n_rows
 
 
-def cpu_baseline(x, budget_s=20.0):
-    """Oracle throughput on a bounded sample: whole heads (or a band of rows for
-    N > 4096), grown until about budget_s CPU-seconds of work."""
-    threads = os.cpu_count() or 1
+def grow_sample(x, threads, budget_s):
+    """Whole heads (or a band of rows for N > 4096), doubled until one timing of the sample
+    takes about budget_s CPU-seconds (or the sample is the whole workload).  Returns
+    (n_heads, n_rows, seconds, flops, heads) of the last timing."""
     B, H, N, d = x.q.shape
     n_heads, n_rows = sample_plan(x, threads)
     while True:
         dt, flops, heads = time_oracle(x, n_heads, n_rows, threads)
         used = min(threads, len(heads))
         if dt * used >= budget_s or (n_heads >= B * H and n_rows >= N) or dt > budget_s:
-            break
+            return n_heads, n_rows, dt, flops, heads
         if n_heads < B * H:
             n_heads = min(B * H, n_heads * 2)
         else:
             n_rows = min(N, n_rows * 2)
-    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": used, "kind": "oracle",
-            "host_cpus": threads, "seconds": dt,
-            "sample": f"FP64 oracle fwd+bwd on {len(heads)} of {B * H} heads, query rows "
-                      f"0..{n_rows - 1} of {N} (FLOPs counted as the metric counts them)"}
+
+
+def sample_text(x, n_heads, n_rows):
+    B, H, N, d = x.q.shape
+    r0, r1 = sample_band(N, n_rows)
+    return (f"FP64 oracle fwd+bwd on {n_heads} of {B * H} heads, query rows {r0}..{r1 - 1} of "
+            f"{N} (FLOPs counted as the metric counts them: the workload's rate per allowed "
+            f"(query, key) entry times the sample's entries)")
+
+
+def cpu_baseline(x, budget_s=20.0):
+    """Oracle throughput on a bounded sample of about budget_s CPU-seconds."""
+    threads = os.cpu_count() or 1
+    n_heads, n_rows, dt, flops, heads = grow_sample(x, threads, budget_s)
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": min(threads, len(heads)),
+            "kind": "oracle", "host_cpus": threads, "seconds": dt,
+            "sample": sample_text(x, len(heads), n_rows)}
 
 
 def run_reference(args):
@@ -620,8 +642,10 @@ def run_reference(args):
     x = workload_or_shape(args)
     threads = os.cpu_count() or 1
     B, H, N, d = x.q.shape
-    n_heads, n_rows = sample_plan(x, threads)
-    n_heads = min(n_heads, B * H)
+    # the kind of sample the CPU baseline takes, sized so that the K + W steps take about
+    # 120 CPU-seconds together (0.5 at least each): the same heads and rows in every step
+    per_step = max(0.5, min(args.cpu_budget, 120.0 / max(1, args.steps + args.warmup)))
+    n_heads, n_rows, _, _, _ = grow_sample(x, threads, per_step)
     for _ in range(args.warmup):
         time_oracle(x, n_heads, n_rows, threads)
     times, flops = [], 0.0
@@ -631,8 +655,7 @@ def run_reference(args):
     ms = 1e3 * sum(times) / len(times)
     value = flops / (ms * 1e-3) / 1e12
     used = min(threads, n_heads)
-    sample = (f"FP64 oracle fwd+bwd on {n_heads} of {B * H} heads, query rows 0..{n_rows - 1} "
-              f"of {N}")
+    sample = sample_text(x, n_heads, n_rows)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,

@@ -18,7 +18,8 @@ import torch
 
 import oracle
 from exact_io_aware_63_b200 import binding, inputs
-from gpu_helpers import BF16_U, LSE_TOL, O_TOL, compare_grads, f64, to_dev
+from gpu_helpers import (BF16_U, LSE_TOL, O_TOL, compare_grads, f64, report_beyond_o_tol,
+                         to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -51,6 +52,7 @@ def compare_forward(o_gpu, lse_gpu, o_ref, lse_ref, pv_abs, where):
         idx = np.unravel_index(np.argmax(err - bound), err.shape)
         raise AssertionError(f"{where}: O error {err[idx]:.3e} > bound {bound[idx]:.3e} at "
                              f"{idx}: gpu {o_gpu[idx]:.6f} ref {o_ref[idx]:.6f}")
+    report_beyond_o_tol(o_gpu, o_ref, where)
     fin = ~empty
     lerr = float(np.abs(lse_gpu[fin] - lse_ref[fin]).max()) if fin.any() else 0.0
     assert lerr <= LSE_TOL, f"{where}: LSE max-abs {lerr:.3e} > {LSE_TOL}"
