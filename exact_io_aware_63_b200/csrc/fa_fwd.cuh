@@ -896,6 +896,18 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
     uint32_t s_cnt = 0, unit_cnt = 0;
     uint32_t q_use = 0;  // units seen: ring index of their Q slot
     uint32_t o_cnt[2] = {0, 0};
+    // Staged epilogue: the Q slot whose O store is still reading it.  The
+    // storing thread does not wait for that read in place (its warp would lag
+    // into the next unit); it waits and releases the slot after its next P,
+    // at the next epilogue, or at the end, whichever comes first.
+    int pend_slot = -1;
+    auto release_pending = [&]() {
+      if (Cfg::kEpiTma && r_local == 0 && pend_slot >= 0) {
+        bulk_wait_group_read0();
+        mbar_arrive(q_empty(pend_slot));
+        pend_slot = -1;
+      }
+    };
     bool ok = true;
     for (int round = 0; ok; ++round) {
       int u = -1;
@@ -905,6 +917,8 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
       const int qs_me = q_use % QSLOTS;
       const uint32_t q_par = (q_use / QSLOTS) & 1;
       ++q_use;
+      // this unit's Q is loaded into the pending slot only after its release
+      if (pend_slot == qs_me) release_pending();
       if (kPair && x == 1 && !w.has1) {
         // pair with no second tile: nothing to compute or write.  The staged
         // epilogue releases this warpgroup's share of the Q slot, once this
@@ -1084,6 +1098,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(p_full(x));
+        release_pending();
         ++cnt;
         if (*abort_flag) { ok = false; break; }
       }
@@ -1115,6 +1130,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
           ok = __all_sync(0xffffffffu, mbar_wait(q_full(qs_me), q_par));
           if (!ok) break;
         }
+        release_pending();
         const float inv_l = (cnt > 0 && l > 0.f) ? (kDrop ? p.drop.w : 1.f) / l : 0.f;
         uint8_t* const stage_row = smem + Cfg::kOffQ +
                                    (qs_me * Cfg::kQPerSlot + x) * Cfg::kTileBytes + r_local * 128;
@@ -1159,9 +1175,10 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
               tma_store_3d(&tm_o, 0, yz.x, yz.y,
                            sbase + Cfg::kOffQ + (qs_me * Cfg::kQPerSlot + x) * Cfg::kTileBytes);
               bulk_commit_group();
-              bulk_wait_group_read0();
+              pend_slot = qs_me;  // released once the store has read it
+            } else {
+              mbar_arrive(q_empty(qs_me));  // the Q slot may be loaded again
             }
-            mbar_arrive(q_empty(qs_me));  // the Q slot may be loaded again
           }
         }
       } else {
@@ -1231,6 +1248,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kPair>::kThreads, 1)
       }
     }
     if (!ok) *abort_flag = 1;
+    release_pending();
     if (Cfg::kEpiTma && r_local == 0) bulk_wait_group0();  // O stores complete before exit
   }
 
