@@ -488,11 +488,7 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_t, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": args.workload + (f" at shape {args.shape}" if args.shape else ""),
-                   "description": w.description,
-                   "B": B, "H": H, "N": N, "d": d, "causal": causal,
-                   "key_padding": x.kv_len is not None, "block_sparse": x.block_mask is not None,
-                   "flop_density": density(x), "seed": w.seed,
+        "config": {**workload_config(args, w, x),
                    "l2": "flushed between timed steps (256 MiB write)",
                    "timing": ("value: K whole steps, CUDA events around each step; ms and "
                               "roofline: K further steps with an event between kernels"),
@@ -560,6 +556,16 @@ def oracle_sample(x, n_heads, n_rows):
     sel = lambda t: torch.stack([t[b, h] for b, h in heads])[:, None].to(torch.float64).numpy()
     kl = None if x.kv_len is None else [int(x.kv_len[b]) for b, _ in heads]
     return heads, sel(x.q), sel(x.k), sel(x.v), sel(x.dout), kl
+
+
+def workload_config(args, w, x):
+    """The keys that name the workload, the same in both arms' lines."""
+    B, H, N, d = x.q.shape
+    return {"workload": args.workload + (f" at shape {args.shape}" if args.shape else ""),
+            "description": w.description, "B": B, "H": H, "N": N, "d": d,
+            "causal": bool(x.causal), "key_padding": x.kv_len is not None,
+            "block_sparse": x.block_mask is not None, "flop_density": density(x),
+            "seed": w.seed}
 
 
 def sample_band(N, n_rows):
@@ -661,9 +667,7 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": args.workload + (f" at shape {args.shape}" if args.shape else ""),
-                       "description": w.description, "B": B, "H": H, "N": N, "d": d,
-                       "parallelism": "cpu threads"},
+            "config": {**workload_config(args, w, x), "parallelism": "cpu threads"},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": used, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,

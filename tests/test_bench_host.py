@@ -120,6 +120,12 @@ def test_reference_arm_prints_one_contract_line():
     assert line["e2e"] == {"value": line["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
     assert line["config"]["N"] == 256 and line["config"]["H"] == 2
+    # the keys naming the workload are the ones the GPU arm's line carries
+    ap = type("A", (), {"workload": "long16k_causal", "shape": "1,2,256,64"})()
+    x = bench.workload_or_shape(ap)
+    want = bench.workload_config(ap, inputs.WORKLOADS["long16k_causal"], x)
+    assert {k: line["config"][k] for k in want} == want
+    assert want["causal"] is True and want["flop_density"] == bench.density(x)
 
 
 def test_reference_arm_runs_on_rank_zero_only():
