@@ -189,8 +189,11 @@ struct FwdCfg {
   static constexpr int kSmemBytes = kOffRing + 4 * kUnitRing;
   static_assert(kSmemBytes <= 232448, "shared memory over the per-block limit");
   static constexpr uint32_t kTmemCols = 512;
-  // pairs (of every 8) whose exponentials ex2_poly2 computes on interior tiles
-  static constexpr int kPolyPer8 = (D == 64) ? 2 : 1;
+  // pairs (of every 8) whose exponentials ex2_poly2 computes on interior tiles.
+  // D = 64 runs both warpgroups' softmax at once, sharing the MUFU unit: a
+  // quarter on the FMA pipe balances the two.  At D = 128 the warpgroups take
+  // turns and the FMA pipe is the busier one: every exponential goes to MUFU.
+  static constexpr int kPolyPer8 = (D == 64) ? 2 : 0;
   // D = 64 leaves 128 TMEM columns after S_0, S_1, O_0, O_1: P gets its own
   // 64 columns per warpgroup, so the next S can be issued as soon as the
   // softmax has read the current one, and each warpgroup has its own MMA
