@@ -131,6 +131,25 @@ def report_beyond_o_tol(o_gpu, o_ref, where=""):
     return rows
 
 
+def dq_edge_bound(do_rows, o_gpu, o_ref, pk_abs, dq_ref, scale, v_abs_max):
+    """Element-wise bound on |dQ_gpu - dQ_ref| for rows with few keys.  The kernels take
+    D_r = sum_x dO_rx O_rx from the bf16 output O (the reading of the D formula), so D_r
+    is off by at most dD_r = sum_x |dO_rx| |O_gpu,rx - O_rx|, which moves dQ_r by
+    scale * dD_r * sum_c P_rc K_c, at most scale * dD_r * sum_c P_rc |K_cx| (pk_abs: the
+    oracle's forward with values |K|).  In a row with few keys and one dominant key
+    dP - D nearly cancels and this term dominates.  The roundings of P, dS and dQ to
+    bf16 add at most a few bf16 units of the row: 2^-6 of |dQ_ref,x| and of the row's
+    root mean square.  D_r and each dP_rc are float32 sums of d products, summed in
+    different orders: each within d * 2^-24 of the sum of the products' magnitudes
+    (|dO_r| |O_r| for D, at most |dO_r| v_abs_max for dP)."""
+    d = do_rows.shape[1]
+    dd = np.sum(np.abs(do_rows) * np.abs(o_gpu - o_ref), axis=1, keepdims=True)
+    dd += d * 2.0 ** -24 * np.sum(np.abs(do_rows) * (np.abs(o_ref) + v_abs_max), axis=1,
+                                  keepdims=True)
+    rms = np.sqrt(np.mean(dq_ref ** 2, axis=1, keepdims=True))
+    return scale * dd * pk_abs + 2.0 ** -6 * (np.abs(dq_ref) + rms) + 1e-6
+
+
 def compare_grads(gpu, ref, where=""):
     errs = {}
     for name in ("dq", "dk", "dv"):

@@ -7,7 +7,9 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_helpers import O_TOL, BeyondOTol, bf16_ulp, report_beyond_o_tol
+import oracle
+from exact_io_aware_63_b200 import inputs
+from gpu_helpers import O_TOL, BeyondOTol, bf16_ulp, dq_edge_bound, f64, report_beyond_o_tol
 
 
 def _next_bf16_up(a):
@@ -41,3 +43,23 @@ def test_report_is_silent_within_the_tolerance():
     with warnings.catch_warnings():
         warnings.simplefilter("error")
         assert report_beyond_o_tol(ref + 0.0099, ref) == []
+
+
+def test_dq_edge_bound_covers_d_from_the_rounded_output():
+    # dQ_r = scale * sum_c P_rc (dP_rc - D_r) K_c: with D_r taken from bf16(O) instead of
+    # O, dQ_r moves by -scale * (D'_r - D_r) * sum_c P_rc K_c (the oracle's forward with
+    # values K).  The bound must cover that shift on the causal edge rows.
+    x = inputs.make_inputs(1, 1, 256, 64, causal=True, seed=3)
+    q, k, v, do = (f64(t[0, 0]) for t in (x.q, x.k, x.v, x.dout))
+    rows = np.array([0, 1, 2, 127, 128, 255])
+    dq, delta = oracle.attention_backward_dq_rows(q[rows], do[rows], rows, k, v, x.scale, True)
+    o, _ = oracle.attention_forward_rows(q[rows], rows, k, v, x.scale, True)
+    pk, _ = oracle.attention_forward_rows(q[rows], rows, k, k, x.scale, True)
+    pk_abs, _ = oracle.attention_forward_rows(q[rows], rows, k, np.abs(k), x.scale, True)
+    o_b = torch.tensor(o).to(torch.bfloat16).double().numpy()
+    d_shift = np.sum(do[rows] * o_b, axis=1) - np.sum(do[rows] * o, axis=1)
+    dq_moved = dq - x.scale * d_shift[:, None] * pk
+    bound = dq_edge_bound(do[rows], o_b, o, pk_abs, dq, x.scale, float(np.abs(v).max()))
+    assert np.all(np.abs(dq_moved - dq) <= bound)
+    # and the bound is not vacuous: it is below |dQ| on most elements of the longer rows
+    assert np.mean(bound[3:] < np.abs(dq[3:])) > 0.5
