@@ -92,6 +92,27 @@ def test_d256_partial_tile_and_key_padding(cuda_device, causal):
     check_all_heads(x)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1, 100])
+def test_d256_single_partial_tile(cuda_device, causal, N):
+    # one query tile and one key tile, both partial; B * H > 1 so that the partial tile
+    # of one head sits next to the next head's rows
+    check_all_heads(inputs.make_inputs(2, 2, N, 256, causal=causal, seed=950 + N + int(causal)))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_d256_key_lengths_outside_zero_to_n(cuda_device, causal):
+    # kv_len values are taken clamped into [0, N]: -3 leaves batch 0 without keys
+    from gpu_helpers import f64
+    N = 384
+    x = inputs.make_inputs(2, 2, N, 256, causal=causal, seed=960 + int(causal),
+                           kv_len=torch.tensor([-3, N + 5], dtype=torch.int32))
+    res, out = check_all_heads(x)
+    assert np.all(f64(out["o"])[0] == 0) and np.all(np.isneginf(f64(out["lse"])[0]))
+    for name in ("dq", "dk", "dv"):
+        assert np.all(f64(out[name])[0] == 0), name
+
+
 def test_d256_block_mask_and_rows_without_keys(cuda_device):
     bm = inputs.draw_block_mask(5, 0.3, torch.Generator().manual_seed(920))
     bm[1, :] = 0  # query tile 1 sees no key tile
