@@ -839,48 +839,70 @@ __global__ void __launch_bounds__(Bwd256Cfg::kThreads, 1)
         //   dQ pass: row = query me, columns = keys t*128 + e
         //   dK / dV: row = key me, columns = queries t*128 + e
         const int col0 = t * kTile;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t rs_[32], rd[32];
-          tmem_ld32(tS + 32 * c, rs_);
-          if constexpr (kMode != kPassDV) tmem_ld32(tDP + 32 * c, rd);
-          tmem_wait_ld();
-          reg_fence32(rs_);
-          if constexpr (kMode != kPassDV) reg_fence32(rd);
+        // tiles with no element mask for this warp's rows take a path without the
+        // per-element tests
+        const bool row_interior =
+            kRowUnits ? (col0 + kTile <= kv_L && (!pq.causal || col0 + kTile - 1 <= me))
+                      : (key_valid && (!pk.causal || me <= col0));
+        const bool interior = __all_sync(0xffffffffu, row_interior);
+        // chunk c (32 columns): S (and dP) from TMEM, bf16 P or dS back over the
+        // score tile's first columns.  The loads of chunk c + 1 are issued before
+        // chunk c is computed, so their latency overlaps it.
+        uint32_t rs_[2][32], rd[2][32];
+        auto load = [&](int c) {
+          tmem_ld32(tS + 32 * c, rs_[c & 1]);
+          if constexpr (kMode != kPassDV) tmem_ld32(tDP + 32 * c, rd[c & 1]);
+        };
+        auto compute = [&](int c, auto interior_tag) {
+          constexpr bool kInterior = decltype(interior_tag)::value;
           uint32_t pk16[16];
 #pragma unroll
-          for (int e2 = 0; e2 < 16; ++e2) {
-            float v[2];
+          for (int e4 = 0; e4 < 8; ++e4) {
+            float4 nl4v, nd4v;
+            if constexpr (kRowUnits) {
+              nl4v = make_float4(my_nlse2, my_nlse2, my_nlse2, my_nlse2);
+              nd4v = make_float4(my_nd, my_nd, my_nd, my_nd);
+            } else {
+              nl4v = nl4[8 * c + e4];
+              nd4v = nd4[8 * c + e4];
+            }
+            const float nlv[4] = {nl4v.x, nl4v.y, nl4v.z, nl4v.w};
+            const float ndv[4] = {nd4v.x, nd4v.y, nd4v.z, nd4v.w};
+            float v[4];
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int e = 2 * e2 + h;
-              const int col = col0 + 32 * c + e;  // key (dQ pass) or query index
-              float nl, nd;
-              bool allowed;
-              if constexpr (kRowUnits) {
-                nl = my_nlse2;
-                nd = my_nd;
-                allowed = col < kv_L && (!pq.causal || col <= me);
-              } else {
-                const float* nlf = reinterpret_cast<const float*>(nl4);
-                const float* ndf = reinterpret_cast<const float*>(nd4);
-                nl = nlf[32 * c + e];
-                nd = ndf[32 * c + e];
-                allowed = key_valid && (!pk.causal || me <= col);
+            for (int h = 0; h < 4; ++h) {
+              const int e = 4 * e4 + h;
+              float pv = ex2_approx(fmaf(__uint_as_float(rs_[c & 1][e]), pk.scale_log2, nlv[h]));
+              if constexpr (!kInterior) {
+                const int col = col0 + 32 * c + e;  // key (dQ pass) or query index
+                const bool allowed = kRowUnits ? (col < kv_L && (!pq.causal || col <= me))
+                                               : (key_valid && (!pk.causal || me <= col));
+                pv = allowed ? pv : 0.f;
               }
-              float pv = ex2_approx(fmaf(__uint_as_float(rs_[e]), pk.scale_log2, nl));
-              pv = allowed ? pv : 0.f;
               if constexpr (kMode == kPassDV) {
                 v[h] = pv;
               } else {
                 // dS = P (dP - D), with P rounded to bf16 as the other kernels use it
                 const float pr = __bfloat162float(__float2bfloat16_rn(pv));
-                v[h] = pr * (__uint_as_float(rd[e]) + nd);
+                v[h] = pr * (__uint_as_float(rd[c & 1][e]) + ndv[h]);
               }
             }
-            pk16[e2] = pack_bf16x2(v[0], v[1]);
+            pk16[2 * e4] = pack_bf16x2(v[0], v[1]);
+            pk16[2 * e4 + 1] = pack_bf16x2(v[2], v[3]);
           }
           tmem_st16(tS + 16 * c, pk16);
+        };
+        load(0);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          tmem_wait_ld();
+          reg_fence32(rs_[c & 1]);
+          if constexpr (kMode != kPassDV) reg_fence32(rd[c & 1]);
+          if (c + 1 < 4) load(c + 1);
+          if (interior)
+            compute(c, std::true_type{});
+          else
+            compute(c, std::false_type{});
         }
         if constexpr (!kRowUnits) {
           __syncwarp();
