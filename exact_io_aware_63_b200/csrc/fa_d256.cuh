@@ -471,8 +471,8 @@ struct Bwd256Cfg {
   static constexpr int kOffRow = kOffRing + kRing * k256Chunk;  // 2 slots x (-LSE2, -D)
   static constexpr int kOffBar = kOffRow + 2 * 2 * kRowBytes;
   // a_full, a_empty, ring_full[R], ring_empty[R], row_full[2], row_empty[2],
-  // s_full[2], p_full, acc_done, drain, staged
-  static constexpr int kNumBars = 12 + 2 * kRing;
+  // s_full[2], p_full, acc_done, drain, staged, dp_free
+  static constexpr int kNumBars = 13 + 2 * kRing;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16;
   static_assert(kSmemBytes <= 232448, "shared memory over the per-block limit");
@@ -506,7 +506,9 @@ __global__ void __launch_bounds__(Bwd256Cfg::kThreads, 1)
   const uint32_t acc_done = bar0 + 8 * (9 + 2 * R);  // the unit's accumulator complete
   const uint32_t drain_bar = bar0 + 8 * (10 + 2 * R);
   const uint32_t staged = bar0 + 8 * (11 + 2 * R);  // the unit's output rows are staged
-  static_assert(Cfg::kNumBars == 12 + 2 * R, "barrier layout");
+  // dQ / dK passes: the math warps hold the tile's dP in registers
+  const uint32_t dp_free = bar0 + 8 * (12 + 2 * R);
+  static_assert(Cfg::kNumBars == 13 + 2 * R, "barrier layout");
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kOffMisc + 4);
   auto chunk = [&](uint32_t c) { return sbase + Cfg::kOffRing + (c % R) * k256Chunk; };
@@ -531,6 +533,7 @@ __global__ void __launch_bounds__(Bwd256Cfg::kThreads, 1)
     mbar_init(acc_done, 1);
     mbar_init(drain_bar, 1);
     mbar_init(staged, 128);
+    mbar_init(dp_free, 128);
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tmap(&tm_q);
@@ -659,20 +662,29 @@ __global__ void __launch_bounds__(Bwd256Cfg::kThreads, 1)
             if (*abort_flag) ok = false;
           }
         } else {
-          for (int t = first_visit(w); t < end_visit(w) && ok; t = next_visit(w, t)) {
-            const int o0 = t * kTile;
-            if constexpr (kMode == kPassDQ) {
-              // S: K_j columns; dP: V_j columns; dQ: K_j rows
-              for (int c = 0; c < 4 && ok; ++c) ok = load_col(&tm_k, o0, z, c);
-              for (int c = 0; c < 4 && ok; ++c) ok = load_col(&tm_v, o0, z, c);
-              for (int m = 0; m < 4 && ok; ++m) ok = load_row(&tm_k32, o0, z, m);
-            } else {
-              // S^T: Q_i columns; dP^T: dO_i columns; dK: Q_i rows
-              ok = load_rows(z, t);
-              for (int c = 0; c < 4 && ok; ++c) ok = load_col(&tm_q, o0, z, c);
-              for (int c = 0; c < 4 && ok; ++c) ok = load_col(&tm_do, o0, z, c);
-              for (int m = 0; m < 4 && ok; ++m) ok = load_row(&tm_q32, o0, z, m);
+          // S: K_j (dQ pass) or Q_i (dK pass) columns; dP: V_j or dO_i columns;
+          // the accumulating product: K_j or Q_i rows.  Consumption order
+          // (dP one visit ahead): S(v0) dP(v0) | dP(v1) rows(v0) S(v1) | ...
+          const CUtensorMap* tm_s = (kMode == kPassDQ) ? &tm_k : &tm_q;
+          const CUtensorMap* tm_dp = (kMode == kPassDQ) ? &tm_v : &tm_do;
+          const CUtensorMap* tm_acc = (kMode == kPassDQ) ? &tm_k32 : &tm_q32;
+          int t = first_visit(w);
+          if (t < end_visit(w)) {
+            if constexpr (kMode == kPassDK) ok = load_rows(z, t);
+            for (int c = 0; c < 4 && ok; ++c) ok = load_col(tm_s, t * kTile, z, c);
+            for (int c = 0; c < 4 && ok; ++c) ok = load_col(tm_dp, t * kTile, z, c);
+          }
+          while (ok && t < end_visit(w)) {
+            const int tn = next_visit(w, t);
+            const bool more = tn < end_visit(w);
+            if (more)
+              for (int c = 0; c < 4 && ok; ++c) ok = load_col(tm_dp, tn * kTile, z, c);
+            for (int m = 0; m < 4 && ok; ++m) ok = load_row(tm_acc, t * kTile, z, m);
+            if (more && ok) {
+              if constexpr (kMode == kPassDK) ok = load_rows(z, tn);
+              for (int c = 0; c < 4 && ok; ++c) ok = load_col(tm_s, tn * kTile, z, c);
             }
+            t = tn;
             if (*abort_flag) ok = false;
           }
         }
@@ -685,7 +697,7 @@ __global__ void __launch_bounds__(Bwd256Cfg::kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t idesc_acc = idesc_bf16_f32(128, 256, 0, 1);
-      uint32_t units = 0, chunks = 0, pcnt = 0;
+      uint32_t units = 0, chunks = 0, pcnt = 0, dpcnt = 0;
       bool ok = true;
       auto wait_chunk = [&]() -> bool {
         return mbar_wait(ring_full(chunks % R), (chunks / R) & 1);
@@ -758,17 +770,36 @@ __global__ void __launch_bounds__(Bwd256Cfg::kThreads, 1)
           }
           n = k > 0 ? k - 1 : 0;  // the unit's visits: the last step issued only dV
         } else {
-          for (int t = first_visit(w); t < end_visit(w) && ok; t = next_visit(w, t)) {
-            // the score tile and dP (both from the resident tiles)
-            ok = issue_cols(Cfg::kColS, Cfg::kOffA, false) && issue_cols(Cfg::kColDP, Cfg::kOffB, false);
+          auto mark = [&](int t) {
+            if constexpr (kRowUnits) {
+              if (pq.visited) pq.visited[((size_t)w.f.bh * pq.n_t + w.f.i0) * pq.n_t + t] = 1;
+            } else {
+              if (pk.visited) pk.visited[((size_t)w.b.bh * pk.n_t + t) * pk.n_t + w.b.j] = 1;
+            }
+          };
+          // Per visit: dP of the next visit as soon as the math warps hold this
+          // one's dP in registers (its MMAs overlap their dS work), then the
+          // accumulating product once dS is in TMEM, then the next score tile
+          // over that dS (issue order).
+          int t = first_visit(w);
+          if (t < end_visit(w)) {
+            ok = issue_cols(Cfg::kColS, Cfg::kOffA, false) &&
+                 issue_cols(Cfg::kColDP, Cfg::kOffB, false);
+            if (ok) {
+              umma_commit(s_full(0));
+              mark(t);
+            }
+          }
+          while (ok && t < end_visit(w)) {
+            const int tn = next_visit(w, t);
+            const bool more = tn < end_visit(w);
+            ok = mbar_wait(dp_free, dpcnt & 1);
+            ++dpcnt;
             if (!ok) break;
-            umma_commit(s_full(0));
-            if (pk.visited || pq.visited) {
-              if constexpr (kRowUnits) {
-                if (pq.visited) pq.visited[((size_t)w.f.bh * pq.n_t + w.f.i0) * pq.n_t + t] = 1;
-              } else {
-                if (pk.visited) pk.visited[((size_t)w.b.bh * pk.n_t + t) * pk.n_t + w.b.j] = 1;
-              }
+            tc_fence_after();
+            if (more) {
+              ok = issue_cols(Cfg::kColDP, Cfg::kOffB, false);
+              if (!ok) break;
             }
             // dS (bf16, over the score tile) x streamed rows into the accumulator
             ok = mbar_wait(p_full, pcnt & 1);
@@ -777,6 +808,14 @@ __global__ void __launch_bounds__(Bwd256Cfg::kThreads, 1)
             tc_fence_after();
             ok = issue_rows(Cfg::kColS, n == 0);
             ++n;
+            if (!ok) break;
+            if (more) {
+              ok = issue_cols(Cfg::kColS, Cfg::kOffA, false);
+              if (!ok) break;
+              umma_commit(s_full(0));
+              mark(tn);
+            }
+            t = tn;
             if (*abort_flag) ok = false;
           }
         }
@@ -848,11 +887,19 @@ __global__ void __launch_bounds__(Bwd256Cfg::kThreads, 1)
         // chunk c (32 columns): S (and dP) from TMEM, bf16 P or dS back over the
         // score tile's first columns.  The loads of chunk c + 1 are issued before
         // chunk c is computed, so their latency overlaps it.
-        uint32_t rs_[2][32], rd[2][32];
-        auto load = [&](int c) {
-          tmem_ld32(tS + 32 * c, rs_[c & 1]);
-          if constexpr (kMode != kPassDV) tmem_ld32(tDP + 32 * c, rd[c & 1]);
-        };
+        // dQ / dK passes: all of dP into registers first; the issuer then
+        // computes the next visit's dP while this tile's dS is formed
+        uint32_t rs_[2][32], rd[kMode != kPassDV ? 4 : 1][32];
+        if constexpr (kMode != kPassDV) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tmem_ld32(tDP + 32 * c, rd[c]);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 4; ++c) reg_fence32(rd[c]);
+          tc_fence_before();
+          mbar_arrive(dp_free);
+        }
+        auto load = [&](int c) { tmem_ld32(tS + 32 * c, rs_[c & 1]); };
         auto compute = [&](int c, auto interior_tag) {
           constexpr bool kInterior = decltype(interior_tag)::value;
           uint32_t pk16[16];
@@ -867,7 +914,7 @@ __global__ void __launch_bounds__(Bwd256Cfg::kThreads, 1)
               nd4v = nd4[8 * c + e4];
             }
             const float nlv[4] = {nl4v.x, nl4v.y, nl4v.z, nl4v.w};
-            const float ndv[4] = {nd4v.x, nd4v.y, nd4v.z, nd4v.w};
+            [[maybe_unused]] const float ndv[4] = {nd4v.x, nd4v.y, nd4v.z, nd4v.w};
             float v[4];
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
@@ -884,7 +931,7 @@ __global__ void __launch_bounds__(Bwd256Cfg::kThreads, 1)
               } else {
                 // dS = P (dP - D), with P rounded to bf16 as the other kernels use it
                 const float pr = __bfloat162float(__float2bfloat16_rn(pv));
-                v[h] = pr * (__uint_as_float(rd[c & 1][e]) + ndv[h]);
+                v[h] = pr * (__uint_as_float(rd[kMode != kPassDV ? c : 0][e]) + ndv[h]);
               }
             }
             pk16[2 * e4] = pack_bf16x2(v[0], v[1]);
@@ -897,7 +944,6 @@ __global__ void __launch_bounds__(Bwd256Cfg::kThreads, 1)
         for (int c = 0; c < 4; ++c) {
           tmem_wait_ld();
           reg_fence32(rs_[c & 1]);
-          if constexpr (kMode != kPassDV) reg_fence32(rd[c & 1]);
           if (c + 1 < 4) load(c + 1);
           if (interior)
             compute(c, std::true_type{});
