@@ -461,7 +461,11 @@ struct Bwd256Params {
 
 struct Bwd256Cfg {
   static constexpr int D = 256;
-  static constexpr int kThreads = 256;
+  // warps 0-3: producer, MMA issuer (TMEM owner), two idle; warps 4-11: two math
+  // warpgroups, warpgroup h on score columns 64h .. 64h + 63 of every row and on
+  // output columns 128h .. 128h + 127 in the epilogue
+  static constexpr int kThreads = 384;
+  static constexpr int kMathThreads = 256;
   static constexpr int kTileBytes = kTile * D * 2;  // 64 KB
   static constexpr int kOffA = 0;                   // resident tile A: Q_i or K_j
   static constexpr int kOffB = kTileBytes;          // resident tile B: dO_i or V_j
@@ -526,14 +530,14 @@ __global__ void __launch_bounds__(Bwd256Cfg::kThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(row_full(s), 1);
-      mbar_init(row_empty(s), 4);  // lane 0 of each math warp
+      mbar_init(row_empty(s), 8);  // lane 0 of each math warp
       mbar_init(s_full(s), 1);
     }
-    mbar_init(p_full, 128);
+    mbar_init(p_full, Cfg::kMathThreads);
     mbar_init(acc_done, 1);
     mbar_init(drain_bar, 1);
-    mbar_init(staged, 128);
-    mbar_init(dp_free, 128);
+    mbar_init(staged, Cfg::kMathThreads);
+    mbar_init(dp_free, Cfg::kMathThreads);
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tmap(&tm_q);
@@ -828,7 +832,8 @@ __global__ void __launch_bounds__(Bwd256Cfg::kThreads, 1)
     }
     __syncwarp();
   } else if (warp >= 4) {
-    // ------------------------------------------------------------ math warpgroup
+    // ------------------------------------------------------------ math warpgroups
+    const int hg = (warp - 4) >> 2;  // warpgroup: score chunks 2hg, 2hg + 1
     const int quarter = warp & 3;
     const int rl = quarter * 32 + lane;  // row within the unit's tile = TMEM lane
     const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
@@ -889,18 +894,21 @@ __global__ void __launch_bounds__(Bwd256Cfg::kThreads, 1)
         // chunk c is computed, so their latency overlaps it.
         // dQ / dK passes: all of dP into registers first; the issuer then
         // computes the next visit's dP while this tile's dS is formed
-        uint32_t rs_[2][32], rd[kMode != kPassDV ? 4 : 1][32];
+        // this warpgroup's two chunks of 32 columns: c0 and c0 + 1
+        const int c0 = 2 * hg;
+        uint32_t rs_[2][32], rd[kMode != kPassDV ? 2 : 1][32];
         if constexpr (kMode != kPassDV) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) tmem_ld32(tDP + 32 * c, rd[c]);
+          for (int i = 0; i < 2; ++i) tmem_ld32(tDP + 32 * (c0 + i), rd[i]);
           tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 4; ++c) reg_fence32(rd[c]);
+          for (int i = 0; i < 2; ++i) reg_fence32(rd[i]);
           tc_fence_before();
           mbar_arrive(dp_free);
         }
-        auto load = [&](int c) { tmem_ld32(tS + 32 * c, rs_[c & 1]); };
-        auto compute = [&](int c, auto interior_tag) {
+        auto load = [&](int i) { tmem_ld32(tS + 32 * (c0 + i), rs_[i]); };
+        auto compute = [&](int i, auto interior_tag) {
+          const int c = c0 + i;
           constexpr bool kInterior = decltype(interior_tag)::value;
           uint32_t pk16[16];
 #pragma unroll
@@ -919,7 +927,7 @@ __global__ void __launch_bounds__(Bwd256Cfg::kThreads, 1)
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
               const int e = 4 * e4 + h;
-              float pv = ex2_approx(fmaf(__uint_as_float(rs_[c & 1][e]), pk.scale_log2, nlv[h]));
+              float pv = ex2_approx(fmaf(__uint_as_float(rs_[i][e]), pk.scale_log2, nlv[h]));
               if constexpr (!kInterior) {
                 const int col = col0 + 32 * c + e;  // key (dQ pass) or query index
                 const bool allowed = kRowUnits ? (col < kv_L && (!pq.causal || col <= me))
@@ -931,7 +939,7 @@ __global__ void __launch_bounds__(Bwd256Cfg::kThreads, 1)
               } else {
                 // dS = P (dP - D), with P rounded to bf16 as the other kernels use it
                 const float pr = __bfloat162float(__float2bfloat16_rn(pv));
-                v[h] = pr * (__uint_as_float(rd[kMode != kPassDV ? c : 0][e]) + ndv[h]);
+                v[h] = pr * (__uint_as_float(rd[kMode != kPassDV ? i : 0][e]) + ndv[h]);
               }
             }
             pk16[2 * e4] = pack_bf16x2(v[0], v[1]);
@@ -941,14 +949,14 @@ __global__ void __launch_bounds__(Bwd256Cfg::kThreads, 1)
         };
         load(0);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int i = 0; i < 2; ++i) {
           tmem_wait_ld();
-          reg_fence32(rs_[c & 1]);
-          if (c + 1 < 4) load(c + 1);
+          reg_fence32(rs_[i]);
+          if (i == 0) load(1);
           if (interior)
-            compute(c, std::true_type{});
+            compute(i, std::true_type{});
           else
-            compute(c, std::false_type{});
+            compute(i, std::false_type{});
         }
         if constexpr (!kRowUnits) {
           __syncwarp();
@@ -972,7 +980,7 @@ __global__ void __launch_bounds__(Bwd256Cfg::kThreads, 1)
       tc_fence_after();
       const float mul = (kMode == kPassDV) ? 1.f : pk.scale;
 #pragma unroll 1
-      for (int c = 0; c < 8; ++c) {
+      for (int c = 4 * hg; c < 4 * hg + 4; ++c) {
         uint32_t pk16[16];
         if (n > 0) {  // warp-uniform: tcgen05.ld is a collective of the whole warp
           uint32_t r[32];
@@ -1000,7 +1008,7 @@ __global__ void __launch_bounds__(Bwd256Cfg::kThreads, 1)
       tc_fence_before();
       fence_proxy_async_smem();
       mbar_arrive(staged);
-      if (rl == 0) {
+      if (hg == 0 && rl == 0) {
         if (mbar_wait(staged, a_par)) {
           for (int c = 0; c < 4; ++c)
             tma_store_3d(&tm_out, 64 * c, own_tile(w) * kTile, bh, sbase + Cfg::kOffA + 16384 * c);
@@ -1013,7 +1021,7 @@ __global__ void __launch_bounds__(Bwd256Cfg::kThreads, 1)
       }
     }
     if (!ok) *abort_flag = 1;
-    if (rl == 0) bulk_wait_group0();
+    if (hg == 0 && rl == 0) bulk_wait_group0();
   }
 
   tc_fence_before();
