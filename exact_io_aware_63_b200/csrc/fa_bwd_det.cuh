@@ -13,12 +13,14 @@
 // order on every run, so dQ is bitwise reproducible; dK and dV from the main
 // kernel already are (one CTA owns each key tile).
 //
-// Roles (8 warps):
+// Roles (12 warps):
 //   warp 0      TMA producer: Q_i, dO_i and the tile's -LSE2 / -D rows
 //               (double-buffered across units for D = 64), then K_j, V_j of
 //               each visited key tile through a kStages ring
 //   warp 1      MMA issuer (one thread), TMEM owner
-//   warps 4-7   math warpgroup, one query row per thread (TMEM lane)
+//   warps 4-11  two math warpgroups, one query row per thread (TMEM lane):
+//               warpgroup h on keys 64h .. 64h + 63 of every key tile and on
+//               dQ columns h D/2 .. (h + 1) D/2 - 1 in the epilogue
 // TMEM columns: S [0,128), dP [128,256), dQ [256,256+D), dS (bf16, two per
 // column) [384,448).
 #pragma once
@@ -37,7 +39,8 @@ struct DetParams {
 
 template <int D>
 struct DetCfg {
-  static constexpr int kThreads = 256;
+  static constexpr int kThreads = 384;
+  static constexpr int kMathThreads = 256;
   static constexpr int kTileBytes = kTile * D * 2;
   static constexpr int kBoxes = D / 64;
   static constexpr int kQSlots = (D == 64) ? 2 : 1;  // Q_i + dO_i per slot
@@ -107,8 +110,8 @@ __global__ void __launch_bounds__(DetCfg<D>::kThreads, 1)
       mbar_init(v_empty(s), 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(s_free, 128);
-    mbar_init(ds_full, 128);
+    mbar_init(s_free, Cfg::kMathThreads);
+    mbar_init(ds_full, Cfg::kMathThreads);
     mbar_init(ds_free, 1);
     mbar_init(dq_full, 1);
     mbar_init(drain_bar, 1);
@@ -266,6 +269,7 @@ __global__ void __launch_bounds__(DetCfg<D>::kThreads, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------------ math
+    const int hh = (warp - 4) >> 2;  // warpgroup: keys 64 hh .. 64 hh + 63 of each tile
     const int quarter = warp & 3;
     const int r_local = quarter * 32 + lane;  // query row within the tile = TMEM lane
     const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
@@ -286,7 +290,7 @@ __global__ void __launch_bounds__(DetCfg<D>::kThreads, 1)
       if (j >= w.j_end) {
         // no key visible to this query tile: dQ = 0 (Q and the rows are not read)
 #pragma unroll
-        for (int c = 0; c < D / 8; ++c)
+        for (int c = hh * D / 16; c < (hh + 1) * D / 16; ++c)
           if (row_ok) out_row[c] = make_uint4(0, 0, 0, 0);
         continue;
       }
@@ -308,8 +312,7 @@ __global__ void __launch_bounds__(DetCfg<D>::kThreads, 1)
         const int kv_lim = w.L - j * kTile;  // keys >= kv_lim are padding
         const int lim = diag ? min(r_local + 1, kv_lim) : kv_lim;
         const bool boundary = diag || kv_lim < kTile;
-#pragma unroll 1
-        for (int hh = 0; hh < 2; ++hh) {
+        {
           uint32_t sr[2][32], pr[2][32];
           tmem_ld32(t_lane + Cfg::kColS + hh * 64, sr[0]);
           tmem_ld32(t_lane + Cfg::kColS + hh * 64 + 32, sr[1]);
@@ -320,11 +323,11 @@ __global__ void __launch_bounds__(DetCfg<D>::kThreads, 1)
           reg_fence32(sr[1]);
           reg_fence32(pr[0]);
           reg_fence32(pr[1]);
-          if (hh == 1) {
-            // all of S and dP are in registers: the next S / dP may overwrite them
-            tc_fence_before();
-            mbar_arrive(s_free);
-          } else if (ds_cnt > 0) {
+          // this warpgroup's half of S and dP is in registers: once both halves
+          // are, the next S / dP may overwrite them
+          tc_fence_before();
+          mbar_arrive(s_free);
+          if (ds_cnt > 0) {
             // dS is overwritten below: the previous dQ MMA must have read it
             ok = __all_sync(0xffffffffu, mbar_wait(ds_free, (ds_cnt - 1) & 1));
             if (!ok) break;
@@ -373,7 +376,7 @@ __global__ void __launch_bounds__(DetCfg<D>::kThreads, 1)
       if (!ok) break;
       tc_fence_after();
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = hh * D / 64; c < (hh + 1) * D / 64; ++c) {
         uint32_t r[32];
         tmem_ld32(t_lane + Cfg::kColDQ + c * 32, r);
         tmem_wait_ld();
