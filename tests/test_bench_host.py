@@ -82,6 +82,13 @@ def test_ideal_bytes_follow_the_rows():
         assert got == (8 * E + 4 * R, 20 * E + 8 * R)
 
 
+def test_launches_per_step():
+    # forward, preprocess, main and a dQ kernel; d = 256 has two main passes
+    for d in (32, 64, 96, 128):
+        assert bench.launches_per_step(d) == 4
+    assert bench.launches_per_step(256) == 5
+
+
 def test_oracle_sample_flops_cover_the_workload_when_the_sample_is_everything():
     # the CPU baseline counts a sample's FLOPs as the metric counts the whole workload,
     # pro rata to allowed entries: a sample of every head and row is the whole count
